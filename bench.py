@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the selective diagonal scan on B200: HybridMamba forward+backward.
+
+One step = the whole hot path over one synthetic batch of the HybridMamba
+workload (batch 8, L = 8192, 32 heads, P = 64, N = 128 = 64 real + 32
+rotation pairs, two-endpoint writes, bf16 I/O, fp32 state): the forward scan
+and the backward scan through the C ABI.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank scans its own batch (weak scaling); per-head
+parameter gradients are summed over ranks with one NCCL all-reduce, the only
+data-parallel exchange the path has.  Inputs (1.6 GB) exceed the 126 MB L2,
+so no flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_diagonal_state_b200 import synthetic as S  # noqa: E402
+
+METRIC = "HybridMamba scan tokens/s (fwd, fwd+bwd) at L=8192; % of HBM/TC roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="hybridmamba", choices=list(S.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target wall time of the bounded oracle sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (read every input once, write every output once)
+# ---------------------------------------------------------------------------
+def tensor_bytes(shape: S.ScanShape) -> dict:
+    s = shape
+    e = 2 if s.dtype_io == S.DTYPE_BF16 else 4
+    BL = s.batch * s.seqlen
+    return {
+        "x": BL * s.nheads * s.rank_in * s.headdim * e,
+        "y": BL * s.nheads * s.rank_out * s.headdim * e,
+        "B": BL * s.ngroups * s.rank_in * s.nstate * e,
+        "C": BL * s.ngroups * s.rank_out * s.nstate * e,
+        "dt": BL * s.nheads * e,
+        "lam": BL * s.nheads * e if s.two_endpoint else 0,
+    }
+
+
+def fwd_bytes(shape):
+    t = tensor_bytes(shape)
+    return t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["y"]
+
+
+def bwd_bytes(shape):
+    t = tensor_bytes(shape)
+    reads = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["y"]  # y-sized dy
+    writes = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
+    return reads + writes
+
+
+def kernel_bytes(shape, name: str) -> int:
+    """Algorithmic bytes of one launch of each kernel of the recurrent path."""
+    s = shape
+    t = tensor_bytes(shape)
+    BLH = s.batch * s.seqlen * s.nheads
+    ins = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
+    if name == "k_fwd":
+        return ins + t["y"]
+    if name == "k_bwd_sweep1":   # inputs + dy -> per-head dC (fp32)
+        return ins + t["y"] + BLH * s.rank_out * s.nstate * 4
+    if name == "k_bwd_sweep2":   # inputs + dy -> dx, sum_p G u^T (fp32), per-token scalars
+        return (ins + t["y"] + t["x"] + BLH * s.rank_in * s.nstate * 4
+                + BLH * (2 + s.rank_in * s.rank_out) * 4)
+    if name == "k_bwd_units":
+        return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["B"] + t["C"]
+                + 2 * t["dt"] + 2 * t["lam"] + BLH * (2 + s.rank_in * s.rank_out) * 4)
+    if name == "k_bwd_groups":
+        return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["C"] + t["B"] + t["C"]
+                + t["dt"] + t["lam"])
+    return 0
+
+
+FWD_KERNELS = ["k_fwd"]
+BWD_KERNELS = ["k_bwd_sweep1", "k_bwd_sweep2", "k_bwd_units", "k_bwd_groups", "k_bwd_params"]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for (ts, r) in self.rows if self.t0 - 0.15 <= ts <= self.t1 + 0.15 and len(r) >= 10]
+        if not rows:
+            rows = [r for (_, r) in self.rows if len(r) >= 10][-3:]
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[6 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (the reported baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_plan(shape, target_s):
+    """(units, seqlen) of a sample taking about target_s of wall time."""
+    import oracle
+    cores = os.cpu_count() or 1
+    cal = shape.replace(batch=1, nheads=1, ngroups=1, seqlen=256)
+    inp = S.make_inputs(cal, seed=99)
+    t = time.perf_counter()
+    oracle.scan_fwd(cal, inp)
+    oracle.scan_bwd(cal, inp, inp["dy"])
+    per_unit_token = (time.perf_counter() - t) / 256.0
+    # units run in parallel over the cores; keep the full sequence length
+    units = max(1, min(shape.nheads * shape.batch, cores))
+    L = shape.seqlen
+    est = per_unit_token * L * -(-units // cores)
+    if est > target_s:
+        L = max(256, int(L * target_s / est))
+    return units, L, cores
+
+
+def oracle_sample_run(shape, units, L, seed=5):
+    """Time one oracle fwd+bwd over `units` (batch row 0, heads 0..units-1) of length L."""
+    import oracle
+    h = min(units, shape.nheads)
+    b = -(-units // shape.nheads)
+    g = shape.ngroups if shape.ngroups == shape.nheads else max(1, shape.ngroups * h // shape.nheads)
+    if shape.ngroups == shape.nheads:
+        g = h
+    sub = shape.replace(batch=b, nheads=h, ngroups=g if h % g == 0 else 1, seqlen=L)
+    inp = S.make_inputs(sub, seed=seed)
+    t = time.perf_counter()
+    oracle.scan_fwd(sub, inp)
+    oracle.scan_bwd(sub, inp, inp["dy"])
+    dt = time.perf_counter() - t
+    unit_tokens = sub.batch * sub.nheads * L
+    return dt, unit_tokens / shape.nheads, sub
+
+
+def cpu_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle as it stands, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    shape = S.WORKLOADS[args.workload]
+    per_step_target = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    units, L, cores = oracle_sample_plan(shape, per_step_target)
+    for _ in range(args.warmup):
+        oracle_sample_run(shape, units, L)
+    total_t, total_tok = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, tok, sub = oracle_sample_run(shape, units, L)
+        total_t += dt
+        total_tok += tok
+    value = total_tok / total_t
+    sample = (f"{sub.batch}x{sub.nheads} (batch rows x heads) of {shape.name} at L={L}, fwd+bwd "
+              f"per step; tokens counted as head-tokens / {shape.nheads}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
+                   "nheads": shape.nheads, "headdim": shape.headdim,
+                   "state": f"{shape.n_real} real + {shape.n_pairs} pairs",
+                   "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from selective_diagonal_state_b200 import abi, scan
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the scan has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    abi.load_library()
+    shape = S.WORKLOADS[args.workload]
+    inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1000 * rank)
+    dev = scan.to_device(shape, inp)
+    desc = abi.make_desc(shape)
+    fwd_out = scan.alloc_fwd(shape)
+    grads = scan.alloc_bwd(shape)
+    ws = scan.alloc_workspace(shape, abi.PASS_BWD, desc=desc)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def allreduce_params():
+        if world > 1:
+            for t in (grads.dA_log, grads.dtheta, grads.dD):
+                if t is not None:
+                    dist.all_reduce(t)
+
+    def step():
+        scan.scan_forward(shape, dev, out=fwd_out, desc=desc)
+        scan.scan_backward(shape, dev, grads=grads, workspace=ws, desc=desc)
+        allreduce_params()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    abi.ssm_scan_poll_device_error()
+
+    # per-kernel events over the timed region (library-owned, on our stream)
+    launches_per_step = len(FWD_KERNELS) + len(BWD_KERNELS)
+    clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    clocks.start()
+    time.sleep(0.3)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    abi.ssm_scan_profile_start(launches_per_step * args.steps)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks.mark(False)
+    prof = abi.ssm_scan_profile_stop()
+    ms_step = start.elapsed_time(stop) / args.steps
+    gpu_launches = sum(c for c, _ in prof.values())
+
+    # forward alone
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    f0.record(stream)
+    for _ in range(args.steps):
+        scan.scan_forward(shape, dev, out=fwd_out, desc=desc)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ms_fwd = f0.elapsed_time(f1) / args.steps
+    clk = clocks.stop()
+    avg = {n: tot / max(1, c) for n, (c, tot) in prof.items()}
+    share = {n: tot / max(1e-9, sum(t for _, t in prof.values())) for n, (c, tot) in prof.items()}
+
+    # max over ranks
+    t = torch.tensor([ms_step, ms_fwd], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step, ms_fwd = float(t[0]), float(t[1])
+
+    tokens = shape.batch * shape.seqlen * world
+    value = tokens / (ms_step * 1e-3)
+    fwd_value = tokens / (ms_fwd * 1e-3)
+
+    peaks = {}
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        peaks = json.load(open(pk))
+    hbm = peaks.get("hbm_gbs")
+    peak_note = "measured" if hbm else "fallback"
+    hbm = hbm or 6650.0
+    dom = max(avg, key=avg.get)
+    dom_bytes = kernel_bytes(shape, dom)
+    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    step_bytes = fwd_bytes(shape) + bwd_bytes(shape)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {k: torch.from_numpy(np.ascontiguousarray(v)).to(scan.io_dtype(shape)
+                if k in ("x", "dt", "lam", "Bm", "Cm", "dy") else torch.float32).pin_memory()
+                for k, v in inp.items() if v is not None}
+        outs = [fwd_out[0], grads.dx, grads.ddt, grads.dBm, grads.dCm, grads.dA_log, grads.dD]
+        outs += [t_ for t_ in (grads.dtheta, grads.dlam) if t_ is not None]
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        dev_map = {"x": dev.x, "dt": dev.dt, "lam": dev.lam, "Bm": dev.Bm, "Cm": dev.Cm,
+                   "dy": dev.dy, "A_log": dev.A_log, "theta": dev.theta, "D": dev.D}
+        h2d = sum(host[k].numel() * host[k].element_size() for k in dev_map
+                  if k in host and dev_map[k] is not None)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for k, d in dev_map.items():
+                if d is not None and k in host:
+                    d.copy_(host[k], non_blocking=True)
+            step()
+            for o, ho in zip(outs, host_out):
+                ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
+        te = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        ms_e2e = float(te[0])
+        e2e = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        units, L, cores = oracle_sample_plan(shape, args.cpu_seconds)
+        dt_s, tok, sub = oracle_sample_run(shape, units, L)
+        cpu = {"value": tok / dt_s, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{sub.batch}x{sub.nheads} (batch rows x heads) of {shape.name} at "
+                         f"L={L}, fwd+bwd, {dt_s:.1f} s; tokens = head-tokens / {shape.nheads}"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": shape.name, "batch_per_gpu": shape.batch, "seqlen": shape.seqlen,
+                   "nheads": shape.nheads, "headdim": shape.headdim,
+                   "state": f"{shape.n_real} real + {shape.n_pairs} rotation pairs",
+                   "two_endpoint": bool(shape.two_endpoint), "io": "bf16, fp32 state",
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "inputs (1.6 GB) larger than L2; no flush"},
+        "fwd_tokens_per_s": fwd_value, "ms_fwd": ms_fwd,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "kernel": dom,
+                     "algorithmic_bytes": dom_bytes, "ms_per_launch": avg[dom],
+                     "peak_source": peak_note},
+        "step_roofline": {"algorithmic_bytes": step_bytes,
+                          "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+                          "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm},
+        "kernel_ms": avg, "kernel_share": share,
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective diagonal scan library.
+ *
+ * The operation (per batch row b and head h) is the linear-transition
+ * state-space recurrence
+ *      h_t = A_t h_{t-1} + B_t u_t,      y_t = C_t h_t + D u_t
+ * of "When a Diagonal State Is Not Enough" (sungsoo.github.io), Part 01
+ * "Definition" and Part 03 "Selective SSM and masked linear attention", in
+ * the HybridMamba / SSD-MIMO form of "Diagonal Equivalence in State Space
+ * Models" (abstract; kongchang.com "From MIMO to HybridMamba"):
+ *
+ *  - state H_t is N x P per head, N = n_real + 2 * n_pairs: n_real real
+ *    coordinates with per-coordinate decay (Mamba-1 style) followed by
+ *    n_pairs complex coordinates stored as (re, im) row pairs and evolved by
+ *    real 2x2 decay-rotation blocks (Mamba-3 style); P channels share one
+ *    transition (Mamba-2-style heads);
+ *  - A_t = exp(dt_t a) on real rows and exp(dt_t a_j) R(dt_t theta_j) on pair
+ *    j, R(phi) = [[cos, -sin], [sin, cos]], a = -exp(A_log);
+ *  - two-endpoint (exponential-trapezoidal) write, sungsoo.github.io Part 05:
+ *        H_t = A_t (H_{t-1} + beta_t W_{t-1}) + gamma_t W_t,   W_t = B_t u_t,
+ *        gamma_t = lam_t dt_t,  beta_t = (1 - lam_t) dt_t
+ *    (two_endpoint = 0 means lam = 1: the Euler write of Mamba-1/2);
+ *  - SSD-MIMO routing (sungsoo.github.io Part 03 "SISO and MIMO"): u_t is
+ *    R x P, B_t is N x R, C_t is O x N; D is used only when O == R.
+ *  Mamba-1, Mamba-2 and Mamba-3-SISO configurations are special cases.
+ *
+ * Memory: the caller owns every buffer.  The library allocates no device or
+ * host memory and launches only on the caller's stream.  All pointers are
+ * device pointers unless stated otherwise.
+ *
+ * Errors: every entry point returns SSM_OK (0) or a negative SSM_ERR_* code
+ * and never aborts; ssm_scan_last_error() gives a message for the calling
+ * thread.  Launches are asynchronous: a fault inside a kernel surfaces as
+ * SSM_ERR_CUDA from a later call or from the caller's own synchronisation.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_SCAN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+enum ssm_status {
+    SSM_OK = 0,
+    SSM_ERR_ARG = -1,         /* bad descriptor, null required pointer, size mismatch */
+    SSM_ERR_UNSUPPORTED = -2, /* valid problem outside what the kernels implement */
+    SSM_ERR_ALIGN = -3,       /* pointer or stride alignment the kernels need is not met */
+    SSM_ERR_CUDA = -4,        /* a CUDA runtime call or a kernel launch failed */
+    SSM_ERR_TIMEOUT = -5,     /* a bounded device-side wait gave up (see ssm_scan_poll_device_error) */
+    SSM_ERR_WORKSPACE = -6    /* workspace missing or smaller than ssm_scan_workspace_size() */
+};
+
+enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 };
+enum ssm_decay_mode { SSM_DECAY_PER_HEAD = 0, SSM_DECAY_PER_COORD = 1 };
+enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1 };
+
+/*
+ * Problem descriptor.  Tensor layouts (innermost last):
+ *   x, dx      [batch][seqlen][nheads][rank_in][headdim]
+ *   y, dy      [batch][seqlen][nheads][rank_out][headdim]
+ *   B, dB      [batch][seqlen][ngroups][rank_in][N]     B_t[n][r] = B[b][t][g][r][n]
+ *   C, dC      [batch][seqlen][ngroups][rank_out][N]    C_t[o][n] = C[b][t][g][o][n]
+ *   dt, lambda, ddt, dlambda   [batch][seqlen][nheads]
+ *   A_log, dA_log  fp32 [nheads][n_decay], n_decay = 1 (SSM_DECAY_PER_HEAD) or
+ *                  n_real + n_pairs (SSM_DECAY_PER_COORD: real rows, then pairs)
+ *   theta, dtheta  fp32 [nheads][n_pairs]   rotation frequency of each pair
+ *   D, dD          fp32 [nheads]
+ *   h0, hT, prev_write, last_write, dh0, dprev_write  fp32 [batch][nheads][N][headdim]
+ * Head h reads group g = h / (nheads / ngroups).  State rows: the n_real real
+ * rows first, then pair j as rows n_real + 2j (re) and n_real + 2j + 1 (im).
+ * The two innermost dimensions of x/y/B/C are dense; the three outer ones
+ * (batch, time, head-or-group) use the element strides below, which also
+ * apply to the matching gradient tensor.  dt/lambda use their own strides.
+ * ssm_desc_set_contiguous() fills every stride for dense tensors.
+ */
+typedef struct ssm_desc {
+    int64_t batch, seqlen, nheads, headdim, ngroups;
+    int32_t n_real, n_pairs;
+    int32_t rank_in, rank_out;  /* R, O; SISO is 1, 1 */
+    int32_t chunk;              /* tuning hint only (0 = library choice); results do not depend on it beyond rounding */
+    int32_t decay_mode;         /* enum ssm_decay_mode */
+    int32_t two_endpoint;       /* 0: lambda not read (lam = 1); 1: lambda used */
+    int32_t dtype_io;           /* enum ssm_dtype of x, dt, B, C, lambda, y and of their gradients */
+    int64_t stride_x[3], stride_y[3], stride_B[3], stride_C[3], stride_dt[3], stride_lambda[3];
+} ssm_desc_t;
+
+/* Fill every stride of *d for dense tensors of the sizes already set. */
+SSM_API void ssm_desc_set_contiguous(ssm_desc_t *d);
+
+/*
+ * Bytes of device workspace that ssm_scan_fwd (pass = SSM_PASS_FWD) or
+ * ssm_scan_bwd (pass = SSM_PASS_BWD) needs for this descriptor; 0 means the
+ * workspace pointer may be NULL.  Returns 0 for an invalid descriptor (the
+ * compute call then reports the error).  The workspace must be 256-byte
+ * aligned; its contents need not be initialised and are clobbered.
+ */
+SSM_API size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass);
+
+/*
+ * Forward scan.  Reads x, dt, A_log, theta (may be NULL when n_pairs == 0),
+ * B, C, D (may be NULL when rank_in != rank_out), lambda (ignored when
+ * two_endpoint == 0), h0 and prev_write (NULL = zero initial state and zero
+ * left endpoint).  Writes y and, when non-NULL, hT = H_{L-1} and
+ * last_write = W_{L-1} = B_{L-1} u_{L-1}; passing (hT, last_write) as
+ * (h0, prev_write) of the next call continues the sequence exactly.
+ * stream is a cudaStream_t (NULL = legacy default stream).
+ */
+SSM_API int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, void *y,
+                 float *hT, float *last_write, void *workspace, size_t workspace_bytes,
+                 void *stream);
+
+/*
+ * Backward scan: gradients of sum(dy * y) with respect to every input of
+ * ssm_scan_fwd, recomputing the forward states (nothing is saved between the
+ * calls).  Inputs as for ssm_scan_fwd plus dy.  Outputs dx, ddt, dB, dC (in
+ * dtype_io), dA_log, dD (fp32), dtheta (fp32; may be NULL when n_pairs == 0),
+ * dlambda (dtype_io; may be NULL, and is not written when two_endpoint == 0),
+ * dh0 and dprev_write (fp32; may be NULL).  Gradients are written, not
+ * accumulated; group-shared dB/dC sum the heads of their group, and the
+ * per-head parameter gradients sum the batch, in a fixed order (deterministic).
+ */
+SSM_API int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, const void *dy,
+                 void *dx, void *ddt, float *dA_log, float *dtheta, void *dB, void *dC,
+                 float *dD, void *dlambda, float *dh0, float *dprev_write, void *workspace,
+                 size_t workspace_bytes, void *stream);
+
+/* Message describing the last failing call on this host thread ("" if none). */
+SSM_API const char *ssm_scan_last_error(void);
+
+/*
+ * Synchronise `stream` and report device-side errors raised by bounded waits
+ * inside the kernels since the previous poll (SSM_ERR_TIMEOUT), or a sticky
+ * CUDA error (SSM_ERR_CUDA).  Clears the device error word.
+ */
+SSM_API int ssm_scan_poll_device_error(void *stream);
+
+/*
+ * Per-kernel device timing (used by the benchmark).  ssm_scan_profile_start
+ * opens a session on the calling host thread and creates up to
+ * `max_launches` + 64 CUDA events up front; until ssm_scan_profile_stop, every
+ * kernel that ssm_scan_fwd / ssm_scan_bwd launch is bracketed by events
+ * recorded on the caller's stream (launches past the capacity are not timed).
+ * ssm_scan_profile_stop waits for the events, writes one entry per distinct
+ * kernel in first-launch order -- its name (NUL-terminated, truncated to
+ * name_len bytes, into names + i * name_len), launch count and summed device
+ * milliseconds -- destroys the events and returns the number of entries
+ * (at most max_kernels) or a negative status.
+ */
+SSM_API int ssm_scan_profile_start(int max_launches);
+SSM_API int ssm_scan_profile_stop(char *names, int name_len, int *counts, double *total_ms,
+                                  int max_kernels);
+
+/* SSM_SCAN_ABI_VERSION of the loaded library. */
+SSM_API int ssm_scan_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSM_SCAN_H */

@@ -1,0 +1,176 @@
+"""Python binding of the C ABI in ``include/ssm_scan.h`` (ctypes, marshalling only).
+
+Functions keep the C names (``ssm_scan_fwd``, ``ssm_scan_bwd``, ...) and take
+torch CUDA tensors (or raw device addresses as ``int``, or ``None`` for NULL).
+Every step of the scan runs in the CUDA library; nothing here computes.  The
+library must have been built (``python -m selective_diagonal_state_b200.build``)
+- there is no fallback: a missing library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .synthetic import ScanShape
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
+
+SSM_OK = 0
+STATUS = {0: "SSM_OK", -1: "SSM_ERR_ARG", -2: "SSM_ERR_UNSUPPORTED", -3: "SSM_ERR_ALIGN",
+          -4: "SSM_ERR_CUDA", -5: "SSM_ERR_TIMEOUT", -6: "SSM_ERR_WORKSPACE"}
+PASS_FWD, PASS_BWD = 0, 1
+
+EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
+            "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
+            "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop"]
+
+
+class SsmError(RuntimeError):
+    def __init__(self, code: int, where: str, msg: str):
+        super().__init__(f"{where} -> {STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Desc(ctypes.Structure):
+    """Mirror of ``ssm_desc_t``."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+        ("headdim", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+        ("n_real", ctypes.c_int32), ("n_pairs", ctypes.c_int32),
+        ("rank_in", ctypes.c_int32), ("rank_out", ctypes.c_int32),
+        ("chunk", ctypes.c_int32), ("decay_mode", ctypes.c_int32),
+        ("two_endpoint", ctypes.c_int32), ("dtype_io", ctypes.c_int32),
+        ("stride_x", ctypes.c_int64 * 3), ("stride_y", ctypes.c_int64 * 3),
+        ("stride_B", ctypes.c_int64 * 3), ("stride_C", ctypes.c_int64 * 3),
+        ("stride_dt", ctypes.c_int64 * 3), ("stride_lambda", ctypes.c_int64 * 3),
+    ]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing: build it with "
+                           "`python -m selective_diagonal_state_b200.build` (no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    lib.ssm_desc_set_contiguous.argtypes = [ctypes.POINTER(Desc)]
+    lib.ssm_desc_set_contiguous.restype = None
+    lib.ssm_scan_workspace_size.argtypes = [ctypes.POINTER(Desc), ctypes.c_int]
+    lib.ssm_scan_workspace_size.restype = ctypes.c_size_t
+    lib.ssm_scan_fwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 14 + [ctypes.c_size_t, _vp]
+    lib.ssm_scan_fwd.restype = ctypes.c_int
+    lib.ssm_scan_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 22 + [ctypes.c_size_t, _vp]
+    lib.ssm_scan_bwd.restype = ctypes.c_int
+    lib.ssm_scan_last_error.argtypes = []
+    lib.ssm_scan_last_error.restype = ctypes.c_char_p
+    lib.ssm_scan_poll_device_error.argtypes = [_vp]
+    lib.ssm_scan_poll_device_error.restype = ctypes.c_int
+    lib.ssm_scan_abi_version.argtypes = []
+    lib.ssm_scan_abi_version.restype = ctypes.c_int
+    lib.ssm_scan_profile_start.argtypes = [ctypes.c_int]
+    lib.ssm_scan_profile_start.restype = ctypes.c_int
+    lib.ssm_scan_profile_stop.argtypes = [ctypes.c_char_p, ctypes.c_int,
+                                          ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_double), ctypes.c_int]
+    lib.ssm_scan_profile_stop.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def make_desc(shape: ScanShape) -> Desc:
+    """Descriptor with dense strides for ``shape``."""
+    d = Desc()
+    d.batch, d.seqlen, d.nheads = shape.batch, shape.seqlen, shape.nheads
+    d.headdim, d.ngroups = shape.headdim, shape.ngroups
+    d.n_real, d.n_pairs = shape.n_real, shape.n_pairs
+    d.rank_in, d.rank_out = shape.rank_in, shape.rank_out
+    d.chunk, d.decay_mode = shape.chunk, shape.decay_mode
+    d.two_endpoint, d.dtype_io = shape.two_endpoint, shape.dtype_io
+    load_library().ssm_desc_set_contiguous(ctypes.byref(d))
+    return d
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not getattr(t, "is_cuda", False):
+        raise ValueError("ssm_scan: every tensor must live on a CUDA device (no CPU path)")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != SSM_OK:
+        msg = load_library().ssm_scan_last_error().decode(errors="replace")
+        raise SsmError(rc, where, msg)
+
+
+def ssm_scan_workspace_size(desc: Desc, pass_: int) -> int:
+    return int(load_library().ssm_scan_workspace_size(ctypes.byref(desc), pass_))
+
+
+def ssm_scan_fwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, y, hT=None,
+                 last_write=None, workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_scan_fwd(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h0, prev_write, y, hT, last_write, workspace)],
+        workspace_bytes, _stream(stream))
+    _check(rc, "ssm_scan_fwd")
+
+
+def ssm_scan_bwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt,
+                 dA_log, dtheta, dB, dC, dD, dlam=None, dh0=None, dprev_write=None,
+                 workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_scan_bwd(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt, dA_log, dtheta, dB, dC,
+        dD, dlam, dh0, dprev_write, workspace)], workspace_bytes, _stream(stream))
+    _check(rc, "ssm_scan_bwd")
+
+
+def ssm_scan_poll_device_error(stream=None) -> None:
+    _check(load_library().ssm_scan_poll_device_error(_stream(stream)),
+           "ssm_scan_poll_device_error")
+
+
+def ssm_scan_abi_version() -> int:
+    return int(load_library().ssm_scan_abi_version())
+
+
+def ssm_scan_profile_start(max_launches: int) -> None:
+    _check(load_library().ssm_scan_profile_start(max_launches), "ssm_scan_profile_start")
+
+
+def ssm_scan_profile_stop(max_kernels: int = 32) -> dict:
+    """Close the timing session; returns {kernel: (launches, total_ms)}."""
+    lib = load_library()
+    name_len = 48
+    names = ctypes.create_string_buffer(name_len * max_kernels)
+    counts = (ctypes.c_int * max_kernels)()
+    tot = (ctypes.c_double * max_kernels)()
+    n = lib.ssm_scan_profile_stop(names, name_len, counts, tot, max_kernels)
+    if n < 0:
+        _check(n, "ssm_scan_profile_stop")
+    out = {}
+    for i in range(n):
+        nm = names.raw[i * name_len:(i + 1) * name_len].split(b"\0", 1)[0].decode()
+        out[nm] = (int(counts[i]), float(tot[i]))
+    return out

@@ -1,0 +1,387 @@
+// C ABI of the selective diagonal scan library: argument validation, workspace
+// sizing, error reporting and dispatch to the kernels.  See include/ssm_scan.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/ssm_scan.h"
+#include "common.cuh"
+
+namespace ssm {
+bool simt_supported(const Params &p);
+cudaError_t simt_forward(const Params &p, cudaStream_t st);
+cudaError_t simt_backward(const Params &p, cudaStream_t st);
+}  // namespace ssm
+
+// Device word raised by bounded waits inside kernels (0 = no error).
+__device__ int ssm_device_error_word;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// per-kernel timing session (see ssm_scan_profile_start)
+struct ProfileRec {
+    const char *name;
+    int ev0, ev1;
+};
+struct ProfileSession {
+    bool active = false;
+    std::vector<cudaEvent_t> pool;
+    size_t used = 0;
+    int cur = -1;  // event that opens the next launch of the current call
+    std::vector<ProfileRec> recs;
+};
+thread_local ProfileSession g_prof;
+
+void profile_begin(cudaStream_t st) {
+    if (!g_prof.active || g_prof.used >= g_prof.pool.size()) {
+        g_prof.cur = -1;
+        return;
+    }
+    cudaEventRecord(g_prof.pool[g_prof.used], st);
+    g_prof.cur = (int)g_prof.used++;
+}
+void profile_end() { g_prof.cur = -1; }
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+    return fail(SSM_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+int nstate(const ssm_desc_t *d) { return d->n_real + 2 * d->n_pairs; }
+int ndecay(const ssm_desc_t *d) {
+    return d->decay_mode == SSM_DECAY_PER_HEAD ? 1 : d->n_real + d->n_pairs;
+}
+
+int validate_desc(const ssm_desc_t *d) {
+    if (!d) return fail(SSM_ERR_ARG, "descriptor is NULL");
+    if (d->batch < 0 || d->seqlen < 0) return fail(SSM_ERR_ARG, "batch and seqlen must be >= 0");
+    if (d->nheads < 1 || d->headdim < 1 || d->ngroups < 1)
+        return fail(SSM_ERR_ARG, "nheads, headdim and ngroups must be >= 1");
+    if (d->nheads % d->ngroups)
+        return fail(SSM_ERR_ARG, "nheads (%lld) must be a multiple of ngroups (%lld)",
+                    (long long)d->nheads, (long long)d->ngroups);
+    if (d->n_real < 0 || d->n_pairs < 0 || nstate(d) < 1)
+        return fail(SSM_ERR_ARG, "need n_real >= 0, n_pairs >= 0 and n_real + 2 n_pairs >= 1");
+    if (d->rank_in < 1 || d->rank_out < 1) return fail(SSM_ERR_ARG, "rank_in, rank_out must be >= 1");
+    if (d->decay_mode != SSM_DECAY_PER_HEAD && d->decay_mode != SSM_DECAY_PER_COORD)
+        return fail(SSM_ERR_ARG, "unknown decay_mode %d", d->decay_mode);
+    if (d->two_endpoint != 0 && d->two_endpoint != 1)
+        return fail(SSM_ERR_ARG, "two_endpoint must be 0 or 1");
+    if (d->dtype_io != SSM_F32 && d->dtype_io != SSM_BF16)
+        return fail(SSM_ERR_ARG, "unknown dtype_io %d", d->dtype_io);
+    if (d->chunk < 0) return fail(SSM_ERR_ARG, "chunk must be >= 0");
+    if (d->batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch > 65535");
+    if (d->seqlen > (1LL << 31) - 1 || d->nheads > (1 << 24) || d->headdim > (1 << 16))
+        return fail(SSM_ERR_UNSUPPORTED, "sizes exceed the 32-bit index ranges of the kernels");
+    const int64_t *st[] = {d->stride_x, d->stride_y, d->stride_B,
+                           d->stride_C, d->stride_dt, d->stride_lambda};
+    for (int i = 0; i < 6; ++i)
+        for (int k = 0; k < 3; ++k)
+            if (st[i][k] < 0) return fail(SSM_ERR_ARG, "negative stride");
+    return SSM_OK;
+}
+
+int check_ptr(const void *ptr, const char *name, size_t align) {
+    if (!ptr) return fail(SSM_ERR_ARG, "%s is NULL", name);
+    if ((uintptr_t)ptr % align) return fail(SSM_ERR_ALIGN, "%s is not %zu-byte aligned", name, align);
+    return SSM_OK;
+}
+
+void fill_params(const ssm_desc_t *d, ssm::Params &p) {
+    memset(&p, 0, sizeof(p));
+    p.Bsz = (int)d->batch;
+    p.L = (int)d->seqlen;
+    p.H = (int)d->nheads;
+    p.P = (int)d->headdim;
+    p.G = (int)d->ngroups;
+    p.nr = d->n_real;
+    p.np = d->n_pairs;
+    p.N = nstate(d);
+    p.R = d->rank_in;
+    p.O = d->rank_out;
+    p.ndec = ndecay(d);
+    p.hpg = (int)(d->nheads / d->ngroups);
+    p.two_ep = d->two_endpoint;
+    p.per_coord = d->decay_mode == SSM_DECAY_PER_COORD;
+    p.bf16 = d->dtype_io == SSM_BF16;
+    for (int k = 0; k < 3; ++k) {
+        p.sx[k] = d->stride_x[k];
+        p.sy[k] = d->stride_y[k];
+        p.sB[k] = d->stride_B[k];
+        p.sC[k] = d->stride_C[k];
+        p.sdt[k] = d->stride_dt[k];
+        p.slam[k] = d->stride_lambda[k];
+    }
+}
+
+struct BwdWs {
+    size_t off_dC, off_gbu, off_tok, off_M2, off_par, total;
+};
+
+BwdWs bwd_layout(const ssm_desc_t *d) {
+    BwdWs w;
+    const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
+    const size_t N = nstate(d);
+    size_t off = 0;
+    w.off_dC = off;
+    off = align256(off + BLH * d->rank_out * N * 4);
+    w.off_gbu = off;
+    off = align256(off + BLH * d->rank_in * N * 4);
+    w.off_tok = off;
+    off = align256(off + BLH * 2 * 4);
+    w.off_M2 = off;
+    off = align256(off + BLH * d->rank_out * d->rank_in * 4);
+    w.off_par = off;
+    off = align256(off + (size_t)d->batch * d->nheads * (ndecay(d) + d->n_pairs + 2) * 4);
+    w.total = off;
+    return w;
+}
+
+int common_inputs(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                  const float *theta, const void *B, const void *C, const float *D,
+                  const void *lambda) {
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    int rc;
+    if ((rc = check_ptr(x, "x", es)) || (rc = check_ptr(dt, "dt", es)) ||
+        (rc = check_ptr(A_log, "A_log", 4)) || (rc = check_ptr(B, "B", es)) ||
+        (rc = check_ptr(C, "C", es)))
+        return rc;
+    if (d->n_pairs > 0 && (rc = check_ptr(theta, "theta", 4))) return rc;
+    if (d->rank_in == d->rank_out && (rc = check_ptr(D, "D", 4))) return rc;
+    if (d->two_endpoint && (rc = check_ptr(lambda, "lambda", es))) return rc;
+    return SSM_OK;
+}
+
+}  // namespace
+
+namespace ssm {
+void profile_mark(cudaStream_t st, const char *name) {
+    if (!g_prof.active || g_prof.cur < 0 || g_prof.used >= g_prof.pool.size()) return;
+    cudaEventRecord(g_prof.pool[g_prof.used], st);
+    g_prof.recs.push_back({name, g_prof.cur, (int)g_prof.used});
+    g_prof.cur = (int)g_prof.used++;
+}
+}  // namespace ssm
+
+extern "C" {
+
+void ssm_desc_set_contiguous(ssm_desc_t *d) {
+    if (!d) return;
+    const int64_t N = d->n_real + 2LL * d->n_pairs;
+    const int64_t H = d->nheads, G = d->ngroups, L = d->seqlen, P = d->headdim;
+    const int64_t R = d->rank_in, O = d->rank_out;
+    d->stride_x[2] = R * P;
+    d->stride_x[1] = H * R * P;
+    d->stride_x[0] = L * H * R * P;
+    d->stride_y[2] = O * P;
+    d->stride_y[1] = H * O * P;
+    d->stride_y[0] = L * H * O * P;
+    d->stride_B[2] = R * N;
+    d->stride_B[1] = G * R * N;
+    d->stride_B[0] = L * G * R * N;
+    d->stride_C[2] = O * N;
+    d->stride_C[1] = G * O * N;
+    d->stride_C[0] = L * G * O * N;
+    d->stride_dt[2] = 1;
+    d->stride_dt[1] = H;
+    d->stride_dt[0] = L * H;
+    for (int k = 0; k < 3; ++k) d->stride_lambda[k] = d->stride_dt[k];
+}
+
+size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
+    if (validate_desc(d) != SSM_OK) return 0;
+    if (pass == SSM_PASS_FWD) return 0;
+    if (pass != SSM_PASS_BWD) return 0;
+    if (d->batch == 0 || d->seqlen == 0) return 0;
+    return bwd_layout(d).total;
+}
+
+int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, void *y,
+                 float *hT, float *last_write, void *workspace, size_t workspace_bytes,
+                 void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    (void)workspace;
+    (void)workspace_bytes;
+    if (d->batch == 0) return SSM_OK;
+    if (d->seqlen > 0) {
+        if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
+        if ((rc = check_ptr(y, "y", d->dtype_io == SSM_BF16 ? 2 : 4))) return rc;
+    }
+    ssm::Params p;
+    fill_params(d, p);
+    p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
+    p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
+    if (!ssm::simt_supported(p))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
+                    d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
+    profile_begin((cudaStream_t)stream);
+    cudaError_t e = ssm::simt_forward(p, (cudaStream_t)stream);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, const void *dy,
+                 void *dx, void *ddt, float *dA_log, float *dtheta, void *dB, void *dC,
+                 float *dD, void *dlambda, float *dh0, float *dprev_write, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(dA_log, "dA_log", 4))) return rc;
+    if (d->rank_in == d->rank_out && (rc = check_ptr(dD, "dD", 4))) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (d->batch == 0) return SSM_OK;
+    if (d->seqlen == 0) {
+        // nothing flows back through an empty sequence: zero parameter and state grads
+        cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * d->nheads * ndecay(d), st);
+        if (e == cudaSuccess && dtheta && d->n_pairs)
+            e = cudaMemsetAsync(dtheta, 0, sizeof(float) * d->nheads * d->n_pairs, st);
+        if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * d->nheads, st);
+        size_t sb = sizeof(float) * d->batch * d->nheads * nstate(d) * d->headdim;
+        if (e == cudaSuccess && dh0) e = cudaMemsetAsync(dh0, 0, sb, st);
+        if (e == cudaSuccess && dprev_write) e = cudaMemsetAsync(dprev_write, 0, sb, st);
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd (empty sequence)");
+        return SSM_OK;
+    }
+    if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
+    if ((rc = check_ptr(dy, "dy", es)) || (rc = check_ptr(dx, "dx", es)) ||
+        (rc = check_ptr(ddt, "ddt", es)) || (rc = check_ptr(dB, "dB", es)) ||
+        (rc = check_ptr(dC, "dC", es)))
+        return rc;
+    if (d->n_pairs > 0 && (rc = check_ptr(dtheta, "dtheta", 4))) return rc;
+    if (dlambda && ((uintptr_t)dlambda % es)) return fail(SSM_ERR_ALIGN, "dlambda misaligned");
+    const BwdWs lay = bwd_layout(d);
+    if (!workspace || workspace_bytes < lay.total)
+        return fail(SSM_ERR_WORKSPACE, "backward needs %zu bytes of workspace, got %zu",
+                    lay.total, workspace ? workspace_bytes : (size_t)0);
+    if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+    ssm::Params p;
+    fill_params(d, p);
+    p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
+    p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.dy = dy;
+    p.dx = dx; p.ddt = ddt; p.dA_log = dA_log; p.dtheta = dtheta; p.dBm = dB; p.dCm = dC;
+    p.dD = dD; p.dlam = d->two_endpoint ? dlambda : nullptr; p.dh0 = dh0; p.dw0 = dprev_write;
+    char *ws = (char *)workspace;
+    p.ws_dC = (float *)(ws + lay.off_dC);
+    p.ws_gbu = (float *)(ws + lay.off_gbu);
+    p.ws_tok = (float *)(ws + lay.off_tok);
+    p.ws_M2 = (float *)(ws + lay.off_M2);
+    p.ws_par = (float *)(ws + lay.off_par);
+    if (!ssm::simt_supported(p))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
+                    d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
+    // dD is written by the parameter pass; keep it defined when R != O
+    profile_begin(st);
+    cudaError_t e = ssm::simt_backward(p, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+const char *ssm_scan_last_error(void) { return g_last_error.c_str(); }
+
+int ssm_scan_poll_device_error(void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_poll_device_error");
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, ssm_device_error_word, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_poll_device_error (read)");
+    if (word != 0) {
+        int zero = 0;
+        cudaMemcpyToSymbol(ssm_device_error_word, &zero, sizeof(int));
+        return fail(SSM_ERR_TIMEOUT, "a bounded device-side wait gave up (code %d)", word);
+    }
+    return SSM_OK;
+}
+
+int ssm_scan_abi_version(void) { return SSM_SCAN_ABI_VERSION; }
+
+int ssm_scan_profile_start(int max_launches) {
+    if (max_launches < 1) return fail(SSM_ERR_ARG, "max_launches must be >= 1");
+    if (g_prof.active) return fail(SSM_ERR_ARG, "a profiling session is already open");
+    g_prof = ProfileSession();
+    const size_t n = (size_t)max_launches + 64;
+    g_prof.pool.resize(n);
+    for (size_t i = 0; i < n; ++i) {
+        cudaError_t e = cudaEventCreate(&g_prof.pool[i]);
+        if (e != cudaSuccess) {
+            for (size_t k = 0; k < i; ++k) cudaEventDestroy(g_prof.pool[k]);
+            g_prof = ProfileSession();
+            return cuda_fail(e, "ssm_scan_profile_start");
+        }
+    }
+    g_prof.active = true;
+    return SSM_OK;
+}
+
+int ssm_scan_profile_stop(char *names, int name_len, int *counts, double *total_ms,
+                          int max_kernels) {
+    if (!g_prof.active) return fail(SSM_ERR_ARG, "no profiling session is open");
+    int rc = SSM_OK;
+    std::vector<std::string> seen;
+    std::vector<int> cnt;
+    std::vector<double> tot;
+    if (g_prof.used > 0) {
+        cudaError_t e = cudaEventSynchronize(g_prof.pool[g_prof.used - 1]);
+        if (e != cudaSuccess) rc = cuda_fail(e, "ssm_scan_profile_stop");
+    }
+    if (rc == SSM_OK) {
+        for (const ProfileRec &r : g_prof.recs) {
+            float ms = 0.f;
+            cudaError_t e = cudaEventElapsedTime(&ms, g_prof.pool[r.ev0], g_prof.pool[r.ev1]);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e, "ssm_scan_profile_stop (elapsed)");
+                break;
+            }
+            size_t k = 0;
+            while (k < seen.size() && seen[k] != r.name) ++k;
+            if (k == seen.size()) {
+                seen.push_back(r.name);
+                cnt.push_back(0);
+                tot.push_back(0.0);
+            }
+            cnt[k] += 1;
+            tot[k] += ms;
+        }
+    }
+    for (cudaEvent_t ev : g_prof.pool) cudaEventDestroy(ev);
+    g_prof = ProfileSession();
+    if (rc != SSM_OK) return rc;
+    int n = (int)seen.size() < max_kernels ? (int)seen.size() : max_kernels;
+    for (int i = 0; i < n; ++i) {
+        if (names && name_len > 0) {
+            strncpy(names + (size_t)i * name_len, seen[i].c_str(), name_len - 1);
+            names[(size_t)i * name_len + name_len - 1] = 0;
+        }
+        if (counts) counts[i] = cnt[i];
+        if (total_ms) total_ms[i] = tot[i];
+    }
+    return n;
+}
+
+}  // extern "C"

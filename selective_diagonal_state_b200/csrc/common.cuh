@@ -1,0 +1,146 @@
+// Shared definitions of the sm_100a selective-diagonal-scan kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Thread/row geometry of the SIMT scan kernels (chosen on the host).
+//  PP: padded head dim (power of two, lanes over p)   NQ: row-groups per head
+//  HC: heads per CTA    T: tokens staged in shared memory per block
+struct Geometry {
+    int PP, NQ, HC, T;
+};
+
+struct Params {
+    // sizes
+    int Bsz, L, H, P, G, nr, np, N, R, O, ndec, hpg;
+    int two_ep, per_coord, bf16;
+    // element strides (batch, time, head-or-group)
+    long long sx[3], sy[3], sB[3], sC[3], sdt[3], slam[3];
+    // inputs
+    const void *x, *dt, *Bm, *Cm, *lam, *dy;
+    const float *A_log, *theta, *D, *h0, *w0;
+    // forward outputs
+    void *y;
+    float *hT, *wT;
+    // backward outputs
+    void *dx, *ddt, *dBm, *dCm, *dlam;
+    float *dA_log, *dtheta, *dD, *dh0, *dw0;
+    // backward workspace (fp32)
+    float *ws_dC;   // [B][L][H][O][N]   per-head dC_t = dy_t H_t^T
+    float *ws_gbu;  // [B][L][H][R][N]   sum_p Gbar_t[n,p] u_t[r,p]
+    float *ws_tok;  // [B][L][H][2]      (dsigma_t, <dy_t, C_t W_t>)
+    float *ws_M2;   // [B][L][H][O][R]   <dy_t[o,:], u_t[r,:]>
+    float *ws_par;  // [B][H][NPAR]      per-unit partials of dA, dtheta, dD, dbeta_0
+    Geometry geo;
+};
+
+// per-unit partial slots in ws_par
+__host__ __device__ inline int npar_of(const Params &p) { return p.ndec + p.np + 2; }
+
+__device__ __forceinline__ float ld_io(const void *ptr, long long i, int bf16) {
+    if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(ptr)[i]);
+    return reinterpret_cast<const float *>(ptr)[i];
+}
+__device__ __forceinline__ void st_io(void *ptr, long long i, float v, int bf16) {
+    if (bf16)
+        reinterpret_cast<__nv_bfloat16 *>(ptr)[i] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float *>(ptr)[i] = v;
+}
+
+__device__ __forceinline__ long long ix_x(const Params &p, int b, int t, int h, int r, int q) {
+    return b * p.sx[0] + t * p.sx[1] + h * p.sx[2] + (long long)r * p.P + q;
+}
+__device__ __forceinline__ long long ix_y(const Params &p, int b, int t, int h, int o, int q) {
+    return b * p.sy[0] + t * p.sy[1] + h * p.sy[2] + (long long)o * p.P + q;
+}
+__device__ __forceinline__ long long ix_B(const Params &p, int b, int t, int g, int r, int n) {
+    return b * p.sB[0] + t * p.sB[1] + g * p.sB[2] + (long long)r * p.N + n;
+}
+__device__ __forceinline__ long long ix_C(const Params &p, int b, int t, int g, int o, int n) {
+    return b * p.sC[0] + t * p.sC[1] + g * p.sC[2] + (long long)o * p.N + n;
+}
+__device__ __forceinline__ long long ix_dt(const Params &p, int b, int t, int h) {
+    return b * p.sdt[0] + t * p.sdt[1] + h * p.sdt[2];
+}
+__device__ __forceinline__ long long ix_lam(const Params &p, int b, int t, int h) {
+    return b * p.slam[0] + t * p.slam[1] + h * p.slam[2];
+}
+__device__ __forceinline__ long long ix_st(const Params &p, int b, int h, int n, int q) {
+    return (((long long)b * p.H + h) * p.N + n) * p.P + q;
+}
+// dense per-head workspace [B][L][H][K][N]
+__device__ __forceinline__ long long ix_wsk(const Params &p, int b, int t, int h, int k, int K,
+                                            int n) {
+    return ((((long long)b * p.L + t) * p.H + h) * K + k) * p.N + n;
+}
+__device__ __forceinline__ long long ix_bth(const Params &p, int b, int t, int h) {
+    return ((long long)b * p.L + t) * p.H + h;
+}
+
+// decay slot of state row n: per-head mode has one slot; per-coordinate mode
+// has one per real row followed by one per rotation pair
+__device__ __forceinline__ int dec_slot(const Params &p, int n) {
+    if (!p.per_coord) return 0;
+    return n < p.nr ? n : p.nr + (n - p.nr) / 2;
+}
+
+// Slot layout: thread-row-group q owns NS = NR + 2*NPR consecutive slots:
+// real rows q, q+NQ, ... (NR of them) then pairs q, q+NQ, ... as (re, im).
+// slot_of maps a state row to its slot index in [0, NQ*NS).
+template <int NR, int NPR>
+__device__ __forceinline__ int slot_of(int n, int nr, int NQ) {
+    constexpr int NS = NR + 2 * NPR;
+    if (n < nr) return (n % NQ) * NS + n / NQ;
+    int j = (n - nr) >> 1, c = (n - nr) & 1;
+    return (j % NQ) * NS + NR + 2 * (j / NQ) + c;
+}
+// inverse: state row of slot s within group q (or -1 for a padding slot)
+template <int NR, int NPR>
+__device__ __forceinline__ int row_of(int q, int s, int nr, int np, int NQ) {
+    if (s < NR) {
+        int n = q + s * NQ;
+        return n < nr ? n : -1;
+    }
+    int j = q + ((s - NR) >> 1) * NQ, c = (s - NR) & 1;
+    return j < np ? nr + 2 * j + c : -1;
+}
+
+// Sum each of K register values over the S lanes that share everything but p
+// (S = 1, 16 or 32 consecutive lanes).  Afterwards, for K >= S lane l holds
+// the totals of values [l*K/S, (l+1)*K/S) in v[0..K/S); for K < S lane l holds
+// the total of value l/(S/K) in v[0].
+template <int K, int S>
+__device__ __forceinline__ void xreduce(float (&v)[K], int lane) {
+    if constexpr (S > 1) {
+        constexpr unsigned FULL = 0xffffffffu;
+        int cur = K;
+#pragma unroll
+        for (int m = S / 2; m >= 1; m >>= 1) {
+            if (cur > 1) {
+                const bool up = (lane & m) != 0;
+                const int hlf = cur / 2;
+#pragma unroll
+                for (int i = 0; i < K / 2; ++i) {
+                    if (i < hlf) {
+                        float send = up ? v[i] : v[i + hlf];
+                        float keep = up ? v[i + hlf] : v[i];
+                        v[i] = keep + __shfl_xor_sync(FULL, send, m);
+                    }
+                }
+                cur = hlf;
+            } else {
+                v[0] += __shfl_xor_sync(FULL, v[0], m);
+            }
+        }
+    }
+}
+
+// Timing hook (defined in abi.cu): call right after every kernel launch with
+// the kernel's name.
+void profile_mark(cudaStream_t st, const char *name);
+
+}  // namespace ssm

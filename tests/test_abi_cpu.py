@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/ssm_scan.h declares, and rejects bad arguments before
+any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_diagonal_state_b200 import abi, build
+from selective_diagonal_state_b200 import synthetic as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"SSM_API\s+[\w\s\*]+?\b(ssm_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    syms = set(declared_symbols())
+    assert {"ssm_scan_fwd", "ssm_scan_bwd", "ssm_scan_workspace_size",
+            "ssm_scan_last_error"} <= syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(abi.EXPORTED) >= set(declared_symbols())
+
+
+def test_abi_version(lib):
+    assert abi.ssm_scan_abi_version() == 1
+
+
+def test_contiguous_strides(lib):
+    sh = S.WORKLOADS["ssd_mimo_r4"]
+    d = abi.make_desc(sh)
+    N, P, R, O, H, G, L = sh.nstate, sh.headdim, sh.rank_in, sh.rank_out, sh.nheads, sh.ngroups, sh.seqlen
+    assert list(d.stride_x) == [L * H * R * P, H * R * P, R * P]
+    assert list(d.stride_y) == [L * H * O * P, H * O * P, O * P]
+    assert list(d.stride_B) == [L * G * R * N, G * R * N, R * N]
+    assert list(d.stride_C) == [L * G * O * N, G * O * N, O * N]
+    assert list(d.stride_dt) == [L * H, H, 1]
+
+
+def test_workspace_size(lib):
+    sh = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=100)
+    d = abi.make_desc(sh)
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+    n = abi.ssm_scan_workspace_size(d, abi.PASS_BWD)
+    BLH = 2 * 100 * 32
+    assert n >= BLH * (2 * 128 + 2 + 1) * 4
+    assert n % 256 == 0
+    bad = abi.make_desc(sh)
+    bad.ngroups = 5
+    assert abi.ssm_scan_workspace_size(bad, abi.PASS_BWD) == 0
+
+
+def _fwd_status(lib, d, **ptrs):
+    names = ["x", "dt", "A_log", "theta", "B", "C", "D", "lam", "h0", "w0", "y", "hT", "wT", "ws"]
+    args = [ptrs.get(n) for n in names]
+    return lib.ssm_scan_fwd(ctypes.byref(d) if d is not None else None, *args, 0, None)
+
+
+FAKE = 1 << 40  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("mutate,code", [
+    (lambda d: setattr(d, "ngroups", 5), -1),
+    (lambda d: setattr(d, "nheads", 0), -1),
+    (lambda d: setattr(d, "decay_mode", 7), -1),
+    (lambda d: setattr(d, "dtype_io", 3), -1),
+    (lambda d: setattr(d, "two_endpoint", 2), -1),
+    (lambda d: (setattr(d, "n_real", 0), setattr(d, "n_pairs", 0)), -1),
+    (lambda d: d.stride_x.__setitem__(1, -4), -1),
+    (lambda d: setattr(d, "batch", 70000), -2),
+])
+def test_bad_descriptor_rejected(lib, mutate, code):
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"])
+    mutate(d)
+    full = dict(x=FAKE, dt=FAKE, A_log=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, lam=FAKE, y=FAKE)
+    assert _fwd_status(lib, d, **full) == code
+    assert lib.ssm_scan_last_error().decode()
+
+
+def test_null_descriptor(lib):
+    assert _fwd_status(lib, None) == -1
+
+
+@pytest.mark.parametrize("missing", ["x", "dt", "A_log", "theta", "B", "C", "D", "lam", "y"])
+def test_missing_pointer_rejected(lib, missing):
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"])
+    full = dict(x=FAKE, dt=FAKE, A_log=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, lam=FAKE, y=FAKE)
+    full[missing] = None
+    assert _fwd_status(lib, d, **full) == -1
+    assert missing in lib.ssm_scan_last_error().decode()
+
+
+def test_misaligned_pointer_rejected(lib):
+    d = abi.make_desc(S.WORKLOADS["mamba2_siso"])
+    full = dict(x=FAKE + 1, dt=FAKE, A_log=FAKE, B=FAKE, C=FAKE, D=FAKE, y=FAKE)
+    assert _fwd_status(lib, d, **full) == -3
+
+
+def test_backward_needs_workspace(lib):
+    d = abi.make_desc(S.WORKLOADS["hybridmamba"].replace(batch=1, seqlen=8))
+    p = [FAKE] * 22
+    rc = lib.ssm_scan_bwd(ctypes.byref(d), *p, 0, None)
+    assert rc == -6
+    assert "workspace" in lib.ssm_scan_last_error().decode()
+
+
+def test_unsupported_rank_reported(lib):
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(rank_in=8, rank_out=8))
+    full = dict(x=FAKE, dt=FAKE, A_log=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, lam=FAKE, y=FAKE)
+    assert _fwd_status(lib, d, **full) == -2
+
+
+def test_host_tensor_refused():
+    torch = pytest.importorskip("torch")
+    with pytest.raises(ValueError):
+        abi._ptr(torch.zeros(3))

@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA scan (through the C ABI) against the fp64 oracle, element
+by element, on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import oracle
+from selective_diagonal_state_b200 import abi, scan
+from selective_diagonal_state_b200 import synthetic as S
+from tests.parity_util import compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from selective_diagonal_state_b200 import build
+    build.build()
+    abi.load_library()
+    assert torch.cuda.is_available()
+
+
+def run_gpu(shape, inp, backward=True):
+    dev = scan.to_device(shape, inp)
+    y, hT, wT = scan.scan_forward(shape, dev)
+    g = scan.scan_backward(shape, dev) if backward else None
+    torch.cuda.synchronize()
+    abi.ssm_scan_poll_device_error()
+    return y, hT, wT, g
+
+
+def check_all(shape, inp, backward=True, report=None):
+    y, hT, wT, g = run_gpu(shape, inp, backward)
+    ref = oracle.scan_fwd(shape, inp)
+    dt = shape.dtype_io
+    compare("y", to_np(y), ref["y"], dt, report)
+    compare("hT", to_np(hT), ref["hT"], dt, report)
+    compare("last_write", to_np(wT), ref["wT"], dt, report)
+    if not backward:
+        return
+    gr = oracle.scan_bwd(shape, inp, inp["dy"])
+    compare("dx", to_np(g.dx), gr["dx"], dt, report)
+    compare("ddt", to_np(g.ddt), gr["ddt"], dt, report)
+    compare("dB", to_np(g.dBm), gr["dBm"], dt, report)
+    compare("dC", to_np(g.dCm), gr["dCm"], dt, report)
+    compare("dA_log", to_np(g.dA_log), gr["dA_log"], dt, report)
+    if shape.rank_in == shape.rank_out:
+        compare("dD", to_np(g.dD), gr["dD"], dt, report)
+    if shape.n_pairs:
+        compare("dtheta", to_np(g.dtheta), gr["dtheta"], dt, report)
+    if shape.two_endpoint:
+        compare("dlambda", to_np(g.dlam), gr["dlam"], dt, report)
+    compare("dh0", to_np(g.dh0), gr["dh0"], dt, report)
+    compare("dprev_write", to_np(g.dw0), gr["dw0"], dt, report)
+
+
+# Reduced copies of the five workloads: same heads/state/rank/group structure,
+# fewer tokens (not a multiple of the 16/32-token staging tile) so the oracle
+# finishes in seconds.
+REDUCED = {
+    "tiny_hybrid_fp32": dict(),
+    "mamba2_siso": dict(batch=2, seqlen=203),
+    "mamba1_siso": dict(batch=2, seqlen=157),
+    "hybridmamba": dict(batch=2, seqlen=181),
+    "ssd_mimo_r4": dict(batch=1, seqlen=133),
+}
+
+
+@pytest.mark.parametrize("name", S.WORKLOAD_ORDER)
+def test_workload_parity(name):
+    shape = S.WORKLOADS[name].replace(**REDUCED[name])
+    inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(name))
+    check_all(shape, inp)
+
+
+@pytest.mark.parametrize("name", S.WORKLOAD_ORDER)
+def test_workload_parity_with_state(name):
+    shape = S.WORKLOADS[name].replace(**REDUCED[name]).replace(seqlen=37)
+    inp = S.make_inputs(shape, seed=100 + S.WORKLOAD_ORDER.index(name), with_state=True)
+    check_all(shape, inp)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=1),
+    dict(seqlen=2),
+    dict(seqlen=33, n_real=0, n_pairs=5),
+    dict(seqlen=47, n_real=7, n_pairs=0),
+    dict(seqlen=20, decay_mode=S.DECAY_PER_HEAD),
+    dict(seqlen=29, rank_in=3, rank_out=3, ngroups=1),
+    dict(seqlen=29, rank_in=2, rank_out=1),
+    dict(seqlen=25, headdim=5, nheads=4, ngroups=2),
+    dict(seqlen=25, headdim=48, nheads=3, ngroups=1),
+    dict(seqlen=64, headdim=128, n_real=32, n_pairs=16, nheads=2),
+])
+@pytest.mark.parametrize("dtype", [S.DTYPE_F32, S.DTYPE_BF16])
+def test_edge_shapes(kw, dtype):
+    base = dict(batch=2, seqlen=16, nheads=2, headdim=16, ngroups=2, n_real=8, n_pairs=4,
+                decay_mode=S.DECAY_PER_COORD, two_endpoint=1, dtype_io=dtype)
+    base.update(kw)
+    shape = S.ScanShape(**base)
+    inp = S.make_inputs(shape, seed=7, with_state=True)
+    check_all(shape, inp)
+
+
+def test_empty_sequence():
+    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=0)
+    inp = S.make_inputs(shape, seed=1, with_state=True)
+    dev = scan.to_device(shape, inp)
+    y, hT, wT = scan.scan_forward(shape, dev)
+    torch.cuda.synchronize()
+    assert y.numel() == 0
+    np.testing.assert_array_equal(to_np(hT), inp["h0"])
+    np.testing.assert_array_equal(to_np(wT), inp["w0"])
+    g = scan.scan_backward(shape, dev)
+    torch.cuda.synchronize()
+    assert float(g.dA_log.abs().max()) == 0.0 and float(g.dh0.abs().max()) == 0.0
+
+
+def test_carry_continuation_on_gpu():
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=1, seqlen=90, dtype_io=S.DTYPE_F32)
+    inp = S.make_inputs(shape, seed=3)
+    full = scan.scan_forward(shape, scan.to_device(shape, inp))
+    L1 = 41
+    cut = lambda a, sl: a[:, sl] if a is not None else None  # noqa: E731
+    part = {k: (cut(v, slice(0, L1)) if k in ("x", "dt", "lam", "Bm", "Cm", "dy") else v)
+            for k, v in inp.items()}
+    s1 = shape.replace(seqlen=L1)
+    y1, h1, w1 = scan.scan_forward(s1, scan.to_device(s1, part))
+    rest = {k: (cut(v, slice(L1, None)) if k in ("x", "dt", "lam", "Bm", "Cm", "dy") else v)
+            for k, v in inp.items()}
+    s2 = shape.replace(seqlen=shape.seqlen - L1)
+    dev2 = scan.to_device(s2, rest)
+    dev2.h0, dev2.w0 = h1, w1
+    y2, h2, _ = scan.scan_forward(s2, dev2)
+    torch.cuda.synchronize()
+    yc = torch.cat([y1, y2], 1)
+    assert float((yc - full[0]).abs().max()) <= 1e-5 * float(full[0].abs().max())
+    assert float((h2 - full[1]).abs().max()) <= 1e-5 * float(full[1].abs().max())
+
+
+def test_strided_views():
+    """x / y / B / C as head-strided views of wider buffers give the dense result."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=40, nheads=4, ngroups=2,
+                                                dtype_io=S.DTYPE_F32)
+    inp = S.make_inputs(shape, seed=11)
+    dev = scan.to_device(shape, inp)
+    y_ref, _, _ = scan.scan_forward(shape, dev)
+    d = abi.make_desc(shape)
+
+    def widen(t, extra):
+        big = torch.zeros(*t.shape[:3], t.shape[3] * t.shape[4] + extra, dtype=t.dtype,
+                          device=t.device)
+        big[..., : t.shape[3] * t.shape[4]] = t.reshape(*t.shape[:3], -1)
+        return big
+
+    xb, Bb, Cb = widen(dev.x, 24), widen(dev.Bm, 8), widen(dev.Cm, 40)
+    yb = torch.zeros(*y_ref.shape[:3], y_ref.shape[3] * y_ref.shape[4] + 16, device="cuda")
+    for arr, big in (("stride_x", xb), ("stride_B", Bb), ("stride_C", Cb), ("stride_y", yb)):
+        st = getattr(d, arr)
+        st[0], st[1], st[2] = big.stride(0), big.stride(1), big.stride(2)
+    y = torch.zeros_like(y_ref)
+    abi.ssm_scan_fwd(d, xb, dev.dt, dev.A_log, dev.theta, Bb, Cb, dev.D, dev.lam, None, None, yb)
+    torch.cuda.synchronize()
+    got = yb[..., : y_ref.shape[3] * y_ref.shape[4]].reshape(y_ref.shape)
+    assert float((got - y_ref).abs().max()) == 0.0
+
+
+def test_backward_deterministic():
+    shape = S.WORKLOADS["mamba2_siso"].replace(batch=2, seqlen=64)
+    inp = S.make_inputs(shape, seed=5)
+    dev = scan.to_device(shape, inp)
+    g1 = scan.scan_backward(shape, dev)
+    a = [t.clone() for t in (g1.dx, g1.ddt, g1.dBm, g1.dCm, g1.dA_log, g1.dD)]
+    g2 = scan.scan_backward(shape, dev)
+    torch.cuda.synchronize()
+    for x1, x2 in zip(a, (g2.dx, g2.ddt, g2.dBm, g2.dCm, g2.dA_log, g2.dD)):
+        assert torch.equal(x1, x2)
