@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target wall time of the bounded oracle sample")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch size (small cases for profiling only)")
     return ap.parse_args()
 
 
@@ -269,6 +271,8 @@ def main():
                                 device_id=torch.device("cuda", local))
     abi.load_library()
     shape = S.WORKLOADS[args.workload]
+    if args.batch:
+        shape = shape.replace(batch=args.batch)
     inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1000 * rank)
     dev = scan.to_device(shape, inp)
     desc = abi.make_desc(shape)
