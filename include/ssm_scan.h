@@ -139,6 +139,38 @@ SSM_API int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, con
                  float *dD, void *dlambda, float *dh0, float *dprev_write, void *workspace,
                  size_t workspace_bytes, void *stream);
 
+/*
+ * Allocation-free backward (no counterpart in the paper; a library service).
+ * Same inputs, outputs and results as ssm_scan_bwd, but it takes no
+ * workspace: its scratch is a fixed 32 MiB array inside the library
+ * (SSM_NOALLOC_SCRATCH_BYTES), which every GPU that loads the library keeps
+ * until the process exits.  It is meant for callers that cannot or must not
+ * call cudaMalloc themselves -- for example code running inside a host
+ * framework that owns all device memory through its own pool, or a
+ * latency-critical path where allocating (and the synchronisation a later
+ * cudaFree brings) is not allowed.  The call itself allocates nothing.
+ *
+ *  - Problems whose backward workspace (ssm_scan_workspace_size with
+ *    SSM_PASS_BWD) exceeds SSM_NOALLOC_SCRATCH_BYTES are rejected with
+ *    SSM_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current (a one-time set-up per device); make that first
+ *    call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents.  Nothing in it has to start at zero (every scratch byte the
+ *    backward reads is written earlier in the same call), but calls whose
+ *    kernels overlap on the GPU (different streams, or several host threads)
+ *    race on it: serialise them.
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (32u << 20)
+SSM_API int ssm_scan_bwd_noalloc(const ssm_desc_t *d, const void *x, const void *dt,
+                                 const float *A_log, const float *theta, const void *B,
+                                 const void *C, const float *D, const void *lambda,
+                                 const float *h0, const float *prev_write, const void *dy,
+                                 void *dx, void *ddt, float *dA_log, float *dtheta, void *dB,
+                                 void *dC, float *dD, void *dlambda, float *dh0,
+                                 float *dprev_write, void *stream);
+
 /* Message describing the last failing call on this host thread ("" if none). */
 SSM_API const char *ssm_scan_last_error(void);
 

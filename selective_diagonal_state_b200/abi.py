@@ -23,7 +23,9 @@ PASS_FWD, PASS_BWD = 0, 1
 
 EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
-            "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop"]
+            "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
+            "ssm_scan_bwd_noalloc"]
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class SsmError(RuntimeError):
@@ -69,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_scan_fwd.restype = ctypes.c_int
     lib.ssm_scan_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 22 + [ctypes.c_size_t, _vp]
     lib.ssm_scan_bwd.restype = ctypes.c_int
+    lib.ssm_scan_bwd_noalloc.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 21 + [_vp]
+    lib.ssm_scan_bwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_last_error.argtypes = []
     lib.ssm_scan_last_error.restype = ctypes.c_char_p
     lib.ssm_scan_poll_device_error.argtypes = [_vp]
@@ -144,6 +148,18 @@ def ssm_scan_bwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, 
         x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt, dA_log, dtheta, dB, dC,
         dD, dlam, dh0, dprev_write, workspace)], workspace_bytes, _stream(stream))
     _check(rc, "ssm_scan_bwd")
+
+
+def ssm_scan_bwd_noalloc(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx,
+                         ddt, dA_log, dtheta, dB, dC, dD, dlam=None, dh0=None, dprev_write=None,
+                         stream=None) -> None:
+    """Backward without a workspace argument: the library's fixed device
+    scratch is used instead (for callers that cannot allocate device memory)."""
+    lib = load_library()
+    rc = lib.ssm_scan_bwd_noalloc(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt, dA_log, dtheta, dB, dC,
+        dD, dlam, dh0, dprev_write)], _stream(stream))
+    _check(rc, "ssm_scan_bwd_noalloc")
 
 
 def ssm_scan_poll_device_error(stream=None) -> None:

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -384,4 +385,58 @@ int ssm_scan_profile_stop(char *names, int name_len, int *counts, double *total_
     return n;
 }
 
+
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward: the scratch lives in this fixed device array.
+// Host code only ever sees the array's host-side shadow symbol, so its device
+// address is looked up once per device (with that device current) and passed
+// to the kernels as an ordinary pointer.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SSM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices];
+
+int noalloc_scratch(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd_noalloc (cudaGetDevice)");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SSM_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return cuda_fail(e, "ssm_scan_bwd_noalloc (cudaGetSymbolAddress)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SSM_OK;
+}
+}  // namespace
+
+extern "C" int ssm_scan_bwd_noalloc(const ssm_desc_t *d, const void *x, const void *dt,
+                                    const float *A_log, const float *theta, const void *B,
+                                    const void *C, const float *D, const void *lambda,
+                                    const float *h0, const float *prev_write, const void *dy,
+                                    void *dx, void *ddt, float *dA_log, float *dtheta, void *dB,
+                                    void *dC, float *dD, void *dlambda, float *dh0,
+                                    float *dprev_write, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    const size_t need = ssm_scan_workspace_size(d, SSM_PASS_BWD);
+    if (need > (size_t)SSM_NOALLOC_SCRATCH_BYTES)
+        return fail(SSM_ERR_WORKSPACE,
+                    "ssm_scan_bwd_noalloc: this problem needs %zu bytes of scratch; the built-in "
+                    "scratch holds %u bytes (use ssm_scan_bwd with a caller workspace)",
+                    need, (unsigned)SSM_NOALLOC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    return ssm_scan_bwd(d, x, dt, A_log, theta, B, C, D, lambda, h0, prev_write, dy, dx, ddt,
+                        dA_log, dtheta, dB, dC, dD, dlambda, dh0, dprev_write, scratch,
+                        SSM_NOALLOC_SCRATCH_BYTES, stream);
+}
