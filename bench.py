@@ -85,7 +85,7 @@ def kernel_bytes(shape, name: str) -> int:
     t = tensor_bytes(shape)
     BLH = s.batch * s.seqlen * s.nheads
     ins = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
-    if name == "k_fwd":
+    if name in ("k_fwd", "k_chunk_fwd"):
         return ins + t["y"]
     if name == "k_bwd_sweep1":   # inputs + dy -> per-head dC (fp32)
         return ins + t["y"] + BLH * s.rank_out * s.nstate * 4

@@ -88,7 +88,10 @@ typedef struct ssm_desc {
     int64_t batch, seqlen, nheads, headdim, ngroups;
     int32_t n_real, n_pairs;
     int32_t rank_in, rank_out;  /* R, O; SISO is 1, 1 */
-    int32_t chunk;              /* tuning hint only (0 = library choice); results do not depend on it beyond rounding */
+    int32_t chunk;              /* kernel choice, results equal up to rounding: 0 = library choice,
+                                   1 = token-by-token recurrent kernels, 64 = 64-token chunked
+                                   tensor-core kernels where supported (bf16, headdim 64,
+                                   rank 1, 64 or 128 state rows) */
     int32_t decay_mode;         /* enum ssm_decay_mode */
     int32_t two_endpoint;       /* 0: lambda not read (lam = 1); 1: lambda used */
     int32_t dtype_io;           /* enum ssm_dtype of x, dt, B, C, lambda, y and of their gradients */

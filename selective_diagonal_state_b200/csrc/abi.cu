@@ -15,10 +15,10 @@ namespace ssm {
 bool simt_supported(const Params &p);
 cudaError_t simt_forward(const Params &p, cudaStream_t st);
 cudaError_t simt_backward(const Params &p, cudaStream_t st);
+bool chunk_fwd_supported(const Params &p);
+cudaError_t chunk_forward(const Params &p, cudaStream_t st);
+int chunk_error_take();
 }  // namespace ssm
-
-// Device word raised by bounded waits inside kernels (0 = no error).
-__device__ int ssm_device_error_word;
 
 namespace {
 
@@ -232,11 +232,14 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     fill_params(d, p);
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
     p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
-    if (!ssm::simt_supported(p))
+    // chunk == 1 asks for the token-by-token recurrent kernels
+    const bool chunked = d->chunk != 1 && ssm::chunk_fwd_supported(p);
+    if (!chunked && !ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
     profile_begin((cudaStream_t)stream);
-    cudaError_t e = ssm::simt_forward(p, (cudaStream_t)stream);
+    cudaError_t e = chunked ? ssm::chunk_forward(p, (cudaStream_t)stream)
+                            : ssm::simt_forward(p, (cudaStream_t)stream);
     profile_end();
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
     g_last_error.clear();
@@ -309,14 +312,10 @@ const char *ssm_scan_last_error(void) { return g_last_error.c_str(); }
 int ssm_scan_poll_device_error(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_poll_device_error");
-    int word = 0;
-    e = cudaMemcpyFromSymbol(&word, ssm_device_error_word, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_poll_device_error (read)");
-    if (word != 0) {
-        int zero = 0;
-        cudaMemcpyToSymbol(ssm_device_error_word, &zero, sizeof(int));
-        return fail(SSM_ERR_TIMEOUT, "a bounded device-side wait gave up (code %d)", word);
-    }
+    const int word = ssm::chunk_error_take();
+    if (word < 0) return fail(SSM_ERR_CUDA, "ssm_scan_poll_device_error: cannot read the error word");
+    if (word == 1) return fail(SSM_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    if (word != 0) return fail(SSM_ERR_TIMEOUT, "device-side error code %d", word);
     return SSM_OK;
 }
 

@@ -1,0 +1,670 @@
+// Chunked tensor-core forward scan for sm_100a (bf16 I/O, fp32 state, SISO,
+// head dim 64, up to 128 state rows).
+//
+// The state-mediated kernel of the scan is masked linear attention ("When a
+// Diagonal State Is Not Enough", sungsoo.github.io Part 03, Thm 24): within a
+// chunk, y_t = sum_{s<=t} Re(conj(c_t) Phi_{t,s} sigma_s b_s) u_s plus the
+// readout of the state carried into the chunk.  With per-coordinate decays
+// and 2x2 rotations the mask is not one scalar per (t, s), so the decay of
+// every state mode is folded into the operands around a reference point:
+//     Phi_{t,s} = exp(lam (S_t - S_ref)) exp(lam (S_ref - S_s)),  lam = a + i theta
+// (the fixed-basis diagonal structure of Thm 8).  References are the starts of
+// 16-token sub-blocks, so every folded factor either decays (|f| <= 1) or
+// grows at most by exp(|a| * sum of 16 steps).
+//
+// Per chunk of Q = 64 tokens (sub-blocks i = 0..3 of 16), S_t = inclusive sum of
+// dt over the chunk, Sb_i = S at the end of sub-block i-1:
+//   Ci_t  = c_t conj(e^{lam (S_t - Sb_i)})           (t in block i)
+//   Ch_t  = c_t conj(e^{lam S_t})                     readout of the carried state
+//   Bi_s  = sigma_s b_s e^{lam (Sb_i - S_s)}          for s <= end of block i
+//   Bh_s  = sigma_s b_s e^{lam (S_63 - S_s)}          chunk-end state contribution
+// and, on the tensor cores (tcgen05, fp32 accumulators in TMEM):
+//   scores^T_i  = Bi (64 s x N) . Ci^T (N x 16 t)          M=64, N=16, K=N
+//   Y^T         = K_prev^T (64 p x N) . Ch^T (N x 64 t)    M=64, N=64, K=N
+//               + X^T (64 p x s) . P^T_i (s x 16 t)        masked scores, M=64, N=16
+//   S_chunk     = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64, K=64
+// while the carried state K_c = e^{lam S_63} K_{c-1} + S_chunk runs in fp32
+// registers (one state row per thread).  The two-endpoint write is used in the
+// pre-state form K_t = A_t K_{t-1} + sigma_t W_t, sigma_t = gamma_t + beta_{t+1},
+// with y_t = C_t K_t - beta_{t+1} (C_t . B_t) u_t + D u_t.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace ssm {
+
+// Device word raised by the bounded waits of the tensor-core kernels
+// (0 = no error; 1 = a wait gave up; 2 = an input outside the folding range).
+__device__ int ssm_chunk_error_word;
+
+namespace chunkfwd {
+
+using namespace umma;
+
+constexpr int Q = 64;
+constexpr int NSB = 4;
+constexpr int NP = 128;   // state rows (K) padded
+constexpr int PD = 64;    // head dim
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+
+// shared-memory map (bytes from a 1024-aligned base)
+constexpr uint32_t SM_X = 0;              // 2 x 8 KB   x tiles (128B-swizzled, rows = t)
+constexpr uint32_t SM_B = 16384;          // 2 x 16 KB  raw B tiles: 2 x (64 t x 64 rows), 128B-swizzled
+constexpr uint32_t SM_C = 49152;          // 2 x 16 KB  raw C tiles, same layout
+constexpr uint32_t SM_CI = 81920;         // 16 KB      Ci   K-major (64 t x 128)
+constexpr uint32_t SM_CH = 98304;         // 16 KB      Ch   K-major
+constexpr uint32_t SM_BI = 114688;        // 40 KB      Bi tiles (16, 32, 48, 64 rows)
+constexpr uint32_t SM_BH = 155648;        // 16 KB      Bh   MN-major (M = 128 rows, K = 64 t)
+constexpr uint32_t SM_P = 172032;         // 8 KB       P^T tiles, MN-major (N = 16 t, K = 64 s)
+constexpr uint32_t SM_KT = 180224;        // 16 KB      K_prev^T MN-major (M = 64 p, K = 128 rows)
+constexpr uint32_t SM_F32 = 196608;       // fp32 scratch
+// fp32 scratch (float offsets from SM_F32)
+constexpr int F_S = 0, F_SIG = 64, F_BN = 128, F_CORR = 192, F_DT = 256, F_LAM = 328;
+constexpr int F_CP = 400;                 // [4][64] corr partials
+constexpr int F_A2 = 656;                 // [128] decay * log2(e) per mode
+constexpr int F_W = 784;                  // [128] rotation frequency per mode
+constexpr int F_KRE = 912;                // [13][128] mode constants, real part
+constexpr int F_KIM = F_KRE + 13 * 128;   // [13][128] imaginary part
+constexpr int F_END = F_KIM + 13 * 128;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;   // 4 mbarriers + TMEM slot + flags
+constexpr uint32_t SMEM_USED = SM_BAR + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+
+constexpr uint32_t KM_LBO = 128, KM_SBO = 2048;  // K-major tiles with K = 128
+
+__device__ __forceinline__ uint32_t bi_off(int i) {
+    return i == 0 ? 0u : (i == 1 ? 4096u : (i == 2 ? 12288u : 24576u));
+}
+// mode-constant slots: F[i][j] = prod_{k=i}^{j-1} E_k (0 <= i < j <= 4), G[i] = conj(F[0][i])
+__device__ __forceinline__ int fslot(int i, int j) {
+    return (i == 0 ? 0 : (i == 1 ? 4 : (i == 2 ? 7 : 9))) + (j - i - 1);
+}
+__device__ __forceinline__ int gslot(int i) { return 10 + (i - 1); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void st16(unsigned char *base, uint32_t off, const float (&v)[8]) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(base + off) = w;
+}
+__device__ __forceinline__ float bf(const unsigned char *p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+}
+// 8 consecutive state rows r0..r0+7 of token t from a raw B/C tile
+// (two 64-row halves, each 64 tokens x 128 bytes with the 128-byte swizzle).
+__device__ __forceinline__ void ld_rows8(const unsigned char *tile, int t, int r0, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(tile + (r0 >> 6) * 8192 +
+                                                     off_sw128(t, r0 & 63));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(u[i] << 16);
+        v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ float ld_row1(const unsigned char *tile, int t, int r) {
+    return bf(tile + (r >> 6) * 8192 + off_sw128(t, r & 63));
+}
+__device__ __forceinline__ void raise_error(int code) { atomicCAS(&ssm_chunk_error_word, 0, code); }
+
+// complex multiply (a + ib)(c + id)
+__device__ __forceinline__ void cmul(float a, float b, float c, float d, float &re, float &im) {
+    re = fmaf(a, c, -b * d);
+    im = fmaf(a, d, b * c);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+            const __grid_constant__ CUtensorMap tmC, Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // [2]
+    uint64_t *bar_mma = bar_tma + 2;                                // [2]: phase A, phase B
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
+    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, L = p.L;
+    const int nmode = p.nr + p.np;
+    const int nchunk = (L + Q - 1) / Q;
+    const uint32_t tile_bytes = Q * PD * 2 + 2u * Q * N * 2;
+    const int nbox = N / 64;   // 64-row TMA boxes per B/C tile
+
+    // ---- set-up ------------------------------------------------------------
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        mbar_fence_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+    }
+    if (warp == 0) tmem_alloc(tslot, TMEM_COLS);
+    for (int m = tid; m < NP; m += THREADS) {
+        float a2 = 0.f, w = 0.f;
+        if (m < nmode) {
+            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
+            if (m >= nr) w = p.theta[h * p.np + (m - nr)];
+        }
+        f32[F_A2 + m] = a2;
+        f32[F_W + m] = w;
+    }
+    // padding rows of every operand stay zero
+    for (int i = tid; i < (int)((SM_F32 - SM_CI) / 16); i += THREADS)
+        reinterpret_cast<uint4 *>(sm + SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_y = tbase;                      // Y^T (M=64, lanes 0-15 of each quarter)
+    const uint32_t t_sc = tbase + (16u << 16);       // scores^T (M=64, lanes 16-31)
+    const uint32_t t_st = tbase + 64u;               // chunk state (M=128), columns 64..127
+
+    // TMA for the first two chunks
+    if (tid == 0) {
+        for (int c = 0; c < 2 && c < nchunk; ++c) {
+            mbar_expect_tx(&bar_tma[c], tile_bytes);
+            tma_load_4d(sm + SM_X + c * 8192, &tmX, &bar_tma[c], 0, h, c * Q, b);
+            for (int k = 0; k < nbox; ++k) {
+                tma_load_4d(sm + SM_B + c * 16384 + k * 8192, &tmB, &bar_tma[c], 64 * k, g, c * Q, b);
+                tma_load_4d(sm + SM_C + c * 16384 + k * 8192, &tmC, &bar_tma[c], 64 * k, g, c * Q, b);
+            }
+        }
+    }
+
+    // carried state: thread n < 128 owns state row n (64 p values, fp32)
+    float K[PD];
+    const bool chain_thr = tid < NP;
+    {
+        float beta0 = 0.f;
+        if (p.two_ep && L > 0)
+            beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+        if (chain_thr) {
+            const int n = tid;
+#pragma unroll
+            for (int q = 0; q < PD; ++q) {
+                float v = 0.f;
+                if (n < N) {
+                    if (p.h0) v = p.h0[ix_st(p, b, h, n, q)];
+                    if (p.w0) v = fmaf(beta0, p.w0[ix_st(p, b, h, n, q)], v);
+                }
+                K[q] = v;
+            }
+            // K_prev^T operand (bf16, MN-major: M = p, K = row)
+#pragma unroll
+            for (int q8 = 0; q8 < PD / 8; ++q8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
+                st16(sm + SM_KT, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
+            }
+        }
+    }
+
+    const float Dh = (p.R == p.O) ? p.D[h] : 0.f;
+    const int t_loc = tid & 63;     // token of this thread in the prep phase
+    const int grp = tid >> 6;       // row-chunk group of this thread (rows 8*(grp + 4k) ..)
+
+    for (int c = 0; c < nchunk; ++c) {
+        const int st = c & 1;
+        const int t0 = c * Q;
+        unsigned char *sX = sm + SM_X + st * 8192;
+        unsigned char *sB = sm + SM_B + st * 16384;
+        unsigned char *sC = sm + SM_C + st * 16384;
+
+        // ---- per-token quantities --------------------------------------------
+        for (int i = tid; i < Q + 1; i += THREADS) {
+            const int t = t0 + i;
+            float dv = 0.f, lv = 1.f;
+            if (t < L) {
+                dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+                if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+            }
+            f32[F_DT + i] = dv;
+            f32[F_LAM + i] = lv;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // inclusive prefix sum of dt over the chunk (two tokens per lane)
+            const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
+            float v = d0 + d1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            f32[F_S + 2 * lane] = v - d1;
+            f32[F_S + 2 * lane + 1] = v;
+        } else if (warp == 1 || warp == 2) {
+            const int t = (warp - 1) * 32 + lane;
+            const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
+            const float bn = (t0 + t + 1 < L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
+            f32[F_SIG + t] = fmaf(lv, dv, bn);
+            f32[F_BN + t] = bn;
+        }
+        // ---- wait for the chunk's tiles ---------------------------------------
+        if (!mbar_wait(&bar_tma[st], (uint32_t)((c >> 1) & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        __syncthreads();
+        if (*abort_flag) break;
+
+        // ---- per-mode chunk constants: E_k = exp(lam dS_k), their products -----
+        for (int m = tid; m < nmode; m += THREADS) {
+            const float a2 = f32[F_A2 + m], w = f32[F_W + m];
+            float er[4], ei[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
+                const float ds = f32[F_S + 16 * k + 15] - lo;
+                const float mag = exp2f(a2 * ds);
+                if (m >= nr) {
+                    float sn, cs;
+                    sincosf(w * ds, &sn, &cs);
+                    er[k] = mag * cs;
+                    ei[k] = mag * sn;
+                } else {
+                    er[k] = mag;
+                    ei[k] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float pr = 1.f, pi = 0.f;
+#pragma unroll
+                for (int j = i + 1; j <= 4; ++j) {
+                    float nr_, ni_;
+                    cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
+                    pr = nr_;
+                    pi = ni_;
+                    f32[F_KRE + fslot(i, j) * NP + m] = pr;
+                    f32[F_KIM + fslot(i, j) * NP + m] = pi;
+                    if (i == 0 && j < 4) {
+                        f32[F_KRE + gslot(j) * NP + m] = pr;
+                        f32[F_KIM + gslot(j) * NP + m] = -pi;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- operand preparation: thread (t, grp) handles rows 8*(grp + 4k) ---
+        {
+            const int t = t_loc;
+            const int ib = t >> 4;
+            const float St = f32[F_S + t];
+            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+            const float ds = St - Sb;
+            const float sig = f32[F_SIG + t];
+            float corr = 0.f;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const int r0 = 8 * (grp + 4 * k);
+                if (r0 >= N) break;
+                float vCI[8], vCH[8], vBI[8], vBH[8], vBX[3][8], rc[8], rb[8];
+                ld_rows8(sC, t, r0, rc);
+                ld_rows8(sB, t, r0, rb);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int r = r0 + j;
+                    // two rows at a time: real rows r, r+1 or one pair (re, im)
+                    const float c0 = rc[j], c1 = rc[j + 1];
+                    const float b0 = rb[j], b1 = rb[j + 1];
+                    corr = fmaf(c0, b0, fmaf(c1, b1, corr));
+                    float ci0, ci1, bi0, bi1;     // folded Ci, own-block Bi
+                    int m0, m1;
+                    bool pair;
+                    if (r < nr) {
+                        pair = false;
+                        m0 = r;
+                        m1 = r + 1;
+                        const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
+                        ci0 = c0 * exp2f(x0);
+                        ci1 = c1 * exp2f(x1);
+                        bi0 = sig * b0 * exp2f(fminf(-x0, 120.f));
+                        bi1 = sig * b1 * exp2f(fminf(-x1, 120.f));
+                    } else {
+                        pair = true;
+                        m0 = m1 = nr + ((r - nr) >> 1);
+                        const float x = f32[F_A2 + m0] * ds;
+                        float sn, cs;
+                        sincosf(f32[F_W + m0] * ds, &sn, &cs);
+                        // rotate by cis(-phi): (u + iv)(cs - i sn)
+                        const float ec = exp2f(x), eb = sig * exp2f(fminf(-x, 120.f));
+                        ci0 = ec * fmaf(c0, cs, c1 * sn);
+                        ci1 = ec * fmaf(c1, cs, -c0 * sn);
+                        bi0 = eb * fmaf(b0, cs, b1 * sn);
+                        bi1 = eb * fmaf(b1, cs, -b0 * sn);
+                    }
+                    vCI[j] = ci0;
+                    vCI[j + 1] = ci1;
+                    vBI[j] = bi0;
+                    vBI[j + 1] = bi1;
+                    // Ch = Ci * G_ib ; other Bi = own Bi * F[ib][i'] ; Bh = own Bi * F[ib][4]
+                    if (!pair) {
+                        const float g0 = ib ? f32[F_KRE + gslot(ib) * NP + m0] : 1.f;
+                        const float g1 = ib ? f32[F_KRE + gslot(ib) * NP + m1] : 1.f;
+                        vCH[j] = ci0 * g0;
+                        vCH[j + 1] = ci1 * g1;
+                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
+                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            const int i2 = ib + 1 + q;
+                            if (i2 < 4) {
+                                vBX[q][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
+                                vBX[q][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                            }
+                        }
+                    } else {
+                        float gr = 1.f, gi = 0.f;
+                        if (ib) {
+                            gr = f32[F_KRE + gslot(ib) * NP + m0];
+                            gi = f32[F_KIM + gslot(ib) * NP + m0];
+                        }
+                        cmul(ci0, ci1, gr, gi, vCH[j], vCH[j + 1]);
+                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m0],
+                             f32[F_KIM + fslot(ib, 4) * NP + m0], vBH[j], vBH[j + 1]);
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            const int i2 = ib + 1 + q;
+                            if (i2 < 4)
+                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m0],
+                                     f32[F_KIM + fslot(ib, i2) * NP + m0], vBX[q][j],
+                                     vBX[q][j + 1]);
+                        }
+                    }
+                }
+                st16(sm + SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
+                st16(sm + SM_CH, off_kmaj(t, r0, KM_LBO, KM_SBO), vCH);
+                st16(sm + SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    const int i2 = ib + 1 + q;
+                    if (i2 < 4) st16(sm + SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[q]);
+                }
+                st16(sm + SM_BH, off_mnmaj(r0, t, 2048u, 128u), vBH);
+            }
+            f32[F_CP + grp * 64 + t] = corr;
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // ---- phase A: scores, chunk state, readout of the carried state --------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t bi_base = smem_u32(sm + SM_BI), ci_base = smem_u32(sm + SM_CI);
+            const uint32_t id_sc = idesc_bf16(64, 16, false, false);
+            for (int i = 0; i < NSB; ++i)
+                for (int s = 0; s < NP / 16; ++s)
+                    mma_bf16(t_sc + 16 * i,
+                             sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
+                             sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
+                             id_sc, s > 0);
+            const uint32_t bh_base = smem_u32(sm + SM_BH), x_base = smem_u32(sX);
+            const uint32_t id_st = idesc_bf16(128, 64, true, true);
+            for (int s = 0; s < Q / 16; ++s)
+                mma_bf16(t_st, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                         sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_st, s > 0);
+            const uint32_t kt_base = smem_u32(sm + SM_KT), ch_base = smem_u32(sm + SM_CH);
+            const uint32_t id_y = idesc_bf16(64, 64, true, false);
+            for (int s = 0; s < NP / 16; ++s)
+                mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),
+                         sdesc(ch_base + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE), id_y, s > 0);
+            mma_commit(&bar_mma[0]);
+        }
+        if (tid < 64) {
+            float cs = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cs += f32[F_CP + q * 64 + tid];
+            f32[F_CORR + tid] = -f32[F_BN + tid] * cs + Dh;
+        }
+        if (!mbar_wait(&bar_mma[0], (uint32_t)(c & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        fence_after_sync();
+        __syncthreads();
+        if (*abort_flag) break;
+
+        if (warp < 4) {
+            // ---- carried state: K_c = e^{lam S_63} K_{c-1} + S_chunk ------------
+            const int n = tid;
+            const int m = n < nr ? n : nr + ((n - nr) >> 1);
+            const bool pr_row = n >= nr && n < N;
+            const bool im_row = pr_row && ((n - nr) & 1);
+            float dr = 0.f, di = 0.f;
+            if (n < N) {
+                dr = f32[F_KRE + fslot(0, 4) * NP + m];
+                di = f32[F_KIM + fslot(0, 4) * NP + m];
+            }
+#pragma unroll
+            for (int c16 = 0; c16 < PD / 16; ++c16) {
+                float sv[16];
+                tmem_ld16(tmem_addr(t_st, 32u * warp, 16u * c16), sv);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int q = c16 * 16 + j;
+                    const float own = K[q];
+                    const float other = __shfl_xor_sync(0xffffffffu, own, 1);
+                    float nv;
+                    if (!pr_row)
+                        nv = fmaf(dr, own, sv[j]);
+                    else if (!im_row)  // re' = dr re - di im
+                        nv = fmaf(dr, own, fmaf(-di, other, sv[j]));
+                    else               // im' = di re + dr im
+                        nv = fmaf(di, other, fmaf(dr, own, sv[j]));
+                    K[q] = n < N ? nv : 0.f;
+                }
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < PD / 8; ++q8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
+                st16(sm + SM_KT, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
+            }
+        } else {
+            // ---- masked scores -> P^T tiles --------------------------------------
+            const int qd = warp - 4;
+            for (int i = 0; i < NSB; ++i) {
+                float v[16];
+                tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
+                const int sl = lane - 16;
+                if (sl >= 0) {
+                    const int s = 16 * qd + sl;
+                    if (s < 16 * (i + 1)) {
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
+                            hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
+                        }
+                        unsigned char *pt = sm + SM_P + i * 2048;
+                        st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
+                        st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // ---- phase B: intra-chunk term Y^T += X^T P^T_i --------------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + SM_P);
+            const uint32_t id_d = idesc_bf16(64, 16, true, true);
+            for (int i = 0; i < NSB; ++i)
+                for (int s = 0; s <= i; ++s)
+                    mma_bf16(t_y + 16 * i, sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128),
+                             sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
+                             true);
+            mma_commit(&bar_mma[1]);
+        }
+        if (!mbar_wait(&bar_mma[1], (uint32_t)(c & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        fence_after_sync();
+        __syncthreads();
+        if (*abort_flag) break;
+
+        // ---- epilogue: y_t[p] = Y^T[p][t] + (corr_t + D) u_t[p] -----------------
+        {
+            const int qd = warp & 3, half = warp >> 2;
+            for (int c16 = 0; c16 < 2; ++c16) {
+                float v[16];
+                const int tc = 32 * half + 16 * c16;
+                tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
+                if (lane < 16) {
+                    const int pp = 16 * qd + lane;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = tc + j;
+                        if (t0 + t < L) {
+                            const float u = bf(sX + off_sw128(t, pp));
+                            const float yv = fmaf(f32[F_CORR + t], u, v[j]);
+                            reinterpret_cast<__nv_bfloat16 *>(p.y)[ix_y(p, b, t0 + t, h, 0, pp)] =
+                                __float2bfloat16_rn(yv);
+                        }
+                    }
+                }
+            }
+        }
+        // last chunk: final state and last write
+        if (c == nchunk - 1 && chain_thr && tid < N) {
+            const int n = tid;
+            const int tl = (L - 1) - t0;
+            const float bl = ld_row1(sB, tl, n);
+#pragma unroll
+            for (int q = 0; q < PD; ++q) {
+                if (p.hT) p.hT[ix_st(p, b, h, n, q)] = K[q];
+                if (p.wT) p.wT[ix_st(p, b, h, n, q)] = bl * bf(sX + off_sw128(tl, q));
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        // refill this stage with chunk c + 2
+        if (tid == 0 && c + 2 < nchunk) {
+            mbar_expect_tx(&bar_tma[st], tile_bytes);
+            tma_load_4d(sm + SM_X + st * 8192, &tmX, &bar_tma[st], 0, h, (c + 2) * Q, b);
+            for (int k = 0; k < nbox; ++k) {
+                tma_load_4d(sm + SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g,
+                            (c + 2) * Q, b);
+                tma_load_4d(sm + SM_C + st * 16384 + k * 8192, &tmC, &bar_tma[st], 64 * k, g,
+                            (c + 2) * Q, b);
+            }
+        }
+    }
+    // on abort: let in-flight loads land before the CTA's shared memory goes away
+    if (*abort_flag && tid == 0) {
+        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
+        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 4-D bf16 map over (inner, dim1, time, batch) with a box of (inner, 1, Q, 1).
+static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t d1, uint64_t L,
+                     uint64_t B, uint64_t s1, uint64_t sL, uint64_t sB, uint32_t box_inner,
+                     bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {inner, d1, L, B};
+    cuuint64_t strides[3] = {s1 * 2, sL * 2, sB * 2};
+    cuuint32_t box[4] = {box_inner, 1, (cuuint32_t)Q, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace chunkfwd
+
+// Whether the tensor-core forward handles this problem.
+bool chunk_fwd_supported(const Params &p) {
+    auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
+    auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
+    return p.bf16 && p.P == chunkfwd::PD && p.R == 1 && p.O == 1 &&
+           (p.N == 64 || p.N == 128) && p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) &&
+           st16(p.sx[0]) && st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) &&
+           st16(p.sB[2]) && st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) &&
+           chunkfwd::encode_fn() != nullptr;
+}
+
+cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
+    using namespace chunkfwd;
+    CUtensorMap mx, mb, mc;
+    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
+        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
+        !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true))
+        return cudaErrorInvalidValue;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(k_chunk_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    k_chunk_fwd<<<dim3(p.H, p.Bsz), THREADS, SMEM_BYTES, st>>>(mx, mb, mc, p);
+    profile_mark(st, "k_chunk_fwd");
+    return cudaGetLastError();
+}
+
+// Read and clear the device error word of the tensor-core kernels.
+int chunk_error_take() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, ssm_chunk_error_word, sizeof(int)) != cudaSuccess) return -1;
+    if (v) cudaMemcpyToSymbol(ssm_chunk_error_word, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace ssm

@@ -74,6 +74,31 @@ def test_workload_parity(name):
     check_all(shape, inp)
 
 
+@pytest.mark.parametrize("name", ["mamba2_siso", "hybridmamba"])
+def test_workload_parity_recurrent_forward(name):
+    """The same workloads through the token-by-token kernels (chunk = 1)."""
+    shape = S.WORKLOADS[name].replace(**REDUCED[name]).replace(chunk=1)
+    inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(name))
+    check_all(shape, inp, backward=False)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=1), dict(seqlen=63), dict(seqlen=64), dict(seqlen=65), dict(seqlen=200),
+    dict(seqlen=130, n_real=128, n_pairs=0),
+    dict(seqlen=130, n_real=0, n_pairs=64),
+    dict(seqlen=100, n_real=32, n_pairs=16),
+    dict(seqlen=100, decay_mode=S.DECAY_PER_HEAD, two_endpoint=0, n_real=128, n_pairs=0,
+         ngroups=2),
+])
+def test_chunked_forward_shapes(kw):
+    """Chunked tensor-core forward: ragged tails around the 64-token chunk,
+    64/128 state rows, real-only, pairs-only, grouped B/C, initial state."""
+    base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, chunk=64)
+    shape = base.replace(**kw)
+    inp = S.make_inputs(shape, seed=31, with_state=True)
+    check_all(shape, inp, backward=False)
+
+
 @pytest.mark.parametrize("name", S.WORKLOAD_ORDER)
 def test_workload_parity_with_state(name):
     shape = S.WORKLOADS[name].replace(**REDUCED[name]).replace(seqlen=37)
