@@ -133,7 +133,7 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
 }
 
 struct BwdWs {
-    size_t off_dC, off_gbu, off_tok, off_M2, off_par, total;
+    size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, total;
 };
 
 BwdWs bwd_layout(const ssm_desc_t *d) {
@@ -151,6 +151,14 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     off = align256(off + BLH * d->rank_out * d->rank_in * 4);
     w.off_par = off;
     off = align256(off + (size_t)d->batch * d->nheads * (ndecay(d) + d->n_pairs + 2) * 4);
+    const size_t ntb = (size_t)(d->seqlen + 127) / 128;  // time blocks of the finalize scan
+    const size_t nmode = (size_t)d->n_real + d->n_pairs;
+    w.off_ddt = off;
+    off = align256(off + BLH * 4);
+    w.off_blk = off;
+    off = align256(off + (size_t)d->batch * d->nheads * ntb * (4 * nmode + 2) * 4);
+    w.off_blkc = off;
+    off = align256(off + (size_t)d->batch * d->nheads * ntb * 4);
     w.total = off;
     return w;
 }
@@ -295,6 +303,9 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     p.ws_tok = (float *)(ws + lay.off_tok);
     p.ws_M2 = (float *)(ws + lay.off_M2);
     p.ws_par = (float *)(ws + lay.off_par);
+    p.ws_ddt = (float *)(ws + lay.off_ddt);
+    p.ws_blk = (float *)(ws + lay.off_blk);
+    p.ws_blkc = (float *)(ws + lay.off_blkc);
     if (!ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);

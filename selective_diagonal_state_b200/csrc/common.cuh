@@ -34,6 +34,9 @@ struct Params {
     float *ws_tok;  // [B][L][H][2]      (dsigma_t, <dy_t, C_t W_t>)
     float *ws_M2;   // [B][L][H][O][R]   <dy_t[o,:], u_t[r,:]>
     float *ws_par;  // [B][H][NPAR]      per-unit partials of dA, dtheta, dD, dbeta_0
+    float *ws_ddt;  // [B][L][H]         local decay part of ddt (within a time block)
+    float *ws_blk;  // [B][H][NTB][4 nmode + 2]  per time block: totals and local sums
+    float *ws_blkc; // [B][H][NTB]       ddt offset of each time block (carried part)
     Geometry geo;
 };
 

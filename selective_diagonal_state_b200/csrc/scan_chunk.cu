@@ -116,6 +116,13 @@ __device__ __forceinline__ float ld_row1(const unsigned char *tile, int t, int r
 }
 __device__ __forceinline__ void raise_error(int code) { atomicCAS(&ssm_chunk_error_word, 0, code); }
 
+// 2^x with the hardware approximation (operands are rounded to bf16 afterwards)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // complex multiply (a + ib)(c + id)
 __device__ __forceinline__ void cmul(float a, float b, float c, float d, float &re, float &im) {
     re = fmaf(a, c, -b * d);
@@ -336,18 +343,18 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                         m0 = r;
                         m1 = r + 1;
                         const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
-                        ci0 = c0 * exp2f(x0);
-                        ci1 = c1 * exp2f(x1);
-                        bi0 = sig * b0 * exp2f(fminf(-x0, 120.f));
-                        bi1 = sig * b1 * exp2f(fminf(-x1, 120.f));
+                        ci0 = c0 * ex2_fast(x0);
+                        ci1 = c1 * ex2_fast(x1);
+                        bi0 = sig * b0 * ex2_fast(fminf(-x0, 120.f));
+                        bi1 = sig * b1 * ex2_fast(fminf(-x1, 120.f));
                     } else {
                         pair = true;
                         m0 = m1 = nr + ((r - nr) >> 1);
                         const float x = f32[F_A2 + m0] * ds;
                         float sn, cs;
-                        sincosf(f32[F_W + m0] * ds, &sn, &cs);
+                        __sincosf(f32[F_W + m0] * ds, &sn, &cs);
                         // rotate by cis(-phi): (u + iv)(cs - i sn)
-                        const float ec = exp2f(x), eb = sig * exp2f(fminf(-x, 120.f));
+                        const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
                         ci0 = ec * fmaf(c0, cs, c1 * sn);
                         ci1 = ec * fmaf(c1, cs, -c0 * sn);
                         bi0 = eb * fmaf(b0, cs, b1 * sn);
@@ -532,21 +539,23 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         // ---- epilogue: y_t[p] = Y^T[p][t] + (corr_t + D) u_t[p] -----------------
         {
             const int qd = warp & 3, half = warp >> 2;
+            const int pp = 16 * qd + (lane & 15);
+            __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
+                                  h * p.sy[2] + pp;
             for (int c16 = 0; c16 < 2; ++c16) {
                 float v[16];
                 const int tc = 32 * half + 16 * c16;
                 tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
                 if (lane < 16) {
-                    const int pp = 16 * qd + lane;
+                    __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = tc + j;
                         if (t0 + t < L) {
                             const float u = bf(sX + off_sw128(t, pp));
-                            const float yv = fmaf(f32[F_CORR + t], u, v[j]);
-                            reinterpret_cast<__nv_bfloat16 *>(p.y)[ix_y(p, b, t0 + t, h, 0, pp)] =
-                                __float2bfloat16_rn(yv);
+                            *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
                         }
+                        yp += p.sy[1];
                     }
                 }
             }

@@ -42,7 +42,25 @@ struct Smem {
     float *corr;              // [HC][T][O][R]   -beta_{t+1} (C_t B_t)[o][r]   (or M for bwd)
     float *red;               // reduction buffer (kernel specific)
     float *misc;              // [HC][T][4]
+    int *slot;                // [N] slot of each state row
 };
+
+// Threads cover a (rows x width) loop as (tid / W, tid % W) with W the
+// smallest power of two >= min(width, blockDim): no division per element.
+struct Lanes2D {
+    int tx, ty, W, ny;
+};
+__device__ __forceinline__ Lanes2D lanes2d(int width) {
+    const int nthr = blockDim.x;
+    int W = 1;
+    while (W < width && W < nthr) W <<= 1;
+    Lanes2D l;
+    l.W = W;
+    l.tx = threadIdx.x & (W - 1);
+    l.ty = threadIdx.x / W;
+    l.ny = nthr / W;
+    return l;
+}
 
 template <int NR, int NPR>
 __device__ __forceinline__ int ngl_of(const Params &p, int hbase, int HC) {
@@ -75,6 +93,7 @@ __host__ __device__ inline size_t carve(Smem &s, float *base, const Params &p, i
     s.dy = with_dy ? take((size_t)g.HC * g.T * p.O * g.PP) : nullptr;
     s.corr = take((size_t)g.HC * g.T * p.O * p.R);
     s.misc = take((size_t)g.HC * g.T * 4);
+    s.slot = reinterpret_cast<int *>(take((size_t)p.N));
     s.red = base ? base + off : nullptr;
     return off;
 }
@@ -98,7 +117,7 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
     const int tid = threadIdx.x, nthr = blockDim.x;
     // dt, lambda for t0 .. t0+T (one past the block for beta_{t+1})
     for (int i = tid; i < HC * (T + 1); i += nthr) {
-        int hc = i / (T + 1), tt = i % (T + 1), h = hbase + hc, t = t0 + tt;
+        int hc = i / (T + 1), tt = i - hc * (T + 1), h = hbase + hc, t = t0 + tt;
         float dv = 0.f, lv = 1.f;
         if (h < p.H && t < p.L) {
             dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
@@ -107,34 +126,52 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
         s.dt[i] = dv;
         s.lam[i] = lv;
     }
-    for (int i = tid; i < NGL * T * p.R * p.N; i += nthr) {
-        int n = i % p.N, r = (i / p.N) % p.R, tt = (i / (p.N * p.R)) % T, gl = i / (p.N * p.R * T);
-        int gg = gbase + gl, t = t0 + tt;
-        float v = (gg < p.G && t < p.L) ? ld_io(p.Bm, ix_B(p, b, t, gg, r, n), p.bf16) : 0.f;
-        s.Bp[((gl * T + tt) * p.R + r) * NSL + slot_of<NR, NPR>(n, p.nr, NQ)] = v;
+    {
+        const Lanes2D l = lanes2d(p.N);
+        for (int gl = 0; gl < NGL; ++gl) {
+            const int gg = gbase + gl;
+            for (int tt = l.ty; tt < T; tt += l.ny) {
+                const int t = t0 + tt;
+                const bool ok = gg < p.G && t < p.L;
+                for (int r = 0; r < p.R; ++r) {
+                    float *dst = s.Bp + ((gl * T + tt) * p.R + r) * NSL;
+                    for (int n = l.tx; n < p.N; n += l.W)
+                        dst[s.slot[n]] = ok ? ld_io(p.Bm, ix_B(p, b, t, gg, r, n), p.bf16) : 0.f;
+                }
+                for (int o = 0; o < p.O; ++o) {
+                    float *dst = s.Cp + ((gl * T + tt) * p.O + o) * NSL;
+                    for (int n = l.tx; n < p.N; n += l.W)
+                        dst[s.slot[n]] = ok ? ld_io(p.Cm, ix_C(p, b, t, gg, o, n), p.bf16) : 0.f;
+                }
+            }
+        }
     }
-    for (int i = tid; i < NGL * T * p.O * p.N; i += nthr) {
-        int n = i % p.N, o = (i / p.N) % p.O, tt = (i / (p.N * p.O)) % T, gl = i / (p.N * p.O * T);
-        int gg = gbase + gl, t = t0 + tt;
-        float v = (gg < p.G && t < p.L) ? ld_io(p.Cm, ix_C(p, b, t, gg, o, n), p.bf16) : 0.f;
-        s.Cp[((gl * T + tt) * p.O + o) * NSL + slot_of<NR, NPR>(n, p.nr, NQ)] = v;
-    }
-    for (int i = tid; i < HC * T * p.R * PP; i += nthr) {
-        int q = i % PP, r = (i / PP) % p.R, tt = (i / (PP * p.R)) % T, hc = i / (PP * p.R * T);
-        int h = hbase + hc, t = t0 + tt;
-        s.u[i] = (h < p.H && t < p.L && q < p.P) ? ld_io(p.x, ix_x(p, b, t, h, r, q), p.bf16) : 0.f;
-    }
-    if (with_dy) {
-        for (int i = tid; i < HC * T * p.O * PP; i += nthr) {
-            int q = i % PP, o = (i / PP) % p.O, tt = (i / (PP * p.O)) % T, hc = i / (PP * p.O * T);
-            int h = hbase + hc, t = t0 + tt;
-            s.dy[i] = (h < p.H && t < p.L && q < p.P) ? ld_io(p.dy, ix_y(p, b, t, h, o, q), p.bf16)
-                                                      : 0.f;
+    {
+        const Lanes2D l = lanes2d(PP);
+        for (int hc = 0; hc < HC; ++hc) {
+            const int h = hbase + hc;
+            for (int tt = l.ty; tt < T; tt += l.ny) {
+                const int t = t0 + tt;
+                const bool ok = h < p.H && t < p.L;
+                for (int r = 0; r < p.R; ++r) {
+                    float *dst = s.u + ((hc * T + tt) * p.R + r) * PP;
+                    for (int q = l.tx; q < PP; q += l.W)
+                        dst[q] = (ok && q < p.P) ? ld_io(p.x, ix_x(p, b, t, h, r, q), p.bf16) : 0.f;
+                }
+                if (with_dy) {
+                    for (int o = 0; o < p.O; ++o) {
+                        float *dst = s.dy + ((hc * T + tt) * p.O + o) * PP;
+                        for (int q = l.tx; q < PP; q += l.W)
+                            dst[q] = (ok && q < p.P) ? ld_io(p.dy, ix_y(p, b, t, h, o, q), p.bf16)
+                                                     : 0.f;
+                    }
+                }
+            }
         }
     }
     __syncthreads();
     for (int i = tid; i < HC * T; i += nthr) {
-        int hc = i / T, tt = i % T, t = t0 + tt;
+        int hc = i / T, tt = i - hc * T, t = t0 + tt;
         float dv = s.dt[hc * (T + 1) + tt], lv = s.lam[hc * (T + 1) + tt];
         float bnext = 0.f;
         if (t + 1 < p.L) bnext = (1.f - s.lam[hc * (T + 1) + tt + 1]) * s.dt[hc * (T + 1) + tt + 1];
@@ -142,24 +179,29 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
         s.bn[i] = bnext;
     }
     const int nmode = p.nr + p.np;
-    for (int i = tid; i < HC * T * nmode; i += nthr) {
-        int m = i % nmode, tt = (i / nmode) % T, hc = i / (nmode * T);
-        float dv = s.dt[hc * (T + 1) + tt];
-        float *cf = s.coef + (hc * T + tt) * NSL;
-        if (m < p.nr) {
-            float a = s.a[hc * p.ndec + (p.per_coord ? m : 0)];
-            cf[slot_of<NR, NPR>(m, p.nr, NQ)] = expf(dv * a);
-        } else {
-            int j = m - p.nr;
-            float a = s.a[hc * p.ndec + (p.per_coord ? m : 0)];
-            float e = expf(dv * a), sn, cs;
-            sincosf(dv * s.w[hc * (p.np > 0 ? p.np : 1) + j], &sn, &cs);
-            int sl = slot_of<NR, NPR>(p.nr + 2 * j, p.nr, NQ);
-            cf[sl] = e * cs;
-            cf[sl + 1] = e * sn;
+    {
+        const Lanes2D l = lanes2d(nmode);
+        for (int hc = 0; hc < HC; ++hc) {
+            for (int tt = l.ty; tt < T; tt += l.ny) {
+                const float dv = s.dt[hc * (T + 1) + tt];
+                float *cf = s.coef + (hc * T + tt) * NSL;
+                for (int m = l.tx; m < nmode; m += l.W) {
+                    const float a = s.a[hc * p.ndec + (p.per_coord ? m : 0)];
+                    if (m < p.nr) {
+                        cf[s.slot[m]] = expf(dv * a);
+                    } else {
+                        const int j = m - p.nr;
+                        float e = expf(dv * a), sn, cs;
+                        sincosf(dv * s.w[hc * (p.np > 0 ? p.np : 1) + j], &sn, &cs);
+                        const int sl = s.slot[p.nr + 2 * j];
+                        cf[sl] = e * cs;
+                        cf[sl + 1] = e * sn;
+                    }
+                }
+            }
         }
     }
-    // M_t[o][r] = sum_n C[o][n] B[n][r] scaled by -beta_{t+1}
+    // M_t[o][r] = sum_n C[o][n] B[n][r] (callers scale by beta_{t+1})
     for (int i = tid; i < HC * T * p.O * p.R; i += nthr) {
         int r = i % p.R, o = (i / p.R) % p.O, tt = (i / (p.R * p.O)) % T, hc = i / (p.R * p.O * T);
         int h = hbase + hc, gl = (h < p.H ? h : hbase) / p.hpg - gbase;
@@ -183,6 +225,7 @@ __device__ void init_rates(const Params &p, Smem &s, int hbase, int NSL, int NGL
         int hc = i / p.np, j = i % p.np, h = min(hbase + hc, p.H - 1);
         s.w[i] = p.theta[h * p.np + j];
     }
+    for (int n = threadIdx.x; n < p.N; n += blockDim.x) s.slot[n] = slot_of<NR, NPR>(n, p.nr, g.NQ);
     // padding slots must read as zero for the whole kernel
     for (int i = threadIdx.x; i < g.HC * g.T * NSL; i += blockDim.x) s.coef[i] = 0.f;
     for (int i = threadIdx.x; i < NGL * g.T * p.R * NSL; i += blockDim.x) s.Bp[i] = 0.f;
@@ -334,9 +377,10 @@ __global__ void __launch_bounds__(MAXT) k_fwd(Params p) {
         }
         __syncthreads();
         // y = C K - beta_{t+1} M u + D u, summed over the row groups
-        for (int i = threadIdx.x; i < HC * T * p.O * p.P; i += blockDim.x) {
-            int q = i % p.P, o = (i / p.P) % p.O, tt = (i / (p.P * p.O)) % T,
-                hc = i / (p.P * p.O * T);
+        const Lanes2D l2 = lanes2d(p.P);
+        for (int row = l2.ty; row < HC * T * p.O; row += l2.ny)
+        for (int q = l2.tx; q < p.P; q += l2.W) {
+            const int o = row % p.O, tt = (row / p.O) % T, hc = row / (p.O * T);
             int h = ln.hbase + hc, t = t0 + tt;
             if (h >= p.H || t >= p.L) continue;
             float v = 0.f;
@@ -451,12 +495,13 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep1(Params p) {
                                lane_in_s);
         }
         __syncthreads();
-        for (int i = threadIdx.x; i < HC * T * p.O * p.N; i += blockDim.x) {
-            int n = i % p.N, o = (i / p.N) % p.O, tt = (i / (p.N * p.O)) % T,
-                hc = i / (p.N * p.O * T);
+        const Lanes2D l2 = lanes2d(p.N);
+        for (int row = l2.ty; row < HC * T * p.O; row += l2.ny)
+        for (int n = l2.tx; n < p.N; n += l2.W) {
+            const int o = row % p.O, tt = (row / p.O) % T, hc = row / (p.O * T);
             int h = ln.hbase + hc, t = t0 + tt;
             if (h >= p.H || t >= p.L) continue;
-            int sl = slot_of<NR, NPR>(n, p.nr, NQ);
+            int sl = s.slot[n];
             int q = sl / NS, k = o * NS + sl % NS;
             float acc = 0.f;
             for (int w2 = 0; w2 < NWP; ++w2) acc += s.red[(((hc * T + tt) * NWP + w2) * NQ + q) * KV + k];
@@ -538,9 +583,10 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
         }
         __syncthreads();
         // dx_t = sigma_t sum_q(B^T G) - beta_{t+1} M^T dy + D dy
-        for (int i = threadIdx.x; i < HC * T * p.R * p.P; i += blockDim.x) {
-            int q = i % p.P, r = (i / p.P) % p.R, tt = (i / (p.P * p.R)) % T,
-                hc = i / (p.P * p.R * T);
+        const Lanes2D lq = lanes2d(p.P);
+        for (int row = lq.ty; row < HC * T * p.R; row += lq.ny)
+        for (int q = lq.tx; q < p.P; q += lq.W) {
+            const int r = row % p.R, tt = (row / p.R) % T, hc = row / (p.R * T);
             int h = ln.hbase + hc, t = t0 + tt;
             if (h >= p.H || t >= p.L) continue;
             float acc = 0.f;
@@ -554,12 +600,13 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
             st_io(p.dx, ix_x(p, ln.b, t, h, r, q), v, p.bf16);
         }
         // gbu_t[r][n] and M2_t[o][r], corr2_t
-        for (int i = threadIdx.x; i < HC * T * p.R * p.N; i += blockDim.x) {
-            int n = i % p.N, r = (i / p.N) % p.R, tt = (i / (p.N * p.R)) % T,
-                hc = i / (p.N * p.R * T);
+        const Lanes2D ln2 = lanes2d(p.N);
+        for (int row = ln2.ty; row < HC * T * p.R; row += ln2.ny)
+        for (int n = ln2.tx; n < p.N; n += ln2.W) {
+            const int r = row % p.R, tt = (row / p.R) % T, hc = row / (p.R * T);
             int h = ln.hbase + hc, t = t0 + tt;
             if (h >= p.H || t >= p.L) continue;
-            int sl = slot_of<NR, NPR>(n, p.nr, NQ);
+            int sl = s.slot[n];
             int q = sl / NS, k = r * NS + sl % NS;
             float acc = 0.f;
             for (int w2 = 0; w2 < NWP; ++w2) acc += redA[(((hc * T + tt) * NWP + w2) * NQ + q) * KV + k];
@@ -578,22 +625,34 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
         }
         __syncthreads();
         // dsigma_t = sum_{r,n} B[n,r] gbu[r][n];  corr2_t = sum_{o,r} M[o][r] M2[o][r]
-        for (int i = threadIdx.x; i < HC * T; i += blockDim.x) {
-            int tt = i % T, hc = i / T, h = ln.hbase + hc, t = t0 + tt;
-            if (h >= p.H || t >= p.L) continue;
-            int gl = h / p.hpg - ln.gbase;
-            float ds = 0.f;
-            for (int r = 0; r < p.R; ++r)
-                for (int n = 0; n < p.N; ++n)
-                    ds = fmaf(s.Bp[((gl * T + tt) * p.R + r) * NSL + slot_of<NR, NPR>(n, p.nr, NQ)],
-                              p.ws_gbu[ix_wsk(p, ln.b, t, h, r, p.R, n)], ds);
-            float c2 = 0.f;
-            for (int o = 0; o < p.O; ++o)
-                for (int r = 0; r < p.R; ++r)
-                    c2 = fmaf(s.corr[((hc * T + tt) * p.O + o) * p.R + r],
-                              p.ws_M2[((ix_bth(p, ln.b, t, h)) * p.O + o) * p.R + r], c2);
-            p.ws_tok[ix_bth(p, ln.b, t, h) * 2 + 0] = ds;
-            p.ws_tok[ix_bth(p, ln.b, t, h) * 2 + 1] = c2;
+        // one warp per token, lanes over (r, n), fixed-order shuffle reduction
+        {
+            const int wid = threadIdx.x >> 5, lid = threadIdx.x & 31, nw = blockDim.x >> 5;
+            for (int i = wid; i < HC * T; i += nw) {
+                const int hc = i / T, tt = i - hc * T, h = ln.hbase + hc, t = t0 + tt;
+                if (h >= p.H || t >= p.L) continue;
+                const int gl = h / p.hpg - ln.gbase;
+                float ds = 0.f;
+                for (int k = lid; k < p.R * p.N; k += 32) {
+                    const int r = k / p.N, n = k - r * p.N;
+                    const int sl = s.slot[n], q = sl / NS;
+                    float g = 0.f;
+                    for (int w2 = 0; w2 < NWP; ++w2)
+                        g += redA[(((hc * T + tt) * NWP + w2) * NQ + q) * KV + r * NS + (sl - q * NS)];
+                    ds = fmaf(s.Bp[((gl * T + tt) * p.R + r) * NSL + sl], g, ds);
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+                if (lid == 0) {
+                    float c2 = 0.f;
+                    for (int o = 0; o < p.O; ++o)
+                        for (int r = 0; r < p.R; ++r)
+                            c2 = fmaf(s.corr[((hc * T + tt) * p.O + o) * p.R + r],
+                                      p.ws_M2[((ix_bth(p, ln.b, t, h)) * p.O + o) * p.R + r], c2);
+                    p.ws_tok[ix_bth(p, ln.b, t, h) * 2 + 0] = ds;
+                    p.ws_tok[ix_bth(p, ln.b, t, h) * 2 + 1] = c2;
+                }
+            }
         }
         __syncthreads();
     }
@@ -629,39 +688,56 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
 }
 
 // ------------------------------------------------------------------------
-// backward finalize per (b, h): decay/angle gradients by reverse cumulative
-// sums over modes, then ddt, dlambda and the per-unit parameter partials.
-// One thread per mode; tokens in reverse blocks of FT.
+// backward finalize: decay/angle gradients by reverse cumulative sums over
+// time, done as a two-level scan.  Blocks of TBL tokens run in parallel
+// (k_bwd_units_local: local suffix sums, block totals), a per-(b, h) pass
+// carries the totals across blocks (k_bwd_units_carry), and an elementwise
+// pass writes ddt and dlambda (k_bwd_units_final).  All sums run in a fixed
+// order.
 // ------------------------------------------------------------------------
 constexpr int FT = 32;
+constexpr int TBL = 128;
 
-__global__ void __launch_bounds__(256) k_bwd_units(Params p) {
-    extern __shared__ __align__(16) float smem[];
-    const int b = blockIdx.y, h = blockIdx.x;
+__host__ __device__ inline int ntb_of(const Params &p) { return (p.L + TBL - 1) / TBL; }
+
+// per-mode constants shared by the finalize kernels
+struct ModeInfo {
+    float a, w;
+    int n0;
+    bool pair, valid;
+};
+__device__ __forceinline__ ModeInfo mode_info(const Params &p, int h, int m) {
+    ModeInfo mi;
     const int nmode = p.nr + p.np;
-    const int m = threadIdx.x;
-    const int nthr = blockDim.x;
-    const int g = h / p.hpg;
-    float *s_c = smem;                 // [FT][nthr]
-    float *s_dd = s_c + FT * nthr;     // [FT] decay part of ddt
-    const bool mv = m < nmode;
-    float a = 0.f, w = 0.f;
-    if (mv) {
-        a = neg_exp(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
-        if (m >= p.nr) w = p.theta[h * p.np + (m - p.nr)];
+    mi.valid = m < nmode;
+    mi.a = mi.w = 0.f;
+    mi.pair = mi.valid && m >= p.nr;
+    mi.n0 = 0;
+    if (mi.valid) {
+        mi.a = neg_exp(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
+        if (mi.pair) mi.w = p.theta[h * p.np + (m - p.nr)];
+        mi.n0 = m < p.nr ? m : p.nr + 2 * (m - p.nr);
     }
-    const int n0 = mv ? (m < p.nr ? m : p.nr + 2 * (m - p.nr)) : 0;
-    const bool pair = mv && m >= p.nr;
-    float cr = 0.f, ci = 0.f;   // running sum_{t >= tau} (X_t - Y_t)
-    float dA = 0.f, dth = 0.f;
-    float dD = 0.f;
-    for (int t1 = p.L; t1 > 0; t1 -= FT) {
-        const int t0 = max(0, t1 - FT), tn = t1 - t0;
+    return mi;
+}
+
+__global__ void __launch_bounds__(256) k_bwd_units_local(Params p) {
+    extern __shared__ __align__(16) float smem[];
+    const int tb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int m = threadIdx.x, nthr = blockDim.x;
+    const int g = h / p.hpg;
+    const int NTB = ntb_of(p), nmode = p.nr + p.np;
+    const int tbeg = tb * TBL, tend = min(p.L, tbeg + TBL);
+    float *s_c = smem;  // [FT][nthr]
+    const ModeInfo mi = mode_info(p, h, m);
+    float cr = 0.f, ci = 0.f, dA = 0.f, dth = 0.f, dD = 0.f, sdt = 0.f;
+    for (int t1 = tend; t1 > tbeg; t1 -= FT) {
+        const int t0 = max(tbeg, t1 - FT), tn = t1 - t0;
         for (int k = tn - 1; k >= 0; --k) {
             const int t = t0 + k;
+            const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
             float contrib = 0.f;
-            if (mv) {
-                const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+            if (mi.valid) {
                 const float lv = p.two_ep ? ld_io(p.lam, ix_lam(p, b, t, h), p.bf16) : 1.f;
                 float bnx = 0.f;
                 if (t + 1 < p.L && p.two_ep)
@@ -669,20 +745,21 @@ __global__ void __launch_bounds__(256) k_bwd_units(Params p) {
                           ld_io(p.dt, ix_dt(p, b, t + 1, h), p.bf16);
                 const float sig = lv * dv + bnx;
                 const float *M2 = p.ws_M2 + ix_bth(p, b, t, h) * p.O * p.R;
+                const int n0 = mi.n0;
+                const bool pair = mi.pair;
                 float xr = 0.f, xi = 0.f, yr = 0.f, yi = 0.f;
                 for (int o = 0; o < p.O; ++o) {
                     // dCK[o][n] = dC[o][n] + beta_{t+1} sum_r B[r][n] M2[o][r]
                     float k0 = p.ws_dC[ix_wsk(p, b, t, h, o, p.O, n0)];
                     float k1 = pair ? p.ws_dC[ix_wsk(p, b, t, h, o, p.O, n0 + 1)] : 0.f;
                     for (int r = 0; r < p.R; ++r) {
-                        float mm = bnx * M2[o * p.R + r];
+                        const float mm = bnx * M2[o * p.R + r];
                         k0 = fmaf(mm, ld_io(p.Bm, ix_B(p, b, t, g, r, n0), p.bf16), k0);
                         if (pair) k1 = fmaf(mm, ld_io(p.Bm, ix_B(p, b, t, g, r, n0 + 1), p.bf16), k1);
                     }
                     const float c0 = ld_io(p.Cm, ix_C(p, b, t, g, o, n0), p.bf16);
                     const float c1 = pair ? ld_io(p.Cm, ix_C(p, b, t, g, o, n0 + 1), p.bf16) : 0.f;
-                    // conj(c) * k
-                    xr += c0 * k0 + c1 * k1;
+                    xr += c0 * k0 + c1 * k1;   // conj(c) * k
                     xi += c0 * k1 - c1 * k0;
                 }
                 for (int r = 0; r < p.R; ++r) {
@@ -690,97 +767,161 @@ __global__ void __launch_bounds__(256) k_bwd_units(Params p) {
                     const float b1 = pair ? ld_io(p.Bm, ix_B(p, b, t, g, r, n0 + 1), p.bf16) : 0.f;
                     const float g0 = sig * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0)];
                     const float g1 = pair ? sig * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0 + 1)] : 0.f;
-                    // b * conj(g)
-                    yr += b0 * g0 + b1 * g1;
+                    yr += b0 * g0 + b1 * g1;   // b * conj(g)
                     yi += b1 * g0 - b0 * g1;
                 }
                 cr += xr - yr;
                 ci += xi - yi;
                 dA = fmaf(dv, cr, dA);
                 if (pair) dth = fmaf(dv, -ci, dth);
-                contrib = a * cr + (pair ? -w * ci : 0.f);
+                contrib = mi.a * cr + (pair ? -mi.w * ci : 0.f);
+            }
+            if (m == 0) {
+                sdt += dv;
+                if (p.O == p.R)
+                    for (int o = 0; o < p.O; ++o)
+                        dD += p.ws_M2[ix_bth(p, b, t, h) * p.O * p.R + o * p.R + o];
             }
             s_c[k * nthr + m] = contrib;
         }
         __syncthreads();
-        if (m < FT && m < tn) {
+        if (m < tn) {
             float acc = 0.f;
             for (int j = 0; j < nthr; ++j) acc += s_c[m * nthr + j];
-            s_dd[m] = acc;
-        }
-        __syncthreads();
-        if (m == 0) {
-            for (int k = tn - 1; k >= 0; --k) {
-                const int t = t0 + k;
-                const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
-                const float lv = p.two_ep ? ld_io(p.lam, ix_lam(p, b, t, h), p.bf16) : 1.f;
-                const float ds = p.ws_tok[ix_bth(p, b, t, h) * 2 + 0];
-                const float c2 = p.ws_tok[ix_bth(p, b, t, h) * 2 + 1];
-                // dgamma_t = dsigma_t ; dbeta_t = dsigma_{t-1} - corr2_{t-1} (t >= 1)
-                float dbeta;
-                if (t >= 1)
-                    dbeta = p.ws_tok[ix_bth(p, b, t - 1, h) * 2 + 0] -
-                            p.ws_tok[ix_bth(p, b, t - 1, h) * 2 + 1];
-                else
-                    dbeta = p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1];
-                float dd = s_dd[k];
-                if (p.two_ep) {
-                    dd += lv * ds + (1.f - lv) * dbeta;
-                    if (p.dlam) st_io(p.dlam, ix_lam(p, b, t, h), dv * (ds - dbeta), p.bf16);
-                } else {
-                    dd += ds;
-                }
-                st_io(p.ddt, ix_dt(p, b, t, h), dd, p.bf16);
-                if (p.O == p.R)
-                    for (int o = 0; o < p.O; ++o) dD += p.ws_M2[ix_bth(p, b, t, h) * p.O * p.R + o * p.R + o];
-                (void)c2;
-            }
+            p.ws_ddt[ix_bth(p, b, t0 + m, h)] = acc;
         }
         __syncthreads();
     }
-    // per-unit partials: dA (per decay slot), dtheta, dD
+    float *blk = p.ws_blk + (((long long)b * p.H + h) * NTB + tb) * (4 * (long long)nmode + 2);
+    if (mi.valid) {
+        blk[4 * m + 0] = cr;
+        blk[4 * m + 1] = ci;
+        blk[4 * m + 2] = dA;
+        blk[4 * m + 3] = dth;
+    }
+    if (m == 0) {
+        blk[4 * nmode + 0] = sdt;
+        blk[4 * nmode + 1] = dD;
+    }
+}
+
+// carry the block totals across time blocks: per (b, h), one thread per mode
+__global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
+    extern __shared__ __align__(16) float smem[];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int m = threadIdx.x, nthr = blockDim.x;
+    const int NTB = ntb_of(p), nmode = p.nr + p.np;
+    const ModeInfo mi = mode_info(p, h, m);
+    float *s_c = smem;  // [nthr]
+    float car = 0.f, cai = 0.f, dA = 0.f, dth = 0.f, dD = 0.f;
+    for (int tb = NTB - 1; tb >= 0; --tb) {
+        const float *blk = p.ws_blk + (((long long)b * p.H + h) * NTB + tb) * (4 * (long long)nmode + 2);
+        const float sdt = blk[4 * nmode + 0];
+        float contrib = 0.f;
+        if (mi.valid) {
+            dA += blk[4 * m + 2] + car * sdt;
+            if (mi.pair) dth += blk[4 * m + 3] - cai * sdt;
+            contrib = mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
+        }
+        s_c[m] = contrib;
+        __syncthreads();
+        if (m == 0) {
+            float acc = 0.f;
+            for (int j = 0; j < nthr; ++j) acc += s_c[j];
+            p.ws_blkc[((long long)b * p.H + h) * NTB + tb] = acc;
+            dD += blk[4 * nmode + 1];
+        }
+        if (mi.valid) {
+            car += blk[4 * m + 0];
+            cai += blk[4 * m + 1];
+        }
+        __syncthreads();
+    }
     float *part = p.ws_par + ((long long)b * p.H + h) * npar_of(p);
-    __syncthreads();
     s_c[m] = dA;
     __syncthreads();
     if (p.per_coord) {
-        if (mv) part[m] = dA;
+        if (mi.valid) part[m] = dA;
     } else if (m == 0) {
         float acc = 0.f;
         for (int j = 0; j < nmode; ++j) acc += s_c[j];
         part[0] = acc;
     }
-    if (pair) part[p.ndec + (m - p.nr)] = dth;
+    if (mi.pair) part[p.ndec + (m - p.nr)] = dth;
     if (m == 0) part[p.ndec + p.np] = dD;
 }
 
-// dB, dC per (b, t, group): sum over the heads of the group
-__global__ void k_bwd_groups(Params p) {
-    const int t = blockIdx.x, b = blockIdx.y;
-    for (int i = threadIdx.x; i < p.G * (p.R + p.O) * p.N; i += blockDim.x) {
-        int n = i % p.N, k = (i / p.N) % (p.R + p.O), g = i / (p.N * (p.R + p.O));
-        float acc = 0.f;
-        if (k < p.R) {
-            const int r = k;
-            for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h) {
-                const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
-                const float lv = p.two_ep ? ld_io(p.lam, ix_lam(p, b, t, h), p.bf16) : 1.f;
-                float bnx = 0.f;
-                if (t + 1 < p.L && p.two_ep)
-                    bnx = (1.f - ld_io(p.lam, ix_lam(p, b, t + 1, h), p.bf16)) *
-                          ld_io(p.dt, ix_dt(p, b, t + 1, h), p.bf16);
-                float v = (lv * dv + bnx) * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n)];
-                const float *M2 = p.ws_M2 + ix_bth(p, b, t, h) * p.O * p.R;
-                for (int o = 0; o < p.O; ++o)
-                    v = fmaf(-bnx * ld_io(p.Cm, ix_C(p, b, t, g, o, n), p.bf16), M2[o * p.R + r], v);
-                acc += v;
-            }
-            st_io(p.dBm, ix_B(p, b, t, g, r, n), acc, p.bf16);
+// ddt and dlambda per (b, t, h)
+__global__ void k_bwd_units_final(Params p) {
+    const long long total = (long long)p.Bsz * p.L * p.H;
+    const int NTB = ntb_of(p);
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int h = (int)(i % p.H);
+        const long long bt = i / p.H;
+        const int t = (int)(bt % p.L), b = (int)(bt / p.L);
+        const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+        const float lv = p.two_ep ? ld_io(p.lam, ix_lam(p, b, t, h), p.bf16) : 1.f;
+        const float ds = p.ws_tok[i * 2 + 0];
+        float dd = p.ws_ddt[i] + p.ws_blkc[((long long)b * p.H + h) * NTB + t / TBL];
+        if (p.two_ep) {
+            // dgamma_t = dsigma_t ; dbeta_t = dsigma_{t-1} - corr2_{t-1} (t >= 1)
+            float dbeta;
+            if (t >= 1)
+                dbeta = p.ws_tok[ix_bth(p, b, t - 1, h) * 2 + 0] -
+                        p.ws_tok[ix_bth(p, b, t - 1, h) * 2 + 1];
+            else
+                dbeta = p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1];
+            dd += lv * ds + (1.f - lv) * dbeta;
+            if (p.dlam) st_io(p.dlam, ix_lam(p, b, t, h), dv * (ds - dbeta), p.bf16);
         } else {
-            const int o = k - p.R;
-            for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h)
-                acc += p.ws_dC[ix_wsk(p, b, t, h, o, p.O, n)];
-            st_io(p.dCm, ix_C(p, b, t, g, o, n), acc, p.bf16);
+            dd += ds;
+        }
+        st_io(p.ddt, ix_dt(p, b, t, h), dd, p.bf16);
+    }
+}
+
+// dB, dC per (b, t): sum over the heads of each group; per-head scalars first
+__global__ void __launch_bounds__(256) k_bwd_groups(Params p) {
+    extern __shared__ __align__(16) float smem[];
+    const int t = blockIdx.x, b = blockIdx.y;
+    float *s_sig = smem, *s_bn = smem + p.H;
+    for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
+        const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+        const float lv = p.two_ep ? ld_io(p.lam, ix_lam(p, b, t, h), p.bf16) : 1.f;
+        float bnx = 0.f;
+        if (t + 1 < p.L && p.two_ep)
+            bnx = (1.f - ld_io(p.lam, ix_lam(p, b, t + 1, h), p.bf16)) *
+                  ld_io(p.dt, ix_dt(p, b, t + 1, h), p.bf16);
+        s_sig[h] = lv * dv + bnx;
+        s_bn[h] = bnx;
+    }
+    __syncthreads();
+    const Lanes2D l = lanes2d(p.N);
+    for (int row = l.ty; row < p.G * (p.R + p.O); row += l.ny) {
+        const int k = row % (p.R + p.O), g = row / (p.R + p.O);
+        for (int n = l.tx; n < p.N; n += l.W) {
+            float acc = 0.f;
+            if (k < p.R) {
+                const int r = k;
+                for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h) {
+                    float v = s_sig[h] * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n)];
+                    const float bnx = s_bn[h];
+                    if (bnx != 0.f) {
+                        const float *M2 = p.ws_M2 + ix_bth(p, b, t, h) * p.O * p.R;
+                        for (int o = 0; o < p.O; ++o)
+                            v = fmaf(-bnx * ld_io(p.Cm, ix_C(p, b, t, g, o, n), p.bf16),
+                                     M2[o * p.R + r], v);
+                    }
+                    acc += v;
+                }
+                st_io(p.dBm, ix_B(p, b, t, g, r, n), acc, p.bf16);
+            } else {
+                const int o = k - p.R;
+                for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h)
+                    acc += p.ws_dC[ix_wsk(p, b, t, h, o, p.O, n)];
+                st_io(p.dCm, ix_C(p, b, t, g, o, n), acc, p.bf16);
+            }
         }
     }
 }
@@ -967,12 +1108,20 @@ cudaError_t simt_backward(const Params &p, cudaStream_t st) {
     {
         int nthr = ((p.nr + p.np + 31) / 32) * 32;
         if (nthr < 32) nthr = 32;
-        size_t sm = (size_t)(FT * nthr + FT + 8) * 4;
-        k_bwd_units<<<dim3(p.H, p.Bsz), nthr, sm, st>>>(p);
-        profile_mark(st, "k_bwd_units");
+        k_bwd_units_local<<<dim3(ntb_of(p), p.H, p.Bsz), nthr, (size_t)FT * nthr * 4, st>>>(p);
+        profile_mark(st, "k_bwd_units_local");
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_bwd_units_carry<<<dim3(p.H, p.Bsz), nthr, (size_t)nthr * 4, st>>>(p);
+        profile_mark(st, "k_bwd_units_carry");
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const long long total = (long long)p.Bsz * p.L * p.H;
+        int blocks = (int)((total + 255) / 256);
+        if (blocks > 148 * 32) blocks = 148 * 32;
+        k_bwd_units_final<<<blocks, 256, 0, st>>>(p);
+        profile_mark(st, "k_bwd_units_final");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    k_bwd_groups<<<dim3(p.L, p.Bsz), 256, 0, st>>>(p);
+    k_bwd_groups<<<dim3(p.L, p.Bsz), 256, (size_t)2 * p.H * 4, st>>>(p);
     profile_mark(st, "k_bwd_groups");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_params<<<4, 256, 0, st>>>(p);
