@@ -258,6 +258,7 @@ def main():
     import torch.distributed as dist
 
     from selective_diagonal_state_b200 import abi, scan
+    from selective_diagonal_state_b200 import dist as sdist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -287,9 +288,7 @@ def main():
 
     def allreduce_params():
         if world > 1:
-            for t in (grads.dA_log, grads.dtheta, grads.dD):
-                if t is not None:
-                    dist.all_reduce(t)
+            sdist.allreduce_param_grads((grads.dA_log, grads.dtheta, grads.dD))
 
     def step():
         scan.scan_forward(shape, dev, out=fwd_out, desc=desc)
