@@ -14,7 +14,8 @@
 namespace ssm {
 bool simt_supported(const Params &p);
 cudaError_t simt_forward(const Params &p, cudaStream_t st);
-cudaError_t simt_backward(const Params &p, cudaStream_t st);
+cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk);
+bool chunk_bwd_supported(const Params &p);
 bool chunk_fwd_supported(const Params &p);
 cudaError_t chunk_forward(const Params &p, cudaStream_t st);
 int chunk_error_take();
@@ -133,8 +134,17 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
 }
 
 struct BwdWs {
-    size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, total;
+    size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, off_kb, off_qb,
+        total;
+    bool boundary;  // chunk-boundary carries (tensor-core backward shapes)
 };
+
+// Shapes the tensor-core backward may take (pointer alignment is checked at call time).
+bool tensor_bwd_shape(const ssm_desc_t *d) {
+    const int N = d->n_real + 2 * d->n_pairs;
+    return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
+           (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0;
+}
 
 BwdWs bwd_layout(const ssm_desc_t *d) {
     BwdWs w;
@@ -151,7 +161,7 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     off = align256(off + BLH * d->rank_out * d->rank_in * 4);
     w.off_par = off;
     off = align256(off + (size_t)d->batch * d->nheads * (ndecay(d) + d->n_pairs + 2) * 4);
-    const size_t ntb = (size_t)(d->seqlen + 127) / 128;  // time blocks of the finalize scan
+    const size_t ntb = (size_t)(d->seqlen + 63) / 64;  // time blocks of the finalize scan
     const size_t nmode = (size_t)d->n_real + d->n_pairs;
     w.off_ddt = off;
     off = align256(off + BLH * 4);
@@ -159,6 +169,14 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     off = align256(off + (size_t)d->batch * d->nheads * ntb * (4 * nmode + 2) * 4);
     w.off_blkc = off;
     off = align256(off + (size_t)d->batch * d->nheads * ntb * 4);
+    w.boundary = tensor_bwd_shape(d);
+    w.off_kb = w.off_qb = off;
+    if (w.boundary) {
+        w.off_kb = off;
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
+        w.off_qb = off;
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * 4 * N * 4);
+    }
     w.total = off;
     return w;
 }
@@ -306,12 +324,18 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     p.ws_ddt = (float *)(ws + lay.off_ddt);
     p.ws_blk = (float *)(ws + lay.off_blk);
     p.ws_blkc = (float *)(ws + lay.off_blkc);
+    p.nc = (int)((d->seqlen + 63) / 64);
     if (!ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
     // dD is written by the parameter pass; keep it defined when R != O
+    const bool chunked = d->chunk != 1 && ssm::chunk_bwd_supported(p);
+    if (chunked && lay.boundary) {
+        p.ws_kb = (float *)(ws + lay.off_kb);
+        p.ws_qb = (float *)(ws + lay.off_qb);
+    }
     profile_begin(st);
-    cudaError_t e = ssm::simt_backward(p, st);
+    cudaError_t e = ssm::simt_backward(p, st, chunked);
     profile_end();
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
     g_last_error.clear();

@@ -37,6 +37,10 @@ struct Params {
     float *ws_ddt;  // [B][L][H]         local decay part of ddt (within a time block)
     float *ws_blk;  // [B][H][NTB][4 nmode + 2]  per time block: totals and local sums
     float *ws_blkc; // [B][H][NTB]       ddt offset of each time block (carried part)
+    // exact decay-gradient carries at 64-token chunk boundaries (tensor-core path):
+    float *ws_kb;   // [B][H][NC][N][P]  pre-state K at the end of every chunk but the last
+    float *ws_qb;   // [B][H][NC][4][N]  per-row sum_p conj(Gbar) A K_prev at chunk starts (per warp of p)
+    int nc;         // number of 64-token chunks
     Geometry geo;
 };
 

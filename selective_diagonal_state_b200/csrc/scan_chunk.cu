@@ -96,6 +96,18 @@ __device__ __forceinline__ void st16(unsigned char *base, uint32_t off, const fl
     w.w = pack_bf16(v[6], v[7]);
     *reinterpret_cast<uint4 *>(base + off) = w;
 }
+// store v as bf16 hi (at hi + off) and the bf16 residual v - hi (at lo + off)
+__device__ __forceinline__ void st16_split(unsigned char *hi, unsigned char *lo, uint32_t off,
+                                           const float (&v)[8]) {
+    float h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+        l[i] = v[i] - h[i];
+    }
+    st16(hi, off, h);
+    st16(lo, off, l);
+}
 __device__ __forceinline__ float bf(const unsigned char *p) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
 }
@@ -599,6 +611,517 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 }
 
 // ---------------------------------------------------------------------------
+// Backward, forward-direction part: dC_t = dy_t H_t^T per head.
+//   H_t = K_t - beta_{t+1} W_t,   K_t = e^{lam S_t} K_prev + sum_{s<=t} Phi_{t,s} sigma_s b_s u_s
+// so, per state mode (complex for rotation pairs, real rows otherwise),
+//   dCK_t = e^{lam S_t} (dy_t . K_prev) + e^{lam (S_t - Sb_i)} sum_{s<=t} (dy_t . u_s) Bi_s
+// which is, on the tensor cores,
+//   V^T  = K_prev (N x 64 p) . dY^T (64 p x 64 t)          M=128, N=64, K=64
+//   G    = dY (64 t x 64 p) . X^T (64 p x 64 s)            M=64,  N=64, K=64
+//   D_i  = Bi^T (N x s) . (G o causal mask)_i^T (s x 16 t) M=128, N=16, K=16(i+1)
+// followed by the per-(t, row) unfolding of the decay factors on the CUDA
+// cores; dC_t = dCK_t - beta_{t+1} (dy_t . u_t) B_t.  The carried state is
+// recomputed exactly as in the forward (chunk-end state MMA + fp32 chain).
+// ---------------------------------------------------------------------------
+namespace chunkbwd {
+using namespace umma;
+using chunkfwd::Q;
+using chunkfwd::NSB;
+using chunkfwd::NP;
+using chunkfwd::PD;
+using chunkfwd::THREADS;
+using chunkfwd::WAIT_LIMIT;
+using chunkfwd::KM_LBO;
+using chunkfwd::KM_SBO;
+constexpr uint32_t TMEM_COLS = 256;
+// Operands that are rounded (folded B, chunk-end B, carried state, masked G)
+// are kept as bf16 pairs hi + lo (lo = v - hi) and every MMA on them runs as
+// hi*hi + hi*lo + lo*hi: about 16 mantissa bits, enough for the decay
+// gradients, which take differences of large sums of these products.
+constexpr uint32_t SM_X = 0;          // 2 x 8 KB   x tiles (128B swizzle)
+constexpr uint32_t SM_B = 16384;      // 2 x 16 KB  raw B tiles (two 64-row swizzled halves)
+constexpr uint32_t SM_DY = 49152;     // 2 x 8 KB   dy tiles (128B swizzle)
+constexpr uint32_t SM_BI = 65536;     // 40 KB      Bi tiles (hi)
+constexpr uint32_t SM_BIL = 106496;   // 40 KB      Bi tiles (lo)
+constexpr uint32_t SM_BH = 147456;    // 16 KB      Bh hi (MN-major, M = rows); masked G hi after phase A
+constexpr uint32_t SM_BHL = 163840;   // 16 KB      Bh lo;                       masked G lo after phase A
+constexpr uint32_t SM_GM = SM_BH;     // 8 KB + 8 KB masked G tiles hi | lo, K-major (N = 16 t, K = s)
+constexpr uint32_t SM_KT = 180224;    // 16 KB      K_prev hi (p-contiguous rows)
+constexpr uint32_t SM_KTL = 196608;   // 16 KB      K_prev lo
+constexpr uint32_t SM_F32 = 212992;
+constexpr uint32_t SM_BAR = SM_F32 + chunkfwd::F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace chunkbwd
+
+__global__ void __launch_bounds__(chunkfwd::THREADS, 1)
+k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmDY, Params p) {
+    using namespace chunkfwd;
+    using namespace umma;
+    namespace cb = chunkbwd;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + cb::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + cb::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 2;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
+    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, L = p.L;
+    const int nmode = p.nr + p.np;
+    const int nchunk = (L + Q - 1) / Q;
+    const int nbox = N / 64;
+    const uint32_t tile_bytes = 2u * Q * PD * 2 + (uint32_t)Q * N * 2;
+
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        mbar_fence_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmDY);
+    }
+    if (warp == 0) tmem_alloc(tslot, cb::TMEM_COLS);
+    for (int m = tid; m < NP; m += THREADS) {
+        float a2 = 0.f, w = 0.f;
+        if (m < nmode) {
+            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
+            if (m >= nr) w = p.theta[h * p.np + (m - nr)];
+        }
+        f32[F_A2 + m] = a2;
+        f32[F_W + m] = w;
+    }
+    for (int i = tid; i < (int)((cb::SM_F32 - cb::SM_BI) / 16); i += THREADS)
+        reinterpret_cast<uint4 *>(sm + cb::SM_BI)[i] = make_uint4(0, 0, 0, 0);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_st = tbase;          // chunk state (M=128), cols 0..63
+    const uint32_t t_v = tbase + 64u;     // V^T (M=128), cols 64..127
+    const uint32_t t_g = tbase + 128u;    // G (M=64, lanes 0-15 per quarter) then D_i (M=128)
+
+    if (tid == 0) {
+        for (int c = 0; c < 2 && c < nchunk; ++c) {
+            mbar_expect_tx(&bar_tma[c], tile_bytes);
+            tma_load_4d(sm + cb::SM_X + c * 8192, &tmX, &bar_tma[c], 0, h, c * Q, b);
+            tma_load_4d(sm + cb::SM_DY + c * 8192, &tmDY, &bar_tma[c], 0, h, c * Q, b);
+            for (int k = 0; k < nbox; ++k)
+                tma_load_4d(sm + cb::SM_B + c * 16384 + k * 8192, &tmB, &bar_tma[c], 64 * k, g,
+                            c * Q, b);
+        }
+    }
+
+    float K[PD];
+    const bool chain_thr = tid < NP;
+    {
+        float beta0 = 0.f;
+        if (p.two_ep && L > 0)
+            beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+        if (chain_thr) {
+            const int n = tid;
+#pragma unroll
+            for (int q = 0; q < PD; ++q) {
+                float v = 0.f;
+                if (n < N) {
+                    if (p.h0) v = p.h0[ix_st(p, b, h, n, q)];
+                    if (p.w0) v = fmaf(beta0, p.w0[ix_st(p, b, h, n, q)], v);
+                }
+                K[q] = v;
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < PD / 8; ++q8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
+                st16_split(sm + cb::SM_KT, sm + cb::SM_KTL, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
+            }
+        }
+    }
+    const int t_loc = tid & 63;
+    const int grp = tid >> 6;
+
+    for (int c = 0; c < nchunk; ++c) {
+        const int st = c & 1;
+        const int t0 = c * Q;
+        unsigned char *sX = sm + cb::SM_X + st * 8192;
+        unsigned char *sB = sm + cb::SM_B + st * 16384;
+        unsigned char *sDY = sm + cb::SM_DY + st * 8192;
+
+        for (int i = tid; i < Q + 1; i += THREADS) {
+            const int t = t0 + i;
+            float dv = 0.f, lv = 1.f;
+            if (t < L) {
+                dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+                if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+            }
+            f32[F_DT + i] = dv;
+            f32[F_LAM + i] = lv;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
+            float v = d0 + d1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            f32[F_S + 2 * lane] = v - d1;
+            f32[F_S + 2 * lane + 1] = v;
+        } else if (warp == 1 || warp == 2) {
+            const int t = (warp - 1) * 32 + lane;
+            const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
+            const float bn = (t0 + t + 1 < L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
+            f32[F_SIG + t] = fmaf(lv, dv, bn);
+            f32[F_BN + t] = bn;
+        }
+        if (!mbar_wait(&bar_tma[st], (uint32_t)((c >> 1) & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        __syncthreads();
+        if (*abort_flag) break;
+
+        // per-mode chunk constants (as in the forward)
+        for (int m = tid; m < nmode; m += THREADS) {
+            const float a2 = f32[F_A2 + m], w = f32[F_W + m];
+            float er[4], ei[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
+                const float ds = f32[F_S + 16 * k + 15] - lo;
+                const float mag = exp2f(a2 * ds);
+                if (m >= nr) {
+                    float sn, cs;
+                    sincosf(w * ds, &sn, &cs);
+                    er[k] = mag * cs;
+                    ei[k] = mag * sn;
+                } else {
+                    er[k] = mag;
+                    ei[k] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float pr = 1.f, pi = 0.f;
+#pragma unroll
+                for (int j = i + 1; j <= 4; ++j) {
+                    float nr_, ni_;
+                    cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
+                    pr = nr_;
+                    pi = ni_;
+                    f32[F_KRE + fslot(i, j) * NP + m] = pr;
+                    f32[F_KIM + fslot(i, j) * NP + m] = pi;
+                    if (i == 0 && j < 4) {
+                        f32[F_KRE + gslot(j) * NP + m] = pr;
+                        f32[F_KIM + gslot(j) * NP + m] = -pi;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // B-side operands: own-block Bi, later-block copies, Bh
+        {
+            const int t = t_loc;
+            const int ib = t >> 4;
+            const float St = f32[F_S + t];
+            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+            const float ds = St - Sb;
+            const float sig = f32[F_SIG + t];
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const int r0 = 8 * (grp + 4 * k);
+                if (r0 >= N) break;
+                float vBI[8], vBH[8], vBX[3][8], rb[8];
+                ld_rows8(sB, t, r0, rb);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int r = r0 + j;
+                    const float b0 = rb[j], b1 = rb[j + 1];
+                    float bi0, bi1;
+                    int m0, m1;
+                    bool pair;
+                    if (r < nr) {
+                        pair = false;
+                        m0 = r;
+                        m1 = r + 1;
+                        bi0 = sig * b0 * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
+                        bi1 = sig * b1 * ex2_fast(fminf(-f32[F_A2 + m1] * ds, 120.f));
+                    } else {
+                        pair = true;
+                        m0 = m1 = nr + ((r - nr) >> 1);
+                        float sn, cs;
+                        __sincosf(f32[F_W + m0] * ds, &sn, &cs);
+                        const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
+                        bi0 = eb * fmaf(b0, cs, b1 * sn);
+                        bi1 = eb * fmaf(b1, cs, -b0 * sn);
+                    }
+                    vBI[j] = bi0;
+                    vBI[j + 1] = bi1;
+                    if (!pair) {
+                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
+                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            const int i2 = ib + 1 + q;
+                            if (i2 < 4) {
+                                vBX[q][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
+                                vBX[q][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                            }
+                        }
+                    } else {
+                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m0],
+                             f32[F_KIM + fslot(ib, 4) * NP + m0], vBH[j], vBH[j + 1]);
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            const int i2 = ib + 1 + q;
+                            if (i2 < 4)
+                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m0],
+                                     f32[F_KIM + fslot(ib, i2) * NP + m0], vBX[q][j],
+                                     vBX[q][j + 1]);
+                        }
+                    }
+                }
+                st16_split(sm + cb::SM_BI + bi_off(ib), sm + cb::SM_BIL + bi_off(ib),
+                           off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    const int i2 = ib + 1 + q;
+                    if (i2 < 4)
+                        st16_split(sm + cb::SM_BI + bi_off(i2), sm + cb::SM_BIL + bi_off(i2),
+                                   off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[q]);
+                }
+                st16_split(sm + cb::SM_BH, sm + cb::SM_BHL, off_mnmaj(r0, t, 2048u, 128u), vBH);
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // phase A: chunk state, V^T = K_prev dY^T, G = dY X^T
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sX), dy_base = smem_u32(sDY);
+            const uint32_t id_st = idesc_bf16(128, 64, true, true);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t bh_base = smem_u32(sm + (part ? cb::SM_BHL : cb::SM_BH));
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(t_st, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                             sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_st,
+                             part > 0 || s > 0);
+            }
+            const uint32_t id_v = idesc_bf16(128, 64, false, false);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t kt_base = smem_u32(sm + (part ? cb::SM_KTL : cb::SM_KT));
+                for (int s = 0; s < PD / 16; ++s)
+                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
+            }
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int s = 0; s < PD / 16; ++s)
+                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
+            mma_commit(&bar_mma[0]);
+        }
+        if (!mbar_wait(&bar_mma[0], (uint32_t)(c & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        fence_after_sync();
+        __syncthreads();
+        if (*abort_flag) break;
+
+        if (warp < 4) {
+            // carried state K_c = e^{lam S_63} K_{c-1} + S_chunk  (as in the forward)
+            const int n = tid;
+            const int m = n < nr ? n : nr + ((n - nr) >> 1);
+            const bool pr_row = n >= nr && n < N;
+            const bool im_row = pr_row && ((n - nr) & 1);
+            float dr = 0.f, di = 0.f;
+            if (n < N) {
+                dr = f32[F_KRE + fslot(0, 4) * NP + m];
+                di = f32[F_KIM + fslot(0, 4) * NP + m];
+            }
+#pragma unroll
+            for (int c16 = 0; c16 < PD / 16; ++c16) {
+                float sv[16];
+                tmem_ld16(tmem_addr(t_st, 32u * warp, 16u * c16), sv);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int q = c16 * 16 + j;
+                    const float own = K[q];
+                    const float other = __shfl_xor_sync(0xffffffffu, own, 1);
+                    float nv;
+                    if (!pr_row)
+                        nv = fmaf(dr, own, sv[j]);
+                    else if (!im_row)
+                        nv = fmaf(dr, own, fmaf(-di, other, sv[j]));
+                    else
+                        nv = fmaf(di, other, fmaf(dr, own, sv[j]));
+                    K[q] = n < N ? nv : 0.f;
+                }
+            }
+        } else {
+            // masked G rows -> K-major tiles (N = 16 t of block i, K = s); diagonal dy_t . u_t
+            const int qd = warp - 4;
+            for (int i = 0; i < NSB; ++i) {
+                float v[16];
+                tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
+                if (lane < 16 && i <= qd) {
+                    const int t = 16 * qd + lane;
+                    float lo[8], hi[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
+                        hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
+                    }
+                    unsigned char *gt = sm + cb::SM_GM + qd * 2048;
+                    st16_split(gt, gt + 8192, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
+                    st16_split(gt, gt + 8192, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
+                    if (i == qd) f32[F_CORR + t] = v[lane];
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // phase B: D_i = Bi^T (G o mask)_i^T into the (now free) G columns
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id_d = idesc_bf16(128, 16, true, false);
+            // hi*hi + hi*lo + lo*hi
+            const uint32_t a_off[3] = {cb::SM_BI, cb::SM_BI, cb::SM_BIL};
+            const uint32_t b_off[3] = {cb::SM_GM, cb::SM_GM + 8192u, cb::SM_GM};
+            for (int i = 0; i < NSB; ++i)
+                for (int part = 0; part < 3; ++part) {
+                    const uint32_t bi_base = smem_u32(sm + a_off[part]);
+                    const uint32_t gm_base = smem_u32(sm + b_off[part]);
+                    for (int s = 0; s <= i; ++s)
+                        mma_bf16(t_g + 16 * i,
+                                 sdesc(bi_base + bi_off(i) + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                                 sdesc(gm_base + i * 2048u + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                                 id_d, part > 0 || s > 0);
+                }
+            mma_commit(&bar_mma[1]);
+        }
+        // the state tile for the next chunk's V^T (phase A of this chunk has consumed it)
+        if (warp < 4) {
+            const int n = tid;
+            if (p.ws_kb && c + 1 < nchunk && n < N) {
+                float4 *kb = reinterpret_cast<float4 *>(
+                    p.ws_kb + ((((long long)b * p.H + h) * p.nc + c) * N + n) * PD);
+#pragma unroll
+                for (int q4 = 0; q4 < PD / 4; ++q4)
+                    kb[q4] = make_float4(K[4 * q4], K[4 * q4 + 1], K[4 * q4 + 2], K[4 * q4 + 3]);
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < PD / 8; ++q8) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
+                st16_split(sm + cb::SM_KT, sm + cb::SM_KTL, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
+            }
+        }
+        if (!mbar_wait(&bar_mma[1], (uint32_t)(c & 1), WAIT_LIMIT)) {
+            raise_error(1);
+            *abort_flag = 1;
+        }
+        fence_after_sync();
+        fence_proxy_async();
+        __syncthreads();
+        if (*abort_flag) break;
+
+        // unfold: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D ; dC_t = dCK_t - beta' (dy.u) B_t
+        {
+            const int n = tid & 127;
+            const int half = tid >> 7;
+            const int qd = warp & 3;
+            const bool valid = n < N;
+            const int m = n < nr ? n : nr + ((n - nr) >> 1);
+            const bool pr_row = valid && n >= nr;
+            const bool im_row = pr_row && ((n - nr) & 1);
+            const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
+            float *dst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+            const long long tstride = (long long)p.H * p.N;
+            for (int c16 = 0; c16 < 2; ++c16) {
+                const int tc = 32 * half + 16 * c16;
+                float vv[16], dd[16];
+                tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
+                tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), dd);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int t = tc + j;
+                    const int ib = t >> 4;
+                    const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+                    const float ds = f32[F_S + t] - Sb;
+                    // E' = e^{lam ds}, E = E' * e^{lam Sb_i} = E' * conj(G_i)
+                    const float mag = ex2_fast(a2 * ds);
+                    float er = mag, ei = 0.f;
+                    if (pr_row) {
+                        float sn, cs;
+                        __sincosf(w * ds, &sn, &cs);
+                        er = mag * cs;
+                        ei = mag * sn;
+                    }
+                    float fr = 1.f, fi = 0.f;
+                    if (ib && valid) {
+                        fr = f32[F_KRE + gslot(ib) * NP + m];
+                        fi = -f32[F_KIM + gslot(ib) * NP + m];
+                    }
+                    float Er, Ei;
+                    cmul(er, ei, fr, fi, Er, Ei);
+                    const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                    const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
+                    float res;
+                    if (!pr_row) {
+                        res = Er * vv[j] + er * dd[j];
+                    } else if (!im_row) {  // real part of E (V_re + i V_im) + E' (D_re + i D_im)
+                        res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
+                    } else {               // imaginary part
+                        res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
+                    }
+                    if (valid && t0 + t < L) {
+                        const float bt = ld_row1(sB, t, n);
+                        dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
+                    }
+                }
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0 && c + 2 < nchunk) {
+            mbar_expect_tx(&bar_tma[st], tile_bytes);
+            tma_load_4d(sm + cb::SM_X + st * 8192, &tmX, &bar_tma[st], 0, h, (c + 2) * Q, b);
+            tma_load_4d(sm + cb::SM_DY + st * 8192, &tmDY, &bar_tma[st], 0, h, (c + 2) * Q, b);
+            for (int k = 0; k < nbox; ++k)
+                tma_load_4d(sm + cb::SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g,
+                            (c + 2) * Q, b);
+        }
+    }
+    if (*abort_flag && tid == 0) {
+        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
+        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, cb::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -649,6 +1172,14 @@ bool chunk_fwd_supported(const Params &p) {
            chunkfwd::encode_fn() != nullptr;
 }
 
+// The tensor-core backward part additionally reads dy through TMA.
+bool chunk_bwd_supported(const Params &p) {
+    auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
+    auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
+    return chunk_fwd_supported(p) && p.dy && al16(p.dy) && st16(p.sy[0]) && st16(p.sy[1]) &&
+           st16(p.sy[2]);
+}
+
 cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     using namespace chunkfwd;
     CUtensorMap mx, mb, mc;
@@ -665,6 +1196,27 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     }
     k_chunk_fwd<<<dim3(p.H, p.Bsz), THREADS, SMEM_BYTES, st>>>(mx, mb, mc, p);
     profile_mark(st, "k_chunk_fwd");
+    return cudaGetLastError();
+}
+
+// Backward forward-direction part on the tensor cores: per-head dC into p.ws_dC.
+cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st) {
+    using namespace chunkfwd;
+    CUtensorMap mx, mb, mdy;
+    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
+        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
+        !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
+        return cudaErrorInvalidValue;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(k_chunk_bwd_dc,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)chunkbwd::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    k_chunk_bwd_dc<<<dim3(p.H, p.Bsz), THREADS, chunkbwd::SMEM_BYTES, st>>>(mx, mb, mdy, p);
+    profile_mark(st, "k_chunk_bwd_dc");
     return cudaGetLastError();
 }
 

@@ -576,9 +576,54 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
             xreduce<KV, S>(v, lane_in_s);
             put_reduced<KV, S>(redA + (((ln.hc * T + tt) * NWP + wp) * NQ + ln.q) * KV, v,
                                lane_in_s);
-            // G <- A_t^T G
             float cf[NS];
             ld_slots<NS>(cf, s.coef + (ln.hc * T + tt) * NSL + ln.q * NS);
+            // at a 64-token chunk start: per row, sum_p conj(Gbar_t) A_t K_{t-1} from the saved
+            // chunk-end state (the exact carry of the decay-gradient scan)
+            const int tg = t0 + tt;
+            if (p.ws_qb && tg > 0 && (tg & 63) == 0) {
+                const int cc = tg >> 6;
+                const float *kb = p.ws_kb + (((long long)ln.b * p.H + (ln.hv ? ln.h : 0)) * p.nc +
+                                             (cc - 1)) * (long long)p.N * p.P;
+                float kv[NS];
+#pragma unroll
+                for (int sl = 0; sl < NS; ++sl) {
+                    const int n = row_of<NR, NPR>(ln.q, sl, p.nr, p.np, NQ);
+                    kv[sl] = (ln.hv && n >= 0 && ln.pl < p.P) ? kb[(long long)n * p.P + ln.pl] : 0.f;
+                }
+                float qv[NS];
+#pragma unroll
+                for (int i = 0; i < NR; ++i) qv[i] = Gv[i] * cf[i] * kv[i];
+#pragma unroll
+                for (int j = 0; j < NPR; ++j) {
+                    const float ec = cf[NR + 2 * j], es = cf[NR + 2 * j + 1];
+                    const float kr = kv[NR + 2 * j], ki = kv[NR + 2 * j + 1];
+                    const float ar = fmaf(ec, kr, -es * ki), ai = fmaf(es, kr, ec * ki);
+                    const float gr = Gv[NR + 2 * j], gi = Gv[NR + 2 * j + 1];
+                    qv[NR + 2 * j] = fmaf(gr, ar, gi * ai);
+                    qv[NR + 2 * j + 1] = fmaf(gr, ai, -gi * ar);
+                }
+                xreduce<NS, S>(qv, lane_in_s);
+                if (ln.hv) {
+                    float *dst = p.ws_qb + ((((long long)ln.b * p.H + ln.h) * p.nc + cc) * 4 + wp) *
+                                               (long long)p.N;
+                    if constexpr (NS >= S) {
+                        constexpr int KS = NS / S;
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            const int n = row_of<NR, NPR>(ln.q, lane_in_s * KS + i, p.nr, p.np, NQ);
+                            if (n >= 0) dst[n] = qv[i];
+                        }
+                    } else {
+                        constexpr int SK = S / NS;
+                        if (lane_in_s % SK == 0) {
+                            const int n = row_of<NR, NPR>(ln.q, lane_in_s / SK, p.nr, p.np, NQ);
+                            if (n >= 0) dst[n] = qv[0];
+                        }
+                    }
+                }
+            }
+            // G <- A_t^T G
             step_adj<NR, NPR>(Gv, cf);
         }
         __syncthreads();
@@ -696,7 +741,7 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
 // order.
 // ------------------------------------------------------------------------
 constexpr int FT = 32;
-constexpr int TBL = 128;
+constexpr int TBL = 64;   // equal to the tensor-core chunk, whose boundaries carry exact values
 
 __host__ __device__ inline int ntb_of(const Params &p) { return (p.L + TBL - 1) / TBL; }
 
@@ -814,9 +859,22 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
     const ModeInfo mi = mode_info(p, h, m);
     float *s_c = smem;  // [nthr]
     float car = 0.f, cai = 0.f, dA = 0.f, dth = 0.f, dD = 0.f;
+    const int nwp = p.P > 32 ? (p.P + 31) / 32 : 1;
     for (int tb = NTB - 1; tb >= 0; --tb) {
         const float *blk = p.ws_blk + (((long long)b * p.H + h) * NTB + tb) * (4 * (long long)nmode + 2);
         const float sdt = blk[4 * nmode + 0];
+        if (p.ws_qb && mi.valid) {
+            // exact carry from the chunk boundary: sum_p conj(Gbar) A K_prev at the next block start
+            car = 0.f;
+            cai = 0.f;
+            if (tb + 1 < NTB) {
+                const float *q = p.ws_qb + (((long long)b * p.H + h) * p.nc + (tb + 1)) * 4 * (long long)p.N;
+                for (int w2 = 0; w2 < nwp; ++w2) {
+                    car += q[w2 * p.N + mi.n0];
+                    if (mi.pair) cai += q[w2 * p.N + mi.n0 + 1];
+                }
+            }
+        }
         float contrib = 0.f;
         if (mi.valid) {
             dA += blk[4 * m + 2] + car * sdt;
@@ -831,7 +889,7 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
             p.ws_blkc[((long long)b * p.H + h) * NTB + tb] = acc;
             dD += blk[4 * nmode + 1];
         }
-        if (mi.valid) {
+        if (mi.valid && !p.ws_qb) {
             car += blk[4 * m + 0];
             cai += blk[4 * m + 1];
         }
@@ -960,14 +1018,15 @@ __global__ void k_copy_state(Params p) {
 struct Combo {
     int NR, NPR;
 };
-static const Combo kCombos[] = {{16, 8}, {32, 0}, {8, 4}, {16, 0}};
+static const Combo kCombos[] = {{16, 8}, {32, 0}, {8, 4}, {16, 0}, {0, 16}};
 
 static int pick_combo(const Params &p, int &NQ) {
     int best = -1, bestw = 1 << 30, bestq = 0;
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 5; ++c) {
         const Combo &k = kCombos[c];
         if (p.np > 0 && k.NPR == 0) continue;
-        int q1 = (p.nr + k.NR - 1) / k.NR;
+        if (p.nr > 0 && k.NR == 0) continue;
+        int q1 = k.NR ? (p.nr + k.NR - 1) / k.NR : 0;
         int q2 = k.NPR ? (p.np + k.NPR - 1) / k.NPR : 0;
         int q = q1 > q2 ? q1 : q2;
         if (q < 1) q = 1;
@@ -1031,7 +1090,7 @@ static size_t plan(Params &p, int kind, int &combo, int &RM, int &S) {
 
 template <int NR, int NPR>
 constexpr int combo_id() {
-    return NR == 16 && NPR == 8 ? 0 : (NR == 32 ? 1 : (NR == 8 ? 2 : 3));
+    return NR == 16 && NPR == 8 ? 0 : (NR == 32 ? 1 : (NR == 8 ? 2 : (NR == 16 ? 3 : 4)));
 }
 
 template <int NR, int NPR, int RM, int S>
@@ -1076,6 +1135,7 @@ static cudaError_t launch_scan(int kind, Params p, cudaStream_t st) {
         SSM_CASES(32, 0)
         SSM_CASES(8, 4)
         SSM_CASES(16, 0)
+        SSM_CASES(0, 16)
         default:
             return cudaErrorInvalidConfiguration;
     }
@@ -1101,9 +1161,17 @@ cudaError_t simt_forward(const Params &p, cudaStream_t st) {
     return launch_scan(KK_FWD, p, st);
 }
 
-cudaError_t simt_backward(const Params &p, cudaStream_t st) {
+bool chunk_bwd_supported(const Params &p);
+cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st);
+
+// use_chunk: per-head dC from the tensor-core kernel instead of sweep 1
+cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk) {
     cudaError_t e;
-    if ((e = launch_scan(KK_S1, p, st)) != cudaSuccess) return e;
+    if (use_chunk)
+        e = chunk_bwd_dc(p, st);
+    else
+        e = launch_scan(KK_S1, p, st);
+    if (e != cudaSuccess) return e;
     if ((e = launch_scan(KK_S2, p, st)) != cudaSuccess) return e;
     {
         int nthr = ((p.nr + p.np + 31) / 32) * 32;

@@ -10,9 +10,11 @@ using namespace ssm::umma;
 
 // layout codes: 0 = K-major no swizzle, 1 = MN-major no swizzle,
 //               2 = MN-major 128-byte swizzle (64-element rows along MN, rows = K)
+//               3 = K-major 128-byte swizzle (64-element rows along K, rows = MN)
 __device__ uint32_t place(int code, int mn, int k, int MN, int K) {
     if (code == 0) return off_kmaj(mn, k, 128u, (uint32_t)(K / 8) * 128u);
     if (code == 1) return off_mnmaj(mn, k, (uint32_t)(MN / 8) * 128u, 128u);
+    if (code == 3) return off_sw128(mn, k);
     return off_sw128(k, mn);
 }
 __device__ uint64_t desc_for(int code, uint32_t base, int step, int MN, int K) {
@@ -21,6 +23,7 @@ __device__ uint64_t desc_for(int code, uint32_t base, int step, int MN, int K) {
         uint32_t lbo = (uint32_t)(MN / 8) * 128u;
         return sdesc(base + step * 2u * lbo, lbo, 128u, LAYOUT_NONE);
     }
+    if (code == 3) return sdesc(base + step * 32u, 16u, 1024u, LAYOUT_SW128);
     return sdesc(base + step * 2048u, 8192u, 1024u, LAYOUT_SW128);
 }
 
@@ -56,7 +59,7 @@ umma_probe(int M, int N, int K, int a_code, int b_code, int d_lane, const float 
     fence_after_sync();
     const uint32_t tbase = tslot;
     if (tid == 0) {
-        const uint32_t id = idesc_bf16(M, N, a_code != 0, b_code != 0);
+        const uint32_t id = idesc_bf16(M, N, a_code == 1 || a_code == 2, b_code == 1 || b_code == 2);
         for (int s = 0; s < K / 16; ++s)
             mma_bf16(tmem_addr(tbase, (uint32_t)d_lane, 0), desc_for(a_code, smem_u32(sA), s, M, K),
                      desc_for(b_code, smem_u32(sB), s, N, K), id, s > 0);

@@ -75,11 +75,11 @@ def test_workload_parity(name):
 
 
 @pytest.mark.parametrize("name", ["mamba2_siso", "hybridmamba"])
-def test_workload_parity_recurrent_forward(name):
+def test_workload_parity_recurrent_path(name):
     """The same workloads through the token-by-token kernels (chunk = 1)."""
     shape = S.WORKLOADS[name].replace(**REDUCED[name]).replace(chunk=1)
     inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(name))
-    check_all(shape, inp, backward=False)
+    check_all(shape, inp)
 
 
 @pytest.mark.parametrize("kw", [
@@ -90,13 +90,13 @@ def test_workload_parity_recurrent_forward(name):
     dict(seqlen=100, decay_mode=S.DECAY_PER_HEAD, two_endpoint=0, n_real=128, n_pairs=0,
          ngroups=2),
 ])
-def test_chunked_forward_shapes(kw):
-    """Chunked tensor-core forward: ragged tails around the 64-token chunk,
+def test_chunked_shapes(kw):
+    """Chunked tensor-core kernels: ragged tails around the 64-token chunk,
     64/128 state rows, real-only, pairs-only, grouped B/C, initial state."""
     base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, chunk=64)
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=31, with_state=True)
-    check_all(shape, inp, backward=False)
+    check_all(shape, inp)
 
 
 @pytest.mark.parametrize("name", S.WORKLOAD_ORDER)

@@ -40,6 +40,9 @@ def bf16(a):
     (64, 64, 64, 2, 1, 0),    # swizzled MN-major A (X^T), MN-major B (P^T)
     (64, 16, 64, 0, 0, 16),   # M=64 accumulator in the upper half-lanes
     (64, 64, 32, 1, 0, 0),    # MN-major A (state^T), K-major B
+    (64, 64, 64, 3, 3, 0),    # 128B-swizzled K-major A and B (dY . X^T)
+    (128, 64, 64, 0, 3, 0),   # K-major A (state rows), swizzled K-major B (K_prev . dY^T)
+    (128, 16, 32, 1, 0, 0),   # MN-major A read from a K-major tile, K-major B (B_i^T . Gm^T)
 ])
 def test_umma_layout(probe, M, N, K, a_code, b_code, d_lane):
     cu, fn = probe
