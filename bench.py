@@ -80,29 +80,45 @@ def bwd_bytes(shape):
 
 
 def kernel_bytes(shape, name: str) -> int:
-    """Algorithmic bytes of one launch of each kernel of the recurrent path."""
+    """Algorithmic bytes of one launch of each kernel: the path's inputs that the
+    kernel has to read and the path's outputs it writes, each counted once.
+    Workspace traffic between kernels is overhead of the design and is not
+    counted, so a kernel that only touches workspace has 0 here."""
     s = shape
     t = tensor_bytes(shape)
     BLH = s.batch * s.seqlen * s.nheads
     ins = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
+    dy = t["y"]
     if name in ("k_fwd", "k_chunk_fwd"):
         return ins + t["y"]
     if name == "k_bwd_sweep1":   # inputs + dy -> per-head dC (fp32)
-        return ins + t["y"] + BLH * s.rank_out * s.nstate * 4
+        return ins + dy + BLH * s.rank_out * s.nstate * 4
     if name == "k_bwd_sweep2":   # inputs + dy -> dx, sum_p G u^T (fp32), per-token scalars
-        return (ins + t["y"] + t["x"] + BLH * s.rank_in * s.nstate * 4
+        return (ins + dy + t["x"] + BLH * s.rank_in * s.nstate * 4
                 + BLH * (2 + s.rank_in * s.rank_out) * 4)
-    if name == "k_bwd_units":
+    if name == "k_bwd_units_local":
         return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["B"] + t["C"]
                 + 2 * t["dt"] + 2 * t["lam"] + BLH * (2 + s.rank_in * s.rank_out) * 4)
     if name == "k_bwd_groups":
         return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["C"] + t["B"] + t["C"]
                 + t["dt"] + t["lam"])
+    # tensor-core backward: path inputs read, path outputs written
+    if name == "k_chunk_bwd_dc":      # x, B, dt, lambda, dy
+        return t["x"] + t["B"] + t["dt"] + t["lam"] + dy
+    if name == "k_chunk_adj_local":   # C, dt, dy
+        return t["C"] + t["dt"] + dy
+    if name == "k_chunk_bwd_dx":      # B, C, dt, lambda, dy -> dx
+        return t["B"] + t["C"] + t["dt"] + t["lam"] + dy + t["x"]
+    if name == "k_chunk_bwd_gbu":     # x, B, C, dt, lambda, dy -> dB, dC (one head per group)
+        out = t["B"] + t["C"] if s.nheads == s.ngroups else 0
+        return ins + dy + out
+    if name == "k_bwd_units_final":   # dt, lambda -> ddt, dlambda
+        return 2 * (t["dt"] + t["lam"])
     return 0
 
 
-FWD_KERNELS = ["k_fwd"]
-BWD_KERNELS = ["k_bwd_sweep1", "k_bwd_sweep2", "k_bwd_units", "k_bwd_groups", "k_bwd_params"]
+# upper bound on library launches per fwd + bwd step (sizes the profiling session)
+LAUNCHES_PER_STEP = 16
 
 
 # ---------------------------------------------------------------------------
@@ -301,7 +317,7 @@ def main():
     abi.ssm_scan_poll_device_error()
 
     # per-kernel events over the timed region (library-owned, on our stream)
-    launches_per_step = len(FWD_KERNELS) + len(BWD_KERNELS)
+    launches_per_step = LAUNCHES_PER_STEP
     clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
     clocks.start()

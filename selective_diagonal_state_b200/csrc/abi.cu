@@ -19,6 +19,7 @@ bool chunk_bwd_supported(const Params &p);
 bool chunk_fwd_supported(const Params &p);
 cudaError_t chunk_forward(const Params &p, cudaStream_t st);
 int chunk_error_take();
+int chunk_rev_error_take();
 }  // namespace ssm
 
 namespace {
@@ -135,7 +136,7 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
 
 struct BwdWs {
     size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, off_kb, off_qb,
-        total;
+        off_gc, off_ce, total;
     bool boundary;  // chunk-boundary carries (tensor-core backward shapes)
 };
 
@@ -170,12 +171,16 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     w.off_blkc = off;
     off = align256(off + (size_t)d->batch * d->nheads * ntb * 4);
     w.boundary = tensor_bwd_shape(d);
-    w.off_kb = w.off_qb = off;
+    w.off_kb = w.off_qb = w.off_gc = w.off_ce = off;
     if (w.boundary) {
         w.off_kb = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
         w.off_qb = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 4 * N * 4);
+        w.off_gc = off;
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
+        w.off_ce = off;
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * 2 * 4);
     }
     w.total = off;
     return w;
@@ -333,6 +338,8 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     if (chunked && lay.boundary) {
         p.ws_kb = (float *)(ws + lay.off_kb);
         p.ws_qb = (float *)(ws + lay.off_qb);
+        p.ws_gc = (float *)(ws + lay.off_gc);
+        p.ws_ce = (float *)(ws + lay.off_ce);
     }
     profile_begin(st);
     cudaError_t e = ssm::simt_backward(p, st, chunked);
@@ -347,7 +354,9 @@ const char *ssm_scan_last_error(void) { return g_last_error.c_str(); }
 int ssm_scan_poll_device_error(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_poll_device_error");
-    const int word = ssm::chunk_error_take();
+    int word = ssm::chunk_error_take();
+    const int word2 = ssm::chunk_rev_error_take();
+    if (word == 0 || word2 < 0) word = word2;
     if (word < 0) return fail(SSM_ERR_CUDA, "ssm_scan_poll_device_error: cannot read the error word");
     if (word == 1) return fail(SSM_ERR_TIMEOUT, "a bounded device-side wait gave up");
     if (word != 0) return fail(SSM_ERR_TIMEOUT, "device-side error code %d", word);

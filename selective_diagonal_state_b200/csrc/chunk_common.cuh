@@ -1,0 +1,135 @@
+// Pieces shared by the chunked tensor-core kernels (64-token chunks of four
+// 16-token sub-blocks, bf16 operands, fp32 accumulation): sizes, the fp32
+// scratch map, bf16 packing, reads of 128-byte-swizzled B/C tiles, mode
+// constants slots, and the host-side TMA descriptor encoder.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace ssm {
+namespace chunkc {
+
+using namespace umma;
+
+constexpr int Q = 64;
+constexpr int NSB = 4;
+constexpr int NP = 128;   // state rows (K) padded
+constexpr int PD = 64;    // head dim
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+
+// fp32 scratch (float offsets from SM_F32)
+constexpr int F_S = 0, F_SIG = 64, F_BN = 128, F_CORR = 192, F_DT = 256, F_LAM = 328;
+constexpr int F_CP = 400;                 // [4][64] corr partials
+constexpr int F_A2 = 656;                 // [128] decay * log2(e) per mode
+constexpr int F_W = 784;                  // [128] rotation frequency per mode
+constexpr int F_KRE = 912;                // [13][128] mode constants, real part
+constexpr int F_KIM = F_KRE + 13 * 128;   // [13][128] imaginary part
+constexpr int F_END = F_KIM + 13 * 128;
+
+constexpr uint32_t KM_LBO = 128, KM_SBO = 2048;  // K-major tiles with K = 128
+
+__device__ __forceinline__ uint32_t bi_off(int i) {
+    return i == 0 ? 0u : (i == 1 ? 4096u : (i == 2 ? 12288u : 24576u));
+}
+// mode-constant slots: F[i][j] = prod_{k=i}^{j-1} E_k (0 <= i < j <= 4), G[i] = conj(F[0][i])
+__device__ __forceinline__ int fslot(int i, int j) {
+    return (i == 0 ? 0 : (i == 1 ? 4 : (i == 2 ? 7 : 9))) + (j - i - 1);
+}
+__device__ __forceinline__ int gslot(int i) { return 10 + (i - 1); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void st16(unsigned char *base, uint32_t off, const float (&v)[8]) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(base + off) = w;
+}
+// store v as bf16 hi (at hi + off) and the bf16 residual v - hi (at lo + off)
+__device__ __forceinline__ void st16_split(unsigned char *hi, unsigned char *lo, uint32_t off,
+                                           const float (&v)[8]) {
+    float h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+        l[i] = v[i] - h[i];
+    }
+    st16(hi, off, h);
+    st16(lo, off, l);
+}
+__device__ __forceinline__ float bf(const unsigned char *p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+}
+// 8 consecutive state rows r0..r0+7 of token t from a raw B/C tile
+// (two 64-row halves, each 64 tokens x 128 bytes with the 128-byte swizzle).
+__device__ __forceinline__ void ld_rows8(const unsigned char *tile, int t, int r0, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(tile + (r0 >> 6) * 8192 +
+                                                     off_sw128(t, r0 & 63));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(u[i] << 16);
+        v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ float ld_row1(const unsigned char *tile, int t, int r) {
+    return bf(tile + (r >> 6) * 8192 + off_sw128(t, r & 63));
+}
+
+// 2^x with the hardware approximation (operands are rounded to bf16 afterwards)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// complex multiply (a + ib)(c + id)
+__device__ __forceinline__ void cmul(float a, float b, float c, float d, float &re, float &im) {
+    re = fmaf(a, c, -b * d);
+    im = fmaf(a, d, b * c);
+}
+
+// ---- host side ---------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 4-D bf16 map over (inner, dim1, time, batch) with a box of (inner, 1, Q, 1).
+static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t d1, uint64_t L,
+                     uint64_t B, uint64_t s1, uint64_t sL, uint64_t sB, uint32_t box_inner,
+                     bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {inner, d1, L, B};
+    cuuint64_t strides[3] = {s1 * 2, sL * 2, sB * 2};
+    cuuint32_t box[4] = {box_inner, 1, (cuuint32_t)Q, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace chunkc
+}  // namespace ssm

@@ -40,6 +40,8 @@ struct Params {
     // exact decay-gradient carries at 64-token chunk boundaries (tensor-core path):
     float *ws_kb;   // [B][H][NC][N][P]  pre-state K at the end of every chunk but the last
     float *ws_qb;   // [B][H][NC][4][N]  per-row sum_p conj(Gbar) A K_prev at chunk starts (per warp of p)
+    float *ws_gc;   // [B][H][NC][N][P]  chunk-local adjoint, then the adjoint carried into each chunk
+    float *ws_ce;   // [B][H][NC][128][2] full-chunk decay e^{lam S_63} per mode (re, im)
     int nc;         // number of 64-token chunks
     Geometry geo;
 };

@@ -1,0 +1,1158 @@
+// Chunk-parallel reverse part of the backward scan on the tensor cores (bf16
+// I/O, fp32 state, SISO, head dim 64, up to 128 state rows).
+//
+// The adjoint of the pre-state, Gbar_t = dL/dK_t, obeys the transposed
+// recurrence Gbar_t = C_t^T dy_t + A_{t+1}^T Gbar_{t+1} ("When a Diagonal State
+// Is Not Enough", sungsoo.github.io Part 01: the linear-transition recurrence,
+// here run backwards).  In the complex packing of a rotation pair, A^T is the
+// conjugate.  Per chunk of 64 tokens with S_t the inclusive sum of dt inside
+// the chunk and Gc the adjoint carried in from later chunks (adjoint of K at
+// the chunk's last token, before that token's own readout term):
+//   Gbar_t = sum_{t' >= t} conj(e^{lam (S_t' - S_t)}) c_t' dy_t'  +  conj(e^{lam (S_63 - S_t)}) Gc
+// so the work splits into
+//   k_chunk_adj_local  (every chunk at once)   Ghat_c = sum_t conj(e^{lam S_t}) c_t dy_t^T
+//   k_chunk_adj_pass   (chunks in reverse)     Gc_{c-1} = conj(e^{lam S_63}) Gc_c + Ghat_c
+//   k_chunk_bwd_dx     (every chunk at once)   dx_s = sum_{t>=s} P_ts dy_t + (Bh_s)^T Gc_c + corr
+//   k_chunk_bwd_gbu    (every chunk at once)   gbu_t = sum_p u_t,p Gbar_t,p
+// where P is the masked score matrix of the forward and Bh_s = sigma_s b_s
+// e^{lam (S_63 - S_s)} (the same folded operands as the chunked forward).  The
+// passing kernel also forms, at every chunk start, the exact boundary value
+// sum_p conj(Gc_{c-1}) K_end_{c-1} of the decay-gradient scan, and writes
+// dL/dh0, dL/dw0 and dL/dbeta_0 after the first chunk.
+#include <cuda.h>
+
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace ssm {
+
+// Device word raised by the bounded waits of these kernels (0 = no error, 1 = a wait gave up).
+__device__ int ssm_chunk_rev_error_word;
+__device__ __forceinline__ void rev_raise_error(int code) {
+    atomicCAS(&ssm_chunk_rev_error_word, 0, code);
+}
+
+namespace chunkrev {
+using namespace umma;
+using namespace chunkc;
+
+// ---- per-chunk token quantities and mode constants ----------------------------
+// Loads dt / lambda of tokens t0 .. t0+64 and writes the inclusive prefix S_t
+// (F_S) and, with `want_sigma`, sigma_t (F_SIG) and beta_{t+1} (F_BN).
+// Call with all threads of the block (>= 96); contains barriers.
+__device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b, int h, int t0,
+                                             bool want_sigma) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < Q + 1; i += blockDim.x) {
+        const int t = t0 + i;
+        float dv = 0.f, lv = 1.f;
+        if (t < p.L) {
+            dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+            if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+        }
+        f32[F_DT + i] = dv;
+        f32[F_LAM + i] = lv;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
+        float v = d0 + d1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        f32[F_S + 2 * lane] = v - d1;
+        f32[F_S + 2 * lane + 1] = v;
+    } else if (want_sigma && (warp == 1 || warp == 2)) {
+        const int t = (warp - 1) * 32 + lane;
+        const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
+        const float bn =
+            (t0 + t + 1 < p.L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
+        f32[F_SIG + t] = fmaf(lv, dv, bn);
+        f32[F_BN + t] = bn;
+    }
+    __syncthreads();
+}
+
+// Per-mode decay over each sub-block, E_k = e^{lam dS_k}, and the products
+// F[i][j] = prod_{k=i}^{j-1} E_k and G_i = conj(F[0][i]) into the F_KRE / F_KIM
+// slots.  Needs F_S, F_A2, F_W.  Ends with a barrier.
+__device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
+    const int nmode = p.nr + p.np;
+    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
+        const float a2 = f32[F_A2 + m], w = f32[F_W + m];
+        float er[4], ei[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
+            const float ds = f32[F_S + 16 * k + 15] - lo;
+            const float mag = exp2f(a2 * ds);
+            if (m >= p.nr) {
+                float sn, cs;
+                sincosf(w * ds, &sn, &cs);
+                er[k] = mag * cs;
+                ei[k] = mag * sn;
+            } else {
+                er[k] = mag;
+                ei[k] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float pr = 1.f, pi = 0.f;
+#pragma unroll
+            for (int j = i + 1; j <= 4; ++j) {
+                float nr_, ni_;
+                cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
+                pr = nr_;
+                pi = ni_;
+                f32[F_KRE + fslot(i, j) * NP + m] = pr;
+                f32[F_KIM + fslot(i, j) * NP + m] = pi;
+                if (i == 0 && j < 4) {
+                    f32[F_KRE + gslot(j) * NP + m] = pr;
+                    f32[F_KIM + gslot(j) * NP + m] = -pi;
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void mode_rates(const Params &p, float *f32, int h) {
+    const int nmode = p.nr + p.np;
+    for (int m = threadIdx.x; m < NP; m += blockDim.x) {
+        float a2 = 0.f, w = 0.f;
+        if (m < nmode) {
+            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
+            if (m >= p.nr) w = p.theta[h * p.np + (m - p.nr)];
+        }
+        f32[F_A2 + m] = a2;
+        f32[F_W + m] = w;
+    }
+}
+
+__device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {
+    return ((long long)b * p.H + h) * p.nc + c;
+}
+
+// ============================================================================
+// k_chunk_adj_local: Ghat_c = Ch^T (N x 64 t) . dY (64 t x 64 p), per chunk.
+//   Ch_t = c_t conj(e^{lam S_t}) = Ci_t G_i (sub-block-relative fold times the
+//   sub-block's start factor), split into bf16 hi + lo.  Also stores the
+//   chunk's full decay F[0][4] per mode for the passing kernel.
+// ============================================================================
+namespace loc {
+constexpr int THREADS = 128;
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint32_t SM_C = 0;        // 16 KB  raw C (two 64-row 128B-swizzled halves)
+constexpr uint32_t SM_DY = 16384;   // 8 KB   dy (128B swizzle)
+constexpr uint32_t SM_CH = 24576;   // 16 KB  Ch hi, K-major (rows t, K = state rows)
+constexpr uint32_t SM_CHL = 40960;  // 16 KB  Ch lo
+constexpr uint32_t SM_F32 = 57344;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace loc
+
+__global__ void __launch_bounds__(loc::THREADS)
+k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                  Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + loc::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + loc::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, nmode = p.nr + p.np;
+    const int t0 = c * Q;
+    const int nbox = N / 64;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmDY);
+        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + Q * N * 2));
+        tma_load_4d(sm + loc::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k)
+            tma_load_4d(sm + loc::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
+    }
+    if (warp == 0) tmem_alloc(tslot, loc::TMEM_COLS);
+    mode_rates(p, f32, h);
+    if (N < NP)  // K padding of the Ch tiles
+        for (int i = tid; i < (int)(32768 / 16); i += loc::THREADS)
+            reinterpret_cast<uint4 *>(sm + loc::SM_CH)[i] = make_uint4(0, 0, 0, 0);
+    chunk_tokens(p, f32, b, h, t0, false);
+    chunk_mode_constants(p, f32);
+    // chunk decay per mode for the passing kernel
+    for (int m = tid; m < nmode; m += loc::THREADS) {
+        float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
+        ce[2 * m] = f32[F_KRE + fslot(0, 4) * NP + m];
+        ce[2 * m + 1] = f32[F_KIM + fslot(0, 4) * NP + m];
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tacc = *tslot;
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) rev_raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // Ch tiles: thread (t, grp) handles rows 8 * (grp + 2k)
+        const int t = tid & 63, grp = tid >> 6;
+        const int ib = t >> 4;
+        const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+        const float ds = f32[F_S + t] - Sb;
+        const unsigned char *sC = sm + loc::SM_C;
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k) {
+            const int r0 = 8 * (grp + 2 * k);
+            if (r0 >= N) break;
+            float rc[8], v[8];
+            ld_rows8(sC, t, r0, rc);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const int r = r0 + j;
+                if (r < nr) {
+                    const float g0 = ib ? f32[F_KRE + gslot(ib) * NP + r] : 1.f;
+                    const float g1 = ib ? f32[F_KRE + gslot(ib) * NP + r + 1] : 1.f;
+                    v[j] = rc[j] * ex2_fast(f32[F_A2 + r] * ds) * g0;
+                    v[j + 1] = rc[j + 1] * ex2_fast(f32[F_A2 + r + 1] * ds) * g1;
+                } else {
+                    const int m = nr + ((r - nr) >> 1);
+                    float sn, cs;
+                    __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                    const float ec = ex2_fast(f32[F_A2 + m] * ds);
+                    const float ci0 = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
+                    const float ci1 = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
+                    float gr = 1.f, gi = 0.f;
+                    if (ib) {
+                        gr = f32[F_KRE + gslot(ib) * NP + m];
+                        gi = f32[F_KIM + gslot(ib) * NP + m];
+                    }
+                    cmul(ci0, ci1, gr, gi, v[j], v[j + 1]);
+                }
+            }
+            st16_split(sm + loc::SM_CH, sm + loc::SM_CHL, off_kmaj(t, r0, KM_LBO, KM_SBO), v);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t dy_base = smem_u32(sm + loc::SM_DY);
+            const uint32_t id = idesc_bf16(128, 64, true, true);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t ch_base = smem_u32(sm + (part ? loc::SM_CHL : loc::SM_CH));
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(tacc, sdesc(ch_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id,
+                             part > 0 || s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            const int n = tid;
+            float *dst = p.ws_gc + (bhc(p, b, h, c) * N + n) * PD;
+#pragma unroll
+            for (int c16 = 0; c16 < PD / 16; ++c16) {
+                float v[16];
+                tmem_ld16(tmem_addr(tacc, 32u * warp, 16u * c16), v);
+                if (n < N) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        reinterpret_cast<float4 *>(dst + 16 * c16)[q4] =
+                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);  // let an in-flight load land before exit
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tacc, loc::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// k_chunk_adj_pass: reverse pass over the chunks of one (batch row, head).
+// Thread (row pair rp, column p) keeps rows 2rp, 2rp+1 of the adjoint carry:
+// two real modes, or one rotation pair as (re, im).  ws_gc[c] holds Ghat_c on
+// entry and the carry into chunk c on exit.
+// ============================================================================
+namespace pass {
+constexpr int THREADS = 512;
+constexpr int KMAX = NP / 16;   // row pairs per thread
+}  // namespace pass
+
+__global__ void __launch_bounds__(pass::THREADS, 2) k_chunk_adj_pass(Params p) {
+    // chunk decays, triple-buffered: chunk c-1's are fetched while chunk c is processed
+    __shared__ float s_ce[3][2 * NP];
+    __shared__ float red[pass::THREADS];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int N = p.N, nr = p.nr, nc = p.nc;
+    const int q = tid & 63, rp0 = tid >> 6, wp = q >> 5;
+    const int nk = N / 16;
+    float g0[pass::KMAX], g1[pass::KMAX];
+#pragma unroll
+    for (int k = 0; k < pass::KMAX; ++k) g0[k] = g1[k] = 0.f;
+    if (tid < 2 * NP) s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
+
+    for (int c = nc - 1; c >= 0; --c) {
+        float *gbase = p.ws_gc + bhc(p, b, h, c) * N * PD + q;
+        const float *kb = (c > 0 && p.ws_qb) ? p.ws_kb + bhc(p, b, h, c - 1) * N * PD + q : nullptr;
+        if (c > 0 && tid < 2 * NP)
+            s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
+        __syncthreads();
+        const float *ce = s_ce[c % 3];
+        float *qb = p.ws_qb ? p.ws_qb + (bhc(p, b, h, c) * 4 + wp) * (long long)N : nullptr;
+        // two halves of KMAX / 2 row pairs; each half issues all of its loads first
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            constexpr int KH = pass::KMAX / 2;
+            float hv0[KH], hv1[KH], kv0[KH], kv1[KH];
+#pragma unroll
+            for (int kk = 0; kk < KH; ++kk) {
+                const int k = hf * KH + kk;
+                hv0[kk] = hv1[kk] = kv0[kk] = kv1[kk] = 0.f;
+                if (k < nk) {
+                    const int n0 = 2 * (rp0 + 8 * k);
+                    hv0[kk] = gbase[(long long)n0 * PD];
+                    hv1[kk] = gbase[(long long)(n0 + 1) * PD];
+                    if (kb) {
+                        kv0[kk] = __ldg(kb + (long long)n0 * PD);
+                        kv1[kk] = __ldg(kb + (long long)(n0 + 1) * PD);
+                    }
+                }
+            }
+#pragma unroll
+            for (int kk = 0; kk < KH; ++kk) {
+                const int k = hf * KH + kk;
+                if (k >= nk) break;
+                const int n0 = 2 * (rp0 + 8 * k);
+                // the carry into chunk c, then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
+                gbase[(long long)n0 * PD] = g0[k];
+                gbase[(long long)(n0 + 1) * PD] = g1[k];
+                float a0, a1;
+                if (n0 < nr) {
+                    a0 = fmaf(ce[2 * n0], g0[k], hv0[kk]);
+                    a1 = fmaf(ce[2 * (n0 + 1)], g1[k], hv1[kk]);
+                } else {
+                    const int m = nr + ((n0 - nr) >> 1);
+                    const float er = ce[2 * m], ei = ce[2 * m + 1];
+                    a0 = fmaf(er, g0[k], fmaf(ei, g1[k], hv0[kk]));
+                    a1 = fmaf(er, g1[k], fmaf(-ei, g0[k], hv1[kk]));
+                }
+                g0[k] = a0;
+                g1[k] = a1;
+                if (kb) {
+                    // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}
+                    float q0, q1;
+                    if (n0 < nr) {
+                        q0 = a0 * kv0[kk];
+                        q1 = a1 * kv1[kk];
+                    } else {
+                        q0 = fmaf(a0, kv0[kk], a1 * kv1[kk]);
+                        q1 = fmaf(a0, kv1[kk], -a1 * kv0[kk]);
+                    }
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) {
+                        q0 += __shfl_xor_sync(0xffffffffu, q0, o);
+                        q1 += __shfl_xor_sync(0xffffffffu, q1, o);
+                    }
+                    if (lane == 0) {
+                        qb[n0] = q0;
+                        qb[n0 + 1] = q1;
+                    }
+                }
+            }
+        }
+    }
+    // carry out of the first chunk = dL/dK_{-1}: dh0, dw0 = beta_0 dh0, dbeta_0 = <dh0, w0>
+    float beta0 = 0.f;
+    if (p.two_ep)
+        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+    float db0 = 0.f;
+#pragma unroll
+    for (int k = 0; k < pass::KMAX; ++k) {
+        if (k >= nk) break;
+        const int n0 = 2 * (rp0 + 8 * k);
+        const long long i0 = ix_st(p, b, h, n0, q), i1 = ix_st(p, b, h, n0 + 1, q);
+        if (p.dh0) {
+            p.dh0[i0] = g0[k];
+            p.dh0[i1] = g1[k];
+        }
+        if (p.dw0) {
+            p.dw0[i0] = beta0 * g0[k];
+            p.dw0[i1] = beta0 * g1[k];
+        }
+        if (p.w0) db0 = fmaf(g0[k], p.w0[i0], fmaf(g1[k], p.w0[i1], db0));
+    }
+    red[tid] = db0;
+    __syncthreads();
+    if (tid == 0) {
+        float acc = 0.f;
+        for (int k = 0; k < pass::THREADS; ++k) acc += red[k];
+        p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1] = acc;
+    }
+}
+
+// ============================================================================
+// k_chunk_bwd_dx: per chunk,
+//   DX = P^T (64 s x 64 t) . dY (64 t x 64 p)  +  Bh (64 s x N) . Gc (N x 64 p)
+//   dx_s = DX_s + (D - beta_{s+1} (C_s . B_s)) dy_s
+// with the scores built exactly as in the forward: scores^T_i = Bi . Ci^T.
+// ============================================================================
+namespace dxk {
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint32_t SM_B = 0;          // 16 KB raw B (swizzled halves)
+constexpr uint32_t SM_C = 16384;      // 16 KB raw C
+constexpr uint32_t SM_DY = 32768;     // 8 KB  dy (swizzled)
+constexpr uint32_t SM_CI = 40960;     // 16 KB Ci K-major (rows t, K = state rows)
+constexpr uint32_t SM_BI = 57344;     // 40 KB Bi tiles (16, 32, 48, 64 rows)
+constexpr uint32_t SM_BH = 98304;     // 16 KB Bh (stored MN-major with M = rows; read K-major, M = s)
+constexpr uint32_t SM_P = 114688;     // 8 KB  P^T, K-major (rows s, K = t)
+constexpr uint32_t SM_GC = 122880;    // 16 KB Gc bf16, MN-major B operand (N = p, K = state rows)
+constexpr uint32_t SM_F32 = 139264;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace dxk
+
+__global__ void __launch_bounds__(dxk::THREADS, 1)
+k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+               const __grid_constant__ CUtensorMap tmDY, Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + dxk::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dxk::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;   // [2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, L = p.L;
+    const int t0 = c * Q;
+    const int nbox = N / 64;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmDY);
+        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + 2 * Q * N * 2));
+        tma_load_4d(sm + dxk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_4d(sm + dxk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+            tma_load_4d(sm + dxk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
+        }
+    }
+    if (warp == 0) tmem_alloc(tslot, dxk::TMEM_COLS);
+    mode_rates(p, f32, h);
+    if (N < NP)  // K padding of Ci, Bi, Bh
+        for (int i = tid; i < (int)((dxk::SM_P - dxk::SM_CI) / 16); i += dxk::THREADS)
+            reinterpret_cast<uint4 *>(sm + dxk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    // Gc (fp32, [n][p]) -> bf16 B operand; rows past N are zero
+    {
+        const float *gsrc = p.ws_gc + bhc(p, b, h, c) * N * PD;
+        for (int it = tid; it < NP * (PD / 8); it += dxk::THREADS) {
+            const int n = it >> 3, p8 = (it & 7) * 8;
+            float v[8];
+            if (n < N) {
+                const float4 a = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8);
+                const float4 d = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8 + 4);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            }
+            st16(sm + dxk::SM_GC, off_mnmaj(p8, n, 1024u, 128u), v);
+        }
+    }
+    chunk_tokens(p, f32, b, h, t0, true);
+    chunk_mode_constants(p, f32);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_dx = tbase;                  // DX (M=64: lanes 0-15 of each quarter), cols 0..63
+    const uint32_t t_sc = tbase + (16u << 16);    // scores^T (M=64: lanes 16-31), cols 0..63
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) rev_raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // ---- operands: Ci, Bi (own block and later blocks), Bh; C.B partials
+        {
+            const int t = tid & 63, grp = tid >> 6;
+            const int ib = t >> 4;
+            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+            const float ds = f32[F_S + t] - Sb;
+            const float sig = f32[F_SIG + t];
+            const unsigned char *sB = sm + dxk::SM_B, *sC = sm + dxk::SM_C;
+            float corr = 0.f;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const int r0 = 8 * (grp + 4 * k);
+                if (r0 >= N) break;
+                float vCI[8], vBI[8], vBH[8], vBX[3][8], rc[8], rb[8];
+                ld_rows8(sC, t, r0, rc);
+                ld_rows8(sB, t, r0, rb);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int r = r0 + j;
+                    const float c0 = rc[j], c1 = rc[j + 1];
+                    const float b0 = rb[j], b1 = rb[j + 1];
+                    corr = fmaf(c0, b0, fmaf(c1, b1, corr));
+                    if (r < nr) {
+                        const int m0 = r, m1 = r + 1;
+                        const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
+                        vCI[j] = c0 * ex2_fast(x0);
+                        vCI[j + 1] = c1 * ex2_fast(x1);
+                        const float bi0 = sig * b0 * ex2_fast(fminf(-x0, 120.f));
+                        const float bi1 = sig * b1 * ex2_fast(fminf(-x1, 120.f));
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
+                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
+                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
+#pragma unroll
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
+                            if (i2 < 4) {
+                                vBX[qq][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
+                                vBX[qq][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                            }
+                        }
+                    } else {
+                        const int m = nr + ((r - nr) >> 1);
+                        const float x = f32[F_A2 + m] * ds;
+                        float sn, cs;
+                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
+                        vCI[j] = ec * fmaf(c0, cs, c1 * sn);
+                        vCI[j + 1] = ec * fmaf(c1, cs, -c0 * sn);
+                        const float bi0 = eb * fmaf(b0, cs, b1 * sn);
+                        const float bi1 = eb * fmaf(b1, cs, -b0 * sn);
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
+                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m],
+                             f32[F_KIM + fslot(ib, 4) * NP + m], vBH[j], vBH[j + 1]);
+#pragma unroll
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
+                            if (i2 < 4)
+                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m],
+                                     f32[F_KIM + fslot(ib, i2) * NP + m], vBX[qq][j],
+                                     vBX[qq][j + 1]);
+                        }
+                    }
+                }
+                st16(sm + dxk::SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
+                st16(sm + dxk::SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+#pragma unroll
+                for (int qq = 0; qq < 3; ++qq) {
+                    const int i2 = ib + 1 + qq;
+                    if (i2 < 4)
+                        st16(sm + dxk::SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
+                }
+                st16(sm + dxk::SM_BH, off_mnmaj(r0, t, 2048u, 128u), vBH);
+            }
+            f32[F_CP + grp * 64 + t] = corr;
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // ---- phase A: scores^T_i = Bi . Ci^T ; DX = Bh . Gc
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t bi_base = smem_u32(sm + dxk::SM_BI), ci_base = smem_u32(sm + dxk::SM_CI);
+            const uint32_t id_sc = idesc_bf16(64, 16, false, false);
+            for (int i = 0; i < NSB; ++i)
+                for (int s = 0; s < NP / 16; ++s)
+                    mma_bf16(t_sc + 16 * i,
+                             sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
+                             sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
+                             id_sc, s > 0);
+            const uint32_t bh_base = smem_u32(sm + dxk::SM_BH), gc_base = smem_u32(sm + dxk::SM_GC);
+            const uint32_t id_dx = idesc_bf16(64, 64, false, true);
+            for (int s = 0; s < NP / 16; ++s)
+                mma_bf16(t_dx, sdesc(bh_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                         sdesc(gc_base + s * 2048u, 1024u, 128u, LAYOUT_NONE), id_dx, s > 0);
+            mma_commit(&bar_mma[0]);
+        }
+        if (tid < 64) {
+            float cs = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cs += f32[F_CP + k * 64 + tid];
+            f32[F_CORR + tid] = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
+        }
+        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            // ---- masked scores -> P^T (K-major rows s, K = t), zero where s > t
+            if (warp >= 4) {
+                const int qd = warp - 4;
+                for (int i = 0; i < NSB; ++i) {
+                    float v[16];
+                    tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
+                    const int sl = lane - 16;
+                    if (sl >= 0) {
+                        const int s = 16 * qd + sl;
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
+                            hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
+                        }
+                        st16(sm + dxk::SM_P, off_kmaj(s, 16 * i, 128u, 1024u), lo);
+                        st16(sm + dxk::SM_P, off_kmaj(s, 16 * i + 8, 128u, 1024u), hi);
+                    }
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            // ---- phase B: DX += P^T dY
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t p_base = smem_u32(sm + dxk::SM_P), dy_base = smem_u32(sm + dxk::SM_DY);
+                const uint32_t id_d = idesc_bf16(64, 64, false, true);
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(t_dx, sdesc(p_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_d, true);
+                mma_commit(&bar_mma[1]);
+            }
+            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
+            if (!ok) rev_raise_error(1);
+            fence_after_sync();
+            if (__syncthreads_and(ok)) {
+                // ---- epilogue: dx_s = DX_s + corr_s dy_s
+                const int qd = warp & 3, half = warp >> 2;
+                const int s = 16 * qd + (lane & 15);
+                const unsigned char *sDY = sm + dxk::SM_DY;
+                __nv_bfloat16 *xrow = reinterpret_cast<__nv_bfloat16 *>(p.dx) + b * p.sx[0] +
+                                      (long long)(t0 + s) * p.sx[1] + h * p.sx[2];
+                const float cr = f32[F_CORR + s];
+                for (int c16 = 0; c16 < 2; ++c16) {
+                    float v[16];
+                    const int pc = 32 * half + 16 * c16;
+                    tmem_ld16(tmem_addr(t_dx, 32u * qd, (uint32_t)pc), v);
+                    if (lane < 16 && t0 + s < L) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float o[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                o[j] = fmaf(cr, bf(sDY + off_sw128(s, pc + 8 * hh + j)), v[8 * hh + j]);
+                            uint4 w;
+                            w.x = pack_bf16(o[0], o[1]);
+                            w.y = pack_bf16(o[2], o[3]);
+                            w.z = pack_bf16(o[4], o[5]);
+                            w.w = pack_bf16(o[6], o[7]);
+                            *reinterpret_cast<uint4 *>(xrow + pc + 8 * hh) = w;
+                        }
+                    }
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, dxk::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// k_chunk_bwd_gbu: per chunk, gbu_t = sum_p u_t,p Gbar_t,p (per state row),
+// with sub-block-END references Se_j (the mirror of the forward's folding):
+//   Gbar_t u_t = conj(e^{lam (Se_j - S_t)}) [ conj(F[j+1][4]) (Gc u_t)
+//                                            + sum_{t' >= t} (u_t . dy_t') Cm^{[j]}_t' ]
+//   Cm^{[j]}_t' = conj(e^{lam (S_t' - Se_j)}) c_t'      for t' >= 16 j  (t in sub-block j)
+// On the tensor cores (all operands split into bf16 hi + lo):
+//   G' = X (64 t x 64 p) . dY^T (64 p x 64 t')                M=64,  N=64, K=64
+//   V2 = Gc (N x 64 p) . X^T (64 p x 64 t)                    M=128, N=64, K=64
+//   E_j = Cm^{[j]} (N x t') . (G' o mask)_j^T (t' x 16 t)      M=128, N=16, K=64-16j
+// Also writes <dy_t, u_t>, dsigma_t = B_t . gbu_t and (C_t . B_t) <dy_t, u_t>.
+// ============================================================================
+namespace gbk {
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t SM_X = 0;           // 8 KB  x (swizzled)
+constexpr uint32_t SM_DY = 8192;       // 8 KB  dy (swizzled)
+constexpr uint32_t SM_B = 16384;       // 16 KB raw B
+constexpr uint32_t SM_C = 32768;       // 16 KB raw C
+constexpr uint32_t SM_CM = 49152;      // 40 KB Cm^{[j]} hi, MN-major (M = rows, K = t' - 16 j)
+constexpr uint32_t SM_CML = 90112;     // 40 KB Cm lo
+constexpr uint32_t SM_GM = 131072;     // 8 KB  masked G' hi: 4 tiles, K-major (rows t, K = t')
+constexpr uint32_t SM_GML = 139264;    // 8 KB  masked G' lo
+constexpr uint32_t SM_GC = 147456;     // 16 KB Gc hi, K-major (rows = state rows, K = p)
+constexpr uint32_t SM_GCL = 163840;    // 16 KB Gc lo
+constexpr uint32_t SM_F32 = 180224;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+constexpr int RED_LD = 65;             // row stride of the dsigma reduction (floats)
+}  // namespace gbk
+
+// byte offset of mirror tile j (64 - 16 j rows of 256 bytes)
+__device__ __forceinline__ uint32_t cm_off(int j) {
+    return j == 0 ? 0u : (j == 1 ? 16384u : (j == 2 ? 28672u : 36864u));
+}
+
+__global__ void __launch_bounds__(gbk::THREADS, 1)
+k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + gbk::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + gbk::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;   // [2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, L = p.L;
+    const int t0 = c * Q;
+    const int nbox = N / 64;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+        tma_prefetch_desc(&tmDY);
+        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + 2 * Q * N * 2));
+        tma_load_4d(sm + gbk::SM_X, &tmX, bar_tma, 0, h, t0, b);
+        tma_load_4d(sm + gbk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_4d(sm + gbk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+            tma_load_4d(sm + gbk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
+        }
+    }
+    if (warp == 0) tmem_alloc(tslot, gbk::TMEM_COLS);
+    mode_rates(p, f32, h);
+    if (N < NP)  // M padding of the mirror tiles
+        for (int i = tid; i < (int)((gbk::SM_GM - gbk::SM_CM) / 16); i += gbk::THREADS)
+            reinterpret_cast<uint4 *>(sm + gbk::SM_CM)[i] = make_uint4(0, 0, 0, 0);
+    // Gc (fp32 [n][p]) -> bf16 hi / lo, K-major (rows n, K = p); rows past N are zero
+    {
+        const float *gsrc = p.ws_gc + bhc(p, b, h, c) * N * PD;
+        for (int it = tid; it < NP * (PD / 8); it += gbk::THREADS) {
+            const int n = it >> 3, p8 = (it & 7) * 8;
+            float v[8];
+            if (n < N) {
+                const float4 a = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8);
+                const float4 d = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8 + 4);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            }
+            st16_split(sm + gbk::SM_GC, sm + gbk::SM_GCL, off_kmaj(n, p8, 128u, 1024u), v);
+        }
+    }
+    chunk_tokens(p, f32, b, h, t0, true);
+    chunk_mode_constants(p, f32);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_v2 = tbase;          // V2 (M=128), cols 0..63
+    const uint32_t t_g = tbase + 64u;     // G' (M=64: lanes 0-15 per quarter), then E_j (M=128)
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) rev_raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // ---- mirror tiles: own sub-block value, copies into earlier sub-blocks' tiles
+        {
+            const int t = tid & 63, grp = tid >> 6;
+            const int kb = t >> 4;
+            const float ds = f32[F_S + t] - f32[F_S + 16 * kb + 15];   // <= 0
+            const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
+            float corr = 0.f;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const int r0 = 8 * (grp + 4 * k);
+                if (r0 >= N) break;
+                float rc[8], rb[8], v[8], vx[3][8];
+                ld_rows8(sC, t, r0, rc);
+                ld_rows8(sB, t, r0, rb);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int r = r0 + j;
+                    corr = fmaf(rc[j], rb[j], fmaf(rc[j + 1], rb[j + 1], corr));
+                    if (r < nr) {
+                        v[j] = rc[j] * ex2_fast(fminf(f32[F_A2 + r] * ds, 120.f));
+                        v[j + 1] = rc[j + 1] * ex2_fast(fminf(f32[F_A2 + r + 1] * ds, 120.f));
+#pragma unroll
+                        for (int jj = 0; jj < 3; ++jj) {
+                            if (jj < kb) {
+                                const int sl = fslot(jj + 1, kb + 1);
+                                vx[jj][j] = v[j] * f32[F_KRE + sl * NP + r];
+                                vx[jj][j + 1] = v[j + 1] * f32[F_KRE + sl * NP + r + 1];
+                            }
+                        }
+                    } else {
+                        const int m = nr + ((r - nr) >> 1);
+                        float sn, cs;
+                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        const float ec = ex2_fast(fminf(f32[F_A2 + m] * ds, 120.f));
+                        v[j] = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
+                        v[j + 1] = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
+#pragma unroll
+                        for (int jj = 0; jj < 3; ++jj) {
+                            if (jj < kb) {
+                                const int sl = fslot(jj + 1, kb + 1);
+                                cmul(v[j], v[j + 1], f32[F_KRE + sl * NP + m],
+                                     -f32[F_KIM + sl * NP + m], vx[jj][j], vx[jj][j + 1]);
+                            }
+                        }
+                    }
+                }
+                st16_split(sm + gbk::SM_CM + cm_off(kb), sm + gbk::SM_CML + cm_off(kb),
+                           off_mnmaj(r0, t - 16 * kb, 2048u, 128u), v);
+#pragma unroll
+                for (int jj = 0; jj < 3; ++jj)
+                    if (jj < kb)
+                        st16_split(sm + gbk::SM_CM + cm_off(jj), sm + gbk::SM_CML + cm_off(jj),
+                                   off_mnmaj(r0, t - 16 * jj, 2048u, 128u), vx[jj]);
+            }
+            f32[F_CP + grp * 64 + t] = corr;
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // this thread's rows of the per-head dC (forward-direction part), in flight during the MMAs
+        float kd[32];
+        {
+            const int n = tid & 127, half = tid >> 7;
+#pragma unroll
+            for (int i2 = 0; i2 < 32; ++i2) {
+                const int t = t0 + 32 * half + i2;
+                kd[i2] = (n < N && t < L) ? __ldg(p.ws_dC + ix_wsk(p, b, t, h, 0, 1, n)) : 0.f;
+            }
+        }
+        // ---- phase A: G' = X dY^T ; V2 = Gc X^T (hi + lo)
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sm + gbk::SM_X), dy_base = smem_u32(sm + gbk::SM_DY);
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int s = 0; s < PD / 16; ++s)
+                mma_bf16(t_g, sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
+            const uint32_t id_v = idesc_bf16(128, 64, false, false);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t gc_base = smem_u32(sm + (part ? gbk::SM_GCL : gbk::SM_GC));
+                for (int s = 0; s < PD / 16; ++s)
+                    mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
+            }
+            mma_commit(&bar_mma[0]);
+        }
+        if (tid < 64) {
+            float cs = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cs += f32[F_CP + k * 64 + tid];
+            f32[F_CORR + tid] = cs;   // C_t . B_t
+        }
+        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            // ---- masked G' rows -> K-major tiles (rows t of sub-block qd, K = t' >= t)
+            if (warp >= 4) {
+                const int qd = warp - 4;
+                for (int i = 0; i < NSB; ++i) {
+                    float v[16];
+                    tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
+                    if (lane < 16 && i >= qd) {
+                        const int t = 16 * qd + lane;
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = (16 * i + j >= t) ? v[j] : 0.f;
+                            hi[j] = (16 * i + 8 + j >= t) ? v[8 + j] : 0.f;
+                        }
+                        unsigned char *gt = sm + gbk::SM_GM + qd * 2048;
+                        unsigned char *gl = sm + gbk::SM_GML + qd * 2048;
+                        st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
+                        st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
+                        if (i == qd) {
+                            float dg = 0.f;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (j == lane) dg = v[j];
+                            f32[F_LAM + t] = dg;   // <dy_t, u_t> (lambda is no longer needed)
+                        }
+                    }
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            // ---- phase B: E_j = Cm^{[j]} (G' o mask)_j^T, hi*hi + hi*lo + lo*hi
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t id_e = idesc_bf16(128, 16, true, false);
+                const uint32_t a_off[3] = {gbk::SM_CM, gbk::SM_CM, gbk::SM_CML};
+                const uint32_t b_off[3] = {gbk::SM_GM, gbk::SM_GML, gbk::SM_GM};
+                for (int j = 0; j < NSB; ++j)
+                    for (int part = 0; part < 3; ++part) {
+                        const uint32_t cm_base = smem_u32(sm + a_off[part]) + cm_off(j);
+                        const uint32_t gm_base = smem_u32(sm + b_off[part]) + j * 2048u;
+                        for (int s = 0; s < NSB - j; ++s)
+                            mma_bf16(t_g + 16 * j, sdesc(cm_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                                     sdesc(gm_base + (j + s) * 256u, 128u, 1024u, LAYOUT_NONE), id_e,
+                                     part > 0 || s > 0);
+                    }
+                mma_commit(&bar_mma[1]);
+            }
+            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
+            if (!ok) rev_raise_error(1);
+            fence_after_sync();
+            if (__syncthreads_and(ok)) {
+                // ---- unfold: gbu_t = conj(e^{lam (Se_j - S_t)}) (conj(F[j+1][4]) V2_t + E_t),
+                // then, per state mode, the within-chunk suffix sums of the decay-gradient
+                // identity (X_t - Y_t, X = conj(c) dCK, Y = b conj(sigma gbu)), walking the
+                // tokens backwards; and dB / dC directly when a group has one head.
+                float *red = reinterpret_cast<float *>(sm + gbk::SM_CM);     // [128][RED_LD] B . gbu
+                float *red2 = reinterpret_cast<float *>(sm + gbk::SM_CML);   // [128][RED_LD] ddt terms
+                float *xch = reinterpret_cast<float *>(sm + gbk::SM_GM);     // [2][128] upper-half totals
+                const int n = tid & 127, half = tid >> 7, qd = warp & 3;
+                const bool valid = n < N;
+                const int m = n < nr ? n : nr + ((n - nr) >> 1);
+                const bool pr_row = valid && n >= nr;
+                const bool im_row = pr_row && ((n - nr) & 1);
+                const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
+                // d ddt / d(suffix sum): a for the real part, -theta for the imaginary part
+                const float coef = !valid ? 0.f : (im_row ? -w : a2 * 0.6931471805599453f);
+                const bool one_head = p.hpg == 1;
+                const long long tstride = (long long)p.H * p.N;
+                float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+                const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
+                float cum = 0.f, dacc = 0.f, sdt = 0.f;
+#pragma unroll
+                for (int c16 = 1; c16 >= 0; --c16) {
+                    const int tc = 32 * half + 16 * c16;
+                    float vv[16], ee[16];
+                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)tc), vv);
+                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), ee);
+#pragma unroll
+                    for (int j = 15; j >= 0; --j) {
+                        const int t = tc + j;
+                        const int jb = t >> 4;
+                        const float ds = f32[F_S + 16 * jb + 15] - f32[F_S + t];   // >= 0
+                        const float mag = ex2_fast(a2 * ds);
+                        float er = mag, ei = 0.f;
+                        if (pr_row) {
+                            float sn, cs;
+                            __sincosf(w * ds, &sn, &cs);
+                            er = mag * cs;
+                            ei = mag * sn;
+                        }
+                        float fr = 1.f, fi = 0.f;
+                        if (jb < 3 && valid) {
+                            fr = f32[F_KRE + fslot(jb + 1, 4) * NP + m];
+                            fi = f32[F_KIM + fslot(jb + 1, 4) * NP + m];
+                        }
+                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                        const float eo = __shfl_xor_sync(0xffffffffu, ee[j], 1);
+                        float res;
+                        if (!pr_row) {
+                            res = er * fmaf(fr, vv[j], ee[j]);
+                        } else {
+                            // own row is re (im_row false) or im; W = conj(F) V + E
+                            const float vr = im_row ? vo : vv[j], vi = im_row ? vv[j] : vo;
+                            const float e_r = im_row ? eo : ee[j], e_i = im_row ? ee[j] : eo;
+                            const float wr = fmaf(fr, vr, fmaf(fi, vi, e_r));
+                            const float wi = fmaf(fr, vi, fmaf(-fi, vr, e_i));
+                            // conj(er + i ei) (wr + i wi)
+                            res = im_row ? fmaf(er, wi, -ei * wr) : fmaf(er, wr, ei * wi);
+                        }
+                        const bool tv = valid && t0 + t < L;
+                        const float m2 = f32[F_LAM + t], bn = f32[F_BN + t];
+                        const float sig = f32[F_SIG + t], dtv = f32[F_DT + t];
+                        const float bt = ld_row1(sB, t, n), ct = ld_row1(sC, t, n);
+                        const float kk = fmaf(bn * m2, bt, kd[16 * c16 + j]);   // dCK = dC + beta' <dy,u> b
+                        const float gg = sig * res;
+                        const float co = __shfl_xor_sync(0xffffffffu, ct, 1);
+                        const float ko = __shfl_xor_sync(0xffffffffu, kk, 1);
+                        const float bo = __shfl_xor_sync(0xffffffffu, bt, 1);
+                        const float go = __shfl_xor_sync(0xffffffffu, gg, 1);
+                        float v;
+                        if (!pr_row)
+                            v = fmaf(ct, kk, -bt * gg);
+                        else if (!im_row)   // Re(conj(c) k) - Re(b conj(g))
+                            v = fmaf(ct, kk, fmaf(co, ko, -fmaf(bt, gg, bo * go)));
+                        else                // Im(conj(c) k) - Im(b conj(g)), own row = im
+                            v = fmaf(co, kk, fmaf(-ct, ko, -fmaf(bt, go, -bo * gg)));
+                        if (!tv) v = 0.f;
+                        cum += v;
+                        dacc = fmaf(dtv, im_row ? -cum : cum, dacc);
+                        sdt += dtv;
+                        red2[n * gbk::RED_LD + t] = coef * cum;
+                        red[n * gbk::RED_LD + t] = tv ? res * bt : 0.f;
+                        if (tv) {
+                            if (one_head) {
+                                const int tg = t0 + t;
+                                reinterpret_cast<__nv_bfloat16 *>(p.dBm)[ix_B(p, b, tg, g, 0, n)] =
+                                    __float2bfloat16_rn(fmaf(-bn * ct, m2, gg));
+                                reinterpret_cast<__nv_bfloat16 *>(p.dCm)[ix_C(p, b, tg, g, 0, n)] =
+                                    __float2bfloat16_rn(kd[16 * c16 + j]);
+                            } else {
+                                gdst[(long long)t * tstride] = res;
+                            }
+                        }
+                    }
+                }
+                // the upper half's totals carry into every token of the lower half
+                if (half == 1) {
+                    xch[n] = cum;
+                    xch[128 + n] = dacc;
+                }
+                __syncthreads();
+                if (half == 0) {
+                    const float tot1 = xch[n];
+                    const float add = coef * tot1;
+                    for (int t = 0; t < 32; ++t) red2[n * gbk::RED_LD + t] += add;
+                    dacc += (im_row ? -tot1 : tot1) * sdt + xch[128 + n];
+                    if (valid) {
+                        const int nmode = p.nr + p.np;
+                        float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
+                        const float tot = cum + tot1;
+                        if (!pr_row) {
+                            blk[4 * m + 0] = tot;
+                            blk[4 * m + 1] = 0.f;
+                            blk[4 * m + 2] = dacc;
+                            blk[4 * m + 3] = 0.f;
+                        } else if (!im_row) {
+                            blk[4 * m + 0] = tot;
+                            blk[4 * m + 2] = dacc;
+                        } else {
+                            blk[4 * m + 1] = tot;
+                            blk[4 * m + 3] = dacc;
+                        }
+                    }
+                }
+                __syncthreads();
+                if (tid < 64 && t0 + tid < L) {
+                    const int t = tid;
+                    float dsig = 0.f, dd = 0.f;
+                    for (int k = 0; k < N; ++k) {
+                        dsig += red[k * gbk::RED_LD + t];
+                        dd += red2[k * gbk::RED_LD + t];
+                    }
+                    const long long i = ix_bth(p, b, t0 + t, h);
+                    const float m2 = f32[F_LAM + t];
+                    p.ws_tok[2 * i] = dsig;
+                    p.ws_tok[2 * i + 1] = f32[F_CORR + t] * m2;
+                    p.ws_M2[i] = m2;
+                    p.ws_ddt[i] = dd;
+                }
+                if (tid == 64) {
+                    const int nmode = p.nr + p.np;
+                    float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
+                    float st_ = 0.f, dD = 0.f;
+                    for (int t = 0; t < Q; ++t) {
+                        st_ += f32[F_DT + t];
+                        if (t0 + t < L) dD += f32[F_LAM + t];
+                    }
+                    blk[4 * nmode + 0] = st_;
+                    blk[4 * nmode + 1] = (p.O == p.R) ? dD : 0.f;
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, gbk::TMEM_COLS);
+    }
+}
+
+}  // namespace chunkrev
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <typename K>
+static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
+    if (done) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
+// Reverse part of the tensor-core backward: dx, gbu / dsigma / <dy, u>, the
+// exact chunk-boundary values, dh0 / dw0 / dbeta_0.  Needs p.ws_gc, p.ws_ce,
+// p.ws_kb (written by the forward-direction part), p.ws_qb.
+cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
+    using namespace chunkrev;
+    CUtensorMap mx, mb, mc, mdy;
+    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
+        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
+        !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true) ||
+        !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
+        return cudaErrorInvalidValue;
+    static bool a1 = false, a3 = false, a4 = false;
+    cudaError_t e;
+    if ((e = set_smem(k_chunk_adj_local, loc::SMEM_BYTES, a1)) != cudaSuccess) return e;
+    if ((e = set_smem(k_chunk_bwd_dx, dxk::SMEM_BYTES, a3)) != cudaSuccess) return e;
+    if ((e = set_smem(k_chunk_bwd_gbu, gbk::SMEM_BYTES, a4)) != cudaSuccess) return e;
+    const dim3 grid(p.nc, p.H, p.Bsz);
+    k_chunk_adj_local<<<grid, loc::THREADS, loc::SMEM_BYTES, st>>>(mc, mdy, p);
+    profile_mark(st, "k_chunk_adj_local");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_chunk_adj_pass<<<dim3(p.H, p.Bsz), pass::THREADS, 0, st>>>(p);
+    profile_mark(st, "k_chunk_adj_pass");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
+    profile_mark(st, "k_chunk_bwd_dx");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_chunk_bwd_gbu<<<grid, gbk::THREADS, gbk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
+    profile_mark(st, "k_chunk_bwd_gbu");
+    return cudaGetLastError();
+}
+
+// Read and clear the device error word of these kernels.
+int chunk_rev_error_take() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, ssm_chunk_rev_error_word, sizeof(int)) != cudaSuccess) return -1;
+    if (v) cudaMemcpyToSymbol(ssm_chunk_rev_error_word, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace ssm

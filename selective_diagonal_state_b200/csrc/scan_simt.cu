@@ -1163,8 +1163,10 @@ cudaError_t simt_forward(const Params &p, cudaStream_t st) {
 
 bool chunk_bwd_supported(const Params &p);
 cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st);
+cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st);
 
-// use_chunk: per-head dC from the tensor-core kernel instead of sweep 1
+// use_chunk: the tensor-core kernels replace both sweeps (forward-direction dC,
+// then the chunk-parallel reverse part); the finalize kernels are shared.
 cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk) {
     cudaError_t e;
     if (use_chunk)
@@ -1172,13 +1174,22 @@ cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk) {
     else
         e = launch_scan(KK_S1, p, st);
     if (e != cudaSuccess) return e;
-    if ((e = launch_scan(KK_S2, p, st)) != cudaSuccess) return e;
+    // the chunk-parallel reverse part also produces the per-block decay sums
+    // (and dB / dC when every group has one head)
+    const bool rev = use_chunk && p.ws_gc;
+    if (rev)
+        e = chunk_bwd_reverse(p, st);
+    else
+        e = launch_scan(KK_S2, p, st);
+    if (e != cudaSuccess) return e;
     {
         int nthr = ((p.nr + p.np + 31) / 32) * 32;
         if (nthr < 32) nthr = 32;
-        k_bwd_units_local<<<dim3(ntb_of(p), p.H, p.Bsz), nthr, (size_t)FT * nthr * 4, st>>>(p);
-        profile_mark(st, "k_bwd_units_local");
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (!rev) {
+            k_bwd_units_local<<<dim3(ntb_of(p), p.H, p.Bsz), nthr, (size_t)FT * nthr * 4, st>>>(p);
+            profile_mark(st, "k_bwd_units_local");
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
         k_bwd_units_carry<<<dim3(p.H, p.Bsz), nthr, (size_t)nthr * 4, st>>>(p);
         profile_mark(st, "k_bwd_units_carry");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1189,9 +1200,11 @@ cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk) {
         profile_mark(st, "k_bwd_units_final");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    k_bwd_groups<<<dim3(p.L, p.Bsz), 256, (size_t)2 * p.H * 4, st>>>(p);
-    profile_mark(st, "k_bwd_groups");
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!(rev && p.hpg == 1)) {
+        k_bwd_groups<<<dim3(p.L, p.Bsz), 256, (size_t)2 * p.H * 4, st>>>(p);
+        profile_mark(st, "k_bwd_groups");
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     k_bwd_params<<<4, 256, 0, st>>>(p);
     profile_mark(st, "k_bwd_params");
     return cudaGetLastError();
