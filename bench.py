@@ -118,7 +118,7 @@ def kernel_bytes(shape, name: str) -> int:
 
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)
-LAUNCHES_PER_STEP = 16
+LAUNCHES_PER_STEP = 32
 
 
 # ---------------------------------------------------------------------------
@@ -315,6 +315,8 @@ def main():
         step()
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
+    route = {abi.ROUTE_CHUNKED: "tensor-core chain", abi.ROUTE_RANGE_FALLBACK:
+             "recurrent (range fallback)", abi.ROUTE_RECURRENT: "recurrent"}[abi.ssm_scan_last_route()]
 
     # per-kernel events over the timed region (library-owned, on our stream)
     launches_per_step = LAUNCHES_PER_STEP
@@ -433,7 +435,7 @@ def main():
                    "state": f"{shape.n_real} real + {shape.n_pairs} rotation pairs",
                    "two_endpoint": bool(shape.two_endpoint), "io": "bf16, fp32 state",
                    "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": "inputs (1.6 GB) larger than L2; no flush"},
+                   "l2": "inputs (1.6 GB) larger than L2; no flush", "route": route},
         "fwd_tokens_per_s": fwd_value, "ms_fwd": ms_fwd,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "kernel": dom,

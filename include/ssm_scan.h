@@ -91,7 +91,14 @@ typedef struct ssm_desc {
     int32_t chunk;              /* kernel choice, results equal up to rounding: 0 = library choice,
                                    1 = token-by-token recurrent kernels, 64 = 64-token chunked
                                    tensor-core kernels where supported (bf16, headdim 64,
-                                   rank 1, 64 or 128 state rows) */
+                                   rank 1, 64 or 128 state rows).  The chunked kernels fold
+                                   each mode's decay into the operands around 16-token
+                                   sub-block references, which needs
+                                   |A| * log2(e) * (sum of dt over any 16 aligned tokens)
+                                   <= 100 for the largest |A| of the head; the call checks
+                                   this on the device and, where it fails, the recurrent
+                                   kernels (launched behind the same device-side check)
+                                   produce the result instead */
     int32_t decay_mode;         /* enum ssm_decay_mode */
     int32_t two_endpoint;       /* 0: lambda not read (lam = 1); 1: lambda used */
     int32_t dtype_io;           /* enum ssm_dtype of x, dt, B, C, lambda, y and of their gradients */
@@ -202,6 +209,20 @@ SSM_API int ssm_scan_profile_stop(char *names, int name_len, int *counts, double
 
 /* SSM_SCAN_ABI_VERSION of the loaded library. */
 SSM_API int ssm_scan_abi_version(void);
+
+/*
+ * Which kernels produced the result of the last ssm_scan_fwd / ssm_scan_bwd
+ * call made on the calling host thread: synchronises `stream` (the stream of
+ * that call) and returns SSM_ROUTE_CHUNKED (tensor-core chain),
+ * SSM_ROUTE_RANGE_FALLBACK (chunk-eligible call whose inputs failed the
+ * device-side range check, taken by the recurrent kernels),
+ * SSM_ROUTE_RECURRENT (recurrent kernels chosen on the host: chunk = 1 or a
+ * shape the chunked kernels do not take), or a negative status (no call yet,
+ * or the gate word cannot be read).  A diagnostic for tests and tuning; the
+ * pages have no counterpart.
+ */
+enum ssm_route { SSM_ROUTE_CHUNKED = 0, SSM_ROUTE_RANGE_FALLBACK = 1, SSM_ROUTE_RECURRENT = 2 };
+SSM_API int ssm_scan_last_route(void *stream);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,8 @@ PASS_FWD, PASS_BWD = 0, 1
 EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
-            "ssm_scan_bwd_noalloc"]
+            "ssm_scan_bwd_noalloc", "ssm_scan_last_route"]
+ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_double), ctypes.c_int]
     lib.ssm_scan_profile_stop.restype = ctypes.c_int
+    lib.ssm_scan_last_route.argtypes = [_vp]
+    lib.ssm_scan_last_route.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -169,6 +172,14 @@ def ssm_scan_poll_device_error(stream=None) -> None:
 
 def ssm_scan_abi_version() -> int:
     return int(load_library().ssm_scan_abi_version())
+
+
+def ssm_scan_last_route(stream=None) -> int:
+    """Route of the last scan call on this thread (ROUTE_*); synchronises the stream."""
+    rc = int(load_library().ssm_scan_last_route(_stream(stream)))
+    if rc < 0:
+        _check(rc, "ssm_scan_last_route")
+    return rc
 
 
 def ssm_scan_profile_start(max_launches: int) -> None:

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -14,7 +15,9 @@
 namespace ssm {
 bool simt_supported(const Params &p);
 cudaError_t simt_forward(const Params &p, cudaStream_t st);
-cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk);
+cudaError_t simt_backward(const Params &p, cudaStream_t st);
+cudaError_t chunk_backward(const Params &p, cudaStream_t st);
+cudaError_t chunk_range_check(const Params &p, int *gate, cudaStream_t st);
 bool chunk_bwd_supported(const Params &p);
 bool chunk_fwd_supported(const Params &p);
 cudaError_t chunk_forward(const Params &p, cudaStream_t st);
@@ -25,6 +28,39 @@ int chunk_rev_error_take();
 namespace {
 
 thread_local std::string g_last_error;
+
+// Gate words of the device-side choice between the tensor-core chain and the
+// recurrent chain (written by the range check of each call).  One slot per
+// call from a ring, so that calls in flight on different streams do not share
+// a word.
+constexpr unsigned kGateSlots = 4096;
+__device__ int g_gate_ring[kGateSlots];
+std::atomic<unsigned> g_gate_next{0};
+std::mutex g_gate_mu;
+int *g_gate_base[64];
+// route of the last call on this host thread: its gate word (chunk-eligible
+// calls) or the recurrent route chosen on the host
+thread_local const int *g_last_gate = nullptr;
+thread_local int g_last_route = -1;
+
+cudaError_t gate_slot(int **out, cudaStream_t st) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(g_gate_mu);
+        if (!g_gate_base[dev]) {
+            void *ptr = nullptr;
+            if ((e = cudaGetSymbolAddress(&ptr, g_gate_ring)) != cudaSuccess) return e;
+            g_gate_base[dev] = static_cast<int *>(ptr);
+        }
+    }
+    int *g = g_gate_base[dev] + (g_gate_next.fetch_add(1) % kGateSlots);
+    if ((e = cudaMemsetAsync(g, 0, sizeof(int), st)) != cudaSuccess) return e;
+    *out = g;
+    return cudaSuccess;
+}
 
 // per-kernel timing session (see ssm_scan_profile_start)
 struct ProfileRec {
@@ -268,9 +304,34 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     if (!chunked && !ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
-    profile_begin((cudaStream_t)stream);
-    cudaError_t e = chunked ? ssm::chunk_forward(p, (cudaStream_t)stream)
-                            : ssm::simt_forward(p, (cudaStream_t)stream);
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    cudaError_t e = cudaSuccess;
+    if (chunked) {
+        // both chains are launched; the range check picks one on the device
+        int *gate = nullptr;
+        const bool fallback = ssm::simt_supported(p);
+        if (fallback) {
+            e = gate_slot(&gate, st);
+            if (e == cudaSuccess) e = ssm::chunk_range_check(p, gate, st);
+        }
+        ssm::Params pc = p;
+        pc.gate = gate;
+        pc.gate_on = 0;
+        if (e == cudaSuccess) e = ssm::chunk_forward(pc, st);
+        if (e == cudaSuccess && fallback) {
+            ssm::Params ps = p;
+            ps.gate = gate;
+            ps.gate_on = 1;
+            e = ssm::simt_forward(ps, st);
+        }
+        g_last_gate = gate;
+        g_last_route = SSM_ROUTE_CHUNKED;
+    } else {
+        e = ssm::simt_forward(p, st);
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_RECURRENT;
+    }
     profile_end();
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
     g_last_error.clear();
@@ -334,15 +395,33 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
     // dD is written by the parameter pass; keep it defined when R != O
-    const bool chunked = d->chunk != 1 && ssm::chunk_bwd_supported(p);
-    if (chunked && lay.boundary) {
-        p.ws_kb = (float *)(ws + lay.off_kb);
-        p.ws_qb = (float *)(ws + lay.off_qb);
-        p.ws_gc = (float *)(ws + lay.off_gc);
-        p.ws_ce = (float *)(ws + lay.off_ce);
-    }
+    const bool chunked = d->chunk != 1 && ssm::chunk_bwd_supported(p) && lay.boundary;
     profile_begin(st);
-    cudaError_t e = ssm::simt_backward(p, st, chunked);
+    cudaError_t e = cudaSuccess;
+    if (chunked) {
+        // both chains are launched; the range check picks one on the device
+        int *gate = nullptr;
+        e = gate_slot(&gate, st);
+        if (e == cudaSuccess) e = ssm::chunk_range_check(p, gate, st);
+        ssm::Params pc = p;
+        pc.ws_kb = (float *)(ws + lay.off_kb);
+        pc.ws_qb = (float *)(ws + lay.off_qb);
+        pc.ws_gc = (float *)(ws + lay.off_gc);
+        pc.ws_ce = (float *)(ws + lay.off_ce);
+        pc.gate = gate;
+        pc.gate_on = 0;
+        if (e == cudaSuccess) e = ssm::chunk_backward(pc, st);
+        ssm::Params ps = p;
+        ps.gate = gate;
+        ps.gate_on = 1;
+        if (e == cudaSuccess) e = ssm::simt_backward(ps, st);
+        g_last_gate = gate;
+        g_last_route = SSM_ROUTE_CHUNKED;
+    } else {
+        e = ssm::simt_backward(p, st);
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_RECURRENT;
+    }
     profile_end();
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
     g_last_error.clear();
@@ -364,6 +443,17 @@ int ssm_scan_poll_device_error(void *stream) {
 }
 
 int ssm_scan_abi_version(void) { return SSM_SCAN_ABI_VERSION; }
+
+int ssm_scan_last_route(void *stream) {
+    if (g_last_route < 0) return fail(SSM_ERR_ARG, "no scan call on this thread yet");
+    if (g_last_route != SSM_ROUTE_CHUNKED || !g_last_gate) return g_last_route;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_last_route");
+    int v = 0;
+    e = cudaMemcpy(&v, g_last_gate, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_last_route (gate word)");
+    return v ? SSM_ROUTE_RANGE_FALLBACK : SSM_ROUTE_CHUNKED;
+}
 
 int ssm_scan_profile_start(int max_launches) {
     if (max_launches < 1) return fail(SSM_ERR_ARG, "max_launches must be >= 1");

@@ -43,8 +43,16 @@ struct Params {
     float *ws_gc;   // [B][H][NC][N][P]  chunk-local adjoint, then the adjoint carried into each chunk
     float *ws_ce;   // [B][H][NC][128][2] full-chunk decay e^{lam S_63} per mode (re, im)
     int nc;         // number of 64-token chunks
+    // device-side choice between two launched kernel chains: a kernel runs
+    // only when (*gate != 0) == gate_on (no gate: always)
+    const int *gate;
+    int gate_on;
     Geometry geo;
 };
+
+__device__ __forceinline__ bool gated_off(const Params &p) {
+    return p.gate && ((*p.gate != 0) != (p.gate_on != 0));
+}
 
 // per-unit partial slots in ws_par
 __host__ __device__ inline int npar_of(const Params &p) { return p.ndec + p.np + 2; }

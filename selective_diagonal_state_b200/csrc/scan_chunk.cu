@@ -66,6 +66,7 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 __global__ void __launch_bounds__(THREADS, 1)
 k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, Params p) {
+    if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -578,6 +579,7 @@ constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 __global__ void __launch_bounds__(chunkfwd::THREADS, 1)
 k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmDY, Params p) {
+    if (gated_off(p)) return;
     using namespace chunkfwd;
     using namespace umma;
     namespace cb = chunkbwd;
@@ -1048,6 +1050,42 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
 // ---------------------------------------------------------------------------
 
 }  // namespace chunkfwd
+
+// Range condition of the folded operands.  Inside a 16-token sub-block the
+// folded factors reach 2^(+-|a| log2(e) sum dt) (|a| the largest decay rate of
+// the head), which must stay inside the bf16 / fp32 exponent range; a call
+// where any sub-block goes past RANGE_LOG2 sets *gate, and the recurrent
+// kernels take the call instead (their chain is launched behind the same gate).
+constexpr float RANGE_LOG2 = 100.f;
+
+__global__ void k_range_check(Params p, int *gate) {
+    const int nsb = (p.L + 15) / 16;
+    const long long items = (long long)p.Bsz * nsb * p.H;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < items;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int h = (int)(i % p.H);
+        const long long r = i / p.H;
+        const int sb = (int)(r % nsb), b = (int)(r / nsb);
+        float amax = p.A_log[h * p.ndec];
+        for (int m = 1; m < p.ndec; ++m) amax = fmaxf(amax, p.A_log[h * p.ndec + m]);
+        float span = 0.f;
+        for (int k = 0; k < 16; ++k) {
+            const int t = 16 * sb + k;
+            if (t < p.L) span += ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+        }
+        if (!(expf(amax) * 1.4426950408889634f * span <= RANGE_LOG2)) *gate = 1;
+    }
+}
+
+cudaError_t chunk_range_check(const Params &p, int *gate, cudaStream_t st) {
+    const long long items = (long long)p.Bsz * ((p.L + 15) / 16) * p.H;
+    long long blocks = (items + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    k_range_check<<<(int)blocks, 256, 0, st>>>(p, gate);
+    profile_mark(st, "k_range_check");
+    return cudaGetLastError();
+}
 
 // Whether the tensor-core forward handles this problem.
 bool chunk_fwd_supported(const Params &p) {

@@ -158,6 +158,7 @@ constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 __global__ void __launch_bounds__(loc::THREADS)
 k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
                   Params p) {
+    if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -298,6 +299,7 @@ constexpr int KMAX = NP / 16;   // row pairs per thread
 }  // namespace pass
 
 __global__ void __launch_bounds__(pass::THREADS, 2) k_chunk_adj_pass(Params p) {
+    if (gated_off(p)) return;
     // chunk decays, triple-buffered: chunk c-1's are fetched while chunk c is processed
     __shared__ float s_ce[3][2 * NP];
     __shared__ float red[pass::THREADS];
@@ -417,7 +419,8 @@ __global__ void __launch_bounds__(pass::THREADS, 2) k_chunk_adj_pass(Params p) {
 // with the scores built exactly as in the forward: scores^T_i = Bi . Ci^T.
 // ============================================================================
 namespace dxk {
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;
+constexpr int RG = THREADS / 64;   // row groups of the operand preparation
 constexpr uint32_t TMEM_COLS = 64;
 constexpr uint32_t SM_B = 0;          // 16 KB raw B (swizzled halves)
 constexpr uint32_t SM_C = 16384;      // 16 KB raw C
@@ -435,6 +438,7 @@ constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 __global__ void __launch_bounds__(dxk::THREADS, 1)
 k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                const __grid_constant__ CUtensorMap tmDY, Params p) {
+    if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -509,8 +513,8 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
             const unsigned char *sB = sm + dxk::SM_B, *sC = sm + dxk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
-            for (int k = 0; k < 4; ++k) {
-                const int r0 = 8 * (grp + 4 * k);
+            for (int k = 0; k < NP / (8 * dxk::RG); ++k) {
+                const int r0 = 8 * (grp + dxk::RG * k);
                 if (r0 >= N) break;
                 float vCI[8], vBI[8], vBH[8], vBX[3][8], rc[8], rb[8];
                 ld_rows8(sC, t, r0, rc);
@@ -574,7 +578,7 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
                 }
                 st16(sm + dxk::SM_BH, off_mnmaj(r0, t, 2048u, 128u), vBH);
             }
-            f32[F_CP + grp * 64 + t] = corr;
+            reinterpret_cast<float *>(sm + dxk::SM_P)[grp * 64 + t] = corr;   // P is written later
         }
         fence_proxy_async();
         fence_before_sync();
@@ -601,7 +605,7 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) cs += f32[F_CP + k * 64 + tid];
+            for (int k = 0; k < dxk::RG; ++k) cs += reinterpret_cast<const float *>(sm + dxk::SM_P)[k * 64 + tid];
             f32[F_CORR + tid] = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
         }
         ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
@@ -609,7 +613,7 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
         fence_after_sync();
         if (__syncthreads_and(ok)) {
             // ---- masked scores -> P^T (K-major rows s, K = t), zero where s > t
-            if (warp >= 4) {
+            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
                 const int qd = warp - 4;
                 for (int i = 0; i < NSB; ++i) {
                     float v[16];
@@ -646,15 +650,16 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
             fence_after_sync();
             if (__syncthreads_and(ok)) {
                 // ---- epilogue: dx_s = DX_s + corr_s dy_s
-                const int qd = warp & 3, half = warp >> 2;
+                const int qd = warp & 3, half = warp >> 2;   // columns split over THREADS / 128 warp sets
+                constexpr int CPW = 64 / (dxk::THREADS / 128);
                 const int s = 16 * qd + (lane & 15);
                 const unsigned char *sDY = sm + dxk::SM_DY;
                 __nv_bfloat16 *xrow = reinterpret_cast<__nv_bfloat16 *>(p.dx) + b * p.sx[0] +
                                       (long long)(t0 + s) * p.sx[1] + h * p.sx[2];
                 const float cr = f32[F_CORR + s];
-                for (int c16 = 0; c16 < 2; ++c16) {
+                for (int c16 = 0; c16 < CPW / 16; ++c16) {
                     float v[16];
-                    const int pc = 32 * half + 16 * c16;
+                    const int pc = CPW * half + 16 * c16;
                     tmem_ld16(tmem_addr(t_dx, 32u * qd, (uint32_t)pc), v);
                     if (lane < 16 && t0 + s < L) {
 #pragma unroll
@@ -698,7 +703,10 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
 // Also writes <dy_t, u_t>, dsigma_t = B_t . gbu_t and (C_t . B_t) <dy_t, u_t>.
 // ============================================================================
 namespace gbk {
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;
+constexpr int RG = THREADS / 64;    // row groups of the operand preparation
+constexpr int TQ = THREADS / 128;   // token groups of the unfold
+constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
 constexpr uint32_t TMEM_COLS = 128;
 constexpr uint32_t SM_X = 0;           // 8 KB  x (swizzled)
 constexpr uint32_t SM_DY = 8192;       // 8 KB  dy (swizzled)
@@ -725,6 +733,7 @@ __global__ void __launch_bounds__(gbk::THREADS, 1)
 k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
                 Params p) {
+    if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -799,8 +808,8 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
-            for (int k = 0; k < 4; ++k) {
-                const int r0 = 8 * (grp + 4 * k);
+            for (int k = 0; k < NP / (8 * gbk::RG); ++k) {
+                const int r0 = 8 * (grp + gbk::RG * k);
                 if (r0 >= N) break;
                 float rc[8], rb[8], v[8], vx[3][8];
                 ld_rows8(sC, t, r0, rc);
@@ -845,19 +854,19 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         st16_split(sm + gbk::SM_CM + cm_off(jj), sm + gbk::SM_CML + cm_off(jj),
                                    off_mnmaj(r0, t - 16 * jj, 2048u, 128u), vx[jj]);
             }
-            f32[F_CP + grp * 64 + t] = corr;
+            reinterpret_cast<float *>(sm + gbk::SM_GM)[grp * 64 + t] = corr;   // G' tiles come later
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
 
         // this thread's rows of the per-head dC (forward-direction part), in flight during the MMAs
-        float kd[32];
+        float kd[gbk::TPT];
         {
-            const int n = tid & 127, half = tid >> 7;
+            const int n = tid & 127, tq = tid >> 7;
 #pragma unroll
-            for (int i2 = 0; i2 < 32; ++i2) {
-                const int t = t0 + 32 * half + i2;
+            for (int i2 = 0; i2 < gbk::TPT; ++i2) {
+                const int t = t0 + gbk::TPT * tq + i2;
                 kd[i2] = (n < N && t < L) ? __ldg(p.ws_dC + ix_wsk(p, b, t, h, 0, 1, n)) : 0.f;
             }
         }
@@ -882,7 +891,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) cs += f32[F_CP + k * 64 + tid];
+            for (int k = 0; k < gbk::RG; ++k) cs += reinterpret_cast<const float *>(sm + gbk::SM_GM)[k * 64 + tid];
             f32[F_CORR + tid] = cs;   // C_t . B_t
         }
         ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
@@ -890,7 +899,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         fence_after_sync();
         if (__syncthreads_and(ok)) {
             // ---- masked G' rows -> K-major tiles (rows t of sub-block qd, K = t' >= t)
-            if (warp >= 4) {
+            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
                 const int qd = warp - 4;
                 for (int i = 0; i < NSB; ++i) {
                     float v[16];
@@ -945,10 +954,11 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 // then, per state mode, the within-chunk suffix sums of the decay-gradient
                 // identity (X_t - Y_t, X = conj(c) dCK, Y = b conj(sigma gbu)), walking the
                 // tokens backwards; and dB / dC directly when a group has one head.
+                // Thread (row n, token group tq) takes tokens TPT tq .. TPT tq + TPT - 1.
                 float *red = reinterpret_cast<float *>(sm + gbk::SM_CM);     // [128][RED_LD] B . gbu
                 float *red2 = reinterpret_cast<float *>(sm + gbk::SM_CML);   // [128][RED_LD] ddt terms
-                float *xch = reinterpret_cast<float *>(sm + gbk::SM_GM);     // [2][128] upper-half totals
-                const int n = tid & 127, half = tid >> 7, qd = warp & 3;
+                float *xch = reinterpret_cast<float *>(sm + gbk::SM_GM);     // [3][TQ][128] group totals
+                const int n = tid & 127, tq = tid >> 7, qd = warp & 3;
                 const bool valid = n < N;
                 const int m = n < nr ? n : nr + ((n - nr) >> 1);
                 const bool pr_row = valid && n >= nr;
@@ -961,17 +971,23 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
                 const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
                 float cum = 0.f, dacc = 0.f, sdt = 0.f;
+                const int tc = gbk::TPT * tq;
 #pragma unroll
-                for (int c16 = 1; c16 >= 0; --c16) {
-                    const int tc = 32 * half + 16 * c16;
+                for (int c16 = gbk::TPT / 16 - 1; c16 >= 0; --c16) {
                     float vv[16], ee[16];
-                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)tc), vv);
-                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), ee);
+                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)(tc + 16 * c16)), vv);
+                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)(tc + 16 * c16)), ee);
+                    const int jb = (tc + 16 * c16) >> 4;   // sub-block of these 16 tokens
+                    const float se = f32[F_S + 16 * jb + 15];
+                    float fr = 1.f, fi = 0.f;
+                    if (jb < 3 && valid) {
+                        fr = f32[F_KRE + fslot(jb + 1, 4) * NP + m];
+                        fi = f32[F_KIM + fslot(jb + 1, 4) * NP + m];
+                    }
 #pragma unroll
                     for (int j = 15; j >= 0; --j) {
-                        const int t = tc + j;
-                        const int jb = t >> 4;
-                        const float ds = f32[F_S + 16 * jb + 15] - f32[F_S + t];   // >= 0
+                        const int t = tc + 16 * c16 + j;
+                        const float ds = se - f32[F_S + t];   // >= 0
                         const float mag = ex2_fast(a2 * ds);
                         float er = mag, ei = 0.f;
                         if (pr_row) {
@@ -979,11 +995,6 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                             __sincosf(w * ds, &sn, &cs);
                             er = mag * cs;
                             ei = mag * sn;
-                        }
-                        float fr = 1.f, fi = 0.f;
-                        if (jb < 3 && valid) {
-                            fr = f32[F_KRE + fslot(jb + 1, 4) * NP + m];
-                            fi = f32[F_KIM + fslot(jb + 1, 4) * NP + m];
                         }
                         const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
                         const float eo = __shfl_xor_sync(0xffffffffu, ee[j], 1);
@@ -1035,42 +1046,59 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         }
                     }
                 }
-                // the upper half's totals carry into every token of the lower half
-                if (half == 1) {
-                    xch[n] = cum;
-                    xch[128 + n] = dacc;
-                }
+                // later token groups carry into every token of earlier ones
+                xch[tq * 128 + n] = cum;
                 __syncthreads();
-                if (half == 0) {
-                    const float tot1 = xch[n];
-                    const float add = coef * tot1;
-                    for (int t = 0; t < 32; ++t) red2[n * gbk::RED_LD + t] += add;
-                    dacc += (im_row ? -tot1 : tot1) * sdt + xch[128 + n];
-                    if (valid) {
-                        const int nmode = p.nr + p.np;
-                        float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
-                        const float tot = cum + tot1;
-                        if (!pr_row) {
-                            blk[4 * m + 0] = tot;
-                            blk[4 * m + 1] = 0.f;
-                            blk[4 * m + 2] = dacc;
-                            blk[4 * m + 3] = 0.f;
-                        } else if (!im_row) {
-                            blk[4 * m + 0] = tot;
-                            blk[4 * m + 2] = dacc;
-                        } else {
-                            blk[4 * m + 1] = tot;
-                            blk[4 * m + 3] = dacc;
-                        }
+                float later = 0.f;
+                for (int k = tq + 1; k < gbk::TQ; ++k) later += xch[k * 128 + n];
+                if (later != 0.f) {
+                    const float add = coef * later;
+                    for (int t = tc; t < tc + gbk::TPT; ++t) red2[n * gbk::RED_LD + t] += add;
+                }
+                dacc += (im_row ? -later : later) * sdt;
+                xch[(gbk::TQ + tq) * 128 + n] = dacc;
+                __syncthreads();
+                if (tq == 0 && valid) {
+                    float tot = 0.f, da = 0.f;
+                    for (int k = 0; k < gbk::TQ; ++k) {
+                        tot += xch[k * 128 + n];
+                        da += xch[(gbk::TQ + k) * 128 + n];
                     }
+                    const int nmode = p.nr + p.np;
+                    float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
+                    if (!pr_row) {
+                        blk[4 * m + 0] = tot;
+                        blk[4 * m + 1] = 0.f;
+                        blk[4 * m + 2] = da;
+                        blk[4 * m + 3] = 0.f;
+                    } else if (!im_row) {
+                        blk[4 * m + 0] = tot;
+                        blk[4 * m + 2] = da;
+                    } else {
+                        blk[4 * m + 1] = tot;
+                        blk[4 * m + 3] = da;
+                    }
+                }
+                // column sums over the state rows: all threads, 128 / RG rows each, fixed order
+                float *part = xch + 2 * gbk::TQ * 128;   // [2][RG][64]
+                {
+                    const int t = tid & 63, rg = tid >> 6;
+                    constexpr int RPG = NP / gbk::RG;
+                    float s1 = 0.f, s2 = 0.f;
+                    for (int k = rg * RPG; k < rg * RPG + RPG && k < N; ++k) {
+                        s1 += red[k * gbk::RED_LD + t];
+                        s2 += red2[k * gbk::RED_LD + t];
+                    }
+                    part[rg * 64 + t] = s1;
+                    part[(gbk::RG + rg) * 64 + t] = s2;
                 }
                 __syncthreads();
                 if (tid < 64 && t0 + tid < L) {
                     const int t = tid;
                     float dsig = 0.f, dd = 0.f;
-                    for (int k = 0; k < N; ++k) {
-                        dsig += red[k * gbk::RED_LD + t];
-                        dd += red2[k * gbk::RED_LD + t];
+                    for (int k = 0; k < gbk::RG; ++k) {
+                        dsig += part[k * 64 + t];
+                        dd += part[(gbk::RG + k) * 64 + t];
                     }
                     const long long i = ix_bth(p, b, t0 + t, h);
                     const float m2 = f32[F_LAM + t];

@@ -301,6 +301,7 @@ __device__ __forceinline__ Lane lane_of(const Params &p) {
 // ------------------------------------------------------------------------
 template <int NR, int NPR, int RM>
 __global__ void __launch_bounds__(MAXT) k_fwd(Params p) {
+    if (gated_off(p)) return;
     extern __shared__ __align__(16) float smem[];
     constexpr int NS = NR + 2 * NPR;
     const Geometry &g = p.geo;
@@ -427,6 +428,7 @@ __device__ __forceinline__ void put_reduced(float *dst, const float (&v)[K], int
 // ------------------------------------------------------------------------
 template <int NR, int NPR, int RM, int S>
 __global__ void __launch_bounds__(MAXT) k_bwd_sweep1(Params p) {
+    if (gated_off(p)) return;
     extern __shared__ __align__(16) float smem[];
     constexpr int NS = NR + 2 * NPR;
     constexpr int KV = RM * NS;
@@ -518,6 +520,7 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep1(Params p) {
 // ------------------------------------------------------------------------
 template <int NR, int NPR, int RM, int S>
 __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
+    if (gated_off(p)) return;
     extern __shared__ __align__(16) float smem[];
     constexpr int NS = NR + 2 * NPR;
     constexpr int KV = RM * NS;
@@ -766,9 +769,8 @@ __device__ __forceinline__ ModeInfo mode_info(const Params &p, int h, int m) {
     return mi;
 }
 
-__global__ void __launch_bounds__(256) k_bwd_units_local(Params p) {
-    extern __shared__ __align__(16) float smem[];
-    const int tb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+__device__ __forceinline__ void units_local_item(const Params &p, float *smem, int tb, int h,
+                                                 int b) {
     const int m = threadIdx.x, nthr = blockDim.x;
     const int g = h / p.hpg;
     const int NTB = ntb_of(p), nmode = p.nr + p.np;
@@ -850,8 +852,23 @@ __global__ void __launch_bounds__(256) k_bwd_units_local(Params p) {
     }
 }
 
+// one (time block, head, batch row) item per block iteration; a capped grid
+// strides over them
+__global__ void __launch_bounds__(256) k_bwd_units_local(Params p) {
+    if (gated_off(p)) return;
+    extern __shared__ __align__(16) float smem[];
+    const int NTB = ntb_of(p);
+    const long long items = (long long)NTB * p.H * p.Bsz;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+        const long long r = it / NTB;
+        units_local_item(p, smem, (int)(it - r * NTB), (int)(r % p.H), (int)(r / p.H));
+        __syncthreads();
+    }
+}
+
 // carry the block totals across time blocks: per (b, h), one thread per mode
 __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
+    if (gated_off(p)) return;
     extern __shared__ __align__(16) float smem[];
     const int h = blockIdx.x, b = blockIdx.y;
     const int m = threadIdx.x, nthr = blockDim.x;
@@ -911,6 +928,7 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
 
 // ddt and dlambda per (b, t, h)
 __global__ void k_bwd_units_final(Params p) {
+    if (gated_off(p)) return;
     const long long total = (long long)p.Bsz * p.L * p.H;
     const int NTB = ntb_of(p);
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -940,9 +958,7 @@ __global__ void k_bwd_units_final(Params p) {
 }
 
 // dB, dC per (b, t): sum over the heads of each group; per-head scalars first
-__global__ void __launch_bounds__(256) k_bwd_groups(Params p) {
-    extern __shared__ __align__(16) float smem[];
-    const int t = blockIdx.x, b = blockIdx.y;
+__device__ __forceinline__ void groups_item(const Params &p, float *smem, int t, int b) {
     float *s_sig = smem, *s_bn = smem + p.H;
     for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
         const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
@@ -984,8 +1000,20 @@ __global__ void __launch_bounds__(256) k_bwd_groups(Params p) {
     }
 }
 
+// one (token, batch row) item per block iteration; a capped grid strides over them
+__global__ void __launch_bounds__(256) k_bwd_groups(Params p) {
+    if (gated_off(p)) return;
+    extern __shared__ __align__(16) float smem[];
+    const long long items = (long long)p.L * p.Bsz;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+        groups_item(p, smem, (int)(it % p.L), (int)(it / p.L));
+        __syncthreads();
+    }
+}
+
 // parameter gradients: sum the per-unit partials over the batch
 __global__ void k_bwd_params(Params p) {
+    if (gated_off(p)) return;
     const int np1 = npar_of(p);
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.H * (p.ndec + p.np + 1);
          i += gridDim.x * blockDim.x) {
@@ -1165,49 +1193,60 @@ bool chunk_bwd_supported(const Params &p);
 cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st);
 cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st);
 
-// use_chunk: the tensor-core kernels replace both sweeps (forward-direction dC,
-// then the chunk-parallel reverse part); the finalize kernels are shared.
-cudaError_t simt_backward(const Params &p, cudaStream_t st, bool use_chunk) {
+// Finalize passes shared by both backward chains: within-block decay sums
+// (when the chain has not produced them), block carries, per-token ddt and
+// dlambda, group sums of dB / dC (when the chain has not written them), and
+// the batch sums of the parameter gradients.  Item grids are capped and
+// strided so that a gated-off chain costs one short launch per kernel.
+static cudaError_t bwd_finalize(const Params &p, cudaStream_t st, bool local, bool groups) {
     cudaError_t e;
-    if (use_chunk)
-        e = chunk_bwd_dc(p, st);
-    else
-        e = launch_scan(KK_S1, p, st);
-    if (e != cudaSuccess) return e;
-    // the chunk-parallel reverse part also produces the per-block decay sums
-    // (and dB / dC when every group has one head)
-    const bool rev = use_chunk && p.ws_gc;
-    if (rev)
-        e = chunk_bwd_reverse(p, st);
-    else
-        e = launch_scan(KK_S2, p, st);
-    if (e != cudaSuccess) return e;
-    {
-        int nthr = ((p.nr + p.np + 31) / 32) * 32;
-        if (nthr < 32) nthr = 32;
-        if (!rev) {
-            k_bwd_units_local<<<dim3(ntb_of(p), p.H, p.Bsz), nthr, (size_t)FT * nthr * 4, st>>>(p);
-            profile_mark(st, "k_bwd_units_local");
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        k_bwd_units_carry<<<dim3(p.H, p.Bsz), nthr, (size_t)nthr * 4, st>>>(p);
-        profile_mark(st, "k_bwd_units_carry");
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const long long total = (long long)p.Bsz * p.L * p.H;
-        int blocks = (int)((total + 255) / 256);
-        if (blocks > 148 * 32) blocks = 148 * 32;
-        k_bwd_units_final<<<blocks, 256, 0, st>>>(p);
-        profile_mark(st, "k_bwd_units_final");
+    int nthr = ((p.nr + p.np + 31) / 32) * 32;
+    if (nthr < 32) nthr = 32;
+    const long long cap = 148LL * 16;
+    if (local) {
+        const long long items = (long long)ntb_of(p) * p.H * p.Bsz;
+        const int blocks = (int)(items < cap ? items : cap);
+        k_bwd_units_local<<<blocks, nthr, (size_t)FT * nthr * 4, st>>>(p);
+        profile_mark(st, "k_bwd_units_local");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (!(rev && p.hpg == 1)) {
-        k_bwd_groups<<<dim3(p.L, p.Bsz), 256, (size_t)2 * p.H * 4, st>>>(p);
+    k_bwd_units_carry<<<dim3(p.H, p.Bsz), nthr, (size_t)nthr * 4, st>>>(p);
+    profile_mark(st, "k_bwd_units_carry");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long total = (long long)p.Bsz * p.L * p.H;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    k_bwd_units_final<<<blocks, 256, 0, st>>>(p);
+    profile_mark(st, "k_bwd_units_final");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (groups) {
+        const long long items = (long long)p.L * p.Bsz;
+        const int gb = (int)(items < cap ? items : cap);
+        k_bwd_groups<<<gb, 256, (size_t)2 * p.H * 4, st>>>(p);
         profile_mark(st, "k_bwd_groups");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     k_bwd_params<<<4, 256, 0, st>>>(p);
     profile_mark(st, "k_bwd_params");
     return cudaGetLastError();
+}
+
+// Recurrent backward: both sweeps token by token, then the finalize passes.
+cudaError_t simt_backward(const Params &p, cudaStream_t st) {
+    cudaError_t e;
+    if ((e = launch_scan(KK_S1, p, st)) != cudaSuccess) return e;
+    if ((e = launch_scan(KK_S2, p, st)) != cudaSuccess) return e;
+    return bwd_finalize(p, st, true, true);
+}
+
+// Tensor-core backward: forward-direction dC, then the chunk-parallel reverse
+// part, which also produces the within-block decay sums (and dB / dC when every
+// group has one head), then the shared finalize passes.
+cudaError_t chunk_backward(const Params &p, cudaStream_t st) {
+    cudaError_t e;
+    if ((e = chunk_bwd_dc(p, st)) != cudaSuccess) return e;
+    if ((e = chunk_bwd_reverse(p, st)) != cudaSuccess) return e;
+    return bwd_finalize(p, st, false, p.hpg != 1);
 }
 
 }  // namespace ssm

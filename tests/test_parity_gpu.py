@@ -21,17 +21,34 @@ def _lib():
     assert torch.cuda.is_available()
 
 
-def run_gpu(shape, inp, backward=True):
+def chunk_eligible(shape):
+    """Shapes the tensor-core kernels take (the rest go to the recurrent ones)."""
+    return (shape.dtype_io == S.DTYPE_BF16 and shape.headdim == 64 and shape.rank_in == 1
+            and shape.rank_out == 1 and shape.nstate in (64, 128) and shape.n_real % 8 == 0
+            and shape.seqlen > 0 and shape.chunk != 1)
+
+
+def expected_route(shape):
+    return abi.ROUTE_CHUNKED if chunk_eligible(shape) else abi.ROUTE_RECURRENT
+
+
+def run_gpu(shape, inp, backward=True, route=None):
+    """Forward (and backward) through the C ABI; checks which kernels ran."""
+    route = expected_route(shape) if route is None else route
     dev = scan.to_device(shape, inp)
     y, hT, wT = scan.scan_forward(shape, dev)
-    g = scan.scan_backward(shape, dev) if backward else None
+    assert abi.ssm_scan_last_route() == route
+    g = None
+    if backward:
+        g = scan.scan_backward(shape, dev)
+        assert abi.ssm_scan_last_route() == route
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
     return y, hT, wT, g
 
 
-def check_all(shape, inp, backward=True, report=None):
-    y, hT, wT, g = run_gpu(shape, inp, backward)
+def check_all(shape, inp, backward=True, report=None, route=None):
+    y, hT, wT, g = run_gpu(shape, inp, backward, route)
     ref = oracle.scan_fwd(shape, inp)
     dt = shape.dtype_io
     compare("y", to_np(y), ref["y"], dt, report)
@@ -201,3 +218,52 @@ def test_backward_deterministic():
     torch.cuda.synchronize()
     for x1, x2 in zip(a, (g2.dx, g2.ddt, g2.dBm, g2.dCm, g2.dA_log, g2.dD)):
         assert torch.equal(x1, x2)
+
+
+def _scaled_dt(shape, inp, factor, rows=None):
+    """Copy of the inputs with dt scaled (bf16-rounded again); `rows` limits it to
+    some batch rows and a token range."""
+    out = dict(inp)
+    dt = inp["dt"].copy()
+    if rows is None:
+        dt = dt * factor
+    else:
+        b, t0, t1 = rows
+        dt[b, t0:t1] = dt[b, t0:t1] * factor
+    out["dt"] = S.round_bf16(dt) if shape.dtype_io == S.DTYPE_BF16 else dt
+    return out
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(decay_mode=S.DECAY_PER_HEAD, two_endpoint=0,
+                                             n_real=128, n_pairs=0, ngroups=2)])
+def test_large_decay_takes_recurrent_route(kw):
+    """Inputs whose per-sub-block decay leaves the folding range (|A| log2(e)
+    sum of 16 dt > 100) give the oracle's result through the recurrent kernels."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=150, nheads=4, ngroups=4).replace(**kw)
+    inp = _scaled_dt(shape, S.make_inputs(shape, seed=41, with_state=True), 60.0)
+    a_max = np.exp(inp["A_log"].max(axis=1))
+    span = np.array([[inp["dt"][b, 16 * k:16 * k + 16, h].sum() for k in range(150 // 16 + 1)]
+                     for b in range(2) for h in range(4)])
+    assert (span.max() * a_max.max() * np.log2(np.e)) > 100.0
+    check_all(shape, inp, route=abi.ROUTE_RANGE_FALLBACK)
+
+
+def test_one_hot_sub_block_takes_recurrent_route():
+    """A single out-of-range stretch in one batch row moves the whole call."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=130, nheads=4, ngroups=4)
+    inp = _scaled_dt(shape, S.make_inputs(shape, seed=43), 200.0, rows=(1, 70, 90))
+    check_all(shape, inp, route=abi.ROUTE_RANGE_FALLBACK)
+
+
+def test_moderate_decay_stays_chunked():
+    """Large but in-range sub-block decays keep the tensor-core kernels and
+    their parity."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=140, nheads=4, ngroups=4)
+    inp = S.make_inputs(shape, seed=45)
+    # scale dt so that the largest sub-block exponent is about 60 (of the 100 allowed)
+    a_max = np.exp(inp["A_log"].max())
+    span = max(inp["dt"][b, 16 * k:16 * k + 16, h].sum()
+               for b in range(2) for h in range(4) for k in range(140 // 16 + 1))
+    f = 60.0 / (a_max * np.log2(np.e) * span)
+    inp = _scaled_dt(shape, inp, f)
+    check_all(shape, inp, route=abi.ROUTE_CHUNKED)
