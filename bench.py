@@ -296,6 +296,7 @@ def main():
     fwd_out = scan.alloc_fwd(shape)
     grads = scan.alloc_bwd(shape)
     ws = scan.alloc_workspace(shape, abi.PASS_BWD, desc=desc)
+    wsf = scan.alloc_workspace(shape, abi.PASS_FWD, desc=desc)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -307,7 +308,7 @@ def main():
             sdist.allreduce_param_grads((grads.dA_log, grads.dtheta, grads.dD))
 
     def step():
-        scan.scan_forward(shape, dev, out=fwd_out, desc=desc)
+        scan.scan_forward(shape, dev, out=fwd_out, desc=desc, workspace=wsf)
         scan.scan_backward(shape, dev, grads=grads, workspace=ws, desc=desc)
         allreduce_params()
 
@@ -346,7 +347,7 @@ def main():
     torch.cuda.synchronize()
     f0.record(stream)
     for _ in range(args.steps):
-        scan.scan_forward(shape, dev, out=fwd_out, desc=desc)
+        scan.scan_forward(shape, dev, out=fwd_out, desc=desc, workspace=wsf)
     f1.record(stream)
     torch.cuda.synchronize()
     ms_fwd = f0.elapsed_time(f1) / args.steps

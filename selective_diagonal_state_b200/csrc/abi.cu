@@ -171,16 +171,34 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
 }
 
 struct BwdWs {
-    size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, off_kb, off_qb,
+    size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, off_kp, off_qb,
         off_gc, off_ce, total;
     bool boundary;  // chunk-boundary carries (tensor-core backward shapes)
 };
 
-// Shapes the tensor-core backward may take (pointer alignment is checked at call time).
-bool tensor_bwd_shape(const ssm_desc_t *d) {
+// Shapes the tensor-core chain may take (pointer alignment is checked at call time).
+bool tensor_chain_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
     return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0;
+}
+
+// Forward workspace of the tensor-core chain: the state entering every
+// 64-token chunk [B][H][L/64][N][P] and the chunk decays [B][H][L/64][128][2].
+struct FwdWs {
+    size_t off_kp, off_ce, total;
+};
+FwdWs fwd_layout(const ssm_desc_t *d) {
+    FwdWs w;
+    w.off_kp = w.off_ce = w.total = 0;
+    if (!tensor_chain_shape(d)) return w;
+    const size_t ntb = (size_t)(d->seqlen + 63) / 64;
+    w.off_kp = 0;
+    size_t off = align256((size_t)d->batch * d->nheads * ntb * nstate(d) * d->headdim * 4);
+    w.off_ce = off;
+    off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * 2 * 4);
+    w.total = off;
+    return w;
 }
 
 BwdWs bwd_layout(const ssm_desc_t *d) {
@@ -206,10 +224,10 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     off = align256(off + (size_t)d->batch * d->nheads * ntb * (4 * nmode + 2) * 4);
     w.off_blkc = off;
     off = align256(off + (size_t)d->batch * d->nheads * ntb * 4);
-    w.boundary = tensor_bwd_shape(d);
-    w.off_kb = w.off_qb = w.off_gc = w.off_ce = off;
+    w.boundary = tensor_chain_shape(d);
+    w.off_kp = w.off_qb = w.off_gc = w.off_ce = off;
     if (w.boundary) {
-        w.off_kb = off;
+        w.off_kp = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
         w.off_qb = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 4 * N * 4);
@@ -275,7 +293,7 @@ void ssm_desc_set_contiguous(ssm_desc_t *d) {
 
 size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
     if (validate_desc(d) != SSM_OK) return 0;
-    if (pass == SSM_PASS_FWD) return 0;
+    if (pass == SSM_PASS_FWD) return (d->batch == 0 || d->seqlen == 0) ? 0 : fwd_layout(d).total;
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
     return bwd_layout(d).total;
@@ -288,8 +306,6 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
                  void *stream) {
     int rc = validate_desc(d);
     if (rc) return rc;
-    (void)workspace;
-    (void)workspace_bytes;
     if (d->batch == 0) return SSM_OK;
     if (d->seqlen > 0) {
         if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
@@ -300,11 +316,22 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
     p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
     // chunk == 1 asks for the token-by-token recurrent kernels
-    const bool chunked = d->chunk != 1 && ssm::chunk_fwd_supported(p);
+    const bool chunked = d->chunk != 1 && ssm::chunk_fwd_supported(p) && tensor_chain_shape(d);
     if (!chunked && !ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
     cudaStream_t st = (cudaStream_t)stream;
+    if (chunked) {
+        const FwdWs lay = fwd_layout(d);
+        if (!workspace || workspace_bytes < lay.total)
+            return fail(SSM_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu",
+                        lay.total, workspace ? workspace_bytes : (size_t)0);
+        if ((uintptr_t)workspace % 256)
+            return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+        p.ws_kp = (float *)((char *)workspace + lay.off_kp);
+        p.ws_ce = (float *)((char *)workspace + lay.off_ce);
+        p.nc = (int)((d->seqlen + 63) / 64);
+    }
     profile_begin(st);
     cudaError_t e = cudaSuccess;
     if (chunked) {
@@ -404,7 +431,7 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         e = gate_slot(&gate, st);
         if (e == cudaSuccess) e = ssm::chunk_range_check(p, gate, st);
         ssm::Params pc = p;
-        pc.ws_kb = (float *)(ws + lay.off_kb);
+        pc.ws_kp = (float *)(ws + lay.off_kp);
         pc.ws_qb = (float *)(ws + lay.off_qb);
         pc.ws_gc = (float *)(ws + lay.off_gc);
         pc.ws_ce = (float *)(ws + lay.off_ce);

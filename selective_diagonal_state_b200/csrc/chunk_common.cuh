@@ -95,6 +95,133 @@ __device__ __forceinline__ void cmul(float a, float b, float c, float d, float &
     im = fmaf(a, d, b * c);
 }
 
+// ---- per-chunk token quantities and mode constants ----------------------------
+// Loads dt / lambda of tokens t0 .. t0+64 and writes the inclusive prefix S_t
+// (F_S) and, with `want_sigma`, sigma_t (F_SIG) and beta_{t+1} (F_BN).
+// Call with all threads of the block (>= 96); contains barriers.
+__device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b, int h, int t0,
+                                             bool want_sigma) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < Q + 1; i += blockDim.x) {
+        const int t = t0 + i;
+        float dv = 0.f, lv = 1.f;
+        if (t < p.L) {
+            dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+            if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+        }
+        f32[F_DT + i] = dv;
+        f32[F_LAM + i] = lv;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
+        float v = d0 + d1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        f32[F_S + 2 * lane] = v - d1;
+        f32[F_S + 2 * lane + 1] = v;
+    } else if (want_sigma && (warp == 1 || warp == 2)) {
+        const int t = (warp - 1) * 32 + lane;
+        const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
+        const float bn =
+            (t0 + t + 1 < p.L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
+        f32[F_SIG + t] = fmaf(lv, dv, bn);
+        f32[F_BN + t] = bn;
+    }
+    __syncthreads();
+}
+
+// Per-mode decay over each sub-block, E_k = e^{lam dS_k}, and the products
+// F[i][j] = prod_{k=i}^{j-1} E_k and G_i = conj(F[0][i]) into the F_KRE / F_KIM
+// slots.  Needs F_S, F_A2, F_W.  Ends with a barrier.
+__device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
+    const int nmode = p.nr + p.np;
+    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
+        const float a2 = f32[F_A2 + m], w = f32[F_W + m];
+        float er[4], ei[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
+            const float ds = f32[F_S + 16 * k + 15] - lo;
+            const float mag = exp2f(a2 * ds);
+            if (m >= p.nr) {
+                float sn, cs;
+                sincosf(w * ds, &sn, &cs);
+                er[k] = mag * cs;
+                ei[k] = mag * sn;
+            } else {
+                er[k] = mag;
+                ei[k] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float pr = 1.f, pi = 0.f;
+#pragma unroll
+            for (int j = i + 1; j <= 4; ++j) {
+                float nr_, ni_;
+                cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
+                pr = nr_;
+                pi = ni_;
+                f32[F_KRE + fslot(i, j) * NP + m] = pr;
+                f32[F_KIM + fslot(i, j) * NP + m] = pi;
+                if (i == 0 && j < 4) {
+                    f32[F_KRE + gslot(j) * NP + m] = pr;
+                    f32[F_KIM + gslot(j) * NP + m] = -pi;
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void mode_rates(const Params &p, float *f32, int h) {
+    const int nmode = p.nr + p.np;
+    for (int m = threadIdx.x; m < NP; m += blockDim.x) {
+        float a2 = 0.f, w = 0.f;
+        if (m < nmode) {
+            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
+            if (m >= p.nr) w = p.theta[h * p.np + (m - p.nr)];
+        }
+        f32[F_A2 + m] = a2;
+        f32[F_W + m] = w;
+    }
+}
+
+__device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {
+    return ((long long)b * p.H + h) * p.nc + c;
+}
+
+// fp32 state-shaped tile [n][64 p] (row stride 64; rows from N on read as 0)
+// -> bf16 operand tile with byte(n, p) = (n/8)*1024 + (p/8)*128 + (n%8)*16 +
+// (p%8)*2, which is both the K-major layout with rows n (K = p) and the
+// MN-major layout with M or N = p (K = n).  With `lo`, the bf16 residual goes
+// to the second tile.  Strided over the block's threads; no barrier.
+__device__ __forceinline__ void load_state_tile(const float *src, int N, unsigned char *hi,
+                                                unsigned char *lo) {
+    for (int it = threadIdx.x; it < NP * (PD / 8); it += blockDim.x) {
+        const int n = it >> 3, p8 = (it & 7) * 8;
+        float v[8];
+        if (n < N) {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8));
+            const float4 d = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8 + 4));
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+        }
+        const uint32_t off = off_kmaj(n, p8, 128u, 1024u);
+        if (lo)
+            st16_split(hi, lo, off, v);
+        else
+            st16(hi, off, v);
+    }
+}
+
 // ---- host side ---------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

@@ -37,8 +37,9 @@ struct Params {
     float *ws_ddt;  // [B][L][H]         local decay part of ddt (within a time block)
     float *ws_blk;  // [B][H][NTB][4 nmode + 2]  per time block: totals and local sums
     float *ws_blkc; // [B][H][NTB]       ddt offset of each time block (carried part)
-    // exact decay-gradient carries at 64-token chunk boundaries (tensor-core path):
-    float *ws_kb;   // [B][H][NC][N][P]  pre-state K at the end of every chunk but the last
+    // chunk states and exact decay-gradient carries at 64-token chunk boundaries
+    // (tensor-core chain; the forward uses ws_kp and ws_ce):
+    float *ws_kp;   // [B][H][NC][N][P]  pre-state K entering every chunk (K_{-1} = h0 + beta_0 w0)
     float *ws_qb;   // [B][H][NC][4][N]  per-row sum_p conj(Gbar) A K_prev at chunk starts (per warp of p)
     float *ws_gc;   // [B][H][NC][N][P]  chunk-local adjoint, then the adjoint carried into each chunk
     float *ws_ce;   // [B][H][NC][128][2] full-chunk decay e^{lam S_63} per mode (re, im)

@@ -1,5 +1,5 @@
-// Chunked tensor-core forward scan for sm_100a (bf16 I/O, fp32 state, SISO,
-// head dim 64, up to 128 state rows).
+// Chunk-parallel tensor-core forward scan for sm_100a (bf16 I/O, fp32 state,
+// SISO, head dim 64, 64 or 128 state rows).
 //
 // The state-mediated kernel of the scan is masked linear attention ("When a
 // Diagonal State Is Not Enough", sungsoo.github.io Part 03, Thm 24): within a
@@ -10,7 +10,7 @@
 //     Phi_{t,s} = exp(lam (S_t - S_ref)) exp(lam (S_ref - S_s)),  lam = a + i theta
 // (the fixed-basis diagonal structure of Thm 8).  References are the starts of
 // 16-token sub-blocks, so every folded factor either decays (|f| <= 1) or
-// grows at most by exp(|a| * sum of 16 steps).
+// grows at most by exp(|a| * sum of 16 steps) (see k_range_check).
 //
 // Per chunk of Q = 64 tokens (sub-blocks i = 0..3 of 16), S_t = inclusive sum of
 // dt over the chunk, Sb_i = S at the end of sub-block i-1:
@@ -18,25 +18,27 @@
 //   Ch_t  = c_t conj(e^{lam S_t})                     readout of the carried state
 //   Bi_s  = sigma_s b_s e^{lam (Sb_i - S_s)}          for s <= end of block i
 //   Bh_s  = sigma_s b_s e^{lam (S_63 - S_s)}          chunk-end state contribution
-// and, on the tensor cores (tcgen05, fp32 accumulators in TMEM):
-//   scores^T_i  = Bi (64 s x N) . Ci^T (N x 16 t)          M=64, N=16, K=N
-//   Y^T         = K_prev^T (64 p x N) . Ch^T (N x 64 t)    M=64, N=64, K=N
-//               + X^T (64 p x s) . P^T_i (s x 16 t)        masked scores, M=64, N=16
-//   S_chunk     = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64, K=64
-// while the carried state K_c = e^{lam S_63} K_{c-1} + S_chunk runs in fp32
-// registers (one state row per thread).  The two-endpoint write is used in the
-// pre-state form K_t = A_t K_{t-1} + sigma_t W_t, sigma_t = gamma_t + beta_{t+1},
-// with y_t = C_t K_t - beta_{t+1} (C_t . B_t) u_t + D u_t.
+// The two-endpoint write is used in the pre-state form
+// K_t = A_t K_{t-1} + sigma_t W_t, sigma_t = gamma_t + beta_{t+1}, with
+// y_t = C_t K_t - beta_{t+1} (C_t . B_t) u_t + D u_t.  Three kernels:
+//   k_chunk_state_local (every chunk at once)  S_c = Bh^T (N x 64 s) . X   M=128, N=64
+//   k_chunk_state_pass  (chunks in order, elementwise over (row pair, p))
+//                        K_c = e^{lam S_63} K_{c-1} + S_c; stores the state
+//                        entering every chunk, hT and the last write
+//   k_chunk_out         (every chunk at once)
+//       scores^T_i  = Bi (64 s x N) . Ci^T (N x 16 t)          M=64, N=16, K=N
+//       Y^T         = K_prev^T (64 p x N) . Ch^T (N x 64 t)    M=64, N=64, K=N
+//                   + X^T (64 p x s) . P^T_i (s x 16 t)        masked scores, M=64, N=16
 #include <cuda.h>
 
-#include "common.cuh"
 #include "chunk_common.cuh"
+#include "common.cuh"
 #include "umma.cuh"
 
 namespace ssm {
 
 // Device word raised by the bounded waits of the tensor-core kernels
-// (0 = no error; 1 = a wait gave up; 2 = an input outside the folding range).
+// (0 = no error; 1 = a wait gave up).
 __device__ int ssm_chunk_error_word;
 __device__ __forceinline__ void raise_error(int code) { atomicCAS(&ssm_chunk_error_word, 0, code); }
 
@@ -45,222 +47,352 @@ namespace chunkfwd {
 using namespace umma;
 using namespace chunkc;
 
+// ============================================================================
+// k_chunk_state_local: chunk-local end state S_c = Bh^T X (Bh split hi + lo, so
+// the state keeps about 16 mantissa bits for the decay gradients), and the
+// chunk's full decay e^{lam S_63} per mode.
+// ============================================================================
+namespace stl {
+constexpr int THREADS = 128;
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint32_t SM_B = 0;        // 16 KB raw B (two 64-row 128B-swizzled halves)
+constexpr uint32_t SM_X = 16384;    // 8 KB  x (128B swizzle)
+constexpr uint32_t SM_BH = 24576;   // 16 KB Bh hi, MN-major (M = state rows, K = s)
+constexpr uint32_t SM_BHL = 40960;  // 16 KB Bh lo
+constexpr uint32_t SM_F32 = 57344;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace stl
+
+__global__ void __launch_bounds__(stl::THREADS)
+k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                    Params p) {
+    if (gated_off(p)) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + stl::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + stl::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, nmode = p.nr + p.np;
+    const int t0 = c * Q;
+    const int nbox = N / 64;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + Q * N * 2));
+        tma_load_4d(sm + stl::SM_X, &tmX, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k)
+            tma_load_4d(sm + stl::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+    }
+    if (warp == 0) tmem_alloc(tslot, stl::TMEM_COLS);
+    mode_rates(p, f32, h);
+    chunk_tokens(p, f32, b, h, t0, true);
+    chunk_mode_constants(p, f32);
+    for (int m = tid; m < nmode; m += stl::THREADS) {
+        float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
+        ce[2 * m] = f32[F_KRE + fslot(0, 4) * NP + m];
+        ce[2 * m + 1] = f32[F_KIM + fslot(0, 4) * NP + m];
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tacc = *tslot;
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // Bh = (own-sub-block Bi) F[ib][4]; thread (t, grp) handles rows 8 (grp + 2k)
+        const int t = tid & 63, grp = tid >> 6;
+        const int ib = t >> 4;
+        const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+        const float ds = f32[F_S + t] - Sb;
+        const float sig = f32[F_SIG + t];
+        const unsigned char *sB = sm + stl::SM_B;
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k) {
+            const int r0 = 8 * (grp + 2 * k);
+            if (r0 >= N) break;
+            float rb[8], v[8];
+            ld_rows8(sB, t, r0, rb);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const int r = r0 + j;
+                if (r < nr) {
+                    v[j] = sig * rb[j] * ex2_fast(fminf(-f32[F_A2 + r] * ds, 120.f)) *
+                           f32[F_KRE + fslot(ib, 4) * NP + r];
+                    v[j + 1] = sig * rb[j + 1] * ex2_fast(fminf(-f32[F_A2 + r + 1] * ds, 120.f)) *
+                               f32[F_KRE + fslot(ib, 4) * NP + r + 1];
+                } else {
+                    const int m = nr + ((r - nr) >> 1);
+                    float sn, cs;
+                    __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                    const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m] * ds, 120.f));
+                    const float bi0 = eb * fmaf(rb[j], cs, rb[j + 1] * sn);
+                    const float bi1 = eb * fmaf(rb[j + 1], cs, -rb[j] * sn);
+                    cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m],
+                         f32[F_KIM + fslot(ib, 4) * NP + m], v[j], v[j + 1]);
+                }
+            }
+            st16_split(sm + stl::SM_BH, sm + stl::SM_BHL, off_mnmaj(r0, t, 2048u, 128u), v);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sm + stl::SM_X);
+            const uint32_t id = idesc_bf16(128, 64, true, true);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t bh_base = smem_u32(sm + (part ? stl::SM_BHL : stl::SM_BH));
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(tacc, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                             sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id,
+                             part > 0 || s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            const int n = tid;
+            float *dst = p.ws_kp + (bhc(p, b, h, c) * N + n) * PD;
+#pragma unroll
+            for (int c16 = 0; c16 < PD / 16; ++c16) {
+                float v[16];
+                tmem_ld16(tmem_addr(tacc, 32u * warp, 16u * c16), v);
+                if (n < N) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        reinterpret_cast<float4 *>(dst + 16 * c16)[q4] =
+                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);  // let an in-flight load land before exit
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tacc, stl::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// k_chunk_state_pass: the carried state over the chunks of one (batch row,
+// head).  Thread (row-pair group, 4 consecutive p) keeps rows 2rp, 2rp+1 for
+// rp = rp0, rp0 + 16, ...: two real modes or one rotation pair as (re, im).
+// Every chunk's loads are issued together (16-byte rows), so that enough bytes
+// are in flight to stream at HBM speed.  ws_kp[c] holds S_c on entry and the
+// state entering chunk c on exit; the state after the last chunk is hT.
+// ============================================================================
+namespace pas {
 constexpr int THREADS = 256;
-constexpr uint32_t TMEM_COLS = 128;
+constexpr int KMAX = NP / 32;   // row pairs per thread
+}  // namespace pas
 
-// shared-memory map (bytes from a 1024-aligned base)
-constexpr uint32_t SM_X = 0;              // 2 x 8 KB   x tiles (128B-swizzled, rows = t)
-constexpr uint32_t SM_B = 16384;          // 2 x 16 KB  raw B tiles: 2 x (64 t x 64 rows), 128B-swizzled
-constexpr uint32_t SM_C = 49152;          // 2 x 16 KB  raw C tiles, same layout
-constexpr uint32_t SM_CI = 81920;         // 16 KB      Ci   K-major (64 t x 128)
-constexpr uint32_t SM_CH = 98304;         // 16 KB      Ch   K-major
-constexpr uint32_t SM_BI = 114688;        // 40 KB      Bi tiles (16, 32, 48, 64 rows)
-constexpr uint32_t SM_BH = 155648;        // 16 KB      Bh   MN-major (M = 128 rows, K = 64 t)
-constexpr uint32_t SM_P = 172032;         // 8 KB       P^T tiles, MN-major (N = 16 t, K = 64 s)
-constexpr uint32_t SM_KT = 180224;        // 16 KB      K_prev^T MN-major (M = 64 p, K = 128 rows)
-constexpr uint32_t SM_F32 = 196608;       // fp32 scratch
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;   // 4 mbarriers + TMEM slot + flags
-constexpr uint32_t SMEM_USED = SM_BAR + 64;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+__global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
+    if (gated_off(p)) return;
+    __shared__ float s_ce[3][2 * NP];   // chunk decays, triple-buffered
+    const int tid = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int N = p.N, nr = p.nr, nc = p.nc;
+    const int q = 4 * (tid & 15), rp0 = tid >> 4;
+    const int nk = N / 32;
+    // K_{-1} = h0 + beta_0 w0
+    float beta0 = 0.f;
+    if (p.two_ep)
+        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+    float4 k0[pas::KMAX], k1[pas::KMAX];
+#pragma unroll
+    for (int k = 0; k < pas::KMAX; ++k) {
+        float a[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+        if (k < nk) {
+            const int n0 = 2 * (rp0 + 16 * k);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+                if (p.h0) {
+                    a[j] = p.h0[i0];
+                    d[j] = p.h0[i1];
+                }
+                if (p.w0) {
+                    a[j] = fmaf(beta0, p.w0[i0], a[j]);
+                    d[j] = fmaf(beta0, p.w0[i1], d[j]);
+                }
+            }
+        }
+        k0[k] = make_float4(a[0], a[1], a[2], a[3]);
+        k1[k] = make_float4(d[0], d[1], d[2], d[3]);
+    }
+    s_ce[0][tid] = __ldg(p.ws_ce + bhc(p, b, h, 0) * (2 * NP) + tid);
+    for (int c = 0; c < nc; ++c) {
+        float *sbase = p.ws_kp + bhc(p, b, h, c) * N * PD + q;
+        float4 sv0[pas::KMAX], sv1[pas::KMAX];
+#pragma unroll
+        for (int k = 0; k < pas::KMAX; ++k) {
+            if (k < nk) {
+                const int n0 = 2 * (rp0 + 16 * k);
+                sv0[k] = *reinterpret_cast<const float4 *>(sbase + (long long)n0 * PD);
+                sv1[k] = *reinterpret_cast<const float4 *>(sbase + (long long)(n0 + 1) * PD);
+            }
+        }
+        if (c + 1 < nc) s_ce[(c + 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c + 1) * (2 * NP) + tid);
+        __syncthreads();
+        const float *ce = s_ce[c % 3];
+#pragma unroll
+        for (int k = 0; k < pas::KMAX; ++k) {
+            if (k >= nk) break;
+            const int n0 = 2 * (rp0 + 16 * k);
+            *reinterpret_cast<float4 *>(sbase + (long long)n0 * PD) = k0[k];
+            *reinterpret_cast<float4 *>(sbase + (long long)(n0 + 1) * PD) = k1[k];
+            float4 &a = k0[k], &d = k1[k];
+            if (n0 < nr) {
+                const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
+                a.x = fmaf(e0, a.x, sv0[k].x); a.y = fmaf(e0, a.y, sv0[k].y);
+                a.z = fmaf(e0, a.z, sv0[k].z); a.w = fmaf(e0, a.w, sv0[k].w);
+                d.x = fmaf(e1, d.x, sv1[k].x); d.y = fmaf(e1, d.y, sv1[k].y);
+                d.z = fmaf(e1, d.z, sv1[k].z); d.w = fmaf(e1, d.w, sv1[k].w);
+            } else {
+                const int m = nr + ((n0 - nr) >> 1);
+                const float er = ce[2 * m], ei = ce[2 * m + 1];
+                // (er + i ei) (a + i d) + S
+                const float4 ao = a;
+                a.x = fmaf(er, ao.x, fmaf(-ei, d.x, sv0[k].x));
+                a.y = fmaf(er, ao.y, fmaf(-ei, d.y, sv0[k].y));
+                a.z = fmaf(er, ao.z, fmaf(-ei, d.z, sv0[k].z));
+                a.w = fmaf(er, ao.w, fmaf(-ei, d.w, sv0[k].w));
+                d.x = fmaf(er, d.x, fmaf(ei, ao.x, sv1[k].x));
+                d.y = fmaf(er, d.y, fmaf(ei, ao.y, sv1[k].y));
+                d.z = fmaf(er, d.z, fmaf(ei, ao.z, sv1[k].z));
+                d.w = fmaf(er, d.w, fmaf(ei, ao.w, sv1[k].w));
+            }
+        }
+    }
+    // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write B_{L-1} u_{L-1}
+    const int g = h / p.hpg, tl = p.L - 1;
+#pragma unroll
+    for (int k = 0; k < pas::KMAX; ++k) {
+        if (k >= nk) break;
+        const int n0 = 2 * (rp0 + 16 * k);
+        const float a[4] = {k0[k].x, k0[k].y, k0[k].z, k0[k].w};
+        const float d[4] = {k1[k].x, k1[k].y, k1[k].z, k1[k].w};
+        const float b0 = p.wT ? ld_io(p.Bm, ix_B(p, b, tl, g, 0, n0), 1) : 0.f;
+        const float b1 = p.wT ? ld_io(p.Bm, ix_B(p, b, tl, g, 0, n0 + 1), 1) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+            if (p.hT) {
+                p.hT[i0] = a[j];
+                p.hT[i1] = d[j];
+            }
+            if (p.wT) {
+                const float ul = ld_io(p.x, ix_x(p, b, tl, h, 0, q + j), 1);
+                p.wT[i0] = b0 * ul;
+                p.wT[i1] = b1 * ul;
+            }
+        }
+    }
+}
 
-__global__ void __launch_bounds__(THREADS, 1)
-k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+// ============================================================================
+// k_chunk_out: per chunk, y_t = readout of the state entering the chunk
+// + masked in-chunk scores x + (D - beta_{t+1} C_t . B_t) u_t.
+// ============================================================================
+namespace outk {
+constexpr int THREADS = 512;
+constexpr int RG = THREADS / 64;   // row groups of the operand preparation
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle, rows = t)
+constexpr uint32_t SM_B = 8192;       // 16 KB raw B (two 64-row swizzled halves)
+constexpr uint32_t SM_C = 24576;      // 16 KB raw C
+constexpr uint32_t SM_CI = 40960;     // 16 KB Ci   K-major (64 t x 128)
+constexpr uint32_t SM_CH = 57344;     // 16 KB Ch   K-major
+constexpr uint32_t SM_BI = 73728;     // 40 KB Bi tiles (16, 32, 48, 64 rows)
+constexpr uint32_t SM_P = 114688;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
+constexpr uint32_t SM_KT = 122880;    // 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
+constexpr uint32_t SM_F32 = 139264;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace outk
+
+__global__ void __launch_bounds__(outk::THREADS, 1)
+k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, Params p) {
     if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // [2]
-    uint64_t *bar_mma = bar_tma + 2;                                // [2]: phase A, phase B
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
-    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
+    float *f32 = reinterpret_cast<float *>(sm + outk::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + outk::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;   // [2]: phase A, phase B
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / p.hpg;
     const int N = p.N, nr = p.nr, L = p.L;
-    const int nmode = p.nr + p.np;
-    const int nchunk = (L + Q - 1) / Q;
-    const uint32_t tile_bytes = Q * PD * 2 + 2u * Q * N * 2;
-    const int nbox = N / 64;   // 64-row TMA boxes per B/C tile
+    const int t0 = c * Q;
+    const int nbox = N / 64;
 
-    // ---- set-up ------------------------------------------------------------
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
+        mbar_init(bar_tma, 1);
         mbar_init(&bar_mma[0], 1);
         mbar_init(&bar_mma[1], 1);
         mbar_fence_init();
-        *abort_flag = 0;
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-    }
-    if (warp == 0) tmem_alloc(tslot, TMEM_COLS);
-    for (int m = tid; m < NP; m += THREADS) {
-        float a2 = 0.f, w = 0.f;
-        if (m < nmode) {
-            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
-            if (m >= nr) w = p.theta[h * p.np + (m - nr)];
+        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + 2 * Q * N * 2));
+        tma_load_4d(sm + outk::SM_X, &tmX, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_4d(sm + outk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+            tma_load_4d(sm + outk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
         }
-        f32[F_A2 + m] = a2;
-        f32[F_W + m] = w;
     }
-    // padding rows of every operand stay zero
-    for (int i = tid; i < (int)((SM_F32 - SM_CI) / 16); i += THREADS)
-        reinterpret_cast<uint4 *>(sm + SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    if (warp == 0) tmem_alloc(tslot, outk::TMEM_COLS);
+    mode_rates(p, f32, h);
+    if (N < NP)  // K padding of Ci, Ch, Bi
+        for (int i = tid; i < (int)((outk::SM_P - outk::SM_CI) / 16); i += outk::THREADS)
+            reinterpret_cast<uint4 *>(sm + outk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    load_state_tile(p.ws_kp + bhc(p, b, h, c) * N * PD, N, sm + outk::SM_KT, nullptr);
+    chunk_tokens(p, f32, b, h, t0, true);
+    chunk_mode_constants(p, f32);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_y = tbase;                      // Y^T (M=64, lanes 0-15 of each quarter)
     const uint32_t t_sc = tbase + (16u << 16);       // scores^T (M=64, lanes 16-31)
-    const uint32_t t_st = tbase + 64u;               // chunk state (M=128), columns 64..127
-
-    // TMA for the first two chunks
-    if (tid == 0) {
-        for (int c = 0; c < 2 && c < nchunk; ++c) {
-            mbar_expect_tx(&bar_tma[c], tile_bytes);
-            tma_load_4d(sm + SM_X + c * 8192, &tmX, &bar_tma[c], 0, h, c * Q, b);
-            for (int k = 0; k < nbox; ++k) {
-                tma_load_4d(sm + SM_B + c * 16384 + k * 8192, &tmB, &bar_tma[c], 64 * k, g, c * Q, b);
-                tma_load_4d(sm + SM_C + c * 16384 + k * 8192, &tmC, &bar_tma[c], 64 * k, g, c * Q, b);
-            }
-        }
-    }
-
-    // carried state: thread n < 128 owns state row n (64 p values, fp32)
-    float K[PD];
-    const bool chain_thr = tid < NP;
-    {
-        float beta0 = 0.f;
-        if (p.two_ep && L > 0)
-            beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
-        if (chain_thr) {
-            const int n = tid;
-#pragma unroll
-            for (int q = 0; q < PD; ++q) {
-                float v = 0.f;
-                if (n < N) {
-                    if (p.h0) v = p.h0[ix_st(p, b, h, n, q)];
-                    if (p.w0) v = fmaf(beta0, p.w0[ix_st(p, b, h, n, q)], v);
-                }
-                K[q] = v;
-            }
-            // K_prev^T operand (bf16, MN-major: M = p, K = row)
-#pragma unroll
-            for (int q8 = 0; q8 < PD / 8; ++q8) {
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
-                st16(sm + SM_KT, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
-            }
-        }
-    }
-
-    const float Dh = (p.R == p.O) ? p.D[h] : 0.f;
-    const int t_loc = tid & 63;     // token of this thread in the prep phase
-    const int grp = tid >> 6;       // row-chunk group of this thread (rows 8*(grp + 4k) ..)
-
-    for (int c = 0; c < nchunk; ++c) {
-        const int st = c & 1;
-        const int t0 = c * Q;
-        unsigned char *sX = sm + SM_X + st * 8192;
-        unsigned char *sB = sm + SM_B + st * 16384;
-        unsigned char *sC = sm + SM_C + st * 16384;
-
-        // ---- per-token quantities --------------------------------------------
-        for (int i = tid; i < Q + 1; i += THREADS) {
-            const int t = t0 + i;
-            float dv = 0.f, lv = 1.f;
-            if (t < L) {
-                dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
-                if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
-            }
-            f32[F_DT + i] = dv;
-            f32[F_LAM + i] = lv;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // inclusive prefix sum of dt over the chunk (two tokens per lane)
-            const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
-            float v = d0 + d1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            f32[F_S + 2 * lane] = v - d1;
-            f32[F_S + 2 * lane + 1] = v;
-        } else if (warp == 1 || warp == 2) {
-            const int t = (warp - 1) * 32 + lane;
-            const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
-            const float bn = (t0 + t + 1 < L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
-            f32[F_SIG + t] = fmaf(lv, dv, bn);
-            f32[F_BN + t] = bn;
-        }
-        // ---- wait for the chunk's tiles ---------------------------------------
-        if (!mbar_wait(&bar_tma[st], (uint32_t)((c >> 1) & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
-        __syncthreads();
-        if (*abort_flag) break;
-
-        // ---- per-mode chunk constants: E_k = exp(lam dS_k), their products -----
-        for (int m = tid; m < nmode; m += THREADS) {
-            const float a2 = f32[F_A2 + m], w = f32[F_W + m];
-            float er[4], ei[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
-                const float ds = f32[F_S + 16 * k + 15] - lo;
-                const float mag = exp2f(a2 * ds);
-                if (m >= nr) {
-                    float sn, cs;
-                    sincosf(w * ds, &sn, &cs);
-                    er[k] = mag * cs;
-                    ei[k] = mag * sn;
-                } else {
-                    er[k] = mag;
-                    ei[k] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float pr = 1.f, pi = 0.f;
-#pragma unroll
-                for (int j = i + 1; j <= 4; ++j) {
-                    float nr_, ni_;
-                    cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
-                    pr = nr_;
-                    pi = ni_;
-                    f32[F_KRE + fslot(i, j) * NP + m] = pr;
-                    f32[F_KIM + fslot(i, j) * NP + m] = pi;
-                    if (i == 0 && j < 4) {
-                        f32[F_KRE + gslot(j) * NP + m] = pr;
-                        f32[F_KIM + gslot(j) * NP + m] = -pi;
-                    }
-                }
-            }
-        }
-        __syncthreads();
-
-        // ---- operand preparation: thread (t, grp) handles rows 8*(grp + 4k) ---
+    float *cpart = reinterpret_cast<float *>(sm + outk::SM_P);   // C.B partials until P is built
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // ---- operand preparation: thread (t, grp) handles rows 8 (grp + RG k) ---
         {
-            const int t = t_loc;
+            const int t = tid & 63, grp = tid >> 6;
             const int ib = t >> 4;
-            const float St = f32[F_S + t];
             const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-            const float ds = St - Sb;
+            const float ds = f32[F_S + t] - Sb;
             const float sig = f32[F_SIG + t];
+            const unsigned char *sB = sm + outk::SM_B, *sC = sm + outk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
-            for (int k = 0; k < 4; ++k) {
-                const int r0 = 8 * (grp + 4 * k);
+            for (int k = 0; k < NP / (8 * outk::RG); ++k) {
+                const int r0 = 8 * (grp + outk::RG * k);
                 if (r0 >= N) break;
-                float vCI[8], vCH[8], vBI[8], vBH[8], vBX[3][8], rc[8], rb[8];
+                float vCI[8], vCH[8], vBI[8], vBX[3][8], rc[8], rb[8];
                 ld_rows8(sC, t, r0, rc);
                 ld_rows8(sB, t, r0, rb);
 #pragma unroll
@@ -270,90 +402,79 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                     const float c0 = rc[j], c1 = rc[j + 1];
                     const float b0 = rb[j], b1 = rb[j + 1];
                     corr = fmaf(c0, b0, fmaf(c1, b1, corr));
-                    float ci0, ci1, bi0, bi1;     // folded Ci, own-block Bi
-                    int m0, m1;
-                    bool pair;
                     if (r < nr) {
-                        pair = false;
-                        m0 = r;
-                        m1 = r + 1;
+                        const int m0 = r, m1 = r + 1;
                         const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
-                        ci0 = c0 * ex2_fast(x0);
-                        ci1 = c1 * ex2_fast(x1);
-                        bi0 = sig * b0 * ex2_fast(fminf(-x0, 120.f));
-                        bi1 = sig * b1 * ex2_fast(fminf(-x1, 120.f));
-                    } else {
-                        pair = true;
-                        m0 = m1 = nr + ((r - nr) >> 1);
-                        const float x = f32[F_A2 + m0] * ds;
-                        float sn, cs;
-                        __sincosf(f32[F_W + m0] * ds, &sn, &cs);
-                        // rotate by cis(-phi): (u + iv)(cs - i sn)
-                        const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
-                        ci0 = ec * fmaf(c0, cs, c1 * sn);
-                        ci1 = ec * fmaf(c1, cs, -c0 * sn);
-                        bi0 = eb * fmaf(b0, cs, b1 * sn);
-                        bi1 = eb * fmaf(b1, cs, -b0 * sn);
-                    }
-                    vCI[j] = ci0;
-                    vCI[j + 1] = ci1;
-                    vBI[j] = bi0;
-                    vBI[j + 1] = bi1;
-                    // Ch = Ci * G_ib ; other Bi = own Bi * F[ib][i'] ; Bh = own Bi * F[ib][4]
-                    if (!pair) {
+                        const float ci0 = c0 * ex2_fast(x0), ci1 = c1 * ex2_fast(x1);
+                        const float bi0 = sig * b0 * ex2_fast(fminf(-x0, 120.f));
+                        const float bi1 = sig * b1 * ex2_fast(fminf(-x1, 120.f));
+                        vCI[j] = ci0;
+                        vCI[j + 1] = ci1;
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
                         const float g0 = ib ? f32[F_KRE + gslot(ib) * NP + m0] : 1.f;
                         const float g1 = ib ? f32[F_KRE + gslot(ib) * NP + m1] : 1.f;
                         vCH[j] = ci0 * g0;
                         vCH[j + 1] = ci1 * g1;
-                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
-                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
 #pragma unroll
-                        for (int q = 0; q < 3; ++q) {
-                            const int i2 = ib + 1 + q;
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
                             if (i2 < 4) {
-                                vBX[q][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
-                                vBX[q][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                                vBX[qq][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
+                                vBX[qq][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
                             }
                         }
                     } else {
+                        const int m = nr + ((r - nr) >> 1);
+                        const float x = f32[F_A2 + m] * ds;
+                        float sn, cs;
+                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        // rotate by cis(-phi): (u + iv)(cs - i sn)
+                        const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
+                        const float ci0 = ec * fmaf(c0, cs, c1 * sn);
+                        const float ci1 = ec * fmaf(c1, cs, -c0 * sn);
+                        const float bi0 = eb * fmaf(b0, cs, b1 * sn);
+                        const float bi1 = eb * fmaf(b1, cs, -b0 * sn);
+                        vCI[j] = ci0;
+                        vCI[j + 1] = ci1;
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
                         float gr = 1.f, gi = 0.f;
                         if (ib) {
-                            gr = f32[F_KRE + gslot(ib) * NP + m0];
-                            gi = f32[F_KIM + gslot(ib) * NP + m0];
+                            gr = f32[F_KRE + gslot(ib) * NP + m];
+                            gi = f32[F_KIM + gslot(ib) * NP + m];
                         }
                         cmul(ci0, ci1, gr, gi, vCH[j], vCH[j + 1]);
-                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m0],
-                             f32[F_KIM + fslot(ib, 4) * NP + m0], vBH[j], vBH[j + 1]);
 #pragma unroll
-                        for (int q = 0; q < 3; ++q) {
-                            const int i2 = ib + 1 + q;
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
                             if (i2 < 4)
-                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m0],
-                                     f32[F_KIM + fslot(ib, i2) * NP + m0], vBX[q][j],
-                                     vBX[q][j + 1]);
+                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m],
+                                     f32[F_KIM + fslot(ib, i2) * NP + m], vBX[qq][j],
+                                     vBX[qq][j + 1]);
                         }
                     }
                 }
-                st16(sm + SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
-                st16(sm + SM_CH, off_kmaj(t, r0, KM_LBO, KM_SBO), vCH);
-                st16(sm + SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+                st16(sm + outk::SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
+                st16(sm + outk::SM_CH, off_kmaj(t, r0, KM_LBO, KM_SBO), vCH);
+                st16(sm + outk::SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
 #pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const int i2 = ib + 1 + q;
-                    if (i2 < 4) st16(sm + SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[q]);
+                for (int qq = 0; qq < 3; ++qq) {
+                    const int i2 = ib + 1 + qq;
+                    if (i2 < 4)
+                        st16(sm + outk::SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
                 }
-                st16(sm + SM_BH, off_mnmaj(r0, t, 2048u, 128u), vBH);
             }
-            f32[F_CP + grp * 64 + t] = corr;
+            cpart[grp * 64 + t] = corr;
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
 
-        // ---- phase A: scores, chunk state, readout of the carried state --------
+        // ---- phase A: scores, readout of the carried state ---------------------
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t bi_base = smem_u32(sm + SM_BI), ci_base = smem_u32(sm + SM_CI);
+            const uint32_t bi_base = smem_u32(sm + outk::SM_BI), ci_base = smem_u32(sm + outk::SM_CI);
             const uint32_t id_sc = idesc_bf16(64, 16, false, false);
             for (int i = 0; i < NSB; ++i)
                 for (int s = 0; s < NP / 16; ++s)
@@ -361,12 +482,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              id_sc, s > 0);
-            const uint32_t bh_base = smem_u32(sm + SM_BH), x_base = smem_u32(sX);
-            const uint32_t id_st = idesc_bf16(128, 64, true, true);
-            for (int s = 0; s < Q / 16; ++s)
-                mma_bf16(t_st, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                         sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_st, s > 0);
-            const uint32_t kt_base = smem_u32(sm + SM_KT), ch_base = smem_u32(sm + SM_CH);
+            const uint32_t kt_base = smem_u32(sm + outk::SM_KT), ch_base = smem_u32(sm + outk::SM_CH);
             const uint32_t id_y = idesc_bf16(64, 64, true, false);
             for (int s = 0; s < NP / 16; ++s)
                 mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),
@@ -376,678 +492,92 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) cs += f32[F_CP + q * 64 + tid];
-            f32[F_CORR + tid] = -f32[F_BN + tid] * cs + Dh;
+            for (int k = 0; k < outk::RG; ++k) cs += cpart[k * 64 + tid];
+            f32[F_CORR + tid] = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
         }
-        if (!mbar_wait(&bar_mma[0], (uint32_t)(c & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
+        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) raise_error(1);
         fence_after_sync();
-        __syncthreads();
-        if (*abort_flag) break;
-
-        if (warp < 4) {
-            // ---- carried state: K_c = e^{lam S_63} K_{c-1} + S_chunk ------------
-            const int n = tid;
-            const int m = n < nr ? n : nr + ((n - nr) >> 1);
-            const bool pr_row = n >= nr && n < N;
-            const bool im_row = pr_row && ((n - nr) & 1);
-            float dr = 0.f, di = 0.f;
-            if (n < N) {
-                dr = f32[F_KRE + fslot(0, 4) * NP + m];
-                di = f32[F_KIM + fslot(0, 4) * NP + m];
-            }
+        if (__syncthreads_and(ok)) {
+            // ---- masked scores -> P^T tiles (one warp per TMEM lane quarter) -------
+            if (warp >= 4 && warp < 8) {
+                const int qd = warp - 4;
+                for (int i = 0; i < NSB; ++i) {
+                    float v[16];
+                    tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
+                    const int sl = lane - 16;
+                    if (sl >= 0) {
+                        const int s = 16 * qd + sl;
+                        if (s < 16 * (i + 1)) {
+                            float lo[8], hi[8];
 #pragma unroll
-            for (int c16 = 0; c16 < PD / 16; ++c16) {
-                float sv[16];
-                tmem_ld16(tmem_addr(t_st, 32u * warp, 16u * c16), sv);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int q = c16 * 16 + j;
-                    const float own = K[q];
-                    const float other = __shfl_xor_sync(0xffffffffu, own, 1);
-                    float nv;
-                    if (!pr_row)
-                        nv = fmaf(dr, own, sv[j]);
-                    else if (!im_row)  // re' = dr re - di im
-                        nv = fmaf(dr, own, fmaf(-di, other, sv[j]));
-                    else               // im' = di re + dr im
-                        nv = fmaf(di, other, fmaf(dr, own, sv[j]));
-                    K[q] = n < N ? nv : 0.f;
-                }
-            }
-#pragma unroll
-            for (int q8 = 0; q8 < PD / 8; ++q8) {
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
-                st16(sm + SM_KT, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
-            }
-        } else {
-            // ---- masked scores -> P^T tiles --------------------------------------
-            const int qd = warp - 4;
-            for (int i = 0; i < NSB; ++i) {
-                float v[16];
-                tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
-                const int sl = lane - 16;
-                if (sl >= 0) {
-                    const int s = 16 * qd + sl;
-                    if (s < 16 * (i + 1)) {
-                        float lo[8], hi[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
-                            hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
-                        }
-                        unsigned char *pt = sm + SM_P + i * 2048;
-                        st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
-                        st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
-                    }
-                }
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-
-        // ---- phase B: intra-chunk term Y^T += X^T P^T_i --------------------------
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + SM_P);
-            const uint32_t id_d = idesc_bf16(64, 16, true, true);
-            for (int i = 0; i < NSB; ++i)
-                for (int s = 0; s <= i; ++s)
-                    mma_bf16(t_y + 16 * i, sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128),
-                             sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
-                             true);
-            mma_commit(&bar_mma[1]);
-        }
-        if (!mbar_wait(&bar_mma[1], (uint32_t)(c & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
-        fence_after_sync();
-        __syncthreads();
-        if (*abort_flag) break;
-
-        // ---- epilogue: y_t[p] = Y^T[p][t] + (corr_t + D) u_t[p] -----------------
-        {
-            const int qd = warp & 3, half = warp >> 2;
-            const int pp = 16 * qd + (lane & 15);
-            __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
-                                  h * p.sy[2] + pp;
-            for (int c16 = 0; c16 < 2; ++c16) {
-                float v[16];
-                const int tc = 32 * half + 16 * c16;
-                tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
-                if (lane < 16) {
-                    __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = tc + j;
-                        if (t0 + t < L) {
-                            const float u = bf(sX + off_sw128(t, pp));
-                            *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
-                        }
-                        yp += p.sy[1];
-                    }
-                }
-            }
-        }
-        // last chunk: final state and last write
-        if (c == nchunk - 1 && chain_thr && tid < N) {
-            const int n = tid;
-            const int tl = (L - 1) - t0;
-            const float bl = ld_row1(sB, tl, n);
-#pragma unroll
-            for (int q = 0; q < PD; ++q) {
-                if (p.hT) p.hT[ix_st(p, b, h, n, q)] = K[q];
-                if (p.wT) p.wT[ix_st(p, b, h, n, q)] = bl * bf(sX + off_sw128(tl, q));
-            }
-        }
-        fence_before_sync();
-        __syncthreads();
-        // refill this stage with chunk c + 2
-        if (tid == 0 && c + 2 < nchunk) {
-            mbar_expect_tx(&bar_tma[st], tile_bytes);
-            tma_load_4d(sm + SM_X + st * 8192, &tmX, &bar_tma[st], 0, h, (c + 2) * Q, b);
-            for (int k = 0; k < nbox; ++k) {
-                tma_load_4d(sm + SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g,
-                            (c + 2) * Q, b);
-                tma_load_4d(sm + SM_C + st * 16384 + k * 8192, &tmC, &bar_tma[st], 64 * k, g,
-                            (c + 2) * Q, b);
-            }
-        }
-    }
-    // on abort: let in-flight loads land before the CTA's shared memory goes away
-    if (*abort_flag && tid == 0) {
-        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
-        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        fence_after_sync();
-        tmem_dealloc(tbase, TMEM_COLS);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Backward, forward-direction part: dC_t = dy_t H_t^T per head.
-//   H_t = K_t - beta_{t+1} W_t,   K_t = e^{lam S_t} K_prev + sum_{s<=t} Phi_{t,s} sigma_s b_s u_s
-// so, per state mode (complex for rotation pairs, real rows otherwise),
-//   dCK_t = e^{lam S_t} (dy_t . K_prev) + e^{lam (S_t - Sb_i)} sum_{s<=t} (dy_t . u_s) Bi_s
-// which is, on the tensor cores,
-//   V^T  = K_prev (N x 64 p) . dY^T (64 p x 64 t)          M=128, N=64, K=64
-//   G    = dY (64 t x 64 p) . X^T (64 p x 64 s)            M=64,  N=64, K=64
-//   D_i  = Bi^T (N x s) . (G o causal mask)_i^T (s x 16 t) M=128, N=16, K=16(i+1)
-// followed by the per-(t, row) unfolding of the decay factors on the CUDA
-// cores; dC_t = dCK_t - beta_{t+1} (dy_t . u_t) B_t.  The carried state is
-// recomputed exactly as in the forward (chunk-end state MMA + fp32 chain).
-// ---------------------------------------------------------------------------
-namespace chunkbwd {
-using namespace umma;
-using chunkfwd::Q;
-using chunkfwd::NSB;
-using chunkfwd::NP;
-using chunkfwd::PD;
-using chunkfwd::THREADS;
-using chunkfwd::WAIT_LIMIT;
-using chunkfwd::KM_LBO;
-using chunkfwd::KM_SBO;
-constexpr uint32_t TMEM_COLS = 256;
-// Operands that are rounded (folded B, chunk-end B, carried state, masked G)
-// are kept as bf16 pairs hi + lo (lo = v - hi) and every MMA on them runs as
-// hi*hi + hi*lo + lo*hi: about 16 mantissa bits, enough for the decay
-// gradients, which take differences of large sums of these products.
-constexpr uint32_t SM_X = 0;          // 2 x 8 KB   x tiles (128B swizzle)
-constexpr uint32_t SM_B = 16384;      // 2 x 16 KB  raw B tiles (two 64-row swizzled halves)
-constexpr uint32_t SM_DY = 49152;     // 2 x 8 KB   dy tiles (128B swizzle)
-constexpr uint32_t SM_BI = 65536;     // 40 KB      Bi tiles (hi)
-constexpr uint32_t SM_BIL = 106496;   // 40 KB      Bi tiles (lo)
-constexpr uint32_t SM_BH = 147456;    // 16 KB      Bh hi (MN-major, M = rows); masked G hi after phase A
-constexpr uint32_t SM_BHL = 163840;   // 16 KB      Bh lo;                       masked G lo after phase A
-constexpr uint32_t SM_GM = SM_BH;     // 8 KB + 8 KB masked G tiles hi | lo, K-major (N = 16 t, K = s)
-constexpr uint32_t SM_KT = 180224;    // 16 KB      K_prev hi (p-contiguous rows)
-constexpr uint32_t SM_KTL = 196608;   // 16 KB      K_prev lo
-constexpr uint32_t SM_F32 = 212992;
-constexpr uint32_t SM_BAR = SM_F32 + chunkfwd::F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
-}  // namespace chunkbwd
-
-__global__ void __launch_bounds__(chunkfwd::THREADS, 1)
-k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmDY, Params p) {
-    if (gated_off(p)) return;
-    using namespace chunkfwd;
-    using namespace umma;
-    namespace cb = chunkbwd;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + cb::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + cb::SM_BAR);
-    uint64_t *bar_mma = bar_tma + 2;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
-    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int g = h / p.hpg;
-    const int N = p.N, nr = p.nr, L = p.L;
-    const int nmode = p.nr + p.np;
-    const int nchunk = (L + Q - 1) / Q;
-    const int nbox = N / 64;
-    const uint32_t tile_bytes = 2u * Q * PD * 2 + (uint32_t)Q * N * 2;
-
-    if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(&bar_mma[0], 1);
-        mbar_init(&bar_mma[1], 1);
-        mbar_fence_init();
-        *abort_flag = 0;
-        tma_prefetch_desc(&tmX);
-        tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmDY);
-    }
-    if (warp == 0) tmem_alloc(tslot, cb::TMEM_COLS);
-    for (int m = tid; m < NP; m += THREADS) {
-        float a2 = 0.f, w = 0.f;
-        if (m < nmode) {
-            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
-            if (m >= nr) w = p.theta[h * p.np + (m - nr)];
-        }
-        f32[F_A2 + m] = a2;
-        f32[F_W + m] = w;
-    }
-    for (int i = tid; i < (int)((cb::SM_F32 - cb::SM_BI) / 16); i += THREADS)
-        reinterpret_cast<uint4 *>(sm + cb::SM_BI)[i] = make_uint4(0, 0, 0, 0);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tbase = *tslot;
-    const uint32_t t_st = tbase;          // chunk state (M=128), cols 0..63
-    const uint32_t t_v = tbase + 64u;     // V^T (M=128), cols 64..127
-    const uint32_t t_g = tbase + 128u;    // G (M=64, lanes 0-15 per quarter) then D_i (M=128)
-
-    if (tid == 0) {
-        for (int c = 0; c < 2 && c < nchunk; ++c) {
-            mbar_expect_tx(&bar_tma[c], tile_bytes);
-            tma_load_4d(sm + cb::SM_X + c * 8192, &tmX, &bar_tma[c], 0, h, c * Q, b);
-            tma_load_4d(sm + cb::SM_DY + c * 8192, &tmDY, &bar_tma[c], 0, h, c * Q, b);
-            for (int k = 0; k < nbox; ++k)
-                tma_load_4d(sm + cb::SM_B + c * 16384 + k * 8192, &tmB, &bar_tma[c], 64 * k, g,
-                            c * Q, b);
-        }
-    }
-
-    float K[PD];
-    const bool chain_thr = tid < NP;
-    {
-        float beta0 = 0.f;
-        if (p.two_ep && L > 0)
-            beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
-        if (chain_thr) {
-            const int n = tid;
-#pragma unroll
-            for (int q = 0; q < PD; ++q) {
-                float v = 0.f;
-                if (n < N) {
-                    if (p.h0) v = p.h0[ix_st(p, b, h, n, q)];
-                    if (p.w0) v = fmaf(beta0, p.w0[ix_st(p, b, h, n, q)], v);
-                }
-                K[q] = v;
-            }
-#pragma unroll
-            for (int q8 = 0; q8 < PD / 8; ++q8) {
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
-                st16_split(sm + cb::SM_KT, sm + cb::SM_KTL, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
-            }
-        }
-    }
-    const int t_loc = tid & 63;
-    const int grp = tid >> 6;
-
-    for (int c = 0; c < nchunk; ++c) {
-        const int st = c & 1;
-        const int t0 = c * Q;
-        unsigned char *sX = sm + cb::SM_X + st * 8192;
-        unsigned char *sB = sm + cb::SM_B + st * 16384;
-        unsigned char *sDY = sm + cb::SM_DY + st * 8192;
-
-        for (int i = tid; i < Q + 1; i += THREADS) {
-            const int t = t0 + i;
-            float dv = 0.f, lv = 1.f;
-            if (t < L) {
-                dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
-                if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
-            }
-            f32[F_DT + i] = dv;
-            f32[F_LAM + i] = lv;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
-            float v = d0 + d1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            f32[F_S + 2 * lane] = v - d1;
-            f32[F_S + 2 * lane + 1] = v;
-        } else if (warp == 1 || warp == 2) {
-            const int t = (warp - 1) * 32 + lane;
-            const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
-            const float bn = (t0 + t + 1 < L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
-            f32[F_SIG + t] = fmaf(lv, dv, bn);
-            f32[F_BN + t] = bn;
-        }
-        if (!mbar_wait(&bar_tma[st], (uint32_t)((c >> 1) & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
-        __syncthreads();
-        if (*abort_flag) break;
-
-        // per-mode chunk constants (as in the forward)
-        for (int m = tid; m < nmode; m += THREADS) {
-            const float a2 = f32[F_A2 + m], w = f32[F_W + m];
-            float er[4], ei[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
-                const float ds = f32[F_S + 16 * k + 15] - lo;
-                const float mag = exp2f(a2 * ds);
-                if (m >= nr) {
-                    float sn, cs;
-                    sincosf(w * ds, &sn, &cs);
-                    er[k] = mag * cs;
-                    ei[k] = mag * sn;
-                } else {
-                    er[k] = mag;
-                    ei[k] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float pr = 1.f, pi = 0.f;
-#pragma unroll
-                for (int j = i + 1; j <= 4; ++j) {
-                    float nr_, ni_;
-                    cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
-                    pr = nr_;
-                    pi = ni_;
-                    f32[F_KRE + fslot(i, j) * NP + m] = pr;
-                    f32[F_KIM + fslot(i, j) * NP + m] = pi;
-                    if (i == 0 && j < 4) {
-                        f32[F_KRE + gslot(j) * NP + m] = pr;
-                        f32[F_KIM + gslot(j) * NP + m] = -pi;
-                    }
-                }
-            }
-        }
-        __syncthreads();
-
-        // B-side operands: own-block Bi, later-block copies, Bh
-        {
-            const int t = t_loc;
-            const int ib = t >> 4;
-            const float St = f32[F_S + t];
-            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-            const float ds = St - Sb;
-            const float sig = f32[F_SIG + t];
-#pragma unroll 1
-            for (int k = 0; k < 4; ++k) {
-                const int r0 = 8 * (grp + 4 * k);
-                if (r0 >= N) break;
-                float vBI[8], vBH[8], vBX[3][8], rb[8];
-                ld_rows8(sB, t, r0, rb);
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    const int r = r0 + j;
-                    const float b0 = rb[j], b1 = rb[j + 1];
-                    float bi0, bi1;
-                    int m0, m1;
-                    bool pair;
-                    if (r < nr) {
-                        pair = false;
-                        m0 = r;
-                        m1 = r + 1;
-                        bi0 = sig * b0 * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
-                        bi1 = sig * b1 * ex2_fast(fminf(-f32[F_A2 + m1] * ds, 120.f));
-                    } else {
-                        pair = true;
-                        m0 = m1 = nr + ((r - nr) >> 1);
-                        float sn, cs;
-                        __sincosf(f32[F_W + m0] * ds, &sn, &cs);
-                        const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
-                        bi0 = eb * fmaf(b0, cs, b1 * sn);
-                        bi1 = eb * fmaf(b1, cs, -b0 * sn);
-                    }
-                    vBI[j] = bi0;
-                    vBI[j + 1] = bi1;
-                    if (!pair) {
-                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
-                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
-#pragma unroll
-                        for (int q = 0; q < 3; ++q) {
-                            const int i2 = ib + 1 + q;
-                            if (i2 < 4) {
-                                vBX[q][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
-                                vBX[q][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                            for (int j = 0; j < 8; ++j) {
+                                lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
+                                hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
                             }
-                        }
-                    } else {
-                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m0],
-                             f32[F_KIM + fslot(ib, 4) * NP + m0], vBH[j], vBH[j + 1]);
-#pragma unroll
-                        for (int q = 0; q < 3; ++q) {
-                            const int i2 = ib + 1 + q;
-                            if (i2 < 4)
-                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m0],
-                                     f32[F_KIM + fslot(ib, i2) * NP + m0], vBX[q][j],
-                                     vBX[q][j + 1]);
+                            unsigned char *pt = sm + outk::SM_P + i * 2048;
+                            st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
+                            st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
                         }
                     }
                 }
-                st16_split(sm + cb::SM_BI + bi_off(ib), sm + cb::SM_BIL + bi_off(ib),
-                           off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const int i2 = ib + 1 + q;
-                    if (i2 < 4)
-                        st16_split(sm + cb::SM_BI + bi_off(i2), sm + cb::SM_BIL + bi_off(i2),
-                                   off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[q]);
-                }
-                st16_split(sm + cb::SM_BH, sm + cb::SM_BHL, off_mnmaj(r0, t, 2048u, 128u), vBH);
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
 
-        // phase A: chunk state, V^T = K_prev dY^T, G = dY X^T
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t x_base = smem_u32(sX), dy_base = smem_u32(sDY);
-            const uint32_t id_st = idesc_bf16(128, 64, true, true);
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t bh_base = smem_u32(sm + (part ? cb::SM_BHL : cb::SM_BH));
-                for (int s = 0; s < Q / 16; ++s)
-                    mma_bf16(t_st, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                             sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_st,
-                             part > 0 || s > 0);
-            }
-            const uint32_t id_v = idesc_bf16(128, 64, false, false);
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t kt_base = smem_u32(sm + (part ? cb::SM_KTL : cb::SM_KT));
-                for (int s = 0; s < PD / 16; ++s)
-                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                             part > 0 || s > 0);
-            }
-            const uint32_t id_g = idesc_bf16(64, 64, false, false);
-            for (int s = 0; s < PD / 16; ++s)
-                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
-            mma_commit(&bar_mma[0]);
-        }
-        if (!mbar_wait(&bar_mma[0], (uint32_t)(c & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
-        fence_after_sync();
-        __syncthreads();
-        if (*abort_flag) break;
-
-        if (warp < 4) {
-            // carried state K_c = e^{lam S_63} K_{c-1} + S_chunk  (as in the forward)
-            const int n = tid;
-            const int m = n < nr ? n : nr + ((n - nr) >> 1);
-            const bool pr_row = n >= nr && n < N;
-            const bool im_row = pr_row && ((n - nr) & 1);
-            float dr = 0.f, di = 0.f;
-            if (n < N) {
-                dr = f32[F_KRE + fslot(0, 4) * NP + m];
-                di = f32[F_KIM + fslot(0, 4) * NP + m];
-            }
-#pragma unroll
-            for (int c16 = 0; c16 < PD / 16; ++c16) {
-                float sv[16];
-                tmem_ld16(tmem_addr(t_st, 32u * warp, 16u * c16), sv);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int q = c16 * 16 + j;
-                    const float own = K[q];
-                    const float other = __shfl_xor_sync(0xffffffffu, own, 1);
-                    float nv;
-                    if (!pr_row)
-                        nv = fmaf(dr, own, sv[j]);
-                    else if (!im_row)
-                        nv = fmaf(dr, own, fmaf(-di, other, sv[j]));
-                    else
-                        nv = fmaf(di, other, fmaf(dr, own, sv[j]));
-                    K[q] = n < N ? nv : 0.f;
-                }
-            }
-        } else {
-            // masked G rows -> K-major tiles (N = 16 t of block i, K = s); diagonal dy_t . u_t
-            const int qd = warp - 4;
-            for (int i = 0; i < NSB; ++i) {
-                float v[16];
-                tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
-                if (lane < 16 && i <= qd) {
-                    const int t = 16 * qd + lane;
-                    float lo[8], hi[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
-                        hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
-                    }
-                    unsigned char *gt = sm + cb::SM_GM + qd * 2048;
-                    st16_split(gt, gt + 8192, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
-                    st16_split(gt, gt + 8192, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
-                    if (i == qd) f32[F_CORR + t] = v[lane];
-                }
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-
-        // phase B: D_i = Bi^T (G o mask)_i^T into the (now free) G columns
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id_d = idesc_bf16(128, 16, true, false);
-            // hi*hi + hi*lo + lo*hi
-            const uint32_t a_off[3] = {cb::SM_BI, cb::SM_BI, cb::SM_BIL};
-            const uint32_t b_off[3] = {cb::SM_GM, cb::SM_GM + 8192u, cb::SM_GM};
-            for (int i = 0; i < NSB; ++i)
-                for (int part = 0; part < 3; ++part) {
-                    const uint32_t bi_base = smem_u32(sm + a_off[part]);
-                    const uint32_t gm_base = smem_u32(sm + b_off[part]);
+            // ---- phase B: intra-chunk term Y^T += X^T P^T_i ----------------------
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t x_base = smem_u32(sm + outk::SM_X), p_base = smem_u32(sm + outk::SM_P);
+                const uint32_t id_d = idesc_bf16(64, 16, true, true);
+                for (int i = 0; i < NSB; ++i)
                     for (int s = 0; s <= i; ++s)
-                        mma_bf16(t_g + 16 * i,
-                                 sdesc(bi_base + bi_off(i) + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                                 sdesc(gm_base + i * 2048u + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                                 id_d, part > 0 || s > 0);
-                }
-            mma_commit(&bar_mma[1]);
-        }
-        // the state tile for the next chunk's V^T (phase A of this chunk has consumed it)
-        if (warp < 4) {
-            const int n = tid;
-            if (p.ws_kb && c + 1 < nchunk && n < N) {
-                float4 *kb = reinterpret_cast<float4 *>(
-                    p.ws_kb + ((((long long)b * p.H + h) * p.nc + c) * N + n) * PD);
-#pragma unroll
-                for (int q4 = 0; q4 < PD / 4; ++q4)
-                    kb[q4] = make_float4(K[4 * q4], K[4 * q4 + 1], K[4 * q4 + 2], K[4 * q4 + 3]);
+                        mma_bf16(t_y + 16 * i, sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128),
+                                 sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
+                                 true);
+                mma_commit(&bar_mma[1]);
             }
+            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
+            if (!ok) raise_error(1);
+            fence_after_sync();
+            if (__syncthreads_and(ok)) {
+                // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p] -----------------
+                const int qd = warp & 3, part = warp >> 2;   // TMEM quarter, column block
+                const int pp = 16 * qd + (lane & 15);
+                const unsigned char *sX = sm + outk::SM_X;
+                __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
+                                      h * p.sy[2] + pp;
+                constexpr int CPW = 64 / (outk::THREADS / 128);
+                for (int c16 = 0; c16 < CPW / 16; ++c16) {
+                    float v[16];
+                    const int tc = CPW * part + 16 * c16;
+                    tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
+                    if (lane < 16) {
+                        __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
 #pragma unroll
-            for (int q8 = 0; q8 < PD / 8; ++q8) {
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = K[q8 * 8 + j];
-                st16_split(sm + cb::SM_KT, sm + cb::SM_KTL, off_mnmaj(q8 * 8, n, 1024u, 128u), v);
-            }
-        }
-        if (!mbar_wait(&bar_mma[1], (uint32_t)(c & 1), WAIT_LIMIT)) {
-            raise_error(1);
-            *abort_flag = 1;
-        }
-        fence_after_sync();
-        fence_proxy_async();
-        __syncthreads();
-        if (*abort_flag) break;
-
-        // unfold: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D ; dC_t = dCK_t - beta' (dy.u) B_t
-        {
-            const int n = tid & 127;
-            const int half = tid >> 7;
-            const int qd = warp & 3;
-            const bool valid = n < N;
-            const int m = n < nr ? n : nr + ((n - nr) >> 1);
-            const bool pr_row = valid && n >= nr;
-            const bool im_row = pr_row && ((n - nr) & 1);
-            const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
-            float *dst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
-            const long long tstride = (long long)p.H * p.N;
-            for (int c16 = 0; c16 < 2; ++c16) {
-                const int tc = 32 * half + 16 * c16;
-                float vv[16], dd[16];
-                tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
-                tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), dd);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = tc + j;
-                    const int ib = t >> 4;
-                    const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-                    const float ds = f32[F_S + t] - Sb;
-                    // E' = e^{lam ds}, E = E' * e^{lam Sb_i} = E' * conj(G_i)
-                    const float mag = ex2_fast(a2 * ds);
-                    float er = mag, ei = 0.f;
-                    if (pr_row) {
-                        float sn, cs;
-                        __sincosf(w * ds, &sn, &cs);
-                        er = mag * cs;
-                        ei = mag * sn;
-                    }
-                    float fr = 1.f, fi = 0.f;
-                    if (ib && valid) {
-                        fr = f32[F_KRE + gslot(ib) * NP + m];
-                        fi = -f32[F_KIM + gslot(ib) * NP + m];
-                    }
-                    float Er, Ei;
-                    cmul(er, ei, fr, fi, Er, Ei);
-                    const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
-                    const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
-                    float res;
-                    if (!pr_row) {
-                        res = Er * vv[j] + er * dd[j];
-                    } else if (!im_row) {  // real part of E (V_re + i V_im) + E' (D_re + i D_im)
-                        res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
-                    } else {               // imaginary part
-                        res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
-                    }
-                    if (valid && t0 + t < L) {
-                        const float bt = ld_row1(sB, t, n);
-                        dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
+                        for (int j = 0; j < 16; ++j) {
+                            const int t = tc + j;
+                            if (t0 + t < L) {
+                                const float u = bf(sX + off_sw128(t, pp));
+                                *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
+                            }
+                            yp += p.sy[1];
+                        }
                     }
                 }
             }
         }
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0 && c + 2 < nchunk) {
-            mbar_expect_tx(&bar_tma[st], tile_bytes);
-            tma_load_4d(sm + cb::SM_X + st * 8192, &tmX, &bar_tma[st], 0, h, (c + 2) * Q, b);
-            tma_load_4d(sm + cb::SM_DY + st * 8192, &tmDY, &bar_tma[st], 0, h, (c + 2) * Q, b);
-            for (int k = 0; k < nbox; ++k)
-                tma_load_4d(sm + cb::SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g,
-                            (c + 2) * Q, b);
-        }
-    }
-    if (*abort_flag && tid == 0) {
-        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
-        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);
     }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         fence_after_sync();
-        tmem_dealloc(tbase, cb::TMEM_COLS);
+        tmem_dealloc(tbase, outk::TMEM_COLS);
     }
 }
-
-// ---------------------------------------------------------------------------
-// host side
-// ---------------------------------------------------------------------------
 
 }  // namespace chunkfwd
 
@@ -1091,14 +621,13 @@ cudaError_t chunk_range_check(const Params &p, int *gate, cudaStream_t st) {
 bool chunk_fwd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
-    return p.bf16 && p.P == chunkfwd::PD && p.R == 1 && p.O == 1 &&
-           (p.N == 64 || p.N == 128) && p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) &&
-           st16(p.sx[0]) && st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) &&
-           st16(p.sB[2]) && st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) &&
-           chunkfwd::encode_fn() != nullptr;
+    return p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 && (p.N == 64 || p.N == 128) &&
+           p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
+           st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) && st16(p.sB[2]) &&
+           st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) && chunkc::encode_fn() != nullptr;
 }
 
-// The tensor-core backward part additionally reads dy through TMA.
+// The tensor-core backward additionally reads dy through TMA and writes dx in 16-byte rows.
 bool chunk_bwd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
@@ -1106,43 +635,46 @@ bool chunk_bwd_supported(const Params &p) {
            st16(p.sy[2]) && (!p.dx || al16(p.dx));
 }
 
+template <typename K>
+static cudaError_t set_smem_once(K kern, uint32_t bytes, bool &done) {
+    if (done) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
+// The state entering every chunk (p.ws_kp) and the chunk decays (p.ws_ce);
+// also hT and the last write when p.hT / p.wT are set.
+cudaError_t chunk_states(const Params &p, cudaStream_t st) {
+    using namespace chunkfwd;
+    CUtensorMap mx, mb;
+    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
+        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true))
+        return cudaErrorInvalidValue;
+    static bool a1 = false;
+    cudaError_t e;
+    if ((e = set_smem_once(k_chunk_state_local, stl::SMEM_BYTES, a1)) != cudaSuccess) return e;
+    k_chunk_state_local<<<dim3(p.nc, p.H, p.Bsz), stl::THREADS, stl::SMEM_BYTES, st>>>(mx, mb, p);
+    profile_mark(st, "k_chunk_state_local");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_chunk_state_pass<<<dim3(p.H, p.Bsz), pas::THREADS, 0, st>>>(p);
+    profile_mark(st, "k_chunk_state_pass");
+    return cudaGetLastError();
+}
+
 cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     using namespace chunkfwd;
+    cudaError_t e = chunk_states(p, st);
+    if (e != cudaSuccess) return e;
     CUtensorMap mx, mb, mc;
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
         !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
         !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true))
         return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k_chunk_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    k_chunk_fwd<<<dim3(p.H, p.Bsz), THREADS, SMEM_BYTES, st>>>(mx, mb, mc, p);
-    profile_mark(st, "k_chunk_fwd");
-    return cudaGetLastError();
-}
-
-// Backward forward-direction part on the tensor cores: per-head dC into p.ws_dC.
-cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st) {
-    using namespace chunkfwd;
-    CUtensorMap mx, mb, mdy;
-    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
-        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
-        !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
-        return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k_chunk_bwd_dc,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)chunkbwd::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
-    k_chunk_bwd_dc<<<dim3(p.H, p.Bsz), THREADS, chunkbwd::SMEM_BYTES, st>>>(mx, mb, mdy, p);
-    profile_mark(st, "k_chunk_bwd_dc");
+    static bool a3 = false;
+    if ((e = set_smem_once(k_chunk_out, outk::SMEM_BYTES, a3)) != cudaSuccess) return e;
+    k_chunk_out<<<dim3(p.nc, p.H, p.Bsz), outk::THREADS, outk::SMEM_BYTES, st>>>(mx, mb, mc, p);
+    profile_mark(st, "k_chunk_out");
     return cudaGetLastError();
 }
 

@@ -37,105 +37,6 @@ namespace chunkrev {
 using namespace umma;
 using namespace chunkc;
 
-// ---- per-chunk token quantities and mode constants ----------------------------
-// Loads dt / lambda of tokens t0 .. t0+64 and writes the inclusive prefix S_t
-// (F_S) and, with `want_sigma`, sigma_t (F_SIG) and beta_{t+1} (F_BN).
-// Call with all threads of the block (>= 96); contains barriers.
-__device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b, int h, int t0,
-                                             bool want_sigma) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < Q + 1; i += blockDim.x) {
-        const int t = t0 + i;
-        float dv = 0.f, lv = 1.f;
-        if (t < p.L) {
-            dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
-            if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
-        }
-        f32[F_DT + i] = dv;
-        f32[F_LAM + i] = lv;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const float d0 = f32[F_DT + 2 * lane], d1 = f32[F_DT + 2 * lane + 1];
-        float v = d0 + d1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += u;
-        }
-        f32[F_S + 2 * lane] = v - d1;
-        f32[F_S + 2 * lane + 1] = v;
-    } else if (want_sigma && (warp == 1 || warp == 2)) {
-        const int t = (warp - 1) * 32 + lane;
-        const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
-        const float bn =
-            (t0 + t + 1 < p.L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
-        f32[F_SIG + t] = fmaf(lv, dv, bn);
-        f32[F_BN + t] = bn;
-    }
-    __syncthreads();
-}
-
-// Per-mode decay over each sub-block, E_k = e^{lam dS_k}, and the products
-// F[i][j] = prod_{k=i}^{j-1} E_k and G_i = conj(F[0][i]) into the F_KRE / F_KIM
-// slots.  Needs F_S, F_A2, F_W.  Ends with a barrier.
-__device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
-    const int nmode = p.nr + p.np;
-    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
-        const float a2 = f32[F_A2 + m], w = f32[F_W + m];
-        float er[4], ei[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
-            const float ds = f32[F_S + 16 * k + 15] - lo;
-            const float mag = exp2f(a2 * ds);
-            if (m >= p.nr) {
-                float sn, cs;
-                sincosf(w * ds, &sn, &cs);
-                er[k] = mag * cs;
-                ei[k] = mag * sn;
-            } else {
-                er[k] = mag;
-                ei[k] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float pr = 1.f, pi = 0.f;
-#pragma unroll
-            for (int j = i + 1; j <= 4; ++j) {
-                float nr_, ni_;
-                cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
-                pr = nr_;
-                pi = ni_;
-                f32[F_KRE + fslot(i, j) * NP + m] = pr;
-                f32[F_KIM + fslot(i, j) * NP + m] = pi;
-                if (i == 0 && j < 4) {
-                    f32[F_KRE + gslot(j) * NP + m] = pr;
-                    f32[F_KIM + gslot(j) * NP + m] = -pi;
-                }
-            }
-        }
-    }
-    __syncthreads();
-}
-
-__device__ __forceinline__ void mode_rates(const Params &p, float *f32, int h) {
-    const int nmode = p.nr + p.np;
-    for (int m = threadIdx.x; m < NP; m += blockDim.x) {
-        float a2 = 0.f, w = 0.f;
-        if (m < nmode) {
-            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
-            if (m >= p.nr) w = p.theta[h * p.np + (m - p.nr)];
-        }
-        f32[F_A2 + m] = a2;
-        f32[F_W + m] = w;
-    }
-}
-
-__device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {
-    return ((long long)b * p.H + h) * p.nc + c;
-}
 
 // ============================================================================
 // k_chunk_adj_local: Ghat_c = Ch^T (N x 64 t) . dY (64 t x 64 p), per chunk.
@@ -170,7 +71,7 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / p.hpg;
-    const int N = p.N, nr = p.nr, nmode = p.nr + p.np;
+    const int N = p.N, nr = p.nr;
     const int t0 = c * Q;
     const int nbox = N / 64;
 
@@ -192,12 +93,6 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
             reinterpret_cast<uint4 *>(sm + loc::SM_CH)[i] = make_uint4(0, 0, 0, 0);
     chunk_tokens(p, f32, b, h, t0, false);
     chunk_mode_constants(p, f32);
-    // chunk decay per mode for the passing kernel
-    for (int m = tid; m < nmode; m += loc::THREADS) {
-        float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
-        ce[2 * m] = f32[F_KRE + fslot(0, 4) * NP + m];
-        ce[2 * m + 1] = f32[F_KIM + fslot(0, 4) * NP + m];
-    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -289,96 +184,105 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
 
 // ============================================================================
 // k_chunk_adj_pass: reverse pass over the chunks of one (batch row, head).
-// Thread (row pair rp, column p) keeps rows 2rp, 2rp+1 of the adjoint carry:
-// two real modes, or one rotation pair as (re, im).  ws_gc[c] holds Ghat_c on
-// entry and the carry into chunk c on exit.
+// Thread (row-pair group, 4 consecutive p) keeps rows 2rp, 2rp+1 of the adjoint
+// carry for rp = rp0, rp0 + 16, ...: two real modes, or one rotation pair as
+// (re, im).  Every chunk's loads are issued together in 16-byte rows.
+// ws_gc[c] holds Ghat_c on entry and the carry into chunk c on exit.
 // ============================================================================
 namespace pass {
-constexpr int THREADS = 512;
-constexpr int KMAX = NP / 16;   // row pairs per thread
+constexpr int THREADS = 256;
+constexpr int KMAX = NP / 32;   // row pairs per thread
 }  // namespace pass
 
-__global__ void __launch_bounds__(pass::THREADS, 2) k_chunk_adj_pass(Params p) {
+__device__ __forceinline__ float sum16(float v) {
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
     if (gated_off(p)) return;
-    // chunk decays, triple-buffered: chunk c-1's are fetched while chunk c is processed
-    __shared__ float s_ce[3][2 * NP];
+    __shared__ float s_ce[3][2 * NP];   // chunk decays, triple-buffered
     __shared__ float red[pass::THREADS];
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const int N = p.N, nr = p.nr, nc = p.nc;
-    const int q = tid & 63, rp0 = tid >> 6, wp = q >> 5;
-    const int nk = N / 16;
-    float g0[pass::KMAX], g1[pass::KMAX];
+    const int q = 4 * (tid & 15), rp0 = tid >> 4;
+    const int nk = N / 32;
+    float4 g0[pass::KMAX], g1[pass::KMAX];
 #pragma unroll
-    for (int k = 0; k < pass::KMAX; ++k) g0[k] = g1[k] = 0.f;
-    if (tid < 2 * NP) s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
+    for (int k = 0; k < pass::KMAX; ++k) g0[k] = g1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
 
     for (int c = nc - 1; c >= 0; --c) {
         float *gbase = p.ws_gc + bhc(p, b, h, c) * N * PD + q;
-        const float *kb = (c > 0 && p.ws_qb) ? p.ws_kb + bhc(p, b, h, c - 1) * N * PD + q : nullptr;
-        if (c > 0 && tid < 2 * NP)
-            s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
-        __syncthreads();
-        const float *ce = s_ce[c % 3];
-        float *qb = p.ws_qb ? p.ws_qb + (bhc(p, b, h, c) * 4 + wp) * (long long)N : nullptr;
-        // two halves of KMAX / 2 row pairs; each half issues all of its loads first
+        // K_end_{c-1}: the state entering chunk c
+        const float *kb = (c > 0 && p.ws_qb) ? p.ws_kp + bhc(p, b, h, c) * N * PD + q : nullptr;
+        float4 hv0[pass::KMAX], hv1[pass::KMAX], kv0[pass::KMAX], kv1[pass::KMAX];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            constexpr int KH = pass::KMAX / 2;
-            float hv0[KH], hv1[KH], kv0[KH], kv1[KH];
-#pragma unroll
-            for (int kk = 0; kk < KH; ++kk) {
-                const int k = hf * KH + kk;
-                hv0[kk] = hv1[kk] = kv0[kk] = kv1[kk] = 0.f;
-                if (k < nk) {
-                    const int n0 = 2 * (rp0 + 8 * k);
-                    hv0[kk] = gbase[(long long)n0 * PD];
-                    hv1[kk] = gbase[(long long)(n0 + 1) * PD];
-                    if (kb) {
-                        kv0[kk] = __ldg(kb + (long long)n0 * PD);
-                        kv1[kk] = __ldg(kb + (long long)(n0 + 1) * PD);
-                    }
+        for (int k = 0; k < pass::KMAX; ++k) {
+            if (k < nk) {
+                const int n0 = 2 * (rp0 + 16 * k);
+                hv0[k] = *reinterpret_cast<const float4 *>(gbase + (long long)n0 * PD);
+                hv1[k] = *reinterpret_cast<const float4 *>(gbase + (long long)(n0 + 1) * PD);
+                if (kb) {
+                    kv0[k] = __ldg(reinterpret_cast<const float4 *>(kb + (long long)n0 * PD));
+                    kv1[k] = __ldg(reinterpret_cast<const float4 *>(kb + (long long)(n0 + 1) * PD));
                 }
             }
+        }
+        if (c > 0) s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
+        __syncthreads();
+        const float *ce = s_ce[c % 3];
+        float *qb = p.ws_qb ? p.ws_qb + bhc(p, b, h, c) * 4 * (long long)N : nullptr;
 #pragma unroll
-            for (int kk = 0; kk < KH; ++kk) {
-                const int k = hf * KH + kk;
-                if (k >= nk) break;
-                const int n0 = 2 * (rp0 + 8 * k);
-                // the carry into chunk c, then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
-                gbase[(long long)n0 * PD] = g0[k];
-                gbase[(long long)(n0 + 1) * PD] = g1[k];
-                float a0, a1;
+        for (int k = 0; k < pass::KMAX; ++k) {
+            if (k >= nk) break;
+            const int n0 = 2 * (rp0 + 16 * k);
+            // the carry into chunk c, then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
+            *reinterpret_cast<float4 *>(gbase + (long long)n0 * PD) = g0[k];
+            *reinterpret_cast<float4 *>(gbase + (long long)(n0 + 1) * PD) = g1[k];
+            float4 &a = g0[k], &d = g1[k];
+            if (n0 < nr) {
+                const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
+                a.x = fmaf(e0, a.x, hv0[k].x); a.y = fmaf(e0, a.y, hv0[k].y);
+                a.z = fmaf(e0, a.z, hv0[k].z); a.w = fmaf(e0, a.w, hv0[k].w);
+                d.x = fmaf(e1, d.x, hv1[k].x); d.y = fmaf(e1, d.y, hv1[k].y);
+                d.z = fmaf(e1, d.z, hv1[k].z); d.w = fmaf(e1, d.w, hv1[k].w);
+            } else {
+                const int m = nr + ((n0 - nr) >> 1);
+                const float er = ce[2 * m], ei = ce[2 * m + 1];
+                // conj(er + i ei) (a + i d) + Ghat
+                const float4 ao = a;
+                a.x = fmaf(er, ao.x, fmaf(ei, d.x, hv0[k].x));
+                a.y = fmaf(er, ao.y, fmaf(ei, d.y, hv0[k].y));
+                a.z = fmaf(er, ao.z, fmaf(ei, d.z, hv0[k].z));
+                a.w = fmaf(er, ao.w, fmaf(ei, d.w, hv0[k].w));
+                d.x = fmaf(er, d.x, fmaf(-ei, ao.x, hv1[k].x));
+                d.y = fmaf(er, d.y, fmaf(-ei, ao.y, hv1[k].y));
+                d.z = fmaf(er, d.z, fmaf(-ei, ao.z, hv1[k].z));
+                d.w = fmaf(er, d.w, fmaf(-ei, ao.w, hv1[k].w));
+            }
+            if (kb) {
+                // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}; 16 lanes hold one row pair
+                float q0, q1;
+                const float4 k0 = kv0[k], k1 = kv1[k];
                 if (n0 < nr) {
-                    a0 = fmaf(ce[2 * n0], g0[k], hv0[kk]);
-                    a1 = fmaf(ce[2 * (n0 + 1)], g1[k], hv1[kk]);
+                    q0 = a.x * k0.x + a.y * k0.y + a.z * k0.z + a.w * k0.w;
+                    q1 = d.x * k1.x + d.y * k1.y + d.z * k1.z + d.w * k1.w;
                 } else {
-                    const int m = nr + ((n0 - nr) >> 1);
-                    const float er = ce[2 * m], ei = ce[2 * m + 1];
-                    a0 = fmaf(er, g0[k], fmaf(ei, g1[k], hv0[kk]));
-                    a1 = fmaf(er, g1[k], fmaf(-ei, g0[k], hv1[kk]));
+                    q0 = (a.x * k0.x + a.y * k0.y + a.z * k0.z + a.w * k0.w) +
+                         (d.x * k1.x + d.y * k1.y + d.z * k1.z + d.w * k1.w);
+                    q1 = (a.x * k1.x + a.y * k1.y + a.z * k1.z + a.w * k1.w) -
+                         (d.x * k0.x + d.y * k0.y + d.z * k0.z + d.w * k0.w);
                 }
-                g0[k] = a0;
-                g1[k] = a1;
-                if (kb) {
-                    // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}
-                    float q0, q1;
-                    if (n0 < nr) {
-                        q0 = a0 * kv0[kk];
-                        q1 = a1 * kv1[kk];
-                    } else {
-                        q0 = fmaf(a0, kv0[kk], a1 * kv1[kk]);
-                        q1 = fmaf(a0, kv1[kk], -a1 * kv0[kk]);
-                    }
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) {
-                        q0 += __shfl_xor_sync(0xffffffffu, q0, o);
-                        q1 += __shfl_xor_sync(0xffffffffu, q1, o);
-                    }
-                    if (lane == 0) {
-                        qb[n0] = q0;
-                        qb[n0 + 1] = q1;
-                    }
+                q0 = sum16(q0);
+                q1 = sum16(q1);
+                if ((tid & 15) == 0) {
+                    qb[n0] = q0;            // slot 0 holds the whole sum over p
+                    qb[n0 + 1] = q1;
+                    qb[N + n0] = 0.f;       // slot 1 (read by the carry pass) stays zero
+                    qb[N + n0 + 1] = 0.f;
                 }
             }
         }
@@ -391,17 +295,22 @@ __global__ void __launch_bounds__(pass::THREADS, 2) k_chunk_adj_pass(Params p) {
 #pragma unroll
     for (int k = 0; k < pass::KMAX; ++k) {
         if (k >= nk) break;
-        const int n0 = 2 * (rp0 + 8 * k);
-        const long long i0 = ix_st(p, b, h, n0, q), i1 = ix_st(p, b, h, n0 + 1, q);
-        if (p.dh0) {
-            p.dh0[i0] = g0[k];
-            p.dh0[i1] = g1[k];
+        const int n0 = 2 * (rp0 + 16 * k);
+        const float a[4] = {g0[k].x, g0[k].y, g0[k].z, g0[k].w};
+        const float d[4] = {g1[k].x, g1[k].y, g1[k].z, g1[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+            if (p.dh0) {
+                p.dh0[i0] = a[j];
+                p.dh0[i1] = d[j];
+            }
+            if (p.dw0) {
+                p.dw0[i0] = beta0 * a[j];
+                p.dw0[i1] = beta0 * d[j];
+            }
+            if (p.w0) db0 = fmaf(a[j], p.w0[i0], fmaf(d[j], p.w0[i1], db0));
         }
-        if (p.dw0) {
-            p.dw0[i0] = beta0 * g0[k];
-            p.dw0[i1] = beta0 * g1[k];
-        }
-        if (p.w0) db0 = fmaf(g0[k], p.w0[i0], fmaf(g1[k], p.w0[i1], db0));
     }
     red[tid] = db0;
     __syncthreads();
@@ -474,24 +383,8 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
     if (N < NP)  // K padding of Ci, Bi, Bh
         for (int i = tid; i < (int)((dxk::SM_P - dxk::SM_CI) / 16); i += dxk::THREADS)
             reinterpret_cast<uint4 *>(sm + dxk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
-    // Gc (fp32, [n][p]) -> bf16 B operand; rows past N are zero
-    {
-        const float *gsrc = p.ws_gc + bhc(p, b, h, c) * N * PD;
-        for (int it = tid; it < NP * (PD / 8); it += dxk::THREADS) {
-            const int n = it >> 3, p8 = (it & 7) * 8;
-            float v[8];
-            if (n < N) {
-                const float4 a = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8);
-                const float4 d = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8 + 4);
-                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.f;
-            }
-            st16(sm + dxk::SM_GC, off_mnmaj(p8, n, 1024u, 128u), v);
-        }
-    }
+    // the adjoint carried into this chunk as the bf16 B operand (N = p, K = rows)
+    load_state_tile(p.ws_gc + bhc(p, b, h, c) * N * PD, N, sm + dxk::SM_GC, nullptr);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
     fence_before_sync();
@@ -771,24 +664,8 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     if (N < NP)  // M padding of the mirror tiles
         for (int i = tid; i < (int)((gbk::SM_GM - gbk::SM_CM) / 16); i += gbk::THREADS)
             reinterpret_cast<uint4 *>(sm + gbk::SM_CM)[i] = make_uint4(0, 0, 0, 0);
-    // Gc (fp32 [n][p]) -> bf16 hi / lo, K-major (rows n, K = p); rows past N are zero
-    {
-        const float *gsrc = p.ws_gc + bhc(p, b, h, c) * N * PD;
-        for (int it = tid; it < NP * (PD / 8); it += gbk::THREADS) {
-            const int n = it >> 3, p8 = (it & 7) * 8;
-            float v[8];
-            if (n < N) {
-                const float4 a = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8);
-                const float4 d = *reinterpret_cast<const float4 *>(gsrc + (long long)n * PD + p8 + 4);
-                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.f;
-            }
-            st16_split(sm + gbk::SM_GC, sm + gbk::SM_GCL, off_kmaj(n, p8, 128u, 1024u), v);
-        }
-    }
+    // the adjoint carried into this chunk, bf16 hi / lo, K-major (rows n, K = p)
+    load_state_tile(p.ws_gc + bhc(p, b, h, c) * N * PD, N, sm + gbk::SM_GC, sm + gbk::SM_GCL);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
     fence_before_sync();
@@ -1131,6 +1008,299 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     }
 }
 
+// ============================================================================
+// k_chunk_bwd_dc: per chunk, dC_t = dy_t H_t^T per head.
+//   H_t = K_t - beta_{t+1} W_t,   K_t = e^{lam S_t} K_prev + sum_{s<=t} Phi_{t,s} sigma_s b_s u_s
+// so, per state mode (complex for rotation pairs, real rows otherwise),
+//   dCK_t = e^{lam S_t} (dy_t . K_prev) + e^{lam (S_t - Sb_i)} sum_{s<=t} (dy_t . u_s) Bi_s
+// which is, on the tensor cores (operands split into bf16 hi + lo),
+//   V^T  = K_prev (N x 64 p) . dY^T (64 p x 64 t)          M=128, N=64, K=64
+//   G    = dY (64 t x 64 p) . X^T (64 p x 64 s)            M=64,  N=64, K=64
+//   D_i  = Bi^T (N x s) . (G o causal mask)_i^T (s x 16 t) M=128, N=16, K=16(i+1)
+// followed by the per-(t, row) unfolding of the decay factors on the CUDA
+// cores; dC_t = dCK_t - beta_{t+1} (dy_t . u_t) B_t.  K_prev is the state
+// entering the chunk (k_chunk_state_pass).
+// ============================================================================
+namespace dck {
+constexpr int THREADS = 512;
+constexpr int RG = THREADS / 64;    // row groups of the operand preparation
+constexpr int TQ = THREADS / 128;   // token groups of the unfold
+constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle)
+constexpr uint32_t SM_DY = 8192;      // 8 KB  dy (128B swizzle)
+constexpr uint32_t SM_B = 16384;      // 16 KB raw B (two 64-row swizzled halves)
+constexpr uint32_t SM_BI = 32768;     // 40 KB Bi tiles (hi)
+constexpr uint32_t SM_BIL = 73728;    // 40 KB Bi tiles (lo)
+constexpr uint32_t SM_GM = 114688;    // 8 KB  masked G hi: 4 tiles, K-major (N = 16 t, K = s)
+constexpr uint32_t SM_GML = 122880;   // 8 KB  masked G lo
+constexpr uint32_t SM_KT = 131072;    // 16 KB K_prev hi, K-major (rows n, K = p)
+constexpr uint32_t SM_KTL = 147456;   // 16 KB K_prev lo
+constexpr uint32_t SM_F32 = 163840;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace dck
+
+__global__ void __launch_bounds__(dck::THREADS, 1)
+k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmDY, Params p) {
+    if (gated_off(p)) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + dck::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dck::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;   // [2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / p.hpg;
+    const int N = p.N, nr = p.nr, L = p.L;
+    const int t0 = c * Q;
+    const int nbox = N / 64;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmDY);
+        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + Q * N * 2));
+        tma_load_4d(sm + dck::SM_X, &tmX, bar_tma, 0, h, t0, b);
+        tma_load_4d(sm + dck::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        for (int k = 0; k < nbox; ++k)
+            tma_load_4d(sm + dck::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+    }
+    if (warp == 0) tmem_alloc(tslot, dck::TMEM_COLS);
+    mode_rates(p, f32, h);
+    if (N < NP)  // M padding of the Bi tiles
+        for (int i = tid; i < (int)((dck::SM_GM - dck::SM_BI) / 16); i += dck::THREADS)
+            reinterpret_cast<uint4 *>(sm + dck::SM_BI)[i] = make_uint4(0, 0, 0, 0);
+    load_state_tile(p.ws_kp + bhc(p, b, h, c) * N * PD, N, sm + dck::SM_KT, sm + dck::SM_KTL);
+    chunk_tokens(p, f32, b, h, t0, true);
+    chunk_mode_constants(p, f32);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_v = tbase;           // V^T (M=128), cols 0..63
+    const uint32_t t_g = tbase + 64u;     // G (M=64, lanes 0-15 per quarter) then D_i (M=128)
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) rev_raise_error(1);
+    if (__syncthreads_and(ok)) {
+        // ---- Bi tiles (own sub-block and later ones), hi + lo ------------------
+        {
+            const int t = tid & 63, grp = tid >> 6;
+            const int ib = t >> 4;
+            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+            const float ds = f32[F_S + t] - Sb;
+            const float sig = f32[F_SIG + t];
+            const unsigned char *sB = sm + dck::SM_B;
+#pragma unroll 1
+            for (int k = 0; k < NP / (8 * dck::RG); ++k) {
+                const int r0 = 8 * (grp + dck::RG * k);
+                if (r0 >= N) break;
+                float vBI[8], vBX[3][8], rb[8];
+                ld_rows8(sB, t, r0, rb);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const int r = r0 + j;
+                    const float b0 = rb[j], b1 = rb[j + 1];
+                    if (r < nr) {
+                        const int m0 = r, m1 = r + 1;
+                        const float bi0 = sig * b0 * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
+                        const float bi1 = sig * b1 * ex2_fast(fminf(-f32[F_A2 + m1] * ds, 120.f));
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
+#pragma unroll
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
+                            if (i2 < 4) {
+                                vBX[qq][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
+                                vBX[qq][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
+                            }
+                        }
+                    } else {
+                        const int m = nr + ((r - nr) >> 1);
+                        float sn, cs;
+                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m] * ds, 120.f));
+                        const float bi0 = eb * fmaf(b0, cs, b1 * sn);
+                        const float bi1 = eb * fmaf(b1, cs, -b0 * sn);
+                        vBI[j] = bi0;
+                        vBI[j + 1] = bi1;
+#pragma unroll
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const int i2 = ib + 1 + qq;
+                            if (i2 < 4)
+                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m],
+                                     f32[F_KIM + fslot(ib, i2) * NP + m], vBX[qq][j],
+                                     vBX[qq][j + 1]);
+                        }
+                    }
+                }
+                st16_split(sm + dck::SM_BI + bi_off(ib), sm + dck::SM_BIL + bi_off(ib),
+                           off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+#pragma unroll
+                for (int qq = 0; qq < 3; ++qq) {
+                    const int i2 = ib + 1 + qq;
+                    if (i2 < 4)
+                        st16_split(sm + dck::SM_BI + bi_off(i2), sm + dck::SM_BIL + bi_off(i2),
+                                   off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // ---- phase A: V^T = K_prev dY^T (hi + lo), G = dY X^T --------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sm + dck::SM_X), dy_base = smem_u32(sm + dck::SM_DY);
+            const uint32_t id_v = idesc_bf16(128, 64, false, false);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t kt_base = smem_u32(sm + (part ? dck::SM_KTL : dck::SM_KT));
+                for (int s = 0; s < PD / 16; ++s)
+                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
+            }
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int s = 0; s < PD / 16; ++s)
+                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
+            mma_commit(&bar_mma[0]);
+        }
+        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            // ---- masked G rows -> K-major tiles (N = 16 t of block i, K = s); dy_t . u_t
+            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
+                const int qd = warp - 4;
+                for (int i = 0; i < NSB; ++i) {
+                    float v[16];
+                    tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
+                    if (lane < 16 && i <= qd) {
+                        const int t = 16 * qd + lane;
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
+                            hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
+                        }
+                        unsigned char *gt = sm + dck::SM_GM + qd * 2048;
+                        unsigned char *gl = sm + dck::SM_GML + qd * 2048;
+                        st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
+                        st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
+                        if (i == qd) {
+                            float dg = 0.f;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (j == lane) dg = v[j];
+                            f32[F_CORR + t] = dg;   // <dy_t, u_t>
+                        }
+                    }
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+
+            // ---- phase B: D_i = Bi^T (G o mask)_i^T into the (now free) G columns
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t id_d = idesc_bf16(128, 16, true, false);
+                // hi*hi + hi*lo + lo*hi
+                const uint32_t a_off[3] = {dck::SM_BI, dck::SM_BI, dck::SM_BIL};
+                const uint32_t b_off[3] = {dck::SM_GM, dck::SM_GML, dck::SM_GM};
+                for (int i = 0; i < NSB; ++i)
+                    for (int part = 0; part < 3; ++part) {
+                        const uint32_t bi_base = smem_u32(sm + a_off[part]);
+                        const uint32_t gm_base = smem_u32(sm + b_off[part]);
+                        for (int s = 0; s <= i; ++s)
+                            mma_bf16(t_g + 16 * i,
+                                     sdesc(bi_base + bi_off(i) + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                                     sdesc(gm_base + i * 2048u + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                                     id_d, part > 0 || s > 0);
+                    }
+                mma_commit(&bar_mma[1]);
+            }
+            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
+            if (!ok) rev_raise_error(1);
+            fence_after_sync();
+            if (__syncthreads_and(ok)) {
+                // ---- unfold: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D ;
+                //      dC_t = dCK_t - beta' (dy.u) B_t
+                const int n = tid & 127, tq = tid >> 7, qd = warp & 3;
+                const bool valid = n < N;
+                const int m = n < nr ? n : nr + ((n - nr) >> 1);
+                const bool pr_row = valid && n >= nr;
+                const bool im_row = pr_row && ((n - nr) & 1);
+                const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
+                float *dst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+                const long long tstride = (long long)p.H * p.N;
+                const unsigned char *sB = sm + dck::SM_B;
+#pragma unroll
+                for (int c16 = 0; c16 < dck::TPT / 16; ++c16) {
+                    const int tc = dck::TPT * tq + 16 * c16;
+                    float vv[16], dd[16];
+                    tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
+                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), dd);
+                    const int ib = tc >> 4;
+                    const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
+                    // E = E' conj(G_i) = E' F[0][i]
+                    float fr = 1.f, fi = 0.f;
+                    if (ib && valid) {
+                        fr = f32[F_KRE + gslot(ib) * NP + m];
+                        fi = -f32[F_KIM + gslot(ib) * NP + m];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = tc + j;
+                        const float ds = f32[F_S + t] - Sb;
+                        const float mag = ex2_fast(a2 * ds);
+                        float er = mag, ei = 0.f;
+                        if (pr_row) {
+                            float sn, cs;
+                            __sincosf(w * ds, &sn, &cs);
+                            er = mag * cs;
+                            ei = mag * sn;
+                        }
+                        float Er, Ei;
+                        cmul(er, ei, fr, fi, Er, Ei);
+                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                        const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
+                        float res;
+                        if (!pr_row)
+                            res = fmaf(Er, vv[j], er * dd[j]);
+                        else if (!im_row)   // real part of E (V_re + i V_im) + E' (D_re + i D_im)
+                            res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
+                        else                // imaginary part
+                            res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
+                        if (valid && t0 + t < L) {
+                            const float bt = ld_row1(sB, t, n);
+                            dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
+                        }
+                    }
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, dck::TMEM_COLS);
+    }
+}
+
 }  // namespace chunkrev
 
 // ---------------------------------------------------------------------------
@@ -1144,9 +1314,29 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
     return e;
 }
 
+cudaError_t chunk_states(const Params &p, cudaStream_t st);
+
+// Forward-direction part of the tensor-core backward: the state entering every
+// chunk (p.ws_kp, p.ws_ce), then the per-head dC of every chunk (p.ws_dC).
+cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st) {
+    using namespace chunkrev;
+    cudaError_t e = chunk_states(p, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mx, mb, mdy;
+    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
+        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
+        !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
+        return cudaErrorInvalidValue;
+    static bool a = false;
+    if ((e = set_smem(k_chunk_bwd_dc, dck::SMEM_BYTES, a)) != cudaSuccess) return e;
+    k_chunk_bwd_dc<<<dim3(p.nc, p.H, p.Bsz), dck::THREADS, dck::SMEM_BYTES, st>>>(mx, mb, mdy, p);
+    profile_mark(st, "k_chunk_bwd_dc");
+    return cudaGetLastError();
+}
+
 // Reverse part of the tensor-core backward: dx, gbu / dsigma / <dy, u>, the
-// exact chunk-boundary values, dh0 / dw0 / dbeta_0.  Needs p.ws_gc, p.ws_ce,
-// p.ws_kb (written by the forward-direction part), p.ws_qb.
+// exact chunk-boundary values, dh0 / dw0 / dbeta_0.  Needs p.ws_gc, p.ws_ce and
+// p.ws_kp (written by the forward-direction part) and p.ws_qb.
 cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     using namespace chunkrev;
     CUtensorMap mx, mb, mc, mdy;

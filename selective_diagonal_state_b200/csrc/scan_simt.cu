@@ -581,51 +581,6 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
                                lane_in_s);
             float cf[NS];
             ld_slots<NS>(cf, s.coef + (ln.hc * T + tt) * NSL + ln.q * NS);
-            // at a 64-token chunk start: per row, sum_p conj(Gbar_t) A_t K_{t-1} from the saved
-            // chunk-end state (the exact carry of the decay-gradient scan)
-            const int tg = t0 + tt;
-            if (p.ws_qb && tg > 0 && (tg & 63) == 0) {
-                const int cc = tg >> 6;
-                const float *kb = p.ws_kb + (((long long)ln.b * p.H + (ln.hv ? ln.h : 0)) * p.nc +
-                                             (cc - 1)) * (long long)p.N * p.P;
-                float kv[NS];
-#pragma unroll
-                for (int sl = 0; sl < NS; ++sl) {
-                    const int n = row_of<NR, NPR>(ln.q, sl, p.nr, p.np, NQ);
-                    kv[sl] = (ln.hv && n >= 0 && ln.pl < p.P) ? kb[(long long)n * p.P + ln.pl] : 0.f;
-                }
-                float qv[NS];
-#pragma unroll
-                for (int i = 0; i < NR; ++i) qv[i] = Gv[i] * cf[i] * kv[i];
-#pragma unroll
-                for (int j = 0; j < NPR; ++j) {
-                    const float ec = cf[NR + 2 * j], es = cf[NR + 2 * j + 1];
-                    const float kr = kv[NR + 2 * j], ki = kv[NR + 2 * j + 1];
-                    const float ar = fmaf(ec, kr, -es * ki), ai = fmaf(es, kr, ec * ki);
-                    const float gr = Gv[NR + 2 * j], gi = Gv[NR + 2 * j + 1];
-                    qv[NR + 2 * j] = fmaf(gr, ar, gi * ai);
-                    qv[NR + 2 * j + 1] = fmaf(gr, ai, -gi * ar);
-                }
-                xreduce<NS, S>(qv, lane_in_s);
-                if (ln.hv) {
-                    float *dst = p.ws_qb + ((((long long)ln.b * p.H + ln.h) * p.nc + cc) * 4 + wp) *
-                                               (long long)p.N;
-                    if constexpr (NS >= S) {
-                        constexpr int KS = NS / S;
-#pragma unroll
-                        for (int i = 0; i < KS; ++i) {
-                            const int n = row_of<NR, NPR>(ln.q, lane_in_s * KS + i, p.nr, p.np, NQ);
-                            if (n >= 0) dst[n] = qv[i];
-                        }
-                    } else {
-                        constexpr int SK = S / NS;
-                        if (lane_in_s % SK == 0) {
-                            const int n = row_of<NR, NPR>(ln.q, lane_in_s / SK, p.nr, p.np, NQ);
-                            if (n >= 0) dst[n] = qv[0];
-                        }
-                    }
-                }
-            }
             // G <- A_t^T G
             step_adj<NR, NPR>(Gv, cf);
         }

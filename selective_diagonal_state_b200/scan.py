@@ -77,12 +77,17 @@ def alloc_fwd(shape: ScanShape, device="cuda"):
     return y, hT, wT
 
 
-def scan_forward(shape: ScanShape, dev: DeviceInputs, out=None, desc=None, stream=None):
-    """Run ``ssm_scan_fwd``; returns (y, hT, last_write)."""
+def scan_forward(shape: ScanShape, dev: DeviceInputs, out=None, desc=None, stream=None,
+                 workspace=None):
+    """Run ``ssm_scan_fwd``; returns (y, hT, last_write).  ``workspace`` is a
+    (tensor, bytes) pair from ``alloc_workspace(shape, PASS_FWD)``; allocated
+    here when not given."""
     desc = desc or abi.make_desc(shape)
     y, hT, wT = out if out is not None else alloc_fwd(shape, dev.x.device)
+    ws, nbytes = workspace if workspace is not None else alloc_workspace(
+        shape, abi.PASS_FWD, dev.x.device, desc)
     abi.ssm_scan_fwd(desc, dev.x, dev.dt, dev.A_log, dev.theta, dev.Bm, dev.Cm, dev.D, dev.lam,
-                     dev.h0, dev.w0, y, hT, wT, None, 0, stream)
+                     dev.h0, dev.w0, y, hT, wT, ws, nbytes, stream)
     return y, hT, wT
 
 

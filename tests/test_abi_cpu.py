@@ -55,7 +55,13 @@ def test_contiguous_strides(lib):
 def test_workspace_size(lib):
     sh = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=100)
     d = abi.make_desc(sh)
-    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+    # tensor-core chain: the state entering every 64-token chunk + chunk decays
+    nc = (100 + 63) // 64
+    nf = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
+    assert nf >= 2 * 32 * nc * (128 * 64 + 128 * 2) * 4 and nf % 256 == 0
+    # the recurrent chain needs none
+    for kw in (dict(chunk=1), dict(dtype_io=S.DTYPE_F32), dict(headdim=32)):
+        assert abi.ssm_scan_workspace_size(abi.make_desc(sh.replace(**kw)), abi.PASS_FWD) == 0
     n = abi.ssm_scan_workspace_size(d, abi.PASS_BWD)
     BLH = 2 * 100 * 32
     assert n >= BLH * (2 * 128 + 2 + 1) * 4
