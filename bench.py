@@ -309,7 +309,7 @@ def main():
 
     def step():
         scan.scan_forward(shape, dev, out=fwd_out, desc=desc, workspace=wsf)
-        scan.scan_backward(shape, dev, grads=grads, workspace=ws, desc=desc)
+        scan.scan_backward(shape, dev, grads=grads, workspace=ws, desc=desc, saved=wsf)
         allreduce_params()
 
     for _ in range(max(3, args.warmup)):

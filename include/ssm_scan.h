@@ -150,6 +150,27 @@ SSM_API int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, con
                  size_t workspace_bytes, void *stream);
 
 /*
+ * Backward that reuses the forward's chunk states: identical to ssm_scan_bwd,
+ * except that fwd_workspace is the workspace of a preceding ssm_scan_fwd call
+ * with the same descriptor and the same inputs (x, dt, A_log, theta, B, lambda,
+ * h0, prev_write), left unchanged since.  The tensor-core backward then reads
+ * the states entering every 64-token chunk from it instead of recomputing them
+ * (the training step "forward saving chunk states, then backward").  For
+ * descriptors whose forward needs no workspace it behaves as ssm_scan_bwd.
+ * Reading a workspace from other inputs gives wrong gradients; nothing checks
+ * it.  fwd_workspace must not be NULL and must hold
+ * ssm_scan_workspace_size(d, SSM_PASS_FWD) bytes, 256-byte aligned.
+ */
+SSM_API int ssm_scan_bwd_saved(const ssm_desc_t *d, const void *x, const void *dt,
+                               const float *A_log, const float *theta, const void *B,
+                               const void *C, const float *D, const void *lambda,
+                               const float *h0, const float *prev_write, const void *dy, void *dx,
+                               void *ddt, float *dA_log, float *dtheta, void *dB, void *dC,
+                               float *dD, void *dlambda, float *dh0, float *dprev_write,
+                               const void *fwd_workspace, size_t fwd_workspace_bytes,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Allocation-free backward (no counterpart in the paper; a library service).
  * Same inputs, outputs and results as ssm_scan_bwd, but it takes no
  * workspace: its scratch is a fixed 32 MiB array inside the library

@@ -24,7 +24,7 @@ PASS_FWD, PASS_BWD = 0, 1
 EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
-            "ssm_scan_bwd_noalloc", "ssm_scan_last_route"]
+            "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved"]
 ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -74,6 +74,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_scan_bwd.restype = ctypes.c_int
     lib.ssm_scan_bwd_noalloc.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 21 + [_vp]
     lib.ssm_scan_bwd_noalloc.restype = ctypes.c_int
+    lib.ssm_scan_bwd_saved.argtypes = ([ctypes.POINTER(Desc)] + [_vp] * 22 +
+                                       [ctypes.c_size_t, _vp, ctypes.c_size_t, _vp])
+    lib.ssm_scan_bwd_saved.restype = ctypes.c_int
     lib.ssm_scan_last_error.argtypes = []
     lib.ssm_scan_last_error.restype = ctypes.c_char_p
     lib.ssm_scan_poll_device_error.argtypes = [_vp]
@@ -151,6 +154,20 @@ def ssm_scan_bwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, 
         x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt, dA_log, dtheta, dB, dC,
         dD, dlam, dh0, dprev_write, workspace)], workspace_bytes, _stream(stream))
     _check(rc, "ssm_scan_bwd")
+
+
+def ssm_scan_bwd_saved(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx,
+                       ddt, dA_log, dtheta, dB, dC, dD, dlam=None, dh0=None, dprev_write=None,
+                       fwd_workspace=None, fwd_workspace_bytes: int = 0, workspace=None,
+                       workspace_bytes: int = 0, stream=None) -> None:
+    """Backward reading the chunk states from the workspace of a preceding
+    forward on the same inputs."""
+    lib = load_library()
+    rc = lib.ssm_scan_bwd_saved(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt, dA_log, dtheta, dB, dC,
+        dD, dlam, dh0, dprev_write, fwd_workspace)], fwd_workspace_bytes, _ptr(workspace),
+        workspace_bytes, _stream(stream))
+    _check(rc, "ssm_scan_bwd_saved")
 
 
 def ssm_scan_bwd_noalloc(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx,

@@ -365,12 +365,16 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     return SSM_OK;
 }
 
-int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
-                 const float *theta, const void *B, const void *C, const float *D,
-                 const void *lambda, const float *h0, const float *prev_write, const void *dy,
-                 void *dx, void *ddt, float *dA_log, float *dtheta, void *dB, void *dC,
-                 float *dD, void *dlambda, float *dh0, float *dprev_write, void *workspace,
-                 size_t workspace_bytes, void *stream) {
+namespace {
+// Backward of both entry points; `saved` (may be NULL) is the workspace of a
+// forward call with the same descriptor and inputs, whose chunk states are
+// then read instead of recomputed.
+int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+             const float *theta, const void *B, const void *C, const float *D, const void *lambda,
+             const float *h0, const float *prev_write, const void *dy, void *dx, void *ddt,
+             float *dA_log, float *dtheta, void *dB, void *dC, float *dD, void *dlambda,
+             float *dh0, float *dprev_write, const void *saved, size_t saved_bytes,
+             void *workspace, size_t workspace_bytes, void *stream) {
     int rc = validate_desc(d);
     if (rc) return rc;
     const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
@@ -402,6 +406,17 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         return fail(SSM_ERR_WORKSPACE, "backward needs %zu bytes of workspace, got %zu",
                     lay.total, workspace ? workspace_bytes : (size_t)0);
     if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+    if (saved) {
+        const size_t need = fwd_layout(d).total;
+        if (need == 0) {
+            saved = nullptr;  // the recurrent kernels save nothing
+        } else if (saved_bytes < need) {
+            return fail(SSM_ERR_WORKSPACE, "saved forward workspace needs %zu bytes, got %zu",
+                        need, saved_bytes);
+        } else if ((uintptr_t)saved % 256) {
+            return fail(SSM_ERR_ALIGN, "saved forward workspace is not 256-byte aligned");
+        }
+    }
     ssm::Params p;
     fill_params(d, p);
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
@@ -435,6 +450,13 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         pc.ws_qb = (float *)(ws + lay.off_qb);
         pc.ws_gc = (float *)(ws + lay.off_gc);
         pc.ws_ce = (float *)(ws + lay.off_ce);
+        if (saved) {
+            // read-only here: the forward wrote them
+            const FwdWs fl = fwd_layout(d);
+            pc.ws_kp = (float *)((const char *)saved + fl.off_kp);
+            pc.ws_ce = (float *)((const char *)saved + fl.off_ce);
+            pc.states_ready = 1;
+        }
         pc.gate = gate;
         pc.gate_on = 0;
         if (e == cudaSuccess) e = ssm::chunk_backward(pc, st);
@@ -453,6 +475,33 @@ int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
     g_last_error.clear();
     return SSM_OK;
+}
+
+}  // namespace
+
+int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, const void *dy,
+                 void *dx, void *ddt, float *dA_log, float *dtheta, void *dB, void *dC,
+                 float *dD, void *dlambda, float *dh0, float *dprev_write, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    return bwd_impl(d, x, dt, A_log, theta, B, C, D, lambda, h0, prev_write, dy, dx, ddt, dA_log,
+                    dtheta, dB, dC, dD, dlambda, dh0, dprev_write, nullptr, 0, workspace,
+                    workspace_bytes, stream);
+}
+
+int ssm_scan_bwd_saved(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                       const float *theta, const void *B, const void *C, const float *D,
+                       const void *lambda, const float *h0, const float *prev_write,
+                       const void *dy, void *dx, void *ddt, float *dA_log, float *dtheta,
+                       void *dB, void *dC, float *dD, void *dlambda, float *dh0,
+                       float *dprev_write, const void *fwd_workspace,
+                       size_t fwd_workspace_bytes, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+    if (!fwd_workspace) return fail(SSM_ERR_ARG, "ssm_scan_bwd_saved: fwd_workspace is NULL");
+    return bwd_impl(d, x, dt, A_log, theta, B, C, D, lambda, h0, prev_write, dy, dx, ddt, dA_log,
+                    dtheta, dB, dC, dD, dlambda, dh0, dprev_write, fwd_workspace,
+                    fwd_workspace_bytes, workspace, workspace_bytes, stream);
 }
 
 const char *ssm_scan_last_error(void) { return g_last_error.c_str(); }

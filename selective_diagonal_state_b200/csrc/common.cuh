@@ -48,6 +48,8 @@ struct Params {
     // only when (*gate != 0) == gate_on (no gate: always)
     const int *gate;
     int gate_on;
+    // the backward takes ws_kp / ws_ce as written by the forward (not recomputed)
+    int states_ready;
     Geometry geo;
 };
 

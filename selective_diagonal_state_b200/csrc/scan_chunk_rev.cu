@@ -1317,10 +1317,11 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
 cudaError_t chunk_states(const Params &p, cudaStream_t st);
 
 // Forward-direction part of the tensor-core backward: the state entering every
-// chunk (p.ws_kp, p.ws_ce), then the per-head dC of every chunk (p.ws_dC).
+// chunk (p.ws_kp, p.ws_ce; taken from the forward when p.states_ready), then the
+// per-head dC of every chunk (p.ws_dC).
 cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st) {
     using namespace chunkrev;
-    cudaError_t e = chunk_states(p, st);
+    cudaError_t e = p.states_ready ? cudaSuccess : chunk_states(p, st);
     if (e != cudaSuccess) return e;
     CUtensorMap mx, mb, mdy;
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||

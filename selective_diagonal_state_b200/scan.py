@@ -135,13 +135,20 @@ def alloc_workspace(shape: ScanShape, pass_: int, device="cuda", desc=None):
 
 
 def scan_backward(shape: ScanShape, dev: DeviceInputs, grads=None, workspace=None, desc=None,
-                  stream=None) -> Grads:
-    """Run ``ssm_scan_bwd`` for ``dev.dy``; returns the gradient buffers."""
+                  stream=None, saved=None) -> Grads:
+    """Run ``ssm_scan_bwd`` for ``dev.dy``; returns the gradient buffers.  With
+    ``saved`` = the (tensor, bytes) forward workspace of a preceding
+    ``scan_forward`` on the same inputs, ``ssm_scan_bwd_saved`` reuses its
+    chunk states."""
     desc = desc or abi.make_desc(shape)
     g = grads or alloc_bwd(shape, dev.x.device)
     ws, nbytes = workspace if workspace is not None else alloc_workspace(
         shape, abi.PASS_BWD, dev.x.device, desc)
-    abi.ssm_scan_bwd(desc, dev.x, dev.dt, dev.A_log, dev.theta, dev.Bm, dev.Cm, dev.D, dev.lam,
-                     dev.h0, dev.w0, dev.dy, g.dx, g.ddt, g.dA_log, g.dtheta, g.dBm, g.dCm, g.dD,
-                     g.dlam, g.dh0, g.dw0, ws, nbytes, stream)
+    args = (desc, dev.x, dev.dt, dev.A_log, dev.theta, dev.Bm, dev.Cm, dev.D, dev.lam, dev.h0,
+            dev.w0, dev.dy, g.dx, g.ddt, g.dA_log, g.dtheta, g.dBm, g.dCm, g.dD, g.dlam, g.dh0,
+            g.dw0)
+    if saved is not None and saved[0] is not None:
+        abi.ssm_scan_bwd_saved(*args, saved[0], saved[1], ws, nbytes, stream)
+    else:
+        abi.ssm_scan_bwd(*args, ws, nbytes, stream)
     return g

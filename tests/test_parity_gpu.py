@@ -267,3 +267,30 @@ def test_moderate_decay_stays_chunked():
     f = 60.0 / (a_max * np.log2(np.e) * span)
     inp = _scaled_dt(shape, inp, f)
     check_all(shape, inp, route=abi.ROUTE_CHUNKED)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(seqlen=64), dict(seqlen=1),
+                                dict(decay_mode=S.DECAY_PER_HEAD, two_endpoint=0, n_real=128,
+                                     n_pairs=0, ngroups=2)])
+def test_backward_from_saved_states(kw):
+    """The backward that reads the forward's chunk states gives the same
+    gradients as the one that recomputes them (bit for bit), and the oracle's."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=150, nheads=4, ngroups=4).replace(**kw)
+    inp = S.make_inputs(shape, seed=47, with_state=True)
+    dev = scan.to_device(shape, inp)
+    wsf = scan.alloc_workspace(shape, abi.PASS_FWD)
+    scan.scan_forward(shape, dev, workspace=wsf)
+    g_saved = scan.scan_backward(shape, dev, saved=wsf)
+    assert abi.ssm_scan_last_route() == expected_route(shape)
+    g_plain = scan.scan_backward(shape, dev)
+    torch.cuda.synchronize()
+    abi.ssm_scan_poll_device_error()
+    for name in ("dx", "ddt", "dBm", "dCm", "dA_log", "dD", "dh0", "dw0", "dtheta", "dlam"):
+        a, b = getattr(g_saved, name), getattr(g_plain, name)
+        if a is not None:
+            assert torch.equal(a, b), name
+    gr = oracle.scan_bwd(shape, inp, inp["dy"])
+    dt = shape.dtype_io
+    compare("dx", to_np(g_saved.dx), gr["dx"], dt)
+    compare("dA_log", to_np(g_saved.dA_log), gr["dA_log"], dt)
+    compare("ddt", to_np(g_saved.ddt), gr["ddt"], dt)
