@@ -63,7 +63,9 @@ enum ssm_status {
 
 enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 };
 enum ssm_decay_mode { SSM_DECAY_PER_HEAD = 0, SSM_DECAY_PER_COORD = 1 };
-enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1 };
+/* SSM_PASS_FWD: a forward that keeps what ssm_scan_bwd_saved reads;
+ * SSM_PASS_FWD_INFER: a forward only (smaller workspace). */
+enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1, SSM_PASS_FWD_INFER = 2 };
 
 /*
  * Problem descriptor.  Tensor layouts (innermost last):
@@ -109,9 +111,12 @@ typedef struct ssm_desc {
 SSM_API void ssm_desc_set_contiguous(ssm_desc_t *d);
 
 /*
- * Bytes of device workspace that ssm_scan_fwd (pass = SSM_PASS_FWD) or
- * ssm_scan_bwd (pass = SSM_PASS_BWD) needs for this descriptor; 0 means the
- * workspace pointer may be NULL.  Returns 0 for an invalid descriptor (the
+ * Bytes of device workspace that ssm_scan_fwd (pass = SSM_PASS_FWD for a
+ * training forward whose workspace a later ssm_scan_bwd_saved reads;
+ * SSM_PASS_FWD_INFER for a forward alone, which is all ssm_scan_fwd requires)
+ * or ssm_scan_bwd (pass = SSM_PASS_BWD) needs for this descriptor; 0 means
+ * the workspace pointer may be NULL.  ssm_scan_fwd given at least the
+ * SSM_PASS_FWD size also writes the per-chunk products the backward reuses.  Returns 0 for an invalid descriptor (the
  * compute call then reports the error).  The workspace must be 256-byte
  * aligned; its contents need not be initialised and are clobbered.
  */
@@ -159,7 +164,8 @@ SSM_API int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, con
  * descriptors whose forward needs no workspace it behaves as ssm_scan_bwd.
  * Reading a workspace from other inputs gives wrong gradients; nothing checks
  * it.  fwd_workspace must not be NULL and must hold
- * ssm_scan_workspace_size(d, SSM_PASS_FWD) bytes, 256-byte aligned.
+ * ssm_scan_workspace_size(d, SSM_PASS_FWD) bytes (a training forward),
+ * 256-byte aligned.
  */
 SSM_API int ssm_scan_bwd_saved(const ssm_desc_t *d, const void *x, const void *dt,
                                const float *A_log, const float *theta, const void *B,

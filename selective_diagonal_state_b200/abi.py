@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libssm_scan.so")
 SSM_OK = 0
 STATUS = {0: "SSM_OK", -1: "SSM_ERR_ARG", -2: "SSM_ERR_UNSUPPORTED", -3: "SSM_ERR_ALIGN",
           -4: "SSM_ERR_CUDA", -5: "SSM_ERR_TIMEOUT", -6: "SSM_ERR_WORKSPACE"}
-PASS_FWD, PASS_BWD = 0, 1
+PASS_FWD, PASS_BWD, PASS_FWD_INFER = 0, 1, 2
 
 EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",

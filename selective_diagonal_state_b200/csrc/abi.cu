@@ -185,18 +185,29 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
 
 // Forward workspace of the tensor-core chain: the state entering every
 // 64-token chunk [B][H][L/64][N][P] and the chunk decays [B][H][L/64][128][2].
+// A training forward (workspace of `total` bytes) also keeps, per chunk, the
+// masked score tiles (8 KB), the chunk-end folded B tile (16 KB) and the
+// diagonal correction (64 floats) for ssm_scan_bwd_saved; an inference forward
+// needs only the first `total_infer` bytes.
 struct FwdWs {
-    size_t off_kp, off_ce, total;
+    size_t off_kp, off_ce, off_P, off_Bh, off_corr, total_infer, total;
 };
 FwdWs fwd_layout(const ssm_desc_t *d) {
     FwdWs w;
-    w.off_kp = w.off_ce = w.total = 0;
+    w.off_kp = w.off_ce = w.off_P = w.off_Bh = w.off_corr = w.total_infer = w.total = 0;
     if (!tensor_chain_shape(d)) return w;
-    const size_t ntb = (size_t)(d->seqlen + 63) / 64;
+    const size_t units = (size_t)d->batch * d->nheads * (size_t)((d->seqlen + 63) / 64);
     w.off_kp = 0;
-    size_t off = align256((size_t)d->batch * d->nheads * ntb * nstate(d) * d->headdim * 4);
+    size_t off = align256(units * nstate(d) * d->headdim * 4);
     w.off_ce = off;
-    off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * 2 * 4);
+    off = align256(off + units * 128 * 2 * 4);
+    w.total_infer = off;
+    w.off_P = off;
+    off = align256(off + units * 8192);
+    w.off_Bh = off;
+    off = align256(off + units * 16384);
+    w.off_corr = off;
+    off = align256(off + units * 64 * 4);
     w.total = off;
     return w;
 }
@@ -294,6 +305,8 @@ void ssm_desc_set_contiguous(ssm_desc_t *d) {
 size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
     if (validate_desc(d) != SSM_OK) return 0;
     if (pass == SSM_PASS_FWD) return (d->batch == 0 || d->seqlen == 0) ? 0 : fwd_layout(d).total;
+    if (pass == SSM_PASS_FWD_INFER)
+        return (d->batch == 0 || d->seqlen == 0) ? 0 : fwd_layout(d).total_infer;
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
     return bwd_layout(d).total;
@@ -323,13 +336,20 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     cudaStream_t st = (cudaStream_t)stream;
     if (chunked) {
         const FwdWs lay = fwd_layout(d);
-        if (!workspace || workspace_bytes < lay.total)
-            return fail(SSM_ERR_WORKSPACE, "forward needs %zu bytes of workspace, got %zu",
-                        lay.total, workspace ? workspace_bytes : (size_t)0);
+        if (!workspace || workspace_bytes < lay.total_infer)
+            return fail(SSM_ERR_WORKSPACE,
+                        "forward needs %zu bytes of workspace (%zu to save for the backward), got %zu",
+                        lay.total_infer, lay.total, workspace ? workspace_bytes : (size_t)0);
         if ((uintptr_t)workspace % 256)
             return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
-        p.ws_kp = (float *)((char *)workspace + lay.off_kp);
-        p.ws_ce = (float *)((char *)workspace + lay.off_ce);
+        char *ws = (char *)workspace;
+        p.ws_kp = (float *)(ws + lay.off_kp);
+        p.ws_ce = (float *)(ws + lay.off_ce);
+        if (workspace_bytes >= lay.total) {  // training forward: keep the products for the backward
+            p.sv_P = (unsigned char *)(ws + lay.off_P);
+            p.sv_Bh = (unsigned char *)(ws + lay.off_Bh);
+            p.sv_corr = (float *)(ws + lay.off_corr);
+        }
         p.nc = (int)((d->seqlen + 63) / 64);
     }
     profile_begin(st);
@@ -453,8 +473,12 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
         if (saved) {
             // read-only here: the forward wrote them
             const FwdWs fl = fwd_layout(d);
-            pc.ws_kp = (float *)((const char *)saved + fl.off_kp);
-            pc.ws_ce = (float *)((const char *)saved + fl.off_ce);
+            const char *sv = (const char *)saved;
+            pc.ws_kp = (float *)(sv + fl.off_kp);
+            pc.ws_ce = (float *)(sv + fl.off_ce);
+            pc.sv_P = (unsigned char *)(sv + fl.off_P);
+            pc.sv_Bh = (unsigned char *)(sv + fl.off_Bh);
+            pc.sv_corr = (float *)(sv + fl.off_corr);
             pc.states_ready = 1;
         }
         pc.gate = gate;

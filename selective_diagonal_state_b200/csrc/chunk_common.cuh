@@ -96,21 +96,30 @@ __device__ __forceinline__ void cmul(float a, float b, float c, float d, float &
 }
 
 // ---- per-chunk token quantities and mode constants ----------------------------
-// Loads dt / lambda of tokens t0 .. t0+64 and writes the inclusive prefix S_t
-// (F_S) and, with `want_sigma`, sigma_t (F_SIG) and beta_{t+1} (F_BN).
-// Call with all threads of the block (>= 96); contains barriers.
-__device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b, int h, int t0,
-                                             bool want_sigma) {
+// One chunk's dt / lambda of tokens t0 .. t0+64, held in registers of threads
+// 0..64 between the load and the use (so that a persistent kernel can fetch
+// the next chunk's while it works on this one).
+struct TokPrefetch {
+    float dv, lv;
+};
+__device__ __forceinline__ TokPrefetch tok_load(const Params &p, int b, int h, int t0) {
+    TokPrefetch r{0.f, 1.f};
+    const int i = threadIdx.x, t = t0 + i;
+    if (i < Q + 1 && t < p.L) {
+        r.dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+        if (p.two_ep) r.lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+    }
+    return r;
+}
+// Writes the inclusive prefix S_t (F_S) and, with `want_sigma`, sigma_t (F_SIG)
+// and beta_{t+1} (F_BN) from prefetched dt / lambda.  Call with all threads of
+// the block (>= 96); contains barriers.
+__device__ __forceinline__ void chunk_tokens_from(const Params &p, float *f32, int t0,
+                                                  const TokPrefetch &r, bool want_sigma) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < Q + 1; i += blockDim.x) {
-        const int t = t0 + i;
-        float dv = 0.f, lv = 1.f;
-        if (t < p.L) {
-            dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
-            if (p.two_ep) lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
-        }
-        f32[F_DT + i] = dv;
-        f32[F_LAM + i] = lv;
+    if (tid < Q + 1) {
+        f32[F_DT + tid] = r.dv;
+        f32[F_LAM + tid] = r.lv;
     }
     __syncthreads();
     if (warp == 0) {
@@ -132,6 +141,12 @@ __device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b,
         f32[F_BN + t] = bn;
     }
     __syncthreads();
+}
+// Loads dt / lambda of tokens t0 .. t0+64 and writes F_S (and F_SIG, F_BN).
+__device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b, int h, int t0,
+                                             bool want_sigma) {
+    const TokPrefetch r = tok_load(p, b, h, t0);
+    chunk_tokens_from(p, f32, t0, r, want_sigma);
 }
 
 // Per-mode decay over each sub-block, E_k = e^{lam dS_k}, and the products
@@ -220,6 +235,58 @@ __device__ __forceinline__ void load_state_tile(const float *src, int N, unsigne
         else
             st16(hi, off, v);
     }
+}
+
+// A state-shaped fp32 tile [n][64 p] held in registers between its global
+// load and its store as a bf16 operand (the load_state_tile layout), so that a
+// persistent kernel can fetch the next chunk's tile while it works on this one.
+template <int THREADS>
+struct StatePrefetch {
+    static constexpr int ITEMS = NP * (PD / 8) / THREADS;
+    float4 v[2 * ITEMS];
+};
+template <int THREADS>
+__device__ __forceinline__ void state_load(const float *src, int N, StatePrefetch<THREADS> &r) {
+#pragma unroll
+    for (int j = 0; j < StatePrefetch<THREADS>::ITEMS; ++j) {
+        const int it = threadIdx.x + j * THREADS;
+        const int n = it >> 3, p8 = (it & 7) * 8;
+        if (n < N) {
+            r.v[2 * j] = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8));
+            r.v[2 * j + 1] = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8 + 4));
+        } else {
+            r.v[2 * j] = r.v[2 * j + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+}
+template <int THREADS>
+__device__ __forceinline__ void state_store(const StatePrefetch<THREADS> &r, unsigned char *hi,
+                                            unsigned char *lo) {
+#pragma unroll
+    for (int j = 0; j < StatePrefetch<THREADS>::ITEMS; ++j) {
+        const int it = threadIdx.x + j * THREADS;
+        const int n = it >> 3, p8 = (it & 7) * 8;
+        const float4 a = r.v[2 * j], d = r.v[2 * j + 1];
+        const float v[8] = {a.x, a.y, a.z, a.w, d.x, d.y, d.z, d.w};
+        const uint32_t off = off_kmaj(n, p8, 128u, 1024u);
+        if (lo)
+            st16_split(hi, lo, off, v);
+        else
+            st16(hi, off, v);
+    }
+}
+
+// Work item of the persistent chunk kernels: chunk fastest, then head, then batch row.
+struct ChunkItem {
+    int c, h, b;
+};
+__device__ __forceinline__ ChunkItem chunk_item(const Params &p, int item) {
+    ChunkItem r;
+    r.c = item % p.nc;
+    const int rest = item / p.nc;
+    r.h = rest % p.H;
+    r.b = rest / p.H;
+    return r;
 }
 
 // ---- host side ---------------------------------------------------------------

@@ -50,6 +50,10 @@ struct Params {
     int gate_on;
     // the backward takes ws_kp / ws_ce as written by the forward (not recomputed)
     int states_ready;
+    // per-chunk products a training forward saves for the backward (null: not saved):
+    unsigned char *sv_P;    // [B][H][NC] 8 KB: masked scores P^T as bf16 operand tiles
+    unsigned char *sv_Bh;   // [B][H][NC] 16 KB: chunk-end folded B (bf16 operand tile)
+    float *sv_corr;         // [B][H][NC][64] D - beta_{t+1} C_t . B_t
     Geometry geo;
 };
 

@@ -117,10 +117,16 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const float ds = f32[F_S + t] - Sb;
         const float sig = f32[F_SIG + t];
         const unsigned char *sB = sm + stl::SM_B;
+        unsigned char *sv = p.sv_Bh ? p.sv_Bh + bhc(p, b, h, c) * 16384 : nullptr;
 #pragma unroll 1
         for (int k = 0; k < 8; ++k) {
             const int r0 = 8 * (grp + 2 * k);
-            if (r0 >= N) break;
+            if (r0 >= N) {
+                if (!sv) break;
+                // K padding of the saved tile
+                *reinterpret_cast<uint4 *>(sv + off_mnmaj(r0, t, 2048u, 128u)) = make_uint4(0, 0, 0, 0);
+                continue;
+            }
             float rb[8], v[8];
             ld_rows8(sB, t, r0, rb);
 #pragma unroll
@@ -143,6 +149,14 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
             }
             st16_split(sm + stl::SM_BH, sm + stl::SM_BHL, off_mnmaj(r0, t, 2048u, 128u), v);
+            if (sv) {  // the bf16 tile (hi part) for the backward's dx
+                uint4 w;
+                w.x = pack_bf16(v[0], v[1]);
+                w.y = pack_bf16(v[2], v[3]);
+                w.z = pack_bf16(v[4], v[5]);
+                w.w = pack_bf16(v[6], v[7]);
+                *reinterpret_cast<uint4 *>(sv + off_mnmaj(r0, t, 2048u, 128u)) = w;
+            }
         }
         fence_proxy_async();
         fence_before_sync();
@@ -309,66 +323,82 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 // ============================================================================
 // k_chunk_out: per chunk, y_t = readout of the state entering the chunk
 // + masked in-chunk scores x + (D - beta_{t+1} C_t . B_t) u_t.
+// Persistent: one CTA per SM walks the chunks with a stride of the grid; the
+// next chunk's tiles (TMA, two stages), dt / lambda and entering state are in
+// flight while the current chunk is computed.
 // ============================================================================
 namespace outk {
 constexpr int THREADS = 512;
 constexpr int RG = THREADS / 64;   // row groups of the operand preparation
 constexpr uint32_t TMEM_COLS = 64;
-constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle, rows = t)
-constexpr uint32_t SM_B = 8192;       // 16 KB raw B (two 64-row swizzled halves)
-constexpr uint32_t SM_C = 24576;      // 16 KB raw C
-constexpr uint32_t SM_CI = 40960;     // 16 KB Ci   K-major (64 t x 128)
-constexpr uint32_t SM_CH = 57344;     // 16 KB Ch   K-major
-constexpr uint32_t SM_BI = 73728;     // 40 KB Bi tiles (16, 32, 48, 64 rows)
-constexpr uint32_t SM_P = 114688;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
-constexpr uint32_t SM_KT = 122880;    // 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
-constexpr uint32_t SM_F32 = 139264;
+constexpr uint32_t SM_X = 0;          // 2 x 8 KB   x (128B swizzle, rows = t)
+constexpr uint32_t SM_B = 16384;      // 2 x 16 KB  raw B (two 64-row swizzled halves)
+constexpr uint32_t SM_C = 49152;      // 2 x 16 KB  raw C
+constexpr uint32_t SM_CI = 81920;     // 16 KB Ci   K-major (64 t x 128)
+constexpr uint32_t SM_CH = 98304;     // 16 KB Ch   K-major
+constexpr uint32_t SM_BI = 114688;    // 40 KB Bi tiles (16, 32, 48, 64 rows)
+constexpr uint32_t SM_P = 155648;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
+constexpr uint32_t SM_KT = 163840;    // 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
+constexpr uint32_t SM_F32 = 180224;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+static_assert(THREADS * 16 == 8192, "one 16-byte piece of the saved P tiles per thread");
 }  // namespace outk
 
 __global__ void __launch_bounds__(outk::THREADS, 1)
 k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, Params p) {
     if (gated_off(p)) return;
+    const int nitems = p.nc * p.H * p.Bsz;
+    if ((int)blockIdx.x >= nitems) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + outk::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + outk::SM_BAR);
-    uint64_t *bar_mma = bar_tma + 1;   // [2]: phase A, phase B
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + outk::SM_BAR);   // [2] stages
+    uint64_t *bar_mma = bar_tma + 2;                                      // [2] phase A, B
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / p.hpg;
     const int N = p.N, nr = p.nr, L = p.L;
-    const int t0 = c * Q;
     const int nbox = N / 64;
+    const uint32_t tile_bytes = (uint32_t)(Q * PD * 2 + 2 * Q * N * 2);
+    auto issue_tma = [&](int item, int st) {
+        const ChunkItem it = chunk_item(p, item);
+        const int g = it.h / p.hpg, t0 = it.c * Q;
+        mbar_expect_tx(&bar_tma[st], tile_bytes);
+        tma_load_4d(sm + outk::SM_X + st * 8192, &tmX, &bar_tma[st], 0, it.h, t0, it.b);
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_4d(sm + outk::SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g, t0,
+                        it.b);
+            tma_load_4d(sm + outk::SM_C + st * 16384 + k * 8192, &tmC, &bar_tma[st], 64 * k, g, t0,
+                        it.b);
+        }
+    };
 
+    int item = blockIdx.x;
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
         mbar_init(&bar_mma[0], 1);
         mbar_init(&bar_mma[1], 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + 2 * Q * N * 2));
-        tma_load_4d(sm + outk::SM_X, &tmX, bar_tma, 0, h, t0, b);
-        for (int k = 0; k < nbox; ++k) {
-            tma_load_4d(sm + outk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
-            tma_load_4d(sm + outk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
-        }
+        issue_tma(item, 0);
     }
     if (warp == 0) tmem_alloc(tslot, outk::TMEM_COLS);
-    mode_rates(p, f32, h);
-    if (N < NP)  // K padding of Ci, Ch, Bi
+    if (N < NP)  // K padding of Ci, Ch, Bi (rows past N are never written)
         for (int i = tid; i < (int)((outk::SM_P - outk::SM_CI) / 16); i += outk::THREADS)
             reinterpret_cast<uint4 *>(sm + outk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
-    load_state_tile(p.ws_kp + bhc(p, b, h, c) * N * PD, N, sm + outk::SM_KT, nullptr);
-    chunk_tokens(p, f32, b, h, t0, true);
-    chunk_mode_constants(p, f32);
+    TokPrefetch tok;
+    StatePrefetch<outk::THREADS> kst;
+    {
+        const ChunkItem it = chunk_item(p, item);
+        tok = tok_load(p, it.b, it.h, it.c * Q);
+        state_load(p.ws_kp + bhc(p, it.b, it.h, it.c) * N * PD, N, kst);
+    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -376,9 +406,36 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     const uint32_t t_y = tbase;                      // Y^T (M=64, lanes 0-15 of each quarter)
     const uint32_t t_sc = tbase + (16u << 16);       // scores^T (M=64, lanes 16-31)
     float *cpart = reinterpret_cast<float *>(sm + outk::SM_P);   // C.B partials until P is built
-    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
-    if (!ok) raise_error(1);
-    if (__syncthreads_and(ok)) {
+    bool aborted = false;
+
+    for (int k = 0; item < nitems; ++k, item += gridDim.x) {
+        const int st = k & 1;
+        const ChunkItem it = chunk_item(p, item);
+        const int c = it.c, h = it.h, b = it.b;
+        const int t0 = c * Q;
+        const int next = item + gridDim.x;
+        unsigned char *sX = sm + outk::SM_X + st * 8192;
+        unsigned char *sB = sm + outk::SM_B + st * 16384;
+        unsigned char *sC = sm + outk::SM_C + st * 16384;
+
+        // ---- this chunk's small inputs; the next chunk's in flight -----------
+        mode_rates(p, f32, h);
+        state_store(kst, sm + outk::SM_KT, nullptr);
+        chunk_tokens_from(p, f32, t0, tok, true);
+        if (next < nitems) {
+            const ChunkItem nx = chunk_item(p, next);
+            tok = tok_load(p, nx.b, nx.h, nx.c * Q);
+            state_load(p.ws_kp + bhc(p, nx.b, nx.h, nx.c) * N * PD, N, kst);
+            // the other stage was last read by the previous chunk, which is complete
+            if (tid == 0) issue_tma(next, st ^ 1);
+        }
+        chunk_mode_constants(p, f32);
+        int ok = mbar_wait(&bar_tma[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) ? 1 : 0;
+        if (!ok) raise_error(1);
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
         // ---- operand preparation: thread (t, grp) handles rows 8 (grp + RG k) ---
         {
             const int t = tid & 63, grp = tid >> 6;
@@ -386,11 +443,10 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
             const float ds = f32[F_S + t] - Sb;
             const float sig = f32[F_SIG + t];
-            const unsigned char *sB = sm + outk::SM_B, *sC = sm + outk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
-            for (int k = 0; k < NP / (8 * outk::RG); ++k) {
-                const int r0 = 8 * (grp + outk::RG * k);
+            for (int kk = 0; kk < NP / (8 * outk::RG); ++kk) {
+                const int r0 = 8 * (grp + outk::RG * kk);
                 if (r0 >= N) break;
                 float vCI[8], vCH[8], vBI[8], vBX[3][8], rc[8], rb[8];
                 ld_rows8(sC, t, r0, rc);
@@ -492,84 +548,104 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int k = 0; k < outk::RG; ++k) cs += cpart[k * 64 + tid];
-            f32[F_CORR + tid] = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
+            for (int kk = 0; kk < outk::RG; ++kk) cs += cpart[kk * 64 + tid];
+            const float corr = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
+            f32[F_CORR + tid] = corr;
+            if (p.sv_corr) p.sv_corr[bhc(p, b, h, c) * Q + tid] = corr;
         }
-        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        ok = mbar_wait(&bar_mma[0], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
         if (!ok) raise_error(1);
         fence_after_sync();
-        if (__syncthreads_and(ok)) {
-            // ---- masked scores -> P^T tiles (one warp per TMEM lane quarter) -------
-            if (warp >= 4 && warp < 8) {
-                const int qd = warp - 4;
-                for (int i = 0; i < NSB; ++i) {
-                    float v[16];
-                    tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
-                    const int sl = lane - 16;
-                    if (sl >= 0) {
-                        const int s = 16 * qd + sl;
-                        if (s < 16 * (i + 1)) {
-                            float lo[8], hi[8];
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // ---- masked scores -> P^T tiles (one warp per TMEM lane quarter) -------
+        if (warp >= 4 && warp < 8) {
+            const int qd = warp - 4;
+            for (int i = 0; i < NSB; ++i) {
+                float v[16];
+                tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
+                const int sl = lane - 16;
+                if (sl >= 0) {
+                    const int s = 16 * qd + sl;
+                    if (s < 16 * (i + 1)) {
+                        float lo[8], hi[8];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
-                                hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
-                            }
-                            unsigned char *pt = sm + outk::SM_P + i * 2048;
-                            st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
-                            st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
+                            hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
                         }
-                    }
-                }
-            }
-            fence_proxy_async();
-            fence_before_sync();
-            __syncthreads();
-
-            // ---- phase B: intra-chunk term Y^T += X^T P^T_i ----------------------
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t x_base = smem_u32(sm + outk::SM_X), p_base = smem_u32(sm + outk::SM_P);
-                const uint32_t id_d = idesc_bf16(64, 16, true, true);
-                for (int i = 0; i < NSB; ++i)
-                    for (int s = 0; s <= i; ++s)
-                        mma_bf16(t_y + 16 * i, sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128),
-                                 sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
-                                 true);
-                mma_commit(&bar_mma[1]);
-            }
-            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
-            if (!ok) raise_error(1);
-            fence_after_sync();
-            if (__syncthreads_and(ok)) {
-                // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p] -----------------
-                const int qd = warp & 3, part = warp >> 2;   // TMEM quarter, column block
-                const int pp = 16 * qd + (lane & 15);
-                const unsigned char *sX = sm + outk::SM_X;
-                __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
-                                      h * p.sy[2] + pp;
-                constexpr int CPW = 64 / (outk::THREADS / 128);
-                for (int c16 = 0; c16 < CPW / 16; ++c16) {
-                    float v[16];
-                    const int tc = CPW * part + 16 * c16;
-                    tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
-                    if (lane < 16) {
-                        __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int t = tc + j;
-                            if (t0 + t < L) {
-                                const float u = bf(sX + off_sw128(t, pp));
-                                *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
-                            }
-                            yp += p.sy[1];
-                        }
+                        unsigned char *pt = sm + outk::SM_P + i * 2048;
+                        st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
+                        st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
+                    } else if (p.sv_P) {
+                        // rows past the block are zero in the saved copy (read there as P^T)
+                        unsigned char *pt = sm + outk::SM_P + i * 2048;
+                        *reinterpret_cast<uint4 *>(pt + off_mnmaj(0, s, 256u, 128u)) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(pt + off_mnmaj(8, s, 256u, 128u)) = make_uint4(0, 0, 0, 0);
                     }
                 }
             }
         }
-    } else if (tid == 0) {
-        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (p.sv_P)  // the masked score tiles, for the backward's dx (512 threads x 16 bytes)
+            *reinterpret_cast<uint4 *>(p.sv_P + bhc(p, b, h, c) * 8192 + tid * 16) =
+                *reinterpret_cast<const uint4 *>(sm + outk::SM_P + tid * 16);
+
+        // ---- phase B: intra-chunk term Y^T += X^T P^T_i ----------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + outk::SM_P);
+            const uint32_t id_d = idesc_bf16(64, 16, true, true);
+            for (int i = 0; i < NSB; ++i)
+                for (int s = 0; s <= i; ++s)
+                    mma_bf16(t_y + 16 * i, sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128),
+                             sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
+                             true);
+            mma_commit(&bar_mma[1]);
+        }
+        ok = mbar_wait(&bar_mma[1], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
+        if (!ok) raise_error(1);
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p] -----------------------
+        {
+            const int qd = warp & 3, part = warp >> 2;   // TMEM quarter, column block
+            const int pp = 16 * qd + (lane & 15);
+            __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
+                                  h * p.sy[2] + pp;
+            constexpr int CPW = 64 / (outk::THREADS / 128);
+            for (int c16 = 0; c16 < CPW / 16; ++c16) {
+                float v[16];
+                const int tc = CPW * part + 16 * c16;
+                tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
+                if (lane < 16) {
+                    __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = tc + j;
+                        if (t0 + t < L) {
+                            const float u = bf(sX + off_sw128(t, pp));
+                            *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
+                        }
+                        yp += p.sy[1];
+                    }
+                }
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+    }
+    if (aborted && tid == 0) {
+        // let loads still in flight land before the CTA's shared memory goes away
+        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
+        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
     }
     fence_before_sync();
     __syncthreads();
@@ -635,6 +711,20 @@ bool chunk_bwd_supported(const Params &p) {
            st16(p.sy[2]) && (!p.dx || al16(p.dx));
 }
 
+// Streaming multiprocessors of the current device (grid of the persistent kernels).
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <typename K>
 static cudaError_t set_smem_once(K kern, uint32_t bytes, bool &done) {
     if (done) return cudaSuccess;
@@ -673,7 +763,9 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     static bool a3 = false;
     if ((e = set_smem_once(k_chunk_out, outk::SMEM_BYTES, a3)) != cudaSuccess) return e;
-    k_chunk_out<<<dim3(p.nc, p.H, p.Bsz), outk::THREADS, outk::SMEM_BYTES, st>>>(mx, mb, mc, p);
+    const long long nitems = (long long)p.nc * p.H * p.Bsz;
+    const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
+    k_chunk_out<<<grid, outk::THREADS, outk::SMEM_BYTES, st>>>(mx, mb, mc, p);
     profile_mark(st, "k_chunk_out");
     return cudaGetLastError();
 }

@@ -584,6 +584,121 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
 }
 
 // ============================================================================
+// k_chunk_bwd_dx_saved: dx from the per-chunk products the training forward
+// saved (masked score tiles P^T, the chunk-end folded B, the diagonal
+// correction), so no operand has to be rebuilt:
+//   DX = P^T (64 s x 64 t) . dY (64 t x 64 p) + Bh (64 s x N) . Gc (N x 64 p)
+//   dx_s = DX_s + (D - beta_{s+1} C_s . B_s) dy_s
+// Small shared memory: several CTAs share an SM.
+// ============================================================================
+namespace dxs {
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 64;
+constexpr uint32_t SM_DY = 0;        // 8 KB  dy (128B swizzle)
+constexpr uint32_t SM_P = 8192;      // 8 KB  P^T, four 16-token tiles (K-major rows s)
+constexpr uint32_t SM_BH = 16384;    // 16 KB Bh (stored MN-major with M = rows; read K-major, M = s)
+constexpr uint32_t SM_GC = 32768;    // 16 KB Gc bf16, MN-major B operand (N = p, K = rows)
+constexpr uint32_t SM_CORR = 49152;  // 64 floats
+constexpr uint32_t SM_BAR = SM_CORR + 256;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+}  // namespace dxs
+
+__global__ void __launch_bounds__(dxs::THREADS)
+k_chunk_bwd_dx_saved(const __grid_constant__ CUtensorMap tmDY, Params p) {
+    if (gated_off(p)) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *corr = reinterpret_cast<float *>(sm + dxs::SM_CORR);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dxs::SM_BAR);
+    uint64_t *bar_mma = bar_tma + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int N = p.N, L = p.L;
+    const int t0 = c * Q;
+    const long long u = bhc(p, b, h, c);
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmDY);
+        mbar_expect_tx(bar_tma, 8192u + 8192u + 16384u);
+        tma_load_4d(sm + dxs::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        bulk_load(sm + dxs::SM_P, p.sv_P + u * 8192, 8192u, bar_tma);
+        bulk_load(sm + dxs::SM_BH, p.sv_Bh + u * 16384, 16384u, bar_tma);
+    }
+    if (warp == 0) tmem_alloc(tslot, dxs::TMEM_COLS);
+    load_state_tile(p.ws_gc + u * N * PD, N, sm + dxs::SM_GC, nullptr);
+    if (tid < Q) corr[tid] = p.sv_corr[u * Q + tid];
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t t_dx = *tslot;
+    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
+    if (!ok) rev_raise_error(1);
+    if (__syncthreads_and(ok)) {
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id = idesc_bf16(64, 64, false, true);
+            const uint32_t p_base = smem_u32(sm + dxs::SM_P), dy_base = smem_u32(sm + dxs::SM_DY);
+            for (int i = 0; i < NSB; ++i)
+                mma_bf16(t_dx, sdesc(p_base + i * 2048u, 128u, 256u, LAYOUT_NONE),
+                         sdesc(dy_base + i * 2048u, 8192u, 1024u, LAYOUT_SW128), id, i > 0);
+            const uint32_t bh_base = smem_u32(sm + dxs::SM_BH), gc_base = smem_u32(sm + dxs::SM_GC);
+            for (int s = 0; s < NP / 16; ++s)
+                mma_bf16(t_dx, sdesc(bh_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                         sdesc(gc_base + s * 2048u, 1024u, 128u, LAYOUT_NONE), id, true);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, 0, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (__syncthreads_and(ok)) {
+            // dx_s = DX_s + corr_s dy_s; warp (quarter qd, half) takes 32 columns of 16 rows
+            const int qd = warp & 3, half = warp >> 2;
+            const int s = 16 * qd + (lane & 15);
+            const unsigned char *sDY = sm + dxs::SM_DY;
+            __nv_bfloat16 *xrow = reinterpret_cast<__nv_bfloat16 *>(p.dx) + b * p.sx[0] +
+                                  (long long)(t0 + s) * p.sx[1] + h * p.sx[2];
+            const float cr = corr[s];
+#pragma unroll
+            for (int c16 = 0; c16 < 2; ++c16) {
+                float v[16];
+                const int pc = 32 * half + 16 * c16;
+                tmem_ld16(tmem_addr(t_dx, 32u * qd, (uint32_t)pc), v);
+                if (lane < 16 && t0 + s < L) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float o[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            o[j] = fmaf(cr, bf(sDY + off_sw128(s, pc + 8 * hh + j)), v[8 * hh + j]);
+                        uint4 w;
+                        w.x = pack_bf16(o[0], o[1]);
+                        w.y = pack_bf16(o[2], o[3]);
+                        w.z = pack_bf16(o[4], o[5]);
+                        w.w = pack_bf16(o[6], o[7]);
+                        *reinterpret_cast<uint4 *>(xrow + pc + 8 * hh) = w;
+                    }
+                }
+            }
+        }
+    } else if (tid == 0) {
+        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(t_dx, dxs::TMEM_COLS);
+    }
+}
+
+// ============================================================================
 // k_chunk_bwd_gbu: per chunk, gbu_t = sum_p u_t,p Gbar_t,p (per state row),
 // with sub-block-END references Se_j (the mirror of the forward's folding):
 //   Gbar_t u_t = conj(e^{lam (Se_j - S_t)}) [ conj(F[j+1][4]) (Gc u_t)
@@ -1358,8 +1473,15 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     k_chunk_adj_pass<<<dim3(p.H, p.Bsz), pass::THREADS, 0, st>>>(p);
     profile_mark(st, "k_chunk_adj_pass");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
-    profile_mark(st, "k_chunk_bwd_dx");
+    if (p.sv_P) {
+        static bool a5 = false;
+        if ((e = set_smem(k_chunk_bwd_dx_saved, dxs::SMEM_BYTES, a5)) != cudaSuccess) return e;
+        k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
+        profile_mark(st, "k_chunk_bwd_dx_saved");
+    } else {
+        k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
+        profile_mark(st, "k_chunk_bwd_dx");
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_chunk_bwd_gbu<<<grid, gbk::THREADS, gbk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
     profile_mark(st, "k_chunk_bwd_gbu");

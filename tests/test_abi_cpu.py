@@ -59,6 +59,11 @@ def test_workspace_size(lib):
     nc = (100 + 63) // 64
     nf = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
     assert nf >= 2 * 32 * nc * (128 * 64 + 128 * 2) * 4 and nf % 256 == 0
+    # a forward alone keeps only the chunk states; a training forward also the
+    # per-chunk products the backward reuses (8 + 16 KB + 64 floats per chunk)
+    ni = abi.ssm_scan_workspace_size(d, abi.PASS_FWD_INFER)
+    assert ni >= 2 * 32 * nc * (128 * 64 + 128 * 2) * 4 and ni % 256 == 0
+    assert nf - ni >= 2 * 32 * nc * (8192 + 16384 + 256)
     # the recurrent chain needs none
     for kw in (dict(chunk=1), dict(dtype_io=S.DTYPE_F32), dict(headdim=32)):
         assert abi.ssm_scan_workspace_size(abi.make_desc(sh.replace(**kw)), abi.PASS_FWD) == 0
