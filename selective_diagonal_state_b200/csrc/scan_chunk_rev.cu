@@ -715,26 +715,32 @@ constexpr int THREADS = 512;
 constexpr int RG = THREADS / 64;    // row groups of the operand preparation
 constexpr int TQ = THREADS / 128;   // token groups of the unfold
 constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
-constexpr uint32_t TMEM_COLS = 128;
+static_assert(TPT == 16, "the unfold takes one 16-token sub-block per thread");
+constexpr uint32_t TMEM_COLS = 512;    // V2 64 | G' 64 | E_{j,k} 10 x 16
 constexpr uint32_t SM_X = 0;           // 8 KB  x (swizzled)
 constexpr uint32_t SM_DY = 8192;       // 8 KB  dy (swizzled)
 constexpr uint32_t SM_B = 16384;       // 16 KB raw B
 constexpr uint32_t SM_C = 32768;       // 16 KB raw C
-constexpr uint32_t SM_CM = 49152;      // 40 KB Cm^{[j]} hi, MN-major (M = rows, K = t' - 16 j)
-constexpr uint32_t SM_CML = 90112;     // 40 KB Cm lo
-constexpr uint32_t SM_GM = 131072;     // 8 KB  masked G' hi: 4 tiles, K-major (rows t, K = t')
-constexpr uint32_t SM_GML = 139264;    // 8 KB  masked G' lo
-constexpr uint32_t SM_GC = 147456;     // 16 KB Gc hi, K-major (rows = state rows, K = p)
-constexpr uint32_t SM_GCL = 163840;    // 16 KB Gc lo
-constexpr uint32_t SM_F32 = 180224;
+constexpr uint32_t SM_CM = 49152;      // 16 KB Cm hi (own sub-block end), MN-major (M = rows, K = t')
+constexpr uint32_t SM_CML = 65536;     // 16 KB Cm lo
+constexpr uint32_t SM_GM = 81920;      // 8 KB  masked G' hi: 4 tiles, K-major (rows t, K = t')
+constexpr uint32_t SM_GML = 90112;     // 8 KB  masked G' lo
+constexpr uint32_t SM_GC = 98304;      // 16 KB Gc hi, K-major (rows = state rows, K = p)
+constexpr uint32_t SM_GCL = 114688;    // 16 KB Gc lo
+constexpr uint32_t SM_F32 = 131072;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
-constexpr int RED_LD = 65;             // row stride of the dsigma reduction (floats)
+constexpr int RED_LD = 65;             // row stride of the column reductions (floats)
+// after phase B the Cm .. Gc regions are free: two [128][RED_LD] reductions, then exchange space
+constexpr uint32_t SM_RED = SM_CM;
+constexpr uint32_t SM_RED2 = SM_RED + 128 * RED_LD * 4;
+constexpr uint32_t SM_XCH = SM_RED2 + 128 * RED_LD * 4;
+static_assert(SM_XCH + 8192 <= SM_F32, "reduction space");
 }  // namespace gbk
 
-// byte offset of mirror tile j (64 - 16 j rows of 256 bytes)
-__device__ __forceinline__ uint32_t cm_off(int j) {
-    return j == 0 ? 0u : (j == 1 ? 16384u : (j == 2 ? 28672u : 36864u));
+// TMEM column of E_{j,k} (k >= j): 10 blocks of 16 columns after V2 and G'
+__device__ __forceinline__ uint32_t ejk_col(int j, int k) {
+    return 128u + 16u * (uint32_t)((j == 0 ? 0 : (j == 1 ? 4 : (j == 2 ? 7 : 9))) + (k - j));
 }
 
 __global__ void __launch_bounds__(gbk::THREADS, 1)
@@ -792,7 +798,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
     if (!ok) rev_raise_error(1);
     if (__syncthreads_and(ok)) {
-        // ---- mirror tiles: own sub-block value, copies into earlier sub-blocks' tiles
+        // ---- Cm: C folded at its own sub-block's end, hi + lo; C.B partials
         {
             const int t = tid & 63, grp = tid >> 6;
             const int kb = t >> 4;
@@ -803,7 +809,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             for (int k = 0; k < NP / (8 * gbk::RG); ++k) {
                 const int r0 = 8 * (grp + gbk::RG * k);
                 if (r0 >= N) break;
-                float rc[8], rb[8], v[8], vx[3][8];
+                float rc[8], rb[8], v[8];
                 ld_rows8(sC, t, r0, rc);
                 ld_rows8(sB, t, r0, rb);
 #pragma unroll
@@ -813,14 +819,6 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     if (r < nr) {
                         v[j] = rc[j] * ex2_fast(fminf(f32[F_A2 + r] * ds, 120.f));
                         v[j + 1] = rc[j + 1] * ex2_fast(fminf(f32[F_A2 + r + 1] * ds, 120.f));
-#pragma unroll
-                        for (int jj = 0; jj < 3; ++jj) {
-                            if (jj < kb) {
-                                const int sl = fslot(jj + 1, kb + 1);
-                                vx[jj][j] = v[j] * f32[F_KRE + sl * NP + r];
-                                vx[jj][j + 1] = v[j + 1] * f32[F_KRE + sl * NP + r + 1];
-                            }
-                        }
                     } else {
                         const int m = nr + ((r - nr) >> 1);
                         float sn, cs;
@@ -828,23 +826,9 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         const float ec = ex2_fast(fminf(f32[F_A2 + m] * ds, 120.f));
                         v[j] = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
                         v[j + 1] = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
-#pragma unroll
-                        for (int jj = 0; jj < 3; ++jj) {
-                            if (jj < kb) {
-                                const int sl = fslot(jj + 1, kb + 1);
-                                cmul(v[j], v[j + 1], f32[F_KRE + sl * NP + m],
-                                     -f32[F_KIM + sl * NP + m], vx[jj][j], vx[jj][j + 1]);
-                            }
-                        }
                     }
                 }
-                st16_split(sm + gbk::SM_CM + cm_off(kb), sm + gbk::SM_CML + cm_off(kb),
-                           off_mnmaj(r0, t - 16 * kb, 2048u, 128u), v);
-#pragma unroll
-                for (int jj = 0; jj < 3; ++jj)
-                    if (jj < kb)
-                        st16_split(sm + gbk::SM_CM + cm_off(jj), sm + gbk::SM_CML + cm_off(jj),
-                                   off_mnmaj(r0, t - 16 * jj, 2048u, 128u), vx[jj]);
+                st16_split(sm + gbk::SM_CM, sm + gbk::SM_CML, off_mnmaj(r0, t, 2048u, 128u), v);
             }
             reinterpret_cast<float *>(sm + gbk::SM_GM)[grp * 64 + t] = corr;   // G' tiles come later
         }
@@ -921,21 +905,21 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
-            // ---- phase B: E_j = Cm^{[j]} (G' o mask)_j^T, hi*hi + hi*lo + lo*hi
+            // ---- phase B: E_{j,k} = Cm_k (G' o mask)_{j,k}^T, hi*hi + hi*lo + lo*hi
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t id_e = idesc_bf16(128, 16, true, false);
                 const uint32_t a_off[3] = {gbk::SM_CM, gbk::SM_CM, gbk::SM_CML};
                 const uint32_t b_off[3] = {gbk::SM_GM, gbk::SM_GML, gbk::SM_GM};
                 for (int j = 0; j < NSB; ++j)
-                    for (int part = 0; part < 3; ++part) {
-                        const uint32_t cm_base = smem_u32(sm + a_off[part]) + cm_off(j);
-                        const uint32_t gm_base = smem_u32(sm + b_off[part]) + j * 2048u;
-                        for (int s = 0; s < NSB - j; ++s)
-                            mma_bf16(t_g + 16 * j, sdesc(cm_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                                     sdesc(gm_base + (j + s) * 256u, 128u, 1024u, LAYOUT_NONE), id_e,
-                                     part > 0 || s > 0);
-                    }
+                    for (int k = j; k < NSB; ++k)
+                        for (int part = 0; part < 3; ++part)
+                            mma_bf16(tbase + ejk_col(j, k),
+                                     sdesc(smem_u32(sm + a_off[part]) + k * 4096u, 2048u, 128u,
+                                           LAYOUT_NONE),
+                                     sdesc(smem_u32(sm + b_off[part]) + j * 2048u + k * 256u, 128u,
+                                           1024u, LAYOUT_NONE),
+                                     id_e, part > 0);
                 mma_commit(&bar_mma[1]);
             }
             ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
@@ -947,9 +931,9 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 // identity (X_t - Y_t, X = conj(c) dCK, Y = b conj(sigma gbu)), walking the
                 // tokens backwards; and dB / dC directly when a group has one head.
                 // Thread (row n, token group tq) takes tokens TPT tq .. TPT tq + TPT - 1.
-                float *red = reinterpret_cast<float *>(sm + gbk::SM_CM);     // [128][RED_LD] B . gbu
-                float *red2 = reinterpret_cast<float *>(sm + gbk::SM_CML);   // [128][RED_LD] ddt terms
-                float *xch = reinterpret_cast<float *>(sm + gbk::SM_GM);     // [3][TQ][128] group totals
+                float *red = reinterpret_cast<float *>(sm + gbk::SM_RED);    // [128][RED_LD] B . gbu
+                float *red2 = reinterpret_cast<float *>(sm + gbk::SM_RED2);  // [128][RED_LD] ddt terms
+                float *xch = reinterpret_cast<float *>(sm + gbk::SM_XCH);    // group totals, partials
                 const int n = tid & 127, tq = tid >> 7, qd = warp & 3;
                 const bool valid = n < N;
                 const int m = n < nr ? n : nr + ((n - nr) >> 1);
@@ -967,9 +951,23 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
                 for (int c16 = gbk::TPT / 16 - 1; c16 >= 0; --c16) {
                     float vv[16], ee[16];
-                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)(tc + 16 * c16)), vv);
-                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)(tc + 16 * c16)), ee);
                     const int jb = (tc + 16 * c16) >> 4;   // sub-block of these 16 tokens
+                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)(tc + 16 * c16)), vv);
+                    tmem_ld16(tmem_addr(tbase + ejk_col(jb, jb), 32u * qd, 0u), ee);
+                    // later sub-blocks' contributions with their per-row factors conj(F[jb+1][k+1])
+                    for (int k = jb + 1; k < NSB; ++k) {
+                        float ek[16];
+                        tmem_ld16(tmem_addr(tbase + ejk_col(jb, k), 32u * qd, 0u), ek);
+                        const float f2r = valid ? f32[F_KRE + fslot(jb + 1, k + 1) * NP + m] : 0.f;
+                        const float f2i = valid ? f32[F_KIM + fslot(jb + 1, k + 1) * NP + m] : 0.f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
+                            // own component of (f2r - i f2i)(re + i im)
+                            ee[j] = pr_row ? fmaf(f2r, ek[j], fmaf(im_row ? -f2i : f2i, other, ee[j]))
+                                           : fmaf(f2r, ek[j], ee[j]);
+                        }
+                    }
                     const float se = f32[F_S + 16 * jb + 15];
                     float fr = 1.f, fi = 0.f;
                     if (jb < 3 && valid) {
@@ -1126,35 +1124,45 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 // ============================================================================
 // k_chunk_bwd_dc: per chunk, dC_t = dy_t H_t^T per head.
 //   H_t = K_t - beta_{t+1} W_t,   K_t = e^{lam S_t} K_prev + sum_{s<=t} Phi_{t,s} sigma_s b_s u_s
-// so, per state mode (complex for rotation pairs, real rows otherwise),
-//   dCK_t = e^{lam S_t} (dy_t . K_prev) + e^{lam (S_t - Sb_i)} sum_{s<=t} (dy_t . u_s) Bi_s
-// which is, on the tensor cores (operands split into bf16 hi + lo),
-//   V^T  = K_prev (N x 64 p) . dY^T (64 p x 64 t)          M=128, N=64, K=64
-//   G    = dY (64 t x 64 p) . X^T (64 p x 64 s)            M=64,  N=64, K=64
-//   D_i  = Bi^T (N x s) . (G o causal mask)_i^T (s x 16 t) M=128, N=16, K=16(i+1)
-// followed by the per-(t, row) unfolding of the decay factors on the CUDA
-// cores; dC_t = dCK_t - beta_{t+1} (dy_t . u_t) B_t.  K_prev is the state
-// entering the chunk (k_chunk_state_pass).
+// so, per state mode (complex for rotation pairs, real rows otherwise), for t
+// in sub-block i,
+//   dCK_t = e^{lam S_t} (dy_t . K_prev)
+//         + e^{lam (S_t - Sb_i)} sum_{k <= i} F[k][i] sum_{s in block k, s <= t} (dy_t . u_s) Bo_s
+// with Bo_s = sigma_s b_s e^{lam (Sb_k - S_s)} folded at its own sub-block's
+// start (the factor F[k][i] = e^{lam (Sb_i - Sb_k)} is per state row, so it is
+// applied after the contraction over tokens).  On the tensor cores (operands
+// split into bf16 hi + lo):
+//   V^T      = K_prev (N x 64 p) . dY^T (64 p x 64 t)                 M=128, N=64, K=64
+//   G        = dY (64 t x 64 p) . X^T (64 p x 64 s)                   M=64,  N=64, K=64
+//   D_{i,k}  = Bo_k^T (N x 16 s) . (G o causal mask)_{i,k}^T (16 s x 16 t)  M=128, N=16, K=16
+// then the per-(t, row) unfold on the CUDA cores; dC_t = dCK_t -
+// beta_{t+1} (dy_t . u_t) B_t.  K_prev is the state entering the chunk.
 // ============================================================================
 namespace dck {
 constexpr int THREADS = 512;
 constexpr int RG = THREADS / 64;    // row groups of the operand preparation
-constexpr int TQ = THREADS / 128;   // token groups of the unfold
+constexpr int TQ = THREADS / 128;   // token groups of the unfold (one sub-block each)
 constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
-constexpr uint32_t TMEM_COLS = 128;
+static_assert(TPT == 16, "the unfold takes one 16-token sub-block per thread");
+constexpr uint32_t TMEM_COLS = 512;   // V 64 | G 64 | D_{i,k} 10 x 16
 constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle)
 constexpr uint32_t SM_DY = 8192;      // 8 KB  dy (128B swizzle)
 constexpr uint32_t SM_B = 16384;      // 16 KB raw B (two 64-row swizzled halves)
-constexpr uint32_t SM_BI = 32768;     // 40 KB Bi tiles (hi)
-constexpr uint32_t SM_BIL = 73728;    // 40 KB Bi tiles (lo)
-constexpr uint32_t SM_GM = 114688;    // 8 KB  masked G hi: 4 tiles, K-major (N = 16 t, K = s)
-constexpr uint32_t SM_GML = 122880;   // 8 KB  masked G lo
-constexpr uint32_t SM_KT = 131072;    // 16 KB K_prev hi, K-major (rows n, K = p)
-constexpr uint32_t SM_KTL = 147456;   // 16 KB K_prev lo
-constexpr uint32_t SM_F32 = 163840;
+constexpr uint32_t SM_BO = 32768;     // 16 KB Bo hi, K-major (rows s, K = state rows)
+constexpr uint32_t SM_BOL = 49152;    // 16 KB Bo lo
+constexpr uint32_t SM_GM = 65536;     // 8 KB  masked G hi: 4 tiles, K-major (N = 16 t, K = s)
+constexpr uint32_t SM_GML = 73728;    // 8 KB  masked G lo
+constexpr uint32_t SM_KT = 81920;     // 16 KB K_prev hi, K-major (rows n, K = p)
+constexpr uint32_t SM_KTL = 98304;    // 16 KB K_prev lo
+constexpr uint32_t SM_F32 = 114688;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 }  // namespace dck
+
+// TMEM column of D_{i,k} (k <= i): 10 blocks of 16 columns after V and G
+__device__ __forceinline__ uint32_t dik_col(int i, int k) {
+    return 128u + 16u * (uint32_t)(i * (i + 1) / 2 + k);
+}
 
 __global__ void __launch_bounds__(dck::THREADS, 1)
 k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -1191,9 +1199,9 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     }
     if (warp == 0) tmem_alloc(tslot, dck::TMEM_COLS);
     mode_rates(p, f32, h);
-    if (N < NP)  // M padding of the Bi tiles
-        for (int i = tid; i < (int)((dck::SM_GM - dck::SM_BI) / 16); i += dck::THREADS)
-            reinterpret_cast<uint4 *>(sm + dck::SM_BI)[i] = make_uint4(0, 0, 0, 0);
+    if (N < NP)  // M padding of the Bo tiles
+        for (int i = tid; i < (int)((dck::SM_GM - dck::SM_BO) / 16); i += dck::THREADS)
+            reinterpret_cast<uint4 *>(sm + dck::SM_BO)[i] = make_uint4(0, 0, 0, 0);
     load_state_tile(p.ws_kp + bhc(p, b, h, c) * N * PD, N, sm + dck::SM_KT, sm + dck::SM_KTL);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
@@ -1202,11 +1210,11 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_v = tbase;           // V^T (M=128), cols 0..63
-    const uint32_t t_g = tbase + 64u;     // G (M=64, lanes 0-15 per quarter) then D_i (M=128)
+    const uint32_t t_g = tbase + 64u;     // G (M=64, lanes 0-15 per quarter), cols 64..127
     int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
     if (!ok) rev_raise_error(1);
     if (__syncthreads_and(ok)) {
-        // ---- Bi tiles (own sub-block and later ones), hi + lo ------------------
+        // ---- Bo: B folded at its own sub-block's start, hi + lo ----------------
         {
             const int t = tid & 63, grp = tid >> 6;
             const int ib = t >> 4;
@@ -1218,54 +1226,25 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             for (int k = 0; k < NP / (8 * dck::RG); ++k) {
                 const int r0 = 8 * (grp + dck::RG * k);
                 if (r0 >= N) break;
-                float vBI[8], vBX[3][8], rb[8];
+                float v[8], rb[8];
                 ld_rows8(sB, t, r0, rb);
 #pragma unroll
                 for (int j = 0; j < 8; j += 2) {
                     const int r = r0 + j;
                     const float b0 = rb[j], b1 = rb[j + 1];
                     if (r < nr) {
-                        const int m0 = r, m1 = r + 1;
-                        const float bi0 = sig * b0 * ex2_fast(fminf(-f32[F_A2 + m0] * ds, 120.f));
-                        const float bi1 = sig * b1 * ex2_fast(fminf(-f32[F_A2 + m1] * ds, 120.f));
-                        vBI[j] = bi0;
-                        vBI[j + 1] = bi1;
-#pragma unroll
-                        for (int qq = 0; qq < 3; ++qq) {
-                            const int i2 = ib + 1 + qq;
-                            if (i2 < 4) {
-                                vBX[qq][j] = bi0 * f32[F_KRE + fslot(ib, i2) * NP + m0];
-                                vBX[qq][j + 1] = bi1 * f32[F_KRE + fslot(ib, i2) * NP + m1];
-                            }
-                        }
+                        v[j] = sig * b0 * ex2_fast(fminf(-f32[F_A2 + r] * ds, 120.f));
+                        v[j + 1] = sig * b1 * ex2_fast(fminf(-f32[F_A2 + r + 1] * ds, 120.f));
                     } else {
                         const int m = nr + ((r - nr) >> 1);
                         float sn, cs;
                         __sincosf(f32[F_W + m] * ds, &sn, &cs);
                         const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m] * ds, 120.f));
-                        const float bi0 = eb * fmaf(b0, cs, b1 * sn);
-                        const float bi1 = eb * fmaf(b1, cs, -b0 * sn);
-                        vBI[j] = bi0;
-                        vBI[j + 1] = bi1;
-#pragma unroll
-                        for (int qq = 0; qq < 3; ++qq) {
-                            const int i2 = ib + 1 + qq;
-                            if (i2 < 4)
-                                cmul(bi0, bi1, f32[F_KRE + fslot(ib, i2) * NP + m],
-                                     f32[F_KIM + fslot(ib, i2) * NP + m], vBX[qq][j],
-                                     vBX[qq][j + 1]);
-                        }
+                        v[j] = eb * fmaf(b0, cs, b1 * sn);
+                        v[j + 1] = eb * fmaf(b1, cs, -b0 * sn);
                     }
                 }
-                st16_split(sm + dck::SM_BI + bi_off(ib), sm + dck::SM_BIL + bi_off(ib),
-                           off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
-#pragma unroll
-                for (int qq = 0; qq < 3; ++qq) {
-                    const int i2 = ib + 1 + qq;
-                    if (i2 < 4)
-                        st16_split(sm + dck::SM_BI + bi_off(i2), sm + dck::SM_BIL + bi_off(i2),
-                                   off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
-                }
+                st16_split(sm + dck::SM_BO, sm + dck::SM_BOL, off_kmaj(t, r0, KM_LBO, KM_SBO), v);
             }
         }
         fence_proxy_async();
@@ -1326,32 +1305,31 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             fence_before_sync();
             __syncthreads();
 
-            // ---- phase B: D_i = Bi^T (G o mask)_i^T into the (now free) G columns
+            // ---- phase B: D_{i,k} = Bo_k^T (G o mask)_{i,k}^T, hi*hi + hi*lo + lo*hi
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t id_d = idesc_bf16(128, 16, true, false);
-                // hi*hi + hi*lo + lo*hi
-                const uint32_t a_off[3] = {dck::SM_BI, dck::SM_BI, dck::SM_BIL};
+                const uint32_t a_off[3] = {dck::SM_BO, dck::SM_BO, dck::SM_BOL};
                 const uint32_t b_off[3] = {dck::SM_GM, dck::SM_GML, dck::SM_GM};
                 for (int i = 0; i < NSB; ++i)
-                    for (int part = 0; part < 3; ++part) {
-                        const uint32_t bi_base = smem_u32(sm + a_off[part]);
-                        const uint32_t gm_base = smem_u32(sm + b_off[part]);
-                        for (int s = 0; s <= i; ++s)
-                            mma_bf16(t_g + 16 * i,
-                                     sdesc(bi_base + bi_off(i) + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                                     sdesc(gm_base + i * 2048u + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                                     id_d, part > 0 || s > 0);
-                    }
+                    for (int k = 0; k <= i; ++k)
+                        for (int part = 0; part < 3; ++part)
+                            mma_bf16(tbase + dik_col(i, k),
+                                     sdesc(smem_u32(sm + a_off[part]) + k * 4096u, 2048u, 128u,
+                                           LAYOUT_NONE),
+                                     sdesc(smem_u32(sm + b_off[part]) + i * 2048u + k * 256u, 128u,
+                                           1024u, LAYOUT_NONE),
+                                     id_d, part > 0);
                 mma_commit(&bar_mma[1]);
             }
             ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
             if (!ok) rev_raise_error(1);
             fence_after_sync();
             if (__syncthreads_and(ok)) {
-                // ---- unfold: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D ;
+                // ---- unfold for the 16 tokens of sub-block i = tq:
+                //      D = sum_k F[k][i] D_{i,k};  dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D
                 //      dC_t = dCK_t - beta' (dy.u) B_t
-                const int n = tid & 127, tq = tid >> 7, qd = warp & 3;
+                const int n = tid & 127, i = tid >> 7, qd = warp & 3;
                 const bool valid = n < N;
                 const int m = n < nr ? n : nr + ((n - nr) >> 1);
                 const bool pr_row = valid && n >= nr;
@@ -1360,47 +1338,57 @@ k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 float *dst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
                 const long long tstride = (long long)p.H * p.N;
                 const unsigned char *sB = sm + dck::SM_B;
-#pragma unroll
-                for (int c16 = 0; c16 < dck::TPT / 16; ++c16) {
-                    const int tc = dck::TPT * tq + 16 * c16;
-                    float vv[16], dd[16];
-                    tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
-                    tmem_ld16(tmem_addr(t_g, 32u * qd, (uint32_t)tc), dd);
-                    const int ib = tc >> 4;
-                    const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-                    // E = E' conj(G_i) = E' F[0][i]
-                    float fr = 1.f, fi = 0.f;
-                    if (ib && valid) {
-                        fr = f32[F_KRE + gslot(ib) * NP + m];
-                        fi = -f32[F_KIM + gslot(ib) * NP + m];
-                    }
+                const int tc = 16 * i;
+                float vv[16], dd[16];
+                tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
+                tmem_ld16(tmem_addr(tbase + dik_col(i, i), 32u * qd, 0u), dd);
+                // earlier sub-blocks' contributions, with their per-row factors F[k][i]
+                for (int k = 0; k < i; ++k) {
+                    float ek[16];
+                    tmem_ld16(tmem_addr(tbase + dik_col(i, k), 32u * qd, 0u), ek);
+                    const float fr = valid ? f32[F_KRE + fslot(k, i) * NP + m] : 0.f;
+                    const float fi = valid ? f32[F_KIM + fslot(k, i) * NP + m] : 0.f;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int t = tc + j;
-                        const float ds = f32[F_S + t] - Sb;
-                        const float mag = ex2_fast(a2 * ds);
-                        float er = mag, ei = 0.f;
-                        if (pr_row) {
-                            float sn, cs;
-                            __sincosf(w * ds, &sn, &cs);
-                            er = mag * cs;
-                            ei = mag * sn;
-                        }
-                        float Er, Ei;
-                        cmul(er, ei, fr, fi, Er, Ei);
-                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
-                        const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
-                        float res;
-                        if (!pr_row)
-                            res = fmaf(Er, vv[j], er * dd[j]);
-                        else if (!im_row)   // real part of E (V_re + i V_im) + E' (D_re + i D_im)
-                            res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
-                        else                // imaginary part
-                            res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
-                        if (valid && t0 + t < L) {
-                            const float bt = ld_row1(sB, t, n);
-                            dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
-                        }
+                        const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
+                        // own component of (fr + i fi)(re + i im)
+                        dd[j] = pr_row ? fmaf(fr, ek[j], fmaf(im_row ? fi : -fi, other, dd[j]))
+                                       : fmaf(fr, ek[j], dd[j]);
+                    }
+                }
+                const float Sb = i == 0 ? 0.f : f32[F_S + 16 * i - 1];
+                // E = E' conj(G_i) = E' F[0][i]
+                float fr = 1.f, fi = 0.f;
+                if (i && valid) {
+                    fr = f32[F_KRE + gslot(i) * NP + m];
+                    fi = -f32[F_KIM + gslot(i) * NP + m];
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int t = tc + j;
+                    const float ds = f32[F_S + t] - Sb;
+                    const float mag = ex2_fast(a2 * ds);
+                    float er = mag, ei = 0.f;
+                    if (pr_row) {
+                        float sn, cs;
+                        __sincosf(w * ds, &sn, &cs);
+                        er = mag * cs;
+                        ei = mag * sn;
+                    }
+                    float Er, Ei;
+                    cmul(er, ei, fr, fi, Er, Ei);
+                    const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                    const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
+                    float res;
+                    if (!pr_row)
+                        res = fmaf(Er, vv[j], er * dd[j]);
+                    else if (!im_row)   // real part of E (V_re + i V_im) + E' (D_re + i D_im)
+                        res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
+                    else                // imaginary part
+                        res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
+                    if (valid && t0 + t < L) {
+                        const float bt = ld_row1(sB, t, n);
+                        dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
                     }
                 }
             }
