@@ -102,14 +102,18 @@ def kernel_bytes(shape, name: str) -> int:
     if name == "k_bwd_groups":
         return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["C"] + t["B"] + t["C"]
                 + t["dt"] + t["lam"])
-    # tensor-core backward: path inputs read, path outputs written
-    if name == "k_chunk_bwd_dc":      # x, B, dt, lambda, dy
-        return t["x"] + t["B"] + t["dt"] + t["lam"] + dy
+    # tensor-core chain: path inputs read, path outputs written
+    if name == "k_chunk_out":         # x, B, C, dt, lambda -> y
+        return ins + t["y"]
+    if name == "k_chunk_state_local":  # x, B, dt, lambda (chunk states go to workspace)
+        return t["x"] + t["B"] + t["dt"] + t["lam"]
     if name == "k_chunk_adj_local":   # C, dt, dy
         return t["C"] + t["dt"] + dy
     if name == "k_chunk_bwd_dx":      # B, C, dt, lambda, dy -> dx
         return t["B"] + t["C"] + t["dt"] + t["lam"] + dy + t["x"]
-    if name == "k_chunk_bwd_gbu":     # x, B, C, dt, lambda, dy -> dB, dC (one head per group)
+    if name == "k_chunk_bwd_dx_saved":  # dy -> dx (the rest comes from the forward's workspace)
+        return dy + t["x"]
+    if name == "k_chunk_bwd_fused":   # x, B, C, dt, lambda, dy -> dB, dC (one head per group)
         out = t["B"] + t["C"] if s.nheads == s.ngroups else 0
         return ins + dy + out
     if name == "k_bwd_units_final":   # dt, lambda -> ddt, dlambda

@@ -699,60 +699,84 @@ k_chunk_bwd_dx_saved(const __grid_constant__ CUtensorMap tmDY, Params p) {
 }
 
 // ============================================================================
-// k_chunk_bwd_gbu: per chunk, gbu_t = sum_p u_t,p Gbar_t,p (per state row),
-// with sub-block-END references Se_j (the mirror of the forward's folding):
-//   Gbar_t u_t = conj(e^{lam (Se_j - S_t)}) [ conj(F[j+1][4]) (Gc u_t)
-//                                            + sum_{t' >= t} (u_t . dy_t') Cm^{[j]}_t' ]
-//   Cm^{[j]}_t' = conj(e^{lam (S_t' - Se_j)}) c_t'      for t' >= 16 j  (t in sub-block j)
-// On the tensor cores (all operands split into bf16 hi + lo):
-//   G' = X (64 t x 64 p) . dY^T (64 p x 64 t')                M=64,  N=64, K=64
-//   V2 = Gc (N x 64 p) . X^T (64 p x 64 t)                    M=128, N=64, K=64
-//   E_j = Cm^{[j]} (N x t') . (G' o mask)_j^T (t' x 16 t)      M=128, N=16, K=64-16j
-// Also writes <dy_t, u_t>, dsigma_t = B_t . gbu_t and (C_t . B_t) <dy_t, u_t>.
+// k_chunk_bwd_fused: per chunk, the per-token backward quantities that need
+// both directions inside the chunk.
+//
+// Forward direction (dC): with K_prev the state entering the chunk and Bo_s =
+// sigma_s b_s e^{lam (Sb_k - S_s)} folded at its own sub-block's start, for t
+// in sub-block i
+//   dCK_t = e^{lam S_t} (dy_t . K_prev)
+//         + e^{lam (S_t - Sb_i)} sum_{k <= i} F[k][i] sum_{s in block k, s <= t} (dy_t . u_s) Bo_s
+// and dC_t = dCK_t - beta_{t+1} (dy_t . u_t) B_t.
+// Reverse direction (gbu = sum_p u_t,p Gbar_t,p): with Gc the adjoint carried
+// into the chunk and Cm_t' = conj(e^{lam (S_t' - Se_k)}) c_t' folded at its own
+// sub-block's end, for t in sub-block j
+//   gbu_t = conj(e^{lam (Se_j - S_t)}) [ conj(F[j+1][4]) (Gc u_t)
+//           + sum_{k >= j} conj(F[j+1][k+1]) sum_{t' in block k, t' >= t} (u_t . dy_t') Cm_t' ]
+// The per-row factors F are applied to accumulators after the contractions
+// over tokens.  Tensor cores (operands split into bf16 hi + lo where rounding
+// reaches the decay gradients):
+//   V       = K_prev (N x 64 p) . dY^T (64 p x 64 t)               M=128, N=64
+//   V2      = Gc (N x 64 p) . X^T (64 p x 64 t)                    M=128, N=64
+//   G       = dY (64 t x 64 p) . X^T (64 p x 64 s)  [masked s <= t] M=64,  N=64
+//   D_{i,k} = Bo_k^T (N x 16 s) . G_{i,k}^T (16 s x 16 t)          M=128, N=16 (k <= i)
+//   E_{j,k} = Cm_k (N x 16 t') . G_{k,j} (16 t' x 16 t)             M=128, N=16 (k >= j)
+// where one stored copy of the masked G serves both: K-major for D, read
+// MN-major (its transpose) for E.  The epilogue then forms, per state mode,
+// the within-chunk suffix sums of the decay-gradient identity (X_t - Y_t,
+// X = conj(c) dCK, Y = b conj(sigma gbu)), the local part of ddt, the chunk's
+// totals, dsigma_t, <dy_t, u_t>, and dB / dC (one head per group) or the
+// per-head dC and gbu (several heads per group).
 // ============================================================================
-namespace gbk {
+namespace fuk {
 constexpr int THREADS = 512;
 constexpr int RG = THREADS / 64;    // row groups of the operand preparation
-constexpr int TQ = THREADS / 128;   // token groups of the unfold
-constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
+constexpr int TQ = THREADS / 128;   // token groups of the unfold (one sub-block each)
+constexpr int TPT = Q / TQ;
 static_assert(TPT == 16, "the unfold takes one 16-token sub-block per thread");
-constexpr uint32_t TMEM_COLS = 512;    // V2 64 | G' 64 | E_{j,k} 10 x 16
-constexpr uint32_t SM_X = 0;           // 8 KB  x (swizzled)
-constexpr uint32_t SM_DY = 8192;       // 8 KB  dy (swizzled)
-constexpr uint32_t SM_B = 16384;       // 16 KB raw B
-constexpr uint32_t SM_C = 32768;       // 16 KB raw C
-constexpr uint32_t SM_CM = 49152;      // 16 KB Cm hi (own sub-block end), MN-major (M = rows, K = t')
-constexpr uint32_t SM_CML = 65536;     // 16 KB Cm lo
-constexpr uint32_t SM_GM = 81920;      // 8 KB  masked G' hi: 4 tiles, K-major (rows t, K = t')
-constexpr uint32_t SM_GML = 90112;     // 8 KB  masked G' lo
-constexpr uint32_t SM_GC = 98304;      // 16 KB Gc hi, K-major (rows = state rows, K = p)
-constexpr uint32_t SM_GCL = 114688;    // 16 KB Gc lo
-constexpr uint32_t SM_F32 = 131072;
+constexpr uint32_t TMEM_COLS = 512;   // V 0 | V2 64 | G 128 | D_{i,k} 192.. | E_{j,k} 352..
+constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle)
+constexpr uint32_t SM_DY = 8192;      // 8 KB  dy (128B swizzle)
+constexpr uint32_t SM_B = 16384;      // 16 KB raw B (two 64-row swizzled halves)
+constexpr uint32_t SM_C = 32768;      // 16 KB raw C
+constexpr uint32_t SM_BO = 49152;     // 16 KB Bo hi (rows s, K = state rows)
+constexpr uint32_t SM_BOL = 65536;    // 16 KB Bo lo
+constexpr uint32_t SM_CM = 81920;     // 16 KB Cm hi (same layout)
+constexpr uint32_t SM_CML = 98304;    // 16 KB Cm lo
+constexpr uint32_t SM_GM = 114688;    // 8 KB  masked G hi: 4 tiles of 16 rows t, K = s
+constexpr uint32_t SM_GML = 122880;   // 8 KB  masked G lo
+constexpr uint32_t SM_KT = 131072;    // 16 KB K_prev hi (rows n, K = p)
+constexpr uint32_t SM_KTL = 147456;   // 16 KB K_prev lo
+constexpr uint32_t SM_GC = 163840;    // 16 KB Gc hi (rows n, K = p)
+constexpr uint32_t SM_GCL = 180224;   // 16 KB Gc lo
+constexpr uint32_t SM_F32 = 196608;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
-constexpr int RED_LD = 65;             // row stride of the column reductions (floats)
-// after phase B the Cm .. Gc regions are free: two [128][RED_LD] reductions, then exchange space
-constexpr uint32_t SM_RED = SM_CM;
+constexpr int RED_LD = 65;            // row stride of the column reductions (floats)
+// after phase B the Bo .. G regions are free: two [128][RED_LD] reductions and exchange space
+constexpr uint32_t SM_RED = SM_BO;
 constexpr uint32_t SM_RED2 = SM_RED + 128 * RED_LD * 4;
 constexpr uint32_t SM_XCH = SM_RED2 + 128 * RED_LD * 4;
-static_assert(SM_XCH + 8192 <= SM_F32, "reduction space");
-}  // namespace gbk
+static_assert(SM_XCH + 8192 <= SM_KT, "reduction space");
+}  // namespace fuk
 
-// TMEM column of E_{j,k} (k >= j): 10 blocks of 16 columns after V2 and G'
-__device__ __forceinline__ uint32_t ejk_col(int j, int k) {
-    return 128u + 16u * (uint32_t)((j == 0 ? 0 : (j == 1 ? 4 : (j == 2 ? 7 : 9))) + (k - j));
+__device__ __forceinline__ uint32_t d_col(int i, int k) {   // k <= i
+    return 192u + 16u * (uint32_t)(i * (i + 1) / 2 + k);
+}
+__device__ __forceinline__ uint32_t e_col(int j, int k) {   // k >= j
+    return 352u + 16u * (uint32_t)((j == 0 ? 0 : (j == 1 ? 4 : (j == 2 ? 7 : 9))) + (k - j));
 }
 
-__global__ void __launch_bounds__(gbk::THREADS, 1)
-k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
-                Params p) {
+__global__ void __launch_bounds__(fuk::THREADS, 1)
+k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                  Params p) {
     if (gated_off(p)) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + gbk::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + gbk::SM_BAR);
+    float *f32 = reinterpret_cast<float *>(sm + fuk::SM_F32);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);
     uint64_t *bar_mma = bar_tma + 1;   // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
 
@@ -762,6 +786,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     const int N = p.N, nr = p.nr, L = p.L;
     const int t0 = c * Q;
     const int nbox = N / 64;
+    const long long u = bhc(p, b, h, c);
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
@@ -773,43 +798,45 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
         mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + 2 * Q * N * 2));
-        tma_load_4d(sm + gbk::SM_X, &tmX, bar_tma, 0, h, t0, b);
-        tma_load_4d(sm + gbk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        tma_load_4d(sm + fuk::SM_X, &tmX, bar_tma, 0, h, t0, b);
+        tma_load_4d(sm + fuk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
         for (int k = 0; k < nbox; ++k) {
-            tma_load_4d(sm + gbk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
-            tma_load_4d(sm + gbk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
+            tma_load_4d(sm + fuk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
+            tma_load_4d(sm + fuk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
         }
     }
-    if (warp == 0) tmem_alloc(tslot, gbk::TMEM_COLS);
+    if (warp == 0) tmem_alloc(tslot, fuk::TMEM_COLS);
     mode_rates(p, f32, h);
-    if (N < NP)  // M padding of the mirror tiles
-        for (int i = tid; i < (int)((gbk::SM_GM - gbk::SM_CM) / 16); i += gbk::THREADS)
-            reinterpret_cast<uint4 *>(sm + gbk::SM_CM)[i] = make_uint4(0, 0, 0, 0);
-    // the adjoint carried into this chunk, bf16 hi / lo, K-major (rows n, K = p)
-    load_state_tile(p.ws_gc + bhc(p, b, h, c) * N * PD, N, sm + gbk::SM_GC, sm + gbk::SM_GCL);
+    if (N < NP)  // M padding of the Bo / Cm tiles
+        for (int i = tid; i < (int)((fuk::SM_GM - fuk::SM_BO) / 16); i += fuk::THREADS)
+            reinterpret_cast<uint4 *>(sm + fuk::SM_BO)[i] = make_uint4(0, 0, 0, 0);
+    load_state_tile(p.ws_kp + u * N * PD, N, sm + fuk::SM_KT, sm + fuk::SM_KTL);
+    load_state_tile(p.ws_gc + u * N * PD, N, sm + fuk::SM_GC, sm + fuk::SM_GCL);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
-    const uint32_t t_v2 = tbase;          // V2 (M=128), cols 0..63
-    const uint32_t t_g = tbase + 64u;     // G' (M=64: lanes 0-15 per quarter), then E_j (M=128)
+    const uint32_t t_v = tbase, t_v2 = tbase + 64u, t_g = tbase + 128u;
     int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
     if (!ok) rev_raise_error(1);
     if (__syncthreads_and(ok)) {
-        // ---- Cm: C folded at its own sub-block's end, hi + lo; C.B partials
+        // ---- Bo (B at its sub-block's start) and Cm (C at its sub-block's end), hi + lo
         {
             const int t = tid & 63, grp = tid >> 6;
             const int kb = t >> 4;
-            const float ds = f32[F_S + t] - f32[F_S + 16 * kb + 15];   // <= 0
-            const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
+            const float St = f32[F_S + t];
+            const float dsb = St - (kb == 0 ? 0.f : f32[F_S + 16 * kb - 1]);   // >= 0
+            const float dse = St - f32[F_S + 16 * kb + 15];                     // <= 0
+            const float sig = f32[F_SIG + t];
+            const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
-            for (int k = 0; k < NP / (8 * gbk::RG); ++k) {
-                const int r0 = 8 * (grp + gbk::RG * k);
+            for (int k = 0; k < NP / (8 * fuk::RG); ++k) {
+                const int r0 = 8 * (grp + fuk::RG * k);
                 if (r0 >= N) break;
-                float rc[8], rb[8], v[8];
+                float rc[8], rb[8], vb[8], vc[8];
                 ld_rows8(sC, t, r0, rc);
                 ld_rows8(sB, t, r0, rb);
 #pragma unroll
@@ -817,79 +844,85 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     const int r = r0 + j;
                     corr = fmaf(rc[j], rb[j], fmaf(rc[j + 1], rb[j + 1], corr));
                     if (r < nr) {
-                        v[j] = rc[j] * ex2_fast(fminf(f32[F_A2 + r] * ds, 120.f));
-                        v[j + 1] = rc[j + 1] * ex2_fast(fminf(f32[F_A2 + r + 1] * ds, 120.f));
+                        const float a0 = f32[F_A2 + r], a1 = f32[F_A2 + r + 1];
+                        vb[j] = sig * rb[j] * ex2_fast(fminf(-a0 * dsb, 120.f));
+                        vb[j + 1] = sig * rb[j + 1] * ex2_fast(fminf(-a1 * dsb, 120.f));
+                        vc[j] = rc[j] * ex2_fast(fminf(a0 * dse, 120.f));
+                        vc[j + 1] = rc[j + 1] * ex2_fast(fminf(a1 * dse, 120.f));
                     } else {
                         const int m = nr + ((r - nr) >> 1);
+                        const float a = f32[F_A2 + m], w = f32[F_W + m];
                         float sn, cs;
-                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
-                        const float ec = ex2_fast(fminf(f32[F_A2 + m] * ds, 120.f));
-                        v[j] = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
-                        v[j + 1] = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
+                        __sincosf(w * dsb, &sn, &cs);
+                        const float eb = sig * ex2_fast(fminf(-a * dsb, 120.f));
+                        vb[j] = eb * fmaf(rb[j], cs, rb[j + 1] * sn);
+                        vb[j + 1] = eb * fmaf(rb[j + 1], cs, -rb[j] * sn);
+                        __sincosf(w * dse, &sn, &cs);
+                        const float ec = ex2_fast(fminf(a * dse, 120.f));
+                        vc[j] = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
+                        vc[j + 1] = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
                     }
                 }
-                st16_split(sm + gbk::SM_CM, sm + gbk::SM_CML, off_mnmaj(r0, t, 2048u, 128u), v);
+                const uint32_t off = off_kmaj(t, r0, KM_LBO, KM_SBO);
+                st16_split(sm + fuk::SM_BO, sm + fuk::SM_BOL, off, vb);
+                st16_split(sm + fuk::SM_CM, sm + fuk::SM_CML, off, vc);
             }
-            reinterpret_cast<float *>(sm + gbk::SM_GM)[grp * 64 + t] = corr;   // G' tiles come later
+            reinterpret_cast<float *>(sm + fuk::SM_GM)[grp * 64 + t] = corr;   // G tiles come later
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
 
-        // this thread's rows of the per-head dC (forward-direction part), in flight during the MMAs
-        float kd[gbk::TPT];
-        {
-            const int n = tid & 127, tq = tid >> 7;
-#pragma unroll
-            for (int i2 = 0; i2 < gbk::TPT; ++i2) {
-                const int t = t0 + gbk::TPT * tq + i2;
-                kd[i2] = (n < N && t < L) ? __ldg(p.ws_dC + ix_wsk(p, b, t, h, 0, 1, n)) : 0.f;
-            }
-        }
-        // ---- phase A: G' = X dY^T ; V2 = Gc X^T (hi + lo)
+        // ---- phase A: V = K_prev dY^T, V2 = Gc X^T (hi + lo), G = dY X^T ---------
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t x_base = smem_u32(sm + gbk::SM_X), dy_base = smem_u32(sm + gbk::SM_DY);
-            const uint32_t id_g = idesc_bf16(64, 64, false, false);
-            for (int s = 0; s < PD / 16; ++s)
-                mma_bf16(t_g, sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
+            const uint32_t x_base = smem_u32(sm + fuk::SM_X), dy_base = smem_u32(sm + fuk::SM_DY);
             const uint32_t id_v = idesc_bf16(128, 64, false, false);
             for (int part = 0; part < 2; ++part) {
-                const uint32_t gc_base = smem_u32(sm + (part ? gbk::SM_GCL : gbk::SM_GC));
-                for (int s = 0; s < PD / 16; ++s)
+                const uint32_t kt_base = smem_u32(sm + (part ? fuk::SM_KTL : fuk::SM_KT));
+                const uint32_t gc_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
+                for (int s = 0; s < PD / 16; ++s) {
+                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
                     mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
                              sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
                              part > 0 || s > 0);
+                }
             }
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int s = 0; s < PD / 16; ++s)
+                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
             mma_commit(&bar_mma[0]);
         }
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int k = 0; k < gbk::RG; ++k) cs += reinterpret_cast<const float *>(sm + gbk::SM_GM)[k * 64 + tid];
+            for (int k = 0; k < fuk::RG; ++k)
+                cs += reinterpret_cast<const float *>(sm + fuk::SM_GM)[k * 64 + tid];
             f32[F_CORR + tid] = cs;   // C_t . B_t
         }
         ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
         if (!ok) rev_raise_error(1);
         fence_after_sync();
         if (__syncthreads_and(ok)) {
-            // ---- masked G' rows -> K-major tiles (rows t of sub-block qd, K = t' >= t)
+            // ---- masked G (s <= t) -> four 16-row tiles (rows t, K = s); dy_t . u_t
             if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
                 const int qd = warp - 4;
                 for (int i = 0; i < NSB; ++i) {
                     float v[16];
                     tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
-                    if (lane < 16 && i >= qd) {
+                    if (lane < 16 && i <= qd) {
                         const int t = 16 * qd + lane;
                         float lo[8], hi[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            lo[j] = (16 * i + j >= t) ? v[j] : 0.f;
-                            hi[j] = (16 * i + 8 + j >= t) ? v[8 + j] : 0.f;
+                            lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
+                            hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
                         }
-                        unsigned char *gt = sm + gbk::SM_GM + qd * 2048;
-                        unsigned char *gl = sm + gbk::SM_GML + qd * 2048;
+                        unsigned char *gt = sm + fuk::SM_GM + qd * 2048;
+                        unsigned char *gl = sm + fuk::SM_GML + qd * 2048;
                         st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
                         st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
                         if (i == qd) {
@@ -905,20 +938,32 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
-            // ---- phase B: E_{j,k} = Cm_k (G' o mask)_{j,k}^T, hi*hi + hi*lo + lo*hi
+
+            // ---- phase B: D_{i,k} and E_{j,k}, hi*hi + hi*lo + lo*hi ---------------
             if (tid == 0) {
                 fence_after_sync();
-                const uint32_t id_e = idesc_bf16(128, 16, true, false);
-                const uint32_t a_off[3] = {gbk::SM_CM, gbk::SM_CM, gbk::SM_CML};
-                const uint32_t b_off[3] = {gbk::SM_GM, gbk::SM_GML, gbk::SM_GM};
+                const uint32_t id_d = idesc_bf16(128, 16, true, false);
+                const uint32_t id_e = idesc_bf16(128, 16, true, true);
+                const uint32_t bo_off[3] = {fuk::SM_BO, fuk::SM_BO, fuk::SM_BOL};
+                const uint32_t cm_off3[3] = {fuk::SM_CM, fuk::SM_CM, fuk::SM_CML};
+                const uint32_t g_off[3] = {fuk::SM_GM, fuk::SM_GML, fuk::SM_GM};
+                for (int i = 0; i < NSB; ++i)
+                    for (int k = 0; k <= i; ++k)
+                        for (int part = 0; part < 3; ++part)
+                            mma_bf16(tbase + d_col(i, k),
+                                     sdesc(smem_u32(sm + bo_off[part]) + k * 4096u, 2048u, 128u,
+                                           LAYOUT_NONE),
+                                     sdesc(smem_u32(sm + g_off[part]) + i * 2048u + k * 256u, 128u,
+                                           1024u, LAYOUT_NONE),
+                                     id_d, part > 0);
                 for (int j = 0; j < NSB; ++j)
                     for (int k = j; k < NSB; ++k)
                         for (int part = 0; part < 3; ++part)
-                            mma_bf16(tbase + ejk_col(j, k),
-                                     sdesc(smem_u32(sm + a_off[part]) + k * 4096u, 2048u, 128u,
+                            mma_bf16(tbase + e_col(j, k),
+                                     sdesc(smem_u32(sm + cm_off3[part]) + k * 4096u, 2048u, 128u,
                                            LAYOUT_NONE),
-                                     sdesc(smem_u32(sm + b_off[part]) + j * 2048u + k * 256u, 128u,
-                                           1024u, LAYOUT_NONE),
+                                     sdesc(smem_u32(sm + g_off[part]) + k * 2048u + j * 256u, 1024u,
+                                           128u, LAYOUT_NONE),
                                      id_e, part > 0);
                 mma_commit(&bar_mma[1]);
             }
@@ -926,40 +971,84 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             if (!ok) rev_raise_error(1);
             fence_after_sync();
             if (__syncthreads_and(ok)) {
-                // ---- unfold: gbu_t = conj(e^{lam (Se_j - S_t)}) (conj(F[j+1][4]) V2_t + E_t),
-                // then, per state mode, the within-chunk suffix sums of the decay-gradient
-                // identity (X_t - Y_t, X = conj(c) dCK, Y = b conj(sigma gbu)), walking the
-                // tokens backwards; and dB / dC directly when a group has one head.
-                // Thread (row n, token group tq) takes tokens TPT tq .. TPT tq + TPT - 1.
-                float *red = reinterpret_cast<float *>(sm + gbk::SM_RED);    // [128][RED_LD] B . gbu
-                float *red2 = reinterpret_cast<float *>(sm + gbk::SM_RED2);  // [128][RED_LD] ddt terms
-                float *xch = reinterpret_cast<float *>(sm + gbk::SM_XCH);    // group totals, partials
-                const int n = tid & 127, tq = tid >> 7, qd = warp & 3;
+                // ---- unfold: thread (row n, sub-block i) -----------------------------
+                float *red = reinterpret_cast<float *>(sm + fuk::SM_RED);    // [128][RED_LD] B . gbu
+                float *red2 = reinterpret_cast<float *>(sm + fuk::SM_RED2);  // [128][RED_LD] ddt terms
+                float *xch = reinterpret_cast<float *>(sm + fuk::SM_XCH);    // group totals, partials
+                const int n = tid & 127, i = tid >> 7, qd = warp & 3;
                 const bool valid = n < N;
                 const int m = n < nr ? n : nr + ((n - nr) >> 1);
                 const bool pr_row = valid && n >= nr;
                 const bool im_row = pr_row && ((n - nr) & 1);
                 const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
-                // d ddt / d(suffix sum): a for the real part, -theta for the imaginary part
+                const int tc = 16 * i;
+
+                // part 1: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} sum_k F[k][i] D_{i,k}
+                float kk[16];
+                {
+                    float vv[16], dd[16];
+                    tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
+                    tmem_ld16(tmem_addr(tbase + d_col(i, i), 32u * qd, 0u), dd);
+                    for (int k = 0; k < i; ++k) {
+                        float ek[16];
+                        tmem_ld16(tmem_addr(tbase + d_col(i, k), 32u * qd, 0u), ek);
+                        const float fr = valid ? f32[F_KRE + fslot(k, i) * NP + m] : 0.f;
+                        const float fi = valid ? f32[F_KIM + fslot(k, i) * NP + m] : 0.f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
+                            // own component of (fr + i fi)(re + i im)
+                            dd[j] = pr_row ? fmaf(fr, ek[j], fmaf(im_row ? fi : -fi, other, dd[j]))
+                                           : fmaf(fr, ek[j], dd[j]);
+                        }
+                    }
+                    const float Sb = i == 0 ? 0.f : f32[F_S + 16 * i - 1];
+                    float fr = 1.f, fi = 0.f;   // F[0][i] = e^{lam Sb_i}
+                    if (i && valid) {
+                        fr = f32[F_KRE + gslot(i) * NP + m];
+                        fi = -f32[F_KIM + gslot(i) * NP + m];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float ds = f32[F_S + tc + j] - Sb;
+                        const float mag = ex2_fast(a2 * ds);
+                        float er = mag, ei = 0.f;
+                        if (pr_row) {
+                            float sn, cs;
+                            __sincosf(w * ds, &sn, &cs);
+                            er = mag * cs;
+                            ei = mag * sn;
+                        }
+                        float Er, Ei;
+                        cmul(er, ei, fr, fi, Er, Ei);
+                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                        const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
+                        if (!pr_row)
+                            kk[j] = fmaf(Er, vv[j], er * dd[j]);
+                        else if (!im_row)
+                            kk[j] = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
+                        else
+                            kk[j] = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
+                    }
+                }
+
+                // part 2: gbu, the decay-gradient suffix sums, dB / dC, walking backwards
                 const float coef = !valid ? 0.f : (im_row ? -w : a2 * 0.6931471805599453f);
                 const bool one_head = p.hpg == 1;
                 const long long tstride = (long long)p.H * p.N;
                 float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
-                const unsigned char *sB = sm + gbk::SM_B, *sC = sm + gbk::SM_C;
+                float *cdst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+                const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
                 float cum = 0.f, dacc = 0.f, sdt = 0.f;
-                const int tc = gbk::TPT * tq;
-#pragma unroll
-                for (int c16 = gbk::TPT / 16 - 1; c16 >= 0; --c16) {
+                {
                     float vv[16], ee[16];
-                    const int jb = (tc + 16 * c16) >> 4;   // sub-block of these 16 tokens
-                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)(tc + 16 * c16)), vv);
-                    tmem_ld16(tmem_addr(tbase + ejk_col(jb, jb), 32u * qd, 0u), ee);
-                    // later sub-blocks' contributions with their per-row factors conj(F[jb+1][k+1])
-                    for (int k = jb + 1; k < NSB; ++k) {
+                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)tc), vv);
+                    tmem_ld16(tmem_addr(tbase + e_col(i, i), 32u * qd, 0u), ee);
+                    for (int k = i + 1; k < NSB; ++k) {
                         float ek[16];
-                        tmem_ld16(tmem_addr(tbase + ejk_col(jb, k), 32u * qd, 0u), ek);
-                        const float f2r = valid ? f32[F_KRE + fslot(jb + 1, k + 1) * NP + m] : 0.f;
-                        const float f2i = valid ? f32[F_KIM + fslot(jb + 1, k + 1) * NP + m] : 0.f;
+                        tmem_ld16(tmem_addr(tbase + e_col(i, k), 32u * qd, 0u), ek);
+                        const float f2r = valid ? f32[F_KRE + fslot(i + 1, k + 1) * NP + m] : 0.f;
+                        const float f2i = valid ? f32[F_KIM + fslot(i + 1, k + 1) * NP + m] : 0.f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
@@ -968,15 +1057,15 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                                            : fmaf(f2r, ek[j], ee[j]);
                         }
                     }
-                    const float se = f32[F_S + 16 * jb + 15];
-                    float fr = 1.f, fi = 0.f;
-                    if (jb < 3 && valid) {
-                        fr = f32[F_KRE + fslot(jb + 1, 4) * NP + m];
-                        fi = f32[F_KIM + fslot(jb + 1, 4) * NP + m];
+                    const float se = f32[F_S + tc + 15];
+                    float fr = 1.f, fi = 0.f;   // F[i+1][4]
+                    if (i < 3 && valid) {
+                        fr = f32[F_KRE + fslot(i + 1, 4) * NP + m];
+                        fi = f32[F_KIM + fslot(i + 1, 4) * NP + m];
                     }
 #pragma unroll
                     for (int j = 15; j >= 0; --j) {
-                        const int t = tc + 16 * c16 + j;
+                        const int t = tc + j;
                         const float ds = se - f32[F_S + t];   // >= 0
                         const float mag = ex2_fast(a2 * ds);
                         float er = mag, ei = 0.f;
@@ -992,7 +1081,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         if (!pr_row) {
                             res = er * fmaf(fr, vv[j], ee[j]);
                         } else {
-                            // own row is re (im_row false) or im; W = conj(F) V + E
+                            // own row is re (im_row false) or im; W = conj(F) V2 + E
                             const float vr = im_row ? vo : vv[j], vi = im_row ? vv[j] : vo;
                             const float e_r = im_row ? eo : ee[j], e_i = im_row ? ee[j] : eo;
                             const float wr = fmaf(fr, vr, fmaf(fi, vi, e_r));
@@ -1004,58 +1093,60 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         const float m2 = f32[F_LAM + t], bn = f32[F_BN + t];
                         const float sig = f32[F_SIG + t], dtv = f32[F_DT + t];
                         const float bt = ld_row1(sB, t, n), ct = ld_row1(sC, t, n);
-                        const float kk = fmaf(bn * m2, bt, kd[16 * c16 + j]);   // dCK = dC + beta' <dy,u> b
+                        const float k_ = kk[j];                          // dCK_t
+                        const float dCt = fmaf(-bn * m2, bt, k_);        // dC_t
                         const float gg = sig * res;
                         const float co = __shfl_xor_sync(0xffffffffu, ct, 1);
-                        const float ko = __shfl_xor_sync(0xffffffffu, kk, 1);
+                        const float ko = __shfl_xor_sync(0xffffffffu, k_, 1);
                         const float bo = __shfl_xor_sync(0xffffffffu, bt, 1);
                         const float go = __shfl_xor_sync(0xffffffffu, gg, 1);
                         float v;
                         if (!pr_row)
-                            v = fmaf(ct, kk, -bt * gg);
+                            v = fmaf(ct, k_, -bt * gg);
                         else if (!im_row)   // Re(conj(c) k) - Re(b conj(g))
-                            v = fmaf(ct, kk, fmaf(co, ko, -fmaf(bt, gg, bo * go)));
+                            v = fmaf(ct, k_, fmaf(co, ko, -fmaf(bt, gg, bo * go)));
                         else                // Im(conj(c) k) - Im(b conj(g)), own row = im
-                            v = fmaf(co, kk, fmaf(-ct, ko, -fmaf(bt, go, -bo * gg)));
+                            v = fmaf(co, k_, fmaf(-ct, ko, -fmaf(bt, go, -bo * gg)));
                         if (!tv) v = 0.f;
                         cum += v;
                         dacc = fmaf(dtv, im_row ? -cum : cum, dacc);
                         sdt += dtv;
-                        red2[n * gbk::RED_LD + t] = coef * cum;
-                        red[n * gbk::RED_LD + t] = tv ? res * bt : 0.f;
+                        red2[n * fuk::RED_LD + t] = coef * cum;
+                        red[n * fuk::RED_LD + t] = tv ? res * bt : 0.f;
                         if (tv) {
                             if (one_head) {
                                 const int tg = t0 + t;
                                 reinterpret_cast<__nv_bfloat16 *>(p.dBm)[ix_B(p, b, tg, g, 0, n)] =
                                     __float2bfloat16_rn(fmaf(-bn * ct, m2, gg));
                                 reinterpret_cast<__nv_bfloat16 *>(p.dCm)[ix_C(p, b, tg, g, 0, n)] =
-                                    __float2bfloat16_rn(kd[16 * c16 + j]);
+                                    __float2bfloat16_rn(dCt);
                             } else {
                                 gdst[(long long)t * tstride] = res;
+                                cdst[(long long)t * tstride] = dCt;
                             }
                         }
                     }
                 }
-                // later token groups carry into every token of earlier ones
-                xch[tq * 128 + n] = cum;
+                // later sub-blocks carry into every token of earlier ones
+                xch[i * 128 + n] = cum;
                 __syncthreads();
                 float later = 0.f;
-                for (int k = tq + 1; k < gbk::TQ; ++k) later += xch[k * 128 + n];
+                for (int k = i + 1; k < fuk::TQ; ++k) later += xch[k * 128 + n];
                 if (later != 0.f) {
                     const float add = coef * later;
-                    for (int t = tc; t < tc + gbk::TPT; ++t) red2[n * gbk::RED_LD + t] += add;
+                    for (int t = tc; t < tc + 16; ++t) red2[n * fuk::RED_LD + t] += add;
                 }
                 dacc += (im_row ? -later : later) * sdt;
-                xch[(gbk::TQ + tq) * 128 + n] = dacc;
+                xch[(fuk::TQ + i) * 128 + n] = dacc;
                 __syncthreads();
-                if (tq == 0 && valid) {
+                if (i == 0 && valid) {
                     float tot = 0.f, da = 0.f;
-                    for (int k = 0; k < gbk::TQ; ++k) {
+                    for (int k = 0; k < fuk::TQ; ++k) {
                         tot += xch[k * 128 + n];
-                        da += xch[(gbk::TQ + k) * 128 + n];
+                        da += xch[(fuk::TQ + k) * 128 + n];
                     }
                     const int nmode = p.nr + p.np;
-                    float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
+                    float *blk = p.ws_blk + u * (4 * nmode + 2);
                     if (!pr_row) {
                         blk[4 * m + 0] = tot;
                         blk[4 * m + 1] = 0.f;
@@ -1070,36 +1161,36 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     }
                 }
                 // column sums over the state rows: all threads, 128 / RG rows each, fixed order
-                float *part = xch + 2 * gbk::TQ * 128;   // [2][RG][64]
+                float *part = xch + 2 * fuk::TQ * 128;   // [2][RG][64]
                 {
                     const int t = tid & 63, rg = tid >> 6;
-                    constexpr int RPG = NP / gbk::RG;
+                    constexpr int RPG = NP / fuk::RG;
                     float s1 = 0.f, s2 = 0.f;
                     for (int k = rg * RPG; k < rg * RPG + RPG && k < N; ++k) {
-                        s1 += red[k * gbk::RED_LD + t];
-                        s2 += red2[k * gbk::RED_LD + t];
+                        s1 += red[k * fuk::RED_LD + t];
+                        s2 += red2[k * fuk::RED_LD + t];
                     }
                     part[rg * 64 + t] = s1;
-                    part[(gbk::RG + rg) * 64 + t] = s2;
+                    part[(fuk::RG + rg) * 64 + t] = s2;
                 }
                 __syncthreads();
                 if (tid < 64 && t0 + tid < L) {
                     const int t = tid;
                     float dsig = 0.f, dd = 0.f;
-                    for (int k = 0; k < gbk::RG; ++k) {
+                    for (int k = 0; k < fuk::RG; ++k) {
                         dsig += part[k * 64 + t];
-                        dd += part[(gbk::RG + k) * 64 + t];
+                        dd += part[(fuk::RG + k) * 64 + t];
                     }
-                    const long long i = ix_bth(p, b, t0 + t, h);
+                    const long long ii = ix_bth(p, b, t0 + t, h);
                     const float m2 = f32[F_LAM + t];
-                    p.ws_tok[2 * i] = dsig;
-                    p.ws_tok[2 * i + 1] = f32[F_CORR + t] * m2;
-                    p.ws_M2[i] = m2;
-                    p.ws_ddt[i] = dd;
+                    p.ws_tok[2 * ii] = dsig;
+                    p.ws_tok[2 * ii + 1] = f32[F_CORR + t] * m2;
+                    p.ws_M2[ii] = m2;
+                    p.ws_ddt[ii] = dd;
                 }
                 if (tid == 64) {
                     const int nmode = p.nr + p.np;
-                    float *blk = p.ws_blk + bhc(p, b, h, c) * (4 * nmode + 2);
+                    float *blk = p.ws_blk + u * (4 * nmode + 2);
                     float st_ = 0.f, dD = 0.f;
                     for (int t = 0; t < Q; ++t) {
                         st_ += f32[F_DT + t];
@@ -1117,290 +1208,7 @@ k_chunk_bwd_gbu(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     __syncthreads();
     if (warp == 0) {
         fence_after_sync();
-        tmem_dealloc(tbase, gbk::TMEM_COLS);
-    }
-}
-
-// ============================================================================
-// k_chunk_bwd_dc: per chunk, dC_t = dy_t H_t^T per head.
-//   H_t = K_t - beta_{t+1} W_t,   K_t = e^{lam S_t} K_prev + sum_{s<=t} Phi_{t,s} sigma_s b_s u_s
-// so, per state mode (complex for rotation pairs, real rows otherwise), for t
-// in sub-block i,
-//   dCK_t = e^{lam S_t} (dy_t . K_prev)
-//         + e^{lam (S_t - Sb_i)} sum_{k <= i} F[k][i] sum_{s in block k, s <= t} (dy_t . u_s) Bo_s
-// with Bo_s = sigma_s b_s e^{lam (Sb_k - S_s)} folded at its own sub-block's
-// start (the factor F[k][i] = e^{lam (Sb_i - Sb_k)} is per state row, so it is
-// applied after the contraction over tokens).  On the tensor cores (operands
-// split into bf16 hi + lo):
-//   V^T      = K_prev (N x 64 p) . dY^T (64 p x 64 t)                 M=128, N=64, K=64
-//   G        = dY (64 t x 64 p) . X^T (64 p x 64 s)                   M=64,  N=64, K=64
-//   D_{i,k}  = Bo_k^T (N x 16 s) . (G o causal mask)_{i,k}^T (16 s x 16 t)  M=128, N=16, K=16
-// then the per-(t, row) unfold on the CUDA cores; dC_t = dCK_t -
-// beta_{t+1} (dy_t . u_t) B_t.  K_prev is the state entering the chunk.
-// ============================================================================
-namespace dck {
-constexpr int THREADS = 512;
-constexpr int RG = THREADS / 64;    // row groups of the operand preparation
-constexpr int TQ = THREADS / 128;   // token groups of the unfold (one sub-block each)
-constexpr int TPT = Q / TQ;         // tokens per thread in the unfold
-static_assert(TPT == 16, "the unfold takes one 16-token sub-block per thread");
-constexpr uint32_t TMEM_COLS = 512;   // V 64 | G 64 | D_{i,k} 10 x 16
-constexpr uint32_t SM_X = 0;          // 8 KB  x (128B swizzle)
-constexpr uint32_t SM_DY = 8192;      // 8 KB  dy (128B swizzle)
-constexpr uint32_t SM_B = 16384;      // 16 KB raw B (two 64-row swizzled halves)
-constexpr uint32_t SM_BO = 32768;     // 16 KB Bo hi, K-major (rows s, K = state rows)
-constexpr uint32_t SM_BOL = 49152;    // 16 KB Bo lo
-constexpr uint32_t SM_GM = 65536;     // 8 KB  masked G hi: 4 tiles, K-major (N = 16 t, K = s)
-constexpr uint32_t SM_GML = 73728;    // 8 KB  masked G lo
-constexpr uint32_t SM_KT = 81920;     // 16 KB K_prev hi, K-major (rows n, K = p)
-constexpr uint32_t SM_KTL = 98304;    // 16 KB K_prev lo
-constexpr uint32_t SM_F32 = 114688;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
-}  // namespace dck
-
-// TMEM column of D_{i,k} (k <= i): 10 blocks of 16 columns after V and G
-__device__ __forceinline__ uint32_t dik_col(int i, int k) {
-    return 128u + 16u * (uint32_t)(i * (i + 1) / 2 + k);
-}
-
-__global__ void __launch_bounds__(dck::THREADS, 1)
-k_chunk_bwd_dc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmDY, Params p) {
-    if (gated_off(p)) return;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + dck::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dck::SM_BAR);
-    uint64_t *bar_mma = bar_tma + 1;   // [2]
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / p.hpg;
-    const int N = p.N, nr = p.nr, L = p.L;
-    const int t0 = c * Q;
-    const int nbox = N / 64;
-
-    if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(&bar_mma[0], 1);
-        mbar_init(&bar_mma[1], 1);
-        mbar_fence_init();
-        tma_prefetch_desc(&tmX);
-        tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + Q * N * 2));
-        tma_load_4d(sm + dck::SM_X, &tmX, bar_tma, 0, h, t0, b);
-        tma_load_4d(sm + dck::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
-        for (int k = 0; k < nbox; ++k)
-            tma_load_4d(sm + dck::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
-    }
-    if (warp == 0) tmem_alloc(tslot, dck::TMEM_COLS);
-    mode_rates(p, f32, h);
-    if (N < NP)  // M padding of the Bo tiles
-        for (int i = tid; i < (int)((dck::SM_GM - dck::SM_BO) / 16); i += dck::THREADS)
-            reinterpret_cast<uint4 *>(sm + dck::SM_BO)[i] = make_uint4(0, 0, 0, 0);
-    load_state_tile(p.ws_kp + bhc(p, b, h, c) * N * PD, N, sm + dck::SM_KT, sm + dck::SM_KTL);
-    chunk_tokens(p, f32, b, h, t0, true);
-    chunk_mode_constants(p, f32);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tbase = *tslot;
-    const uint32_t t_v = tbase;           // V^T (M=128), cols 0..63
-    const uint32_t t_g = tbase + 64u;     // G (M=64, lanes 0-15 per quarter), cols 64..127
-    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
-    if (!ok) rev_raise_error(1);
-    if (__syncthreads_and(ok)) {
-        // ---- Bo: B folded at its own sub-block's start, hi + lo ----------------
-        {
-            const int t = tid & 63, grp = tid >> 6;
-            const int ib = t >> 4;
-            const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-            const float ds = f32[F_S + t] - Sb;
-            const float sig = f32[F_SIG + t];
-            const unsigned char *sB = sm + dck::SM_B;
-#pragma unroll 1
-            for (int k = 0; k < NP / (8 * dck::RG); ++k) {
-                const int r0 = 8 * (grp + dck::RG * k);
-                if (r0 >= N) break;
-                float v[8], rb[8];
-                ld_rows8(sB, t, r0, rb);
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    const int r = r0 + j;
-                    const float b0 = rb[j], b1 = rb[j + 1];
-                    if (r < nr) {
-                        v[j] = sig * b0 * ex2_fast(fminf(-f32[F_A2 + r] * ds, 120.f));
-                        v[j + 1] = sig * b1 * ex2_fast(fminf(-f32[F_A2 + r + 1] * ds, 120.f));
-                    } else {
-                        const int m = nr + ((r - nr) >> 1);
-                        float sn, cs;
-                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
-                        const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m] * ds, 120.f));
-                        v[j] = eb * fmaf(b0, cs, b1 * sn);
-                        v[j + 1] = eb * fmaf(b1, cs, -b0 * sn);
-                    }
-                }
-                st16_split(sm + dck::SM_BO, sm + dck::SM_BOL, off_kmaj(t, r0, KM_LBO, KM_SBO), v);
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-
-        // ---- phase A: V^T = K_prev dY^T (hi + lo), G = dY X^T --------------------
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t x_base = smem_u32(sm + dck::SM_X), dy_base = smem_u32(sm + dck::SM_DY);
-            const uint32_t id_v = idesc_bf16(128, 64, false, false);
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t kt_base = smem_u32(sm + (part ? dck::SM_KTL : dck::SM_KT));
-                for (int s = 0; s < PD / 16; ++s)
-                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                             part > 0 || s > 0);
-            }
-            const uint32_t id_g = idesc_bf16(64, 64, false, false);
-            for (int s = 0; s < PD / 16; ++s)
-                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
-            mma_commit(&bar_mma[0]);
-        }
-        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
-        fence_after_sync();
-        if (__syncthreads_and(ok)) {
-            // ---- masked G rows -> K-major tiles (N = 16 t of block i, K = s); dy_t . u_t
-            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
-                const int qd = warp - 4;
-                for (int i = 0; i < NSB; ++i) {
-                    float v[16];
-                    tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
-                    if (lane < 16 && i <= qd) {
-                        const int t = 16 * qd + lane;
-                        float lo[8], hi[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
-                            hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
-                        }
-                        unsigned char *gt = sm + dck::SM_GM + qd * 2048;
-                        unsigned char *gl = sm + dck::SM_GML + qd * 2048;
-                        st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
-                        st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
-                        if (i == qd) {
-                            float dg = 0.f;
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (j == lane) dg = v[j];
-                            f32[F_CORR + t] = dg;   // <dy_t, u_t>
-                        }
-                    }
-                }
-            }
-            fence_proxy_async();
-            fence_before_sync();
-            __syncthreads();
-
-            // ---- phase B: D_{i,k} = Bo_k^T (G o mask)_{i,k}^T, hi*hi + hi*lo + lo*hi
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t id_d = idesc_bf16(128, 16, true, false);
-                const uint32_t a_off[3] = {dck::SM_BO, dck::SM_BO, dck::SM_BOL};
-                const uint32_t b_off[3] = {dck::SM_GM, dck::SM_GML, dck::SM_GM};
-                for (int i = 0; i < NSB; ++i)
-                    for (int k = 0; k <= i; ++k)
-                        for (int part = 0; part < 3; ++part)
-                            mma_bf16(tbase + dik_col(i, k),
-                                     sdesc(smem_u32(sm + a_off[part]) + k * 4096u, 2048u, 128u,
-                                           LAYOUT_NONE),
-                                     sdesc(smem_u32(sm + b_off[part]) + i * 2048u + k * 256u, 128u,
-                                           1024u, LAYOUT_NONE),
-                                     id_d, part > 0);
-                mma_commit(&bar_mma[1]);
-            }
-            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
-            if (!ok) rev_raise_error(1);
-            fence_after_sync();
-            if (__syncthreads_and(ok)) {
-                // ---- unfold for the 16 tokens of sub-block i = tq:
-                //      D = sum_k F[k][i] D_{i,k};  dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} D
-                //      dC_t = dCK_t - beta' (dy.u) B_t
-                const int n = tid & 127, i = tid >> 7, qd = warp & 3;
-                const bool valid = n < N;
-                const int m = n < nr ? n : nr + ((n - nr) >> 1);
-                const bool pr_row = valid && n >= nr;
-                const bool im_row = pr_row && ((n - nr) & 1);
-                const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
-                float *dst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
-                const long long tstride = (long long)p.H * p.N;
-                const unsigned char *sB = sm + dck::SM_B;
-                const int tc = 16 * i;
-                float vv[16], dd[16];
-                tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
-                tmem_ld16(tmem_addr(tbase + dik_col(i, i), 32u * qd, 0u), dd);
-                // earlier sub-blocks' contributions, with their per-row factors F[k][i]
-                for (int k = 0; k < i; ++k) {
-                    float ek[16];
-                    tmem_ld16(tmem_addr(tbase + dik_col(i, k), 32u * qd, 0u), ek);
-                    const float fr = valid ? f32[F_KRE + fslot(k, i) * NP + m] : 0.f;
-                    const float fi = valid ? f32[F_KIM + fslot(k, i) * NP + m] : 0.f;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
-                        // own component of (fr + i fi)(re + i im)
-                        dd[j] = pr_row ? fmaf(fr, ek[j], fmaf(im_row ? fi : -fi, other, dd[j]))
-                                       : fmaf(fr, ek[j], dd[j]);
-                    }
-                }
-                const float Sb = i == 0 ? 0.f : f32[F_S + 16 * i - 1];
-                // E = E' conj(G_i) = E' F[0][i]
-                float fr = 1.f, fi = 0.f;
-                if (i && valid) {
-                    fr = f32[F_KRE + gslot(i) * NP + m];
-                    fi = -f32[F_KIM + gslot(i) * NP + m];
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = tc + j;
-                    const float ds = f32[F_S + t] - Sb;
-                    const float mag = ex2_fast(a2 * ds);
-                    float er = mag, ei = 0.f;
-                    if (pr_row) {
-                        float sn, cs;
-                        __sincosf(w * ds, &sn, &cs);
-                        er = mag * cs;
-                        ei = mag * sn;
-                    }
-                    float Er, Ei;
-                    cmul(er, ei, fr, fi, Er, Ei);
-                    const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
-                    const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
-                    float res;
-                    if (!pr_row)
-                        res = fmaf(Er, vv[j], er * dd[j]);
-                    else if (!im_row)   // real part of E (V_re + i V_im) + E' (D_re + i D_im)
-                        res = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
-                    else                // imaginary part
-                        res = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
-                    if (valid && t0 + t < L) {
-                        const float bt = ld_row1(sB, t, n);
-                        dst[(long long)t * tstride] = res - f32[F_BN + t] * f32[F_CORR + t] * bt;
-                    }
-                }
-            }
-        }
-    } else if (tid == 0) {
-        mbar_wait(bar_tma, 0, WAIT_LIMIT);
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        fence_after_sync();
-        tmem_dealloc(tbase, dck::TMEM_COLS);
+        tmem_dealloc(tbase, fuk::TMEM_COLS);
     }
 }
 
@@ -1419,28 +1227,16 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
 
 cudaError_t chunk_states(const Params &p, cudaStream_t st);
 
-// Forward-direction part of the tensor-core backward: the state entering every
-// chunk (p.ws_kp, p.ws_ce; taken from the forward when p.states_ready), then the
-// per-head dC of every chunk (p.ws_dC).
-cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st) {
-    using namespace chunkrev;
-    cudaError_t e = p.states_ready ? cudaSuccess : chunk_states(p, st);
-    if (e != cudaSuccess) return e;
-    CUtensorMap mx, mb, mdy;
-    if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
-        !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
-        !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
-        return cudaErrorInvalidValue;
-    static bool a = false;
-    if ((e = set_smem(k_chunk_bwd_dc, dck::SMEM_BYTES, a)) != cudaSuccess) return e;
-    k_chunk_bwd_dc<<<dim3(p.nc, p.H, p.Bsz), dck::THREADS, dck::SMEM_BYTES, st>>>(mx, mb, mdy, p);
-    profile_mark(st, "k_chunk_bwd_dc");
-    return cudaGetLastError();
+// The state entering every chunk for the tensor-core backward (p.ws_kp,
+// p.ws_ce), unless the forward's are given (p.states_ready).
+cudaError_t chunk_bwd_states(const Params &p, cudaStream_t st) {
+    return p.states_ready ? cudaSuccess : chunk_states(p, st);
 }
 
-// Reverse part of the tensor-core backward: dx, gbu / dsigma / <dy, u>, the
-// exact chunk-boundary values, dh0 / dw0 / dbeta_0.  Needs p.ws_gc, p.ws_ce and
-// p.ws_kp (written by the forward-direction part) and p.ws_qb.
+// The rest of the tensor-core backward: the chunk-local adjoints, the reverse
+// pass (exact chunk-boundary values, dh0 / dw0 / dbeta_0), dx, and the fused
+// per-chunk kernel (dC, gbu, dsigma, <dy, u>, the within-chunk decay sums, dB
+// / dC).  Needs p.ws_kp and p.ws_ce from chunk_bwd_states.
 cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     using namespace chunkrev;
     CUtensorMap mx, mb, mc, mdy;
@@ -1453,7 +1249,7 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     cudaError_t e;
     if ((e = set_smem(k_chunk_adj_local, loc::SMEM_BYTES, a1)) != cudaSuccess) return e;
     if ((e = set_smem(k_chunk_bwd_dx, dxk::SMEM_BYTES, a3)) != cudaSuccess) return e;
-    if ((e = set_smem(k_chunk_bwd_gbu, gbk::SMEM_BYTES, a4)) != cudaSuccess) return e;
+    if ((e = set_smem(k_chunk_bwd_fused, fuk::SMEM_BYTES, a4)) != cudaSuccess) return e;
     const dim3 grid(p.nc, p.H, p.Bsz);
     k_chunk_adj_local<<<grid, loc::THREADS, loc::SMEM_BYTES, st>>>(mc, mdy, p);
     profile_mark(st, "k_chunk_adj_local");
@@ -1471,8 +1267,8 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         profile_mark(st, "k_chunk_bwd_dx");
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_chunk_bwd_gbu<<<grid, gbk::THREADS, gbk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
-    profile_mark(st, "k_chunk_bwd_gbu");
+    k_chunk_bwd_fused<<<grid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
+    profile_mark(st, "k_chunk_bwd_fused");
     return cudaGetLastError();
 }
 

@@ -1145,7 +1145,7 @@ cudaError_t simt_forward(const Params &p, cudaStream_t st) {
 }
 
 bool chunk_bwd_supported(const Params &p);
-cudaError_t chunk_bwd_dc(const Params &p, cudaStream_t st);
+cudaError_t chunk_bwd_states(const Params &p, cudaStream_t st);
 cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st);
 
 // Finalize passes shared by both backward chains: within-block decay sums
@@ -1194,12 +1194,12 @@ cudaError_t simt_backward(const Params &p, cudaStream_t st) {
     return bwd_finalize(p, st, true, true);
 }
 
-// Tensor-core backward: forward-direction dC, then the chunk-parallel reverse
-// part, which also produces the within-block decay sums (and dB / dC when every
-// group has one head), then the shared finalize passes.
+// Tensor-core backward: the chunk states (unless the forward's are given), the
+// chunk-parallel kernels, which also produce the within-block decay sums (and
+// dB / dC when every group has one head), then the shared finalize passes.
 cudaError_t chunk_backward(const Params &p, cudaStream_t st) {
     cudaError_t e;
-    if ((e = chunk_bwd_dc(p, st)) != cudaSuccess) return e;
+    if ((e = chunk_bwd_states(p, st)) != cudaSuccess) return e;
     if ((e = chunk_bwd_reverse(p, st)) != cudaSuccess) return e;
     return bwd_finalize(p, st, false, p.hpg != 1);
 }
