@@ -198,7 +198,8 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
     if (!tensor_chain_shape(d)) return w;
     const size_t units = (size_t)d->batch * d->nheads * (size_t)((d->seqlen + 63) / 64);
     w.off_kp = 0;
-    size_t off = align256(units * nstate(d) * d->headdim * 4);
+    // one 32 KB slot per chunk (128 state rows x 64, bf16 hi + lo tiles or the fp32 local sum)
+    size_t off = align256(units * 128 * d->headdim * 4);
     w.off_ce = off;
     off = align256(off + units * 128 * 2 * 4);
     w.total_infer = off;
@@ -239,11 +240,11 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     w.off_kp = w.off_qb = w.off_gc = w.off_ce = off;
     if (w.boundary) {
         w.off_kp = off;
-        off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * d->headdim * 4);
         w.off_qb = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 4 * N * 4);
         w.off_gc = off;
-        off = align256(off + (size_t)d->batch * d->nheads * ntb * N * d->headdim * 4);
+        off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * d->headdim * 4);
         w.off_ce = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * 2 * 4);
     }

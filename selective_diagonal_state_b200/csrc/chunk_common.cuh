@@ -210,70 +210,53 @@ __device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {
     return ((long long)b * p.H + h) * p.nc + c;
 }
 
-// fp32 state-shaped tile [n][64 p] (row stride 64; rows from N on read as 0)
-// -> bf16 operand tile with byte(n, p) = (n/8)*1024 + (p/8)*128 + (n%8)*16 +
-// (p%8)*2, which is both the K-major layout with rows n (K = p) and the
-// MN-major layout with M or N = p (K = n).  With `lo`, the bf16 residual goes
-// to the second tile.  Strided over the block's threads; no barrier.
-__device__ __forceinline__ void load_state_tile(const float *src, int N, unsigned char *hi,
-                                                unsigned char *lo) {
-    for (int it = threadIdx.x; it < NP * (PD / 8); it += blockDim.x) {
-        const int n = it >> 3, p8 = (it & 7) * 8;
-        float v[8];
-        if (n < N) {
-            const float4 a = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8));
-            const float4 d = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8 + 4));
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = 0.f;
-        }
-        const uint32_t off = off_kmaj(n, p8, 128u, 1024u);
-        if (lo)
-            st16_split(hi, lo, off, v);
-        else
-            st16(hi, off, v);
-    }
-}
+// ---- chunk states in the operand-tile format ----------------------------------
+// The state entering a chunk (and the adjoint carried into it) are stored per
+// chunk as 32 KB: the bf16 tile with byte(n, p) = (n/8)*1024 + (p/8)*128 +
+// (n%8)*16 + (p%8)*2 for 128 rows x 64 p (rows past N zero), then the tile of
+// the bf16 residuals v - hi.  That layout is both K-major with rows n (K = p)
+// and MN-major with M or N = p (K = n); consumers bulk-copy it straight into
+// their operand tiles.  Before the passes rewrite a slot, it holds the
+// chunk-local fp32 sum [N][64].
+constexpr int SLOT_FLOATS = NP * PD;            // floats per chunk slot
+constexpr uint32_t TILE_BYTES = NP * PD * 2;    // one bf16 tile
 
-// A state-shaped fp32 tile [n][64 p] held in registers between its global
-// load and its store as a bf16 operand (the load_state_tile layout), so that a
-// persistent kernel can fetch the next chunk's tile while it works on this one.
-template <int THREADS>
-struct StatePrefetch {
-    static constexpr int ITEMS = NP * (PD / 8) / THREADS;
-    float4 v[2 * ITEMS];
-};
-template <int THREADS>
-__device__ __forceinline__ void state_load(const float *src, int N, StatePrefetch<THREADS> &r) {
+// rows n0, n0 + 1 at p .. p + 3 (p a multiple of 4) -> hi / lo tiles
+__device__ __forceinline__ void tile_store_rows2(unsigned char *slot, int n0, int p,
+                                                 const float4 &a, const float4 &d) {
+    const uint32_t off = off_kmaj(n0, p, 128u, 1024u);   // row n0 + 1 is 16 bytes further
+    const float v[2][4] = {{a.x, a.y, a.z, a.w}, {d.x, d.y, d.z, d.w}};
 #pragma unroll
-    for (int j = 0; j < StatePrefetch<THREADS>::ITEMS; ++j) {
-        const int it = threadIdx.x + j * THREADS;
-        const int n = it >> 3, p8 = (it & 7) * 8;
-        if (n < N) {
-            r.v[2 * j] = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8));
-            r.v[2 * j + 1] = __ldg(reinterpret_cast<const float4 *>(src + (long long)n * PD + p8 + 4));
-        } else {
-            r.v[2 * j] = r.v[2 * j + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < 2; ++r) {
+        float h[4], l[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h[j] = __bfloat162float(__float2bfloat16_rn(v[r][j]));
+            l[j] = v[r][j] - h[j];
         }
+        *reinterpret_cast<uint2 *>(slot + off + 16 * r) =
+            make_uint2(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]));
+        *reinterpret_cast<uint2 *>(slot + TILE_BYTES + off + 16 * r) =
+            make_uint2(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
     }
 }
-template <int THREADS>
-__device__ __forceinline__ void state_store(const StatePrefetch<THREADS> &r, unsigned char *hi,
-                                            unsigned char *lo) {
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// hi + lo of rows n0, n0 + 1 at p .. p + 3
+__device__ __forceinline__ void tile_load_rows2(const unsigned char *slot, int n0, int p, float4 &a,
+                                                float4 &d) {
+    const uint32_t off = off_kmaj(n0, p, 128u, 1024u);
+    float4 o[2];
 #pragma unroll
-    for (int j = 0; j < StatePrefetch<THREADS>::ITEMS; ++j) {
-        const int it = threadIdx.x + j * THREADS;
-        const int n = it >> 3, p8 = (it & 7) * 8;
-        const float4 a = r.v[2 * j], d = r.v[2 * j + 1];
-        const float v[8] = {a.x, a.y, a.z, a.w, d.x, d.y, d.z, d.w};
-        const uint32_t off = off_kmaj(n, p8, 128u, 1024u);
-        if (lo)
-            st16_split(hi, lo, off, v);
-        else
-            st16(hi, off, v);
+    for (int r = 0; r < 2; ++r) {
+        const uint2 h = __ldg(reinterpret_cast<const uint2 *>(slot + off + 16 * r));
+        const uint2 l = __ldg(reinterpret_cast<const uint2 *>(slot + TILE_BYTES + off + 16 * r));
+        const float2 h0 = bf2_to_f2(h.x), h1 = bf2_to_f2(h.y), l0 = bf2_to_f2(l.x), l1 = bf2_to_f2(l.y);
+        o[r] = make_float4(h0.x + l0.x, h0.y + l0.y, h1.x + l1.x, h1.y + l1.y);
     }
+    a = o[0];
+    d = o[1];
 }
 
 // Work item of the persistent chunk kernels: chunk fastest, then head, then batch row.

@@ -53,7 +53,8 @@ using namespace chunkc;
 // chunk's full decay e^{lam S_63} per mode.
 // ============================================================================
 namespace stl {
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;
+constexpr int RG = THREADS / 64;   // row groups of the operand preparation
 constexpr uint32_t TMEM_COLS = 64;
 constexpr uint32_t SM_B = 0;        // 16 KB raw B (two 64-row 128B-swizzled halves)
 constexpr uint32_t SM_X = 16384;    // 8 KB  x (128B swizzle)
@@ -110,7 +111,7 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
     if (!ok) raise_error(1);
     if (__syncthreads_and(ok)) {
-        // Bh = (own-sub-block Bi) F[ib][4]; thread (t, grp) handles rows 8 (grp + 2k)
+        // Bh = (own-sub-block Bi) F[ib][4]; thread (t, grp) handles rows 8 (grp + RG k)
         const int t = tid & 63, grp = tid >> 6;
         const int ib = t >> 4;
         const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
@@ -119,8 +120,8 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const unsigned char *sB = sm + stl::SM_B;
         unsigned char *sv = p.sv_Bh ? p.sv_Bh + bhc(p, b, h, c) * 16384 : nullptr;
 #pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
-            const int r0 = 8 * (grp + 2 * k);
+        for (int k = 0; k < NP / (8 * stl::RG); ++k) {
+            const int r0 = 8 * (grp + stl::RG * k);
             if (r0 >= N) {
                 if (!sv) break;
                 // K padding of the saved tile
@@ -178,12 +179,13 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         if (!ok) raise_error(1);
         fence_after_sync();
         if (__syncthreads_and(ok)) {
-            const int n = tid;
-            float *dst = p.ws_kp + (bhc(p, b, h, c) * N + n) * PD;
+            // the chunk-local fp32 sum [N][64] at the start of the chunk's slot
+            const int n = 32 * (warp & 3) + (tid & 31), half = warp >> 2;
+            float *dst = p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS + n * PD;
 #pragma unroll
-            for (int c16 = 0; c16 < PD / 16; ++c16) {
+            for (int c16 = 2 * half; c16 < 2 * half + 2; ++c16) {
                 float v[16];
-                tmem_ld16(tmem_addr(tacc, 32u * warp, 16u * c16), v);
+                tmem_ld16(tmem_addr(tacc, 32u * (warp & 3), 16u * c16), v);
                 if (n < N) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
@@ -252,7 +254,8 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
     }
     s_ce[0][tid] = __ldg(p.ws_ce + bhc(p, b, h, 0) * (2 * NP) + tid);
     for (int c = 0; c < nc; ++c) {
-        float *sbase = p.ws_kp + bhc(p, b, h, c) * N * PD + q;
+        float *slot = p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS;
+        float *sbase = slot + q;
         float4 sv0[pas::KMAX], sv1[pas::KMAX];
 #pragma unroll
         for (int k = 0; k < pas::KMAX; ++k) {
@@ -263,14 +266,19 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
             }
         }
         if (c + 1 < nc) s_ce[(c + 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c + 1) * (2 * NP) + tid);
+        // every thread has read its part of S_c: the slot can take the state entering chunk c
         __syncthreads();
         const float *ce = s_ce[c % 3];
+        unsigned char *tile = reinterpret_cast<unsigned char *>(slot);
 #pragma unroll
         for (int k = 0; k < pas::KMAX; ++k) {
-            if (k >= nk) break;
             const int n0 = 2 * (rp0 + 16 * k);
-            *reinterpret_cast<float4 *>(sbase + (long long)n0 * PD) = k0[k];
-            *reinterpret_cast<float4 *>(sbase + (long long)(n0 + 1) * PD) = k1[k];
+            if (k >= nk) {   // rows past N read as zero by the consumers
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                tile_store_rows2(tile, n0, q, z, z);
+                continue;
+            }
+            tile_store_rows2(tile, n0, q, k0[k], k1[k]);
             float4 &a = k0[k], &d = k1[k];
             if (n0 < nr) {
                 const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
@@ -338,8 +346,8 @@ constexpr uint32_t SM_CI = 81920;     // 16 KB Ci   K-major (64 t x 128)
 constexpr uint32_t SM_CH = 98304;     // 16 KB Ch   K-major
 constexpr uint32_t SM_BI = 114688;    // 40 KB Bi tiles (16, 32, 48, 64 rows)
 constexpr uint32_t SM_P = 155648;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
-constexpr uint32_t SM_KT = 163840;    // 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
-constexpr uint32_t SM_F32 = 180224;
+constexpr uint32_t SM_KT = 163840;    // 2 x 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
+constexpr uint32_t SM_F32 = 196608;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 static_assert(THREADS * 16 == 8192, "one 16-byte piece of the saved P tiles per thread");
@@ -362,12 +370,15 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
     const int nbox = N / 64;
-    const uint32_t tile_bytes = (uint32_t)(Q * PD * 2 + 2 * Q * N * 2);
+    const uint32_t tile_bytes = (uint32_t)(Q * PD * 2 + 2 * Q * N * 2) + TILE_BYTES;
     auto issue_tma = [&](int item, int st) {
         const ChunkItem it = chunk_item(p, item);
         const int g = it.h / p.hpg, t0 = it.c * Q;
         mbar_expect_tx(&bar_tma[st], tile_bytes);
         tma_load_4d(sm + outk::SM_X + st * 8192, &tmX, &bar_tma[st], 0, it.h, t0, it.b);
+        // the state entering the chunk (bf16 tile, the hi part of its slot)
+        bulk_load(sm + outk::SM_KT + st * TILE_BYTES,
+                  p.ws_kp + bhc(p, it.b, it.h, it.c) * SLOT_FLOATS, TILE_BYTES, &bar_tma[st]);
         for (int k = 0; k < nbox; ++k) {
             tma_load_4d(sm + outk::SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g, t0,
                         it.b);
@@ -393,11 +404,9 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         for (int i = tid; i < (int)((outk::SM_P - outk::SM_CI) / 16); i += outk::THREADS)
             reinterpret_cast<uint4 *>(sm + outk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
     TokPrefetch tok;
-    StatePrefetch<outk::THREADS> kst;
     {
         const ChunkItem it = chunk_item(p, item);
         tok = tok_load(p, it.b, it.h, it.c * Q);
-        state_load(p.ws_kp + bhc(p, it.b, it.h, it.c) * N * PD, N, kst);
     }
     fence_before_sync();
     __syncthreads();
@@ -420,12 +429,10 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 
         // ---- this chunk's small inputs; the next chunk's in flight -----------
         mode_rates(p, f32, h);
-        state_store(kst, sm + outk::SM_KT, nullptr);
         chunk_tokens_from(p, f32, t0, tok, true);
         if (next < nitems) {
             const ChunkItem nx = chunk_item(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
-            state_load(p.ws_kp + bhc(p, nx.b, nx.h, nx.c) * N * PD, N, kst);
             // the other stage was last read by the previous chunk, which is complete
             if (tid == 0) issue_tma(next, st ^ 1);
         }
@@ -538,7 +545,8 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              id_sc, s > 0);
-            const uint32_t kt_base = smem_u32(sm + outk::SM_KT), ch_base = smem_u32(sm + outk::SM_CH);
+            const uint32_t kt_base = smem_u32(sm + outk::SM_KT + st * TILE_BYTES);
+            const uint32_t ch_base = smem_u32(sm + outk::SM_CH);
             const uint32_t id_y = idesc_bf16(64, 64, true, false);
             for (int s = 0; s < NP / 16; ++s)
                 mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),

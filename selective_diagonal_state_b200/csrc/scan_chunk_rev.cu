@@ -13,7 +13,8 @@
 //   k_chunk_adj_local  (every chunk at once)   Ghat_c = sum_t conj(e^{lam S_t}) c_t dy_t^T
 //   k_chunk_adj_pass   (chunks in reverse)     Gc_{c-1} = conj(e^{lam S_63}) Gc_c + Ghat_c
 //   k_chunk_bwd_dx     (every chunk at once)   dx_s = sum_{t>=s} P_ts dy_t + (Bh_s)^T Gc_c + corr
-//   k_chunk_bwd_gbu    (every chunk at once)   gbu_t = sum_p u_t,p Gbar_t,p
+//   k_chunk_bwd_fused  (every chunk at once)   dC_t and gbu_t = sum_p u_t,p Gbar_t,p, then the
+//                                              decay-gradient sums of the chunk
 // where P is the masked score matrix of the forward and Bh_s = sigma_s b_s
 // e^{lam (S_63 - S_s)} (the same folded operands as the chunked forward).  The
 // passing kernel also forms, at every chunk start, the exact boundary value
@@ -41,11 +42,11 @@ using namespace chunkc;
 // ============================================================================
 // k_chunk_adj_local: Ghat_c = Ch^T (N x 64 t) . dY (64 t x 64 p), per chunk.
 //   Ch_t = c_t conj(e^{lam S_t}) = Ci_t G_i (sub-block-relative fold times the
-//   sub-block's start factor), split into bf16 hi + lo.  Also stores the
-//   chunk's full decay F[0][4] per mode for the passing kernel.
+//   sub-block's start factor), split into bf16 hi + lo.
 // ============================================================================
 namespace loc {
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;
+constexpr int RG = THREADS / 64;   // row groups of the operand preparation
 constexpr uint32_t TMEM_COLS = 64;
 constexpr uint32_t SM_C = 0;        // 16 KB  raw C (two 64-row 128B-swizzled halves)
 constexpr uint32_t SM_DY = 16384;   // 8 KB   dy (128B swizzle)
@@ -100,15 +101,15 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
     int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
     if (!ok) rev_raise_error(1);
     if (__syncthreads_and(ok)) {
-        // Ch tiles: thread (t, grp) handles rows 8 * (grp + 2k)
+        // Ch tiles: thread (t, grp) handles rows 8 * (grp + RG k)
         const int t = tid & 63, grp = tid >> 6;
         const int ib = t >> 4;
         const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
         const float ds = f32[F_S + t] - Sb;
         const unsigned char *sC = sm + loc::SM_C;
 #pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
-            const int r0 = 8 * (grp + 2 * k);
+        for (int k = 0; k < NP / (8 * loc::RG); ++k) {
+            const int r0 = 8 * (grp + loc::RG * k);
             if (r0 >= N) break;
             float rc[8], v[8];
             ld_rows8(sC, t, r0, rc);
@@ -157,12 +158,13 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
         if (!ok) rev_raise_error(1);
         fence_after_sync();
         if (__syncthreads_and(ok)) {
-            const int n = tid;
-            float *dst = p.ws_gc + (bhc(p, b, h, c) * N + n) * PD;
+            // the chunk-local fp32 sum [N][64] at the start of the chunk's slot
+            const int n = 32 * (warp & 3) + (tid & 31), half = warp >> 2;
+            float *dst = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS + n * PD;
 #pragma unroll
-            for (int c16 = 0; c16 < PD / 16; ++c16) {
+            for (int c16 = 2 * half; c16 < 2 * half + 2; ++c16) {
                 float v[16];
-                tmem_ld16(tmem_addr(tacc, 32u * warp, 16u * c16), v);
+                tmem_ld16(tmem_addr(tacc, 32u * (warp & 3), 16u * c16), v);
                 if (n < N) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
@@ -215,9 +217,12 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
     s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
 
     for (int c = nc - 1; c >= 0; --c) {
-        float *gbase = p.ws_gc + bhc(p, b, h, c) * N * PD + q;
-        // K_end_{c-1}: the state entering chunk c
-        const float *kb = (c > 0 && p.ws_qb) ? p.ws_kp + bhc(p, b, h, c) * N * PD + q : nullptr;
+        float *slot = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS;
+        float *gbase = slot + q;
+        // K_end_{c-1}: the state entering chunk c (tile format)
+        const unsigned char *kb = (c > 0 && p.ws_qb)
+            ? reinterpret_cast<const unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
+            : nullptr;
         float4 hv0[pass::KMAX], hv1[pass::KMAX], kv0[pass::KMAX], kv1[pass::KMAX];
 #pragma unroll
         for (int k = 0; k < pass::KMAX; ++k) {
@@ -225,23 +230,25 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
                 const int n0 = 2 * (rp0 + 16 * k);
                 hv0[k] = *reinterpret_cast<const float4 *>(gbase + (long long)n0 * PD);
                 hv1[k] = *reinterpret_cast<const float4 *>(gbase + (long long)(n0 + 1) * PD);
-                if (kb) {
-                    kv0[k] = __ldg(reinterpret_cast<const float4 *>(kb + (long long)n0 * PD));
-                    kv1[k] = __ldg(reinterpret_cast<const float4 *>(kb + (long long)(n0 + 1) * PD));
-                }
+                if (kb) tile_load_rows2(kb, n0, q, kv0[k], kv1[k]);
             }
         }
         if (c > 0) s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
+        // every thread has read its part of Ghat_c: the slot can take the carry into chunk c
         __syncthreads();
         const float *ce = s_ce[c % 3];
         float *qb = p.ws_qb ? p.ws_qb + bhc(p, b, h, c) * 4 * (long long)N : nullptr;
+        unsigned char *tile = reinterpret_cast<unsigned char *>(slot);
 #pragma unroll
         for (int k = 0; k < pass::KMAX; ++k) {
-            if (k >= nk) break;
             const int n0 = 2 * (rp0 + 16 * k);
-            // the carry into chunk c, then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
-            *reinterpret_cast<float4 *>(gbase + (long long)n0 * PD) = g0[k];
-            *reinterpret_cast<float4 *>(gbase + (long long)(n0 + 1) * PD) = g1[k];
+            if (k >= nk) {   // rows past N read as zero by the consumers
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                tile_store_rows2(tile, n0, q, z, z);
+                continue;
+            }
+            // the carry into chunk c (tile format), then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
+            tile_store_rows2(tile, n0, q, g0[k], g1[k]);
             float4 &a = g0[k], &d = g1[k];
             if (n0 < nr) {
                 const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
@@ -371,8 +378,10 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + 2 * Q * N * 2));
+        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + 2 * Q * N * 2) + TILE_BYTES);
         tma_load_4d(sm + dxk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        // the adjoint carried into this chunk (bf16 tile: B operand, N = p, K = rows)
+        bulk_load(sm + dxk::SM_GC, p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS, TILE_BYTES, bar_tma);
         for (int k = 0; k < nbox; ++k) {
             tma_load_4d(sm + dxk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
             tma_load_4d(sm + dxk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
@@ -383,8 +392,6 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
     if (N < NP)  // K padding of Ci, Bi, Bh
         for (int i = tid; i < (int)((dxk::SM_P - dxk::SM_CI) / 16); i += dxk::THREADS)
             reinterpret_cast<uint4 *>(sm + dxk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
-    // the adjoint carried into this chunk as the bf16 B operand (N = p, K = rows)
-    load_state_tile(p.ws_gc + bhc(p, b, h, c) * N * PD, N, sm + dxk::SM_GC, nullptr);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
     fence_before_sync();
@@ -616,7 +623,7 @@ k_chunk_bwd_dx_saved(const __grid_constant__ CUtensorMap tmDY, Params p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int N = p.N, L = p.L;
+    const int L = p.L;
     const int t0 = c * Q;
     const long long u = bhc(p, b, h, c);
 
@@ -625,13 +632,13 @@ k_chunk_bwd_dx_saved(const __grid_constant__ CUtensorMap tmDY, Params p) {
         mbar_init(bar_mma, 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, 8192u + 8192u + 16384u);
+        mbar_expect_tx(bar_tma, 8192u + 8192u + 16384u + TILE_BYTES);
         tma_load_4d(sm + dxs::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        bulk_load(sm + dxs::SM_GC, p.ws_gc + u * SLOT_FLOATS, TILE_BYTES, bar_tma);
         bulk_load(sm + dxs::SM_P, p.sv_P + u * 8192, 8192u, bar_tma);
         bulk_load(sm + dxs::SM_BH, p.sv_Bh + u * 16384, 16384u, bar_tma);
     }
     if (warp == 0) tmem_alloc(tslot, dxs::TMEM_COLS);
-    load_state_tile(p.ws_gc + u * N * PD, N, sm + dxs::SM_GC, nullptr);
     if (tid < Q) corr[tid] = p.sv_corr[u * Q + tid];
     fence_proxy_async();
     fence_before_sync();
@@ -797,9 +804,12 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + 2 * Q * N * 2));
+        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + 2 * Q * N * 2) + 4 * TILE_BYTES);
         tma_load_4d(sm + fuk::SM_X, &tmX, bar_tma, 0, h, t0, b);
         tma_load_4d(sm + fuk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
+        // the state entering the chunk and the adjoint carried into it, hi + lo tiles
+        bulk_load(sm + fuk::SM_KT, p.ws_kp + u * SLOT_FLOATS, 2 * TILE_BYTES, bar_tma);
+        bulk_load(sm + fuk::SM_GC, p.ws_gc + u * SLOT_FLOATS, 2 * TILE_BYTES, bar_tma);
         for (int k = 0; k < nbox; ++k) {
             tma_load_4d(sm + fuk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
             tma_load_4d(sm + fuk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
@@ -810,8 +820,6 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     if (N < NP)  // M padding of the Bo / Cm tiles
         for (int i = tid; i < (int)((fuk::SM_GM - fuk::SM_BO) / 16); i += fuk::THREADS)
             reinterpret_cast<uint4 *>(sm + fuk::SM_BO)[i] = make_uint4(0, 0, 0, 0);
-    load_state_tile(p.ws_kp + u * N * PD, N, sm + fuk::SM_KT, sm + fuk::SM_KTL);
-    load_state_tile(p.ws_gc + u * N * PD, N, sm + fuk::SM_GC, sm + fuk::SM_GCL);
     chunk_tokens(p, f32, b, h, t0, true);
     chunk_mode_constants(p, f32);
     fence_before_sync();
