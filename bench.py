@@ -121,14 +121,14 @@ def kernel_bytes(shape, name: str) -> int:
     return 0
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# dominant kernel from the ncu capture summarised in
-# profiles/chunk_parallel_step_hybridmamba.md, taken at batch 1 and scaled to
-# the 8 batch rows of the workload (the traffic is per 64-token chunk).  An
-# entry is removed whenever its kernel changes after the capture.
-NCU_TRAFFIC = {
-    ("hybridmamba", "k_chunk_bwd_fused"): 8 * (472.464896 + 124.908288) * 1e6,
-    ("hybridmamba", "k_chunk_out"): 8 * (236.2304 + 52.0064) * 1e6,
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per batch row of
+# the workload for the largest kernels, from the ncu capture summarised in
+# profiles/chunk_parallel_step_hybridmamba.md (taken at batch 1; the traffic
+# is per 64-token chunk, so a launch moves batch x this).  An entry is removed
+# whenever its kernel changes after the capture.
+NCU_TRAFFIC_PER_ROW = {
+    ("hybridmamba", "k_chunk_bwd_fused"): (472.464896 + 124.908288) * 1e6,
+    ("hybridmamba", "k_chunk_out"): (236.2304 + 52.0064) * 1e6,
 }
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)
@@ -453,7 +453,8 @@ def main():
                    "l2": "inputs (1.6 GB) larger than L2; no flush", "route": route},
         "fwd_tokens_per_s": fwd_value, "ms_fwd": ms_fwd,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": NCU_TRAFFIC.get((shape.name, dom)), "kernel": dom,
+                     "frac": achieved / hbm, "traffic": (NCU_TRAFFIC_PER_ROW[(shape.name, dom)] * shape.batch
+                                 if (shape.name, dom) in NCU_TRAFFIC_PER_ROW else None), "kernel": dom,
                      "algorithmic_bytes": dom_bytes, "ms_per_launch": avg[dom],
                      "peak_source": peak_note},
         "step_roofline": {"algorithmic_bytes": step_bytes,
