@@ -149,36 +149,43 @@ __device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b,
     chunk_tokens_from(p, f32, t0, r, want_sigma);
 }
 
-// Per-mode decay over each sub-block, E_k = e^{lam dS_k}, and the products
-// F[i][j] = prod_{k=i}^{j-1} E_k and G_i = conj(F[0][i]) into the F_KRE / F_KIM
-// slots.  Needs F_S, F_A2, F_W.  Ends with a barrier.
+// Per-mode decay over each sub-block, E_k = e^{lam dS_k} (one thread per mode
+// and sub-block), then the products F[i][j] = prod_{k=i}^{j-1} E_k and
+// G_i = conj(F[0][i]) (one thread per mode) into the F_KRE / F_KIM slots; E_k
+// itself is F[k][k+1].  Needs F_S, F_A2, F_W.  Contains barriers.
 __device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
     const int nmode = p.nr + p.np;
-    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
+    for (int it = threadIdx.x; it < 4 * nmode; it += blockDim.x) {
+        const int m = it >> 2, k = it & 3;
         const float a2 = f32[F_A2 + m], w = f32[F_W + m];
-        float er[4], ei[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
-            const float ds = f32[F_S + 16 * k + 15] - lo;
-            const float mag = exp2f(a2 * ds);
-            if (m >= p.nr) {
-                float sn, cs;
-                sincosf(w * ds, &sn, &cs);
-                er[k] = mag * cs;
-                ei[k] = mag * sn;
-            } else {
-                er[k] = mag;
-                ei[k] = 0.f;
-            }
+        const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
+        const float ds = f32[F_S + 16 * k + 15] - lo;
+        const float mag = exp2f(a2 * ds);
+        float er = mag, ei = 0.f;
+        if (m >= p.nr) {
+            float sn, cs;
+            sincosf(w * ds, &sn, &cs);
+            er = mag * cs;
+            ei = mag * sn;
         }
+        f32[F_KRE + fslot(k, k + 1) * NP + m] = er;
+        f32[F_KIM + fslot(k, k + 1) * NP + m] = ei;
+    }
+    __syncthreads();
+    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float pr = 1.f, pi = 0.f;
+        for (int i = 0; i < 3; ++i) {
+            float pr = f32[F_KRE + fslot(i, i + 1) * NP + m];
+            float pi = f32[F_KIM + fslot(i, i + 1) * NP + m];
+            if (i == 0) {
+                f32[F_KRE + gslot(1) * NP + m] = pr;
+                f32[F_KIM + gslot(1) * NP + m] = -pi;
+            }
 #pragma unroll
-            for (int j = i + 1; j <= 4; ++j) {
+            for (int j = i + 2; j <= 4; ++j) {
                 float nr_, ni_;
-                cmul(pr, pi, er[j - 1], ei[j - 1], nr_, ni_);
+                cmul(pr, pi, f32[F_KRE + fslot(j - 1, j) * NP + m],
+                     f32[F_KIM + fslot(j - 1, j) * NP + m], nr_, ni_);
                 pr = nr_;
                 pi = ni_;
                 f32[F_KRE + fslot(i, j) * NP + m] = pr;

@@ -569,9 +569,9 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             break;
         }
         // ---- masked scores -> P^T tiles (one warp per TMEM lane quarter) -------
-        if (warp >= 4 && warp < 8) {
-            const int qd = warp - 4;
-            for (int i = 0; i < NSB; ++i) {
+        if (warp >= 4 && warp < 12) {   // two warps per TMEM lane quarter, two blocks each
+            const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);
+            for (int i = i0; i < i0 + 2; ++i) {
                 float v[16];
                 tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
                 const int sl = lane - 16;

@@ -513,9 +513,9 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
         fence_after_sync();
         if (__syncthreads_and(ok)) {
             // ---- masked scores -> P^T (K-major rows s, K = t), zero where s > t
-            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
-                const int qd = warp - 4;
-                for (int i = 0; i < NSB; ++i) {
+            if (warp >= 4 && warp < 12) {   // two warps per TMEM lane quarter, two blocks each
+                const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);
+                for (int i = i0; i < i0 + 2; ++i) {
                     float v[16];
                     tmem_ld16(tmem_addr(t_sc - (16u << 16), 32u * qd, 16u * i), v);
                     const int sl = lane - 16;
@@ -779,57 +779,89 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
                   Params p) {
     if (gated_off(p)) return;
+    const int nitems = p.nc * p.H * p.Bsz;
+    if ((int)blockIdx.x >= nitems) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + fuk::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);
-    uint64_t *bar_mma = bar_tma + 1;   // [2]
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);   // [2]: x/dy/states, B/C
+    uint64_t *bar_mma = bar_in + 2;                                      // [2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / p.hpg;
     const int N = p.N, nr = p.nr, L = p.L;
-    const int t0 = c * Q;
     const int nbox = N / 64;
-    const long long u = bhc(p, b, h, c);
+    // the next chunk's inputs go into regions as soon as this chunk is done with them:
+    // x, dy and the state tiles after phase A, B and C after the unfold's token loop
+    auto issue_xs = [&](int item) {
+        const ChunkItem it = chunk_item(p, item);
+        const int t0_ = it.c * Q;
+        const long long u_ = bhc(p, it.b, it.h, it.c);
+        mbar_expect_tx(&bar_in[0], (uint32_t)(2 * Q * PD * 2) + 4 * TILE_BYTES);
+        tma_load_4d(sm + fuk::SM_X, &tmX, &bar_in[0], 0, it.h, t0_, it.b);
+        tma_load_4d(sm + fuk::SM_DY, &tmDY, &bar_in[0], 0, it.h, t0_, it.b);
+        bulk_load(sm + fuk::SM_KT, p.ws_kp + u_ * SLOT_FLOATS, 2 * TILE_BYTES, &bar_in[0]);
+        bulk_load(sm + fuk::SM_GC, p.ws_gc + u_ * SLOT_FLOATS, 2 * TILE_BYTES, &bar_in[0]);
+    };
+    auto issue_bc = [&](int item) {
+        const ChunkItem it = chunk_item(p, item);
+        const int t0_ = it.c * Q, g_ = it.h / p.hpg;
+        mbar_expect_tx(&bar_in[1], (uint32_t)(2 * Q * N * 2));
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_4d(sm + fuk::SM_B + k * 8192, &tmB, &bar_in[1], 64 * k, g_, t0_, it.b);
+            tma_load_4d(sm + fuk::SM_C + k * 8192, &tmC, &bar_in[1], 64 * k, g_, t0_, it.b);
+        }
+    };
 
+    int item = blockIdx.x;
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(&bar_mma[0], 1);
-        mbar_init(&bar_mma[1], 1);
+        mbar_init(&bar_in[0], 1);
+        mbar_init(&bar_in[1], 1);
+        mbar_init(&bar_mma[0], 2);   // two issuing threads commit each phase
+        mbar_init(&bar_mma[1], 2);
         mbar_fence_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, (uint32_t)(2 * Q * PD * 2 + 2 * Q * N * 2) + 4 * TILE_BYTES);
-        tma_load_4d(sm + fuk::SM_X, &tmX, bar_tma, 0, h, t0, b);
-        tma_load_4d(sm + fuk::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
-        // the state entering the chunk and the adjoint carried into it, hi + lo tiles
-        bulk_load(sm + fuk::SM_KT, p.ws_kp + u * SLOT_FLOATS, 2 * TILE_BYTES, bar_tma);
-        bulk_load(sm + fuk::SM_GC, p.ws_gc + u * SLOT_FLOATS, 2 * TILE_BYTES, bar_tma);
-        for (int k = 0; k < nbox; ++k) {
-            tma_load_4d(sm + fuk::SM_B + k * 8192, &tmB, bar_tma, 64 * k, g, t0, b);
-            tma_load_4d(sm + fuk::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
-        }
+        issue_xs(item);
+        issue_bc(item);
     }
     if (warp == 0) tmem_alloc(tslot, fuk::TMEM_COLS);
-    mode_rates(p, f32, h);
-    if (N < NP)  // M padding of the Bo / Cm tiles
-        for (int i = tid; i < (int)((fuk::SM_GM - fuk::SM_BO) / 16); i += fuk::THREADS)
-            reinterpret_cast<uint4 *>(sm + fuk::SM_BO)[i] = make_uint4(0, 0, 0, 0);
-    chunk_tokens(p, f32, b, h, t0, true);
-    chunk_mode_constants(p, f32);
+    TokPrefetch tok;
+    {
+        const ChunkItem it = chunk_item(p, item);
+        tok = tok_load(p, it.b, it.h, it.c * Q);
+    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_v = tbase, t_v2 = tbase + 64u, t_g = tbase + 128u;
-    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
-    if (!ok) rev_raise_error(1);
-    if (__syncthreads_and(ok)) {
+    bool aborted = false;
+
+    for (int kit = 0; item < nitems; ++kit, item += gridDim.x) {
+        const ChunkItem it = chunk_item(p, item);
+        const int c = it.c, h = it.h, b = it.b;
+        const int g = h / p.hpg;
+        const int t0 = c * Q;
+        const long long u = bhc(p, b, h, c);
+        const int next = item + gridDim.x;
+        const uint32_t par = (uint32_t)(kit & 1);
+        mode_rates(p, f32, h);
+        chunk_tokens_from(p, f32, t0, tok, true);
+        if (next < nitems) {
+            const ChunkItem nx = chunk_item(p, next);
+            tok = tok_load(p, nx.b, nx.h, nx.c * Q);
+        }
+        chunk_mode_constants(p, f32);
+        int ok = (mbar_wait(&bar_in[0], par, WAIT_LIMIT) && mbar_wait(&bar_in[1], par, WAIT_LIMIT)) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
         // ---- Bo (B at its sub-block's start) and Cm (C at its sub-block's end), hi + lo
         {
             const int t = tid & 63, grp = tid >> 6;
@@ -882,26 +914,32 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         __syncthreads();
 
         // ---- phase A: V = K_prev dY^T, V2 = Gc X^T (hi + lo), G = dY X^T ---------
-        if (tid == 0) {
+        // (two threads in different warps issue the independent accumulators)
+        if (tid == 0 || tid == 32) {
             fence_after_sync();
             const uint32_t x_base = smem_u32(sm + fuk::SM_X), dy_base = smem_u32(sm + fuk::SM_DY);
             const uint32_t id_v = idesc_bf16(128, 64, false, false);
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t kt_base = smem_u32(sm + (part ? fuk::SM_KTL : fuk::SM_KT));
-                const uint32_t gc_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
-                for (int s = 0; s < PD / 16; ++s) {
-                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                             part > 0 || s > 0);
-                    mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                             sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                             part > 0 || s > 0);
+            if (tid == 0) {
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t kt_base = smem_u32(sm + (part ? fuk::SM_KTL : fuk::SM_KT));
+                    for (int s = 0; s < PD / 16; ++s)
+                        mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                                 sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                                 part > 0 || s > 0);
+                }
+                const uint32_t id_g = idesc_bf16(64, 64, false, false);
+                for (int s = 0; s < PD / 16; ++s)
+                    mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                             sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
+            } else {
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t gc_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
+                    for (int s = 0; s < PD / 16; ++s)
+                        mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                                 sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                                 part > 0 || s > 0);
                 }
             }
-            const uint32_t id_g = idesc_bf16(64, 64, false, false);
-            for (int s = 0; s < PD / 16; ++s)
-                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
             mma_commit(&bar_mma[0]);
         }
         if (tid < 64) {
@@ -911,306 +949,323 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 cs += reinterpret_cast<const float *>(sm + fuk::SM_GM)[k * 64 + tid];
             f32[F_CORR + tid] = cs;   // C_t . B_t
         }
-        ok = mbar_wait(&bar_mma[0], 0, WAIT_LIMIT) ? 1 : 0;
+        ok = mbar_wait(&bar_mma[0], par, WAIT_LIMIT) ? 1 : 0;
         if (!ok) rev_raise_error(1);
         fence_after_sync();
-        if (__syncthreads_and(ok)) {
-            // ---- masked G (s <= t) -> four 16-row tiles (rows t, K = s); dy_t . u_t
-            if (warp >= 4 && warp < 8) {   // one warp per TMEM lane quarter
-                const int qd = warp - 4;
-                for (int i = 0; i < NSB; ++i) {
-                    float v[16];
-                    tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
-                    if (lane < 16 && i <= qd) {
-                        const int t = 16 * qd + lane;
-                        float lo[8], hi[8];
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // phase A has read x, dy and the state tiles: fetch the next chunk's
+        if (tid == 0 && next < nitems) issue_xs(next);
+        // ---- masked G (s <= t) -> four 16-row tiles (rows t, K = s); dy_t . u_t
+        if (warp >= 4 && warp < 12) {   // two warps per TMEM lane quarter, two blocks each
+            const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);
+            for (int i = i0; i < i0 + 2; ++i) {
+                float v[16];
+                tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
+                if (lane < 16 && i <= qd) {
+                    const int t = 16 * qd + lane;
+                    float lo[8], hi[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
-                            hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
-                        }
-                        unsigned char *gt = sm + fuk::SM_GM + qd * 2048;
-                        unsigned char *gl = sm + fuk::SM_GML + qd * 2048;
-                        st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
-                        st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
-                        if (i == qd) {
-                            float dg = 0.f;
+                    for (int j = 0; j < 8; ++j) {
+                        lo[j] = (16 * i + j <= t) ? v[j] : 0.f;
+                        hi[j] = (16 * i + 8 + j <= t) ? v[8 + j] : 0.f;
+                    }
+                    unsigned char *gt = sm + fuk::SM_GM + qd * 2048;
+                    unsigned char *gl = sm + fuk::SM_GML + qd * 2048;
+                    st16_split(gt, gl, off_kmaj(lane, 16 * i, 128u, 1024u), lo);
+                    st16_split(gt, gl, off_kmaj(lane, 16 * i + 8, 128u, 1024u), hi);
+                    if (i == qd) {
+                        float dg = 0.f;
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (j == lane) dg = v[j];
-                            f32[F_LAM + t] = dg;   // <dy_t, u_t> (lambda is no longer needed)
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            if (j == lane) dg = v[j];
+                        f32[F_LAM + t] = dg;   // <dy_t, u_t> (lambda is no longer needed)
                     }
-                }
-            }
-            fence_proxy_async();
-            fence_before_sync();
-            __syncthreads();
-
-            // ---- phase B: D_{i,k} and E_{j,k}, hi*hi + hi*lo + lo*hi ---------------
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t id_d = idesc_bf16(128, 16, true, false);
-                const uint32_t id_e = idesc_bf16(128, 16, true, true);
-                const uint32_t bo_off[3] = {fuk::SM_BO, fuk::SM_BO, fuk::SM_BOL};
-                const uint32_t cm_off3[3] = {fuk::SM_CM, fuk::SM_CM, fuk::SM_CML};
-                const uint32_t g_off[3] = {fuk::SM_GM, fuk::SM_GML, fuk::SM_GM};
-                for (int i = 0; i < NSB; ++i)
-                    for (int k = 0; k <= i; ++k)
-                        for (int part = 0; part < 3; ++part)
-                            mma_bf16(tbase + d_col(i, k),
-                                     sdesc(smem_u32(sm + bo_off[part]) + k * 4096u, 2048u, 128u,
-                                           LAYOUT_NONE),
-                                     sdesc(smem_u32(sm + g_off[part]) + i * 2048u + k * 256u, 128u,
-                                           1024u, LAYOUT_NONE),
-                                     id_d, part > 0);
-                for (int j = 0; j < NSB; ++j)
-                    for (int k = j; k < NSB; ++k)
-                        for (int part = 0; part < 3; ++part)
-                            mma_bf16(tbase + e_col(j, k),
-                                     sdesc(smem_u32(sm + cm_off3[part]) + k * 4096u, 2048u, 128u,
-                                           LAYOUT_NONE),
-                                     sdesc(smem_u32(sm + g_off[part]) + k * 2048u + j * 256u, 1024u,
-                                           128u, LAYOUT_NONE),
-                                     id_e, part > 0);
-                mma_commit(&bar_mma[1]);
-            }
-            ok = mbar_wait(&bar_mma[1], 0, WAIT_LIMIT) ? 1 : 0;
-            if (!ok) rev_raise_error(1);
-            fence_after_sync();
-            if (__syncthreads_and(ok)) {
-                // ---- unfold: thread (row n, sub-block i) -----------------------------
-                float *red = reinterpret_cast<float *>(sm + fuk::SM_RED);    // [128][RED_LD] B . gbu
-                float *red2 = reinterpret_cast<float *>(sm + fuk::SM_RED2);  // [128][RED_LD] ddt terms
-                float *xch = reinterpret_cast<float *>(sm + fuk::SM_XCH);    // group totals, partials
-                const int n = tid & 127, i = tid >> 7, qd = warp & 3;
-                const bool valid = n < N;
-                const int m = n < nr ? n : nr + ((n - nr) >> 1);
-                const bool pr_row = valid && n >= nr;
-                const bool im_row = pr_row && ((n - nr) & 1);
-                const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
-                const int tc = 16 * i;
-
-                // part 1: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} sum_k F[k][i] D_{i,k}
-                float kk[16];
-                {
-                    float vv[16], dd[16];
-                    tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
-                    tmem_ld16(tmem_addr(tbase + d_col(i, i), 32u * qd, 0u), dd);
-                    for (int k = 0; k < i; ++k) {
-                        float ek[16];
-                        tmem_ld16(tmem_addr(tbase + d_col(i, k), 32u * qd, 0u), ek);
-                        const float fr = valid ? f32[F_KRE + fslot(k, i) * NP + m] : 0.f;
-                        const float fi = valid ? f32[F_KIM + fslot(k, i) * NP + m] : 0.f;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
-                            // own component of (fr + i fi)(re + i im)
-                            dd[j] = pr_row ? fmaf(fr, ek[j], fmaf(im_row ? fi : -fi, other, dd[j]))
-                                           : fmaf(fr, ek[j], dd[j]);
-                        }
-                    }
-                    const float Sb = i == 0 ? 0.f : f32[F_S + 16 * i - 1];
-                    float fr = 1.f, fi = 0.f;   // F[0][i] = e^{lam Sb_i}
-                    if (i && valid) {
-                        fr = f32[F_KRE + gslot(i) * NP + m];
-                        fi = -f32[F_KIM + gslot(i) * NP + m];
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float ds = f32[F_S + tc + j] - Sb;
-                        const float mag = ex2_fast(a2 * ds);
-                        float er = mag, ei = 0.f;
-                        if (pr_row) {
-                            float sn, cs;
-                            __sincosf(w * ds, &sn, &cs);
-                            er = mag * cs;
-                            ei = mag * sn;
-                        }
-                        float Er, Ei;
-                        cmul(er, ei, fr, fi, Er, Ei);
-                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
-                        const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
-                        if (!pr_row)
-                            kk[j] = fmaf(Er, vv[j], er * dd[j]);
-                        else if (!im_row)
-                            kk[j] = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
-                        else
-                            kk[j] = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
-                    }
-                }
-
-                // part 2: gbu, the decay-gradient suffix sums, dB / dC, walking backwards
-                const float coef = !valid ? 0.f : (im_row ? -w : a2 * 0.6931471805599453f);
-                const bool one_head = p.hpg == 1;
-                const long long tstride = (long long)p.H * p.N;
-                float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
-                float *cdst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
-                const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
-                float cum = 0.f, dacc = 0.f, sdt = 0.f;
-                {
-                    float vv[16], ee[16];
-                    tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)tc), vv);
-                    tmem_ld16(tmem_addr(tbase + e_col(i, i), 32u * qd, 0u), ee);
-                    for (int k = i + 1; k < NSB; ++k) {
-                        float ek[16];
-                        tmem_ld16(tmem_addr(tbase + e_col(i, k), 32u * qd, 0u), ek);
-                        const float f2r = valid ? f32[F_KRE + fslot(i + 1, k + 1) * NP + m] : 0.f;
-                        const float f2i = valid ? f32[F_KIM + fslot(i + 1, k + 1) * NP + m] : 0.f;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
-                            // own component of (f2r - i f2i)(re + i im)
-                            ee[j] = pr_row ? fmaf(f2r, ek[j], fmaf(im_row ? -f2i : f2i, other, ee[j]))
-                                           : fmaf(f2r, ek[j], ee[j]);
-                        }
-                    }
-                    const float se = f32[F_S + tc + 15];
-                    float fr = 1.f, fi = 0.f;   // F[i+1][4]
-                    if (i < 3 && valid) {
-                        fr = f32[F_KRE + fslot(i + 1, 4) * NP + m];
-                        fi = f32[F_KIM + fslot(i + 1, 4) * NP + m];
-                    }
-#pragma unroll
-                    for (int j = 15; j >= 0; --j) {
-                        const int t = tc + j;
-                        const float ds = se - f32[F_S + t];   // >= 0
-                        const float mag = ex2_fast(a2 * ds);
-                        float er = mag, ei = 0.f;
-                        if (pr_row) {
-                            float sn, cs;
-                            __sincosf(w * ds, &sn, &cs);
-                            er = mag * cs;
-                            ei = mag * sn;
-                        }
-                        const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
-                        const float eo = __shfl_xor_sync(0xffffffffu, ee[j], 1);
-                        float res;
-                        if (!pr_row) {
-                            res = er * fmaf(fr, vv[j], ee[j]);
-                        } else {
-                            // own row is re (im_row false) or im; W = conj(F) V2 + E
-                            const float vr = im_row ? vo : vv[j], vi = im_row ? vv[j] : vo;
-                            const float e_r = im_row ? eo : ee[j], e_i = im_row ? ee[j] : eo;
-                            const float wr = fmaf(fr, vr, fmaf(fi, vi, e_r));
-                            const float wi = fmaf(fr, vi, fmaf(-fi, vr, e_i));
-                            // conj(er + i ei) (wr + i wi)
-                            res = im_row ? fmaf(er, wi, -ei * wr) : fmaf(er, wr, ei * wi);
-                        }
-                        const bool tv = valid && t0 + t < L;
-                        const float m2 = f32[F_LAM + t], bn = f32[F_BN + t];
-                        const float sig = f32[F_SIG + t], dtv = f32[F_DT + t];
-                        const float bt = ld_row1(sB, t, n), ct = ld_row1(sC, t, n);
-                        const float k_ = kk[j];                          // dCK_t
-                        const float dCt = fmaf(-bn * m2, bt, k_);        // dC_t
-                        const float gg = sig * res;
-                        const float co = __shfl_xor_sync(0xffffffffu, ct, 1);
-                        const float ko = __shfl_xor_sync(0xffffffffu, k_, 1);
-                        const float bo = __shfl_xor_sync(0xffffffffu, bt, 1);
-                        const float go = __shfl_xor_sync(0xffffffffu, gg, 1);
-                        float v;
-                        if (!pr_row)
-                            v = fmaf(ct, k_, -bt * gg);
-                        else if (!im_row)   // Re(conj(c) k) - Re(b conj(g))
-                            v = fmaf(ct, k_, fmaf(co, ko, -fmaf(bt, gg, bo * go)));
-                        else                // Im(conj(c) k) - Im(b conj(g)), own row = im
-                            v = fmaf(co, k_, fmaf(-ct, ko, -fmaf(bt, go, -bo * gg)));
-                        if (!tv) v = 0.f;
-                        cum += v;
-                        dacc = fmaf(dtv, im_row ? -cum : cum, dacc);
-                        sdt += dtv;
-                        red2[n * fuk::RED_LD + t] = coef * cum;
-                        red[n * fuk::RED_LD + t] = tv ? res * bt : 0.f;
-                        if (tv) {
-                            if (one_head) {
-                                const int tg = t0 + t;
-                                reinterpret_cast<__nv_bfloat16 *>(p.dBm)[ix_B(p, b, tg, g, 0, n)] =
-                                    __float2bfloat16_rn(fmaf(-bn * ct, m2, gg));
-                                reinterpret_cast<__nv_bfloat16 *>(p.dCm)[ix_C(p, b, tg, g, 0, n)] =
-                                    __float2bfloat16_rn(dCt);
-                            } else {
-                                gdst[(long long)t * tstride] = res;
-                                cdst[(long long)t * tstride] = dCt;
-                            }
-                        }
-                    }
-                }
-                // later sub-blocks carry into every token of earlier ones
-                xch[i * 128 + n] = cum;
-                __syncthreads();
-                float later = 0.f;
-                for (int k = i + 1; k < fuk::TQ; ++k) later += xch[k * 128 + n];
-                if (later != 0.f) {
-                    const float add = coef * later;
-                    for (int t = tc; t < tc + 16; ++t) red2[n * fuk::RED_LD + t] += add;
-                }
-                dacc += (im_row ? -later : later) * sdt;
-                xch[(fuk::TQ + i) * 128 + n] = dacc;
-                __syncthreads();
-                if (i == 0 && valid) {
-                    float tot = 0.f, da = 0.f;
-                    for (int k = 0; k < fuk::TQ; ++k) {
-                        tot += xch[k * 128 + n];
-                        da += xch[(fuk::TQ + k) * 128 + n];
-                    }
-                    const int nmode = p.nr + p.np;
-                    float *blk = p.ws_blk + u * (4 * nmode + 2);
-                    if (!pr_row) {
-                        blk[4 * m + 0] = tot;
-                        blk[4 * m + 1] = 0.f;
-                        blk[4 * m + 2] = da;
-                        blk[4 * m + 3] = 0.f;
-                    } else if (!im_row) {
-                        blk[4 * m + 0] = tot;
-                        blk[4 * m + 2] = da;
-                    } else {
-                        blk[4 * m + 1] = tot;
-                        blk[4 * m + 3] = da;
-                    }
-                }
-                // column sums over the state rows: all threads, 128 / RG rows each, fixed order
-                float *part = xch + 2 * fuk::TQ * 128;   // [2][RG][64]
-                {
-                    const int t = tid & 63, rg = tid >> 6;
-                    constexpr int RPG = NP / fuk::RG;
-                    float s1 = 0.f, s2 = 0.f;
-                    for (int k = rg * RPG; k < rg * RPG + RPG && k < N; ++k) {
-                        s1 += red[k * fuk::RED_LD + t];
-                        s2 += red2[k * fuk::RED_LD + t];
-                    }
-                    part[rg * 64 + t] = s1;
-                    part[(fuk::RG + rg) * 64 + t] = s2;
-                }
-                __syncthreads();
-                if (tid < 64 && t0 + tid < L) {
-                    const int t = tid;
-                    float dsig = 0.f, dd = 0.f;
-                    for (int k = 0; k < fuk::RG; ++k) {
-                        dsig += part[k * 64 + t];
-                        dd += part[(fuk::RG + k) * 64 + t];
-                    }
-                    const long long ii = ix_bth(p, b, t0 + t, h);
-                    const float m2 = f32[F_LAM + t];
-                    p.ws_tok[2 * ii] = dsig;
-                    p.ws_tok[2 * ii + 1] = f32[F_CORR + t] * m2;
-                    p.ws_M2[ii] = m2;
-                    p.ws_ddt[ii] = dd;
-                }
-                if (tid == 64) {
-                    const int nmode = p.nr + p.np;
-                    float *blk = p.ws_blk + u * (4 * nmode + 2);
-                    float st_ = 0.f, dD = 0.f;
-                    for (int t = 0; t < Q; ++t) {
-                        st_ += f32[F_DT + t];
-                        if (t0 + t < L) dD += f32[F_LAM + t];
-                    }
-                    blk[4 * nmode + 0] = st_;
-                    blk[4 * nmode + 1] = (p.O == p.R) ? dD : 0.f;
                 }
             }
         }
-    } else if (tid == 0) {
-        mbar_wait(bar_tma, 0, WAIT_LIMIT);
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+
+        // ---- phase B: D_{i,k} and E_{j,k}, hi*hi + hi*lo + lo*hi ---------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id_d = idesc_bf16(128, 16, true, false);
+            const uint32_t bo_off[3] = {fuk::SM_BO, fuk::SM_BO, fuk::SM_BOL};
+            const uint32_t g_off[3] = {fuk::SM_GM, fuk::SM_GML, fuk::SM_GM};
+            for (int i = 0; i < NSB; ++i)
+                for (int k = 0; k <= i; ++k)
+                    for (int part = 0; part < 3; ++part)
+                        mma_bf16(tbase + d_col(i, k),
+                                 sdesc(smem_u32(sm + bo_off[part]) + k * 4096u, 2048u, 128u,
+                                       LAYOUT_NONE),
+                                 sdesc(smem_u32(sm + g_off[part]) + i * 2048u + k * 256u, 128u,
+                                       1024u, LAYOUT_NONE),
+                                 id_d, part > 0);
+            mma_commit(&bar_mma[1]);
+        } else if (tid == 32) {
+            fence_after_sync();
+            const uint32_t id_e = idesc_bf16(128, 16, true, true);
+            const uint32_t cm_off3[3] = {fuk::SM_CM, fuk::SM_CM, fuk::SM_CML};
+            const uint32_t g_off[3] = {fuk::SM_GM, fuk::SM_GML, fuk::SM_GM};
+            for (int j = 0; j < NSB; ++j)
+                for (int k = j; k < NSB; ++k)
+                    for (int part = 0; part < 3; ++part)
+                        mma_bf16(tbase + e_col(j, k),
+                                 sdesc(smem_u32(sm + cm_off3[part]) + k * 4096u, 2048u, 128u,
+                                       LAYOUT_NONE),
+                                 sdesc(smem_u32(sm + g_off[part]) + k * 2048u + j * 256u, 1024u,
+                                       128u, LAYOUT_NONE),
+                                 id_e, part > 0);
+            mma_commit(&bar_mma[1]);
+        }
+        ok = mbar_wait(&bar_mma[1], par, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // ---- unfold: thread (row n, sub-block i) -----------------------------
+        float *red = reinterpret_cast<float *>(sm + fuk::SM_RED);    // [128][RED_LD] B . gbu
+        float *red2 = reinterpret_cast<float *>(sm + fuk::SM_RED2);  // [128][RED_LD] ddt terms
+        float *xch = reinterpret_cast<float *>(sm + fuk::SM_XCH);    // group totals, partials
+        const int n = tid & 127, i = tid >> 7, qd = warp & 3;
+        const bool valid = n < N;
+        const int m = n < nr ? n : nr + ((n - nr) >> 1);
+        const bool pr_row = valid && n >= nr;
+        const bool im_row = pr_row && ((n - nr) & 1);
+        const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
+        const int tc = 16 * i;
+
+        // part 1: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} sum_k F[k][i] D_{i,k}
+        float kk[16];
+        {
+            float vv[16], dd[16];
+            tmem_ld16(tmem_addr(t_v, 32u * qd, (uint32_t)tc), vv);
+            tmem_ld16(tmem_addr(tbase + d_col(i, i), 32u * qd, 0u), dd);
+            for (int k = 0; k < i; ++k) {
+                float ek[16];
+                tmem_ld16(tmem_addr(tbase + d_col(i, k), 32u * qd, 0u), ek);
+                const float fr = valid ? f32[F_KRE + fslot(k, i) * NP + m] : 0.f;
+                const float fi = valid ? f32[F_KIM + fslot(k, i) * NP + m] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
+                    // own component of (fr + i fi)(re + i im)
+                    dd[j] = pr_row ? fmaf(fr, ek[j], fmaf(im_row ? fi : -fi, other, dd[j]))
+                                   : fmaf(fr, ek[j], dd[j]);
+                }
+            }
+            const float Sb = i == 0 ? 0.f : f32[F_S + 16 * i - 1];
+            float fr = 1.f, fi = 0.f;   // F[0][i] = e^{lam Sb_i}
+            if (i && valid) {
+                fr = f32[F_KRE + gslot(i) * NP + m];
+                fi = -f32[F_KIM + gslot(i) * NP + m];
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float ds = f32[F_S + tc + j] - Sb;
+                const float mag = ex2_fast(a2 * ds);
+                float er = mag, ei = 0.f;
+                if (pr_row) {
+                    float sn, cs;
+                    __sincosf(w * ds, &sn, &cs);
+                    er = mag * cs;
+                    ei = mag * sn;
+                }
+                float Er, Ei;
+                cmul(er, ei, fr, fi, Er, Ei);
+                const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                const float dO = __shfl_xor_sync(0xffffffffu, dd[j], 1);
+                if (!pr_row)
+                    kk[j] = fmaf(Er, vv[j], er * dd[j]);
+                else if (!im_row)
+                    kk[j] = Er * vv[j] - Ei * vo + er * dd[j] - ei * dO;
+                else
+                    kk[j] = Ei * vo + Er * vv[j] + ei * dO + er * dd[j];
+            }
+        }
+
+        // part 2: gbu, the decay-gradient suffix sums, dB / dC, walking backwards
+        const float coef = !valid ? 0.f : (im_row ? -w : a2 * 0.6931471805599453f);
+        const bool one_head = p.hpg == 1;
+        const long long tstride = (long long)p.H * p.N;
+        float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+        float *cdst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
+        const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
+        float cum = 0.f, dacc = 0.f, sdt = 0.f;
+        {
+            float vv[16], ee[16];
+            tmem_ld16(tmem_addr(t_v2, 32u * qd, (uint32_t)tc), vv);
+            tmem_ld16(tmem_addr(tbase + e_col(i, i), 32u * qd, 0u), ee);
+            for (int k = i + 1; k < NSB; ++k) {
+                float ek[16];
+                tmem_ld16(tmem_addr(tbase + e_col(i, k), 32u * qd, 0u), ek);
+                const float f2r = valid ? f32[F_KRE + fslot(i + 1, k + 1) * NP + m] : 0.f;
+                const float f2i = valid ? f32[F_KIM + fslot(i + 1, k + 1) * NP + m] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float other = __shfl_xor_sync(0xffffffffu, ek[j], 1);
+                    // own component of (f2r - i f2i)(re + i im)
+                    ee[j] = pr_row ? fmaf(f2r, ek[j], fmaf(im_row ? -f2i : f2i, other, ee[j]))
+                                   : fmaf(f2r, ek[j], ee[j]);
+                }
+            }
+            const float se = f32[F_S + tc + 15];
+            float fr = 1.f, fi = 0.f;   // F[i+1][4]
+            if (i < 3 && valid) {
+                fr = f32[F_KRE + fslot(i + 1, 4) * NP + m];
+                fi = f32[F_KIM + fslot(i + 1, 4) * NP + m];
+            }
+#pragma unroll
+            for (int j = 15; j >= 0; --j) {
+                const int t = tc + j;
+                const float ds = se - f32[F_S + t];   // >= 0
+                const float mag = ex2_fast(a2 * ds);
+                float er = mag, ei = 0.f;
+                if (pr_row) {
+                    float sn, cs;
+                    __sincosf(w * ds, &sn, &cs);
+                    er = mag * cs;
+                    ei = mag * sn;
+                }
+                const float vo = __shfl_xor_sync(0xffffffffu, vv[j], 1);
+                const float eo = __shfl_xor_sync(0xffffffffu, ee[j], 1);
+                float res;
+                if (!pr_row) {
+                    res = er * fmaf(fr, vv[j], ee[j]);
+                } else {
+                    // own row is re (im_row false) or im; W = conj(F) V2 + E
+                    const float vr = im_row ? vo : vv[j], vi = im_row ? vv[j] : vo;
+                    const float e_r = im_row ? eo : ee[j], e_i = im_row ? ee[j] : eo;
+                    const float wr = fmaf(fr, vr, fmaf(fi, vi, e_r));
+                    const float wi = fmaf(fr, vi, fmaf(-fi, vr, e_i));
+                    // conj(er + i ei) (wr + i wi)
+                    res = im_row ? fmaf(er, wi, -ei * wr) : fmaf(er, wr, ei * wi);
+                }
+                const bool tv = valid && t0 + t < L;
+                const float m2 = f32[F_LAM + t], bn = f32[F_BN + t];
+                const float sig = f32[F_SIG + t], dtv = f32[F_DT + t];
+                const float bt = ld_row1(sB, t, n), ct = ld_row1(sC, t, n);
+                const float k_ = kk[j];                          // dCK_t
+                const float dCt = fmaf(-bn * m2, bt, k_);        // dC_t
+                const float gg = sig * res;
+                const float co = __shfl_xor_sync(0xffffffffu, ct, 1);
+                const float ko = __shfl_xor_sync(0xffffffffu, k_, 1);
+                const float bo = __shfl_xor_sync(0xffffffffu, bt, 1);
+                const float go = __shfl_xor_sync(0xffffffffu, gg, 1);
+                float v;
+                if (!pr_row)
+                    v = fmaf(ct, k_, -bt * gg);
+                else if (!im_row)   // Re(conj(c) k) - Re(b conj(g))
+                    v = fmaf(ct, k_, fmaf(co, ko, -fmaf(bt, gg, bo * go)));
+                else                // Im(conj(c) k) - Im(b conj(g)), own row = im
+                    v = fmaf(co, k_, fmaf(-ct, ko, -fmaf(bt, go, -bo * gg)));
+                if (!tv) v = 0.f;
+                cum += v;
+                dacc = fmaf(dtv, im_row ? -cum : cum, dacc);
+                sdt += dtv;
+                red2[n * fuk::RED_LD + t] = coef * cum;
+                red[n * fuk::RED_LD + t] = tv ? res * bt : 0.f;
+                if (tv) {
+                    if (one_head) {
+                        const int tg = t0 + t;
+                        reinterpret_cast<__nv_bfloat16 *>(p.dBm)[ix_B(p, b, tg, g, 0, n)] =
+                            __float2bfloat16_rn(fmaf(-bn * ct, m2, gg));
+                        reinterpret_cast<__nv_bfloat16 *>(p.dCm)[ix_C(p, b, tg, g, 0, n)] =
+                            __float2bfloat16_rn(dCt);
+                    } else {
+                        gdst[(long long)t * tstride] = res;
+                        cdst[(long long)t * tstride] = dCt;
+                    }
+                }
+            }
+        }
+        // later sub-blocks carry into every token of earlier ones
+        xch[i * 128 + n] = cum;
+        __syncthreads();
+        // every token loop is done with the raw B / C tiles: fetch the next chunk's
+        if (tid == 0 && next < nitems) issue_bc(next);
+        float later = 0.f;
+        for (int k = i + 1; k < fuk::TQ; ++k) later += xch[k * 128 + n];
+        if (later != 0.f) {
+            const float add = coef * later;
+            for (int t = tc; t < tc + 16; ++t) red2[n * fuk::RED_LD + t] += add;
+        }
+        dacc += (im_row ? -later : later) * sdt;
+        xch[(fuk::TQ + i) * 128 + n] = dacc;
+        __syncthreads();
+        if (i == 0 && valid) {
+            float tot = 0.f, da = 0.f;
+            for (int k = 0; k < fuk::TQ; ++k) {
+                tot += xch[k * 128 + n];
+                da += xch[(fuk::TQ + k) * 128 + n];
+            }
+            const int nmode = p.nr + p.np;
+            float *blk = p.ws_blk + u * (4 * nmode + 2);
+            if (!pr_row) {
+                blk[4 * m + 0] = tot;
+                blk[4 * m + 1] = 0.f;
+                blk[4 * m + 2] = da;
+                blk[4 * m + 3] = 0.f;
+            } else if (!im_row) {
+                blk[4 * m + 0] = tot;
+                blk[4 * m + 2] = da;
+            } else {
+                blk[4 * m + 1] = tot;
+                blk[4 * m + 3] = da;
+            }
+        }
+        // column sums over the state rows: all threads, 128 / RG rows each, fixed order
+        float *part = xch + 2 * fuk::TQ * 128;   // [2][RG][64]
+        {
+            const int t = tid & 63, rg = tid >> 6;
+            constexpr int RPG = NP / fuk::RG;
+            float s1 = 0.f, s2 = 0.f;
+            for (int k = rg * RPG; k < rg * RPG + RPG && k < N; ++k) {
+                s1 += red[k * fuk::RED_LD + t];
+                s2 += red2[k * fuk::RED_LD + t];
+            }
+            part[rg * 64 + t] = s1;
+            part[(fuk::RG + rg) * 64 + t] = s2;
+        }
+        __syncthreads();
+        if (tid < 64 && t0 + tid < L) {
+            const int t = tid;
+            float dsig = 0.f, dd = 0.f;
+            for (int k = 0; k < fuk::RG; ++k) {
+                dsig += part[k * 64 + t];
+                dd += part[(fuk::RG + k) * 64 + t];
+            }
+            const long long ii = ix_bth(p, b, t0 + t, h);
+            const float m2 = f32[F_LAM + t];
+            p.ws_tok[2 * ii] = dsig;
+            p.ws_tok[2 * ii + 1] = f32[F_CORR + t] * m2;
+            p.ws_M2[ii] = m2;
+            p.ws_ddt[ii] = dd;
+        }
+        if (tid == 64) {
+            const int nmode = p.nr + p.np;
+            float *blk = p.ws_blk + u * (4 * nmode + 2);
+            float st_ = 0.f, dD = 0.f;
+            for (int t = 0; t < Q; ++t) {
+                st_ += f32[F_DT + t];
+                if (t0 + t < L) dD += f32[F_LAM + t];
+            }
+            blk[4 * nmode + 0] = st_;
+            blk[4 * nmode + 1] = (p.O == p.R) ? dD : 0.f;
+        }
+        fence_before_sync();
+        __syncthreads();
+    }
+    if (aborted && tid == 0) {
+        // let loads still in flight land before the CTA's shared memory goes away
+        mbar_wait(&bar_in[0], 0, WAIT_LIMIT);
+        mbar_wait(&bar_in[1], 0, WAIT_LIMIT);
     }
     fence_before_sync();
     __syncthreads();
@@ -1234,6 +1289,7 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
 }
 
 cudaError_t chunk_states(const Params &p, cudaStream_t st);
+int sm_count();
 
 // The state entering every chunk for the tensor-core backward (p.ws_kp,
 // p.ws_ce), unless the forward's are given (p.states_ready).
@@ -1275,7 +1331,11 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         profile_mark(st, "k_chunk_bwd_dx");
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_chunk_bwd_fused<<<grid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
+    {
+        const long long nitems = (long long)p.nc * p.H * p.Bsz;
+        const int pgrid = (int)(nitems < sm_count() ? nitems : sm_count());
+        k_chunk_bwd_fused<<<pgrid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
+    }
     profile_mark(st, "k_chunk_bwd_fused");
     return cudaGetLastError();
 }
