@@ -128,7 +128,6 @@ def kernel_bytes(shape, name: str) -> int:
 # whenever its kernel changes after the capture.
 NCU_TRAFFIC_PER_ROW = {
     ("hybridmamba", "k_chunk_bwd_fused"): (472.179456 + 121.520896) * 1e6,
-    ("hybridmamba", "k_chunk_out"): (236.2304 + 52.0064) * 1e6,
 }
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)

@@ -228,42 +228,57 @@ __device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {
 constexpr int SLOT_FLOATS = NP * PD;            // floats per chunk slot
 constexpr uint32_t TILE_BYTES = NP * PD * 2;    // one bf16 tile
 
-// rows n0, n0 + 1 at p .. p + 3 (p a multiple of 4) -> hi / lo tiles
-__device__ __forceinline__ void tile_store_rows2(unsigned char *slot, int n0, int p,
-                                                 const float4 &a, const float4 &d) {
-    const uint32_t off = off_kmaj(n0, p, 128u, 1024u);   // row n0 + 1 is 16 bytes further
-    const float v[2][4] = {{a.x, a.y, a.z, a.w}, {d.x, d.y, d.z, d.w}};
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        float h[4], l[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            h[j] = __bfloat162float(__float2bfloat16_rn(v[r][j]));
-            l[j] = v[r][j] - h[j];
-        }
-        *reinterpret_cast<uint2 *>(slot + off + 16 * r) =
-            make_uint2(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]));
-        *reinterpret_cast<uint2 *>(slot + TILE_BYTES + off + 16 * r) =
-            make_uint2(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
-    }
-}
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
-// hi + lo of rows n0, n0 + 1 at p .. p + 3
-__device__ __forceinline__ void tile_load_rows2(const unsigned char *slot, int n0, int p, float4 &a,
-                                                float4 &d) {
-    const uint32_t off = off_kmaj(n0, p, 128u, 1024u);
-    float4 o[2];
+
+// 8 consecutive p of two state rows n0, n0 + 1 (n0 even): the unit of the
+// elementwise passes, moved in 16-byte pieces.
+struct Rows2x8 {
+    float a[8], d[8];
+};
+__device__ __forceinline__ void rows_load_f32(const float *slot, int n0, int p8, Rows2x8 &r) {
+    const float4 *s0 = reinterpret_cast<const float4 *>(slot + (long long)n0 * PD + p8);
+    const float4 *s1 = reinterpret_cast<const float4 *>(slot + (long long)(n0 + 1) * PD + p8);
+    const float4 a0 = s0[0], a1 = s0[1], d0 = s1[0], d1 = s1[1];
+    r.a[0] = a0.x; r.a[1] = a0.y; r.a[2] = a0.z; r.a[3] = a0.w;
+    r.a[4] = a1.x; r.a[5] = a1.y; r.a[6] = a1.z; r.a[7] = a1.w;
+    r.d[0] = d0.x; r.d[1] = d0.y; r.d[2] = d0.z; r.d[3] = d0.w;
+    r.d[4] = d1.x; r.d[5] = d1.y; r.d[6] = d1.z; r.d[7] = d1.w;
+}
+// -> hi / lo operand tiles of a chunk slot (row n0 + 1 lies 16 bytes after row n0)
+__device__ __forceinline__ void rows_store_tile(unsigned char *slot, int n0, int p8,
+                                                const Rows2x8 &r) {
+    const uint32_t off = off_kmaj(n0, p8, 128u, 1024u);
+    const float *v[2] = {r.a, r.d};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const uint2 h = __ldg(reinterpret_cast<const uint2 *>(slot + off + 16 * r));
-        const uint2 l = __ldg(reinterpret_cast<const uint2 *>(slot + TILE_BYTES + off + 16 * r));
-        const float2 h0 = bf2_to_f2(h.x), h1 = bf2_to_f2(h.y), l0 = bf2_to_f2(l.x), l1 = bf2_to_f2(l.y);
-        o[r] = make_float4(h0.x + l0.x, h0.y + l0.y, h1.x + l1.x, h1.y + l1.y);
+    for (int q = 0; q < 2; ++q) {
+        float hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            hi[j] = __bfloat162float(__float2bfloat16_rn(v[q][j]));
+            lo[j] = v[q][j] - hi[j];
+        }
+        st16(slot, off + 16 * q, hi);
+        st16(slot + TILE_BYTES, off + 16 * q, lo);
     }
-    a = o[0];
-    d = o[1];
+}
+__device__ __forceinline__ void rows_load_tile(const unsigned char *slot, int n0, int p8,
+                                               Rows2x8 &r) {
+    const uint32_t off = off_kmaj(n0, p8, 128u, 1024u);
+    float *v[2] = {r.a, r.d};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 h = __ldg(reinterpret_cast<const uint4 *>(slot + off + 16 * q));
+        const uint4 l = __ldg(reinterpret_cast<const uint4 *>(slot + TILE_BYTES + off + 16 * q));
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 hh = bf2_to_f2(hw[j]), ll = bf2_to_f2(lw[j]);
+            v[q][2 * j] = hh.x + ll.x;
+            v[q][2 * j + 1] = hh.y + ll.y;
+        }
+    }
 }
 
 // Work item of the persistent chunk kernels: chunk fastest, then head, then batch row.

@@ -213,9 +213,16 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 // are in flight to stream at HBM speed.  ws_kp[c] holds S_c on entry and the
 // state entering chunk c on exit; the state after the last chunk is hT.
 // ============================================================================
+// k_chunk_state_pass: the carried state over the chunks of one (batch row,
+// head).  Thread (row-pair group, 8 consecutive p) keeps rows 2rp, 2rp+1 for
+// rp = rp0, rp0 + 32: two real modes or one rotation pair as (re, im).  Every
+// chunk's loads are issued together, in 16-byte pieces.  ws_kp[c] holds S_c
+// (fp32) on entry and the state entering chunk c (hi / lo tiles) on exit; the
+// state after the last chunk is hT.
+// ============================================================================
 namespace pas {
 constexpr int THREADS = 256;
-constexpr int KMAX = NP / 32;   // row pairs per thread
+constexpr int KMAX = NP / 64;   // row pairs per thread
 }  // namespace pas
 
 __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
@@ -224,47 +231,41 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
     const int tid = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const int N = p.N, nr = p.nr, nc = p.nc;
-    const int q = 4 * (tid & 15), rp0 = tid >> 4;
-    const int nk = N / 32;
+    const int p8 = 8 * (tid & 7), rp0 = tid >> 3;
+    const int nk = N / 64;
     // K_{-1} = h0 + beta_0 w0
     float beta0 = 0.f;
     if (p.two_ep)
         beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
-    float4 k0[pas::KMAX], k1[pas::KMAX];
+    Rows2x8 kst[pas::KMAX];
 #pragma unroll
     for (int k = 0; k < pas::KMAX; ++k) {
-        float a[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
-        if (k < nk) {
-            const int n0 = 2 * (rp0 + 16 * k);
+        const int n0 = 2 * (rp0 + 32 * k);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+        for (int j = 0; j < 8; ++j) {
+            float a = 0.f, d = 0.f;
+            if (k < nk) {
+                const long long i0 = ix_st(p, b, h, n0, p8 + j), i1 = ix_st(p, b, h, n0 + 1, p8 + j);
                 if (p.h0) {
-                    a[j] = p.h0[i0];
-                    d[j] = p.h0[i1];
+                    a = p.h0[i0];
+                    d = p.h0[i1];
                 }
                 if (p.w0) {
-                    a[j] = fmaf(beta0, p.w0[i0], a[j]);
-                    d[j] = fmaf(beta0, p.w0[i1], d[j]);
+                    a = fmaf(beta0, p.w0[i0], a);
+                    d = fmaf(beta0, p.w0[i1], d);
                 }
             }
+            kst[k].a[j] = a;
+            kst[k].d[j] = d;
         }
-        k0[k] = make_float4(a[0], a[1], a[2], a[3]);
-        k1[k] = make_float4(d[0], d[1], d[2], d[3]);
     }
     s_ce[0][tid] = __ldg(p.ws_ce + bhc(p, b, h, 0) * (2 * NP) + tid);
     for (int c = 0; c < nc; ++c) {
         float *slot = p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS;
-        float *sbase = slot + q;
-        float4 sv0[pas::KMAX], sv1[pas::KMAX];
+        Rows2x8 sv[pas::KMAX];
 #pragma unroll
-        for (int k = 0; k < pas::KMAX; ++k) {
-            if (k < nk) {
-                const int n0 = 2 * (rp0 + 16 * k);
-                sv0[k] = *reinterpret_cast<const float4 *>(sbase + (long long)n0 * PD);
-                sv1[k] = *reinterpret_cast<const float4 *>(sbase + (long long)(n0 + 1) * PD);
-            }
-        }
+        for (int k = 0; k < pas::KMAX; ++k)
+            if (k < nk) rows_load_f32(slot, 2 * (rp0 + 32 * k), p8, sv[k]);
         if (c + 1 < nc) s_ce[(c + 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c + 1) * (2 * NP) + tid);
         // every thread has read its part of S_c: the slot can take the state entering chunk c
         __syncthreads();
@@ -272,33 +273,31 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
         unsigned char *tile = reinterpret_cast<unsigned char *>(slot);
 #pragma unroll
         for (int k = 0; k < pas::KMAX; ++k) {
-            const int n0 = 2 * (rp0 + 16 * k);
+            const int n0 = 2 * (rp0 + 32 * k);
             if (k >= nk) {   // rows past N read as zero by the consumers
-                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-                tile_store_rows2(tile, n0, q, z, z);
+                Rows2x8 z;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) z.a[j] = z.d[j] = 0.f;
+                rows_store_tile(tile, n0, p8, z);
                 continue;
             }
-            tile_store_rows2(tile, n0, q, k0[k], k1[k]);
-            float4 &a = k0[k], &d = k1[k];
+            rows_store_tile(tile, n0, p8, kst[k]);
             if (n0 < nr) {
                 const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
-                a.x = fmaf(e0, a.x, sv0[k].x); a.y = fmaf(e0, a.y, sv0[k].y);
-                a.z = fmaf(e0, a.z, sv0[k].z); a.w = fmaf(e0, a.w, sv0[k].w);
-                d.x = fmaf(e1, d.x, sv1[k].x); d.y = fmaf(e1, d.y, sv1[k].y);
-                d.z = fmaf(e1, d.z, sv1[k].z); d.w = fmaf(e1, d.w, sv1[k].w);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    kst[k].a[j] = fmaf(e0, kst[k].a[j], sv[k].a[j]);
+                    kst[k].d[j] = fmaf(e1, kst[k].d[j], sv[k].d[j]);
+                }
             } else {
                 const int m = nr + ((n0 - nr) >> 1);
                 const float er = ce[2 * m], ei = ce[2 * m + 1];
-                // (er + i ei) (a + i d) + S
-                const float4 ao = a;
-                a.x = fmaf(er, ao.x, fmaf(-ei, d.x, sv0[k].x));
-                a.y = fmaf(er, ao.y, fmaf(-ei, d.y, sv0[k].y));
-                a.z = fmaf(er, ao.z, fmaf(-ei, d.z, sv0[k].z));
-                a.w = fmaf(er, ao.w, fmaf(-ei, d.w, sv0[k].w));
-                d.x = fmaf(er, d.x, fmaf(ei, ao.x, sv1[k].x));
-                d.y = fmaf(er, d.y, fmaf(ei, ao.y, sv1[k].y));
-                d.z = fmaf(er, d.z, fmaf(ei, ao.z, sv1[k].z));
-                d.w = fmaf(er, d.w, fmaf(ei, ao.w, sv1[k].w));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {   // (er + i ei) (a + i d) + S
+                    const float ao = kst[k].a[j], dd = kst[k].d[j];
+                    kst[k].a[j] = fmaf(er, ao, fmaf(-ei, dd, sv[k].a[j]));
+                    kst[k].d[j] = fmaf(er, dd, fmaf(ei, ao, sv[k].d[j]));
+                }
             }
         }
     }
@@ -307,20 +306,18 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 #pragma unroll
     for (int k = 0; k < pas::KMAX; ++k) {
         if (k >= nk) break;
-        const int n0 = 2 * (rp0 + 16 * k);
-        const float a[4] = {k0[k].x, k0[k].y, k0[k].z, k0[k].w};
-        const float d[4] = {k1[k].x, k1[k].y, k1[k].z, k1[k].w};
+        const int n0 = 2 * (rp0 + 32 * k);
         const float b0 = p.wT ? ld_io(p.Bm, ix_B(p, b, tl, g, 0, n0), 1) : 0.f;
         const float b1 = p.wT ? ld_io(p.Bm, ix_B(p, b, tl, g, 0, n0 + 1), 1) : 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+        for (int j = 0; j < 8; ++j) {
+            const long long i0 = ix_st(p, b, h, n0, p8 + j), i1 = ix_st(p, b, h, n0 + 1, p8 + j);
             if (p.hT) {
-                p.hT[i0] = a[j];
-                p.hT[i1] = d[j];
+                p.hT[i0] = kst[k].a[j];
+                p.hT[i1] = kst[k].d[j];
             }
             if (p.wT) {
-                const float ul = ld_io(p.x, ix_x(p, b, tl, h, 0, q + j), 1);
+                const float ul = ld_io(p.x, ix_x(p, b, tl, h, 0, p8 + j), 1);
                 p.wT[i0] = b0 * ul;
                 p.wT[i1] = b1 * ul;
             }

@@ -186,19 +186,20 @@ k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant
 
 // ============================================================================
 // k_chunk_adj_pass: reverse pass over the chunks of one (batch row, head).
-// Thread (row-pair group, 4 consecutive p) keeps rows 2rp, 2rp+1 of the adjoint
-// carry for rp = rp0, rp0 + 16, ...: two real modes, or one rotation pair as
-// (re, im).  Every chunk's loads are issued together in 16-byte rows.
-// ws_gc[c] holds Ghat_c on entry and the carry into chunk c on exit.
+// Thread (row-pair group, 8 consecutive p) keeps rows 2rp, 2rp+1 of the adjoint
+// carry for rp = rp0, rp0 + 32: two real modes, or one rotation pair as
+// (re, im).  Every chunk's loads are issued together, in 16-byte pieces.
+// ws_gc[c] holds Ghat_c (fp32) on entry and the carry into chunk c (hi / lo
+// tiles) on exit.
 // ============================================================================
 namespace pass {
 constexpr int THREADS = 256;
-constexpr int KMAX = NP / 32;   // row pairs per thread
+constexpr int KMAX = NP / 64;   // row pairs per thread
 }  // namespace pass
 
-__device__ __forceinline__ float sum16(float v) {
+__device__ __forceinline__ float sum8(float v) {
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 4; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
@@ -209,28 +210,28 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
     const int tid = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const int N = p.N, nr = p.nr, nc = p.nc;
-    const int q = 4 * (tid & 15), rp0 = tid >> 4;
-    const int nk = N / 32;
-    float4 g0[pass::KMAX], g1[pass::KMAX];
+    const int p8 = 8 * (tid & 7), rp0 = tid >> 3;
+    const int nk = N / 64;
+    Rows2x8 g[pass::KMAX];
 #pragma unroll
-    for (int k = 0; k < pass::KMAX; ++k) g0[k] = g1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < pass::KMAX; ++k)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g[k].a[j] = g[k].d[j] = 0.f;
     s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
 
     for (int c = nc - 1; c >= 0; --c) {
         float *slot = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS;
-        float *gbase = slot + q;
         // K_end_{c-1}: the state entering chunk c (tile format)
         const unsigned char *kb = (c > 0 && p.ws_qb)
             ? reinterpret_cast<const unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
             : nullptr;
-        float4 hv0[pass::KMAX], hv1[pass::KMAX], kv0[pass::KMAX], kv1[pass::KMAX];
+        Rows2x8 hv[pass::KMAX], kv[pass::KMAX];
 #pragma unroll
         for (int k = 0; k < pass::KMAX; ++k) {
             if (k < nk) {
-                const int n0 = 2 * (rp0 + 16 * k);
-                hv0[k] = *reinterpret_cast<const float4 *>(gbase + (long long)n0 * PD);
-                hv1[k] = *reinterpret_cast<const float4 *>(gbase + (long long)(n0 + 1) * PD);
-                if (kb) tile_load_rows2(kb, n0, q, kv0[k], kv1[k]);
+                const int n0 = 2 * (rp0 + 32 * k);
+                rows_load_f32(slot, n0, p8, hv[k]);
+                if (kb) rows_load_tile(kb, n0, p8, kv[k]);
             }
         }
         if (c > 0) s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
@@ -241,51 +242,55 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
         unsigned char *tile = reinterpret_cast<unsigned char *>(slot);
 #pragma unroll
         for (int k = 0; k < pass::KMAX; ++k) {
-            const int n0 = 2 * (rp0 + 16 * k);
+            const int n0 = 2 * (rp0 + 32 * k);
             if (k >= nk) {   // rows past N read as zero by the consumers
-                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-                tile_store_rows2(tile, n0, q, z, z);
+                Rows2x8 z;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) z.a[j] = z.d[j] = 0.f;
+                rows_store_tile(tile, n0, p8, z);
                 continue;
             }
             // the carry into chunk c (tile format), then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
-            tile_store_rows2(tile, n0, q, g0[k], g1[k]);
-            float4 &a = g0[k], &d = g1[k];
+            rows_store_tile(tile, n0, p8, g[k]);
+            float *a = g[k].a, *d = g[k].d;
             if (n0 < nr) {
                 const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
-                a.x = fmaf(e0, a.x, hv0[k].x); a.y = fmaf(e0, a.y, hv0[k].y);
-                a.z = fmaf(e0, a.z, hv0[k].z); a.w = fmaf(e0, a.w, hv0[k].w);
-                d.x = fmaf(e1, d.x, hv1[k].x); d.y = fmaf(e1, d.y, hv1[k].y);
-                d.z = fmaf(e1, d.z, hv1[k].z); d.w = fmaf(e1, d.w, hv1[k].w);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    a[j] = fmaf(e0, a[j], hv[k].a[j]);
+                    d[j] = fmaf(e1, d[j], hv[k].d[j]);
+                }
             } else {
                 const int m = nr + ((n0 - nr) >> 1);
                 const float er = ce[2 * m], ei = ce[2 * m + 1];
-                // conj(er + i ei) (a + i d) + Ghat
-                const float4 ao = a;
-                a.x = fmaf(er, ao.x, fmaf(ei, d.x, hv0[k].x));
-                a.y = fmaf(er, ao.y, fmaf(ei, d.y, hv0[k].y));
-                a.z = fmaf(er, ao.z, fmaf(ei, d.z, hv0[k].z));
-                a.w = fmaf(er, ao.w, fmaf(ei, d.w, hv0[k].w));
-                d.x = fmaf(er, d.x, fmaf(-ei, ao.x, hv1[k].x));
-                d.y = fmaf(er, d.y, fmaf(-ei, ao.y, hv1[k].y));
-                d.z = fmaf(er, d.z, fmaf(-ei, ao.z, hv1[k].z));
-                d.w = fmaf(er, d.w, fmaf(-ei, ao.w, hv1[k].w));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {   // conj(er + i ei) (a + i d) + Ghat
+                    const float ao = a[j];
+                    a[j] = fmaf(er, ao, fmaf(ei, d[j], hv[k].a[j]));
+                    d[j] = fmaf(er, d[j], fmaf(-ei, ao, hv[k].d[j]));
+                }
             }
             if (kb) {
-                // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}; 16 lanes hold one row pair
-                float q0, q1;
-                const float4 k0 = kv0[k], k1 = kv1[k];
-                if (n0 < nr) {
-                    q0 = a.x * k0.x + a.y * k0.y + a.z * k0.z + a.w * k0.w;
-                    q1 = d.x * k1.x + d.y * k1.y + d.z * k1.z + d.w * k1.w;
-                } else {
-                    q0 = (a.x * k0.x + a.y * k0.y + a.z * k0.z + a.w * k0.w) +
-                         (d.x * k1.x + d.y * k1.y + d.z * k1.z + d.w * k1.w);
-                    q1 = (a.x * k1.x + a.y * k1.y + a.z * k1.z + a.w * k1.w) -
-                         (d.x * k0.x + d.y * k0.y + d.z * k0.z + d.w * k0.w);
+                // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}; 8 lanes hold one row pair
+                float aa = 0.f, dd = 0.f, ad = 0.f, da = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    aa = fmaf(a[j], kv[k].a[j], aa);
+                    dd = fmaf(d[j], kv[k].d[j], dd);
+                    ad = fmaf(a[j], kv[k].d[j], ad);
+                    da = fmaf(d[j], kv[k].a[j], da);
                 }
-                q0 = sum16(q0);
-                q1 = sum16(q1);
-                if ((tid & 15) == 0) {
+                float q0, q1;
+                if (n0 < nr) {
+                    q0 = aa;
+                    q1 = dd;
+                } else {
+                    q0 = aa + dd;
+                    q1 = ad - da;
+                }
+                q0 = sum8(q0);
+                q1 = sum8(q1);
+                if ((tid & 7) == 0) {
                     qb[n0] = q0;            // slot 0 holds the whole sum over p
                     qb[n0 + 1] = q1;
                     qb[N + n0] = 0.f;       // slot 1 (read by the carry pass) stays zero
@@ -302,21 +307,19 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
 #pragma unroll
     for (int k = 0; k < pass::KMAX; ++k) {
         if (k >= nk) break;
-        const int n0 = 2 * (rp0 + 16 * k);
-        const float a[4] = {g0[k].x, g0[k].y, g0[k].z, g0[k].w};
-        const float d[4] = {g1[k].x, g1[k].y, g1[k].z, g1[k].w};
+        const int n0 = 2 * (rp0 + 32 * k);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const long long i0 = ix_st(p, b, h, n0, q + j), i1 = ix_st(p, b, h, n0 + 1, q + j);
+        for (int j = 0; j < 8; ++j) {
+            const long long i0 = ix_st(p, b, h, n0, p8 + j), i1 = ix_st(p, b, h, n0 + 1, p8 + j);
             if (p.dh0) {
-                p.dh0[i0] = a[j];
-                p.dh0[i1] = d[j];
+                p.dh0[i0] = g[k].a[j];
+                p.dh0[i1] = g[k].d[j];
             }
             if (p.dw0) {
-                p.dw0[i0] = beta0 * a[j];
-                p.dw0[i1] = beta0 * d[j];
+                p.dw0[i0] = beta0 * g[k].a[j];
+                p.dw0[i1] = beta0 * g[k].d[j];
             }
-            if (p.w0) db0 = fmaf(a[j], p.w0[i0], fmaf(d[j], p.w0[i1], db0));
+            if (p.w0) db0 = fmaf(g[k].a[j], p.w0[i0], fmaf(g[k].d[j], p.w0[i1], db0));
         }
     }
     red[tid] = db0;
