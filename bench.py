@@ -103,8 +103,6 @@ def kernel_bytes(shape, name: str) -> int:
         return (BLH * (s.rank_in + s.rank_out) * s.nstate * 4 + t["C"] + t["B"] + t["C"]
                 + t["dt"] + t["lam"])
     # tensor-core chain: path inputs read, path outputs written
-    if name == "k_chunk_out":         # x, B, C, dt, lambda -> y
-        return ins + t["y"]
     if name == "k_chunk_state_local":  # x, B, dt, lambda (chunk states go to workspace)
         return t["x"] + t["B"] + t["dt"] + t["lam"]
     if name == "k_chunk_adj_local":   # C, dt, dy

@@ -183,26 +183,36 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0;
 }
 
-// Forward workspace of the tensor-core chain: the state entering every
-// 64-token chunk [B][H][L/64][N][P] and the chunk decays [B][H][L/64][128][2].
-// A training forward (workspace of `total` bytes) also keeps, per chunk, the
-// masked score tiles (8 KB), the chunk-end folded B tile (16 KB) and the
-// diagonal correction (64 floats) for ssm_scan_bwd_saved; an inference forward
-// needs only the first `total_infer` bytes.
+// Forward workspace of the tensor-core chain.  Every forward carries the fp32
+// state from one 64-token chunk to the next through two 32 KB slots and one
+// counter per (b, h) (the first `total_infer` bytes).  A training forward
+// (workspace of `total` bytes) also keeps, per chunk, the state entering it
+// (bf16 hi + lo tiles, 32 KB), the chunk decays (128 x 2 floats), the masked
+// score tiles (8 KB), the chunk-end folded B tile (16 KB) and the diagonal
+// correction (64 floats) for ssm_scan_bwd_saved.
 struct FwdWs {
-    size_t off_kp, off_ce, off_P, off_Bh, off_corr, total_infer, total;
+    size_t off_ring, off_flag, off_kp, off_ce, off_P, off_Bh, off_corr, total_infer, total;
 };
 FwdWs fwd_layout(const ssm_desc_t *d) {
     FwdWs w;
-    w.off_kp = w.off_ce = w.off_P = w.off_Bh = w.off_corr = w.total_infer = w.total = 0;
+    w.off_ring = w.off_flag = w.off_kp = w.off_ce = w.off_P = w.off_Bh = w.off_corr = 0;
+    w.total_infer = w.total = 0;
     if (!tensor_chain_shape(d)) return w;
-    const size_t units = (size_t)d->batch * d->nheads * (size_t)((d->seqlen + 63) / 64);
-    w.off_kp = 0;
-    // one 32 KB slot per chunk (128 state rows x 64, bf16 hi + lo tiles or the fp32 local sum)
-    size_t off = align256(units * 128 * d->headdim * 4);
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const size_t units = bh * (size_t)((d->seqlen + 63) / 64);
+    const size_t slot = 128 * (size_t)d->headdim * 4;   // 128 state rows x P, fp32 (32 KB)
+    // every forward: the two carry slots and the carry counter of each (b, h)
+    w.off_ring = 0;
+    size_t off = align256(2 * bh * slot);
+    w.off_flag = off;
+    off = align256(off + bh * 4);
+    w.total_infer = off;
+    // a training forward also keeps, per chunk, the state entering it (bf16 hi + lo
+    // tiles), the chunk decays and the products the backward reuses
+    w.off_kp = off;
+    off = align256(off + units * slot);
     w.off_ce = off;
     off = align256(off + units * 128 * 2 * 4);
-    w.total_infer = off;
     w.off_P = off;
     off = align256(off + units * 8192);
     w.off_Bh = off;
@@ -344,9 +354,11 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         if ((uintptr_t)workspace % 256)
             return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
         char *ws = (char *)workspace;
-        p.ws_kp = (float *)(ws + lay.off_kp);
-        p.ws_ce = (float *)(ws + lay.off_ce);
-        if (workspace_bytes >= lay.total) {  // training forward: keep the products for the backward
+        p.ws_ring = (float *)(ws + lay.off_ring);
+        p.ws_flag = (int *)(ws + lay.off_flag);
+        if (workspace_bytes >= lay.total) {  // training forward: keep the states and products
+            p.ws_kp = (float *)(ws + lay.off_kp);
+            p.ws_ce = (float *)(ws + lay.off_ce);
             p.sv_P = (unsigned char *)(ws + lay.off_P);
             p.sv_Bh = (unsigned char *)(ws + lay.off_Bh);
             p.sv_corr = (float *)(ws + lay.off_corr);

@@ -99,15 +99,18 @@ __device__ __forceinline__ void cmul(float a, float b, float c, float d, float &
 // One chunk's dt / lambda of tokens t0 .. t0+64, held in registers of threads
 // 0..64 between the load and the use (so that a persistent kernel can fetch
 // the next chunk's while it works on this one).
+// dt / lambda of one token (bf16 bits), loaded one chunk ahead: the values
+// are converted only when chunk_tokens_from stores them, so the loads stay in
+// flight until then.
 struct TokPrefetch {
-    float dv, lv;
+    unsigned short dv, lv;
 };
 __device__ __forceinline__ TokPrefetch tok_load(const Params &p, int b, int h, int t0) {
-    TokPrefetch r{0.f, 1.f};
+    TokPrefetch r{0, 0x3f80};   // dt 0, lambda 1
     const int i = threadIdx.x, t = t0 + i;
     if (i < Q + 1 && t < p.L) {
-        r.dv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
-        if (p.two_ep) r.lv = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+        r.dv = __ldg(reinterpret_cast<const unsigned short *>(p.dt) + ix_dt(p, b, t, h));
+        if (p.two_ep) r.lv = __ldg(reinterpret_cast<const unsigned short *>(p.lam) + ix_lam(p, b, t, h));
     }
     return r;
 }
@@ -118,8 +121,8 @@ __device__ __forceinline__ void chunk_tokens_from(const Params &p, float *f32, i
                                                   const TokPrefetch &r, bool want_sigma) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < Q + 1) {
-        f32[F_DT + tid] = r.dv;
-        f32[F_LAM + tid] = r.lv;
+        f32[F_DT + tid] = __uint_as_float((uint32_t)r.dv << 16);
+        f32[F_LAM + tid] = __uint_as_float((uint32_t)r.lv << 16);
     }
     __syncthreads();
     if (warp == 0) {
@@ -149,68 +152,92 @@ __device__ __forceinline__ void chunk_tokens(const Params &p, float *f32, int b,
     chunk_tokens_from(p, f32, t0, r, want_sigma);
 }
 
-// Per-mode decay over each sub-block, E_k = e^{lam dS_k} (one thread per mode
-// and sub-block), then the products F[i][j] = prod_{k=i}^{j-1} E_k and
-// G_i = conj(F[0][i]) (one thread per mode) into the F_KRE / F_KIM slots; E_k
-// itself is F[k][k+1].  Needs F_S, F_A2, F_W.  Contains barriers.
+// sin / cos of x after reducing it to [-pi, pi] (the fast intrinsic is only
+// accurate near zero).
+__device__ __forceinline__ void sincos_red(float x, float *sn, float *cs) {
+    const float r = fmaf(-6.28318530717958648f, rintf(x * 0.159154943091895336f), x);
+    __sincosf(r, sn, cs);
+}
+
+// Per-mode decay over each sub-block, E_k = e^{lam dS_k}, the products
+// F[i][j] = prod_{k=i}^{j-1} E_k (E_k itself is F[k][k+1]) and
+// G_i = conj(F[0][i]) into the F_KRE / F_KIM slots.  Four consecutive lanes
+// take one mode, lane k its sub-block k; the four factors are exchanged by
+// shuffles inside the group.  Needs F_S, F_A2, F_W; ends with a barrier.
 __device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
     const int nmode = p.nr + p.np;
     for (int it = threadIdx.x; it < 4 * nmode; it += blockDim.x) {
         const int m = it >> 2, k = it & 3;
+        const unsigned gm = 0xfu << (threadIdx.x & 28);   // the four lanes of this mode
         const float a2 = f32[F_A2 + m], w = f32[F_W + m];
         const float lo = k == 0 ? 0.f : f32[F_S + 16 * k - 1];
         const float ds = f32[F_S + 16 * k + 15] - lo;
-        const float mag = exp2f(a2 * ds);
+        const float mag = ex2_fast(a2 * ds);
         float er = mag, ei = 0.f;
         if (m >= p.nr) {
             float sn, cs;
-            sincosf(w * ds, &sn, &cs);
+            sincos_red(w * ds, &sn, &cs);
             er = mag * cs;
             ei = mag * sn;
         }
-        f32[F_KRE + fslot(k, k + 1) * NP + m] = er;
-        f32[F_KIM + fslot(k, k + 1) * NP + m] = ei;
-    }
-    __syncthreads();
-    for (int m = threadIdx.x; m < nmode; m += blockDim.x) {
+        float Er[4], Ei[4];
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            float pr = f32[F_KRE + fslot(i, i + 1) * NP + m];
-            float pi = f32[F_KIM + fslot(i, i + 1) * NP + m];
-            if (i == 0) {
-                f32[F_KRE + gslot(1) * NP + m] = pr;
-                f32[F_KIM + gslot(1) * NP + m] = -pi;
-            }
+        for (int q = 0; q < 4; ++q) {
+            Er[q] = __shfl_sync(gm, er, q, 4);
+            Ei[q] = __shfl_sync(gm, ei, q, 4);
+        }
+        float *fr = f32 + F_KRE + m, *fi = f32 + F_KIM + m;
+        fr[fslot(k, k + 1) * NP] = er;
+        fi[fslot(k, k + 1) * NP] = ei;
+        // lane k forms F[k][j] for j = k+2 .. 4; lane 0 also the G_i
+        float pr = er, pi = ei;
+        if (k == 0) {
+            fr[gslot(1) * NP] = pr;
+            fi[gslot(1) * NP] = -pi;
+        }
 #pragma unroll
-            for (int j = i + 2; j <= 4; ++j) {
-                float nr_, ni_;
-                cmul(pr, pi, f32[F_KRE + fslot(j - 1, j) * NP + m],
-                     f32[F_KIM + fslot(j - 1, j) * NP + m], nr_, ni_);
-                pr = nr_;
-                pi = ni_;
-                f32[F_KRE + fslot(i, j) * NP + m] = pr;
-                f32[F_KIM + fslot(i, j) * NP + m] = pi;
-                if (i == 0 && j < 4) {
-                    f32[F_KRE + gslot(j) * NP + m] = pr;
-                    f32[F_KIM + gslot(j) * NP + m] = -pi;
-                }
+        for (int j2 = 2; j2 <= 4; ++j2) {
+            const int jj = k + j2;
+            if (jj > 4) break;
+            float nr_, ni_;
+            cmul(pr, pi, Er[jj - 1], Ei[jj - 1], nr_, ni_);
+            pr = nr_;
+            pi = ni_;
+            fr[fslot(k, jj) * NP] = pr;
+            fi[fslot(k, jj) * NP] = pi;
+            if (k == 0 && jj < 4) {
+                fr[gslot(jj) * NP] = pr;
+                fi[gslot(jj) * NP] = -pi;
             }
         }
     }
     __syncthreads();
 }
 
-__device__ __forceinline__ void mode_rates(const Params &p, float *f32, int h) {
-    const int nmode = p.nr + p.np;
-    for (int m = threadIdx.x; m < NP; m += blockDim.x) {
-        float a2 = 0.f, w = 0.f;
-        if (m < nmode) {
-            a2 = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]) * 1.4426950408889634f;
-            if (m >= p.nr) w = p.theta[h * p.np + (m - p.nr)];
-        }
-        f32[F_A2 + m] = a2;
-        f32[F_W + m] = w;
+// Decay rate (times log2 e) and rotation frequency of mode m = threadIdx.x of
+// head h, loaded one chunk ahead; mode_rates_from writes them to F_A2 / F_W.
+struct ModePrefetch {
+    float alog, w;
+};
+__device__ __forceinline__ ModePrefetch mode_load(const Params &p, int h) {
+    ModePrefetch r{0.f, 0.f};
+    const int m = threadIdx.x;
+    if (m < p.nr + p.np) {
+        r.alog = __ldg(p.A_log + h * p.ndec + (p.per_coord ? m : 0));
+        if (m >= p.nr) r.w = __ldg(p.theta + h * p.np + (m - p.nr));
     }
+    return r;
+}
+__device__ __forceinline__ void mode_rates_from(const Params &p, float *f32, const ModePrefetch &r) {
+    const int m = threadIdx.x;
+    if (m < NP) {
+        const bool on = m < p.nr + p.np;
+        f32[F_A2 + m] = on ? -expf(r.alog) * 1.4426950408889634f : 0.f;
+        f32[F_W + m] = on ? r.w : 0.f;
+    }
+}
+__device__ __forceinline__ void mode_rates(const Params &p, float *f32, int h) {
+    mode_rates_from(p, f32, mode_load(p, h));
 }
 
 __device__ __forceinline__ long long bhc(const Params &p, int b, int h, int c) {

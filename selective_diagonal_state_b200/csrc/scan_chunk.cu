@@ -20,15 +20,18 @@
 //   Bh_s  = sigma_s b_s e^{lam (S_63 - S_s)}          chunk-end state contribution
 // The two-endpoint write is used in the pre-state form
 // K_t = A_t K_{t-1} + sigma_t W_t, sigma_t = gamma_t + beta_{t+1}, with
-// y_t = C_t K_t - beta_{t+1} (C_t . B_t) u_t + D u_t.  Three kernels:
-//   k_chunk_state_local (every chunk at once)  S_c = Bh^T (N x 64 s) . X   M=128, N=64
+// y_t = C_t K_t - beta_{t+1} (C_t . B_t) u_t + D u_t.
+//   k_chunk_fwd (persistent, chunks of a (b, h) chained through an fp32 carry)
+//       scores^T_i  = Bi (64 s x N) . Ci^T (N x 16 t)          M=64,  N=16, K=N
+//       Y^T         = K_c^T (64 p x N) . Ch^T (N x 64 t)       M=64,  N=64, K=N
+//       S_c         = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64
+//       K_{c+1}     = e^{lam S_63} K_c + S_c                   elementwise, to the next chunk
+//       Y^T        += X^T (64 p x s) . P^T_i (s x 16 t)        masked scores, M=64, N=16
+// The backward, when it is not handed the forward's workspace, rebuilds the
+// states entering every chunk with two kernels:
+//   k_chunk_state_local (every chunk at once)  S_c = Bh^T X
 //   k_chunk_state_pass  (chunks in order, elementwise over (row pair, p))
-//                        K_c = e^{lam S_63} K_{c-1} + S_c; stores the state
-//                        entering every chunk, hT and the last write
-//   k_chunk_out         (every chunk at once)
-//       scores^T_i  = Bi (64 s x N) . Ci^T (N x 16 t)          M=64, N=16, K=N
-//       Y^T         = K_prev^T (64 p x N) . Ch^T (N x 64 t)    M=64, N=64, K=N
-//                   + X^T (64 p x s) . P^T_i (s x 16 t)        masked scores, M=64, N=16
+//                        K_c = e^{lam S_63} K_{c-1} + S_c; hT and the last write
 #include <cuda.h>
 
 #include "chunk_common.cuh"
@@ -207,13 +210,6 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 
 // ============================================================================
 // k_chunk_state_pass: the carried state over the chunks of one (batch row,
-// head).  Thread (row-pair group, 4 consecutive p) keeps rows 2rp, 2rp+1 for
-// rp = rp0, rp0 + 16, ...: two real modes or one rotation pair as (re, im).
-// Every chunk's loads are issued together (16-byte rows), so that enough bytes
-// are in flight to stream at HBM speed.  ws_kp[c] holds S_c on entry and the
-// state entering chunk c on exit; the state after the last chunk is hT.
-// ============================================================================
-// k_chunk_state_pass: the carried state over the chunks of one (batch row,
 // head).  Thread (row-pair group, 8 consecutive p) keeps rows 2rp, 2rp+1 for
 // rp = rp0, rp0 + 32: two real modes or one rotation pair as (re, im).  Every
 // chunk's loads are issued together, in 16-byte pieces.  ws_kp[c] holds S_c
@@ -326,84 +322,175 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 }
 
 // ============================================================================
-// k_chunk_out: per chunk, y_t = readout of the state entering the chunk
-// + masked in-chunk scores x + (D - beta_{t+1} C_t . B_t) u_t.
-// Persistent: one CTA per SM walks the chunks with a stride of the grid; the
-// next chunk's tiles (TMA, two stages), dt / lambda and entering state are in
-// flight while the current chunk is computed.
+// k_chunk_fwd: the whole forward of one chunk per work item, chunks of a
+// (batch row, head) chained through a carry in global memory.
+//
+// Items run chunk-slowest (item = c * B*H + b*H + h), one persistent CTA per SM
+// with a stride of the grid, so the item of chunk c - 1 of the same (b, h) was
+// taken about B*H items earlier.  Per item:
+//   - K_c, the state entering the chunk, is read from a two-slot fp32 carry
+//     once the item of chunk c - 1 has published it (bounded wait on a
+//     per-(b, h) counter); K_0 = h0 + beta_0 w0.  Its bf16 tile feeds the
+//     readout; with a saving workspace its hi / lo tiles are kept for the
+//     backward.
+//   - operands Ci, Ch, Bi (as for the scores) and Bh (hi + lo) are folded from
+//     raw B / C; the tensor cores form, in one phase,
+//       scores^T_i = Bi (64 s x N) . Ci^T (N x 16 t)          M=64,  N=16, K=N
+//       Y^T        = K_c^T (64 p x N) . Ch^T (N x 64 t)       M=64,  N=64, K=N
+//       S_c        = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64 (hi, lo)
+//   - K_{c+1} = e^{lam S_63} K_c + S_c goes to the carry (hT and the last write
+//     after the last chunk), and the counter of (b, h) is advanced;
+//   - masked scores P^T, then Y^T += X^T (64 p x s) . P^T_i (s x 16 t), and
+//     y_t = Y_t + (D - beta_{t+1} C_t . B_t) u_t.
+// The carry slots (2 x 32 KB per (b, h)) stay in L2.  Every item waits only on
+// an item with a smaller index, which its CTA took earlier, so the chain makes
+// progress whenever the CTAs owning earlier items run.
 // ============================================================================
-namespace outk {
+namespace fwk {
 constexpr int THREADS = 512;
-constexpr int RG = THREADS / 64;   // row groups of the operand preparation
-constexpr uint32_t TMEM_COLS = 64;
+constexpr int RG = THREADS / 64;      // row groups of the operand preparation
+constexpr uint32_t TMEM_COLS = 128;   // Y^T | scores^T (M = 64) in 0..63, S_c (M = 128) in 64..127
 constexpr uint32_t SM_X = 0;          // 2 x 8 KB   x (128B swizzle, rows = t)
-constexpr uint32_t SM_B = 16384;      // 2 x 16 KB  raw B (two 64-row swizzled halves)
-constexpr uint32_t SM_C = 49152;      // 2 x 16 KB  raw C
-constexpr uint32_t SM_CI = 81920;     // 16 KB Ci   K-major (64 t x 128)
-constexpr uint32_t SM_CH = 98304;     // 16 KB Ch   K-major
-constexpr uint32_t SM_BI = 114688;    // 40 KB Bi tiles (16, 32, 48, 64 rows)
-constexpr uint32_t SM_P = 155648;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
-constexpr uint32_t SM_KT = 163840;    // 2 x 16 KB K_prev^T, MN-major (M = 64 p, K = 128 rows)
-constexpr uint32_t SM_F32 = 196608;
+constexpr uint32_t SM_B = 16384;      // 16 KB raw B (two 64-row swizzled halves)
+constexpr uint32_t SM_C = 32768;      // 16 KB raw C
+constexpr uint32_t SM_CI = 49152;     // 16 KB Ci   K-major (64 t x 128)
+constexpr uint32_t SM_CH = 65536;     // 16 KB Ch   K-major
+constexpr uint32_t SM_BI = 81920;     // 40 KB Bi tiles (16, 32, 48, 64 rows)
+constexpr uint32_t SM_BH = 122880;    // 16 KB Bh hi, MN-major (M = state rows, K = s)
+constexpr uint32_t SM_BHL = 139264;   // 16 KB Bh lo
+constexpr uint32_t SM_KT = 155648;    // 16 KB K_c hi tile (MN-major: M = 64 p, K = 128 rows)
+constexpr uint32_t SM_P = 172032;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
+constexpr uint32_t SM_F32 = 180224;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 static_assert(THREADS * 16 == 8192, "one 16-byte piece of the saved P tiles per thread");
-}  // namespace outk
+static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
+constexpr long long FLAG_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
+}  // namespace fwk
 
-__global__ void __launch_bounds__(outk::THREADS, 1)
-k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+// item -> (chunk, head, batch row), chunk slowest
+__device__ __forceinline__ ChunkItem chunk_item_cs(const Params &p, int item) {
+    ChunkItem r;
+    const int bh_n = p.Bsz * p.H;
+    r.c = item / bh_n;
+    const int rest = item - r.c * bh_n;
+    r.b = rest / p.H;
+    r.h = rest - r.b * p.H;
+    return r;
+}
+
+// 4 float4 of the carry: thread (row n, column block cq) holds p = 16 cq + 4 j4 + 0..3;
+// slot layout [cq][j4][row][4] so that a warp reads 32 consecutive rows.
+__device__ __forceinline__ float4 *carry_ptr(const Params &p, int slot, int bh, int cq, int n) {
+    return reinterpret_cast<float4 *>(p.ws_ring) +
+           (((long long)(slot * p.Bsz * p.H + bh) * 4 + cq) * 4) * NP + n;
+}
+
+__device__ __forceinline__ bool wait_count(const int *flag, int target) {
+    for (long long i = 0; i < fwk::FLAG_WAIT_LIMIT; ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v >= target) return true;
+        __nanosleep(64);
+    }
+    return false;
+}
+__device__ __forceinline__ void publish_count(int *flag, int v) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+// K_c of thread (n, cq): the carry slot, or K_0 = h0 + beta_0 w0 for the first chunk
+__device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int n, int cq,
+                                       float (&kc)[16]) {
+    if (n >= p.N) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) kc[j] = 0.f;
+        return;
+    }
+    if (c > 0) {
+        const float4 *src = carry_ptr(p, c & 1, b * p.H + h, cq, n);
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 v = __ldcg(src + j4 * NP);
+            kc[4 * j4] = v.x;
+            kc[4 * j4 + 1] = v.y;
+            kc[4 * j4 + 2] = v.z;
+            kc[4 * j4 + 3] = v.w;
+        }
+        return;
+    }
+    float beta0 = 0.f;
+    if (p.two_ep)
+        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
+        float a = p.h0 ? p.h0[i0] : 0.f;
+        if (p.w0) a = fmaf(beta0, p.w0[i0], a);
+        kc[j] = a;
+    }
+}
+
+__global__ void __launch_bounds__(fwk::THREADS, 1)
+k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, Params p) {
     if (gated_off(p)) return;
-    const int nitems = p.nc * p.H * p.Bsz;
+    const int BH = p.Bsz * p.H;
+    const int nitems = p.nc * BH;
     if ((int)blockIdx.x >= nitems) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + outk::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + outk::SM_BAR);   // [2] stages
-    uint64_t *bar_mma = bar_tma + 2;                                      // [2] phase A, B
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 4);
+    float *f32 = reinterpret_cast<float *>(sm + fwk::SM_F32);
+    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + fwk::SM_BAR);   // [2] x stages
+    uint64_t *bar_bc = bar_x + 2;                                       // raw B, C
+    uint64_t *bar_mma = bar_x + 3;                                      // [2] phase A, B
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 5);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
     const int nbox = N / 64;
-    const uint32_t tile_bytes = (uint32_t)(Q * PD * 2 + 2 * Q * N * 2) + TILE_BYTES;
-    auto issue_tma = [&](int item, int st) {
-        const ChunkItem it = chunk_item(p, item);
+    const int kn_row = 32 * (warp & 3) + lane, kcq = warp >> 2;   // carry: row, column block
+    auto issue_x = [&](int item, int st) {
+        const ChunkItem it = chunk_item_cs(p, item);
+        mbar_expect_tx(&bar_x[st], (uint32_t)(Q * PD * 2));
+        tma_load_4d(sm + fwk::SM_X + st * 8192, &tmX, &bar_x[st], 0, it.h, it.c * Q, it.b);
+    };
+    auto issue_bc = [&](int item) {
+        const ChunkItem it = chunk_item_cs(p, item);
         const int g = it.h / p.hpg, t0 = it.c * Q;
-        mbar_expect_tx(&bar_tma[st], tile_bytes);
-        tma_load_4d(sm + outk::SM_X + st * 8192, &tmX, &bar_tma[st], 0, it.h, t0, it.b);
-        // the state entering the chunk (bf16 tile, the hi part of its slot)
-        bulk_load(sm + outk::SM_KT + st * TILE_BYTES,
-                  p.ws_kp + bhc(p, it.b, it.h, it.c) * SLOT_FLOATS, TILE_BYTES, &bar_tma[st]);
+        mbar_expect_tx(bar_bc, (uint32_t)(2 * Q * N * 2));
         for (int k = 0; k < nbox; ++k) {
-            tma_load_4d(sm + outk::SM_B + st * 16384 + k * 8192, &tmB, &bar_tma[st], 64 * k, g, t0,
-                        it.b);
-            tma_load_4d(sm + outk::SM_C + st * 16384 + k * 8192, &tmC, &bar_tma[st], 64 * k, g, t0,
-                        it.b);
+            tma_load_4d(sm + fwk::SM_B + k * 8192, &tmB, bar_bc, 64 * k, g, t0, it.b);
+            tma_load_4d(sm + fwk::SM_C + k * 8192, &tmC, bar_bc, 64 * k, g, t0, it.b);
         }
     };
 
     int item = blockIdx.x;
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_x[0], 1);
+        mbar_init(&bar_x[1], 1);
+        mbar_init(bar_bc, 1);
+        mbar_init(&bar_mma[0], 2);   // two issuing threads commit phase A
         mbar_init(&bar_mma[1], 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-        issue_tma(item, 0);
+        issue_x(item, 0);
+        issue_bc(item);
     }
-    if (warp == 0) tmem_alloc(tslot, outk::TMEM_COLS);
-    if (N < NP)  // K padding of Ci, Ch, Bi (rows past N are never written)
-        for (int i = tid; i < (int)((outk::SM_P - outk::SM_CI) / 16); i += outk::THREADS)
-            reinterpret_cast<uint4 *>(sm + outk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    if (warp == 0) tmem_alloc(tslot, fwk::TMEM_COLS);
+    if (N < NP)  // K padding of Ci, Ch, Bi and M padding of Bh (rows past N are never written)
+        for (int i = tid; i < (int)((fwk::SM_KT - fwk::SM_CI) / 16); i += fwk::THREADS)
+            reinterpret_cast<uint4 *>(sm + fwk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
     TokPrefetch tok;
+    ModePrefetch mp;
     {
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_cs(p, item);
         tok = tok_load(p, it.b, it.h, it.c * Q);
+        mp = mode_load(p, it.h);
     }
     fence_before_sync();
     __syncthreads();
@@ -411,30 +498,63 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     const uint32_t tbase = *tslot;
     const uint32_t t_y = tbase;                      // Y^T (M=64, lanes 0-15 of each quarter)
     const uint32_t t_sc = tbase + (16u << 16);       // scores^T (M=64, lanes 16-31)
-    float *cpart = reinterpret_cast<float *>(sm + outk::SM_P);   // C.B partials until P is built
+    const uint32_t t_s = tbase + 64u;                // S_c (M=128)
+    float *cpart = reinterpret_cast<float *>(sm + fwk::SM_P);   // C.B partials until P is built
     bool aborted = false;
 
     for (int k = 0; item < nitems; ++k, item += gridDim.x) {
         const int st = k & 1;
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_cs(p, item);
         const int c = it.c, h = it.h, b = it.b;
+        const int bh = b * p.H + h;
         const int t0 = c * Q;
         const int next = item + gridDim.x;
-        unsigned char *sX = sm + outk::SM_X + st * 8192;
-        unsigned char *sB = sm + outk::SM_B + st * 16384;
-        unsigned char *sC = sm + outk::SM_C + st * 16384;
+        unsigned char *sX = sm + fwk::SM_X + st * 8192;
+        const unsigned char *sB = sm + fwk::SM_B, *sC = sm + fwk::SM_C;
 
-        // ---- this chunk's small inputs; the next chunk's in flight -----------
-        mode_rates(p, f32, h);
-        chunk_tokens_from(p, f32, t0, tok, true);
+        // ---- this chunk's small inputs; K_c once the previous chunk has published it
+        mode_rates_from(p, f32, mp);
+        if (tid == 0 && c > 0 && !wait_count(p.ws_flag + bh, c)) raise_error(2);
+        chunk_tokens_from(p, f32, t0, tok, true);   // its barriers order the wait before the loads
+        float kc[16];
+        load_k(p, c, b, h, kn_row, kcq, kc);
         if (next < nitems) {
-            const ChunkItem nx = chunk_item(p, next);
+            const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
-            // the other stage was last read by the previous chunk, which is complete
-            if (tid == 0) issue_tma(next, st ^ 1);
+            mp = mode_load(p, nx.h);
+            // the other x stage was last read by the previous chunk, which is complete
+            if (tid == 0) issue_x(next, st ^ 1);
         }
         chunk_mode_constants(p, f32);
-        int ok = mbar_wait(&bar_tma[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) ? 1 : 0;
+        if (p.ws_ce && tid < p.nr + p.np) {
+            float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
+            ce[2 * tid] = f32[F_KRE + fslot(0, 4) * NP + tid];
+            ce[2 * tid + 1] = f32[F_KIM + fslot(0, 4) * NP + tid];
+        }
+        // K_c: bf16 tile for the readout; hi / lo tiles of the chunk's slot for the backward
+        {
+            unsigned char *slot = p.ws_kp
+                ? reinterpret_cast<unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
+                : nullptr;
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const uint32_t off = off_kmaj(kn_row, 16 * kcq + 8 * g8, 128u, 1024u);
+                float hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float v = kc[8 * g8 + j];
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+                    lo[j] = v - hi[j];
+                }
+                st16(sm + fwk::SM_KT, off, hi);
+                if (slot) {
+                    st16(slot, off, hi);
+                    st16(slot + TILE_BYTES, off, lo);
+                }
+            }
+        }
+        int ok = (mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) &&
+                  mbar_wait(bar_bc, (uint32_t)(k & 1), WAIT_LIMIT)) ? 1 : 0;
         if (!ok) raise_error(1);
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -447,12 +567,18 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
             const float ds = f32[F_S + t] - Sb;
             const float sig = f32[F_SIG + t];
+            unsigned char *sv = p.sv_Bh ? p.sv_Bh + bhc(p, b, h, c) * 16384 : nullptr;
             float corr = 0.f;
 #pragma unroll 1
-            for (int kk = 0; kk < NP / (8 * outk::RG); ++kk) {
-                const int r0 = 8 * (grp + outk::RG * kk);
-                if (r0 >= N) break;
-                float vCI[8], vCH[8], vBI[8], vBX[3][8], rc[8], rb[8];
+            for (int kk = 0; kk < NP / (8 * fwk::RG); ++kk) {
+                const int r0 = 8 * (grp + fwk::RG * kk);
+                if (r0 >= N) {
+                    if (!sv) break;
+                    // K padding of the saved Bh tile
+                    *reinterpret_cast<uint4 *>(sv + off_mnmaj(r0, t, 2048u, 128u)) = make_uint4(0, 0, 0, 0);
+                    continue;
+                }
+                float vCI[8], vCH[8], vBI[8], vBH[8], vBX[3][8], rc[8], rb[8];
                 ld_rows8(sC, t, r0, rc);
                 ld_rows8(sB, t, r0, rb);
 #pragma unroll
@@ -472,6 +598,8 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                         vCI[j + 1] = ci1;
                         vBI[j] = bi0;
                         vBI[j + 1] = bi1;
+                        vBH[j] = bi0 * f32[F_KRE + fslot(ib, 4) * NP + m0];
+                        vBH[j + 1] = bi1 * f32[F_KRE + fslot(ib, 4) * NP + m1];
                         const float g0 = ib ? f32[F_KRE + gslot(ib) * NP + m0] : 1.f;
                         const float g1 = ib ? f32[F_KRE + gslot(ib) * NP + m1] : 1.f;
                         vCH[j] = ci0 * g0;
@@ -499,6 +627,8 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                         vCI[j + 1] = ci1;
                         vBI[j] = bi0;
                         vBI[j + 1] = bi1;
+                        cmul(bi0, bi1, f32[F_KRE + fslot(ib, 4) * NP + m],
+                             f32[F_KIM + fslot(ib, 4) * NP + m], vBH[j], vBH[j + 1]);
                         float gr = 1.f, gi = 0.f;
                         if (ib) {
                             gr = f32[F_KRE + gslot(ib) * NP + m];
@@ -515,14 +645,23 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                         }
                     }
                 }
-                st16(sm + outk::SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
-                st16(sm + outk::SM_CH, off_kmaj(t, r0, KM_LBO, KM_SBO), vCH);
-                st16(sm + outk::SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
+                st16(sm + fwk::SM_CI, off_kmaj(t, r0, KM_LBO, KM_SBO), vCI);
+                st16(sm + fwk::SM_CH, off_kmaj(t, r0, KM_LBO, KM_SBO), vCH);
+                st16(sm + fwk::SM_BI + bi_off(ib), off_kmaj(t, r0, KM_LBO, KM_SBO), vBI);
 #pragma unroll
                 for (int qq = 0; qq < 3; ++qq) {
                     const int i2 = ib + 1 + qq;
                     if (i2 < 4)
-                        st16(sm + outk::SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
+                        st16(sm + fwk::SM_BI + bi_off(i2), off_kmaj(t, r0, KM_LBO, KM_SBO), vBX[qq]);
+                }
+                st16_split(sm + fwk::SM_BH, sm + fwk::SM_BHL, off_mnmaj(r0, t, 2048u, 128u), vBH);
+                if (sv) {  // the bf16 Bh tile (hi part) for the backward's dx
+                    uint4 w;
+                    w.x = pack_bf16(vBH[0], vBH[1]);
+                    w.y = pack_bf16(vBH[2], vBH[3]);
+                    w.z = pack_bf16(vBH[4], vBH[5]);
+                    w.w = pack_bf16(vBH[6], vBH[7]);
+                    *reinterpret_cast<uint4 *>(sv + off_mnmaj(r0, t, 2048u, 128u)) = w;
                 }
             }
             cpart[grp * 64 + t] = corr;
@@ -530,11 +669,13 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        // raw B and C are consumed: fetch the next chunk's
+        if (tid == 0 && next < nitems) issue_bc(next);
 
-        // ---- phase A: scores, readout of the carried state ---------------------
+        // ---- phase A: scores, readout of K_c, chunk-local state ---------------
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t bi_base = smem_u32(sm + outk::SM_BI), ci_base = smem_u32(sm + outk::SM_CI);
+            const uint32_t bi_base = smem_u32(sm + fwk::SM_BI), ci_base = smem_u32(sm + fwk::SM_CI);
             const uint32_t id_sc = idesc_bf16(64, 16, false, false);
             for (int i = 0; i < NSB; ++i)
                 for (int s = 0; s < NP / 16; ++s)
@@ -542,22 +683,36 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              id_sc, s > 0);
-            const uint32_t kt_base = smem_u32(sm + outk::SM_KT + st * TILE_BYTES);
-            const uint32_t ch_base = smem_u32(sm + outk::SM_CH);
+            const uint32_t kt_base = smem_u32(sm + fwk::SM_KT);
+            const uint32_t ch_base = smem_u32(sm + fwk::SM_CH);
             const uint32_t id_y = idesc_bf16(64, 64, true, false);
             for (int s = 0; s < NP / 16; ++s)
                 mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),
                          sdesc(ch_base + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE), id_y, s > 0);
             mma_commit(&bar_mma[0]);
+        } else if (tid == 32) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sX);
+            const uint32_t id_s = idesc_bf16(128, 64, true, true);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t bh_base = smem_u32(sm + (part ? fwk::SM_BHL : fwk::SM_BH));
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(t_s, sdesc(bh_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                             sdesc(x_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_s,
+                             part > 0 || s > 0);
+            }
+            mma_commit(&bar_mma[0]);
         }
         if (tid < 64) {
             float cs = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < outk::RG; ++kk) cs += cpart[kk * 64 + tid];
+            for (int kk = 0; kk < fwk::RG; ++kk) cs += cpart[kk * 64 + tid];
             const float corr = -f32[F_BN + tid] * cs + ((p.R == p.O) ? p.D[h] : 0.f);
             f32[F_CORR + tid] = corr;
             if (p.sv_corr) p.sv_corr[bhc(p, b, h, c) * Q + tid] = corr;
         }
+        // K_c again (fp32), in flight while the tensor cores work
+        load_k(p, c, b, h, kn_row, kcq, kc);
         ok = mbar_wait(&bar_mma[0], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
         if (!ok) raise_error(1);
         fence_after_sync();
@@ -565,8 +720,50 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             aborted = true;
             break;
         }
-        // ---- masked scores -> P^T tiles (one warp per TMEM lane quarter) -------
-        if (warp >= 4 && warp < 12) {   // two warps per TMEM lane quarter, two blocks each
+        // ---- carry: K_{c+1} = e^{lam S_63} K_c + S_c (thread: row n, 16 columns) ----
+        {
+            float sv16[16];
+            tmem_ld16(tmem_addr(t_s, 32u * (warp & 3), 16u * kcq), sv16);
+            const int n = kn_row;
+            const bool vrow = n < N;
+            const bool pr = vrow && n >= nr;
+            const bool im = pr && ((n - nr) & 1);
+            const int m = pr ? nr + ((n - nr) >> 1) : (vrow ? n : 0);
+            const float er = f32[F_KRE + fslot(0, 4) * NP + m];
+            const float ei = pr ? f32[F_KIM + fslot(0, 4) * NP + m] : 0.f;
+            float kn[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float other = __shfl_xor_sync(0xffffffffu, kc[j], 1);
+                if (!vrow)
+                    kn[j] = 0.f;
+                else if (!pr)
+                    kn[j] = fmaf(er, kc[j], sv16[j]);
+                else if (!im)   // (er + i ei)(a + i d) + S, own row = re
+                    kn[j] = fmaf(er, kc[j], fmaf(-ei, other, sv16[j]));
+                else            // own row = im
+                    kn[j] = fmaf(er, kc[j], fmaf(ei, other, sv16[j]));
+            }
+            if (c + 1 < p.nc) {
+                float4 *dst = carry_ptr(p, (c + 1) & 1, bh, kcq, n);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(kn[4 * j4], kn[4 * j4 + 1], kn[4 * j4 + 2],
+                                                      kn[4 * j4 + 3]));
+            } else if (vrow) {
+                // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write B_{L-1} u_{L-1}
+                const int g = h / p.hpg, tl = L - 1;
+                const float bl = p.wT ? ld_io(p.Bm, ix_B(p, b, tl, g, 0, n), 1) : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const long long i0 = ix_st(p, b, h, n, 16 * kcq + j);
+                    if (p.hT) p.hT[i0] = kn[j];
+                    if (p.wT) p.wT[i0] = bl * ld_io(p.x, ix_x(p, b, tl, h, 0, 16 * kcq + j), 1);
+                }
+            }
+        }
+        // ---- masked scores -> P^T tiles (two warps per TMEM lane quarter) -------
+        if (warp >= 4 && warp < 12) {
             const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);
             for (int i = i0; i < i0 + 2; ++i) {
                 float v[16];
@@ -581,12 +778,12 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                             lo[j] = (s <= 16 * i + j) ? v[j] : 0.f;
                             hi[j] = (s <= 16 * i + 8 + j) ? v[8 + j] : 0.f;
                         }
-                        unsigned char *pt = sm + outk::SM_P + i * 2048;
+                        unsigned char *pt = sm + fwk::SM_P + i * 2048;
                         st16(pt, off_mnmaj(0, s, 256u, 128u), lo);
                         st16(pt, off_mnmaj(8, s, 256u, 128u), hi);
                     } else if (p.sv_P) {
                         // rows past the block are zero in the saved copy (read there as P^T)
-                        unsigned char *pt = sm + outk::SM_P + i * 2048;
+                        unsigned char *pt = sm + fwk::SM_P + i * 2048;
                         *reinterpret_cast<uint4 *>(pt + off_mnmaj(0, s, 256u, 128u)) = make_uint4(0, 0, 0, 0);
                         *reinterpret_cast<uint4 *>(pt + off_mnmaj(8, s, 256u, 128u)) = make_uint4(0, 0, 0, 0);
                     }
@@ -596,14 +793,16 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        // the carry of (b, h) is in place: let the next chunk's item go
+        if (tid == 0 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
         if (p.sv_P)  // the masked score tiles, for the backward's dx (512 threads x 16 bytes)
             *reinterpret_cast<uint4 *>(p.sv_P + bhc(p, b, h, c) * 8192 + tid * 16) =
-                *reinterpret_cast<const uint4 *>(sm + outk::SM_P + tid * 16);
+                *reinterpret_cast<const uint4 *>(sm + fwk::SM_P + tid * 16);
 
         // ---- phase B: intra-chunk term Y^T += X^T P^T_i ----------------------
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + outk::SM_P);
+            const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + fwk::SM_P);
             const uint32_t id_d = idesc_bf16(64, 16, true, true);
             for (int i = 0; i < NSB; ++i)
                 for (int s = 0; s <= i; ++s)
@@ -625,7 +824,7 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             const int pp = 16 * qd + (lane & 15);
             __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
                                   h * p.sy[2] + pp;
-            constexpr int CPW = 64 / (outk::THREADS / 128);
+            constexpr int CPW = 64 / (fwk::THREADS / 128);
             for (int c16 = 0; c16 < CPW / 16; ++c16) {
                 float v[16];
                 const int tc = CPW * part + 16 * c16;
@@ -649,14 +848,15 @@ k_chunk_out(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     }
     if (aborted && tid == 0) {
         // let loads still in flight land before the CTA's shared memory goes away
-        mbar_wait(&bar_tma[0], 0, WAIT_LIMIT);
-        mbar_wait(&bar_tma[1], 0, WAIT_LIMIT);
+        mbar_wait(&bar_x[0], 0, WAIT_LIMIT);
+        mbar_wait(&bar_x[1], 0, WAIT_LIMIT);
+        mbar_wait(bar_bc, 0, WAIT_LIMIT);
     }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         fence_after_sync();
-        tmem_dealloc(tbase, outk::TMEM_COLS);
+        tmem_dealloc(tbase, fwk::TMEM_COLS);
     }
 }
 
@@ -759,19 +959,22 @@ cudaError_t chunk_states(const Params &p, cudaStream_t st) {
 
 cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     using namespace chunkfwd;
-    cudaError_t e = chunk_states(p, st);
-    if (e != cudaSuccess) return e;
     CUtensorMap mx, mb, mc;
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
         !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
         !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true))
         return cudaErrorInvalidValue;
+    if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
     static bool a3 = false;
-    if ((e = set_smem_once(k_chunk_out, outk::SMEM_BYTES, a3)) != cudaSuccess) return e;
+    cudaError_t e;
+    if ((e = set_smem_once(k_chunk_fwd, fwk::SMEM_BYTES, a3)) != cudaSuccess) return e;
+    // the per-(b, h) carry counters start at zero on every call
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
+        return e;
     const long long nitems = (long long)p.nc * p.H * p.Bsz;
     const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
-    k_chunk_out<<<grid, outk::THREADS, outk::SMEM_BYTES, st>>>(mx, mb, mc, p);
-    profile_mark(st, "k_chunk_out");
+    k_chunk_fwd<<<grid, fwk::THREADS, fwk::SMEM_BYTES, st>>>(mx, mb, mc, p);
+    profile_mark(st, "k_chunk_fwd");
     return cudaGetLastError();
 }
 

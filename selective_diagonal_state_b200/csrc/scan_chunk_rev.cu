@@ -833,9 +833,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     }
     if (warp == 0) tmem_alloc(tslot, fuk::TMEM_COLS);
     TokPrefetch tok;
+    ModePrefetch mp;
     {
         const ChunkItem it = chunk_item(p, item);
         tok = tok_load(p, it.b, it.h, it.c * Q);
+        mp = mode_load(p, it.h);
     }
     fence_before_sync();
     __syncthreads();
@@ -852,11 +854,12 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const long long u = bhc(p, b, h, c);
         const int next = item + gridDim.x;
         const uint32_t par = (uint32_t)(kit & 1);
-        mode_rates(p, f32, h);
+        mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
         if (next < nitems) {
             const ChunkItem nx = chunk_item(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
+            mp = mode_load(p, nx.h);
         }
         chunk_mode_constants(p, f32);
         int ok = (mbar_wait(&bar_in[0], par, WAIT_LIMIT) && mbar_wait(&bar_in[1], par, WAIT_LIMIT)) ? 1 : 0;
@@ -1251,16 +1254,21 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             p.ws_M2[ii] = m2;
             p.ws_ddt[ii] = dd;
         }
-        if (tid == 64) {
-            const int nmode = p.nr + p.np;
-            float *blk = p.ws_blk + u * (4 * nmode + 2);
-            float st_ = 0.f, dD = 0.f;
-            for (int t = 0; t < Q; ++t) {
-                st_ += f32[F_DT + t];
-                if (t0 + t < L) dD += f32[F_LAM + t];
+        if (warp == 2) {   // the chunk's sum of dt and of <dy_t, u_t>
+            float st_ = f32[F_DT + lane] + f32[F_DT + lane + 32];
+            float dD = (t0 + lane < L ? f32[F_LAM + lane] : 0.f) +
+                       (t0 + lane + 32 < L ? f32[F_LAM + lane + 32] : 0.f);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                st_ += __shfl_xor_sync(0xffffffffu, st_, o);
+                dD += __shfl_xor_sync(0xffffffffu, dD, o);
             }
-            blk[4 * nmode + 0] = st_;
-            blk[4 * nmode + 1] = (p.O == p.R) ? dD : 0.f;
+            if (lane == 0) {
+                const int nmode = p.nr + p.np;
+                float *blk = p.ws_blk + u * (4 * nmode + 2);
+                blk[4 * nmode + 0] = st_;
+                blk[4 * nmode + 1] = (p.O == p.R) ? dD : 0.f;
+            }
         }
         fence_before_sync();
         __syncthreads();

@@ -55,15 +55,16 @@ def test_contiguous_strides(lib):
 def test_workspace_size(lib):
     sh = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=100)
     d = abi.make_desc(sh)
-    # tensor-core chain: the state entering every 64-token chunk + chunk decays
+    # tensor-core chain: a forward alone needs the two fp32 carry slots and the
+    # counter of every (b, h); a training forward also keeps, per chunk, the
+    # entering state (32 KB), the chunk decays and the products the backward
+    # reuses (8 + 16 KB + 64 floats)
     nc = (100 + 63) // 64
-    nf = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
-    assert nf >= 2 * 32 * nc * (128 * 64 + 128 * 2) * 4 and nf % 256 == 0
-    # a forward alone keeps only the chunk states; a training forward also the
-    # per-chunk products the backward reuses (8 + 16 KB + 64 floats per chunk)
     ni = abi.ssm_scan_workspace_size(d, abi.PASS_FWD_INFER)
-    assert ni >= 2 * 32 * nc * (128 * 64 + 128 * 2) * 4 and ni % 256 == 0
-    assert nf - ni >= 2 * 32 * nc * (8192 + 16384 + 256)
+    assert ni >= 2 * 32 * (2 * 128 * 64 * 4 + 4) and ni % 256 == 0
+    nf = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
+    assert nf % 256 == 0
+    assert nf - ni >= 2 * 32 * nc * (128 * 64 * 4 + 128 * 2 * 4 + 8192 + 16384 + 256)
     # the recurrent chain needs none
     for kw in (dict(chunk=1), dict(dtype_io=S.DTYPE_F32), dict(headdim=32)):
         assert abi.ssm_scan_workspace_size(abi.make_desc(sh.replace(**kw)), abi.PASS_FWD) == 0
