@@ -321,6 +321,45 @@ __device__ __forceinline__ ChunkItem chunk_item(const Params &p, int item) {
     return r;
 }
 
+// ---- chunks chained through a carry in global memory ---------------------------
+// A persistent kernel walks the chunks of every (b, h) in order, chunk slowest.
+// The item of chunk c reads the fp32 carry from slot c & 1 once the counter of
+// (b, h) reaches c, writes the next carry to slot (c + 1) & 1 and sets the
+// counter to c + 1.
+constexpr long long FLAG_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
+
+// item -> (chunk, head, batch row), chunk slowest
+__device__ __forceinline__ ChunkItem chunk_item_cs(const Params &p, int item) {
+    ChunkItem r;
+    const int bh_n = p.Bsz * p.H;
+    r.c = item / bh_n;
+    const int rest = item - r.c * bh_n;
+    r.b = rest / p.H;
+    r.h = rest - r.b * p.H;
+    return r;
+}
+
+// 4 float4 of the carry: thread (row n, column block cq) holds p = 16 cq + 4 j4 + 0..3;
+// slot layout [cq][j4][row][4] so that a warp reads 32 consecutive rows.
+__device__ __forceinline__ float4 *carry_ptr(const Params &p, int slot, int bh, int cq, int n) {
+    return reinterpret_cast<float4 *>(p.ws_ring) +
+           (((long long)(slot * p.Bsz * p.H + bh) * 4 + cq) * 4) * NP + n;
+}
+
+__device__ __forceinline__ bool wait_count(const int *flag, int target) {
+    for (long long i = 0; i < FLAG_WAIT_LIMIT; ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v >= target) return true;
+        __nanosleep(64);
+    }
+    return false;
+}
+__device__ __forceinline__ void publish_count(int *flag, int v) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
 // ---- host side ---------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

@@ -365,40 +365,7 @@ constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
 static_assert(THREADS * 16 == 8192, "one 16-byte piece of the saved P tiles per thread");
 static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
-constexpr long long FLAG_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
 }  // namespace fwk
-
-// item -> (chunk, head, batch row), chunk slowest
-__device__ __forceinline__ ChunkItem chunk_item_cs(const Params &p, int item) {
-    ChunkItem r;
-    const int bh_n = p.Bsz * p.H;
-    r.c = item / bh_n;
-    const int rest = item - r.c * bh_n;
-    r.b = rest / p.H;
-    r.h = rest - r.b * p.H;
-    return r;
-}
-
-// 4 float4 of the carry: thread (row n, column block cq) holds p = 16 cq + 4 j4 + 0..3;
-// slot layout [cq][j4][row][4] so that a warp reads 32 consecutive rows.
-__device__ __forceinline__ float4 *carry_ptr(const Params &p, int slot, int bh, int cq, int n) {
-    return reinterpret_cast<float4 *>(p.ws_ring) +
-           (((long long)(slot * p.Bsz * p.H + bh) * 4 + cq) * 4) * NP + n;
-}
-
-__device__ __forceinline__ bool wait_count(const int *flag, int target) {
-    for (long long i = 0; i < fwk::FLAG_WAIT_LIMIT; ++i) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-        if (v >= target) return true;
-        __nanosleep(64);
-    }
-    return false;
-}
-__device__ __forceinline__ void publish_count(int *flag, int v) {
-    __threadfence();
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
-}
 
 // K_c of thread (n, cq): the carry slot, or K_0 = h0 + beta_0 w0 for the first chunk
 __device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int n, int cq,
@@ -793,8 +760,9 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        // the carry of (b, h) is in place: let the next chunk's item go
-        if (tid == 0 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
+        // the carry of (b, h) is in place: let the next chunk's item go (a thread off the
+        // tensor-core issue path)
+        if (tid == fwk::THREADS - 32 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
         if (p.sv_P)  // the masked score tiles, for the backward's dx (512 threads x 16 bytes)
             *reinterpret_cast<uint4 *>(p.sv_P + bhc(p, b, h, c) * 8192 + tid * 16) =
                 *reinterpret_cast<const uint4 *>(sm + fwk::SM_P + tid * 16);
