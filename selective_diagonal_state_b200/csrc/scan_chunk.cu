@@ -328,20 +328,23 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 // Items run chunk-slowest (item = c * B*H + b*H + h), one persistent CTA per SM
 // with a stride of the grid, so the item of chunk c - 1 of the same (b, h) was
 // taken about B*H items earlier.  Per item:
+//   - operands Ci, Ch, Bi (as for the scores) and Bh (hi + lo) are folded from
+//     raw B / C; phase A of the tensor cores needs no carried state:
+//       scores^T_i = Bi (64 s x N) . Ci^T (N x 16 t)          M=64,  N=16, K=N
+//       S_c        = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64 (hi, lo)
 //   - K_c, the state entering the chunk, is read from a two-slot fp32 carry
 //     once the item of chunk c - 1 has published it (bounded wait on a
-//     per-(b, h) counter); K_0 = h0 + beta_0 w0.  Its bf16 tile feeds the
-//     readout; with a saving workspace its hi / lo tiles are kept for the
-//     backward.
-//   - operands Ci, Ch, Bi (as for the scores) and Bh (hi + lo) are folded from
-//     raw B / C; the tensor cores form, in one phase,
-//       scores^T_i = Bi (64 s x N) . Ci^T (N x 16 t)          M=64,  N=16, K=N
+//     per-(b, h) counter; K_0 = h0 + beta_0 w0); K_{c+1} = e^{lam S_63} K_c + S_c
+//     goes to the other slot (hT and the last write after the last chunk) and
+//     the counter of (b, h) is advanced.  K_c's bf16 tile feeds the readout;
+//     with a saving workspace its hi / lo tiles are kept for the backward;
+//   - masked scores P^T, then phase B
 //       Y^T        = K_c^T (64 p x N) . Ch^T (N x 64 t)       M=64,  N=64, K=N
-//       S_c        = Bh^T (N x 64 s) . X (64 s x 64 p)        M=128, N=64 (hi, lo)
-//   - K_{c+1} = e^{lam S_63} K_c + S_c goes to the carry (hT and the last write
-//     after the last chunk), and the counter of (b, h) is advanced;
-//   - masked scores P^T, then Y^T += X^T (64 p x s) . P^T_i (s x 16 t), and
-//     y_t = Y_t + (D - beta_{t+1} C_t . B_t) u_t.
+//                  + X^T (64 p x s) . P^T_i (s x 16 t)        M=64,  N=16
+//     and y_t = Y_t + (D - beta_{t+1} C_t . B_t) u_t.
+// Only the carry step sits on the chain of a (b, h), so the chain stays short
+// even when B*H is below the number of SMs and the chunks of one (b, h) run
+// side by side.
 // The carry slots (2 x 32 KB per (b, h)) stay in L2.  Every item waits only on
 // an item with a smaller index, which its CTA took earlier, so the chain makes
 // progress whenever the CTAs owning earlier items run.
@@ -481,10 +484,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 
         // ---- this chunk's small inputs; K_c once the previous chunk has published it
         mode_rates_from(p, f32, mp);
-        if (tid == 0 && c > 0 && !wait_count(p.ws_flag + bh, c)) raise_error(2);
-        chunk_tokens_from(p, f32, t0, tok, true);   // its barriers order the wait before the loads
-        float kc[16];
-        load_k(p, c, b, h, kn_row, kcq, kc);
+        chunk_tokens_from(p, f32, t0, tok, true);
         if (next < nitems) {
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
@@ -497,28 +497,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
             ce[2 * tid] = f32[F_KRE + fslot(0, 4) * NP + tid];
             ce[2 * tid + 1] = f32[F_KIM + fslot(0, 4) * NP + tid];
-        }
-        // K_c: bf16 tile for the readout; hi / lo tiles of the chunk's slot for the backward
-        {
-            unsigned char *slot = p.ws_kp
-                ? reinterpret_cast<unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
-                : nullptr;
-#pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-                const uint32_t off = off_kmaj(kn_row, 16 * kcq + 8 * g8, 128u, 1024u);
-                float hi[8], lo[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float v = kc[8 * g8 + j];
-                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
-                    lo[j] = v - hi[j];
-                }
-                st16(sm + fwk::SM_KT, off, hi);
-                if (slot) {
-                    st16(slot, off, hi);
-                    st16(slot + TILE_BYTES, off, lo);
-                }
-            }
         }
         int ok = (mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) &&
                   mbar_wait(bar_bc, (uint32_t)(k & 1), WAIT_LIMIT)) ? 1 : 0;
@@ -633,13 +611,15 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             }
             cpart[grp * 64 + t] = corr;
         }
+        // K_c is published by the item of chunk c - 1 (everything above does not need it)
+        if (tid == 0 && c > 0 && !wait_count(p.ws_flag + bh, c)) raise_error(2);
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();
+        __syncthreads();   // also orders the wait before every thread's loads of K_c
         // raw B and C are consumed: fetch the next chunk's
         if (tid == 0 && next < nitems) issue_bc(next);
 
-        // ---- phase A: scores, readout of K_c, chunk-local state ---------------
+        // ---- phase A: scores, chunk-local state --------------------------------
         if (tid == 0) {
             fence_after_sync();
             const uint32_t bi_base = smem_u32(sm + fwk::SM_BI), ci_base = smem_u32(sm + fwk::SM_CI);
@@ -650,12 +630,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(bi_base + bi_off(i) + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              id_sc, s > 0);
-            const uint32_t kt_base = smem_u32(sm + fwk::SM_KT);
-            const uint32_t ch_base = smem_u32(sm + fwk::SM_CH);
-            const uint32_t id_y = idesc_bf16(64, 64, true, false);
-            for (int s = 0; s < NP / 16; ++s)
-                mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),
-                         sdesc(ch_base + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE), id_y, s > 0);
             mma_commit(&bar_mma[0]);
         } else if (tid == 32) {
             fence_after_sync();
@@ -678,7 +652,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             f32[F_CORR + tid] = corr;
             if (p.sv_corr) p.sv_corr[bhc(p, b, h, c) * Q + tid] = corr;
         }
-        // K_c again (fp32), in flight while the tensor cores work
+        // K_c (fp32), in flight while the tensor cores work
+        float kc[16];
         load_k(p, c, b, h, kn_row, kcq, kc);
         ok = mbar_wait(&bar_mma[0], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
         if (!ok) raise_error(1);
@@ -686,6 +661,28 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (!__syncthreads_and(ok)) {
             aborted = true;
             break;
+        }
+        // K_c: bf16 tile for the readout; hi / lo tiles of the chunk's slot for the backward
+        {
+            unsigned char *slot = p.ws_kp
+                ? reinterpret_cast<unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
+                : nullptr;
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const uint32_t off = off_kmaj(kn_row, 16 * kcq + 8 * g8, 128u, 1024u);
+                float hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float v = kc[8 * g8 + j];
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+                    lo[j] = v - hi[j];
+                }
+                st16(sm + fwk::SM_KT, off, hi);
+                if (slot) {
+                    st16(slot, off, hi);
+                    st16(slot + TILE_BYTES, off, lo);
+                }
+            }
         }
         // ---- carry: K_{c+1} = e^{lam S_63} K_c + S_c (thread: row n, 16 columns) ----
         {
@@ -767,9 +764,15 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             *reinterpret_cast<uint4 *>(p.sv_P + bhc(p, b, h, c) * 8192 + tid * 16) =
                 *reinterpret_cast<const uint4 *>(sm + fwk::SM_P + tid * 16);
 
-        // ---- phase B: intra-chunk term Y^T += X^T P^T_i ----------------------
+        // ---- phase B: Y^T = K_c^T Ch^T (readout) + X^T P^T_i (intra-chunk) ----------
         if (tid == 0) {
             fence_after_sync();
+            const uint32_t kt_base = smem_u32(sm + fwk::SM_KT);
+            const uint32_t ch_base = smem_u32(sm + fwk::SM_CH);
+            const uint32_t id_y = idesc_bf16(64, 64, true, false);
+            for (int s = 0; s < NP / 16; ++s)
+                mma_bf16(t_y, sdesc(kt_base + s * 2048u, 1024u, 128u, LAYOUT_NONE),
+                         sdesc(ch_base + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE), id_y, s > 0);
             const uint32_t x_base = smem_u32(sX), p_base = smem_u32(sm + fwk::SM_P);
             const uint32_t id_d = idesc_bf16(64, 16, true, true);
             for (int i = 0; i < NSB; ++i)
