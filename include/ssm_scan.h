@@ -208,6 +208,28 @@ SSM_API int ssm_scan_bwd_noalloc(const ssm_desc_t *d, const void *x, const void 
                                  void *dC, float *dD, void *dlambda, float *dh0,
                                  float *dprev_write, void *stream);
 
+/*
+ * One recurrent step (autoregressive decoding): the recurrence of
+ * ssm_scan_fwd for a single token, with the state kept by the caller
+ * ("State Space Models", robocikowo.com: glossary item 2, the discretised
+ * recurrence, and the complexity entry, constant memory per token in
+ * autoregressive inference).  For every (batch row, head):
+ *     h <- A_t (h + beta_t w) + gamma_t W_t,   W_t = B_t u_t,   w <- W_t
+ *     y_t = C_t h + D u_t
+ * h and w are fp32 [batch][nheads][N][headdim], read and overwritten in
+ * place: h holds H_{t-1} on entry and H_t on return; w holds the previous
+ * write W_{t-1} on entry and W_t on return.  w may be NULL when
+ * two_endpoint == 0 (then nothing is read from or written to it).
+ * The token's x, dt, B, C, lambda and y use the layouts and strides of
+ * ssm_scan_fwd with time index 0; d->seqlen must be 1.  Starting from
+ * h = h0, w = prev_write and calling this once per token gives the y, hT and
+ * last_write of ssm_scan_fwd over the sequence up to rounding.  rank_in and
+ * rank_out up to 8.  No workspace; errors as ssm_scan_fwd.
+ */
+SSM_API int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                          const float *theta, const void *B, const void *C, const float *D,
+                          const void *lambda, float *h, float *w, void *y, void *stream);
+
 /* Message describing the last failing call on this host thread ("" if none). */
 SSM_API const char *ssm_scan_last_error(void);
 

@@ -24,7 +24,8 @@ PASS_FWD, PASS_BWD, PASS_FWD_INFER = 0, 1, 2
 EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd",
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
-            "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved"]
+            "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
+            "ssm_scan_step"]
 ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -77,6 +78,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_scan_bwd_saved.argtypes = ([ctypes.POINTER(Desc)] + [_vp] * 22 +
                                        [ctypes.c_size_t, _vp, ctypes.c_size_t, _vp])
     lib.ssm_scan_bwd_saved.restype = ctypes.c_int
+    lib.ssm_scan_step.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 12
+    lib.ssm_scan_step.restype = ctypes.c_int
     lib.ssm_scan_last_error.argtypes = []
     lib.ssm_scan_last_error.restype = ctypes.c_char_p
     lib.ssm_scan_poll_device_error.argtypes = [_vp]
@@ -144,6 +147,15 @@ def ssm_scan_fwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, 
         x, dt, A_log, theta, B, C, D, lam, h0, prev_write, y, hT, last_write, workspace)],
         workspace_bytes, _stream(stream))
     _check(rc, "ssm_scan_fwd")
+
+
+def ssm_scan_step(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h, w, y, stream=None) -> None:
+    """One recurrent step; ``h`` and ``w`` (fp32 state and previous write) are
+    updated in place."""
+    lib = load_library()
+    rc = lib.ssm_scan_step(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h, w, y)], _stream(stream))
+    _check(rc, "ssm_scan_step")
 
 
 def ssm_scan_bwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt,

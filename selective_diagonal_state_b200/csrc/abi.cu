@@ -23,6 +23,8 @@ bool chunk_fwd_supported(const Params &p);
 cudaError_t chunk_forward(const Params &p, cudaStream_t st);
 int chunk_error_take();
 int chunk_rev_error_take();
+bool step_supported(const Params &p);
+cudaError_t scan_step(const Params &p, float *h, float *w, cudaStream_t st);
 }  // namespace ssm
 
 namespace {
@@ -321,6 +323,35 @@ size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
     return bwd_layout(d).total;
+}
+
+int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                  const float *theta, const void *B, const void *C, const float *D,
+                  const void *lambda, float *h, float *w, void *y, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (d->seqlen != 1) return fail(SSM_ERR_ARG, "ssm_scan_step takes one token (seqlen %lld)",
+                                    (long long)d->seqlen);
+    if (d->batch == 0) return SSM_OK;
+    if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
+    if ((rc = check_ptr(y, "y", d->dtype_io == SSM_BF16 ? 2 : 4))) return rc;
+    if ((rc = check_ptr(h, "h", 4))) return rc;
+    if (d->two_endpoint && (rc = check_ptr(w, "w", 4))) return rc;
+    if (w && (uintptr_t)w % 4) return fail(SSM_ERR_ALIGN, "w is not 4-byte aligned");
+    ssm::Params p;
+    fill_params(d, p);
+    if (!ssm::step_supported(p))
+        return fail(SSM_ERR_UNSUPPORTED, "ssm_scan_step: rank_in %d / rank_out %d above 8",
+                    d->rank_in, d->rank_out);
+    p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
+    p.lam = lambda; p.y = y;
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::scan_step(p, h, w, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_step launch");
+    g_last_error.clear();
+    return SSM_OK;
 }
 
 int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,

@@ -141,3 +141,22 @@ def test_host_tensor_refused():
     torch = pytest.importorskip("torch")
     with pytest.raises(ValueError):
         abi._ptr(torch.zeros(3))
+
+
+def _step_status(lib, d, **ptrs):
+    names = ["x", "dt", "A_log", "theta", "B", "C", "D", "lam", "h", "w", "y"]
+    return lib.ssm_scan_step(ctypes.byref(d), *[ptrs.get(n) for n in names], None)
+
+
+def test_step_argument_checks(lib):
+    full = dict(x=FAKE, dt=FAKE, A_log=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, lam=FAKE,
+                h=FAKE, w=FAKE, y=FAKE)
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=3))
+    assert _step_status(lib, d, **full) == -1          # one token per call
+    assert "one token" in lib.ssm_scan_last_error().decode()
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=1))
+    assert _step_status(lib, d, **dict(full, w=None)) == -1     # two-endpoint needs w
+    assert "w" in lib.ssm_scan_last_error().decode()
+    assert _step_status(lib, d, **dict(full, h=None)) == -1
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=1, rank_in=9, rank_out=9))
+    assert _step_status(lib, d, **full) == -2
