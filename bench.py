@@ -121,11 +121,11 @@ def kernel_bytes(shape, name: str) -> int:
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per batch row of
 # the workload for the largest kernels, from the ncu capture summarised in
-# profiles/chunk_parallel_step_hybridmamba.md (taken at batch 1; the traffic
+# profiles/chunk_parallel_step_hybridmamba.md (taken at batch 2; the traffic
 # is per 64-token chunk, so a launch moves batch x this).  An entry is removed
 # whenever its kernel changes after the capture.
 NCU_TRAFFIC_PER_ROW = {
-    ("hybridmamba", "k_chunk_bwd_fused"): (472.179456 + 121.520896) * 1e6,
+    ("hybridmamba", "k_chunk_bwd_fused"): (944.152320 + 270.234112) * 1e6 / 2,
 }
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)
