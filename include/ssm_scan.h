@@ -230,6 +230,33 @@ SSM_API int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, co
                           const float *theta, const void *B, const void *C, const float *D,
                           const void *lambda, float *h, float *w, void *y, void *stream);
 
+/*
+ * Pre-activations of the scan's step size and two-endpoint weight (the
+ * positivity maps in front of ssm_scan_fwd; the pages give the log-uniform
+ * initialisation of the step, "State Space Models", robocikowo.com; the maps
+ * themselves are the reading the workloads use):
+ *     dt[b][t][h] = softplus(z[b][t][h] + dt_bias[h])
+ *     lambda[b][t][h] = sigmoid(lambda_logit[b][t][h])   (two_endpoint == 1)
+ * z and dt use d's dt layout and strides, lambda_logit and lambda its lambda
+ * layout; all in dtype_io, dt_bias fp32 [nheads].  lambda_logit / lambda may
+ * be NULL when two_endpoint == 0.  The outputs may alias the inputs.
+ * seqlen may be anything (one elementwise pass).
+ */
+SSM_API int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
+                           const void *lambda_logit, void *dt, void *lambda, void *stream);
+
+/*
+ * Gradients through the pre-activations, from ddt and dlambda (as written by
+ * ssm_scan_bwd):  dz = ddt * sigmoid(z + dt_bias),
+ * ddt_bias[h] = sum over (b, t) of dz (fp32, written, fixed summation order),
+ * dlambda_logit = dlambda * lambda (1 - lambda).  dz may alias ddt and
+ * dlambda_logit may alias dlambda; ddt_bias may be NULL; the lambda pointers
+ * may be NULL when two_endpoint == 0.
+ */
+SSM_API int ssm_preact_bwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
+                           const void *lambda_logit, const void *ddt, const void *dlambda,
+                           void *dz, float *ddt_bias, void *dlambda_logit, void *stream);
+
 /* Message describing the last failing call on this host thread ("" if none). */
 SSM_API const char *ssm_scan_last_error(void);
 

@@ -126,3 +126,42 @@ def scan_bwd(shape, inp: dict, dy, lib_path=None) -> dict:
     if s.n_pairs > 0:
         out["dtheta"] = dth
     return out
+
+
+# ---------------------------------------------------------------------------
+# Pre-activations of dt and lambda (fp64).  The pages give the log-uniform
+# initialisation of the step ("State Space Models", robocikowo.com, the entries
+# on the discretisation step); the positivity maps are the reading the
+# workloads use: dt = softplus(z + dt_bias[h]), lambda = sigmoid(logit).
+# Parity pinned by closed forms and central differences in
+# tests/test_preact_pins.py.
+# ---------------------------------------------------------------------------
+def _softplus(x):
+    return np.logaddexp(0.0, x)
+
+
+def _sigmoid(x):
+    # 1 / (1 + e^-x), written with e^-|x| so that neither side loses relative precision
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def preact_fwd(z, dt_bias, lam_logit=None):
+    """dt[b,t,h] = softplus(z[b,t,h] + dt_bias[h]); lam = sigmoid(lam_logit)."""
+    z = np.asarray(z, dtype=np.float64)
+    dt = _softplus(z + np.asarray(dt_bias, dtype=np.float64)[None, None, :])
+    lam = None if lam_logit is None else _sigmoid(np.asarray(lam_logit, dtype=np.float64))
+    return dt, lam
+
+
+def preact_bwd(z, dt_bias, lam_logit, ddt, dlam=None):
+    """Chain rule through preact_fwd: (dz, ddt_bias, dlam_logit)."""
+    x = np.asarray(z, dtype=np.float64) + np.asarray(dt_bias, dtype=np.float64)[None, None, :]
+    dz = np.asarray(ddt, dtype=np.float64) * _sigmoid(x)
+    dbias = dz.sum(axis=(0, 1))
+    dlogit = None
+    if lam_logit is not None and dlam is not None:
+        lam = _sigmoid(np.asarray(lam_logit, dtype=np.float64))
+        dlogit = np.asarray(dlam, dtype=np.float64) * lam * (1.0 - lam)
+    return dz, dbias, dlogit

@@ -25,7 +25,7 @@ EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd"
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
             "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
-            "ssm_scan_step"]
+            "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd"]
 ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -80,6 +80,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_scan_bwd_saved.restype = ctypes.c_int
     lib.ssm_scan_step.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 12
     lib.ssm_scan_step.restype = ctypes.c_int
+    lib.ssm_preact_fwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 6
+    lib.ssm_preact_fwd.restype = ctypes.c_int
+    lib.ssm_preact_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 9
+    lib.ssm_preact_bwd.restype = ctypes.c_int
     lib.ssm_scan_last_error.argtypes = []
     lib.ssm_scan_last_error.restype = ctypes.c_char_p
     lib.ssm_scan_poll_device_error.argtypes = [_vp]
@@ -156,6 +160,22 @@ def ssm_scan_step(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h, w, y, stream
     rc = lib.ssm_scan_step(ctypes.byref(desc), *[_ptr(t) for t in (
         x, dt, A_log, theta, B, C, D, lam, h, w, y)], _stream(stream))
     _check(rc, "ssm_scan_step")
+
+
+def ssm_preact_fwd(desc: Desc, z, dt_bias, lam_logit, dt, lam, stream=None) -> None:
+    """dt = softplus(z + dt_bias[h]); lam = sigmoid(lam_logit) (two-endpoint)."""
+    lib = load_library()
+    rc = lib.ssm_preact_fwd(ctypes.byref(desc), *[_ptr(t) for t in (
+        z, dt_bias, lam_logit, dt, lam)], _stream(stream))
+    _check(rc, "ssm_preact_fwd")
+
+
+def ssm_preact_bwd(desc: Desc, z, dt_bias, lam_logit, ddt, dlam, dz, ddt_bias=None,
+                   dlam_logit=None, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_preact_bwd(ctypes.byref(desc), *[_ptr(t) for t in (
+        z, dt_bias, lam_logit, ddt, dlam, dz, ddt_bias, dlam_logit)], _stream(stream))
+    _check(rc, "ssm_preact_bwd")
 
 
 def ssm_scan_bwd(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, dy, dx, ddt,

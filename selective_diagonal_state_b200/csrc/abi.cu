@@ -24,6 +24,14 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st);
 int chunk_error_take();
 int chunk_rev_error_take();
 bool step_supported(const Params &p);
+struct PreactArgs {
+    const void *z, *lam_logit, *ddt, *dlam;
+    const float *bias;
+    void *dt, *lam, *dz, *dlam_logit;
+    float *dbias;
+};
+cudaError_t preact_forward(const Params &p, const PreactArgs &a, cudaStream_t st);
+cudaError_t preact_backward(const Params &p, const PreactArgs &a, cudaStream_t st);
 cudaError_t scan_step(const Params &p, float *h, float *w, cudaStream_t st);
 }  // namespace ssm
 
@@ -323,6 +331,66 @@ size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
     return bwd_layout(d).total;
+}
+
+int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
+                   const void *lambda_logit, void *dt, void *lambda, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (d->batch == 0 || d->seqlen == 0) return SSM_OK;
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(z, "z", es)) || (rc = check_ptr(dt_bias, "dt_bias", 4)) ||
+        (rc = check_ptr(dt, "dt", es)))
+        return rc;
+    if (d->two_endpoint && ((rc = check_ptr(lambda_logit, "lambda_logit", es)) ||
+                            (rc = check_ptr(lambda, "lambda", es))))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    ssm::PreactArgs a = {};
+    a.z = z; a.bias = dt_bias; a.lam_logit = lambda_logit; a.dt = dt; a.lam = lambda;
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::preact_forward(p, a, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_preact_fwd launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_preact_bwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
+                   const void *lambda_logit, const void *ddt, const void *dlambda, void *dz,
+                   float *ddt_bias, void *dlambda_logit, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (d->batch == 0 || d->seqlen == 0) {
+        if (ddt_bias) {
+            const cudaError_t e = cudaMemsetAsync(ddt_bias, 0, sizeof(float) * d->nheads, st);
+            if (e != cudaSuccess) return cuda_fail(e, "ssm_preact_bwd (empty)");
+        }
+        return SSM_OK;
+    }
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(z, "z", es)) || (rc = check_ptr(dt_bias, "dt_bias", 4)) ||
+        (rc = check_ptr(ddt, "ddt", es)) || (rc = check_ptr(dz, "dz", es)))
+        return rc;
+    if (ddt_bias && (uintptr_t)ddt_bias % 4) return fail(SSM_ERR_ALIGN, "ddt_bias is not 4-byte aligned");
+    if (d->two_endpoint && ((rc = check_ptr(lambda_logit, "lambda_logit", es)) ||
+                            (rc = check_ptr(dlambda, "dlambda", es)) ||
+                            (rc = check_ptr(dlambda_logit, "dlambda_logit", es))))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    ssm::PreactArgs a = {};
+    a.z = z; a.bias = dt_bias; a.lam_logit = lambda_logit; a.ddt = ddt; a.dlam = dlambda;
+    a.dz = dz; a.dbias = ddt_bias; a.dlam_logit = dlambda_logit;
+    profile_begin(st);
+    const cudaError_t e = ssm::preact_backward(p, a, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_preact_bwd launch");
+    g_last_error.clear();
+    return SSM_OK;
 }
 
 int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,

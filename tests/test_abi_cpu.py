@@ -160,3 +160,17 @@ def test_step_argument_checks(lib):
     assert _step_status(lib, d, **dict(full, h=None)) == -1
     d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=1, rank_in=9, rank_out=9))
     assert _step_status(lib, d, **full) == -2
+
+
+def test_preact_argument_checks(lib):
+    d = abi.make_desc(S.WORKLOADS["hybridmamba"].replace(batch=1, seqlen=8))
+    ok = dict(z=FAKE, bias=FAKE, logit=FAKE, dt=FAKE, lam=FAKE)
+    def fwd(**kw):
+        a = dict(ok, **kw)
+        return lib.ssm_preact_fwd(ctypes.byref(d), a["z"], a["bias"], a["logit"], a["dt"], a["lam"], None)
+    assert fwd(z=None) == -1 and "z" in lib.ssm_scan_last_error().decode()
+    assert fwd(bias=None) == -1
+    assert fwd(lam=None) == -1          # two-endpoint shapes need lambda
+    assert fwd(z=FAKE + 1) == -3        # bf16 tensors need 2-byte alignment
+    assert lib.ssm_preact_bwd(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                              None) == -1
