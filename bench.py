@@ -125,7 +125,6 @@ def kernel_bytes(shape, name: str) -> int:
 # is per 64-token chunk, so a launch moves batch x this).  An entry is removed
 # whenever its kernel changes after the capture.
 NCU_TRAFFIC_PER_ROW = {
-    ("hybridmamba", "k_chunk_bwd_fused"): (944.152320 + 270.234112) * 1e6 / 2,
 }
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)

@@ -82,6 +82,11 @@ __device__ __forceinline__ float ld_row1(const unsigned char *tile, int t, int r
     return bf(tile + (r >> 6) * 8192 + off_sw128(t, r & 63));
 }
 
+__device__ __forceinline__ void st_row1(unsigned char *tile, int t, int r, float v) {
+    *reinterpret_cast<__nv_bfloat16 *>(tile + (r >> 6) * 8192 + off_sw128(t, r & 63)) =
+        __float2bfloat16_rn(v);
+}
+
 // 2^x with the hardware approximation (operands are rounded to bf16 afterwards)
 __device__ __forceinline__ float ex2_fast(float x) {
     float y;

@@ -879,12 +879,15 @@ bool chunk_fwd_supported(const Params &p) {
            st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) && chunkc::encode_fn() != nullptr;
 }
 
-// The tensor-core backward additionally reads dy through TMA and writes dx in 16-byte rows.
+// The tensor-core backward additionally reads dy through TMA, writes dx in 16-byte rows and
+// dB / dC through TMA.
 bool chunk_bwd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
+    // dB / dC go out by TMA stores when every group has one head
+    const bool dbc = p.hpg != 1 || (al16(p.dBm) && al16(p.dCm));
     return chunk_fwd_supported(p) && p.dy && al16(p.dy) && st16(p.sy[0]) && st16(p.sy[1]) &&
-           st16(p.sy[2]) && (!p.dx || al16(p.dx));
+           st16(p.sy[2]) && (!p.dx || al16(p.dx)) && dbc;
 }
 
 // Streaming multiprocessors of the current device (grid of the persistent kernels).

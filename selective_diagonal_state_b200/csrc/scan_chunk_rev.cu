@@ -780,6 +780,7 @@ __device__ __forceinline__ uint32_t e_col(int j, int k) {   // k >= j
 __global__ void __launch_bounds__(fuk::THREADS, 1)
 k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
+                  const __grid_constant__ CUtensorMap tmDB, const __grid_constant__ CUtensorMap tmDC,
                   Params p) {
     if (gated_off(p)) return;
     const int nitems = p.nc * p.H * p.Bsz;
@@ -1103,6 +1104,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
         float *cdst = p.ws_dC + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
         const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
+        unsigned char *sBw = sm + fuk::SM_B, *sCw = sm + fuk::SM_C;
         float cum = 0.f, dacc = 0.f, sdt = 0.f;
         {
             float vv[16], ee[16];
@@ -1177,25 +1179,35 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 sdt += dtv;
                 red2[n * fuk::RED_LD + t] = coef * cum;
                 red[n * fuk::RED_LD + t] = tv ? res * bt : 0.f;
-                if (tv) {
-                    if (one_head) {
-                        const int tg = t0 + t;
-                        reinterpret_cast<__nv_bfloat16 *>(p.dBm)[ix_B(p, b, tg, g, 0, n)] =
-                            __float2bfloat16_rn(fmaf(-bn * ct, m2, gg));
-                        reinterpret_cast<__nv_bfloat16 *>(p.dCm)[ix_C(p, b, tg, g, 0, n)] =
-                            __float2bfloat16_rn(dCt);
-                    } else {
-                        gdst[(long long)t * tstride] = res;
-                        cdst[(long long)t * tstride] = dCt;
+                if (one_head) {
+                    // dB / dC replace the (t, n) element of the raw B / C tiles that only this
+                    // thread reads; the tiles go out by TMA stores (rows past L are clipped)
+                    if (valid) {
+                        st_row1(sBw, t, n, fmaf(-bn * ct, m2, gg));
+                        st_row1(sCw, t, n, dCt);
                     }
+                } else if (tv) {
+                    gdst[(long long)t * tstride] = res;
+                    cdst[(long long)t * tstride] = dCt;
                 }
             }
         }
         // later sub-blocks carry into every token of earlier ones
         xch[i * 128 + n] = cum;
+        fence_proxy_async();   // the staged dB / dC tiles are read by TMA stores
         __syncthreads();
-        // every token loop is done with the raw B / C tiles: fetch the next chunk's
-        if (tid == 0 && next < nitems) issue_bc(next);
+        if (tid == 0) {
+            if (one_head) {
+                for (int k = 0; k < nbox; ++k) {
+                    tma_store_4d(&tmDB, sm + fuk::SM_B + k * 8192, 64 * k, g, t0, b);
+                    tma_store_4d(&tmDC, sm + fuk::SM_C + k * 8192, 64 * k, g, t0, b);
+                }
+                bulk_commit();
+            } else if (next < nitems) {
+                // every token loop is done with the raw B / C tiles: fetch the next chunk's
+                issue_bc(next);
+            }
+        }
         float later = 0.f;
         for (int k = i + 1; k < fuk::TQ; ++k) later += xch[k * 128 + n];
         if (later != 0.f) {
@@ -1240,6 +1252,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             part[(fuk::RG + rg) * 64 + t] = s2;
         }
         __syncthreads();
+        if (tid == 0 && one_head) {
+            // the dB / dC stores have read the B / C tiles: fetch the next chunk's
+            bulk_wait_read_all();
+            if (next < nitems) issue_bc(next);
+        }
         if (tid < 64 && t0 + tid < L) {
             const int t = tid;
             float dsig = 0.f, dd = 0.f;
@@ -1278,6 +1295,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         mbar_wait(&bar_in[0], 0, WAIT_LIMIT);
         mbar_wait(&bar_in[1], 0, WAIT_LIMIT);
     }
+    if (tid == 0) bulk_wait_read_all();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -1345,7 +1363,13 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     {
         const long long nitems = (long long)p.nc * p.H * p.Bsz;
         const int pgrid = (int)(nitems < sm_count() ? nitems : sm_count());
-        k_chunk_bwd_fused<<<pgrid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, p);
+        // dB / dC leave the fused kernel by TMA stores when every group has one head
+        CUtensorMap mdb = mb, mdc = mc;
+        if (p.hpg == 1 &&
+            (!make_map(&mdb, p.dBm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
+             !make_map(&mdc, p.dCm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true)))
+            return cudaErrorInvalidValue;
+        k_chunk_bwd_fused<<<pgrid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, mdb, mdc, p);
     }
     profile_mark(st, "k_chunk_bwd_fused");
     return cudaGetLastError();
