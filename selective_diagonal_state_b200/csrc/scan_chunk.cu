@@ -404,7 +404,8 @@ __device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int
 
 __global__ void __launch_bounds__(fwk::THREADS, 1)
 k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-            const __grid_constant__ CUtensorMap tmC, Params p) {
+            const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+            Params p) {
     if (gated_off(p)) return;
     const int BH = p.Bsz * p.H;
     const int nitems = p.nc * BH;
@@ -498,6 +499,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             ce[2 * tid] = f32[F_KRE + fslot(0, 4) * NP + tid];
             ce[2 * tid + 1] = f32[F_KIM + fslot(0, 4) * NP + tid];
         }
+        // the previous chunk's y store has to have read the P region (corr partials below)
+        if (tid == 0) bulk_wait_read_all();
         int ok = (mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) &&
                   mbar_wait(bar_bc, (uint32_t)(k & 1), WAIT_LIMIT)) ? 1 : 0;
         if (!ok) raise_error(1);
@@ -789,34 +792,37 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             aborted = true;
             break;
         }
-        // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p] -----------------------
+        // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p], staged in the P tiles'
+        // place (phase B is done with them) and written by one TMA store --------
         {
             const int qd = warp & 3, part = warp >> 2;   // TMEM quarter, column block
             const int pp = 16 * qd + (lane & 15);
-            __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + b * p.sy[0] +
-                                  h * p.sy[2] + pp;
+            unsigned char *ys = sm + fwk::SM_P;
             constexpr int CPW = 64 / (fwk::THREADS / 128);
             for (int c16 = 0; c16 < CPW / 16; ++c16) {
                 float v[16];
                 const int tc = CPW * part + 16 * c16;
                 tmem_ld16(tmem_addr(t_y, 32u * qd, (uint32_t)tc), v);
                 if (lane < 16) {
-                    __nv_bfloat16 *yp = yrow + (long long)(t0 + tc) * p.sy[1];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = tc + j;
-                        if (t0 + t < L) {
-                            const float u = bf(sX + off_sw128(t, pp));
-                            *yp = __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
-                        }
-                        yp += p.sy[1];
+                        const float u = bf(sX + off_sw128(t, pp));
+                        *reinterpret_cast<__nv_bfloat16 *>(ys + off_sw128(t, pp)) =
+                            __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
                     }
                 }
             }
         }
+        fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        if (tid == 0) {   // tokens past the sequence end are clipped by the store
+            tma_store_4d(&tmY, sm + fwk::SM_P, 0, h, t0, b);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_read_all();
     if (aborted && tid == 0) {
         // let loads still in flight land before the CTA's shared memory goes away
         mbar_wait(&bar_x[0], 0, WAIT_LIMIT);
@@ -873,7 +879,9 @@ cudaError_t chunk_range_check(const Params &p, int *gate, cudaStream_t st) {
 bool chunk_fwd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
-    return p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 && (p.N == 64 || p.N == 128) &&
+    // y (forward) leaves by TMA stores
+    const bool yok = !p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]));
+    return yok && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 && (p.N == 64 || p.N == 128) &&
            p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
            st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) && st16(p.sB[2]) &&
            st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) && chunkc::encode_fn() != nullptr;
@@ -947,7 +955,10 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         return e;
     const long long nitems = (long long)p.nc * p.H * p.Bsz;
     const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
-    k_chunk_fwd<<<grid, fwk::THREADS, fwk::SMEM_BYTES, st>>>(mx, mb, mc, p);
+    CUtensorMap my;
+    if (!make_map(&my, p.y, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
+        return cudaErrorInvalidValue;
+    k_chunk_fwd<<<grid, fwk::THREADS, fwk::SMEM_BYTES, st>>>(mx, mb, mc, my, p);
     profile_mark(st, "k_chunk_fwd");
     return cudaGetLastError();
 }
