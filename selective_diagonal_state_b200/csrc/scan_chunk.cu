@@ -256,7 +256,13 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
         }
     }
     s_ce[0][tid] = __ldg(p.ws_ce + bhc(p, b, h, 0) * (2 * NP) + tid);
+    // the two chunks after this one stream into L2 while this one is processed
+    constexpr int PF = 2;
+    for (int k = 1; k <= PF && k < nc; ++k)
+        if (tid == 0) bulk_prefetch_l2(p.ws_kp + bhc(p, b, h, k) * SLOT_FLOATS, SLOT_FLOATS * 4);
     for (int c = 0; c < nc; ++c) {
+        if (tid == 0 && c + PF + 1 < nc)
+            bulk_prefetch_l2(p.ws_kp + bhc(p, b, h, c + PF + 1) * SLOT_FLOATS, SLOT_FLOATS * 4);
         float *slot = p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS;
         Rows2x8 sv[pas::KMAX];
 #pragma unroll

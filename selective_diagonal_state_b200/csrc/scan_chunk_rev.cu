@@ -219,7 +219,18 @@ __global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
         for (int j = 0; j < 8; ++j) g[k].a[j] = g[k].d[j] = 0.f;
     s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
 
+    // the two chunks after this one stream into L2 while this one is processed
+    constexpr int PF = 2;
+    auto prefetch = [&](int cc) {
+        if (tid == 0 && cc >= 0) {
+            bulk_prefetch_l2(p.ws_gc + bhc(p, b, h, cc) * SLOT_FLOATS, SLOT_FLOATS * 4);
+            if (cc > 0 && p.ws_qb)
+                bulk_prefetch_l2(p.ws_kp + bhc(p, b, h, cc) * SLOT_FLOATS, 2 * TILE_BYTES);
+        }
+    };
+    for (int k = 1; k <= PF; ++k) prefetch(nc - 1 - k);
     for (int c = nc - 1; c >= 0; --c) {
+        prefetch(c - PF - 1);
         float *slot = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS;
         // K_end_{c-1}: the state entering chunk c (tile format)
         const unsigned char *kb = (c > 0 && p.ws_qb)
