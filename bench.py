@@ -105,8 +105,6 @@ def kernel_bytes(shape, name: str) -> int:
     # tensor-core chain: path inputs read, path outputs written
     if name == "k_chunk_state_local":  # x, B, dt, lambda (chunk states go to workspace)
         return t["x"] + t["B"] + t["dt"] + t["lam"]
-    if name == "k_chunk_adj_local":   # C, dt, dy
-        return t["C"] + t["dt"] + dy
     if name == "k_chunk_bwd_dx":      # B, C, dt, lambda, dy -> dx
         return t["B"] + t["C"] + t["dt"] + t["lam"] + dy + t["x"]
     if name == "k_chunk_bwd_dx_saved":  # dy -> dx (the rest comes from the forward's workspace)

@@ -182,7 +182,7 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
 
 struct BwdWs {
     size_t off_dC, off_gbu, off_tok, off_M2, off_par, off_ddt, off_blk, off_blkc, off_kp, off_qb,
-        off_gc, off_ce, total;
+        off_gc, off_ce, off_ring, off_flag, total;
     bool boundary;  // chunk-boundary carries (tensor-core backward shapes)
 };
 
@@ -257,7 +257,7 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
     w.off_blkc = off;
     off = align256(off + (size_t)d->batch * d->nheads * ntb * 4);
     w.boundary = tensor_chain_shape(d);
-    w.off_kp = w.off_qb = w.off_gc = w.off_ce = off;
+    w.off_kp = w.off_qb = w.off_gc = w.off_ce = w.off_ring = w.off_flag = off;
     if (w.boundary) {
         w.off_kp = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * d->headdim * 4);
@@ -267,6 +267,11 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * d->headdim * 4);
         w.off_ce = off;
         off = align256(off + (size_t)d->batch * d->nheads * ntb * 128 * 2 * 4);
+        // the adjoint carried between chunks: two fp32 slots and a counter per (b, h)
+        w.off_ring = off;
+        off = align256(off + 2 * (size_t)d->batch * d->nheads * 128 * d->headdim * 4);
+        w.off_flag = off;
+        off = align256(off + (size_t)d->batch * d->nheads * 4);
     }
     w.total = off;
     return w;
@@ -582,6 +587,8 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
         pc.ws_qb = (float *)(ws + lay.off_qb);
         pc.ws_gc = (float *)(ws + lay.off_gc);
         pc.ws_ce = (float *)(ws + lay.off_ce);
+        pc.ws_ring = (float *)(ws + lay.off_ring);
+        pc.ws_flag = (int *)(ws + lay.off_flag);
         if (saved) {
             // read-only here: the forward wrote them
             const FwdWs fl = fwd_layout(d);

@@ -327,10 +327,11 @@ __device__ __forceinline__ ChunkItem chunk_item(const Params &p, int item) {
 }
 
 // ---- chunks chained through a carry in global memory ---------------------------
-// A persistent kernel walks the chunks of every (b, h) in order, chunk slowest.
-// The item of chunk c reads the fp32 carry from slot c & 1 once the counter of
-// (b, h) reaches c, writes the next carry to slot (c + 1) & 1 and sets the
-// counter to c + 1.
+// A persistent kernel walks the chunks of every (b, h) in order (forward) or in
+// reverse (backward), chunk slowest.  The item of the r-th chunk of a (b, h) in
+// walking order reads the fp32 carry from slot r & 1 once the counter of
+// (b, h) reaches r, writes the next carry to slot (r + 1) & 1 and sets the
+// counter to r + 1.
 constexpr long long FLAG_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
 
 // item -> (chunk, head, batch row), chunk slowest
@@ -363,6 +364,14 @@ __device__ __forceinline__ bool wait_count(const int *flag, int target) {
 __device__ __forceinline__ void publish_count(int *flag, int v) {
     __threadfence();
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+// item -> (chunk, head, batch row), chunk slowest, last chunk first (the walk of
+// the backward, whose carry runs from the end of the sequence)
+__device__ __forceinline__ ChunkItem chunk_item_rcs(const Params &p, int item) {
+    ChunkItem r = chunk_item_cs(p, item);
+    r.c = p.nc - 1 - r.c;
+    return r;
 }
 
 // ---- host side ---------------------------------------------------------------

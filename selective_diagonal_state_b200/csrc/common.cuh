@@ -40,13 +40,13 @@ struct Params {
     // chunk states and exact decay-gradient carries at 64-token chunk boundaries
     // (tensor-core chain; the forward uses ws_kp and ws_ce):
     float *ws_kp;   // [B][H][NC] 32 KB: pre-state K entering every chunk (K_{-1} = h0 + beta_0 w0)
-    float *ws_qb;   // [B][H][NC][4][N]  per-row sum_p conj(Gbar) A K_prev at chunk starts (per warp of p)
-    float *ws_gc;   // [B][H][NC][N][P]  chunk-local adjoint, then the adjoint carried into each chunk
+    float *ws_qb;   // [B][H][NC][4][N]  per-row sum_p conj(Gbar) A K_prev at chunk starts (4 partials over p)
+    float *ws_gc;   // [B][H][NC] 32 KB: the adjoint carried into each chunk (hi / lo tiles)
     float *ws_ce;   // [B][H][NC][128][2] full-chunk decay e^{lam S_63} per mode (re, im)
     // forward chain: fp32 state carried from chunk c to c + 1 through two slots per
     // (b, h), and the count of chunks of (b, h) whose outgoing state is in place
     float *ws_ring; // [2][B][H][4][4][128][4] carry slots (row-contiguous per 4 columns)
-    int *ws_flag;   // [B][H]
+    int *ws_flag;   // [B][H]           (the backward carries its adjoint the same way)
     int nc;         // number of 64-token chunks
     // device-side choice between two launched kernel chains: a kernel runs
     // only when (*gate != 0) == gate_on (no gate: always)

@@ -10,16 +10,17 @@
 // the chunk's last token, before that token's own readout term):
 //   Gbar_t = sum_{t' >= t} conj(e^{lam (S_t' - S_t)}) c_t' dy_t'  +  conj(e^{lam (S_63 - S_t)}) Gc
 // so the work splits into
-//   k_chunk_adj_local  (every chunk at once)   Ghat_c = sum_t conj(e^{lam S_t}) c_t dy_t^T
-//   k_chunk_adj_pass   (chunks in reverse)     Gc_{c-1} = conj(e^{lam S_63}) Gc_c + Ghat_c
+//   k_chunk_bwd_fused  (persistent, the chunks of every (b, h) last to first, chained
+//                       through an fp32 carry in L2): the chunk-local adjoint
+//                       Ghat_c = sum_t conj(e^{lam S_t}) c_t dy_t^T, the carry step
+//                       Gc_{c-1} = conj(e^{lam S_63}) Gc_c + Ghat_c, and dC_t and
+//                       gbu_t = sum_p u_t,p Gbar_t,p, then the decay-gradient sums of the chunk
 //   k_chunk_bwd_dx     (every chunk at once)   dx_s = sum_{t>=s} P_ts dy_t + (Bh_s)^T Gc_c + corr
-//   k_chunk_bwd_fused  (every chunk at once)   dC_t and gbu_t = sum_p u_t,p Gbar_t,p, then the
-//                                              decay-gradient sums of the chunk
 // where P is the masked score matrix of the forward and Bh_s = sigma_s b_s
 // e^{lam (S_63 - S_s)} (the same folded operands as the chunked forward).  The
-// passing kernel also forms, at every chunk start, the exact boundary value
+// fused kernel also forms, at every chunk start, the exact boundary value
 // sum_p conj(Gc_{c-1}) K_end_{c-1} of the decay-gradient scan, and writes
-// dL/dh0, dL/dw0 and dL/dbeta_0 after the first chunk.
+// dL/dh0, dL/dw0 and dL/dbeta_0 at the first chunk.
 #include <cuda.h>
 
 #include "chunk_common.cuh"
@@ -38,309 +39,6 @@ namespace chunkrev {
 using namespace umma;
 using namespace chunkc;
 
-
-// ============================================================================
-// k_chunk_adj_local: Ghat_c = Ch^T (N x 64 t) . dY (64 t x 64 p), per chunk.
-//   Ch_t = c_t conj(e^{lam S_t}) = Ci_t G_i (sub-block-relative fold times the
-//   sub-block's start factor), split into bf16 hi + lo.
-// ============================================================================
-namespace loc {
-constexpr int THREADS = 256;
-constexpr int RG = THREADS / 64;   // row groups of the operand preparation
-constexpr uint32_t TMEM_COLS = 64;
-constexpr uint32_t SM_C = 0;        // 16 KB  raw C (two 64-row 128B-swizzled halves)
-constexpr uint32_t SM_DY = 16384;   // 8 KB   dy (128B swizzle)
-constexpr uint32_t SM_CH = 24576;   // 16 KB  Ch hi, K-major (rows t, K = state rows)
-constexpr uint32_t SM_CHL = 40960;  // 16 KB  Ch lo
-constexpr uint32_t SM_F32 = 57344;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
-}  // namespace loc
-
-__global__ void __launch_bounds__(loc::THREADS)
-k_chunk_adj_local(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
-                  Params p) {
-    if (gated_off(p)) return;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *f32 = reinterpret_cast<float *>(sm + loc::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + loc::SM_BAR);
-    uint64_t *bar_mma = bar_tma + 1;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 2);
-
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / p.hpg;
-    const int N = p.N, nr = p.nr;
-    const int t0 = c * Q;
-    const int nbox = N / 64;
-
-    if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
-        mbar_fence_init();
-        tma_prefetch_desc(&tmC);
-        tma_prefetch_desc(&tmDY);
-        mbar_expect_tx(bar_tma, (uint32_t)(Q * PD * 2 + Q * N * 2));
-        tma_load_4d(sm + loc::SM_DY, &tmDY, bar_tma, 0, h, t0, b);
-        for (int k = 0; k < nbox; ++k)
-            tma_load_4d(sm + loc::SM_C + k * 8192, &tmC, bar_tma, 64 * k, g, t0, b);
-    }
-    if (warp == 0) tmem_alloc(tslot, loc::TMEM_COLS);
-    mode_rates(p, f32, h);
-    if (N < NP)  // K padding of the Ch tiles
-        for (int i = tid; i < (int)(32768 / 16); i += loc::THREADS)
-            reinterpret_cast<uint4 *>(sm + loc::SM_CH)[i] = make_uint4(0, 0, 0, 0);
-    chunk_tokens(p, f32, b, h, t0, false);
-    chunk_mode_constants(p, f32);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tacc = *tslot;
-    int ok = mbar_wait(bar_tma, 0, WAIT_LIMIT) ? 1 : 0;
-    if (!ok) rev_raise_error(1);
-    if (__syncthreads_and(ok)) {
-        // Ch tiles: thread (t, grp) handles rows 8 * (grp + RG k)
-        const int t = tid & 63, grp = tid >> 6;
-        const int ib = t >> 4;
-        const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
-        const float ds = f32[F_S + t] - Sb;
-        const unsigned char *sC = sm + loc::SM_C;
-#pragma unroll 1
-        for (int k = 0; k < NP / (8 * loc::RG); ++k) {
-            const int r0 = 8 * (grp + loc::RG * k);
-            if (r0 >= N) break;
-            float rc[8], v[8];
-            ld_rows8(sC, t, r0, rc);
-#pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-                const int r = r0 + j;
-                if (r < nr) {
-                    const float g0 = ib ? f32[F_KRE + gslot(ib) * NP + r] : 1.f;
-                    const float g1 = ib ? f32[F_KRE + gslot(ib) * NP + r + 1] : 1.f;
-                    v[j] = rc[j] * ex2_fast(f32[F_A2 + r] * ds) * g0;
-                    v[j + 1] = rc[j + 1] * ex2_fast(f32[F_A2 + r + 1] * ds) * g1;
-                } else {
-                    const int m = nr + ((r - nr) >> 1);
-                    float sn, cs;
-                    __sincosf(f32[F_W + m] * ds, &sn, &cs);
-                    const float ec = ex2_fast(f32[F_A2 + m] * ds);
-                    const float ci0 = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
-                    const float ci1 = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
-                    float gr = 1.f, gi = 0.f;
-                    if (ib) {
-                        gr = f32[F_KRE + gslot(ib) * NP + m];
-                        gi = f32[F_KIM + gslot(ib) * NP + m];
-                    }
-                    cmul(ci0, ci1, gr, gi, v[j], v[j + 1]);
-                }
-            }
-            st16_split(sm + loc::SM_CH, sm + loc::SM_CHL, off_kmaj(t, r0, KM_LBO, KM_SBO), v);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t dy_base = smem_u32(sm + loc::SM_DY);
-            const uint32_t id = idesc_bf16(128, 64, true, true);
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t ch_base = smem_u32(sm + (part ? loc::SM_CHL : loc::SM_CH));
-                for (int s = 0; s < Q / 16; ++s)
-                    mma_bf16(tacc, sdesc(ch_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                             sdesc(dy_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id,
-                             part > 0 || s > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        ok = mbar_wait(bar_mma, 0, WAIT_LIMIT) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
-        fence_after_sync();
-        if (__syncthreads_and(ok)) {
-            // the chunk-local fp32 sum [N][64] at the start of the chunk's slot
-            const int n = 32 * (warp & 3) + (tid & 31), half = warp >> 2;
-            float *dst = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS + n * PD;
-#pragma unroll
-            for (int c16 = 2 * half; c16 < 2 * half + 2; ++c16) {
-                float v[16];
-                tmem_ld16(tmem_addr(tacc, 32u * (warp & 3), 16u * c16), v);
-                if (n < N) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        reinterpret_cast<float4 *>(dst + 16 * c16)[q4] =
-                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                }
-            }
-        }
-    } else if (tid == 0) {
-        mbar_wait(bar_tma, 0, WAIT_LIMIT);  // let an in-flight load land before exit
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        fence_after_sync();
-        tmem_dealloc(tacc, loc::TMEM_COLS);
-    }
-}
-
-// ============================================================================
-// k_chunk_adj_pass: reverse pass over the chunks of one (batch row, head).
-// Thread (row-pair group, 8 consecutive p) keeps rows 2rp, 2rp+1 of the adjoint
-// carry for rp = rp0, rp0 + 32: two real modes, or one rotation pair as
-// (re, im).  Every chunk's loads are issued together, in 16-byte pieces.
-// ws_gc[c] holds Ghat_c (fp32) on entry and the carry into chunk c (hi / lo
-// tiles) on exit.
-// ============================================================================
-namespace pass {
-constexpr int THREADS = 256;
-constexpr int KMAX = NP / 64;   // row pairs per thread
-}  // namespace pass
-
-__device__ __forceinline__ float sum8(float v) {
-#pragma unroll
-    for (int o = 4; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-__global__ void __launch_bounds__(pass::THREADS) k_chunk_adj_pass(Params p) {
-    if (gated_off(p)) return;
-    __shared__ float s_ce[3][2 * NP];   // chunk decays, triple-buffered
-    __shared__ float red[pass::THREADS];
-    const int tid = threadIdx.x;
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int N = p.N, nr = p.nr, nc = p.nc;
-    const int p8 = 8 * (tid & 7), rp0 = tid >> 3;
-    const int nk = N / 64;
-    Rows2x8 g[pass::KMAX];
-#pragma unroll
-    for (int k = 0; k < pass::KMAX; ++k)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) g[k].a[j] = g[k].d[j] = 0.f;
-    s_ce[(nc - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, nc - 1) * (2 * NP) + tid);
-
-    // the two chunks after this one stream into L2 while this one is processed
-    constexpr int PF = 2;
-    auto prefetch = [&](int cc) {
-        if (tid == 0 && cc >= 0) {
-            bulk_prefetch_l2(p.ws_gc + bhc(p, b, h, cc) * SLOT_FLOATS, SLOT_FLOATS * 4);
-            if (cc > 0 && p.ws_qb)
-                bulk_prefetch_l2(p.ws_kp + bhc(p, b, h, cc) * SLOT_FLOATS, 2 * TILE_BYTES);
-        }
-    };
-    for (int k = 1; k <= PF; ++k) prefetch(nc - 1 - k);
-    for (int c = nc - 1; c >= 0; --c) {
-        prefetch(c - PF - 1);
-        float *slot = p.ws_gc + bhc(p, b, h, c) * SLOT_FLOATS;
-        // K_end_{c-1}: the state entering chunk c (tile format)
-        const unsigned char *kb = (c > 0 && p.ws_qb)
-            ? reinterpret_cast<const unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
-            : nullptr;
-        Rows2x8 hv[pass::KMAX], kv[pass::KMAX];
-#pragma unroll
-        for (int k = 0; k < pass::KMAX; ++k) {
-            if (k < nk) {
-                const int n0 = 2 * (rp0 + 32 * k);
-                rows_load_f32(slot, n0, p8, hv[k]);
-                if (kb) rows_load_tile(kb, n0, p8, kv[k]);
-            }
-        }
-        if (c > 0) s_ce[(c - 1) % 3][tid] = __ldg(p.ws_ce + bhc(p, b, h, c - 1) * (2 * NP) + tid);
-        // every thread has read its part of Ghat_c: the slot can take the carry into chunk c
-        __syncthreads();
-        const float *ce = s_ce[c % 3];
-        float *qb = p.ws_qb ? p.ws_qb + bhc(p, b, h, c) * 4 * (long long)N : nullptr;
-        unsigned char *tile = reinterpret_cast<unsigned char *>(slot);
-#pragma unroll
-        for (int k = 0; k < pass::KMAX; ++k) {
-            const int n0 = 2 * (rp0 + 32 * k);
-            if (k >= nk) {   // rows past N read as zero by the consumers
-                Rows2x8 z;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) z.a[j] = z.d[j] = 0.f;
-                rows_store_tile(tile, n0, p8, z);
-                continue;
-            }
-            // the carry into chunk c (tile format), then Gc_{c-1} = conj(E_c) Gc_c + Ghat_c
-            rows_store_tile(tile, n0, p8, g[k]);
-            float *a = g[k].a, *d = g[k].d;
-            if (n0 < nr) {
-                const float e0 = ce[2 * n0], e1 = ce[2 * (n0 + 1)];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    a[j] = fmaf(e0, a[j], hv[k].a[j]);
-                    d[j] = fmaf(e1, d[j], hv[k].d[j]);
-                }
-            } else {
-                const int m = nr + ((n0 - nr) >> 1);
-                const float er = ce[2 * m], ei = ce[2 * m + 1];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {   // conj(er + i ei) (a + i d) + Ghat
-                    const float ao = a[j];
-                    a[j] = fmaf(er, ao, fmaf(ei, d[j], hv[k].a[j]));
-                    d[j] = fmaf(er, d[j], fmaf(-ei, ao, hv[k].d[j]));
-                }
-            }
-            if (kb) {
-                // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1}; 8 lanes hold one row pair
-                float aa = 0.f, dd = 0.f, ad = 0.f, da = 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    aa = fmaf(a[j], kv[k].a[j], aa);
-                    dd = fmaf(d[j], kv[k].d[j], dd);
-                    ad = fmaf(a[j], kv[k].d[j], ad);
-                    da = fmaf(d[j], kv[k].a[j], da);
-                }
-                float q0, q1;
-                if (n0 < nr) {
-                    q0 = aa;
-                    q1 = dd;
-                } else {
-                    q0 = aa + dd;
-                    q1 = ad - da;
-                }
-                q0 = sum8(q0);
-                q1 = sum8(q1);
-                if ((tid & 7) == 0) {
-                    qb[n0] = q0;            // slot 0 holds the whole sum over p
-                    qb[n0 + 1] = q1;
-                    qb[N + n0] = 0.f;       // slot 1 (read by the carry pass) stays zero
-                    qb[N + n0 + 1] = 0.f;
-                }
-            }
-        }
-    }
-    // carry out of the first chunk = dL/dK_{-1}: dh0, dw0 = beta_0 dh0, dbeta_0 = <dh0, w0>
-    float beta0 = 0.f;
-    if (p.two_ep)
-        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
-    float db0 = 0.f;
-#pragma unroll
-    for (int k = 0; k < pass::KMAX; ++k) {
-        if (k >= nk) break;
-        const int n0 = 2 * (rp0 + 32 * k);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const long long i0 = ix_st(p, b, h, n0, p8 + j), i1 = ix_st(p, b, h, n0 + 1, p8 + j);
-            if (p.dh0) {
-                p.dh0[i0] = g[k].a[j];
-                p.dh0[i1] = g[k].d[j];
-            }
-            if (p.dw0) {
-                p.dw0[i0] = beta0 * g[k].a[j];
-                p.dw0[i1] = beta0 * g[k].d[j];
-            }
-            if (p.w0) db0 = fmaf(g[k].a[j], p.w0[i0], fmaf(g[k].d[j], p.w0[i1], db0));
-        }
-    }
-    red[tid] = db0;
-    __syncthreads();
-    if (tid == 0) {
-        float acc = 0.f;
-        for (int k = 0; k < pass::THREADS; ++k) acc += red[k];
-        p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1] = acc;
-    }
-}
 
 // ============================================================================
 // k_chunk_bwd_dx: per chunk,
@@ -801,26 +499,25 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + fuk::SM_F32);
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);   // [2]: x/dy/states, B/C
-    uint64_t *bar_mma = bar_in + 2;                                      // [2]
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 4);
+    uint64_t *bar_mma = bar_in + 2;                                      // [3] phases A, B, C
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 5);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
     const int nbox = N / 64;
     // the next chunk's inputs go into regions as soon as this chunk is done with them:
-    // x, dy and the state tiles after phase A, B and C after the unfold's token loop
+    // x, dy and the entering state after phase C, B and C after the unfold's token loop
     auto issue_xs = [&](int item) {
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_rcs(p, item);
         const int t0_ = it.c * Q;
         const long long u_ = bhc(p, it.b, it.h, it.c);
-        mbar_expect_tx(&bar_in[0], (uint32_t)(2 * Q * PD * 2) + 4 * TILE_BYTES);
+        mbar_expect_tx(&bar_in[0], (uint32_t)(2 * Q * PD * 2) + 2 * TILE_BYTES);
         tma_load_4d(sm + fuk::SM_X, &tmX, &bar_in[0], 0, it.h, t0_, it.b);
         tma_load_4d(sm + fuk::SM_DY, &tmDY, &bar_in[0], 0, it.h, t0_, it.b);
         bulk_load(sm + fuk::SM_KT, p.ws_kp + u_ * SLOT_FLOATS, 2 * TILE_BYTES, &bar_in[0]);
-        bulk_load(sm + fuk::SM_GC, p.ws_gc + u_ * SLOT_FLOATS, 2 * TILE_BYTES, &bar_in[0]);
     };
     auto issue_bc = [&](int item) {
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_rcs(p, item);
         const int t0_ = it.c * Q, g_ = it.h / p.hpg;
         mbar_expect_tx(&bar_in[1], (uint32_t)(2 * Q * N * 2));
         for (int k = 0; k < nbox; ++k) {
@@ -833,8 +530,9 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     if (tid == 0) {
         mbar_init(&bar_in[0], 1);
         mbar_init(&bar_in[1], 1);
-        mbar_init(&bar_mma[0], 2);   // two issuing threads commit each phase
-        mbar_init(&bar_mma[1], 2);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 2);   // two issuing threads commit phase B
+        mbar_init(&bar_mma[2], 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
@@ -847,7 +545,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     TokPrefetch tok;
     ModePrefetch mp;
     {
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_rcs(p, item);
         tok = tok_load(p, it.b, it.h, it.c * Q);
         mp = mode_load(p, it.h);
     }
@@ -856,20 +554,22 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_v = tbase, t_v2 = tbase + 64u, t_g = tbase + 128u;
+    const int cn = 32 * (warp & 3) + lane, ccq = warp >> 2;   // chain step: row, 16-column block
     bool aborted = false;
 
     for (int kit = 0; item < nitems; ++kit, item += gridDim.x) {
-        const ChunkItem it = chunk_item(p, item);
+        const ChunkItem it = chunk_item_rcs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int g = h / p.hpg;
         const int t0 = c * Q;
         const long long u = bhc(p, b, h, c);
+        const int bh = b * p.H + h, rr = p.nc - 1 - c;   // chunks of (b, h) walked before this one
         const int next = item + gridDim.x;
         const uint32_t par = (uint32_t)(kit & 1);
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
         if (next < nitems) {
-            const ChunkItem nx = chunk_item(p, next);
+            const ChunkItem nx = chunk_item_rcs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
             mp = mode_load(p, nx.h);
         }
@@ -931,33 +631,22 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         fence_before_sync();
         __syncthreads();
 
-        // ---- phase A: V = K_prev dY^T, V2 = Gc X^T (hi + lo), G = dY X^T ---------
-        // (two threads in different warps issue the independent accumulators)
-        if (tid == 0 || tid == 32) {
+        // ---- phase A: V = K_prev dY^T (hi + lo), G = dY X^T ---------------------
+        if (tid == 0) {
             fence_after_sync();
             const uint32_t x_base = smem_u32(sm + fuk::SM_X), dy_base = smem_u32(sm + fuk::SM_DY);
             const uint32_t id_v = idesc_bf16(128, 64, false, false);
-            if (tid == 0) {
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t kt_base = smem_u32(sm + (part ? fuk::SM_KTL : fuk::SM_KT));
-                    for (int s = 0; s < PD / 16; ++s)
-                        mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                                 sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                                 part > 0 || s > 0);
-                }
-                const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t kt_base = smem_u32(sm + (part ? fuk::SM_KTL : fuk::SM_KT));
                 for (int s = 0; s < PD / 16; ++s)
-                    mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                             sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
-            } else {
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t gc_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
-                    for (int s = 0; s < PD / 16; ++s)
-                        mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
-                                 sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
-                                 part > 0 || s > 0);
-                }
+                    mma_bf16(t_v, sdesc(kt_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
             }
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            for (int s = 0; s < PD / 16; ++s)
+                mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
             mma_commit(&bar_mma[0]);
         }
         if (tid < 64) {
@@ -974,11 +663,9 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             aborted = true;
             break;
         }
-        // phase A has read x, dy and the state tiles: fetch the next chunk's
-        if (tid == 0 && next < nitems) issue_xs(next);
-        // ---- masked G (s <= t) -> four 16-row tiles (rows t, K = s); dy_t . u_t
-        if (warp >= 4 && warp < 12) {   // two warps per TMEM lane quarter, two blocks each
-            const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);
+        if (warp >= 4 && warp < 12) {
+            // ---- masked G (s <= t) -> four 16-row tiles (rows t, K = s); dy_t . u_t
+            const int qd = warp & 3, i0 = 2 * ((warp - 4) >> 2);   // two warps per lane quarter
             for (int i = i0; i < i0 + 2; ++i) {
                 float v[16];
                 tmem_ld16(tmem_addr(t_g, 32u * qd, 16u * i), v);
@@ -1003,12 +690,53 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     }
                 }
             }
+        } else {
+            // ---- Ch_t = c_t conj(e^{lam S_t}) = Cm_t conj(F[0][k+1]) (t in sub-block k),
+            // hi + lo, into the Gc tiles' place (the carried adjoint arrives later)
+            const int th = (warp < 4 ? warp : warp - 8) * 32 + lane;
+            for (int pc = th; pc < 64 * (N / 8); pc += 256) {
+                const int t = pc & 63, r0 = 8 * (pc >> 6), kb = t >> 4;
+                const uint32_t off = off_kmaj(t, r0, KM_LBO, KM_SBO);
+                const uint4 hq = *reinterpret_cast<const uint4 *>(sm + fuk::SM_CM + off);
+                const uint4 lq = *reinterpret_cast<const uint4 *>(sm + fuk::SM_CML + off);
+                const uint32_t hw[4] = {hq.x, hq.y, hq.z, hq.w}, lw[4] = {lq.x, lq.y, lq.z, lq.w};
+                const float *fre = f32 + F_KRE + fslot(0, kb + 1) * NP;
+                const float *fim = f32 + F_KIM + fslot(0, kb + 1) * NP;
+                float v[8];
+#pragma unroll
+                for (int w2 = 0; w2 < 4; ++w2) {
+                    const float2 a2_ = bf2_to_f2(hw[w2]), l2_ = bf2_to_f2(lw[w2]);
+                    const float a = a2_.x + l2_.x, d = a2_.y + l2_.y;   // rows r0 + 2 w2, + 1
+                    const int r = r0 + 2 * w2;
+                    if (r < nr) {
+                        v[2 * w2] = a * fre[r];
+                        v[2 * w2 + 1] = d * fre[r + 1];
+                    } else {   // (a + i d) conj(fr + i fi)
+                        const int m = nr + ((r - nr) >> 1);
+                        v[2 * w2] = fmaf(a, fre[m], d * fim[m]);
+                        v[2 * w2 + 1] = fmaf(d, fre[m], -a * fim[m]);
+                    }
+                }
+                st16_split(sm + fuk::SM_GC, sm + fuk::SM_GCL, off, v);
+            }
         }
+        // the adjoint carried into this chunk is published by the item of chunk c + 1
+        if (tid == 0 && rr > 0 && !wait_count(p.ws_flag + bh, rr)) rev_raise_error(2);
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();
+        __syncthreads();   // also orders the wait before every thread's loads of Gc_c
+        float gcv[16];     // Gc_c of row cn, columns 16 ccq ..; in flight during phase B
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+            float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (rr > 0 && cn < N) a4 = __ldcg(carry_ptr(p, rr & 1, bh, ccq, cn) + j4 * NP);
+            gcv[4 * j4] = a4.x;
+            gcv[4 * j4 + 1] = a4.y;
+            gcv[4 * j4 + 2] = a4.z;
+            gcv[4 * j4 + 3] = a4.w;
+        }
 
-        // ---- phase B: D_{i,k} and E_{j,k}, hi*hi + hi*lo + lo*hi ---------------
+        // ---- phase B: D_{i,k}, E_{j,k} (hi*hi + hi*lo + lo*hi), Ghat = Ch^T dY ------
         if (tid == 0) {
             fence_after_sync();
             const uint32_t id_d = idesc_bf16(128, 16, true, false);
@@ -1038,6 +766,16 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                                  sdesc(smem_u32(sm + g_off[part]) + k * 2048u + j * 256u, 1024u,
                                        128u, LAYOUT_NONE),
                                  id_e, part > 0);
+            // Ghat (M = 128 state rows, N = 64 p) into G's columns, which masking has read
+            const uint32_t dy_base = smem_u32(sm + fuk::SM_DY);
+            const uint32_t id_h = idesc_bf16(128, 64, true, true);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t ch_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
+                for (int s = 0; s < Q / 16; ++s)
+                    mma_bf16(t_g, sdesc(ch_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                             sdesc(dy_base + s * 2048u, 8192u, 1024u, LAYOUT_SW128), id_h,
+                             part > 0 || s > 0);
+            }
             mma_commit(&bar_mma[1]);
         }
         ok = mbar_wait(&bar_mma[1], par, WAIT_LIMIT) ? 1 : 0;
@@ -1047,6 +785,139 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             aborted = true;
             break;
         }
+        // ---- chain step: Gc_c tiles, Gc_{c-1} = conj(E_c) Gc_c + Ghat_c, boundary value --
+        {
+            const bool c_valid = cn < N, c_pair = c_valid && cn >= nr;
+            const bool c_im = c_pair && ((cn - nr) & 1);
+            float ghv[16];
+            tmem_ld16(tmem_addr(t_g, 32u * (warp & 3), 16u * ccq), ghv);
+            // Gc_c as hi / lo operand tiles: shared memory (for V2) and the chunk's slot (for dx)
+            unsigned char *slot = reinterpret_cast<unsigned char *>(p.ws_gc + u * SLOT_FLOATS);
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const uint32_t off = off_kmaj(cn, 16 * ccq + 8 * g8, 128u, 1024u);
+                float hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float v = gcv[8 * g8 + j];
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+                    lo[j] = v - hi[j];
+                }
+                st16(sm + fuk::SM_GC, off, hi);
+                st16(sm + fuk::SM_GCL, off, lo);
+                st16(slot, off, hi);
+                st16(slot + TILE_BYTES, off, lo);
+            }
+            const int m = c_pair ? nr + ((cn - nr) >> 1) : (c_valid ? cn : 0);
+            const float er = f32[F_KRE + fslot(0, 4) * NP + m];
+            const float ei = c_pair ? f32[F_KIM + fslot(0, 4) * NP + m] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float other = __shfl_xor_sync(0xffffffffu, gcv[j], 1);
+                if (!c_valid)
+                    gcv[j] = 0.f;
+                else if (!c_pair)
+                    gcv[j] = fmaf(er, gcv[j], ghv[j]);
+                else if (!c_im)   // conj(er + i ei)(a + i d) + Ghat, own row = re
+                    gcv[j] = fmaf(er, gcv[j], fmaf(ei, other, ghv[j]));
+                else              // own row = im
+                    gcv[j] = fmaf(er, gcv[j], fmaf(-ei, other, ghv[j]));
+            }
+            if (c > 0) {
+                float4 *dst = carry_ptr(p, (rr + 1) & 1, bh, ccq, cn);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(gcv[4 * j4], gcv[4 * j4 + 1], gcv[4 * j4 + 2],
+                                                      gcv[4 * j4 + 3]));
+                if (p.ws_qb) {
+                    // exact boundary value sum_p conj(Gc_{c-1}) K_end_{c-1} of the decay-gradient
+                    // scan (K_end_{c-1} = the state entering this chunk, hi + lo tiles); each
+                    // 16-column block writes its own partial slot
+                    float kv[16];
+#pragma unroll
+                    for (int g8 = 0; g8 < 2; ++g8) {
+                        const uint32_t off = off_kmaj(cn, 16 * ccq + 8 * g8, 128u, 1024u);
+                        const uint4 hq = *reinterpret_cast<const uint4 *>(sm + fuk::SM_KT + off);
+                        const uint4 lq = *reinterpret_cast<const uint4 *>(sm + fuk::SM_KTL + off);
+                        const uint32_t hw[4] = {hq.x, hq.y, hq.z, hq.w};
+                        const uint32_t lw[4] = {lq.x, lq.y, lq.z, lq.w};
+#pragma unroll
+                        for (int w2 = 0; w2 < 4; ++w2) {
+                            const float2 a2_ = bf2_to_f2(hw[w2]), l2_ = bf2_to_f2(lw[w2]);
+                            kv[8 * g8 + 2 * w2] = a2_.x + l2_.x;
+                            kv[8 * g8 + 2 * w2 + 1] = a2_.y + l2_.y;
+                        }
+                    }
+                    float q = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float og = __shfl_xor_sync(0xffffffffu, gcv[j], 1);
+                        const float ok_ = __shfl_xor_sync(0xffffffffu, kv[j], 1);
+                        if (!c_pair)
+                            q = fmaf(gcv[j], kv[j], q);
+                        else if (!c_im)   // a ka + d kd
+                            q = fmaf(gcv[j], kv[j], fmaf(og, ok_, q));
+                        else              // a kd - d ka
+                            q = fmaf(og, kv[j], fmaf(-gcv[j], ok_, q));
+                    }
+                    if (c_valid) p.ws_qb[u * 4 * N + ccq * N + cn] = q;
+                }
+            } else {
+                // carry out of the first chunk = dL/dK_{-1}: dh0, dw0 = beta_0 dh0,
+                // dbeta_0 = <dh0, w0>
+                float beta0 = 0.f;
+                if (p.two_ep)
+                    beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+                float db0 = 0.f;
+                if (c_valid) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const long long i0 = ix_st(p, b, h, cn, 16 * ccq + j);
+                        if (p.dh0) p.dh0[i0] = gcv[j];
+                        if (p.dw0) p.dw0[i0] = beta0 * gcv[j];
+                        if (p.w0) db0 = fmaf(gcv[j], p.w0[i0], db0);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) db0 += __shfl_xor_sync(0xffffffffu, db0, o);
+                if (lane == 0) f32[F_CP + warp] = db0;   // summed after the next barrier
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // ---- phase C: V2 = Gc_c X^T (hi + lo) ------------------------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t x_base = smem_u32(sm + fuk::SM_X);
+            const uint32_t id_v = idesc_bf16(128, 64, false, false);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t gc_base = smem_u32(sm + (part ? fuk::SM_GCL : fuk::SM_GC));
+                for (int s = 0; s < PD / 16; ++s)
+                    mma_bf16(t_v2, sdesc(gc_base + s * 256u, 128u, 1024u, LAYOUT_NONE),
+                             sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_v,
+                             part > 0 || s > 0);
+            }
+            mma_commit(&bar_mma[2]);
+        } else if (tid == fuk::THREADS - 32) {
+            // the carry of chunk c - 1 is in place: let its item go (off the issue path)
+            if (c > 0) publish_count(p.ws_flag + bh, rr + 1);
+            if (c == 0) {
+                float acc = 0.f;
+                for (int k = 0; k < fuk::THREADS / 32; ++k) acc += f32[F_CP + k];
+                p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1] = acc;
+            }
+        }
+        ok = mbar_wait(&bar_mma[2], par, WAIT_LIMIT) ? 1 : 0;
+        if (!ok) rev_raise_error(1);
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // the tensor cores and the boundary value are done with x, dy and the entering
+        // state: fetch the next chunk's
+        if (tid == 0 && next < nitems) issue_xs(next);
         // ---- unfold: thread (row n, sub-block i) -----------------------------
         float *red = reinterpret_cast<float *>(sm + fuk::SM_RED);    // [128][RED_LD] B . gbu
         float *red2 = reinterpret_cast<float *>(sm + fuk::SM_RED2);  // [128][RED_LD] ddt terms
@@ -1349,28 +1220,14 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true) ||
         !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
-    static bool a1 = false, a3 = false, a4 = false;
+    if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
+    static bool a3 = false, a4 = false;
     cudaError_t e;
-    if ((e = set_smem(k_chunk_adj_local, loc::SMEM_BYTES, a1)) != cudaSuccess) return e;
     if ((e = set_smem(k_chunk_bwd_dx, dxk::SMEM_BYTES, a3)) != cudaSuccess) return e;
     if ((e = set_smem(k_chunk_bwd_fused, fuk::SMEM_BYTES, a4)) != cudaSuccess) return e;
-    const dim3 grid(p.nc, p.H, p.Bsz);
-    k_chunk_adj_local<<<grid, loc::THREADS, loc::SMEM_BYTES, st>>>(mc, mdy, p);
-    profile_mark(st, "k_chunk_adj_local");
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_chunk_adj_pass<<<dim3(p.H, p.Bsz), pass::THREADS, 0, st>>>(p);
-    profile_mark(st, "k_chunk_adj_pass");
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (p.sv_P) {
-        static bool a5 = false;
-        if ((e = set_smem(k_chunk_bwd_dx_saved, dxs::SMEM_BYTES, a5)) != cudaSuccess) return e;
-        k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
-        profile_mark(st, "k_chunk_bwd_dx_saved");
-    } else {
-        k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
-        profile_mark(st, "k_chunk_bwd_dx");
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the per-(b, h) carry counters start at zero on every call
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
+        return e;
     {
         const long long nitems = (long long)p.nc * p.H * p.Bsz;
         const int pgrid = (int)(nitems < sm_count() ? nitems : sm_count());
@@ -1383,6 +1240,18 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         k_chunk_bwd_fused<<<pgrid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, mdb, mdc, p);
     }
     profile_mark(st, "k_chunk_bwd_fused");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dx reads the adjoint carries the fused kernel left in every chunk's slot
+    const dim3 grid(p.nc, p.H, p.Bsz);
+    if (p.sv_P) {
+        static bool a5 = false;
+        if ((e = set_smem(k_chunk_bwd_dx_saved, dxs::SMEM_BYTES, a5)) != cudaSuccess) return e;
+        k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
+        profile_mark(st, "k_chunk_bwd_dx_saved");
+    } else {
+        k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
+        profile_mark(st, "k_chunk_bwd_dx");
+    }
     return cudaGetLastError();
 }
 

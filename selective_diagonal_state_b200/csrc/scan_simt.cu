@@ -831,7 +831,6 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
     const ModeInfo mi = mode_info(p, h, m);
     float *s_c = smem;  // [nthr]
     float car = 0.f, cai = 0.f, dA = 0.f, dth = 0.f, dD = 0.f;
-    const int nwp = p.P > 32 ? (p.P + 31) / 32 : 1;
     for (int tb = NTB - 1; tb >= 0; --tb) {
         const float *blk = p.ws_blk + (((long long)b * p.H + h) * NTB + tb) * (4 * (long long)nmode + 2);
         const float sdt = blk[4 * nmode + 0];
@@ -841,7 +840,7 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
             cai = 0.f;
             if (tb + 1 < NTB) {
                 const float *q = p.ws_qb + (((long long)b * p.H + h) * p.nc + (tb + 1)) * 4 * (long long)p.N;
-                for (int w2 = 0; w2 < nwp; ++w2) {
+                for (int w2 = 0; w2 < 4; ++w2) {   // four partial sums over column blocks of p
                     car += q[w2 * p.N + mi.n0];
                     if (mi.pair) cai += q[w2 * p.N + mi.n0 + 1];
                 }
