@@ -123,6 +123,7 @@ def kernel_bytes(shape, name: str) -> int:
 # is per 64-token chunk, so a launch moves batch x this).  An entry is removed
 # whenever its kernel changes after the capture.
 NCU_TRAFFIC_PER_ROW = {
+    ("hybridmamba", "k_chunk_bwd_fused"): (673.438720 + 541.037056) * 1e6 / 2,
 }
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)
