@@ -10,8 +10,11 @@ and the backward scan through the C ABI.  Prints one JSON line (rank 0).
 
 Under torchrun each rank scans its own batch (weak scaling); per-head
 parameter gradients are summed over ranks with one NCCL all-reduce, the only
-data-parallel exchange the path has.  Inputs (1.6 GB) exceed the 126 MB L2,
-so no flush is needed between steps.
+data-parallel exchange the path has.  HybridMamba's inputs (1.6 GB) exceed
+the 126 MB L2, so steps run back to back; for a workload whose inputs fit in
+twice the L2 (--workload mamba2_siso) every step is timed on its own and L2 is
+flushed between steps.  --workload picks one of the other configured
+workloads (their lines name it in config.workload).
 """
 from __future__ import annotations
 
@@ -118,13 +121,33 @@ def kernel_bytes(shape, name: str) -> int:
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per batch row of
-# the workload for the largest kernels, from the ncu capture summarised in
-# profiles/chunk_parallel_step_hybridmamba.md (taken at batch 2; the traffic
-# is per 64-token chunk, so a launch moves batch x this).  An entry is removed
-# whenever its kernel changes after the capture.
-NCU_TRAFFIC_PER_ROW = {
-    ("hybridmamba", "k_chunk_bwd_fused"): (673.438720 + 541.037056) * 1e6 / 2,
-}
+# the workload for the largest kernels, from one ncu capture of a smaller
+# batch (the traffic is per 64-token chunk, so a launch moves batch x this),
+# keyed by the kernel's source file and the first 16 hex digits of its SHA-256
+# at capture time: an entry whose source has changed since is not reported
+# (traffic null) instead of going stale.
+NCU_TRAFFIC_PER_ROW = {}
+
+
+def _source_sha16(rel):
+    import hashlib
+    path = os.path.join(ROOT, "selective_diagonal_state_b200", "csrc", rel)
+    try:
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def ncu_traffic(shape, kernel):
+    """Measured DRAM bytes of one launch of `kernel`, or None when there is no
+    capture of the kernel's current source."""
+    ent = NCU_TRAFFIC_PER_ROW.get((shape.name, kernel))
+    if ent is None:
+        return None
+    per_row, src, sha = ent
+    if _source_sha16(src) != sha:
+        return None
+    return per_row * shape.batch
 
 # upper bound on library launches per fwd + bwd step (sizes the profiling session)
 LAUNCHES_PER_STEP = 32
@@ -274,6 +297,34 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+L2_BYTES = 126 * 2 ** 20
+
+
+def roofline_of(shape, dom, ms_launch, peaks):
+    """Roofline entry of the dominant kernel: HBM bytes for every workload but
+    the Mamba-1 recovery, whose per-(token, channel, state) exponentials make it
+    bound by the special-function unit (MUFU)."""
+    hbm = peaks.get("hbm_gbs")
+    src = "measured" if hbm else "fallback"
+    hbm = hbm or 6650.0
+    if shape.name == "mamba1_siso" and dom in ("k_fwd", "k_bwd_sweep1", "k_bwd_sweep2"):
+        # one ex2 per (token, channel, state row) in each sweep over the sequence:
+        # 16 ex2 per SM and clock, 148 SMs, at the clock sampled under load
+        ex2 = shape.batch * shape.seqlen * shape.nheads * shape.nstate
+        clk = peaks.get("sm_mhz_under_load") or 1965.0
+        peak = 16 * 148 * clk * 1e6 / 1e9   # G ex2 / s
+        ach = ex2 / (ms_launch * 1e-3) / 1e9
+        return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "G ex2/s",
+                "frac": ach / peak, "traffic": ncu_traffic(shape, dom), "kernel": dom,
+                "algorithmic_ex2": ex2, "ms_per_launch": ms_launch,
+                "peak_source": "MUFU ex2 16/clk/SM x 148 SMs x SM clock"}
+    b = kernel_bytes(shape, dom)
+    ach = b / (ms_launch * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+            "traffic": ncu_traffic(shape, dom), "kernel": dom, "algorithmic_bytes": b,
+            "ms_per_launch": ms_launch, "peak_source": src}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -307,6 +358,9 @@ def main():
     ws = scan.alloc_workspace(shape, abi.PASS_BWD, desc=desc)
     wsf = scan.alloc_workspace(shape, abi.PASS_FWD, desc=desc)
     stream = torch.cuda.current_stream()
+    in_bytes = fwd_bytes(shape)   # x, B, C, dt, lambda and the y-sized dy
+    flush = in_bytes < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
 
     def barrier():
         if world > 1:
@@ -321,48 +375,75 @@ def main():
         scan.scan_backward(shape, dev, grads=grads, workspace=ws, desc=desc, saved=wsf)
         allreduce_params()
 
+    def fwd_only():
+        scan.scan_forward(shape, dev, out=fwd_out, desc=desc, workspace=wsf)
+
+    def timed(fn, n):
+        """Device ms per call of fn over n calls (CUDA events on our stream).  With
+        inputs that fit in L2, every call is timed on its own and L2 is flushed by
+        writing a buffer of twice its size between calls, outside the events."""
+        if not flush:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            scratch.fill_(1.0)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / n
+
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
-    route = {abi.ROUTE_CHUNKED: "tensor-core chain", abi.ROUTE_RANGE_FALLBACK:
-             "recurrent (range fallback)", abi.ROUTE_RECURRENT: "recurrent"}[abi.ssm_scan_last_route()]
+    names = {abi.ROUTE_CHUNKED: "per-coordinate tensor-core chain",
+             abi.ROUTE_RANGE_FALLBACK: "recurrent (range fallback)",
+             abi.ROUTE_RECURRENT: "recurrent", abi.ROUTE_SSD: "scalar-decay tensor-core chain"}
+    route_bwd = names[abi.ssm_scan_last_route()]
+    fwd_only()
+    route = {"fwd": names[abi.ssm_scan_last_route()], "bwd": route_bwd}
 
-    # per-kernel events over the timed region (library-owned, on our stream)
-    launches_per_step = LAUNCHES_PER_STEP
+    # ---- the headline: K steps, nothing else on the stream -----------------------
     clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
     clocks.start()
     time.sleep(0.3)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    abi.ssm_scan_profile_start(launches_per_step * args.steps)
     barrier()
     torch.cuda.synchronize()
     clocks.mark(True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    stop.record(stream)
-    torch.cuda.synchronize()
+    ms_step = timed(step, args.steps)
     barrier()
     clocks.mark(False)
-    prof = abi.ssm_scan_profile_stop()
-    ms_step = start.elapsed_time(stop) / args.steps
-    gpu_launches = sum(c for c, _ in prof.values())
-
-    # forward alone
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    f0.record(stream)
-    for _ in range(args.steps):
-        scan.scan_forward(shape, dev, out=fwd_out, desc=desc, workspace=wsf)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    ms_fwd = f0.elapsed_time(f1) / args.steps
+    ms_fwd = timed(fwd_only, args.steps)
     clk = clocks.stop()
+
+    # ---- per-kernel device times: a separate pass of K steps bracketed per launch
+    abi.ssm_scan_profile_start(LAUNCHES_PER_STEP * args.steps)
+    timed(step, args.steps)
+    prof = abi.ssm_scan_profile_stop()
+    launches_per_step = sum(c for c, _ in prof.values()) / args.steps
     avg = {n: tot / max(1, c) for n, (c, tot) in prof.items()}
     share = {n: tot / max(1e-9, sum(t for _, t in prof.values())) for n, (c, tot) in prof.items()}
+
+    # ---- memory: what the training forward keeps for the backward, and the peak
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base_alloc = torch.cuda.memory_allocated()
+    step()
+    torch.cuda.synchronize()
+    peak_alloc = torch.cuda.max_memory_allocated()
+    saved_bytes = int(wsf[1]) if wsf[0] is not None else 0
+    memory = {"saved_for_backward_bytes": saved_bytes,
+              "backward_workspace_bytes": int(ws[1]) if ws[0] is not None else 0,
+              "peak_alloc_bytes": int(peak_alloc), "resident_alloc_bytes": int(base_alloc)}
 
     # max over ranks
     t = torch.tensor([ms_step, ms_fwd], dtype=torch.float64, device="cuda")
@@ -378,12 +459,11 @@ def main():
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk):
         peaks = json.load(open(pk))
-    hbm = peaks.get("hbm_gbs")
-    peak_note = "measured" if hbm else "fallback"
-    hbm = hbm or 6650.0
+    if clk.get("sm_mhz"):
+        peaks = dict(peaks, sm_mhz_under_load=clk["sm_mhz"])
+    hbm = peaks.get("hbm_gbs") or 6650.0
     dom = max(avg, key=avg.get)
-    dom_bytes = kernel_bytes(shape, dom)
-    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    roof = roofline_of(shape, dom, avg[dom], peaks)
     step_bytes = fwd_bytes(shape) + bwd_bytes(shape)
 
     # end to end through the public API with host buffers
@@ -400,20 +480,18 @@ def main():
         h2d = sum(host[k].numel() * host[k].element_size() for k in dev_map
                   if k in host and dev_map[k] is not None)
         d2h = sum(o.numel() * o.element_size() for o in outs)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
+
+        def e2e_step():
             for k, d in dev_map.items():
                 if d is not None and k in host:
                     d.copy_(host[k], non_blocking=True)
             step()
             for o, ho in zip(outs, host_out):
                 ho.copy_(o, non_blocking=True)
-        e1.record(stream)
+
+        barrier()
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
+        ms_e2e = timed(e2e_step, args.e2e_steps)
         te = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -435,28 +513,31 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
+    io = "bf16, fp32 state" if shape.dtype_io == S.DTYPE_BF16 else "fp32"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype_io == S.DTYPE_BF16 else "f32",
         "data": "synthetic",
         "config": {"workload": shape.name, "batch_per_gpu": shape.batch, "seqlen": shape.seqlen,
-                   "nheads": shape.nheads, "headdim": shape.headdim,
+                   "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
                    "state": f"{shape.n_real} real + {shape.n_pairs} rotation pairs",
-                   "two_endpoint": bool(shape.two_endpoint), "io": "bf16, fp32 state",
+                   "rank_in": shape.rank_in, "rank_out": shape.rank_out,
+                   "two_endpoint": bool(shape.two_endpoint), "io": io,
                    "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": "inputs (1.6 GB) larger than L2; no flush", "route": route},
+                   "l2": (f"inputs ({in_bytes / 1e9:.2f} GB) fit in L2: each step timed alone, "
+                          f"L2 flushed between steps" if flush else
+                          f"inputs ({in_bytes / 1e9:.2f} GB) larger than L2; no flush"),
+                   "route": route},
         "fwd_tokens_per_s": fwd_value, "ms_fwd": ms_fwd,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": (NCU_TRAFFIC_PER_ROW[(shape.name, dom)] * shape.batch
-                                 if (shape.name, dom) in NCU_TRAFFIC_PER_ROW else None), "kernel": dom,
-                     "algorithmic_bytes": dom_bytes, "ms_per_launch": avg[dom],
-                     "peak_source": peak_note},
+        "roofline": roof,
         "step_roofline": {"algorithmic_bytes": step_bytes,
                           "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
                           "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm},
         "kernel_ms": avg, "kernel_share": share,
-        "gpu_launches": gpu_launches,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "memory": memory,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -91,9 +91,14 @@ typedef struct ssm_desc {
     int32_t n_real, n_pairs;
     int32_t rank_in, rank_out;  /* R, O; SISO is 1, 1 */
     int32_t chunk;              /* kernel choice, results equal up to rounding: 0 = library choice,
-                                   1 = token-by-token recurrent kernels, 64 = 64-token chunked
-                                   tensor-core kernels where supported (bf16, headdim 64,
-                                   rank 1, 64 or 128 state rows).  The chunked kernels fold
+                                   1 = token-by-token recurrent kernels, other values = the
+                                   chunked tensor-core kernels where supported.  A per-head
+                                   decay without rotation pairs (bf16, headdim 64, 64 or 128
+                                   state rows, rank_in == rank_out in {1, 2, 4}) takes the
+                                   scalar-decay chain, 128 / rank_in tokens per chunk, with no
+                                   range condition.  Other shapes with bf16, headdim 64,
+                                   rank 1 and 64 or 128 state rows take the 64-token
+                                   per-coordinate chain.  That chain folds
                                    each mode's decay into the operands around 16-token
                                    sub-block references, which needs
                                    |A| * log2(e) * (sum of dt over any 16 aligned tokens)
@@ -283,6 +288,20 @@ SSM_API int ssm_scan_profile_start(int max_launches);
 SSM_API int ssm_scan_profile_stop(char *names, int name_len, int *counts, double *total_ms,
                                   int max_kernels);
 
+/*
+ * Failure-path diagnostic (the pages have no counterpart).  The chained
+ * tensor-core kernels wait, on the device, for the chunk before (forward) or
+ * after (backward) to publish its carry; each such wait polls at most this
+ * many times (default 2^22, about half a second) before it gives up.  A wait
+ * that gives up stops every kernel of that call early (its outputs are then
+ * undefined), and the next ssm_scan_poll_device_error reports SSM_ERR_TIMEOUT;
+ * later calls are unaffected.  0 makes every such wait give up at once: tests
+ * use it to exercise the timeout path without a fault.  Applies to calls made
+ * after it returns (the value is read when a call is issued).  Returns the
+ * previous limit, or SSM_ERR_ARG for a negative value.
+ */
+SSM_API int64_t ssm_scan_set_wait_limit(int64_t polls);
+
 /* SSM_SCAN_ABI_VERSION of the loaded library. */
 SSM_API int ssm_scan_abi_version(void);
 
@@ -293,11 +312,19 @@ SSM_API int ssm_scan_abi_version(void);
  * SSM_ROUTE_RANGE_FALLBACK (chunk-eligible call whose inputs failed the
  * device-side range check, taken by the recurrent kernels),
  * SSM_ROUTE_RECURRENT (recurrent kernels chosen on the host: chunk = 1 or a
- * shape the chunked kernels do not take), or a negative status (no call yet,
+ * shape the chunked kernels do not take), SSM_ROUTE_SSD (per-head decay,
+ * bf16, head dim 64, 64 or 128 state rows, no rotation pairs, rank_in ==
+ * rank_out in {1, 2, 4}), or a negative status (no call yet,
  * or the gate word cannot be read).  A diagnostic for tests and tuning; the
  * pages have no counterpart.
  */
-enum ssm_route { SSM_ROUTE_CHUNKED = 0, SSM_ROUTE_RANGE_FALLBACK = 1, SSM_ROUTE_RECURRENT = 2 };
+enum ssm_route {
+    SSM_ROUTE_CHUNKED = 0,
+    SSM_ROUTE_RANGE_FALLBACK = 1,
+    SSM_ROUTE_RECURRENT = 2,
+    SSM_ROUTE_SSD = 3   /* tensor-core chain of a per-head (scalar) decay: masked linear
+                           attention with an exact segment-sum mask, 128 / R tokens per chunk */
+};
 SSM_API int ssm_scan_last_route(void *stream);
 
 #ifdef __cplusplus

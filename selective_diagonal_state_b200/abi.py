@@ -25,8 +25,8 @@ EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd"
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
             "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
-            "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd"]
-ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT = 0, 1, 2
+            "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd", "ssm_scan_set_wait_limit"]
+ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT, ROUTE_SSD = 0, 1, 2, 3
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -98,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_scan_profile_stop.restype = ctypes.c_int
     lib.ssm_scan_last_route.argtypes = [_vp]
     lib.ssm_scan_last_route.restype = ctypes.c_int
+    lib.ssm_scan_set_wait_limit.argtypes = [ctypes.c_int64]
+    lib.ssm_scan_set_wait_limit.restype = ctypes.c_int64
     _lib = lib
     return lib
 
@@ -217,6 +219,15 @@ def ssm_scan_bwd_noalloc(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev
 def ssm_scan_poll_device_error(stream=None) -> None:
     _check(load_library().ssm_scan_poll_device_error(_stream(stream)),
            "ssm_scan_poll_device_error")
+
+
+def ssm_scan_set_wait_limit(polls: int) -> int:
+    """Polls of a carry counter before a chained kernel's wait gives up (0: every
+    such wait gives up); returns the previous limit."""
+    rc = int(load_library().ssm_scan_set_wait_limit(int(polls)))
+    if rc < 0:
+        _check(rc, "ssm_scan_set_wait_limit")
+    return rc
 
 
 def ssm_scan_abi_version() -> int:

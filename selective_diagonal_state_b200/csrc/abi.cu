@@ -33,11 +33,19 @@ struct PreactArgs {
 cudaError_t preact_forward(const Params &p, const PreactArgs &a, cudaStream_t st);
 cudaError_t preact_backward(const Params &p, const PreactArgs &a, cudaStream_t st);
 cudaError_t scan_step(const Params &p, float *h, float *w, cudaStream_t st);
+bool ssd_supported(const Params &p);
+int ssd_chunk_tokens(int R);
+cudaError_t ssd_forward(const Params &p, cudaStream_t st);
+cudaError_t ssd_backward(const Params &p, cudaStream_t st);
+int ssd_error_take();
 }  // namespace ssm
 
 namespace {
 
 thread_local std::string g_last_error;
+
+// polls of a carry counter before a chained kernel's wait gives up
+std::atomic<long long> g_wait_limit{1ll << 22};
 
 // Gate words of the device-side choice between the tensor-core chain and the
 // recurrent chain (written by the range check of each call).  One slot per
@@ -170,6 +178,7 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
     p.two_ep = d->two_endpoint;
     p.per_coord = d->decay_mode == SSM_DECAY_PER_COORD;
     p.bf16 = d->dtype_io == SSM_BF16;
+    p.wait_limit = g_wait_limit.load();
     for (int k = 0; k < 3; ++k) {
         p.sx[k] = d->stride_x[k];
         p.sy[k] = d->stride_y[k];
@@ -193,6 +202,16 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0;
 }
 
+// Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and
+// SSD-MIMO with R = O in {1, 2, 4} (pointer alignment is checked at call time).
+bool ssd_shape(const ssm_desc_t *d) {
+    const int N = d->n_real + 2 * d->n_pairs;
+    return d->dtype_io == SSM_BF16 && d->decay_mode == SSM_DECAY_PER_HEAD && d->n_pairs == 0 &&
+           d->headdim == 64 && (N == 64 || N == 128) && d->rank_in == d->rank_out &&
+           (d->rank_in == 1 || d->rank_in == 2 || d->rank_in == 4) && d->chunk != 1 &&
+           d->seqlen > 0;
+}
+
 // Forward workspace of the tensor-core chain.  Every forward carries the fp32
 // state from one 64-token chunk to the next through two 32 KB slots and one
 // counter per (b, h) (the first `total_infer` bytes).  A training forward
@@ -207,6 +226,23 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
     FwdWs w;
     w.off_ring = w.off_flag = w.off_kp = w.off_ce = w.off_P = w.off_Bh = w.off_corr = 0;
     w.total_infer = w.total = 0;
+    if (ssd_shape(d)) {
+        // scalar-decay chain: the two fp32 carry slots and the counter of every (b, h),
+        // the ticket and abort words; a training forward also keeps the state entering
+        // every chunk of ssm::ssd_chunk_tokens tokens (bf16 hi + lo tiles, 32 KB)
+        const size_t bh = (size_t)d->batch * d->nheads;
+        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        const size_t units = bh * (size_t)((d->seqlen + qt - 1) / qt);
+        const size_t slot = 128 * (size_t)d->headdim * 4;
+        size_t off = align256(2 * bh * slot);
+        w.off_flag = off;
+        off = align256(off + (bh + 2) * 4);
+        w.total_infer = off;
+        w.off_kp = off;
+        off = align256(off + units * slot);
+        w.total = off;
+        return w;
+    }
     if (!tensor_chain_shape(d)) return w;
     const size_t bh = (size_t)d->batch * d->nheads;
     const size_t units = bh * (size_t)((d->seqlen + 63) / 64);
@@ -214,8 +250,8 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
     // every forward: the two carry slots and the carry counter of each (b, h)
     w.off_ring = 0;
     size_t off = align256(2 * bh * slot);
-    w.off_flag = off;
-    off = align256(off + bh * 4);
+    w.off_flag = off;   // carry counters, then the work-item ticket and the abort word
+    off = align256(off + (bh + 2) * 4);
     w.total_infer = off;
     // a training forward also keeps, per chunk, the state entering it (bf16 hi + lo
     // tiles), the chunk decays and the products the backward reuses
@@ -229,6 +265,45 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
     off = align256(off + units * 16384);
     w.off_corr = off;
     off = align256(off + units * 64 * 4);
+    w.total = off;
+    return w;
+}
+
+// Backward workspace of the scalar-decay chain: the adjoint carry slots and
+// counters, the entering states of every chunk (unless a training forward's are
+// given), per-token and per-chunk sums, and the per-head dB / dC of groups that
+// hold several heads.
+struct SsdBwdWs {
+    size_t off_ring, off_flag, off_kp, off_tok, off_par, off_db0, off_dBh, off_dCh, total;
+};
+SsdBwdWs ssd_bwd_layout(const ssm_desc_t *d) {
+    SsdBwdWs w;
+    const size_t bh = (size_t)d->batch * d->nheads;
+    const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+    const size_t nc = (size_t)((d->seqlen + qt - 1) / qt);
+    const size_t slot = 128 * (size_t)d->headdim * 4;
+    const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
+    const size_t N = nstate(d);
+    size_t off = 0;
+    w.off_ring = off;
+    off = align256(off + 2 * bh * slot);
+    w.off_flag = off;
+    off = align256(off + (bh + 2) * 4);
+    w.off_kp = off;
+    off = align256(off + bh * nc * slot);
+    w.off_tok = off;
+    off = align256(off + BLH * 3 * 4);
+    w.off_par = off;
+    off = align256(off + bh * nc * 2 * 4);
+    w.off_db0 = off;
+    off = align256(off + bh * 4);
+    w.off_dBh = w.off_dCh = off;
+    if (d->nheads != d->ngroups) {
+        w.off_dBh = off;
+        off = align256(off + BLH * d->rank_in * N * 4);
+        w.off_dCh = off;
+        off = align256(off + BLH * d->rank_out * N * 4);
+    }
     w.total = off;
     return w;
 }
@@ -270,8 +345,8 @@ BwdWs bwd_layout(const ssm_desc_t *d) {
         // the adjoint carried between chunks: two fp32 slots and a counter per (b, h)
         w.off_ring = off;
         off = align256(off + 2 * (size_t)d->batch * d->nheads * 128 * d->headdim * 4);
-        w.off_flag = off;
-        off = align256(off + (size_t)d->batch * d->nheads * 4);
+        w.off_flag = off;   // carry counters, then the work-item ticket and the abort word
+        off = align256(off + ((size_t)d->batch * d->nheads + 2) * 4);
     }
     w.total = off;
     return w;
@@ -335,7 +410,14 @@ size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
         return (d->batch == 0 || d->seqlen == 0) ? 0 : fwd_layout(d).total_infer;
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
-    return bwd_layout(d).total;
+    const size_t t = bwd_layout(d).total;
+    if (ssd_shape(d)) {
+        // either chain may take the call (the scalar-decay one unless pointer
+        // alignment rules it out): room for both
+        const size_t t2 = ssd_bwd_layout(d).total;
+        return t2 > t ? t2 : t;
+    }
+    return t;
 }
 
 int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
@@ -444,11 +526,36 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
     p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
     // chunk == 1 asks for the token-by-token recurrent kernels
-    const bool chunked = d->chunk != 1 && ssm::chunk_fwd_supported(p) && tensor_chain_shape(d);
-    if (!chunked && !ssm::simt_supported(p))
+    const bool ssd = ssd_shape(d) && ssm::ssd_supported(p);
+    const bool chunked =
+        !ssd && d->chunk != 1 && ssm::chunk_fwd_supported(p) && tensor_chain_shape(d);
+    if (!ssd && !chunked && !ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
     cudaStream_t st = (cudaStream_t)stream;
+    if (ssd) {
+        const FwdWs lay = fwd_layout(d);
+        if (!workspace || workspace_bytes < lay.total_infer)
+            return fail(SSM_ERR_WORKSPACE,
+                        "forward needs %zu bytes of workspace (%zu to save for the backward), got %zu",
+                        lay.total_infer, lay.total, workspace ? workspace_bytes : (size_t)0);
+        if ((uintptr_t)workspace % 256)
+            return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+        char *ws = (char *)workspace;
+        p.ws_ring = (float *)(ws + lay.off_ring);
+        p.ws_flag = (int *)(ws + lay.off_flag);
+        if (workspace_bytes >= lay.total) p.ws_kp = (float *)(ws + lay.off_kp);
+        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        p.nc = (int)((d->seqlen + qt - 1) / qt);
+        profile_begin(st);
+        const cudaError_t e = ssm::ssd_forward(p, st);
+        profile_end();
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_SSD;
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
+        g_last_error.clear();
+        return SSM_OK;
+    }
     if (chunked) {
         const FwdWs lay = fwd_layout(d);
         if (!workspace || workspace_bytes < lay.total_infer)
@@ -539,9 +646,10 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     if (d->n_pairs > 0 && (rc = check_ptr(dtheta, "dtheta", 4))) return rc;
     if (dlambda && ((uintptr_t)dlambda % es)) return fail(SSM_ERR_ALIGN, "dlambda misaligned");
     const BwdWs lay = bwd_layout(d);
-    if (!workspace || workspace_bytes < lay.total)
+    const size_t need_ws = ssm_scan_workspace_size(d, SSM_PASS_BWD);
+    if (!workspace || workspace_bytes < need_ws)
         return fail(SSM_ERR_WORKSPACE, "backward needs %zu bytes of workspace, got %zu",
-                    lay.total, workspace ? workspace_bytes : (size_t)0);
+                    need_ws, workspace ? workspace_bytes : (size_t)0);
     if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
     if (saved) {
         const size_t need = fwd_layout(d).total;
@@ -570,6 +678,38 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     p.ws_blk = (float *)(ws + lay.off_blk);
     p.ws_blkc = (float *)(ws + lay.off_blkc);
     p.nc = (int)((d->seqlen + 63) / 64);
+    if (ssd_shape(d) && ssm::ssd_supported(p) && ((uintptr_t)dy & 15) == 0 &&
+        ((uintptr_t)dx & 15) == 0 &&
+        (d->nheads != d->ngroups || ((((uintptr_t)dB | (uintptr_t)dC) & 15) == 0))) {
+        // scalar-decay chain
+        const SsdBwdWs sl = ssd_bwd_layout(d);
+        ssm::Params pc = p;
+        pc.ws_ring = (float *)(ws + sl.off_ring);
+        pc.ws_flag = (int *)(ws + sl.off_flag);
+        pc.ws_kp = (float *)(ws + sl.off_kp);
+        pc.sd_tok = (float *)(ws + sl.off_tok);
+        pc.sd_par = (float *)(ws + sl.off_par);
+        pc.sd_db0 = (float *)(ws + sl.off_db0);
+        if (d->nheads != d->ngroups) {
+            pc.sd_dBh = (float *)(ws + sl.off_dBh);
+            pc.sd_dCh = (float *)(ws + sl.off_dCh);
+        }
+        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        pc.nc = (int)((d->seqlen + qt - 1) / qt);
+        if (saved) {
+            pc.ws_kp = (float *)((const char *)saved + fwd_layout(d).off_kp);
+            pc.states_ready = 1;
+        }
+        profile_begin(st);
+        const cudaError_t e = ssm::ssd_backward(pc, st);
+        profile_end();
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_SSD;
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
+        g_last_error.clear();
+        return SSM_OK;
+    }
+    if (saved && ssd_shape(d)) saved = nullptr;   // scalar-decay forward states: not read here
     if (!ssm::simt_supported(p))
         return fail(SSM_ERR_UNSUPPORTED, "no kernel for n_real=%d n_pairs=%d P=%lld R=%d O=%d",
                     d->n_real, d->n_pairs, (long long)d->headdim, d->rank_in, d->rank_out);
@@ -655,6 +795,8 @@ int ssm_scan_poll_device_error(void *stream) {
     int word = ssm::chunk_error_take();
     const int word2 = ssm::chunk_rev_error_take();
     if (word == 0 || word2 < 0) word = word2;
+    const int word3 = ssm::ssd_error_take();
+    if (word == 0 || word3 < 0) word = word3;
     if (word < 0) return fail(SSM_ERR_CUDA, "ssm_scan_poll_device_error: cannot read the error word");
     if (word == 1) return fail(SSM_ERR_TIMEOUT, "a bounded device-side wait gave up");
     if (word != 0) return fail(SSM_ERR_TIMEOUT, "device-side error code %d", word);
@@ -662,6 +804,11 @@ int ssm_scan_poll_device_error(void *stream) {
 }
 
 int ssm_scan_abi_version(void) { return SSM_SCAN_ABI_VERSION; }
+
+int64_t ssm_scan_set_wait_limit(int64_t polls) {
+    if (polls < 0) return fail(SSM_ERR_ARG, "wait limit must be >= 0");
+    return (int64_t)g_wait_limit.exchange((long long)polls);
+}
 
 int ssm_scan_last_route(void *stream) {
     if (g_last_route < 0) return fail(SSM_ERR_ARG, "no scan call on this thread yet");

@@ -332,7 +332,61 @@ __device__ __forceinline__ ChunkItem chunk_item(const Params &p, int item) {
 // walking order reads the fp32 carry from slot r & 1 once the counter of
 // (b, h) reaches r, writes the next carry to slot (r + 1) & 1 and sets the
 // counter to r + 1.
-constexpr long long FLAG_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
+//
+// Work items are handed out by a ticket counter in the workspace (zeroed with
+// the carry counters on every call): a CTA takes its next item, one ahead of
+// the one it works on, with an atomic increment.  Tickets only go to CTAs that
+// are running, in increasing order, so the item an item waits on (the same
+// (b, h), one chunk earlier in walking order, hence a smaller ticket) is held
+// by a running CTA; the smallest unfinished item never waits, so the chain
+// always progresses, whatever number of CTAs is resident.
+// A carry wait gives up after Params::wait_limit polls; the CTA then raises the
+// device error word, sets the call's abort word (so that every other wait of
+// the call gives up at once instead of polling to its own limit) and stops.
+constexpr long long DEFAULT_WAIT_LIMIT = 1ll << 22;   // polls of a carry counter (~0.5 s)
+
+__device__ __forceinline__ int *chain_ticket(const Params &p) { return p.ws_flag + p.Bsz * p.H; }
+__device__ __forceinline__ int *chain_abort_word(const Params &p) {
+    return p.ws_flag + p.Bsz * p.H + 1;
+}
+
+// Wait until *flag >= target: at most `limit` polls (none for limit 0, which
+// makes every wait give up), and none after the call's abort word is set.
+__device__ __forceinline__ bool wait_count(const int *flag, int target, const int *abort_word,
+                                           long long limit) {
+    for (long long i = 0; i < limit; ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v >= target) return true;
+        if ((i & 15) == 15) {
+            int a;
+            asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(a) : "l"(abort_word) : "memory");
+            if (a) return false;
+        }
+        __nanosleep(64);
+    }
+    return false;
+}
+__device__ __forceinline__ void publish_count(int *flag, int v) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+__device__ __forceinline__ void chain_abort(const Params &p) { atomicExch(chain_abort_word(p), 1); }
+
+// Loads (TMA / bulk copies) and MMA commits completing on one mbarrier, counted
+// by the issuing thread, so that a CTA that stops early can wait for every
+// phase still outstanding before its shared memory and TMEM go away.
+struct PhaseCount {
+    uint32_t issued, done;
+};
+// Wait for every outstanding phase (bounded); false if one did not complete.
+__device__ __forceinline__ bool drain_phases(uint64_t *bar, PhaseCount &pc) {
+    while (pc.done < pc.issued) {
+        if (!mbar_wait(bar, pc.done & 1u, WAIT_LIMIT)) return false;
+        ++pc.done;
+    }
+    return true;
+}
 
 // item -> (chunk, head, batch row), chunk slowest
 __device__ __forceinline__ ChunkItem chunk_item_cs(const Params &p, int item) {
@@ -350,20 +404,6 @@ __device__ __forceinline__ ChunkItem chunk_item_cs(const Params &p, int item) {
 __device__ __forceinline__ float4 *carry_ptr(const Params &p, int slot, int bh, int cq, int n) {
     return reinterpret_cast<float4 *>(p.ws_ring) +
            (((long long)(slot * p.Bsz * p.H + bh) * 4 + cq) * 4) * NP + n;
-}
-
-__device__ __forceinline__ bool wait_count(const int *flag, int target) {
-    for (long long i = 0; i < FLAG_WAIT_LIMIT; ++i) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-        if (v >= target) return true;
-        __nanosleep(64);
-    }
-    return false;
-}
-__device__ __forceinline__ void publish_count(int *flag, int v) {
-    __threadfence();
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
 }
 
 // item -> (chunk, head, batch row), chunk slowest, last chunk first (the walk of

@@ -46,7 +46,9 @@ struct Params {
     // forward chain: fp32 state carried from chunk c to c + 1 through two slots per
     // (b, h), and the count of chunks of (b, h) whose outgoing state is in place
     float *ws_ring; // [2][B][H][4][4][128][4] carry slots (row-contiguous per 4 columns)
-    int *ws_flag;   // [B][H]           (the backward carries its adjoint the same way)
+    int *ws_flag;   // [B][H] counters, then [0] the next work item (ticket) and [1] the
+                    // abort word of this call (the backward carries its adjoint the same way)
+    long long wait_limit;   // polls of a carry counter before a wait gives up
     int nc;         // number of 64-token chunks
     // device-side choice between two launched kernel chains: a kernel runs
     // only when (*gate != 0) == gate_on (no gate: always)
@@ -58,6 +60,11 @@ struct Params {
     unsigned char *sv_P;    // [B][H][NC] 8 KB: masked scores P^T as bf16 operand tiles
     unsigned char *sv_Bh;   // [B][H][NC] 16 KB: chunk-end folded B (bf16 operand tile)
     float *sv_corr;         // [B][H][NC][64] D - beta_{t+1} C_t . B_t
+    // scalar-decay chain backward (chunks of 128 / R tokens):
+    float *sd_tok;          // [B][L][H][3] dsigma_t, diag_t (the gamma_t part), drho_t
+    float *sd_par;          // [B][H][NC][2] per chunk: sum_t dt_t drho_t, sum <dy, x>
+    float *sd_db0;          // [B][H] dbeta_0 = <dL/dK_{-1}, w0>
+    float *sd_dBh, *sd_dCh; // [B][L][H][R or O][N] fp32 per-head dB / dC (several heads per group)
     Geometry geo;
 };
 

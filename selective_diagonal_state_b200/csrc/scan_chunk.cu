@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 // (batch row, head) chained through a carry in global memory.
 //
 // Items run chunk-slowest (item = c * B*H + b*H + h), one persistent CTA per SM
-// with a stride of the grid, so the item of chunk c - 1 of the same (b, h) was
-// taken about B*H items earlier.  Per item:
+// taking tickets from a counter in the workspace, so the item of chunk c - 1 of
+// the same (b, h) was taken B*H tickets earlier.  Per item:
 //   - operands Ci, Ch, Bi (as for the scores) and Bh (hi + lo) are folded from
 //     raw B / C; phase A of the tensor cores needs no carried state:
 //       scores^T_i = Bi (64 s x N) . Ci^T (N x 16 t)          M=64,  N=16, K=N
@@ -352,8 +352,8 @@ __global__ void __launch_bounds__(pas::THREADS) k_chunk_state_pass(Params p) {
 // even when B*H is below the number of SMs and the chunks of one (b, h) run
 // side by side.
 // The carry slots (2 x 32 KB per (b, h)) stay in L2.  Every item waits only on
-// an item with a smaller index, which its CTA took earlier, so the chain makes
-// progress whenever the CTAs owning earlier items run.
+// an item with a smaller ticket, which a running CTA holds, so the chain makes
+// progress whatever number of CTAs is resident.
 // ============================================================================
 namespace fwk {
 constexpr int THREADS = 512;
@@ -424,6 +424,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     uint64_t *bar_bc = bar_x + 2;                                       // raw B, C
     uint64_t *bar_mma = bar_x + 3;                                      // [2] phase A, B
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 5);
+    int *s_item = reinterpret_cast<int *>(bar_x + 6);                  // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
@@ -444,7 +445,9 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         }
     };
 
-    int item = blockIdx.x;
+    // phases issued / completed on each mbarrier (counted by thread 0, which issues
+    // every load and the first MMA batch of a phase), for the drain of a CTA that stops
+    PhaseCount pc_x[2] = {{0u, 0u}, {0u, 0u}}, pc_bc = {0u, 0u}, pc_a = {0u, 0u}, pc_b = {0u, 0u};
     if (tid == 0) {
         mbar_init(&bar_x[0], 1);
         mbar_init(&bar_x[1], 1);
@@ -455,13 +458,21 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-        issue_x(item, 0);
-        issue_bc(item);
+        const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
+        s_item[0] = first;
+        issue_x(first, 0);
+        ++pc_x[0].issued;
+        issue_bc(first);
+        ++pc_bc.issued;
     }
     if (warp == 0) tmem_alloc(tslot, fwk::TMEM_COLS);
     if (N < NP)  // K padding of Ci, Ch, Bi and M padding of Bh (rows past N are never written)
         for (int i = tid; i < (int)((fwk::SM_KT - fwk::SM_CI) / 16); i += fwk::THREADS)
             reinterpret_cast<uint4 *>(sm + fwk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    int item = s_item[0];
     TokPrefetch tok;
     ModePrefetch mp;
     {
@@ -469,9 +480,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         tok = tok_load(p, it.b, it.h, it.c * Q);
         mp = mode_load(p, it.h);
     }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_y = tbase;                      // Y^T (M=64, lanes 0-15 of each quarter)
     const uint32_t t_sc = tbase + (16u << 16);       // scores^T (M=64, lanes 16-31)
@@ -479,25 +487,30 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     float *cpart = reinterpret_cast<float *>(sm + fwk::SM_P);   // C.B partials until P is built
     bool aborted = false;
 
-    for (int k = 0; item < nitems; ++k, item += gridDim.x) {
+    for (int k = 0; item < nitems; ++k) {
+        // the item after this one (read by every thread after the next barrier)
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const int st = k & 1;
         const ChunkItem it = chunk_item_cs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int bh = b * p.H + h;
         const int t0 = c * Q;
-        const int next = item + gridDim.x;
         unsigned char *sX = sm + fwk::SM_X + st * 8192;
         const unsigned char *sB = sm + fwk::SM_B, *sC = sm + fwk::SM_C;
 
         // ---- this chunk's small inputs; K_c once the previous chunk has published it
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
+        const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
             mp = mode_load(p, nx.h);
             // the other x stage was last read by the previous chunk, which is complete
-            if (tid == 0) issue_x(next, st ^ 1);
+            if (tid == 0) {
+                issue_x(next, st ^ 1);
+                ++pc_x[st ^ 1].issued;
+            }
         }
         chunk_mode_constants(p, f32);
         if (p.ws_ce && tid < p.nr + p.np) {
@@ -507,9 +520,17 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         }
         // the previous chunk's y store has to have read the P region (corr partials below)
         if (tid == 0) bulk_wait_read_all();
-        int ok = (mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT) &&
-                  mbar_wait(bar_bc, (uint32_t)(k & 1), WAIT_LIMIT)) ? 1 : 0;
-        if (!ok) raise_error(1);
+        const bool okx = mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT);
+        const bool okb = okx && mbar_wait(bar_bc, (uint32_t)(k & 1), WAIT_LIMIT);
+        if (tid == 0) {
+            pc_x[st].done += okx ? 1u : 0u;
+            pc_bc.done += okb ? 1u : 0u;
+        }
+        int ok = okb ? 1 : 0;
+        if (!ok) {
+            raise_error(1);
+            chain_abort(p);
+        }
         if (!__syncthreads_and(ok)) {
             aborted = true;
             break;
@@ -621,12 +642,25 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             cpart[grp * 64 + t] = corr;
         }
         // K_c is published by the item of chunk c - 1 (everything above does not need it)
-        if (tid == 0 && c > 0 && !wait_count(p.ws_flag + bh, c)) raise_error(2);
+        int cw = 1;
+        if (tid == 0 && c > 0 &&
+            !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
+            raise_error(2);
+            chain_abort(p);
+            cw = 0;
+        }
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();   // also orders the wait before every thread's loads of K_c
+        // also orders the wait before every thread's loads of K_c
+        if (!__syncthreads_and(cw)) {
+            aborted = true;
+            break;
+        }
         // raw B and C are consumed: fetch the next chunk's
-        if (tid == 0 && next < nitems) issue_bc(next);
+        if (tid == 0 && next < nitems) {
+            issue_bc(next);
+            ++pc_bc.issued;
+        }
 
         // ---- phase A: scores, chunk-local state --------------------------------
         if (tid == 0) {
@@ -640,6 +674,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(ci_base + 2u * i * KM_SBO + s * 256u, KM_LBO, KM_SBO, LAYOUT_NONE),
                              id_sc, s > 0);
             mma_commit(&bar_mma[0]);
+            ++pc_a.issued;
         } else if (tid == 32) {
             fence_after_sync();
             const uint32_t x_base = smem_u32(sX);
@@ -665,7 +700,11 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         float kc[16];
         load_k(p, c, b, h, kn_row, kcq, kc);
         ok = mbar_wait(&bar_mma[0], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
-        if (!ok) raise_error(1);
+        if (tid == 0) pc_a.done += (uint32_t)ok;
+        if (!ok) {
+            raise_error(1);
+            chain_abort(p);
+        }
         fence_after_sync();
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -790,9 +829,14 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              sdesc(p_base + i * 2048u + s * 512u, 256u, 128u, LAYOUT_NONE), id_d,
                              true);
             mma_commit(&bar_mma[1]);
+            ++pc_b.issued;
         }
         ok = mbar_wait(&bar_mma[1], (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
-        if (!ok) raise_error(1);
+        if (tid == 0) pc_b.done += (uint32_t)ok;
+        if (!ok) {
+            raise_error(1);
+            chain_abort(p);
+        }
         fence_after_sync();
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -827,13 +871,17 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             tma_store_4d(&tmY, sm + fwk::SM_P, 0, h, t0, b);
             bulk_commit();
         }
+        item = next;
     }
     if (tid == 0) bulk_wait_read_all();
     if (aborted && tid == 0) {
-        // let loads still in flight land before the CTA's shared memory goes away
-        mbar_wait(&bar_x[0], 0, WAIT_LIMIT);
-        mbar_wait(&bar_x[1], 0, WAIT_LIMIT);
-        mbar_wait(bar_bc, 0, WAIT_LIMIT);
+        // every load and MMA still in flight lands before the CTA's shared memory and
+        // TMEM go away
+        drain_phases(&bar_x[0], pc_x[0]);
+        drain_phases(&bar_x[1], pc_x[1]);
+        drain_phases(bar_bc, pc_bc);
+        drain_phases(&bar_mma[0], pc_a);
+        drain_phases(&bar_mma[1], pc_b);
     }
     fence_before_sync();
     __syncthreads();
@@ -918,11 +966,16 @@ int sm_count() {
     return cached[dev];
 }
 
+// Opt-in to the dynamic shared memory of a kernel on the current device (the
+// attribute is per device, so the flag is kept per device ordinal).
 template <typename K>
-static cudaError_t set_smem_once(K kern, uint32_t bytes, bool &done) {
-    if (done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) done = true;
+static cudaError_t set_smem_once(K kern, uint32_t bytes, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
     return e;
 }
 
@@ -934,7 +987,7 @@ cudaError_t chunk_states(const Params &p, cudaStream_t st) {
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
         !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true))
         return cudaErrorInvalidValue;
-    static bool a1 = false;
+    static bool a1[64] = {};
     cudaError_t e;
     if ((e = set_smem_once(k_chunk_state_local, stl::SMEM_BYTES, a1)) != cudaSuccess) return e;
     k_chunk_state_local<<<dim3(p.nc, p.H, p.Bsz), stl::THREADS, stl::SMEM_BYTES, st>>>(mx, mb, p);
@@ -953,11 +1006,12 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
-    static bool a3 = false;
+    static bool a3[64] = {};
     cudaError_t e;
     if ((e = set_smem_once(k_chunk_fwd, fwk::SMEM_BYTES, a3)) != cudaSuccess) return e;
-    // the per-(b, h) carry counters start at zero on every call
-    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
+    // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
+        cudaSuccess)
         return e;
     const long long nitems = (long long)p.nc * p.H * p.Bsz;
     const int grid = (int)(nitems < sm_count() ? nitems : sm_count());

@@ -501,6 +501,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);   // [2]: x/dy/states, B/C
     uint64_t *bar_mma = bar_in + 2;                                      // [3] phases A, B, C
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 5);
+    int *s_item = reinterpret_cast<int *>(bar_in + 6);                  // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
@@ -526,7 +527,9 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     };
 
-    int item = blockIdx.x;
+    // phases issued / completed on each mbarrier (counted by thread 0, which issues
+    // every load and the first MMA batch of a phase), for the drain of a CTA that stops
+    PhaseCount pc_in[2] = {{0u, 0u}, {0u, 0u}}, pc_m[3] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
     if (tid == 0) {
         mbar_init(&bar_in[0], 1);
         mbar_init(&bar_in[1], 1);
@@ -538,10 +541,18 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
-        issue_xs(item);
-        issue_bc(item);
+        const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
+        s_item[0] = first;
+        issue_xs(first);
+        ++pc_in[0].issued;
+        issue_bc(first);
+        ++pc_in[1].issued;
     }
     if (warp == 0) tmem_alloc(tslot, fuk::TMEM_COLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    int item = s_item[0];
     TokPrefetch tok;
     ModePrefetch mp;
     {
@@ -549,33 +560,41 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tok = tok_load(p, it.b, it.h, it.c * Q);
         mp = mode_load(p, it.h);
     }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
     const uint32_t tbase = *tslot;
     const uint32_t t_v = tbase, t_v2 = tbase + 64u, t_g = tbase + 128u;
     const int cn = 32 * (warp & 3) + lane, ccq = warp >> 2;   // chain step: row, 16-column block
     bool aborted = false;
 
-    for (int kit = 0; item < nitems; ++kit, item += gridDim.x) {
+    for (int kit = 0; item < nitems; ++kit) {
+        // the item after this one (read by every thread after the next barrier)
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const ChunkItem it = chunk_item_rcs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int g = h / p.hpg;
         const int t0 = c * Q;
         const long long u = bhc(p, b, h, c);
         const int bh = b * p.H + h, rr = p.nc - 1 - c;   // chunks of (b, h) walked before this one
-        const int next = item + gridDim.x;
         const uint32_t par = (uint32_t)(kit & 1);
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
+        const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
             mp = mode_load(p, nx.h);
         }
         chunk_mode_constants(p, f32);
-        int ok = (mbar_wait(&bar_in[0], par, WAIT_LIMIT) && mbar_wait(&bar_in[1], par, WAIT_LIMIT)) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
+        const bool ok0 = mbar_wait(&bar_in[0], par, WAIT_LIMIT);
+        const bool ok1 = ok0 && mbar_wait(&bar_in[1], par, WAIT_LIMIT);
+        if (tid == 0) {
+            pc_in[0].done += ok0 ? 1u : 0u;
+            pc_in[1].done += ok1 ? 1u : 0u;
+        }
+        int ok = ok1 ? 1 : 0;
+        if (!ok) {
+            rev_raise_error(1);
+            chain_abort(p);
+        }
         if (!__syncthreads_and(ok)) {
             aborted = true;
             break;
@@ -648,6 +667,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 mma_bf16(t_g, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
                          sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_g, s > 0);
             mma_commit(&bar_mma[0]);
+            ++pc_m[0].issued;
         }
         if (tid < 64) {
             float cs = 0.f;
@@ -657,7 +677,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             f32[F_CORR + tid] = cs;   // C_t . B_t
         }
         ok = mbar_wait(&bar_mma[0], par, WAIT_LIMIT) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
+        if (tid == 0) pc_m[0].done += (uint32_t)ok;
+        if (!ok) {
+            rev_raise_error(1);
+            chain_abort(p);
+        }
         fence_after_sync();
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -721,10 +745,20 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
         }
         // the adjoint carried into this chunk is published by the item of chunk c + 1
-        if (tid == 0 && rr > 0 && !wait_count(p.ws_flag + bh, rr)) rev_raise_error(2);
+        int cw = 1;
+        if (tid == 0 && rr > 0 &&
+            !wait_count(p.ws_flag + bh, rr, chain_abort_word(p), p.wait_limit)) {
+            rev_raise_error(2);
+            chain_abort(p);
+            cw = 0;
+        }
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();   // also orders the wait before every thread's loads of Gc_c
+        // also orders the wait before every thread's loads of Gc_c
+        if (!__syncthreads_and(cw)) {
+            aborted = true;
+            break;
+        }
         float gcv[16];     // Gc_c of row cn, columns 16 ccq ..; in flight during phase B
 #pragma unroll
         for (int j4 = 0; j4 < 4; ++j4) {
@@ -752,6 +786,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                                        1024u, LAYOUT_NONE),
                                  id_d, part > 0);
             mma_commit(&bar_mma[1]);
+            ++pc_m[1].issued;
         } else if (tid == 32) {
             fence_after_sync();
             const uint32_t id_e = idesc_bf16(128, 16, true, true);
@@ -779,7 +814,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             mma_commit(&bar_mma[1]);
         }
         ok = mbar_wait(&bar_mma[1], par, WAIT_LIMIT) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
+        if (tid == 0) pc_m[1].done += (uint32_t)ok;
+        if (!ok) {
+            rev_raise_error(1);
+            chain_abort(p);
+        }
         fence_after_sync();
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -899,6 +938,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                              part > 0 || s > 0);
             }
             mma_commit(&bar_mma[2]);
+            ++pc_m[2].issued;
         } else if (tid == fuk::THREADS - 32) {
             // the carry of chunk c - 1 is in place: let its item go (off the issue path)
             if (c > 0) publish_count(p.ws_flag + bh, rr + 1);
@@ -909,7 +949,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             }
         }
         ok = mbar_wait(&bar_mma[2], par, WAIT_LIMIT) ? 1 : 0;
-        if (!ok) rev_raise_error(1);
+        if (tid == 0) pc_m[2].done += (uint32_t)ok;
+        if (!ok) {
+            rev_raise_error(1);
+            chain_abort(p);
+        }
         fence_after_sync();
         if (!__syncthreads_and(ok)) {
             aborted = true;
@@ -917,7 +961,10 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         // the tensor cores and the boundary value are done with x, dy and the entering
         // state: fetch the next chunk's
-        if (tid == 0 && next < nitems) issue_xs(next);
+        if (tid == 0 && next < nitems) {
+            issue_xs(next);
+            ++pc_in[0].issued;
+        }
         // ---- unfold: thread (row n, sub-block i) -----------------------------
         float *red = reinterpret_cast<float *>(sm + fuk::SM_RED);    // [128][RED_LD] B . gbu
         float *red2 = reinterpret_cast<float *>(sm + fuk::SM_RED2);  // [128][RED_LD] ddt terms
@@ -1088,6 +1135,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             } else if (next < nitems) {
                 // every token loop is done with the raw B / C tiles: fetch the next chunk's
                 issue_bc(next);
+                ++pc_in[1].issued;
             }
         }
         float later = 0.f;
@@ -1137,7 +1185,10 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (tid == 0 && one_head) {
             // the dB / dC stores have read the B / C tiles: fetch the next chunk's
             bulk_wait_read_all();
-            if (next < nitems) issue_bc(next);
+            if (next < nitems) {
+                issue_bc(next);
+                ++pc_in[1].issued;
+            }
         }
         if (tid < 64 && t0 + tid < L) {
             const int t = tid;
@@ -1171,11 +1222,14 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         fence_before_sync();
         __syncthreads();
+        item = next;
     }
     if (aborted && tid == 0) {
-        // let loads still in flight land before the CTA's shared memory goes away
-        mbar_wait(&bar_in[0], 0, WAIT_LIMIT);
-        mbar_wait(&bar_in[1], 0, WAIT_LIMIT);
+        // every load and MMA still in flight lands before the CTA's shared memory and
+        // TMEM go away
+        drain_phases(&bar_in[0], pc_in[0]);
+        drain_phases(&bar_in[1], pc_in[1]);
+        for (int q = 0; q < 3; ++q) drain_phases(&bar_mma[q], pc_m[q]);
     }
     if (tid == 0) bulk_wait_read_all();
     fence_before_sync();
@@ -1191,11 +1245,16 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// Opt-in to the dynamic shared memory of a kernel on the current device (the
+// attribute is per device, so the flag is kept per device ordinal).
 template <typename K>
-static cudaError_t set_smem(K kern, uint32_t bytes, bool &done) {
-    if (done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) done = true;
+static cudaError_t set_smem(K kern, uint32_t bytes, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
     return e;
 }
 
@@ -1221,12 +1280,13 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
-    static bool a3 = false, a4 = false;
+    static bool a3[64] = {}, a4[64] = {};
     cudaError_t e;
     if ((e = set_smem(k_chunk_bwd_dx, dxk::SMEM_BYTES, a3)) != cudaSuccess) return e;
     if ((e = set_smem(k_chunk_bwd_fused, fuk::SMEM_BYTES, a4)) != cudaSuccess) return e;
-    // the per-(b, h) carry counters start at zero on every call
-    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
+    // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
+        cudaSuccess)
         return e;
     {
         const long long nitems = (long long)p.nc * p.H * p.Bsz;
@@ -1244,7 +1304,7 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
     // dx reads the adjoint carries the fused kernel left in every chunk's slot
     const dim3 grid(p.nc, p.H, p.Bsz);
     if (p.sv_P) {
-        static bool a5 = false;
+        static bool a5[64] = {};
         if ((e = set_smem(k_chunk_bwd_dx_saved, dxs::SMEM_BYTES, a5)) != cudaSuccess) return e;
         k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
         profile_mark(st, "k_chunk_bwd_dx_saved");

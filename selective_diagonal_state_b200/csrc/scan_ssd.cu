@@ -1,0 +1,1467 @@
+// Chunked tensor-core scan for a per-head (scalar) decay: the Mamba-2 SISO and
+// SSD-MIMO configurations ("When a Diagonal State Is Not Enough",
+// sungsoo.github.io, Part 03 "Selective SSM and masked linear attention" and
+// "SISO and MIMO"; Part 08 item 3), bf16 I/O, fp32 state, head dim 64, 64 or
+// 128 state rows, rank R = O in {1, 2, 4}, optional two-endpoint writes.
+//
+// With one decay a per head the transition between tokens s < t is the scalar
+// exp(a (S_t - S_s)), S the cumulative sum of dt, so the state-mediated part
+// of the scan is unnormalised masked linear attention (Thm 24 of Part 03): a
+// chunk's output is
+//     Y = (C B^T (.) W) X + diag(e) C K_in + D X
+// where the rows of X, B (sources) and of Y, C (targets) are the chunk's
+// (token, rank) pairs -- R value rows per token, so SSD-MIMO is the SISO form
+// with R source and O target rows per token (Part 03 "SISO and MIMO") --,
+// W[j, i] = exp(a (S_tj - S_ti)) sigma_ti for t_i < t_j, gamma_tj for
+// t_i = t_j and 0 after (the two-endpoint write in the pre-state form
+// K_t = A_t K_{t-1} + sigma_t W_t, sigma_t = gamma_t + beta_{t+1}, whose
+// readout C_t K_t - beta_{t+1} C_t W_t leaves gamma_t on the diagonal),
+// e_t = exp(a S_t) and K_in the state entering the chunk.  The chunk's end
+// state is
+//     K_out = E K_in + B^T diag(f) X,   f_t = exp(a (S_end - S_t)) sigma_t,
+//     E = exp(a S_end).
+// Every exponent is <= 0, so no range condition applies.
+//
+// A chunk has 128 (token, rank) rows: 128 / R tokens.  Per chunk, on the
+// tensor cores (M = 128 everywhere, fp32 accumulators in TMEM):
+//     CB   = C (128 j x N) . B^T (N x 128 i)
+//     S_c  = B^T (N x 128 i) . X' (128 i x 64 p),   X' = diag(f) X
+//     Y_d  = P (128 j x 128 i) . X (128 i x 64 p),  P = CB (.) W  (bf16)
+//     Y_o  = C (128 j x N) . K_in (N x 64 p)
+// and y = Y_d + e Y_o + D x.  k_ssd_fwd is persistent: items are (chunk, head,
+// batch row) with the chunk slowest, handed out by a ticket counter; the state
+// is carried between the chunks of a (b, h) through two fp32 slots in global
+// memory (L2), the same chain as the per-coordinate kernels.
+#include <cuda.h>
+
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace ssm {
+
+// Device word raised by the bounded waits of these kernels (0 = no error).
+__device__ int ssm_ssd_error_word;
+__device__ __forceinline__ void ssd_raise_error(int code) {
+    atomicCAS(&ssm_ssd_error_word, 0, code);
+}
+
+namespace ssdk {
+
+using namespace umma;
+using namespace chunkc;
+
+constexpr int ROWS = 128;                 // (token, rank) rows per chunk
+constexpr int THREADS = 512;
+constexpr uint32_t TILE = 16384;          // 128 rows x 128 bytes (64 bf16), 128-byte swizzle
+constexpr uint32_t TMEM_COLS = 256;       // CB 0..127 (then Y_o 0..63) | S_c 128.. | Y_d 192..
+constexpr uint32_t SM_X = 0;              // 2 x 16 KB x tiles (rows (t, r)), double-buffered
+constexpr uint32_t SM_B = 32768;          // 2 x 16 KB B (state rows 0-63 | 64-127), rows (t, r)
+constexpr uint32_t SM_C = 65536;          // 2 x 16 KB C, rows (t, o)
+constexpr uint32_t SM_P = 98304;          // 32 KB masked scores, no-swizzle K-major (rows j, K = i)
+constexpr uint32_t SM_XS = 131072;        // 16 KB diag(f) x, then the y tile
+constexpr uint32_t SM_K = 147456;         // 16 KB entering state, bf16 [n][p] (128-byte swizzle)
+constexpr uint32_t SM_F32 = 163840;
+// fp32 scratch (float offsets)
+constexpr int F_DT = 0;      // [129] dt of the chunk's tokens and of the token after it
+constexpr int F_LAM = 132;   // [129] lambda of the same tokens
+constexpr int F_S = 264;     // [128] inclusive cumulative sum of dt inside the chunk
+constexpr int F_SIG = 392;   // [128] sigma_t = gamma_t + beta_{t+1}
+constexpr int F_GAM = 520;   // [128] gamma_t
+constexpr int F_FW = 648;    // [128] f_t = e^{a (S_end - S_t)} sigma_t
+constexpr int F_EW = 776;    // [128] e_t = e^{a S_t}
+constexpr int F_SC = 904;    // [0] a log2(e), [1] D, [2] E = e^{a S_end}
+constexpr int F_END = 912;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 128 + 1024;
+static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
+
+// Tokens of one chunk: dt and lambda (bf16 bits) of tokens t0 .. t0 + Qt, loaded
+// one item ahead and converted when stored.
+struct Tok {
+    unsigned short dv, lv;
+};
+__device__ __forceinline__ Tok tok_load_q(const Params &p, int b, int h, int t0, int Qt) {
+    Tok r{0, 0x3f80};   // dt 0 (tokens past L add nothing), lambda 1
+    const int i = threadIdx.x, t = t0 + i;
+    if (i <= Qt && t < p.L) {
+        r.dv = __ldg(reinterpret_cast<const unsigned short *>(p.dt) + ix_dt(p, b, t, h));
+        if (p.two_ep)
+            r.lv = __ldg(reinterpret_cast<const unsigned short *>(p.lam) + ix_lam(p, b, t, h));
+    }
+    return r;
+}
+
+// Per-token quantities of the chunk (S, sigma, gamma, f, e) and E, from the
+// prefetched dt / lambda; contains barriers (all threads).
+__device__ __forceinline__ void chunk_scalars(const Params &p, float *f32, int t0, int Qt,
+                                              const Tok &r, float alog, float *fe = nullptr) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid <= Qt) {
+        f32[F_DT + tid] = __uint_as_float((uint32_t)r.dv << 16);
+        f32[F_LAM + tid] = __uint_as_float((uint32_t)r.lv << 16);
+    }
+    if (tid == 0) f32[F_SC] = -expf(alog) * 1.4426950408889634f;
+    __syncthreads();
+    if (warp == 0) {
+        // inclusive prefix of dt: lane l takes tokens [l * per, (l + 1) * per)
+        const int per = Qt >> 5;
+        float loc[4];
+        float run = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k < per) run += f32[F_DT + lane * per + k];
+            loc[k] = run;
+        }
+        float v = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        const float base = v - run;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < per) f32[F_S + lane * per + k] = base + loc[k];
+    } else if (tid >= 32 && tid < 32 + Qt) {
+        const int t = tid - 32;
+        const float dv = f32[F_DT + t], lv = f32[F_LAM + t];
+        const float bn = (t0 + t + 1 < p.L) ? (1.f - f32[F_LAM + t + 1]) * f32[F_DT + t + 1] : 0.f;
+        const float g = lv * dv;
+        f32[F_GAM + t] = g;
+        f32[F_SIG + t] = g + bn;
+    }
+    __syncthreads();
+    if (tid < Qt) {
+        const float a2 = f32[F_SC], se = f32[F_S + Qt - 1], st = f32[F_S + tid];
+        const float dend = ex2_fast(a2 * (se - st));
+        f32[F_FW + tid] = dend * f32[F_SIG + tid];
+        f32[F_EW + tid] = ex2_fast(a2 * st);
+        if (fe) fe[tid] = dend;
+        if (tid == 0) f32[F_SC + 2] = ex2_fast(a2 * se);
+    }
+    __syncthreads();
+}
+
+// K_in of thread (state row n, 16 columns from 16 cq): the carry slot, or
+// h0 + beta_0 w0 for the first chunk.
+__device__ __forceinline__ void load_kin(const Params &p, int c, int b, int h, int n, int cq,
+                                         float (&kc)[16]) {
+    if (n >= p.N) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) kc[j] = 0.f;
+        return;
+    }
+    if (c > 0) {
+        const float4 *src = carry_ptr(p, c & 1, b * p.H + h, cq, n);
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 v = __ldcg(src + j4 * NP);
+            kc[4 * j4] = v.x;
+            kc[4 * j4 + 1] = v.y;
+            kc[4 * j4 + 2] = v.z;
+            kc[4 * j4 + 3] = v.w;
+        }
+        return;
+    }
+    float beta0 = 0.f;
+    if (p.two_ep)
+        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
+        float a = p.h0 ? p.h0[i0] : 0.f;
+        if (p.w0) a = fmaf(beta0, p.w0[i0], a);
+        kc[j] = a;
+    }
+}
+
+// 8 bf16 of row `row`, logical 16-byte chunk `lc` of a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t sw_off(int row, int lc) {
+    return (uint32_t)row * 128u + ((uint32_t)(lc ^ (row & 7)) << 4);
+}
+__device__ __forceinline__ void unpack8(const uint4 w, float (&v)[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(u[i] << 16);
+        v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    return w;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+          const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+          Params p, int lgR) {
+    const int BH = p.Bsz * p.H;
+    const int nitems = p.nc * BH;
+    if ((int)blockIdx.x >= nitems) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + SM_F32);
+    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // [2] x stages
+    uint64_t *bar_b = bar_x + 2, *bar_c = bar_x + 3;               // B, C tiles
+    uint64_t *bar_cb = bar_x + 4, *bar_sc = bar_x + 5, *bar_y = bar_x + 6;   // MMA phases
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 7);
+    int *s_item = reinterpret_cast<int *>(bar_x + 8);               // [2] claimed tickets
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int N = p.N, L = p.L;
+    const int nbox = N / 64;
+    const int Qt = ROWS >> lgR;   // tokens per chunk
+    const bool want_y = p.y != nullptr;
+    const int qd = warp & 3, cb4 = warp >> 2;   // TMEM lane quarter, column block
+    const int row = 32 * qd + lane;             // TMEM lane = row of every M = 128 tile
+
+    auto issue_x = [&](int item, int st) {
+        const ChunkItem it = chunk_item_cs(p, item);
+        mbar_expect_tx(&bar_x[st], TILE);
+        tma_load_5d(sm + SM_X + st * TILE, &tmX, &bar_x[st], 0, 0, it.h, it.c * Qt, it.b);
+    };
+    auto issue_b = [&](int item) {
+        const ChunkItem it = chunk_item_cs(p, item);
+        mbar_expect_tx(bar_b, TILE * nbox);
+        for (int k = 0; k < nbox; ++k)
+            tma_load_5d(sm + SM_B + k * TILE, &tmB, bar_b, 64 * k, 0, it.h / p.hpg, it.c * Qt, it.b);
+    };
+    auto issue_c = [&](int item) {
+        const ChunkItem it = chunk_item_cs(p, item);
+        mbar_expect_tx(bar_c, TILE * nbox);
+        for (int k = 0; k < nbox; ++k)
+            tma_load_5d(sm + SM_C + k * TILE, &tmC, bar_c, 64 * k, 0, it.h / p.hpg, it.c * Qt, it.b);
+    };
+
+    PhaseCount pc_x[2] = {{0u, 0u}, {0u, 0u}}, pc_b = {0u, 0u}, pc_c = {0u, 0u};
+    PhaseCount pc_cb = {0u, 0u}, pc_sc = {0u, 0u}, pc_y = {0u, 0u};
+    if (tid == 0) {
+        for (int i = 0; i < 7; ++i) mbar_init(&bar_x[i], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+        if (want_y) tma_prefetch_desc(&tmY);
+        const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
+        s_item[0] = first;
+        issue_x(first, 0);
+        ++pc_x[0].issued;
+        issue_b(first);
+        ++pc_b.issued;
+        if (want_y) {   // C is read by the outputs only
+            issue_c(first);
+            ++pc_c.issued;
+        }
+    }
+    if (warp == 0) tmem_alloc(tslot, TMEM_COLS);
+    if (N < NP) {   // state rows 64-127 of B / C are never loaded: keep them zero
+        for (int i = tid; i < (int)(TILE / 16); i += THREADS) {
+            reinterpret_cast<uint4 *>(sm + SM_B + TILE)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4 *>(sm + SM_C + TILE)[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const uint32_t t_cb = tbase, t_yo = tbase, t_sc = tbase + 128u, t_yd = tbase + 192u;
+    const uint32_t lane_q = (32u * qd) << 16;
+    int item = s_item[0];
+    Tok tok;
+    float alog;
+    {
+        const ChunkItem it = chunk_item_cs(p, item);
+        tok = tok_load_q(p, it.b, it.h, it.c * Qt, Qt);
+        alog = __ldg(p.A_log + it.h * p.ndec);
+    }
+    bool aborted = false;
+
+    for (int k = 0; item < nitems; ++k) {
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
+        const int st = k & 1;
+        const ChunkItem it = chunk_item_cs(p, item);
+        const int c = it.c, h = it.h, b = it.b;
+        const int bh = b * p.H + h;
+        const int t0 = c * Qt;
+        unsigned char *sX = sm + SM_X + st * TILE;
+        // the previous item's y store has read the staging tile
+        if (tid == 0) bulk_wait_read_all();
+        chunk_scalars(p, f32, t0, Qt, tok, alog);
+        const int next = s_item[1];
+        if (next < nitems) {
+            const ChunkItem nx = chunk_item_cs(p, next);
+            tok = tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
+            alog = __ldg(p.A_log + nx.h * p.ndec);
+            // the other x stage was last read by the previous item, which is complete
+            if (tid == 0) {
+                issue_x(next, st ^ 1);
+                ++pc_x[st ^ 1].issued;
+            }
+        }
+        const bool okx = mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT);
+        const bool okb = okx && mbar_wait(bar_b, (uint32_t)(k & 1), WAIT_LIMIT);
+        const bool okc = okb && (!want_y || mbar_wait(bar_c, (uint32_t)(k & 1), WAIT_LIMIT));
+        if (tid == 0) {
+            pc_x[st].done += okx ? 1u : 0u;
+            pc_b.done += okb ? 1u : 0u;
+            pc_c.done += (want_y && okc) ? 1u : 0u;
+        }
+        int ok = okc ? 1 : 0;
+        if (!ok) {
+            ssd_raise_error(1);
+            chain_abort(p);
+        }
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        // ---- CB = C B^T ----------------------------------------------------------
+        if (tid == 0 && want_y) {
+            fence_after_sync();
+            const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
+            const uint32_t id = idesc_bf16(128, 128, false, false);
+            for (int s = 0; s < N / 16; ++s) {
+                const uint32_t off = (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u;
+                mma_bf16(t_cb, sdesc(c_base + off, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(b_base + off, 16u, 1024u, LAYOUT_SW128), id, s > 0);
+            }
+            mma_commit(bar_cb);
+            ++pc_cb.issued;
+        }
+        // ---- X' = diag(f) X (same swizzled positions) -------------------------------
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int ch = tid + THREADS * q;    // 16-byte chunk: row ch >> 3, position ch & 7
+            const int r = ch >> 3;
+            const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
+            const float f = f32[F_FW + (r >> lgR)];
+            float v[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sX + off), v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= f;
+            *reinterpret_cast<uint4 *>(sm + SM_XS + off) = pack8(v);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // ---- S_c = B^T X' (A = B read MN-major over both 64-row halves) ----------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t b_base = smem_u32(sm + SM_B), xs_base = smem_u32(sm + SM_XS);
+            const uint32_t id = idesc_bf16(128, 64, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(t_sc, sdesc(b_base + s * 2048u, TILE, 1024u, LAYOUT_SW128),
+                         sdesc(xs_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id, s > 0);
+            mma_commit(bar_sc);
+            ++pc_sc.issued;
+        }
+        if (want_y) {
+            // ---- masked scores P = CB (.) W -> bf16 tile ------------------------------
+            ok = mbar_wait(bar_cb, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_cb.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            fence_after_sync();
+            if (ok) {
+                float v[32];
+                tmem_ld16(t_cb + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(t_cb + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(v + 16));
+                const int tj = row >> lgR;
+                const float a2 = f32[F_SC], stj = f32[F_S + tj], gj = f32[F_GAM + tj];
+                const int i0 = 32 * cb4;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float w8[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int ti = (i0 + 8 * q8 + j) >> lgR;
+                        float wt = 0.f;
+                        if (ti < tj)
+                            wt = ex2_fast(a2 * (stj - f32[F_S + ti])) * f32[F_SIG + ti];
+                        else if (ti == tj)
+                            wt = gj;
+                        w8[j] = v[8 * q8 + j] * wt;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + SM_P + off_kmaj(row, i0 + 8 * q8, 128u, 2048u)) =
+                        pack8(w8);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+            // ---- Y_d = P X ------------------------------------------------------------
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t p_base = smem_u32(sm + SM_P), x_base = smem_u32(sX);
+                const uint32_t id = idesc_bf16(128, 64, false, true);
+                for (int s = 0; s < ROWS / 16; ++s)
+                    mma_bf16(t_yd, sdesc(p_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                             sdesc(x_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id, s > 0);
+            }
+        }
+        // ---- chain: K_out = E K_in + S_c -------------------------------------------
+        ok = mbar_wait(bar_sc, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
+        if (tid == 0) pc_sc.done += (uint32_t)ok;
+        if (!ok) {
+            ssd_raise_error(1);
+            chain_abort(p);
+        }
+        if (tid == 0 && ok && c > 0 &&
+            !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
+            ssd_raise_error(2);
+            chain_abort(p);
+            ok = 0;
+        }
+        fence_after_sync();
+        if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of K_in
+            aborted = true;
+            break;
+        }
+        // B and X' are consumed (CB and S_c complete): fetch the next item's B
+        if (tid == 0 && next < nitems) {
+            issue_b(next);
+            ++pc_b.issued;
+        }
+        {
+            const int n = row, cq = cb4;
+            float kc[16], sc[16];
+            load_kin(p, c, b, h, n, cq, kc);
+            tmem_ld16(t_sc + lane_q + 16u * cq, sc);
+            const float E = f32[F_SC + 2];
+            unsigned char *sv = p.ws_kp
+                ? reinterpret_cast<unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
+                : nullptr;
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float v = kc[8 * g8 + j];
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+                    lo[j] = v - hi[j];
+                }
+                const uint32_t off = sw_off(n, 2 * cq + g8);
+                const uint4 wh = pack8(hi);
+                *reinterpret_cast<uint4 *>(sm + SM_K + off) = wh;
+                if (sv) {
+                    *reinterpret_cast<uint4 *>(sv + off) = wh;
+                    *reinterpret_cast<uint4 *>(sv + TILE + off) = pack8(lo);
+                }
+            }
+            float kn[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) kn[j] = n < N ? fmaf(E, kc[j], sc[j]) : 0.f;
+            if (c + 1 < p.nc) {
+                float4 *dst = carry_ptr(p, (c + 1) & 1, bh, cq, n);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(kn[4 * j4], kn[4 * j4 + 1], kn[4 * j4 + 2],
+                                                      kn[4 * j4 + 3]));
+            } else if (n < N) {
+                // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write
+                // W_{L-1} = B_{L-1} u_{L-1} (summed over the R value rows)
+                const int g = h / p.hpg, tl = L - 1;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
+                    if (p.hT) p.hT[i0] = kn[j];
+                    if (p.wT) {
+                        float w = 0.f;
+                        for (int r = 0; r < p.R; ++r)
+                            w = fmaf(ld_io(p.Bm, ix_B(p, b, tl, g, r, n), 1),
+                                     ld_io(p.x, ix_x(p, b, tl, h, r, 16 * cq + j), 1), w);
+                        p.wT[i0] = w;
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // the carry of (b, h) is in place: let the next chunk's item go (off the issue path)
+        if (tid == THREADS - 32 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
+        if (want_y) {
+            // ---- Y_o = C K_in, then the epilogue -----------------------------------------
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t c_base = smem_u32(sm + SM_C), k_base = smem_u32(sm + SM_K);
+                const uint32_t id = idesc_bf16(128, 64, false, true);
+                for (int s = 0; s < N / 16; ++s)
+                    mma_bf16(t_yo,
+                             sdesc(c_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u,
+                                   16u, 1024u, LAYOUT_SW128),
+                             sdesc(k_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id, s > 0);
+                mma_commit(bar_y);
+                ++pc_y.issued;
+            }
+            ok = mbar_wait(bar_y, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_y.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+            // C is consumed: fetch the next item's
+            if (tid == 0 && next < nitems) {
+                issue_c(next);
+                ++pc_c.issued;
+            }
+            {
+                float yd[16], yo[16];
+                tmem_ld16(t_yd + lane_q + 16u * cb4, yd);
+                tmem_ld16(t_yo + lane_q + 16u * cb4, yo);
+                const float e = f32[F_EW + (row >> lgR)];
+                const float D = (p.R == p.O && p.D) ? __ldg(p.D + h) : 0.f;
+#pragma unroll
+                for (int g8 = 0; g8 < 2; ++g8) {
+                    const uint32_t off = sw_off(row, 2 * cb4 + g8);
+                    float xv[8], yv[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sX + off), xv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        yv[j] = fmaf(D, xv[j], fmaf(e, yo[8 * g8 + j], yd[8 * g8 + j]));
+                    *reinterpret_cast<uint4 *>(sm + SM_XS + off) = pack8(yv);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {   // rows past the sequence end are clipped by the store
+                tma_store_5d(&tmY, sm + SM_XS, 0, 0, h, t0, b);
+                bulk_commit();
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        item = next;
+    }
+    if (tid == 0) bulk_wait_read_all();
+    if (aborted && tid == 0) {
+        drain_phases(&bar_x[0], pc_x[0]);
+        drain_phases(&bar_x[1], pc_x[1]);
+        drain_phases(bar_b, pc_b);
+        drain_phases(bar_c, pc_c);
+        drain_phases(bar_cb, pc_cb);
+        drain_phases(bar_sc, pc_sc);
+        drain_phases(bar_y, pc_y);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, TMEM_COLS);
+    }
+}
+
+}  // namespace ssdk
+
+// ============================================================================
+// k_ssd_bwd: reverse-mode of one chunk per work item, chunks of a (b, h) walked
+// last to first and chained through the adjoint G = dL/dK carried between them
+// (two fp32 slots in L2, the same chain as the forward).  With dS = dY X^T,
+// w the mask weights and G_out the adjoint of the chunk's end state:
+//     dX  = P^T dY + diag(f) B G_out + D dY
+//     dB  = (dS (.) W)^T C + diag(f) X G_out^T
+//     dC  = (dS (.) W) B + diag(e) dY K_in^T
+//     G_in = E G_out + C^T diag(e) dY
+// and the gradient of the log-decay rho_u = a dt_u of token u is, exactly,
+// the sum over the (write, read) pairs that step u lies between:
+//     drho_u = sum_{t_i < u <= t_j} Z[j, i]              (Z = dS (.) CB (.) W)
+//            + sum_{t_j >= u} R[j] + sum_{t_i < u} F[i] + Q
+// with R[j] = <dY_j, e_j (C K_in)_j> (the entering state read in the chunk),
+// F[i] = f_i <X_i, (B G_out)_i> (writes read after the chunk) and
+// Q = <G_out, E K_in> (the entering state read after the chunk).  dsigma_t and
+// the gamma_t part of the diagonal go to a per-token workspace for the
+// token pass (k_ssd_tokens).  Tensor cores (M = 128):
+//   phase 1: CB = C B^T, dS = dY X^T, dC <- diag(e) dY K_in^T, G_loc = C^T diag(e) dY
+//   phase 2: dX_d = P^T dY, dC += (dS (.) W) B, dB = (dS (.) W)^T C
+//   phase 3 (after the chain step): dX_s = B G_out, dB += diag(f) X G_out^T
+// ============================================================================
+namespace ssdb {
+using ssdk::F_DT;
+using ssdk::F_EW;
+using ssdk::F_FW;
+using ssdk::F_GAM;
+using ssdk::F_LAM;
+using ssdk::F_S;
+using ssdk::F_SC;
+using ssdk::F_SIG;
+using ssdk::ROWS;
+using ssdk::TILE;
+
+constexpr int THREADS = 512;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_CB = 0, T_DB = 0;       // CB, then dB (128 columns)
+constexpr uint32_t T_DS = 128, T_DXS = 128;  // dS, then dX_s (64)
+constexpr uint32_t T_DC = 256;               // diag(e) dY K_in^T, then dC (128)
+constexpr uint32_t T_GL = 384;               // G_loc (64)
+constexpr uint32_t T_DXD = 448;              // dX_d (64)
+constexpr uint32_t SM_X = 0;         // 16 KB x (rows (t, r))
+constexpr uint32_t SM_DY = 16384;    // 16 KB dy (rows (t, o))
+constexpr uint32_t SM_B = 32768;     // 2 x 16 KB B
+constexpr uint32_t SM_C = 65536;     // 2 x 16 KB C
+constexpr uint32_t SM_K = 98304;     // 16 KB K_in (bf16 hi tile [n][p])
+constexpr uint32_t SM_P = 114688;    // 32 KB P; then diag(f) X (16 KB) + G_out [n][p] (16 KB); then dB
+constexpr uint32_t SM_DCB = 147456;  // 32 KB dS (.) W; then dC
+constexpr uint32_t SM_DYS = 180224;  // 16 KB diag(e) dy, then dx
+constexpr uint32_t SM_F32 = 196608;
+constexpr int F_FE = 912;            // [128] e^{a (S_end - S_t)}
+constexpr int F_RED = 1040;          // [6][4][128] partial row / column sums
+constexpr int R_ROWZ = 0, R_DIAG = 512, R_ROFF = 1024, R_COLZ = 1536, R_WQ = 2048, R_DD = 2560;
+constexpr int F_QB = F_RED + 3072;   // [16] per-warp partials of Q, then [16] of dbeta_0
+constexpr int F_END = F_QB + 32;
+constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 128 + 1024;
+static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
+}  // namespace ssdb
+
+__global__ void __launch_bounds__(ssdb::THREADS, 1)
+k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDY,
+          const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+          const __grid_constant__ CUtensorMap tmDX, const __grid_constant__ CUtensorMap tmDB,
+          const __grid_constant__ CUtensorMap tmDC, Params p, int lgR) {
+    using namespace ssdb;
+    using namespace umma;
+    using chunkc::bhc;
+    using chunkc::carry_ptr;
+    using chunkc::chain_abort;
+    using chunkc::chain_abort_word;
+    using chunkc::chain_ticket;
+    using chunkc::ChunkItem;
+    using chunkc::chunk_item_rcs;
+    using chunkc::drain_phases;
+    using chunkc::ex2_fast;
+    using chunkc::NP;
+    using chunkc::PhaseCount;
+    using chunkc::publish_count;
+    using chunkc::SLOT_FLOATS;
+    using chunkc::wait_count;
+    using chunkc::WAIT_LIMIT;
+    using ssdk::pack8;
+    using ssdk::sw_off;
+    using ssdk::unpack8;
+    const int BH = p.Bsz * p.H;
+    const int nitems = p.nc * BH;
+    if ((int)blockIdx.x >= nitems) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + SM_F32);
+    float *red = f32 + F_RED;
+    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // x + dy
+    uint64_t *bar_k = bar_x + 1, *bar_bc = bar_x + 2;                 // K_in; B + C
+    uint64_t *bar_p1 = bar_x + 3, *bar_p2 = bar_x + 4, *bar_p3 = bar_x + 5;   // MMA phases
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 6);
+    int *s_item = reinterpret_cast<int *>(bar_x + 7);                // [2] claimed tickets
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int N = p.N, L = p.L;
+    const int nbox = N / 64;
+    const int Qt = ROWS >> lgR;
+    const int Rm = (1 << lgR) - 1;
+    const bool one_head = p.hpg == 1;
+    const int qd = warp & 3, cb4 = warp >> 2;
+    const int row = 32 * qd + lane;
+    const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+
+    auto issue_x = [&](int item) {
+        const ChunkItem it = chunk_item_rcs(p, item);
+        mbar_expect_tx(bar_x, 2 * TILE);
+        tma_load_5d(sm + SM_X, &tmX, bar_x, 0, 0, it.h, it.c * Qt, it.b);
+        tma_load_5d(sm + SM_DY, &tmDY, bar_x, 0, 0, it.h, it.c * Qt, it.b);
+    };
+    auto issue_k = [&](int item) {
+        const ChunkItem it = chunk_item_rcs(p, item);
+        mbar_expect_tx(bar_k, TILE);
+        bulk_load(sm + SM_K, p.ws_kp + bhc(p, it.b, it.h, it.c) * SLOT_FLOATS, TILE, bar_k);
+    };
+    auto issue_bc = [&](int item) {
+        const ChunkItem it = chunk_item_rcs(p, item);
+        const int g = it.h / p.hpg;
+        mbar_expect_tx(bar_bc, 2 * TILE * nbox);
+        for (int k = 0; k < nbox; ++k) {
+            tma_load_5d(sm + SM_B + k * TILE, &tmB, bar_bc, 64 * k, 0, g, it.c * Qt, it.b);
+            tma_load_5d(sm + SM_C + k * TILE, &tmC, bar_bc, 64 * k, 0, g, it.c * Qt, it.b);
+        }
+    };
+
+    PhaseCount pc_x = {0u, 0u}, pc_k = {0u, 0u}, pc_bc = {0u, 0u};
+    PhaseCount pc_1 = {0u, 0u}, pc_2 = {0u, 0u}, pc_3 = {0u, 0u};
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(&bar_x[i], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmDY);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+        const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
+        s_item[0] = first;
+        issue_x(first);
+        ++pc_x.issued;
+        issue_k(first);
+        ++pc_k.issued;
+        issue_bc(first);
+        ++pc_bc.issued;
+    }
+    if (warp == 0) tmem_alloc(tslot, TMEM_COLS);
+    if (N < NP) {   // state rows 64-127 of B / C are never loaded: keep them zero
+        for (int i = tid; i < (int)(TILE / 16); i += THREADS) {
+            reinterpret_cast<uint4 *>(sm + SM_B + TILE)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4 *>(sm + SM_C + TILE)[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tb = *tslot;
+    int item = s_item[0];
+    ssdk::Tok tok;
+    float alog;
+    {
+        const ChunkItem it = chunk_item_rcs(p, item);
+        tok = ssdk::tok_load_q(p, it.b, it.h, it.c * Qt, Qt);
+        alog = __ldg(p.A_log + it.h * p.ndec);
+    }
+    bool aborted = false;
+
+    for (int k = 0; item < nitems; ++k) {
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
+        const uint32_t par = (uint32_t)(k & 1);
+        const ChunkItem it = chunk_item_rcs(p, item);
+        const int c = it.c, h = it.h, b = it.b;
+        const int g = h / p.hpg;
+        const int bh = b * p.H + h, rr = p.nc - 1 - c;   // chunks of (b, h) walked before this one
+        const int t0 = c * Qt;
+        const long long u = bhc(p, b, h, c);
+        // the previous item's stores have read their staging tiles
+        if (tid == 0) bulk_wait_read_all();
+        ssdk::chunk_scalars(p, f32, t0, Qt, tok, alog, f32 + F_FE);
+        const int next = s_item[1];
+        if (next < nitems) {
+            const ChunkItem nx = chunk_item_rcs(p, next);
+            tok = ssdk::tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
+            alog = __ldg(p.A_log + nx.h * p.ndec);
+        }
+        const float a2 = f32[F_SC], E = f32[F_SC + 2];
+        {
+            const bool o1 = mbar_wait(bar_x, par, WAIT_LIMIT);
+            const bool o2 = o1 && mbar_wait(bar_k, par, WAIT_LIMIT);
+            const bool o3 = o2 && mbar_wait(bar_bc, par, WAIT_LIMIT);
+            if (tid == 0) {
+                pc_x.done += o1 ? 1u : 0u;
+                pc_k.done += o2 ? 1u : 0u;
+                pc_bc.done += o3 ? 1u : 0u;
+            }
+            int ok = o3 ? 1 : 0;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+        }
+        // ---- phase 1a: CB = C B^T, dS = dY X^T --------------------------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
+            const uint32_t x_base = smem_u32(sm + SM_X), dy_base = smem_u32(sm + SM_DY);
+            const uint32_t id128 = idesc_bf16(128, 128, false, false);
+            for (int s = 0; s < N / 16; ++s) {
+                const uint32_t off = (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u;
+                mma_bf16(tb + T_CB, sdesc(c_base + off, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(b_base + off, 16u, 1024u, LAYOUT_SW128), id128, s > 0);
+            }
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tb + T_DS, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id128, s > 0);
+        }
+        // diag(e) dy (same swizzled positions)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int ch = tid + THREADS * q;
+            const int r = ch >> 3;
+            const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
+            const float e = f32[F_EW + (r >> lgR)];
+            float v[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sm + SM_DY + off), v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= e;
+            *reinterpret_cast<uint4 *>(sm + SM_DYS + off) = pack8(v);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // ---- phase 1b: dC <- diag(e) dY K_in^T, G_loc = C^T diag(e) dY ----------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t c_base = smem_u32(sm + SM_C), k_base = smem_u32(sm + SM_K);
+            const uint32_t dys_base = smem_u32(sm + SM_DYS);
+            const uint32_t id128 = idesc_bf16(128, 128, false, false);
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tb + T_DC, sdesc(dys_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(k_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id128, s > 0);
+            const uint32_t id64 = idesc_bf16(128, 64, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_GL, sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128),
+                         sdesc(dys_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id64, s > 0);
+            mma_commit(bar_p1);
+            ++pc_1.issued;
+        }
+        {
+            int ok = mbar_wait(bar_p1, par, WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_1.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            fence_after_sync();
+            if (ok) {
+                // ---- masking: P = CB (.) W, dCB = dS (.) W, the sums of Z, and R ----------
+                float cbv[32], dsv[32], colz[32];
+                tmem_ld16(tb + T_CB + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(cbv));
+                tmem_ld16(tb + T_CB + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(cbv + 16));
+                tmem_ld16(tb + T_DS + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(dsv));
+                tmem_ld16(tb + T_DS + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(dsv + 16));
+                const int tj = row >> lgR;
+                const float stj = f32[F_S + tj], gj = f32[F_GAM + tj];
+                const int i0 = 32 * cb4;
+                float rowz = 0.f, diag = 0.f;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float pv[8], dv[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int kk = 8 * q8 + j;
+                        const int ti = (i0 + kk) >> lgR;
+                        const float cb = cbv[kk], ds = dsv[kk];
+                        float z = 0.f, pw = 0.f, dw = 0.f;
+                        if (ti < tj) {
+                            const float wd = ex2_fast(a2 * (stj - f32[F_S + ti]));
+                            const float sg = f32[F_SIG + ti];
+                            z = ds * cb * wd;             // per unit sigma
+                            rowz = fmaf(z, sg, rowz);
+                            pw = cb * wd * sg;
+                            dw = ds * wd * sg;
+                        } else if (ti == tj) {
+                            diag = fmaf(ds, cb, diag);
+                            pw = cb * gj;
+                            dw = ds * gj;
+                        }
+                        colz[kk] = z;
+                        pv[j] = pw;
+                        dv[j] = dw;
+                    }
+                    const uint32_t off = off_kmaj(row, i0 + 8 * q8, 128u, 2048u);
+                    *reinterpret_cast<uint4 *>(sm + SM_P + off) = pack8(pv);
+                    *reinterpret_cast<uint4 *>(sm + SM_DCB + off) = pack8(dv);
+                }
+                xreduce<32, 32>(colz, lane);   // lane l: column i0 + l over the warp's 32 rows
+                red[R_COLZ + qd * 128 + i0 + lane] = colz[0];
+                red[R_ROWZ + cb4 * 128 + row] = rowz;
+                red[R_DIAG + cb4 * 128 + row] = diag;
+                // R[j] = sum_n C[j][n] (diag(e) dY K_in^T)[j][n] over this thread's 32 n
+                float dcs[32];
+                tmem_ld16(tb + T_DC + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(dcs));
+                tmem_ld16(tb + T_DC + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(dcs + 16));
+                const unsigned char *ct = sm + SM_C + (cb4 >> 1) * TILE;
+                float roff = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float cv[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(ct + sw_off(row, 4 * (cb4 & 1) + q)), cv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) roff = fmaf(cv[j], dcs[8 * q + j], roff);
+                }
+                red[R_ROFF + cb4 * 128 + row] = roff;
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+        }
+        // ---- phase 2: dX_d = P^T dY, dC += dCB B, dB = dCB^T C ------------------------
+        if (tid == 0) {
+            fence_after_sync();
+            // K_in is consumed: fetch the next item's
+            if (next < nitems) {
+                issue_k(next);
+                ++pc_k.issued;
+            }
+            const uint32_t p_base = smem_u32(sm + SM_P), dcb_base = smem_u32(sm + SM_DCB);
+            const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
+            const uint32_t dy_base = smem_u32(sm + SM_DY);
+            const uint32_t id_x = idesc_bf16(128, 64, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DXD, sdesc(p_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                         sdesc(dy_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_x, s > 0);
+            const uint32_t id_c = idesc_bf16(128, 128, false, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DC, sdesc(dcb_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                         sdesc(b_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_c, true);
+            const uint32_t id_b = idesc_bf16(128, 128, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DB, sdesc(dcb_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                         sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_b, s > 0);
+            mma_commit(bar_p2);
+            ++pc_2.issued;
+        }
+        {
+            int ok = mbar_wait(bar_p2, par, WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_2.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            // the adjoint leaving this chunk is published by the item of chunk c + 1
+            if (tid == 0 && ok && rr > 0 &&
+                !wait_count(p.ws_flag + bh, rr, chain_abort_word(p), p.wait_limit)) {
+                ssd_raise_error(2);
+                chain_abort(p);
+                ok = 0;
+            }
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of G_out
+                aborted = true;
+                break;
+            }
+        }
+        // ---- diag(f) X into P's place (phase 2 has read P) --------------------------
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int ch = tid + THREADS * q;
+            const int r = ch >> 3;
+            const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
+            const float f = f32[F_FW + (r >> lgR)];
+            float v[8];
+            unpack8(*reinterpret_cast<const uint4 *>(sm + SM_X + off), v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= f;
+            *reinterpret_cast<uint4 *>(sm + SM_P + off) = pack8(v);
+        }
+        // ---- chain step: G_in = E G_out + G_loc; Q = <G_out, E K_in> ------------------
+        {
+            const int n = row, cq = cb4;
+            float go[16], gl[16];
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rr > 0 && n < N) a4 = __ldcg(carry_ptr(p, rr & 1, bh, cq, n) + j4 * NP);
+                go[4 * j4] = a4.x;
+                go[4 * j4 + 1] = a4.y;
+                go[4 * j4 + 2] = a4.z;
+                go[4 * j4 + 3] = a4.w;
+            }
+            tmem_ld16(tb + T_GL + lane_q + 16u * cq, gl);
+            const unsigned char *kslot =
+                reinterpret_cast<const unsigned char *>(p.ws_kp + u * SLOT_FLOATS);
+            float qb = 0.f;
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const uint32_t off = sw_off(n, 2 * cq + g8);
+                float gh[8], kh[8], kl[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) gh[j] = go[8 * g8 + j];
+                *reinterpret_cast<uint4 *>(sm + SM_P + TILE + off) = pack8(gh);
+                // K_in hi / lo from the chunk's slot (the next item's K_in may be landing in
+                // the shared-memory copy already)
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(kslot + off)), kh);
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(kslot + TILE + off)), kl);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) qb = fmaf(gh[j], kh[j] + kl[j], qb);
+            }
+            float gi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) gi[j] = n < N ? fmaf(E, go[j], gl[j]) : 0.f;
+            float db0 = 0.f;
+            if (c > 0) {
+                float4 *dst = carry_ptr(p, (rr + 1) & 1, bh, cq, n);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(gi[4 * j4], gi[4 * j4 + 1], gi[4 * j4 + 2],
+                                                      gi[4 * j4 + 3]));
+            } else if (n < N) {
+                // the adjoint of K_{-1} = h0 + beta_0 w0: dh0, dw0 = beta_0 dh0, dbeta_0
+                float beta0 = 0.f;
+                if (p.two_ep)
+                    beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
+                    if (p.dh0) p.dh0[i0] = gi[j];
+                    if (p.dw0) p.dw0[i0] = beta0 * gi[j];
+                    if (p.w0) db0 = fmaf(gi[j], p.w0[i0], db0);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                qb += __shfl_xor_sync(0xffffffffu, qb, o);
+                db0 += __shfl_xor_sync(0xffffffffu, db0, o);
+            }
+            if (lane == 0) {
+                f32[F_QB + warp] = qb;
+                f32[F_QB + 16 + warp] = db0;
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // the carry of chunk c - 1 is in place: let its item go (off the issue path)
+        if (tid == THREADS - 32 && c > 0) publish_count(p.ws_flag + bh, rr + 1);
+        // ---- phase 3: dX_s = B G_out, dB += diag(f) X G_out^T ---------------------------
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t b_base = smem_u32(sm + SM_B), xs_base = smem_u32(sm + SM_P);
+            const uint32_t g_base = smem_u32(sm + SM_P + TILE);
+            const uint32_t id_x = idesc_bf16(128, 64, false, true);
+            for (int s = 0; s < N / 16; ++s)
+                mma_bf16(tb + T_DXS,
+                         sdesc(b_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u, 16u,
+                               1024u, LAYOUT_SW128),
+                         sdesc(g_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_x, s > 0);
+            const uint32_t id_b = idesc_bf16(128, 128, false, false);
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tb + T_DB, sdesc(xs_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                         sdesc(g_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_b, true);
+            mma_commit(bar_p3);
+            ++pc_3.issued;
+        }
+        {
+            int ok = mbar_wait(bar_p3, par, WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_3.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+        }
+        // B and C are consumed: fetch the next item's
+        if (tid == 0 && next < nitems) {
+            issue_bc(next);
+            ++pc_bc.issued;
+        }
+        // ---- epilogue: dx (into the e dy tile), dB (into P's place), dC (into dCB's) ----
+        {
+            const int ti = row >> lgR;
+            const float f = f32[F_FW + ti];
+            const float D = (p.R == p.O && p.D) ? __ldg(p.D + h) : 0.f;
+            float dxd[16], dxs[16];
+            tmem_ld16(tb + T_DXD + lane_q + 16u * cb4, dxd);
+            tmem_ld16(tb + T_DXS + lane_q + 16u * cb4, dxs);
+            float wq = 0.f, dd = 0.f;
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const uint32_t off = sw_off(row, 2 * cb4 + g8);
+                float xv[8], dyv[8], o8[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + SM_X + off), xv);
+                unpack8(*reinterpret_cast<const uint4 *>(sm + SM_DY + off), dyv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float s_ = dxs[8 * g8 + j];
+                    wq = fmaf(xv[j], s_, wq);
+                    dd = fmaf(dyv[j], xv[j], dd);
+                    o8[j] = fmaf(D, dyv[j], fmaf(f, s_, dxd[8 * g8 + j]));
+                }
+                *reinterpret_cast<uint4 *>(sm + SM_DYS + off) = pack8(o8);
+            }
+            red[R_WQ + cb4 * 128 + row] = wq;
+            red[R_DD + cb4 * 128 + row] = dd;
+            const bool tvalid = t0 + ti < L;
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t tcol = half ? T_DC : T_DB;
+                float v[32];
+                tmem_ld16(tb + tcol + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(tb + tcol + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(v + 16));
+                const int n0 = 32 * cb4;
+                if (one_head) {
+                    unsigned char *stg = sm + (half ? SM_DCB : SM_P) + (cb4 >> 1) * TILE;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float o8[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o8[j] = v[8 * q + j];
+                        *reinterpret_cast<uint4 *>(stg + sw_off(row, 4 * (cb4 & 1) + q)) = pack8(o8);
+                    }
+                } else if (tvalid && n0 < N) {
+                    float *dst = (half ? p.sd_dCh : p.sd_dBh) +
+                                 ix_wsk(p, b, t0 + ti, h, row & Rm, p.R, n0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        reinterpret_cast<float4 *>(dst)[q] =
+                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {   // rows past the sequence end are clipped by the stores
+            tma_store_5d(&tmDX, sm + SM_DYS, 0, 0, h, t0, b);
+            if (one_head)
+                for (int kb = 0; kb < nbox; ++kb) {
+                    tma_store_5d(&tmDB, sm + SM_P + kb * TILE, 64 * kb, 0, g, t0, b);
+                    tma_store_5d(&tmDC, sm + SM_DCB + kb * TILE, 64 * kb, 0, g, t0, b);
+                }
+            bulk_commit();
+        } else if (warp == 1) {
+            // ---- per-token sums and the drho scans (one warp; lane: Qt / 32 tokens) --------
+            const int per = Qt >> 5;
+            const int R = 1 << lgR;
+            float qb = 0.f, db0 = 0.f;
+            for (int w = 0; w < THREADS / 32; ++w) {
+                qb += f32[F_QB + w];
+                db0 += f32[F_QB + 16 + w];
+            }
+            qb *= E;
+            float cz[4], rz[4], dg[4], ro[4], wf[4], dsg[4];
+            float tot_in = 0.f, tot_w = 0.f, tot_r = 0.f;
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                cz[kq] = rz[kq] = dg[kq] = ro[kq] = wf[kq] = dsg[kq] = 0.f;
+                if (kq >= per) continue;
+                const int t = lane * per + kq;
+                float czs = 0.f, wq = 0.f;
+                for (int j = t * R; j < t * R + R; ++j) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        rz[kq] += red[R_ROWZ + q * 128 + j];
+                        dg[kq] += red[R_DIAG + q * 128 + j];
+                        ro[kq] += red[R_ROFF + q * 128 + j];
+                        czs += red[R_COLZ + q * 128 + j];
+                        wq += red[R_WQ + q * 128 + j];
+                    }
+                }
+                cz[kq] = czs * f32[F_SIG + t];
+                wf[kq] = wq * f32[F_FW + t];
+                dsg[kq] = czs + wq * f32[F_FE + t];
+                tot_in += cz[kq] - rz[kq];
+                tot_w += wf[kq];
+                tot_r += ro[kq];
+            }
+            // exclusive prefix over lanes of (colZ - rowZ) and F; suffix of R
+            float pin = tot_in, pw = tot_w, sr = tot_r;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float a_ = __shfl_up_sync(0xffffffffu, pin, o);
+                const float b_ = __shfl_up_sync(0xffffffffu, pw, o);
+                const float c_ = __shfl_down_sync(0xffffffffu, sr, o);
+                if (lane >= o) {
+                    pin += a_;
+                    pw += b_;
+                }
+                if (lane + o < 32) sr += c_;
+            }
+            float run_in = pin - tot_in, run_w = pw - tot_w, run_r = sr;   // suffix includes own
+            float sdr = 0.f, sdd = 0.f;
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                if (kq >= per) continue;
+                const int t = lane * per + kq;
+                const float drho = run_in + run_w + run_r + qb;
+                run_in += cz[kq] - rz[kq];
+                run_w += wf[kq];
+                run_r -= ro[kq];
+                if (t0 + t < L) {
+                    float *dst = p.sd_tok + 3 * ix_bth(p, b, t0 + t, h);
+                    dst[0] = dsg[kq];
+                    dst[1] = dg[kq];
+                    dst[2] = drho;
+                    sdr = fmaf(f32[F_DT + t], drho, sdr);
+                }
+            }
+            for (int j = lane; j < ROWS; j += 32)
+                if (t0 + (j >> lgR) < L)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sdd += red[R_DD + q * 128 + j];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                sdr += __shfl_xor_sync(0xffffffffu, sdr, o);
+                sdd += __shfl_xor_sync(0xffffffffu, sdd, o);
+            }
+            if (lane == 0) {
+                p.sd_par[2 * u] = sdr;
+                p.sd_par[2 * u + 1] = sdd;
+                if (c == 0) p.sd_db0[bh] = db0;
+            }
+        }
+        // x and dy are consumed: fetch the next item's
+        if (tid == 0 && next < nitems) {
+            issue_x(next);
+            ++pc_x.issued;
+        }
+        fence_before_sync();
+        __syncthreads();
+        item = next;
+    }
+    if (tid == 0) bulk_wait_read_all();
+    if (aborted && tid == 0) {
+        drain_phases(bar_x, pc_x);
+        drain_phases(bar_k, pc_k);
+        drain_phases(bar_bc, pc_bc);
+        drain_phases(bar_p1, pc_1);
+        drain_phases(bar_p2, pc_2);
+        drain_phases(bar_p3, pc_3);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tb, TMEM_COLS);
+    }
+}
+
+// Per-token gradients of the scalar-decay backward: dgamma_t = dsigma_t +
+// diag_t, dbeta_t = dsigma_{t-1} (dbeta_0 from the chain), then
+//   ddt_t = lam_t dgamma_t + (1 - lam_t) dbeta_t + a drho_t,
+//   dlambda_t = dt_t (dgamma_t - dbeta_t).
+__global__ void k_ssd_tokens(Params p) {
+    const long long total = (long long)p.Bsz * p.L * p.H;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int h = (int)(i % p.H);
+        const long long r = i / p.H;
+        const int t = (int)(r % p.L), b = (int)(r / p.L);
+        const float *tk = p.sd_tok + 3 * ix_bth(p, b, t, h);
+        const float a = -expf(__ldg(p.A_log + h * p.ndec));
+        const float dgam = tk[0] + tk[1];
+        const float dtv = ld_io(p.dt, ix_dt(p, b, t, h), 1);
+        float ddt = fmaf(a, tk[2], dgam);
+        if (p.two_ep) {
+            const float dbet = t > 0 ? p.sd_tok[3 * ix_bth(p, b, t - 1, h)] : p.sd_db0[b * p.H + h];
+            const float lam = ld_io(p.lam, ix_lam(p, b, t, h), 1);
+            ddt = fmaf(a, tk[2], fmaf(lam, dgam, (1.f - lam) * dbet));
+            if (p.dlam) st_io(p.dlam, ix_lam(p, b, t, h), dtv * (dgam - dbet), 1);
+        }
+        st_io(p.ddt, ix_dt(p, b, t, h), ddt, 1);
+    }
+}
+
+// Per-head parameter gradients (fixed summation order over batch rows and
+// chunks): dA_log = a sum dt drho, dD = sum <dy, x>.
+__global__ void k_ssd_params(Params p) {
+    for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < p.H; h += gridDim.x * blockDim.x) {
+        float sa = 0.f, sd = 0.f;
+        for (int b = 0; b < p.Bsz; ++b)
+            for (int c = 0; c < p.nc; ++c) {
+                const long long u = chunkc::bhc(p, b, h, c);
+                sa += p.sd_par[2 * u];
+                sd += p.sd_par[2 * u + 1];
+            }
+        const float a = -expf(__ldg(p.A_log + h * p.ndec));
+        p.dA_log[h * p.ndec] = a * sa;
+        if (p.dD) p.dD[h] = sd;
+    }
+}
+
+// dB / dC of groups with several heads: the fixed-order sum of the per-head parts.
+__global__ void k_ssd_group_sum(Params p) {
+    const int RN = p.R * p.N;
+    const long long total = (long long)p.Bsz * p.L * p.G * RN;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int e = (int)(i % RN);
+        const long long r = i / RN;
+        const int g = (int)(r % p.G);
+        const long long r2 = r / p.G;
+        const int t = (int)(r2 % p.L), b = (int)(r2 / p.L);
+        const int rr = e / p.N, n = e % p.N;
+        float sb = 0.f, sc = 0.f;
+        for (int k = 0; k < p.hpg; ++k) {
+            const int h = g * p.hpg + k;
+            sb += p.sd_dBh[ix_wsk(p, b, t, h, rr, p.R, n)];
+            sc += p.sd_dCh[ix_wsk(p, b, t, h, rr, p.O, n)];
+        }
+        st_io(p.dBm, ix_B(p, b, t, g, rr, n), sb, 1);
+        st_io(p.dCm, ix_C(p, b, t, g, rr, n), sc, 1);
+    }
+}
+
+namespace ssdk {
+
+// 5-D bf16 map over (inner, rank, head-or-group, time, batch), box
+// (64, rank, 1, tokens, 1), 128-byte swizzle: one box is the chunk's 128
+// (token, rank) rows of 64 elements.
+static bool make_map5(CUtensorMap *m, const void *base, uint64_t inner, uint64_t R, uint64_t d2,
+                      uint64_t L, uint64_t B, uint64_t sR, uint64_t s2, uint64_t sL, uint64_t sB,
+                      uint32_t Qt) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[5] = {inner, R, d2, L, B};
+    cuuint64_t strides[4] = {sR * 2, s2 * 2, sL * 2, sB * 2};
+    cuuint32_t box[5] = {64, (cuuint32_t)R, 1, Qt, 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+}  // namespace ssdk
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+int sm_count();
+
+static int ssd_lg_rank(int R) { return R == 1 ? 0 : (R == 2 ? 1 : (R == 4 ? 2 : -1)); }
+
+// Tokens per chunk of the scalar-decay kernels (128 (token, rank) rows).
+int ssd_chunk_tokens(int R) {
+    const int lg = ssd_lg_rank(R);
+    return lg < 0 ? 0 : (ssdk::ROWS >> lg);
+}
+
+// Shapes the scalar-decay kernels take (alignment of the call's pointers and
+// strides included).
+bool ssd_supported(const Params &p) {
+    auto al16 = [](const void *ptr) { return ptr == nullptr || ((uintptr_t)ptr & 15) == 0; };
+    auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
+    return p.bf16 && !p.per_coord && p.np == 0 && p.P == 64 && (p.N == 64 || p.N == 128) &&
+           p.R == p.O && ssd_lg_rank(p.R) >= 0 && p.L > 0 && al16(p.x) && al16(p.Bm) &&
+           al16(p.Cm) && al16(p.y) && st16(p.sx[0]) && st16(p.sx[1]) && st16(p.sx[2]) &&
+           st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]) && st16(p.sB[0]) && st16(p.sB[1]) &&
+           st16(p.sB[2]) && st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) &&
+           chunkc::encode_fn() != nullptr;
+}
+
+template <typename K>
+static cudaError_t ssd_set_smem(K kern, uint32_t bytes, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    return e;
+}
+
+// Forward of the scalar-decay path: y (when p.y is set), hT / last write, and
+// with p.ws_kp the state entering every chunk (bf16 hi / lo tiles) for the
+// backward.  Needs p.ws_ring, p.ws_flag and p.nc = chunks of ssd_chunk_tokens.
+cudaError_t ssd_forward(const Params &p, cudaStream_t st) {
+    using namespace ssdk;
+    const int lgR = ssd_lg_rank(p.R);
+    const uint32_t Qt = (uint32_t)(ROWS >> lgR);
+    CUtensorMap mx, mb, mc, my;
+    if (!make_map5(&mx, p.x, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
+        !make_map5(&mb, p.Bm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+        !make_map5(&mc, p.Cm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt))
+        return cudaErrorInvalidValue;
+    my = mx;
+    if (p.y &&
+        !make_map5(&my, p.y, 64, p.O, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt))
+        return cudaErrorInvalidValue;
+    if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
+    static bool done[64] = {};
+    cudaError_t e;
+    if ((e = ssd_set_smem(k_ssd_fwd, SMEM_BYTES, done)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
+        cudaSuccess)
+        return e;
+    const long long nitems = (long long)p.nc * p.H * p.Bsz;
+    const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
+    k_ssd_fwd<<<grid, THREADS, SMEM_BYTES, st>>>(mx, mb, mc, my, p, lgR);
+    profile_mark(st, "k_ssd_fwd");
+    return cudaGetLastError();
+}
+
+// Backward of the scalar-decay path.  p.ws_kp holds the state entering every
+// chunk (the training forward's tiles, p.states_ready), or is filled here by a
+// forward pass that writes the states only.  Needs p.ws_ring, p.ws_flag,
+// p.sd_tok, p.sd_par, p.sd_db0 (and p.sd_dBh / p.sd_dCh when groups hold
+// several heads).
+cudaError_t ssd_backward(const Params &p, cudaStream_t st) {
+    using namespace ssdk;
+    cudaError_t e;
+    if (!p.states_ready) {
+        Params pf = p;
+        pf.y = nullptr;
+        pf.hT = nullptr;
+        pf.wT = nullptr;
+        if ((e = ssd_forward(pf, st)) != cudaSuccess) return e;
+    }
+    const int lgR = ssd_lg_rank(p.R);
+    const uint32_t Qt = (uint32_t)(ROWS >> lgR);
+    CUtensorMap mx, mdy, mb, mc, mdx, mdb, mdc;
+    if (!make_map5(&mx, p.x, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
+        !make_map5(&mdy, p.dy, 64, p.O, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt) ||
+        !make_map5(&mb, p.Bm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+        !make_map5(&mc, p.Cm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt) ||
+        !make_map5(&mdx, p.dx, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt))
+        return cudaErrorInvalidValue;
+    mdb = mb;
+    mdc = mc;
+    if (p.hpg == 1 &&
+        (!make_map5(&mdb, p.dBm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+         !make_map5(&mdc, p.dCm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt)))
+        return cudaErrorInvalidValue;
+    if (!p.ws_ring || !p.ws_flag || !p.ws_kp || !p.sd_tok || !p.sd_par || !p.sd_db0 ||
+        (p.hpg != 1 && (!p.sd_dBh || !p.sd_dCh)))
+        return cudaErrorInvalidValue;
+    static bool done[64] = {};
+    if ((e = ssd_set_smem(k_ssd_bwd, ssdb::SMEM_BYTES, done)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
+        cudaSuccess)
+        return e;
+    // dbeta_0 stays zero without a left endpoint
+    if ((e = cudaMemsetAsync(p.sd_db0, 0, sizeof(float) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
+        return e;
+    const long long nitems = (long long)p.nc * p.H * p.Bsz;
+    const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
+    k_ssd_bwd<<<grid, ssdb::THREADS, ssdb::SMEM_BYTES, st>>>(mx, mdy, mb, mc, mdx, mdb, mdc, p,
+                                                             lgR);
+    profile_mark(st, "k_ssd_bwd");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long tot = (long long)p.Bsz * p.L * p.H;
+    int blocks = (int)((tot + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_ssd_tokens<<<blocks, 256, 0, st>>>(p);
+    profile_mark(st, "k_ssd_tokens");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.hpg != 1) {
+        const long long tg = (long long)p.Bsz * p.L * p.G * p.R * p.N;
+        int gb = (int)((tg + 255) / 256);
+        if (gb > 148 * 16) gb = 148 * 16;
+        k_ssd_group_sum<<<gb, 256, 0, st>>>(p);
+        profile_mark(st, "k_ssd_group_sum");
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    k_ssd_params<<<(p.H + 127) / 128, 128, 0, st>>>(p);
+    profile_mark(st, "k_ssd_params");
+    return cudaGetLastError();
+}
+
+// Read and clear the device error word of these kernels.
+int ssd_error_take() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, ssm_ssd_error_word, sizeof(int)) != cudaSuccess) return -1;
+    if (v) cudaMemcpyToSymbol(ssm_ssd_error_word, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace ssm

@@ -156,6 +156,26 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, uint64_
         "r"(smem_u32(bar))
         : "memory");
 }
+// 5-D tile load into shared memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_5d(void *dst, const void *tmap, uint64_t *bar, int c0,
+                                            int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "r"(smem_u32(bar))
+        : "memory");
+}
+// 5-D tile store from shared memory (bulk-group completion); coordinates past
+// the tensor's extent are not written.  Innermost coordinate 16-byte aligned.
+__device__ __forceinline__ void tma_store_5d(const void *tmap, const void *src, int c0, int c1,
+                                             int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];\n" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(src))
+        : "memory");
+}
 // 1-D bulk copy global -> shared completing on `bar` (no multicast); both
 // addresses 16-byte aligned, `bytes` a multiple of 16.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,

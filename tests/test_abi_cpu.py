@@ -41,6 +41,16 @@ def test_abi_version(lib):
     assert abi.ssm_scan_abi_version() == 1
 
 
+def test_wait_limit_setter(lib):
+    old = abi.ssm_scan_set_wait_limit(123)
+    assert old == 1 << 22
+    assert abi.ssm_scan_set_wait_limit(old) == 123
+    with pytest.raises(abi.SsmError) as ei:
+        abi.ssm_scan_set_wait_limit(-1)
+    assert ei.value.code == -1
+    assert abi.ssm_scan_set_wait_limit(old) == old
+
+
 def test_contiguous_strides(lib):
     sh = S.WORKLOADS["ssd_mimo_r4"]
     d = abi.make_desc(sh)
@@ -61,7 +71,7 @@ def test_workspace_size(lib):
     # reuses (8 + 16 KB + 64 floats)
     nc = (100 + 63) // 64
     ni = abi.ssm_scan_workspace_size(d, abi.PASS_FWD_INFER)
-    assert ni >= 2 * 32 * (2 * 128 * 64 * 4 + 4) and ni % 256 == 0
+    assert ni >= 2 * 32 * 2 * 128 * 64 * 4 + (2 * 32 + 2) * 4 and ni % 256 == 0
     nf = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
     assert nf % 256 == 0
     assert nf - ni >= 2 * 32 * nc * (128 * 64 * 4 + 128 * 2 * 4 + 8192 + 16384 + 256)

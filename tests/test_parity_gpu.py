@@ -22,26 +22,41 @@ def _lib():
 
 
 def chunk_eligible(shape):
-    """Shapes the tensor-core kernels take (the rest go to the recurrent ones)."""
+    """Shapes the per-coordinate tensor-core kernels take."""
     return (shape.dtype_io == S.DTYPE_BF16 and shape.headdim == 64 and shape.rank_in == 1
             and shape.rank_out == 1 and shape.nstate in (64, 128) and shape.n_real % 8 == 0
             and shape.seqlen > 0 and shape.chunk != 1)
 
 
-def expected_route(shape):
+def ssd_eligible(shape):
+    """Shapes the scalar-decay (per-head) tensor-core kernels take."""
+    return (shape.dtype_io == S.DTYPE_BF16 and shape.decay_mode == S.DECAY_PER_HEAD
+            and shape.n_pairs == 0 and shape.headdim == 64 and shape.nstate in (64, 128)
+            and shape.rank_in == shape.rank_out and shape.rank_in in (1, 2, 4)
+            and shape.seqlen > 0 and shape.chunk != 1)
+
+
+def expected_route(shape, backward=False):
+    """Kernels expected to run the forward (backward) of `shape`."""
+    if ssd_eligible(shape):
+        return abi.ROUTE_SSD
     return abi.ROUTE_CHUNKED if chunk_eligible(shape) else abi.ROUTE_RECURRENT
 
 
 def run_gpu(shape, inp, backward=True, route=None):
-    """Forward (and backward) through the C ABI; checks which kernels ran."""
-    route = expected_route(shape) if route is None else route
+    """Forward (and backward) through the C ABI; checks which kernels ran.  `route`
+    overrides the expected route of both directions (a pair: each its own)."""
+    if route is None:
+        route = (expected_route(shape), expected_route(shape, backward=True))
+    elif not isinstance(route, tuple):
+        route = (route, route)
     dev = scan.to_device(shape, inp)
     y, hT, wT = scan.scan_forward(shape, dev)
-    assert abi.ssm_scan_last_route() == route
+    assert abi.ssm_scan_last_route() == route[0]
     g = None
     if backward:
         g = scan.scan_backward(shape, dev)
-        assert abi.ssm_scan_last_route() == route
+        assert abi.ssm_scan_last_route() == route[1]
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
     return y, hT, wT, g
@@ -238,14 +253,16 @@ def _scaled_dt(shape, inp, factor, rows=None):
                                              n_real=128, n_pairs=0, ngroups=2)])
 def test_large_decay_takes_recurrent_route(kw):
     """Inputs whose per-sub-block decay leaves the folding range (|A| log2(e)
-    sum of 16 dt > 100) give the oracle's result through the recurrent kernels."""
+    sum of 16 dt > 100) give the oracle's result through the recurrent kernels
+    in the per-coordinate chain; the scalar-decay chain has no range condition
+    and keeps them."""
     shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=150, nheads=4, ngroups=4).replace(**kw)
     inp = _scaled_dt(shape, S.make_inputs(shape, seed=41, with_state=True), 60.0)
     a_max = np.exp(inp["A_log"].max(axis=1))
     span = np.array([[inp["dt"][b, 16 * k:16 * k + 16, h].sum() for k in range(150 // 16 + 1)]
                      for b in range(2) for h in range(4)])
     assert (span.max() * a_max.max() * np.log2(np.e)) > 100.0
-    check_all(shape, inp, route=abi.ROUTE_RANGE_FALLBACK)
+    check_all(shape, inp, route=abi.ROUTE_SSD if ssd_eligible(shape) else abi.ROUTE_RANGE_FALLBACK)
 
 
 def test_one_hot_sub_block_takes_recurrent_route():
@@ -286,7 +303,7 @@ def test_backward_from_saved_states(kw):
     torch.cuda.synchronize()
     assert torch.equal(y_inf, y_tr)   # saving the backward's products changes nothing
     g_saved = scan.scan_backward(shape, dev, saved=wsf)
-    assert abi.ssm_scan_last_route() == expected_route(shape)
+    assert abi.ssm_scan_last_route() == expected_route(shape, backward=True)
     g_plain = scan.scan_backward(shape, dev)
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
