@@ -117,6 +117,23 @@ def kernel_bytes(shape, name: str) -> int:
         return ins + dy + out
     if name == "k_bwd_units_final":   # dt, lambda -> ddt, dlambda
         return 2 * (t["dt"] + t["lam"])
+    # scalar-decay chain
+    if name == "k_ssd_fwd":           # x, B, C, dt, lambda -> y
+        return ins + t["y"]
+    if name == "k_ssd_bwd":           # x, B, C, dt, lambda, dy -> dx (+ dB, dC, one head per group)
+        out = t["B"] + t["C"] if s.nheads == s.ngroups else 0
+        return ins + dy + t["x"] + out
+    if name == "k_ssd_tokens":        # dt, lambda -> ddt, dlambda
+        return 2 * (t["dt"] + t["lam"])
+    if name == "k_ssd_group_sum":     # -> dB, dC (groups of several heads)
+        return t["B"] + t["C"]
+    # channel scan
+    if name == "k_m1_fwd":
+        return ins + t["y"]
+    if name == "k_m1_bwd":            # inputs + dy -> dx, ddt, dlambda
+        return ins + dy + t["x"] + t["dt"] + t["lam"]
+    if name == "k_m1_bc_sum":         # -> dB, dC
+        return t["B"] + t["C"]
     return 0
 
 
@@ -307,9 +324,12 @@ def roofline_of(shape, dom, ms_launch, peaks):
     hbm = peaks.get("hbm_gbs")
     src = "measured" if hbm else "fallback"
     hbm = hbm or 6650.0
-    if shape.name == "mamba1_siso" and dom in ("k_fwd", "k_bwd_sweep1", "k_bwd_sweep2"):
-        # one ex2 per (token, channel, state row) in each sweep over the sequence:
-        # 16 ex2 per SM and clock, 148 SMs, at the clock sampled under load
+    if shape.name == "mamba1_siso" and dom in ("k_fwd", "k_bwd_sweep1", "k_bwd_sweep2",
+                                                "k_m1_fwd", "k_m1_bwd"):
+        # one ex2 per (token, channel, state row): the minimum of a pass over the
+        # sequence (the channel-scan backward recomputes the states and does two, which
+        # is overhead of the design and not counted); 16 ex2 per SM and clock, 148 SMs,
+        # at the clock sampled under load
         ex2 = shape.batch * shape.seqlen * shape.nheads * shape.nstate
         clk = peaks.get("sm_mhz_under_load") or 1965.0
         peak = 16 * 148 * clk * 1e6 / 1e9   # G ex2 / s
@@ -406,7 +426,8 @@ def main():
     abi.ssm_scan_poll_device_error()
     names = {abi.ROUTE_CHUNKED: "per-coordinate tensor-core chain",
              abi.ROUTE_RANGE_FALLBACK: "recurrent (range fallback)",
-             abi.ROUTE_RECURRENT: "recurrent", abi.ROUTE_SSD: "scalar-decay tensor-core chain"}
+             abi.ROUTE_RECURRENT: "recurrent", abi.ROUTE_SSD: "scalar-decay tensor-core chain",
+             abi.ROUTE_CHANNEL: "channel scan"}
     route_bwd = names[abi.ssm_scan_last_route()]
     fwd_only()
     route = {"fwd": names[abi.ssm_scan_last_route()], "bwd": route_bwd}

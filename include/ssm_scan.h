@@ -314,7 +314,8 @@ SSM_API int ssm_scan_abi_version(void);
  * SSM_ROUTE_RECURRENT (recurrent kernels chosen on the host: chunk = 1 or a
  * shape the chunked kernels do not take), SSM_ROUTE_SSD (per-head decay,
  * bf16, head dim 64, 64 or 128 state rows, no rotation pairs, rank_in ==
- * rank_out in {1, 2, 4}), or a negative status (no call yet,
+ * rank_out in {1, 2, 4}), SSM_ROUTE_CHANNEL (the Mamba-1 channel scan), or a
+ * negative status (no call yet,
  * or the gate word cannot be read).  A diagnostic for tests and tuning; the
  * pages have no counterpart.
  */
@@ -322,8 +323,10 @@ enum ssm_route {
     SSM_ROUTE_CHUNKED = 0,
     SSM_ROUTE_RANGE_FALLBACK = 1,
     SSM_ROUTE_RECURRENT = 2,
-    SSM_ROUTE_SSD = 3   /* tensor-core chain of a per-head (scalar) decay: masked linear
+    SSM_ROUTE_SSD = 3,  /* tensor-core chain of a per-head (scalar) decay: masked linear
                            attention with an exact segment-sum mask, 128 / R tokens per chunk */
+    SSM_ROUTE_CHANNEL = 4 /* channel scan: head dim 1 (Mamba-1 channels), 8 or 16 real state
+                             rows, groups of a multiple of 64 channels, bf16 */
 };
 SSM_API int ssm_scan_last_route(void *stream);
 

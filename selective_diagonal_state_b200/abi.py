@@ -26,7 +26,7 @@ EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd"
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
             "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
             "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd", "ssm_scan_set_wait_limit"]
-ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT, ROUTE_SSD = 0, 1, 2, 3
+ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT, ROUTE_SSD, ROUTE_CHANNEL = 0, 1, 2, 3, 4
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 

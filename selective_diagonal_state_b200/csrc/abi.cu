@@ -38,6 +38,12 @@ int ssd_chunk_tokens(int R);
 cudaError_t ssd_forward(const Params &p, cudaStream_t st);
 cudaError_t ssd_backward(const Params &p, cudaStream_t st);
 int ssd_error_take();
+bool m1_supported(const Params &p);
+size_t m1_kept_floats(long long B, long long L, long long H, int N);
+size_t m1_part_floats(long long B, long long L, long long H, int N);
+cudaError_t m1_forward(const Params &p, float *kept, cudaStream_t st);
+cudaError_t m1_backward(const Params &p, float *kept, bool kept_ready, float *part,
+                        cudaStream_t st);
 }  // namespace ssm
 
 namespace {
@@ -212,6 +218,15 @@ bool ssd_shape(const ssm_desc_t *d) {
            d->seqlen > 0;
 }
 
+// Shapes of the channel scan (Mamba-1: head dim 1, 8 or 16 real state rows,
+// groups of a multiple of 64 channels).
+bool m1_shape(const ssm_desc_t *d) {
+    const int N = d->n_real + 2 * d->n_pairs;
+    return d->dtype_io == SSM_BF16 && d->headdim == 1 && d->rank_in == 1 && d->rank_out == 1 &&
+           d->n_pairs == 0 && (N == 8 || N == 16) && (d->nheads / d->ngroups) % 64 == 0 &&
+           d->chunk != 1 && d->seqlen > 0;
+}
+
 // Forward workspace of the tensor-core chain.  Every forward carries the fp32
 // state from one 64-token chunk to the next through two 32 KB slots and one
 // counter per (b, h) (the first `total_infer` bytes).  A training forward
@@ -226,6 +241,13 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
     FwdWs w;
     w.off_ring = w.off_flag = w.off_kp = w.off_ce = w.off_P = w.off_Bh = w.off_corr = 0;
     w.total_infer = w.total = 0;
+    if (m1_shape(d)) {
+        // channel scan: a forward alone needs nothing; a training forward keeps the
+        // state entering every 16-token tile
+        w.off_kp = 0;
+        w.total = align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
+        return w;
+    }
     if (ssd_shape(d)) {
         // scalar-decay chain: the two fp32 carry slots and the counter of every (b, h),
         // the ticket and abort words; a training forward also keeps the state entering
@@ -411,6 +433,11 @@ size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
     const size_t t = bwd_layout(d).total;
+    if (m1_shape(d)) {
+        const size_t t2 = align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4) +
+                          align256(ssm::m1_part_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
+        return t2 > t ? t2 : t;
+    }
     if (ssd_shape(d)) {
         // either chain may take the call (the scalar-decay one unless pointer
         // alignment rules it out): room for both
@@ -526,6 +553,23 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
     p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
     // chunk == 1 asks for the token-by-token recurrent kernels
+    if (m1_shape(d) && ssm::m1_supported(p)) {
+        const FwdWs lay = fwd_layout(d);
+        float *kept = nullptr;
+        if (workspace && workspace_bytes >= lay.total) {
+            if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+            kept = (float *)workspace;
+        }
+        cudaStream_t st = (cudaStream_t)stream;
+        profile_begin(st);
+        const cudaError_t e = ssm::m1_forward(p, kept, st);
+        profile_end();
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_CHANNEL;
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
+        g_last_error.clear();
+        return SSM_OK;
+    }
     const bool ssd = ssd_shape(d) && ssm::ssd_supported(p);
     const bool chunked =
         !ssd && d->chunk != 1 && ssm::chunk_fwd_supported(p) && tensor_chain_shape(d);
@@ -678,6 +722,24 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     p.ws_blk = (float *)(ws + lay.off_blk);
     p.ws_blkc = (float *)(ws + lay.off_blkc);
     p.nc = (int)((d->seqlen + 63) / 64);
+    if (m1_shape(d) && ssm::m1_supported(p)) {
+        const size_t kb = align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
+        float *kept = (float *)ws;
+        bool ready = false;
+        if (saved) {
+            kept = (float *)saved;
+            ready = true;
+        }
+        profile_begin(st);
+        const cudaError_t e = ssm::m1_backward(p, kept, ready, (float *)(ws + kb), st);
+        profile_end();
+        g_last_gate = nullptr;
+        g_last_route = SSM_ROUTE_CHANNEL;
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_bwd launch");
+        g_last_error.clear();
+        return SSM_OK;
+    }
+    if (saved && m1_shape(d)) saved = nullptr;   // states kept by the channel scan: not read here
     if (ssd_shape(d) && ssm::ssd_supported(p) && ((uintptr_t)dy & 15) == 0 &&
         ((uintptr_t)dx & 15) == 0 &&
         (d->nheads != d->ngroups || ((((uintptr_t)dB | (uintptr_t)dC) & 15) == 0))) {

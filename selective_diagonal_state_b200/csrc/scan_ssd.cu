@@ -52,16 +52,15 @@ using namespace umma;
 using namespace chunkc;
 
 constexpr int ROWS = 128;                 // (token, rank) rows per chunk
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;              // two CTAs per SM
 constexpr uint32_t TILE = 16384;          // 128 rows x 128 bytes (64 bf16), 128-byte swizzle
 constexpr uint32_t TMEM_COLS = 256;       // CB 0..127 (then Y_o 0..63) | S_c 128.. | Y_d 192..
-constexpr uint32_t SM_X = 0;              // 2 x 16 KB x tiles (rows (t, r)), double-buffered
-constexpr uint32_t SM_B = 32768;          // 2 x 16 KB B (state rows 0-63 | 64-127), rows (t, r)
-constexpr uint32_t SM_C = 65536;          // 2 x 16 KB C, rows (t, o)
-constexpr uint32_t SM_P = 98304;          // 32 KB masked scores, no-swizzle K-major (rows j, K = i)
-constexpr uint32_t SM_XS = 131072;        // 16 KB diag(f) x, then the y tile
-constexpr uint32_t SM_K = 147456;         // 16 KB entering state, bf16 [n][p] (128-byte swizzle)
-constexpr uint32_t SM_F32 = 163840;
+constexpr uint32_t SM_X = 0;              // 16 KB x tile (rows (t, r))
+constexpr uint32_t SM_B = 16384;          // 2 x 16 KB B (state rows 0-63 | 64-127), rows (t, r);
+                                          // then the masked scores P, no-swizzle K-major
+constexpr uint32_t SM_C = 49152;          // 2 x 16 KB C, rows (t, o)
+constexpr uint32_t SM_XS = 81920;         // 16 KB diag(f) x, then K_in (bf16 [n][p]), then y
+constexpr uint32_t SM_F32 = 98304;
 // fp32 scratch (float offsets)
 constexpr int F_DT = 0;      // [129] dt of the chunk's tokens and of the token after it
 constexpr int F_LAM = 132;   // [129] lambda of the same tokens
@@ -74,7 +73,7 @@ constexpr int F_SC = 904;    // [0] a log2(e), [1] D, [2] E = e^{a S_end}
 constexpr int F_END = 912;
 constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 128 + 1024;
-static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
+static_assert(SM_BAR % 8 == 0 && 2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 
 // Tokens of one chunk: dt and lambda (bf16 bits) of tokens t0 .. t0 + Qt, loaded
 // one item ahead and converted when stored.
@@ -197,7 +196,7 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
     return w;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
 k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
           Params p, int lgR) {
@@ -208,24 +207,25 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + SM_F32);
-    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // [2] x stages
-    uint64_t *bar_b = bar_x + 2, *bar_c = bar_x + 3;               // B, C tiles
-    uint64_t *bar_cb = bar_x + 4, *bar_sc = bar_x + 5, *bar_y = bar_x + 6;   // MMA phases
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 7);
-    int *s_item = reinterpret_cast<int *>(bar_x + 8);               // [2] claimed tickets
+    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // x tile
+    uint64_t *bar_b = bar_x + 1, *bar_c = bar_x + 2;               // B, C tiles
+    uint64_t *bar_sc = bar_x + 3, *bar_y = bar_x + 4;              // MMA phases
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 5);
+    int *s_item = reinterpret_cast<int *>(bar_x + 6);               // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, L = p.L;
     const int nbox = N / 64;
     const int Qt = ROWS >> lgR;   // tokens per chunk
     const bool want_y = p.y != nullptr;
-    const int qd = warp & 3, cb4 = warp >> 2;   // TMEM lane quarter, column block
+    const int qd = warp & 3, cb2 = warp >> 2;   // TMEM lane quarter, column half
     const int row = 32 * qd + lane;             // TMEM lane = row of every M = 128 tile
+    unsigned char *sX = sm + SM_X;
 
-    auto issue_x = [&](int item, int st) {
+    auto issue_x = [&](int item) {
         const ChunkItem it = chunk_item_cs(p, item);
-        mbar_expect_tx(&bar_x[st], TILE);
-        tma_load_5d(sm + SM_X + st * TILE, &tmX, &bar_x[st], 0, 0, it.h, it.c * Qt, it.b);
+        mbar_expect_tx(bar_x, TILE);
+        tma_load_5d(sX, &tmX, bar_x, 0, 0, it.h, it.c * Qt, it.b);
     };
     auto issue_b = [&](int item) {
         const ChunkItem it = chunk_item_cs(p, item);
@@ -240,10 +240,10 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             tma_load_5d(sm + SM_C + k * TILE, &tmC, bar_c, 64 * k, 0, it.h / p.hpg, it.c * Qt, it.b);
     };
 
-    PhaseCount pc_x[2] = {{0u, 0u}, {0u, 0u}}, pc_b = {0u, 0u}, pc_c = {0u, 0u};
-    PhaseCount pc_cb = {0u, 0u}, pc_sc = {0u, 0u}, pc_y = {0u, 0u};
+    PhaseCount pc_x = {0u, 0u}, pc_b = {0u, 0u}, pc_c = {0u, 0u};
+    PhaseCount pc_sc = {0u, 0u}, pc_y = {0u, 0u};
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bar_x[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bar_x[i], 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
@@ -251,8 +251,8 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         if (want_y) tma_prefetch_desc(&tmY);
         const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
         s_item[0] = first;
-        issue_x(first, 0);
-        ++pc_x[0].issued;
+        issue_x(first);
+        ++pc_x.issued;
         issue_b(first);
         ++pc_b.issued;
         if (want_y) {   // C is read by the outputs only
@@ -261,13 +261,6 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         }
     }
     if (warp == 0) tmem_alloc(tslot, TMEM_COLS);
-    if (N < NP) {   // state rows 64-127 of B / C are never loaded: keep them zero
-        for (int i = tid; i < (int)(TILE / 16); i += THREADS) {
-            reinterpret_cast<uint4 *>(sm + SM_B + TILE)[i] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4 *>(sm + SM_C + TILE)[i] = make_uint4(0, 0, 0, 0);
-        }
-    }
-    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -286,12 +279,11 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
 
     for (int k = 0; item < nitems; ++k) {
         if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
-        const int st = k & 1;
+        const uint32_t par = (uint32_t)(k & 1);
         const ChunkItem it = chunk_item_cs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int bh = b * p.H + h;
         const int t0 = c * Qt;
-        unsigned char *sX = sm + SM_X + st * TILE;
         // the previous item's y store has read the staging tile
         if (tid == 0) bulk_wait_read_all();
         chunk_scalars(p, f32, t0, Qt, tok, alog);
@@ -300,30 +292,27 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
             alog = __ldg(p.A_log + nx.h * p.ndec);
-            // the other x stage was last read by the previous item, which is complete
+        }
+        {
+            const bool okx = mbar_wait(bar_x, par, WAIT_LIMIT);
+            const bool okb = okx && mbar_wait(bar_b, par, WAIT_LIMIT);
+            const bool okc = okb && (!want_y || mbar_wait(bar_c, par, WAIT_LIMIT));
             if (tid == 0) {
-                issue_x(next, st ^ 1);
-                ++pc_x[st ^ 1].issued;
+                pc_x.done += okx ? 1u : 0u;
+                pc_b.done += okb ? 1u : 0u;
+                pc_c.done += (want_y && okc) ? 1u : 0u;
+            }
+            int ok = okc ? 1 : 0;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
             }
         }
-        const bool okx = mbar_wait(&bar_x[st], (uint32_t)((k >> 1) & 1), WAIT_LIMIT);
-        const bool okb = okx && mbar_wait(bar_b, (uint32_t)(k & 1), WAIT_LIMIT);
-        const bool okc = okb && (!want_y || mbar_wait(bar_c, (uint32_t)(k & 1), WAIT_LIMIT));
-        if (tid == 0) {
-            pc_x[st].done += okx ? 1u : 0u;
-            pc_b.done += okb ? 1u : 0u;
-            pc_c.done += (want_y && okc) ? 1u : 0u;
-        }
-        int ok = okc ? 1 : 0;
-        if (!ok) {
-            ssd_raise_error(1);
-            chain_abort(p);
-        }
-        if (!__syncthreads_and(ok)) {
-            aborted = true;
-            break;
-        }
-        // ---- CB = C B^T ----------------------------------------------------------
+        // ---- CB = C B^T (completion tracked by the S_c commit, which covers it) -----
         if (tid == 0 && want_y) {
             fence_after_sync();
             const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
@@ -333,12 +322,10 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 mma_bf16(t_cb, sdesc(c_base + off, 16u, 1024u, LAYOUT_SW128),
                          sdesc(b_base + off, 16u, 1024u, LAYOUT_SW128), id, s > 0);
             }
-            mma_commit(bar_cb);
-            ++pc_cb.issued;
         }
         // ---- X' = diag(f) X (same swizzled positions) -------------------------------
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 4; ++q) {
             const int ch = tid + THREADS * q;    // 16-byte chunk: row ch >> 3, position ch & 7
             const int r = ch >> 3;
             const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
@@ -363,80 +350,35 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             mma_commit(bar_sc);
             ++pc_sc.issued;
         }
-        if (want_y) {
-            // ---- masked scores P = CB (.) W -> bf16 tile ------------------------------
-            ok = mbar_wait(bar_cb, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
-            if (tid == 0) pc_cb.done += (uint32_t)ok;
+        // ---- chain: K_out = E K_in + S_c -------------------------------------------
+        {
+            int ok = mbar_wait(bar_sc, par, WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_sc.done += (uint32_t)ok;
             if (!ok) {
                 ssd_raise_error(1);
                 chain_abort(p);
             }
-            fence_after_sync();
-            if (ok) {
-                float v[32];
-                tmem_ld16(t_cb + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(v));
-                tmem_ld16(t_cb + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(v + 16));
-                const int tj = row >> lgR;
-                const float a2 = f32[F_SC], stj = f32[F_S + tj], gj = f32[F_GAM + tj];
-                const int i0 = 32 * cb4;
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float w8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int ti = (i0 + 8 * q8 + j) >> lgR;
-                        float wt = 0.f;
-                        if (ti < tj)
-                            wt = ex2_fast(a2 * (stj - f32[F_S + ti])) * f32[F_SIG + ti];
-                        else if (ti == tj)
-                            wt = gj;
-                        w8[j] = v[8 * q8 + j] * wt;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + SM_P + off_kmaj(row, i0 + 8 * q8, 128u, 2048u)) =
-                        pack8(w8);
-                }
+            if (tid == 0 && ok && c > 0 &&
+                !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
+                ssd_raise_error(2);
+                chain_abort(p);
+                ok = 0;
             }
-            fence_proxy_async();
-            fence_before_sync();
-            if (!__syncthreads_and(ok)) {
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of K_in
                 aborted = true;
                 break;
             }
-            // ---- Y_d = P X ------------------------------------------------------------
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t p_base = smem_u32(sm + SM_P), x_base = smem_u32(sX);
-                const uint32_t id = idesc_bf16(128, 64, false, true);
-                for (int s = 0; s < ROWS / 16; ++s)
-                    mma_bf16(t_yd, sdesc(p_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
-                             sdesc(x_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id, s > 0);
-            }
         }
-        // ---- chain: K_out = E K_in + S_c -------------------------------------------
-        ok = mbar_wait(bar_sc, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
-        if (tid == 0) pc_sc.done += (uint32_t)ok;
-        if (!ok) {
-            ssd_raise_error(1);
-            chain_abort(p);
-        }
-        if (tid == 0 && ok && c > 0 &&
-            !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
-            ssd_raise_error(2);
-            chain_abort(p);
-            ok = 0;
-        }
-        fence_after_sync();
-        if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of K_in
-            aborted = true;
-            break;
-        }
-        // B and X' are consumed (CB and S_c complete): fetch the next item's B
-        if (tid == 0 && next < nitems) {
+        // states only: B is consumed (CB is not issued): fetch the next item's
+        if (!want_y && tid == 0 && next < nitems) {
             issue_b(next);
             ++pc_b.issued;
         }
-        {
-            const int n = row, cq = cb4;
+#pragma unroll 1
+        for (int cq = 2 * cb2; cq < 2 * cb2 + 2; ++cq) {
+            // K_in as the bf16 tile of the readout, in X''s place (S_c has read X')
+            const int n = row;
             float kc[16], sc[16];
             load_kin(p, c, b, h, n, cq, kc);
             tmem_ld16(t_sc + lane_q + 16u * cq, sc);
@@ -455,7 +397,7 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 }
                 const uint32_t off = sw_off(n, 2 * cq + g8);
                 const uint4 wh = pack8(hi);
-                *reinterpret_cast<uint4 *>(sm + SM_K + off) = wh;
+                *reinterpret_cast<uint4 *>(sm + SM_XS + off) = wh;
                 if (sv) {
                     *reinterpret_cast<uint4 *>(sv + off) = wh;
                     *reinterpret_cast<uint4 *>(sv + TILE + off) = pack8(lo);
@@ -494,11 +436,45 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         // the carry of (b, h) is in place: let the next chunk's item go (off the issue path)
         if (tid == THREADS - 32 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
         if (want_y) {
-            // ---- Y_o = C K_in, then the epilogue -----------------------------------------
+            // ---- masked scores P = CB (.) W -> bf16 tile in B's place (CB and S_c have
+            // read B; CB completed with S_c) -------------------------------------------------
+#pragma unroll 1
+            for (int sub = 0; sub < 2; ++sub) {
+                const int i0 = 64 * cb2 + 32 * sub;
+                float v[32];
+                tmem_ld16(t_cb + lane_q + (uint32_t)i0, *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(t_cb + lane_q + (uint32_t)i0 + 16u, *reinterpret_cast<float(*)[16]>(v + 16));
+                const int tj = row >> lgR;
+                const float a2 = f32[F_SC], stj = f32[F_S + tj], gj = f32[F_GAM + tj];
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float w8[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int ti = (i0 + 8 * q8 + j) >> lgR;
+                        float wt = 0.f;
+                        if (ti < tj)
+                            wt = ex2_fast(a2 * (stj - f32[F_S + ti])) * f32[F_SIG + ti];
+                        else if (ti == tj)
+                            wt = gj;
+                        w8[j] = v[8 * q8 + j] * wt;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + SM_B + off_kmaj(row, i0 + 8 * q8, 128u, 2048u)) =
+                        pack8(w8);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            // ---- Y_d = P X, Y_o = C K_in ------------------------------------------------
             if (tid == 0) {
                 fence_after_sync();
-                const uint32_t c_base = smem_u32(sm + SM_C), k_base = smem_u32(sm + SM_K);
+                const uint32_t p_base = smem_u32(sm + SM_B), x_base = smem_u32(sX);
                 const uint32_t id = idesc_bf16(128, 64, false, true);
+                for (int s = 0; s < ROWS / 16; ++s)
+                    mma_bf16(t_yd, sdesc(p_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                             sdesc(x_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id, s > 0);
+                const uint32_t c_base = smem_u32(sm + SM_C), k_base = smem_u32(sm + SM_XS);
                 for (int s = 0; s < N / 16; ++s)
                     mma_bf16(t_yo,
                              sdesc(c_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u,
@@ -507,31 +483,37 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 mma_commit(bar_y);
                 ++pc_y.issued;
             }
-            ok = mbar_wait(bar_y, (uint32_t)(k & 1), WAIT_LIMIT) ? 1 : 0;
-            if (tid == 0) pc_y.done += (uint32_t)ok;
-            if (!ok) {
-                ssd_raise_error(1);
-                chain_abort(p);
+            {
+                int ok = mbar_wait(bar_y, par, WAIT_LIMIT) ? 1 : 0;
+                if (tid == 0) pc_y.done += (uint32_t)ok;
+                if (!ok) {
+                    ssd_raise_error(1);
+                    chain_abort(p);
+                }
+                fence_after_sync();
+                if (!__syncthreads_and(ok)) {
+                    aborted = true;
+                    break;
+                }
             }
-            fence_after_sync();
-            if (!__syncthreads_and(ok)) {
-                aborted = true;
-                break;
-            }
-            // C is consumed: fetch the next item's
+            // P (in B's place), C and K_in are consumed: fetch the next item's B and C
             if (tid == 0 && next < nitems) {
+                issue_b(next);
+                ++pc_b.issued;
                 issue_c(next);
                 ++pc_c.issued;
             }
-            {
+            // ---- epilogue: y into K_in's place ------------------------------------------
+#pragma unroll 1
+            for (int cq = 2 * cb2; cq < 2 * cb2 + 2; ++cq) {
                 float yd[16], yo[16];
-                tmem_ld16(t_yd + lane_q + 16u * cb4, yd);
-                tmem_ld16(t_yo + lane_q + 16u * cb4, yo);
+                tmem_ld16(t_yd + lane_q + 16u * cq, yd);
+                tmem_ld16(t_yo + lane_q + 16u * cq, yo);
                 const float e = f32[F_EW + (row >> lgR)];
                 const float D = (p.R == p.O && p.D) ? __ldg(p.D + h) : 0.f;
 #pragma unroll
                 for (int g8 = 0; g8 < 2; ++g8) {
-                    const uint32_t off = sw_off(row, 2 * cb4 + g8);
+                    const uint32_t off = sw_off(row, 2 * cq + g8);
                     float xv[8], yv[8];
                     unpack8(*reinterpret_cast<const uint4 *>(sX + off), xv);
 #pragma unroll
@@ -550,15 +532,18 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         }
         fence_before_sync();
         __syncthreads();
+        // x is consumed: fetch the next item's
+        if (tid == 0 && next < nitems) {
+            issue_x(next);
+            ++pc_x.issued;
+        }
         item = next;
     }
     if (tid == 0) bulk_wait_read_all();
     if (aborted && tid == 0) {
-        drain_phases(&bar_x[0], pc_x[0]);
-        drain_phases(&bar_x[1], pc_x[1]);
+        drain_phases(bar_x, pc_x);
         drain_phases(bar_b, pc_b);
         drain_phases(bar_c, pc_c);
-        drain_phases(bar_cb, pc_cb);
         drain_phases(bar_sc, pc_sc);
         drain_phases(bar_y, pc_y);
     }
@@ -611,8 +596,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t T_CB = 0, T_DB = 0;       // CB, then dB (128 columns)
 constexpr uint32_t T_DS = 128, T_DXS = 128;  // dS, then dX_s (64)
 constexpr uint32_t T_DC = 256;               // diag(e) dY K_in^T, then dC (128)
-constexpr uint32_t T_GL = 384;               // G_loc (64)
-constexpr uint32_t T_DXD = 448;              // dX_d (64)
+constexpr uint32_t T_GL = 384;               // G_loc (64), read by the chain step
+constexpr uint32_t T_BS0 = 192, T_BS1 = 384;  // X G_out^T, state rows 0-63 | 64-127 (phase 3)
+constexpr uint32_t T_DXD = 448, T_YO = 448;  // Y_o = C K_in (read by the masking), then dX_d (64)
 constexpr uint32_t SM_X = 0;         // 16 KB x (rows (t, r))
 constexpr uint32_t SM_DY = 16384;    // 16 KB dy (rows (t, o))
 constexpr uint32_t SM_B = 32768;     // 2 x 16 KB B
@@ -795,35 +781,65 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 mma_bf16(tb + T_DS, sdesc(dy_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
                          sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id128, s > 0);
         }
-        // diag(e) dy (same swizzled positions)
+        // diag(e) dy as bf16 hi (SM_DYS) + lo (dCB's place, free until the masking), and the
+        // K_in lo tile after it (same swizzled positions throughout)
+        {
+            const unsigned char *klo =
+                reinterpret_cast<const unsigned char *>(p.ws_kp + u * SLOT_FLOATS) + TILE;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int ch = tid + THREADS * q;
-            const int r = ch >> 3;
-            const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
-            const float e = f32[F_EW + (r >> lgR)];
-            float v[8];
-            unpack8(*reinterpret_cast<const uint4 *>(sm + SM_DY + off), v);
+            for (int q = 0; q < 2; ++q) {
+                const int ch = tid + THREADS * q;
+                const int r = ch >> 3;
+                const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
+                const float e = f32[F_EW + (r >> lgR)];
+                float v[8], hi[8], lo[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + SM_DY + off), v);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] *= e;
-            *reinterpret_cast<uint4 *>(sm + SM_DYS + off) = pack8(v);
+                for (int j = 0; j < 8; ++j) {
+                    v[j] *= e;
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
+                    lo[j] = v[j] - hi[j];
+                }
+                *reinterpret_cast<uint4 *>(sm + SM_DYS + off) = pack8(hi);
+                *reinterpret_cast<uint4 *>(sm + SM_DCB + off) = pack8(lo);
+                *reinterpret_cast<uint4 *>(sm + SM_DCB + TILE + off) =
+                    __ldg(reinterpret_cast<const uint4 *>(klo + off));
+            }
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        // ---- phase 1b: dC <- diag(e) dY K_in^T, G_loc = C^T diag(e) dY ----------------
+        // ---- phase 1b: dC <- diag(e) dY K_in^T; Y_o = C K_in (hi + lo, for R);
+        //      G_loc = C^T diag(e) dY (hi + lo) ------------------------------------------
         if (tid == 0) {
             fence_after_sync();
             const uint32_t c_base = smem_u32(sm + SM_C), k_base = smem_u32(sm + SM_K);
-            const uint32_t dys_base = smem_u32(sm + SM_DYS);
+            const uint32_t klo_base = smem_u32(sm + SM_DCB + TILE);
+            const uint32_t dys_base = smem_u32(sm + SM_DYS), dyl_base = smem_u32(sm + SM_DCB);
             const uint32_t id128 = idesc_bf16(128, 128, false, false);
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tb + T_DC, sdesc(dys_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(k_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id128, s > 0);
+            // hi * hi + hi * lo + lo * hi
+            const uint32_t a_of[3] = {dys_base, dys_base, dyl_base};
+            const uint32_t b_of[3] = {k_base, klo_base, k_base};
+            for (int part = 0; part < 3; ++part)
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tb + T_DC, sdesc(a_of[part] + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                             sdesc(b_of[part] + s * 32u, 16u, 1024u, LAYOUT_SW128), id128,
+                             part > 0 || s > 0);
+            const uint32_t id_yo = idesc_bf16(128, 64, false, true);
+            for (int part = 0; part < 2; ++part)
+                for (int s = 0; s < N / 16; ++s)
+                    mma_bf16(tb + T_YO,
+                             sdesc(c_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u,
+                                   16u, 1024u, LAYOUT_SW128),
+                             sdesc((part ? klo_base : k_base) + s * 2048u, TILE, 1024u, LAYOUT_SW128),
+                             id_yo, part > 0 || s > 0);
             const uint32_t id64 = idesc_bf16(128, 64, true, true);
-            for (int s = 0; s < ROWS / 16; ++s)
-                mma_bf16(tb + T_GL, sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128),
-                         sdesc(dys_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id64, s > 0);
+            for (int part = 0; part < 2; ++part)
+                for (int s = 0; s < ROWS / 16; ++s)
+                    mma_bf16(tb + T_GL, sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128),
+                             sdesc((part ? dyl_base : dys_base) + s * 2048u, TILE, 1024u,
+                                   LAYOUT_SW128),
+                             id64, part > 0 || s > 0);
             mma_commit(bar_p1);
             ++pc_1.issued;
         }
@@ -879,20 +895,18 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 red[R_COLZ + qd * 128 + i0 + lane] = colz[0];
                 red[R_ROWZ + cb4 * 128 + row] = rowz;
                 red[R_DIAG + cb4 * 128 + row] = diag;
-                // R[j] = sum_n C[j][n] (diag(e) dY K_in^T)[j][n] over this thread's 32 n
-                float dcs[32];
-                tmem_ld16(tb + T_DC + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(dcs));
-                tmem_ld16(tb + T_DC + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(dcs + 16));
-                const unsigned char *ct = sm + SM_C + (cb4 >> 1) * TILE;
+                // R[j] = e_j <dY_j, (C K_in)_j> over this thread's 16 p
+                float yo[16];
+                tmem_ld16(tb + T_YO + lane_q + 16u * cb4, yo);
                 float roff = 0.f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float cv[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(ct + sw_off(row, 4 * (cb4 & 1) + q)), cv);
+                for (int g8 = 0; g8 < 2; ++g8) {
+                    float dyv[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + SM_DY + sw_off(row, 2 * cb4 + g8)), dyv);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) roff = fmaf(cv[j], dcs[8 * q + j], roff);
+                    for (int j = 0; j < 8; ++j) roff = fmaf(dyv[j], yo[8 * g8 + j], roff);
                 }
-                red[R_ROFF + cb4 * 128 + row] = roff;
+                red[R_ROFF + cb4 * 128 + row] = roff * f32[F_EW + tj];
             }
             fence_proxy_async();
             fence_before_sync();
@@ -901,69 +915,25 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 break;
             }
         }
-        // ---- phase 2: dX_d = P^T dY, dC += dCB B, dB = dCB^T C ------------------------
-        if (tid == 0) {
-            fence_after_sync();
-            // K_in is consumed: fetch the next item's
-            if (next < nitems) {
-                issue_k(next);
-                ++pc_k.issued;
-            }
-            const uint32_t p_base = smem_u32(sm + SM_P), dcb_base = smem_u32(sm + SM_DCB);
-            const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
-            const uint32_t dy_base = smem_u32(sm + SM_DY);
-            const uint32_t id_x = idesc_bf16(128, 64, true, true);
-            for (int s = 0; s < ROWS / 16; ++s)
-                mma_bf16(tb + T_DXD, sdesc(p_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                         sdesc(dy_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_x, s > 0);
-            const uint32_t id_c = idesc_bf16(128, 128, false, true);
-            for (int s = 0; s < ROWS / 16; ++s)
-                mma_bf16(tb + T_DC, sdesc(dcb_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
-                         sdesc(b_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_c, true);
-            const uint32_t id_b = idesc_bf16(128, 128, true, true);
-            for (int s = 0; s < ROWS / 16; ++s)
-                mma_bf16(tb + T_DB, sdesc(dcb_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
-                         sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_b, s > 0);
-            mma_commit(bar_p2);
-            ++pc_2.issued;
-        }
+        // ---- chain step (needs only G_loc): G_in = E G_out + G_loc; Q = <G_out, E K_in> ----
         {
-            int ok = mbar_wait(bar_p2, par, WAIT_LIMIT) ? 1 : 0;
-            if (tid == 0) pc_2.done += (uint32_t)ok;
-            if (!ok) {
-                ssd_raise_error(1);
-                chain_abort(p);
-            }
+            int ok = 1;
             // the adjoint leaving this chunk is published by the item of chunk c + 1
-            if (tid == 0 && ok && rr > 0 &&
+            if (tid == 0 && rr > 0 &&
                 !wait_count(p.ws_flag + bh, rr, chain_abort_word(p), p.wait_limit)) {
                 ssd_raise_error(2);
                 chain_abort(p);
                 ok = 0;
             }
-            fence_after_sync();
             if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of G_out
                 aborted = true;
                 break;
             }
         }
-        // ---- diag(f) X into P's place (phase 2 has read P) --------------------------
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int ch = tid + THREADS * q;
-            const int r = ch >> 3;
-            const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
-            const float f = f32[F_FW + (r >> lgR)];
-            float v[8];
-            unpack8(*reinterpret_cast<const uint4 *>(sm + SM_X + off), v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] *= f;
-            *reinterpret_cast<uint4 *>(sm + SM_P + off) = pack8(v);
-        }
-        // ---- chain step: G_in = E G_out + G_loc; Q = <G_out, E K_in> ------------------
+        float go[16];   // G_out of (state row `row`, 16 columns from 16 cb4), kept for phase 3
         {
             const int n = row, cq = cb4;
-            float go[16], gl[16];
+            float gl[16];
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
                 float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -980,16 +950,11 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
                 const uint32_t off = sw_off(n, 2 * cq + g8);
-                float gh[8], kh[8], kl[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) gh[j] = go[8 * g8 + j];
-                *reinterpret_cast<uint4 *>(sm + SM_P + TILE + off) = pack8(gh);
-                // K_in hi / lo from the chunk's slot (the next item's K_in may be landing in
-                // the shared-memory copy already)
+                float kh[8], kl[8];
                 unpack8(__ldg(reinterpret_cast<const uint4 *>(kslot + off)), kh);
                 unpack8(__ldg(reinterpret_cast<const uint4 *>(kslot + TILE + off)), kl);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) qb = fmaf(gh[j], kh[j] + kl[j], qb);
+                for (int j = 0; j < 8; ++j) qb = fmaf(go[8 * g8 + j], kh[j] + kl[j], qb);
             }
             float gi[16];
 #pragma unroll
@@ -1024,26 +989,88 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 f32[F_QB + 16 + warp] = db0;
             }
         }
-        fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         // the carry of chunk c - 1 is in place: let its item go (off the issue path)
         if (tid == THREADS - 32 && c > 0) publish_count(p.ws_flag + bh, rr + 1);
-        // ---- phase 3: dX_s = B G_out, dB += diag(f) X G_out^T ---------------------------
+        // ---- phase 2: dX_d = P^T dY, dC += dCB B, dB = dCB^T C ------------------------
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t b_base = smem_u32(sm + SM_B), xs_base = smem_u32(sm + SM_P);
-            const uint32_t g_base = smem_u32(sm + SM_P + TILE);
+            // K_in is consumed: fetch the next item's
+            if (next < nitems) {
+                issue_k(next);
+                ++pc_k.issued;
+            }
+            const uint32_t p_base = smem_u32(sm + SM_P), dcb_base = smem_u32(sm + SM_DCB);
+            const uint32_t b_base = smem_u32(sm + SM_B), c_base = smem_u32(sm + SM_C);
+            const uint32_t dy_base = smem_u32(sm + SM_DY);
+            const uint32_t id_x = idesc_bf16(128, 64, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DXD, sdesc(p_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                         sdesc(dy_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_x, s > 0);
+            const uint32_t id_c = idesc_bf16(128, 128, false, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DC, sdesc(dcb_base + s * 256u, 128u, 2048u, LAYOUT_NONE),
+                         sdesc(b_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_c, true);
+            const uint32_t id_b = idesc_bf16(128, 128, true, true);
+            for (int s = 0; s < ROWS / 16; ++s)
+                mma_bf16(tb + T_DB, sdesc(dcb_base + s * 4096u, 2048u, 128u, LAYOUT_NONE),
+                         sdesc(c_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_b, s > 0);
+            mma_commit(bar_p2);
+            ++pc_2.issued;
+        }
+        {
+            int ok = mbar_wait(bar_p2, par, WAIT_LIMIT) ? 1 : 0;
+            if (tid == 0) pc_2.done += (uint32_t)ok;
+            if (!ok) {
+                ssd_raise_error(1);
+                chain_abort(p);
+            }
+            fence_after_sync();
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+        }
+        // ---- phase 2 has read P and dCB: G_out hi in P's place (after 16 KB) and lo in
+        // dCB's ------------------------------------------------------------------------
+#pragma unroll
+        for (int g8 = 0; g8 < 2; ++g8) {
+            const uint32_t off = sw_off(row, 2 * cb4 + g8);
+            float gh[8], glo[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                gh[j] = __bfloat162float(__float2bfloat16_rn(go[8 * g8 + j]));
+                glo[j] = go[8 * g8 + j] - gh[j];
+            }
+            *reinterpret_cast<uint4 *>(sm + SM_P + TILE + off) = pack8(gh);
+            *reinterpret_cast<uint4 *>(sm + SM_DCB + off) = pack8(glo);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // ---- phase 3: dX_s = B G_out, X G_out^T (G_out as hi + lo; diag(f) applied after) --
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t b_base = smem_u32(sm + SM_B), x_base = smem_u32(sm + SM_X);
+            const uint32_t g_base = smem_u32(sm + SM_P + TILE), gl_base = smem_u32(sm + SM_DCB);
             const uint32_t id_x = idesc_bf16(128, 64, false, true);
-            for (int s = 0; s < N / 16; ++s)
-                mma_bf16(tb + T_DXS,
-                         sdesc(b_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u, 16u,
-                               1024u, LAYOUT_SW128),
-                         sdesc(g_base + s * 2048u, TILE, 1024u, LAYOUT_SW128), id_x, s > 0);
-            const uint32_t id_b = idesc_bf16(128, 128, false, false);
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tb + T_DB, sdesc(xs_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
-                         sdesc(g_base + s * 32u, 16u, 1024u, LAYOUT_SW128), id_b, true);
+            for (int part = 0; part < 2; ++part)
+                for (int s = 0; s < N / 16; ++s)
+                    mma_bf16(tb + T_DXS,
+                             sdesc(b_base + (uint32_t)(s >> 2) * TILE + (uint32_t)(s & 3) * 32u,
+                                   16u, 1024u, LAYOUT_SW128),
+                             sdesc((part ? gl_base : g_base) + s * 2048u, TILE, 1024u, LAYOUT_SW128),
+                             id_x, part > 0 || s > 0);
+            const uint32_t id_b = idesc_bf16(128, 64, false, false);
+            for (int nh = 0; nh < 2; ++nh)        // state rows 64 nh .. 64 nh + 63 (N = 64 each)
+                for (int part = 0; part < 2; ++part)
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tb + (nh ? T_BS1 : T_BS0),
+                                 sdesc(x_base + s * 32u, 16u, 1024u, LAYOUT_SW128),
+                                 sdesc((part ? gl_base : g_base) + (uint32_t)nh * 8192u + s * 32u, 16u,
+                                       1024u, LAYOUT_SW128),
+                                 id_b, part > 0 || s > 0);
             mma_commit(bar_p3);
             ++pc_3.issued;
         }
@@ -1097,6 +1124,14 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 float v[32];
                 tmem_ld16(tb + tcol + lane_q + 32u * cb4, *reinterpret_cast<float(*)[16]>(v));
                 tmem_ld16(tb + tcol + lane_q + 32u * cb4 + 16u, *reinterpret_cast<float(*)[16]>(v + 16));
+                if (!half) {   // dB = (dS (.) W)^T C + diag(f) X G_out^T
+                    const uint32_t ts = ((cb4 >> 1) ? T_BS1 : T_BS0) + 32u * (cb4 & 1);
+                    float w2[32];
+                    tmem_ld16(tb + ts + lane_q, *reinterpret_cast<float(*)[16]>(w2));
+                    tmem_ld16(tb + ts + lane_q + 16u, *reinterpret_cast<float(*)[16]>(w2 + 16));
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = fmaf(f, w2[j], v[j]);
+                }
                 const int n0 = 32 * cb4;
                 if (one_head) {
                     unsigned char *stg = sm + (half ? SM_DCB : SM_P) + (cb4 >> 1) * TILE;

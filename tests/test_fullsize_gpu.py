@@ -138,7 +138,8 @@ def mamba1_run():
 
 
 def test_mamba1_sampled_batch_row(mamba1_run):
-    shape, inp, out, _ = mamba1_run
+    shape, inp, out, routes = mamba1_run
+    assert routes == (abi.ROUTE_CHANNEL, abi.ROUTE_CHANNEL)
     b = 5
     bs = slice(b, b + 1)
     hs = slice(None)

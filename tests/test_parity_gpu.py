@@ -36,8 +36,18 @@ def ssd_eligible(shape):
             and shape.seqlen > 0 and shape.chunk != 1)
 
 
+def channel_eligible(shape):
+    """Shapes the channel scan (Mamba-1 channels) takes."""
+    return (shape.dtype_io == S.DTYPE_BF16 and shape.headdim == 1 and shape.rank_in == 1
+            and shape.rank_out == 1 and shape.n_pairs == 0 and shape.nstate in (8, 16)
+            and (shape.nheads // shape.ngroups) % 64 == 0 and shape.seqlen > 0
+            and shape.chunk != 1)
+
+
 def expected_route(shape, backward=False):
     """Kernels expected to run the forward (backward) of `shape`."""
+    if channel_eligible(shape):
+        return abi.ROUTE_CHANNEL
     if ssd_eligible(shape):
         return abi.ROUTE_SSD
     return abi.ROUTE_CHUNKED if chunk_eligible(shape) else abi.ROUTE_RECURRENT
@@ -128,6 +138,23 @@ def test_chunked_shapes(kw):
     base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, chunk=64)
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=31, with_state=True)
+    check_all(shape, inp)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),                                  # Mamba-1: 16 state rows, B / C shared by all channels
+    dict(n_real=8),                          # 8 state rows: one thread per channel
+    dict(two_endpoint=1),                    # two-endpoint writes
+    dict(decay_mode=S.DECAY_PER_HEAD),       # one decay per channel
+    dict(nheads=256, ngroups=4),             # groups of 64 channels
+    dict(seqlen=1), dict(seqlen=16), dict(seqlen=17),
+])
+def test_channel_scan_shapes(kw):
+    """The channel scan (head dim 1) around its 16-token tiles and 64-channel
+    blocks, with an initial state and a left endpoint."""
+    base = S.WORKLOADS["mamba1_siso"].replace(batch=2, seqlen=70, nheads=128)
+    shape = base.replace(**kw)
+    inp = S.make_inputs(shape, seed=71, with_state=True)
     check_all(shape, inp)
 
 
