@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define SSM_SCAN_ABI_VERSION 1
+#define SSM_SCAN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define SSM_API __attribute__((visibility("default")))
@@ -63,6 +63,11 @@ enum ssm_status {
 
 enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 };
 enum ssm_decay_mode { SSM_DECAY_PER_HEAD = 0, SSM_DECAY_PER_COORD = 1 };
+/* Rotation angle of pair j at step t: SSM_ANGLE_STATIC phi = dt_t theta[h][j]
+ * (a fixed frequency scaled by the step), SSM_ANGLE_PER_TOKEN phi =
+ * theta[b][t][h][j] (a data-dependent angle per token, the complex state of
+ * Mamba-3 written as 2x2 rotations, sungsoo.github.io Part 05). */
+enum ssm_angle_mode { SSM_ANGLE_STATIC = 0, SSM_ANGLE_PER_TOKEN = 1 };
 /* SSM_PASS_FWD: a forward that keeps what ssm_scan_bwd_saved reads;
  * SSM_PASS_FWD_INFER: a forward only (smaller workspace). */
 enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1, SSM_PASS_FWD_INFER = 2 };
@@ -77,6 +82,8 @@ enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1, SSM_PASS_FWD_INFER = 2 };
  *   A_log, dA_log  fp32 [nheads][n_decay], n_decay = 1 (SSM_DECAY_PER_HEAD) or
  *                  n_real + n_pairs (SSM_DECAY_PER_COORD: real rows, then pairs)
  *   theta, dtheta  fp32 [nheads][n_pairs]   rotation frequency of each pair
+ *                  (SSM_ANGLE_STATIC), or fp32 [batch][seqlen][nheads][n_pairs],
+ *                  dense, the angle of each pair at each token (SSM_ANGLE_PER_TOKEN)
  *   D, dD          fp32 [nheads]
  *   h0, hT, prev_write, last_write, dh0, dprev_write  fp32 [batch][nheads][N][headdim]
  * Head h reads group g = h / (nheads / ngroups).  State rows: the n_real real
@@ -110,6 +117,14 @@ typedef struct ssm_desc {
     int32_t two_endpoint;       /* 0: lambda not read (lam = 1); 1: lambda used */
     int32_t dtype_io;           /* enum ssm_dtype of x, dt, B, C, lambda, y and of their gradients */
     int64_t stride_x[3], stride_y[3], stride_B[3], stride_C[3], stride_dt[3], stride_lambda[3];
+    int32_t angle_mode;         /* enum ssm_angle_mode (ignored when n_pairs == 0).  Per-token
+                                   angles are taken by the token-by-token recurrent kernels */
+    int32_t n_static;           /* 0 <= n_static <= n_real: the first n_static real rows are
+                                   static, with the transition exp(a_n) at every step whatever
+                                   dt_t (HybridMamba's real static rows next to its real and
+                                   complex dynamic ones, sungsoo.github.io Part 08 item 3);
+                                   their write is that of every row.  n_static > 0 is taken
+                                   by the token-by-token recurrent kernels */
 } ssm_desc_t;
 
 /* Fill every stride of *d for dense tensors of the sizes already set. */
@@ -221,6 +236,8 @@ SSM_API int ssm_scan_bwd_noalloc(const ssm_desc_t *d, const void *x, const void 
  * autoregressive inference).  For every (batch row, head):
  *     h <- A_t (h + beta_t w) + gamma_t W_t,   W_t = B_t u_t,   w <- W_t
  *     y_t = C_t h + D u_t
+ * With SSM_ANGLE_PER_TOKEN, theta is the token's angles, fp32
+ * [batch][nheads][n_pairs].
  * h and w are fp32 [batch][nheads][N][headdim], read and overwritten in
  * place: h holds H_{t-1} on entry and H_t on return; w holds the previous
  * write W_{t-1} on entry and W_t on return.  w may be NULL when

@@ -29,6 +29,8 @@ class _Desc(ctypes.Structure):
         ("n_real", ctypes.c_int), ("n_pairs", ctypes.c_int),
         ("rank_in", ctypes.c_int), ("rank_out", ctypes.c_int),
         ("per_coord_decay", ctypes.c_int), ("two_endpoint", ctypes.c_int),
+        ("angle_per_token", ctypes.c_int),
+        ("n_static", ctypes.c_int),
     ]
 
 
@@ -57,7 +59,8 @@ def _load(path=None):
 def _desc(shape) -> _Desc:
     return _Desc(shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups,
                  shape.n_real, shape.n_pairs, shape.rank_in, shape.rank_out,
-                 1 if shape.decay_mode == 1 else 0, shape.two_endpoint)
+                 1 if shape.decay_mode == 1 else 0, shape.two_endpoint,
+                 1 if getattr(shape, "angle_mode", 0) == 1 else 0, getattr(shape, "n_static", 0))
 
 
 def _p(a):
@@ -108,7 +111,8 @@ def scan_bwd(shape, inp: dict, dy, lib_path=None) -> dict:
     out = {
         "dx": np.zeros_like(a["x"]), "ddt": np.zeros_like(a["dt"]),
         "dA_log": np.zeros_like(a["A_log"]),
-        "dtheta": np.zeros((s.nheads, s.n_pairs)),
+        "dtheta": (np.zeros((s.batch, s.seqlen, s.nheads, s.n_pairs))
+                   if getattr(s, "angle_mode", 0) == 1 else np.zeros((s.nheads, s.n_pairs))),
         "dBm": np.zeros_like(a["Bm"]), "dCm": np.zeros_like(a["Cm"]),
         "dD": np.zeros_like(a["D"]), "dlam": np.zeros((s.batch, s.seqlen, s.nheads)),
         "dh0": np.zeros((s.batch, s.nheads, s.nstate, s.headdim)),

@@ -40,6 +40,15 @@
  *  n_real+2j = re, n_real+2j+1 = im) the block
  *      exp(dt_t a_j) [[cos phi, -sin phi], [sin phi, cos phi]],  phi = dt_t theta_j,
  *  with a = -exp(A_log) (one value per head, or one per real row / pair).
+ *  Real static rows (n_static > 0: the first n_static real rows; HybridMamba
+ *  mixes real static, real dynamic and complex dynamic rows, sungsoo.github.io
+ *  Part 08 item 3): the transition of such a row is exp(a_n) at every step,
+ *  independent of dt_t (read: "static" = not selective); its write is that of
+ *  every other row.
+ *  Per-token rotation angles (angle_per_token = 1, the data-dependent angles of
+ *  Mamba-3's complex state, sungsoo.github.io Part 05): phi = theta_t[j] is an
+ *  input per (batch, token, head, pair) instead of dt_t theta_j, and its
+ *  gradient is returned per token.
  *
  * Parity pins that do not go through this file (see tests/): the quadratic
  * masked-attention form, a complex128 recurrence, the LTI Vandermonde
@@ -70,6 +79,8 @@ typedef struct {
     int n_real, n_pairs, rank_in, rank_out;
     int per_coord_decay; /* 0: one decay per head; 1: one per real row / pair */
     int two_endpoint;    /* 0: lam == 1 (Euler write) */
+    int angle_per_token; /* 0: phi = dt_t theta[h][j]; 1: phi = theta[b][t][h][j] */
+    int n_static;        /* the first n_static real rows decay by exp(a_n) per step */
 } oracle_desc;
 
 /* ---- index helpers ---------------------------------------------------- */
@@ -107,15 +118,17 @@ static long dec_of_row(const oracle_desc *d, long n) {
 typedef struct { double *er, *ep, *cp, *sp; } step_coef;
 
 static void make_step(const oracle_desc *d, const double *A_log, const double *theta,
-                      long h, double dtv, step_coef *sc) {
+                      long b, long t, long h, double dtv, step_coef *sc) {
     long nd = NDEC(d);
     for (long n = 0; n < d->n_real; ++n) {
         double a = -exp(A_log[h * nd + dec_of_row(d, n)]);
-        sc->er[n] = exp(dtv * a);
+        sc->er[n] = (n < d->n_static && !MUT(10)) ? exp(a) : exp(dtv * a);
     }
     for (long j = 0; j < d->n_pairs; ++j) {
         double a = -exp(A_log[h * nd + dec_of_row(d, d->n_real + 2 * j)]);
-        double phi = dtv * theta[h * d->n_pairs + j];
+        double phi = d->angle_per_token
+                         ? theta[((b * d->seqlen + t) * d->nheads + h) * d->n_pairs + j]
+                         : dtv * theta[h * d->n_pairs + j];
         sc->ep[j] = exp(dtv * a);
         sc->cp[j] = cos(phi);
         sc->sp[j] = sin(phi);
@@ -199,7 +212,7 @@ static void fwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
     for (long t = 0; t < d->seqlen; ++t) {
         double gamma, beta, lv;
         step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
-        make_step(d, A_log, theta, h, dt[ix_bl(d, b, t, h)], &sc);
+        make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
         make_write(d, x, Bm, b, t, h, g, W);
         for (long i = 0; i < NP; ++i) Z[i] = H[i] + (MUT(1) ? 0.0 : beta) * Wp[i];
         apply_transition(d, &sc, Z, tmp);
@@ -265,8 +278,8 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
                      const double *A_log, const double *theta, const double *Bm,
                      const double *Cm, const double *D, const double *lam, const double *h0,
                      const double *w0, const double *dy, double *dx, double *ddt,
-                     double *dA_unit, double *dth_unit, double *dB_head, double *dC_head,
-                     double *dD_unit, double *dlam, double *dh0, double *dw0) {
+                     double *dA_unit, double *dth_unit, double *dtheta, double *dB_head,
+                     double *dC_head, double *dD_unit, double *dlam, double *dh0, double *dw0) {
     long N = NST(d), P = d->headdim, NP = N * P, L = d->seqlen, nd = NDEC(d);
     long g = h / (d->nheads / d->ngroups);
     long nseg = (L + SEG - 1) / SEG;
@@ -298,7 +311,7 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
         }
         double gamma, beta, lv;
         step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
-        make_step(d, A_log, theta, h, dt[ix_bl(d, b, t, h)], &sc);
+        make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
         for (long i = 0; i < NP; ++i) Z[i] = H[i] + beta * W[i];
         apply_transition(d, &sc, Z, AZ);
         make_write(d, x, Bm, b, t, h, g, W);
@@ -315,7 +328,7 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
             long k = t - t0 + 1;
             double gamma, beta, lv;
             step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
-            make_step(d, A_log, theta, h, dt[ix_bl(d, b, t, h)], &sc);
+            make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
             for (long i = 0; i < NP; ++i) Z[i] = segH[(k - 1) * NP + i] + beta * segW[(k - 1) * NP + i];
             apply_transition(d, &sc, Z, AZ);
             make_write(d, x, Bm, b, t, h, g, segW + k * NP);
@@ -327,7 +340,7 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
             const double *Wt = segW + k * NP, *Wm = segW + (k - 1) * NP;
             double gamma, beta, lv, dtv = dt[ix_bl(d, b, t, h)];
             step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
-            make_step(d, A_log, theta, h, dtv, &sc);
+            make_step(d, A_log, theta, b, t, h, dtv, &sc);
             /* output y_t = C_t H_t + D u_t */
             for (long n = 0; n < N; ++n)
                 for (long p = 0; p < P; ++p) {
@@ -365,8 +378,13 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
                 double grho = 0.0;
                 for (long p = 0; p < P; ++p) grho += G[n * P + p] * AZ[n * P + p];
                 double a = -exp(A_log[h * nd + dec_of_row(d, n)]);
-                ddt_acc += a * grho;
-                dA_unit[dec_of_row(d, n)] += dtv * grho;
+                if (n < d->n_static) {
+                    /* static row: log-transition a_n, independent of the step */
+                    dA_unit[dec_of_row(d, n)] += (MUT(11) ? dtv : 1.0) * grho;
+                } else {
+                    ddt_acc += a * grho;
+                    dA_unit[dec_of_row(d, n)] += dtv * grho;
+                }
             }
             for (long j = 0; j < d->n_pairs; ++j) {
                 long re = d->n_real + 2 * j, im = re + 1;
@@ -381,10 +399,16 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
                 }
                 long di = dec_of_row(d, re);
                 double a = -exp(A_log[h * nd + di]);
-                double w = theta[h * d->n_pairs + j];
-                ddt_acc += a * grho + w * gphi;
+                ddt_acc += a * grho;
                 dA_unit[di] += dtv * grho;
-                dth_unit[j] += (MUT(5) ? -dtv : dtv) * gphi;
+                if (d->angle_per_token) {
+                    /* phi is an input of its own: its gradient, per token */
+                    dtheta[((b * L + t) * d->nheads + h) * d->n_pairs + j] = MUT(12) ? -gphi : gphi;
+                } else {
+                    double w = theta[h * d->n_pairs + j];
+                    ddt_acc += w * gphi;
+                    dth_unit[j] += (MUT(5) ? -dtv : dtv) * gphi;
+                }
             }
             double dbeta = 0.0;
             for (long i = 0; i < NP; ++i) dbeta += Gz[i] * (MUT(6) ? Wt[i] : Wm[i]);
@@ -437,8 +461,8 @@ int oracle_scan_bwd(const oracle_desc *d, const double *x, const double *dt, con
 #pragma omp parallel for schedule(dynamic, 1)
     for (long u = 0; u < units; ++u) {
         bwd_unit(d, u / H, u % H, x, dt, A_log, theta, Bm, Cm, D, lam, h0, w0, dy, dx, ddt,
-                 dA_u + u * nd, dth_u + u * (d->n_pairs + 1), dBh, dCh, dD_u + u, dlam, dh0,
-                 dw0);
+                 dA_u + u * nd, dth_u + u * (d->n_pairs + 1), dtheta, dBh, dCh, dD_u + u, dlam,
+                 dh0, dw0);
     }
     /* reductions in a fixed order: over batch for the per-head parameters,
        over the heads of a group for the shared B and C */
@@ -448,7 +472,7 @@ int oracle_scan_bwd(const oracle_desc *d, const double *x, const double *dt, con
             for (long b = 0; b < Bt; ++b) acc += dA_u[(b * H + h) * nd + k];
             dA_log[h * nd + k] = acc * (-exp(A_log[h * nd + k]));
         }
-        for (long j = 0; j < d->n_pairs; ++j) {
+        for (long j = 0; j < d->n_pairs && !d->angle_per_token; ++j) {
             double acc = 0.0;
             for (long b = 0; b < Bt; ++b) acc += dth_u[(b * H + h) * (d->n_pairs + 1) + j];
             dtheta[h * d->n_pairs + j] = acc;

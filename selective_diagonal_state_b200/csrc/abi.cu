@@ -35,6 +35,7 @@ cudaError_t preact_backward(const Params &p, const PreactArgs &a, cudaStream_t s
 cudaError_t scan_step(const Params &p, float *h, float *w, cudaStream_t st);
 bool ssd_supported(const Params &p);
 int ssd_chunk_tokens(int R);
+size_t ssd_ring_bytes(long long B, long long H);
 cudaError_t ssd_forward(const Params &p, cudaStream_t st);
 cudaError_t ssd_backward(const Params &p, cudaStream_t st);
 int ssd_error_take();
@@ -150,6 +151,10 @@ int validate_desc(const ssm_desc_t *d) {
     if (d->dtype_io != SSM_F32 && d->dtype_io != SSM_BF16)
         return fail(SSM_ERR_ARG, "unknown dtype_io %d", d->dtype_io);
     if (d->chunk < 0) return fail(SSM_ERR_ARG, "chunk must be >= 0");
+    if (d->angle_mode != SSM_ANGLE_STATIC && d->angle_mode != SSM_ANGLE_PER_TOKEN)
+        return fail(SSM_ERR_ARG, "unknown angle_mode %d", d->angle_mode);
+    if (d->n_static < 0 || d->n_static > d->n_real)
+        return fail(SSM_ERR_ARG, "n_static (%d) must lie in [0, n_real = %d]", d->n_static, d->n_real);
     if (d->batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch > 65535");
     if (d->seqlen > (1LL << 31) - 1 || d->nheads > (1 << 24) || d->headdim > (1 << 16))
         return fail(SSM_ERR_UNSUPPORTED, "sizes exceed the 32-bit index ranges of the kernels");
@@ -184,6 +189,8 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
     p.two_ep = d->two_endpoint;
     p.per_coord = d->decay_mode == SSM_DECAY_PER_COORD;
     p.bf16 = d->dtype_io == SSM_BF16;
+    p.angle_tok = d->angle_mode == SSM_ANGLE_PER_TOKEN && d->n_pairs > 0;
+    p.nst = d->n_static;
     p.wait_limit = g_wait_limit.load();
     for (int k = 0; k < 3; ++k) {
         p.sx[k] = d->stride_x[k];
@@ -204,8 +211,10 @@ struct BwdWs {
 // Shapes the tensor-core chain may take (pointer alignment is checked at call time).
 bool tensor_chain_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
+    const bool static_angles = d->angle_mode == SSM_ANGLE_STATIC || d->n_pairs == 0;
     return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
-           (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0;
+           (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0 &&
+           static_angles && d->n_static == 0;
 }
 
 // Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and
@@ -215,7 +224,7 @@ bool ssd_shape(const ssm_desc_t *d) {
     return d->dtype_io == SSM_BF16 && d->decay_mode == SSM_DECAY_PER_HEAD && d->n_pairs == 0 &&
            d->headdim == 64 && (N == 64 || N == 128) && d->rank_in == d->rank_out &&
            (d->rank_in == 1 || d->rank_in == 2 || d->rank_in == 4) && d->chunk != 1 &&
-           d->seqlen > 0;
+           d->seqlen > 0 && d->n_static == 0;
 }
 
 // Shapes of the channel scan (Mamba-1: head dim 1, 8 or 16 real state rows,
@@ -224,7 +233,7 @@ bool m1_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
     return d->dtype_io == SSM_BF16 && d->headdim == 1 && d->rank_in == 1 && d->rank_out == 1 &&
            d->n_pairs == 0 && (N == 8 || N == 16) && (d->nheads / d->ngroups) % 64 == 0 &&
-           d->chunk != 1 && d->seqlen > 0;
+           d->chunk != 1 && d->seqlen > 0 && d->n_static == 0;
 }
 
 // Forward workspace of the tensor-core chain.  Every forward carries the fp32
@@ -249,14 +258,14 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
         return w;
     }
     if (ssd_shape(d)) {
-        // scalar-decay chain: the two fp32 carry slots and the counter of every (b, h),
+        // scalar-decay chain: the two tagged carry slots and the counter of every (b, h),
         // the ticket and abort words; a training forward also keeps the state entering
         // every chunk of ssm::ssd_chunk_tokens tokens (bf16 hi + lo tiles, 32 KB)
         const size_t bh = (size_t)d->batch * d->nheads;
         const int qt = ssm::ssd_chunk_tokens(d->rank_in);
         const size_t units = bh * (size_t)((d->seqlen + qt - 1) / qt);
         const size_t slot = 128 * (size_t)d->headdim * 4;
-        size_t off = align256(2 * bh * slot);
+        size_t off = align256(ssm::ssd_ring_bytes(d->batch, d->nheads));   // tagged carry slots
         w.off_flag = off;
         off = align256(off + (bh + 2) * 4);
         w.total_infer = off;
@@ -307,8 +316,8 @@ SsdBwdWs ssd_bwd_layout(const ssm_desc_t *d) {
     const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
     const size_t N = nstate(d);
     size_t off = 0;
-    w.off_ring = off;
-    off = align256(off + 2 * bh * slot);
+    w.off_ring = off;   // tagged carry slots
+    off = align256(off + ssm::ssd_ring_bytes(d->batch, d->nheads));
     w.off_flag = off;
     off = align256(off + (bh + 2) * 4);
     w.off_kp = off;
@@ -673,7 +682,7 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     if (d->seqlen == 0) {
         // nothing flows back through an empty sequence: zero parameter and state grads
         cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * d->nheads * ndecay(d), st);
-        if (e == cudaSuccess && dtheta && d->n_pairs)
+        if (e == cudaSuccess && dtheta && d->n_pairs && d->angle_mode == SSM_ANGLE_STATIC)
             e = cudaMemsetAsync(dtheta, 0, sizeof(float) * d->nheads * d->n_pairs, st);
         if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * d->nheads, st);
         size_t sb = sizeof(float) * d->batch * d->nheads * nstate(d) * d->headdim;

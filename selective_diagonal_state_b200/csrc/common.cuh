@@ -17,6 +17,8 @@ struct Params {
     // sizes
     int Bsz, L, H, P, G, nr, np, N, R, O, ndec, hpg;
     int two_ep, per_coord, bf16;
+    int angle_tok;  // rotation angles given per token: theta / dtheta are [B][L][H][np]
+    int nst;        // the first nst real rows are static (transition e^{a} whatever dt)
     // element strides (batch, time, head-or-group)
     long long sx[3], sy[3], sB[3], sC[3], sdt[3], slam[3];
     // inputs
@@ -103,6 +105,10 @@ __device__ __forceinline__ long long ix_dt(const Params &p, int b, int t, int h)
 }
 __device__ __forceinline__ long long ix_lam(const Params &p, int b, int t, int h) {
     return b * p.slam[0] + t * p.slam[1] + h * p.slam[2];
+}
+// per-token rotation angle of pair j (dense [B][L][H][np])
+__device__ __forceinline__ long long ix_th(const Params &p, int b, int t, int h, int j) {
+    return (((long long)b * p.L + t) * p.H + h) * p.np + j;
 }
 __device__ __forceinline__ long long ix_st(const Params &p, int b, int h, int n, int q) {
     return (((long long)b * p.H + h) * p.N + n) * p.P + q;

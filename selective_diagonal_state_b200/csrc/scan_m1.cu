@@ -7,8 +7,9 @@
 //
 // The work is a sequential recurrence per channel whose cost is one exp per
 // (token, channel, state row): the special-function unit (MUFU) bounds it.
-// A thread keeps 8 state rows of one channel in registers (two threads per
-// channel for N = 16) and walks the sequence; 64 channels form a CTA, which
+// A thread keeps 4 state rows of one channel in registers (S = N / 4 threads
+// per channel, their readouts summed with shuffles) and walks the sequence;
+// 64 channels form a CTA, which
 // stages 16 tokens of dt, lambda, x (and dy), B_t and C_t in shared memory with
 // cp.async, double-buffered, so that the loads of the next tile overlap the
 // recurrence of this one.  Pre-state form K_t = A_t K_{t-1} + sigma_t B_t x_t,
@@ -34,7 +35,7 @@ namespace m1 {
 
 constexpr int CPB = 64;   // channels per CTA
 constexpr int TT = 16;    // tokens per staged tile
-constexpr int NSL = 8;    // state rows per thread
+constexpr int NSL = 4;    // state rows per thread
 
 __device__ __forceinline__ float bfu(unsigned short v) { return __uint_as_float((uint32_t)v << 16); }
 
@@ -90,14 +91,20 @@ __device__ __forceinline__ void stage(const Params &p, Tile &tl, int b, int hb, 
     cp_async_commit();
 }
 
-__device__ __forceinline__ void ld8(const unsigned short *src, float (&v)[8]) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(src);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+// 4 consecutive bf16 (8-byte aligned) as floats
+__device__ __forceinline__ void ld4(const unsigned short *src, float (&v)[NSL]) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(src);
+    v[0] = __uint_as_float(w.x << 16);
+    v[1] = __uint_as_float(w.x & 0xffff0000u);
+    v[2] = __uint_as_float(w.y << 16);
+    v[3] = __uint_as_float(w.y & 0xffff0000u);
+}
+// sum over the S lanes of a channel (consecutive lanes)
+template <int S>
+__device__ __forceinline__ float lane_sum(float v) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(u[i] << 16);
-        v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-    }
+    for (int m = 1; m < S; m <<= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
 }
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -106,7 +113,7 @@ __device__ __forceinline__ float ex2f(float x) {
     return y;
 }
 
-// decay rates (times log2 e) of this thread's 8 state rows
+// decay rates (times log2 e) of this thread's state rows
 __device__ __forceinline__ void rates(const Params &p, int h, int half, float (&a)[NSL],
                                       float (&a2)[NSL]) {
 #pragma unroll
@@ -121,7 +128,7 @@ __device__ __forceinline__ void rates(const Params &p, int h, int half, float (&
 
 // ============================================================================
 template <int S>
-__global__ void __launch_bounds__(64 * S) k_m1_fwd(Params p, float *kept) {
+__global__ void __launch_bounds__(64 * S, 2) k_m1_fwd(Params p, float *kept) {
     using namespace m1;
     __shared__ __align__(16) Tile tiles[2];
     __shared__ float s_cb[2][TT];
@@ -163,11 +170,10 @@ __global__ void __launch_bounds__(64 * S) k_m1_fwd(Params p, float *kept) {
         }
         if (kept) {   // the state entering this tile, for the backward
             float *dst = kept + (((long long)b * p.H + h) * ntile + k) * p.N + NSL * half;
-            reinterpret_cast<float4 *>(dst)[0] = make_float4(K[0], K[1], K[2], K[3]);
-            reinterpret_cast<float4 *>(dst)[1] = make_float4(K[4], K[5], K[6], K[7]);
+            *reinterpret_cast<float4 *>(dst) = make_float4(K[0], K[1], K[2], K[3]);
         }
         __syncthreads();
-#pragma unroll 1
+#pragma unroll 4
         for (int j = 0; j < TT; ++j) {
             const int t = t0 + j;
             const float dt = bfu(tl.dt[j][ch]), x = bfu(tl.x[j][ch]);
@@ -178,15 +184,15 @@ __global__ void __launch_bounds__(64 * S) k_m1_fwd(Params p, float *kept) {
             }
             const float w = fmaf(lam, dt, bn) * x;
             float Bv[NSL], Cv[NSL];
-            ld8(&tl.B[j][NSL * half], Bv);
-            ld8(&tl.C[j][NSL * half], Cv);
+            ld4(&tl.B[j][NSL * half], Bv);
+            ld4(&tl.C[j][NSL * half], Cv);
             float yp = 0.f;
 #pragma unroll
             for (int i = 0; i < NSL; ++i) {
                 K[i] = fmaf(ex2f(a2[i] * dt), K[i], w * Bv[i]);
                 yp = fmaf(Cv[i], K[i], yp);
             }
-            if (S == 2) yp += __shfl_xor_sync(0xffffffffu, yp, 1);
+            yp = lane_sum<S>(yp);
             if (half == 0)
                 s_y[j][ch] = __bfloat16_as_ushort(
                     __float2bfloat16_rn(fmaf(fmaf(-bn, s_cb[buf][j], D), x, yp)));
@@ -216,19 +222,22 @@ __global__ void __launch_bounds__(64 * S) k_m1_fwd(Params p, float *kept) {
 }
 
 // ============================================================================
-// Sum of 16 values over the 32 / S lanes of a warp that share `half`: afterwards
-// lane l holds, in v[0], the total of value ((l / S) & 15) of its half
-// (butterfly reduce-scatter over lane bits S .. 16, fixed order).
+// Sum of 2 NSL = 8 values over the 32 / S lanes of a warp that hold the same
+// rows of different channels (lane = S * channel + sub): butterfly
+// reduce-scatter over lane bits 16 .. S in a fixed order.  Afterwards lane l
+// holds, in v[0], the total of value (l >> 2) & 7 of its `sub` (for S = 2 the
+// last level adds lane pairs that already hold the same value index, so both
+// lanes of a pair end with the same total).
 template <int S>
-__device__ __forceinline__ void chan_reduce16(float (&v)[16], int lane) {
-    int cur = 16;
+__device__ __forceinline__ void chan_reduce8(float (&v)[2 * m1::NSL], int lane) {
+    int cur = 2 * m1::NSL;
 #pragma unroll
     for (int m = 16; m >= S; m >>= 1) {
         if (cur > 1) {
             const bool up = (lane & m) != 0;
             const int hl = cur / 2;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < m1::NSL; ++i) {
                 if (i < hl) {
                     const float send = up ? v[i] : v[i + hl];
                     const float keep = up ? v[i + hl] : v[i];
@@ -243,8 +252,8 @@ __device__ __forceinline__ void chan_reduce16(float (&v)[16], int lane) {
 }
 
 template <int S>
-__global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, float *bc_part,
-                                                   float *par_part) {
+__global__ void __launch_bounds__(64 * S, 2) k_m1_bwd(Params p, const float *kept, float *bc_part,
+                                                      float *par_part) {
     using namespace m1;
     constexpr int NT = 64 * S;
     constexpr int NW = NT / 32;
@@ -294,11 +303,10 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
         {
             const float *src = kept + (((long long)b * p.H + h) * ntile + k) * p.N + NSL * half;
             const float4 k0 = __ldg(reinterpret_cast<const float4 *>(src));
-            const float4 k1 = __ldg(reinterpret_cast<const float4 *>(src) + 1);
-            float K[NSL] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            float K[NSL] = {k0.x, k0.y, k0.z, k0.w};
 #pragma unroll
             for (int i = 0; i < NSL; ++i) Ks[i * NT + tid] = K[i];
-#pragma unroll 1
+#pragma unroll 4
             for (int j = 0; j < TT; ++j) {
                 const int t = t0 + j;
                 const float dt = bfu(tl.dt[j][ch]), x = bfu(tl.x[j][ch]);
@@ -309,7 +317,7 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
                 }
                 const float w = fmaf(lam, dt, bn) * x;
                 float Bv[NSL];
-                ld8(&tl.B[j][NSL * half], Bv);
+                ld4(&tl.B[j][NSL * half], Bv);
 #pragma unroll
                 for (int i = 0; i < NSL; ++i) {
                     K[i] = fmaf(ex2f(a2[i] * dt), K[i], w * Bv[i]);
@@ -322,7 +330,7 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
 #pragma unroll 1
         for (int j = TT - 1; j >= 0; --j) {
             const int t = t0 + j;
-            float v[16];   // dB (8), dC (8) of this thread's rows
+            float v[2 * NSL];   // dB, dC of this thread's rows
             if (t < L) {
                 const float dt = bfu(tl.dt[j][ch]), x = bfu(tl.x[j][ch]), dy = bfu(tl.dy[j][ch]);
                 float lam = 1.f, bn = 0.f;
@@ -332,8 +340,8 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
                 }
                 const float sig = fmaf(lam, dt, bn), cbt = s_cb[j];
                 float Bv[NSL], Cv[NSL];
-                ld8(&tl.B[j][NSL * half], Bv);
-                ld8(&tl.C[j][NSL * half], Cv);
+                ld4(&tl.B[j][NSL * half], Bv);
+                ld4(&tl.C[j][NSL * half], Cv);
                 const float bxd = bn * x * dy;
                 float sBG = 0.f, adr = 0.f;
 #pragma unroll
@@ -350,10 +358,8 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
                     adr = fmaf(a[i], dr, adr);
                     G[i] *= e;
                 }
-                if (S == 2) {
-                    sBG += __shfl_xor_sync(0xffffffffu, sBG, 1);
-                    adr += __shfl_xor_sync(0xffffffffu, adr, 1);
-                }
+                sBG = lane_sum<S>(sBG);
+                adr = lane_sum<S>(adr);
                 const float dsig = sBG * x;                 // = dgamma_t = part of dbeta_{t+1}
                 const float dbn = dsig - cbt * x * dy;      // dbeta_{t+1}
                 finish(dbn);                                // token t + 1 is complete
@@ -369,21 +375,21 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                for (int i = 0; i < 2 * NSL; ++i) v[i] = 0.f;
             }
-            chan_reduce16<S>(v, lane);
-            // after the reduction lane l holds value ((l >> 1) & 15) of its half (for S = 1
-            // the two lanes of a pair hold the same total)
-            red[(warp * TT + j) * 32 + ((lane >> 1) & 15) * 2 + (S == 2 ? half : 0)] = v[0];
+            chan_reduce8<S>(v, lane);
+            // lane l now holds value (l >> 2) & 7 (dB rows for 0..3, dC rows for 4..7) of
+            // its sub-block `half` of rows, summed over the warp's channels
+            red[(warp * TT + j) * 32 + ((lane >> 2) & 7) * S + half] = v[0];
         }
         __syncthreads();
         // ---- the CTA's partial dB / dC of the tile: sum over its warps in order -------
-        // red[w][j][vi * 2 + half]: vi < 8 -> dB row 8 half + vi, vi >= 8 -> dC row 8 half + vi - 8
+        // red[w][j][vi * S + sub]: vi < NSL -> dB row NSL sub + vi, else dC row NSL sub + vi - NSL
         for (int i = tid; i < TT * 2 * p.N; i += NT) {
             const int j = i / (2 * p.N), r = i % (2 * p.N);
             const int kind = r / p.N, n = r % p.N;           // kind 0 = dB, 1 = dC
-            const int hf = n / NSL, vi = kind * NSL + n % NSL;
-            const int slot = S == 2 ? vi * 2 + hf : vi * 2;
+            const int sub = n / NSL, vi = kind * NSL + n % NSL;
+            const int slot = vi * S + sub;
             float s = 0.f;
             for (int w = 0; w < NW; ++w) s += red[(w * TT + j) * 32 + slot];
             const int t = t0 + j;
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(64 * S) k_m1_bwd(Params p, const float *kept, 
         if (p.dw0) p.dw0[ii] = beta0 * G[i];
         if (p.w0) db0 = fmaf(G[i], p.w0[ii], db0);
     }
-    if (S == 2) db0 += __shfl_xor_sync(0xffffffffu, db0, 1);
+    db0 = lane_sum<S>(db0);
     finish(db0);
     // per-(b, h) partial parameter gradients: sum_t dt drho per row, <dy, x>
 #pragma unroll
@@ -478,9 +484,9 @@ size_t m1_part_floats(long long B, long long L, long long H, int N) {
 cudaError_t m1_forward(const Params &p, float *kept, cudaStream_t st) {
     const dim3 grid(p.H / m1::CPB, p.Bsz);
     if (p.N == 16) {
-        k_m1_fwd<2><<<grid, 128, 0, st>>>(p, kept);
+        k_m1_fwd<4><<<grid, 256, 0, st>>>(p, kept);
     } else {
-        k_m1_fwd<1><<<grid, 64, 0, st>>>(p, kept);
+        k_m1_fwd<2><<<grid, 128, 0, st>>>(p, kept);
     }
     profile_mark(st, "k_m1_fwd");
     return cudaGetLastError();
@@ -509,17 +515,17 @@ cudaError_t m1_backward(const Params &p, float *kept, bool kept_ready, float *pa
     float *par_part = part + (size_t)p.Bsz * p.L * (p.H / m1::CPB) * 2 * p.N;
     const dim3 grid(p.H / m1::CPB, p.Bsz);
     if (p.N == 16) {
+        const size_t sm = m1_bwd_smem<4>();
+        if ((e = cudaFuncSetAttribute(k_m1_bwd<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)sm)) != cudaSuccess)
+            return e;
+        k_m1_bwd<4><<<grid, 256, sm, st>>>(p, kept, bc_part, par_part);
+    } else {
         const size_t sm = m1_bwd_smem<2>();
         if ((e = cudaFuncSetAttribute(k_m1_bwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)sm)) != cudaSuccess)
             return e;
         k_m1_bwd<2><<<grid, 128, sm, st>>>(p, kept, bc_part, par_part);
-    } else {
-        const size_t sm = m1_bwd_smem<1>();
-        if ((e = cudaFuncSetAttribute(k_m1_bwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)sm)) != cudaSuccess)
-            return e;
-        k_m1_bwd<1><<<grid, 64, sm, st>>>(p, kept, bc_part, par_part);
     }
     profile_mark(st, "k_m1_bwd");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -182,17 +182,23 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
     {
         const Lanes2D l = lanes2d(nmode);
         for (int hc = 0; hc < HC; ++hc) {
+            const int h = hbase + hc;
             for (int tt = l.ty; tt < T; tt += l.ny) {
                 const float dv = s.dt[hc * (T + 1) + tt];
+                const bool tok_ok = h < p.H && t0 + tt < p.L;
                 float *cf = s.coef + (hc * T + tt) * NSL;
                 for (int m = l.tx; m < nmode; m += l.W) {
                     const float a = s.a[hc * p.ndec + (p.per_coord ? m : 0)];
                     if (m < p.nr) {
-                        cf[s.slot[m]] = expf(dv * a);
+                        cf[s.slot[m]] = expf(m < p.nst ? a : dv * a);   // static rows: e^{a}
                     } else {
                         const int j = m - p.nr;
                         float e = expf(dv * a), sn, cs;
-                        sincosf(dv * s.w[hc * (p.np > 0 ? p.np : 1) + j], &sn, &cs);
+                        // angle of step t: per token, or the pair's frequency times dt_t
+                        const float phi =
+                            p.angle_tok ? (tok_ok ? p.theta[ix_th(p, b, t0 + tt, h, j)] : 0.f)
+                                        : dv * s.w[hc * (p.np > 0 ? p.np : 1) + j];
+                        sincosf(phi, &sn, &cs);
                         const int sl = s.slot[p.nr + 2 * j];
                         cf[sl] = e * cs;
                         cf[sl + 1] = e * sn;
@@ -223,7 +229,7 @@ __device__ void init_rates(const Params &p, Smem &s, int hbase, int NSL, int NGL
     }
     for (int i = threadIdx.x; i < g.HC * p.np; i += blockDim.x) {
         int hc = i / p.np, j = i % p.np, h = min(hbase + hc, p.H - 1);
-        s.w[i] = p.theta[h * p.np + j];
+        s.w[i] = p.angle_tok ? 0.f : p.theta[h * p.np + j];
     }
     for (int n = threadIdx.x; n < p.N; n += blockDim.x) s.slot[n] = slot_of<NR, NPR>(n, p.nr, g.NQ);
     // padding slots must read as zero for the whole kernel
@@ -718,7 +724,8 @@ __device__ __forceinline__ ModeInfo mode_info(const Params &p, int h, int m) {
     mi.n0 = 0;
     if (mi.valid) {
         mi.a = neg_exp(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
-        if (mi.pair) mi.w = p.theta[h * p.np + (m - p.nr)];
+        // per-token angles: the angle's gradient leaves through dtheta, not ddt
+        if (mi.pair && !p.angle_tok) mi.w = p.theta[h * p.np + (m - p.nr)];
         mi.n0 = m < p.nr ? m : p.nr + 2 * (m - p.nr);
     }
     return mi;
@@ -774,9 +781,14 @@ __device__ __forceinline__ void units_local_item(const Params &p, float *smem, i
                 }
                 cr += xr - yr;
                 ci += xi - yi;
-                dA = fmaf(dv, cr, dA);
+                // a static row's log-transition is a itself: weight 1, nothing to ddt
+                const bool stat = m < p.nst;
+                dA = fmaf(stat ? 1.f : dv, cr, dA);
                 if (pair) dth = fmaf(dv, -ci, dth);
-                contrib = mi.a * cr + (pair ? -mi.w * ci : 0.f);
+                // per-token angle: the local part of dL/dphi_t (the carry from
+                // later time blocks is added by k_bwd_units_carry)
+                if (pair && p.angle_tok) p.dtheta[ix_th(p, b, t, h, m - p.nr)] = -ci;
+                contrib = stat ? 0.f : mi.a * cr + (pair ? -mi.w * ci : 0.f);
             }
             if (m == 0) {
                 sdt += dv;
@@ -848,9 +860,17 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
         }
         float contrib = 0.f;
         if (mi.valid) {
-            dA += blk[4 * m + 2] + car * sdt;
+            const bool stat = m < p.nst;
+            // static rows: the carried sum counts once per token of the block
+            const float ntok = (float)(min(p.L, (tb + 1) * TBL) - tb * TBL);
+            dA += blk[4 * m + 2] + car * (stat ? ntok : sdt);
             if (mi.pair) dth += blk[4 * m + 3] - cai * sdt;
-            contrib = mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
+            contrib = stat ? 0.f : mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
+            if (mi.pair && p.angle_tok && cai != 0.f) {
+                const int tend = min(p.L, (tb + 1) * TBL);
+                for (int t = tb * TBL; t < tend; ++t)
+                    p.dtheta[ix_th(p, b, t, h, m - p.nr)] -= cai;
+            }
         }
         s_c[m] = contrib;
         __syncthreads();
@@ -876,7 +896,7 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
         for (int j = 0; j < nmode; ++j) acc += s_c[j];
         part[0] = acc;
     }
-    if (mi.pair) part[p.ndec + (m - p.nr)] = dth;
+    if (mi.pair && !p.angle_tok) part[p.ndec + (m - p.nr)] = dth;
     if (m == 0) part[p.ndec + p.np] = dD;
 }
 
@@ -977,7 +997,7 @@ __global__ void k_bwd_params(Params p) {
         if (k < p.ndec) {
             p.dA_log[h * p.ndec + k] = acc * neg_exp(p.A_log[h * p.ndec + k]);
         } else if (k < p.ndec + p.np) {
-            if (p.dtheta) p.dtheta[h * p.np + (k - p.ndec)] = acc;
+            if (p.dtheta && !p.angle_tok) p.dtheta[h * p.np + (k - p.ndec)] = acc;
         } else if (p.dD) {
             p.dD[h] = (p.O == p.R) ? acc : 0.f;
         }

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(stepk::THREADS) k_scan_step(Params p, float *h
         };
         for (int n = 0; n < p.nr; ++n) {
             const float a = -expf(p.A_log[h * p.ndec + (p.per_coord ? n : 0)]);
-            const float e = expf(dt * a);
+            const float e = expf(n < p.nst ? a : dt * a);   // static rows: e^{a}
             const long long i0 = ix_st(p, b, h, n, q);
             const float wn = write_of(n);
             const float wp = (p.two_ep && ws) ? ws[i0] : 0.f;
@@ -65,7 +65,10 @@ __global__ void __launch_bounds__(stepk::THREADS) k_scan_step(Params p, float *h
             const float a = -expf(p.A_log[h * p.ndec + (p.per_coord ? p.nr + j : 0)]);
             const float mag = expf(dt * a);
             float sn, cs;
-            sincosf(dt * p.theta[h * p.np + j], &sn, &cs);
+            // per-token angles: theta holds this token's [B][H][np] angles
+            sincosf(p.angle_tok ? p.theta[((long long)b * p.H + h) * p.np + j]
+                                : dt * p.theta[h * p.np + j],
+                    &sn, &cs);
             const float er = mag * cs, ei = mag * sn;
             const long long i0 = ix_st(p, b, h, n0, q), i1 = ix_st(p, b, h, n0 + 1, q);
             const float wr = write_of(n0), wi = write_of(n0 + 1);

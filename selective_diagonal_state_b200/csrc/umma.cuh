@@ -176,6 +176,16 @@ __device__ __forceinline__ void tma_store_5d(const void *tmap, const void *src, 
         "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(src))
         : "memory");
 }
+// Prefetch of the 5-D tile at the given coordinates into L2 (no shared memory
+// involved; coordinates past the tensor's extent are ignored).
+__device__ __forceinline__ void tma_prefetch_5d(const void *tmap, int c0, int c1, int c2, int c3,
+                                                int c4) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];\n" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
 // 1-D bulk copy global -> shared completing on `bar` (no multicast); both
 // addresses 16-byte aligned, `bytes` a multiple of 16.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,

@@ -12,7 +12,7 @@ import dataclasses
 import numpy as np
 
 from . import abi
-from .synthetic import DTYPE_BF16, ScanShape
+from .synthetic import ANGLE_PER_TOKEN, DTYPE_BF16, ScanShape
 
 
 def _torch():
@@ -115,7 +115,9 @@ def alloc_bwd(shape: ScanShape, device="cuda"):
         dx=e(s.batch, s.seqlen, s.nheads, s.rank_in, s.headdim),
         ddt=e(s.batch, s.seqlen, s.nheads),
         dA_log=e(s.nheads, s.n_decay, dt=f),
-        dtheta=e(s.nheads, s.n_pairs, dt=f) if s.n_pairs else None,
+        dtheta=(None if not s.n_pairs else
+                e(s.batch, s.seqlen, s.nheads, s.n_pairs, dt=f) if s.angle_mode == ANGLE_PER_TOKEN
+                else e(s.nheads, s.n_pairs, dt=f)),
         dBm=e(s.batch, s.seqlen, s.ngroups, s.rank_in, s.nstate),
         dCm=e(s.batch, s.seqlen, s.ngroups, s.rank_out, s.nstate),
         dD=e(s.nheads, dt=f),

@@ -18,6 +18,9 @@ these synthetic draws stand in for their five H100 workloads):
 * ``theta ~ U(0, pi)`` per (head, rotation pair).
 * ``B, C ~ N(0, 1/N)`` (``1/(N R)`` for rank-R routing), ``D ~ N(0, 1)``,
   ``x, dy ~ N(0, 1)``.
+* per-token angles (``angle_mode = 1``): ``theta_t = dt_t theta_j (1 + 0.5 xi)``
+  with ``xi ~ N(0, 1)``, drawn after every other tensor, fp32;
+  ``inp["theta"]`` then holds them, ``[B, L, H, n_pairs]``.
 
 Draw order, from one ``numpy.random.Generator(PCG64(seed))``:
 ``A_log, theta, D, dt0, z, lambda_logit, B, C, x, dy``.
@@ -34,6 +37,8 @@ DTYPE_F32 = 0
 DTYPE_BF16 = 1
 DECAY_PER_HEAD = 0
 DECAY_PER_COORD = 1
+ANGLE_STATIC = 0
+ANGLE_PER_TOKEN = 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,6 +61,12 @@ class ScanShape:
     # Mamba-1 recovery: A_n = -(n+1) instead of the random draw
     fixed_mamba1_A: bool = False
     name: str = ""
+    # 0: rotation angle dt_t theta[h][j]; 1: per-token angles theta[b][t][h][j]
+    # (the data-dependent angles of Mamba-3's complex state)
+    angle_mode: int = 0
+    # the first n_static real rows are static: transition exp(a_n) per step,
+    # independent of dt_t (HybridMamba's real static rows)
+    n_static: int = 0
 
     @property
     def nstate(self) -> int:
@@ -166,4 +177,7 @@ def make_inputs(shape: ScanShape, seed: int, with_dy: bool = True,
         for k in ("dt", "lam", "Bm", "Cm", "x", "dy"):
             if k in out:
                 out[k] = round_bf16(out[k])
+    if s.angle_mode == ANGLE_PER_TOKEN:
+        xi = g.standard_normal((Bt, L, H, s.n_pairs), dtype=f32)
+        out["theta"] = (out["dt"][..., None] * theta[None, None] * (1.0 + 0.5 * xi)).astype(f32)
     return out

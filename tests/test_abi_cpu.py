@@ -38,7 +38,35 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert abi.ssm_scan_abi_version() == 1
+    assert abi.ssm_scan_abi_version() == 2
+
+
+def test_desc_layout_matches_header(lib):
+    """ssm_desc_t: five int64 sizes, eight int32 fields, six int64[3] stride
+    arrays, angle_mode and n_static: 200 bytes, no padding."""
+    assert ctypes.sizeof(abi.Desc) == 5 * 8 + 8 * 4 + 6 * 3 * 8 + 2 * 4
+    assert abi.Desc.angle_mode.offset == 5 * 8 + 8 * 4 + 6 * 3 * 8
+
+
+def test_angle_mode_validation(lib):
+    sh = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=100)
+    d = abi.make_desc(sh)
+    d.angle_mode = 2
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+    assert b"angle_mode" in lib.ssm_scan_last_error()
+    d.angle_mode = 0
+    for bad in (-1, sh.n_real + 1):
+        d.n_static = bad
+        assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+        assert b"n_static" in lib.ssm_scan_last_error()
+    # static rows run on the recurrent kernels too
+    st = abi.make_desc(sh.replace(n_static=16))
+    assert st.n_static == 16
+    assert abi.ssm_scan_workspace_size(st, abi.PASS_FWD) == 0
+    # per-token angles run on the recurrent kernels: no chunk workspace
+    pt = abi.make_desc(sh.replace(angle_mode=S.ANGLE_PER_TOKEN))
+    assert abi.ssm_scan_workspace_size(pt, abi.PASS_FWD) == 0
+    assert abi.ssm_scan_workspace_size(abi.make_desc(sh), abi.PASS_FWD) > 0
 
 
 def test_wait_limit_setter(lib):

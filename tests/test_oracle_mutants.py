@@ -5,6 +5,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_pins as pins
+from selective_diagonal_state_b200 import synthetic as S
 
 MUTANTS = {
     1: "two-endpoint (beta) term dropped",
@@ -16,6 +17,9 @@ MUTANTS = {
     7: "lam * dgamma missing from ddt",
     8: "adjoint uses A instead of A^T",
     9: "feedthrough D u dropped",
+    10: "static rows decay by e^{dt a} instead of e^{a}",
+    11: "static rows' decay gradient weighted by dt",
+    12: "sign of the per-token angle gradient flipped",
 }
 
 PIN_CALLS = [
@@ -30,6 +34,10 @@ PIN_CALLS = [
     lambda: pins.test_gradients_match_central_differences(dict(rank_in=2, rank_out=2, ngroups=2)),
     lambda: pins.test_gradients_match_central_differences(dict(nheads=4, ngroups=2, headdim=1,
                                                                seqlen=8)),
+    lambda: pins.test_static_rows_lti_vandermonde(),
+    lambda: pins.test_static_row_gradients_match_central_differences(S.DECAY_PER_COORD),
+    lambda: pins.test_per_token_angles_equal_complex_modes(),
+    lambda: pins.test_per_token_angle_gradients_match_central_differences(),
 ]
 
 

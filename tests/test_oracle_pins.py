@@ -380,3 +380,156 @@ def test_gradients_match_central_differences(kw):
             an = g[gkey].reshape(-1)[i]
             scale = max(1.0, abs(fd))
             assert abs(fd - an) <= 1e-6 * scale, (key, i, fd, an)
+
+
+# ---------------------------------------------------------------------------
+# per-token rotation angles (the data-dependent angles of Mamba-3's complex
+# state, sungsoo.github.io Part 05)
+# ---------------------------------------------------------------------------
+def test_per_token_angles_reduce_to_static_angles():
+    """theta_t = dt_t theta_j gives the static-angle scan exactly, and the
+    gradients split by the chain rule: ddt_static = ddt + sum_j theta_j dtheta_t,
+    dtheta_static = sum_{b,t} dt_t dtheta_t; every other gradient is unchanged."""
+    sh = tiny(n_real=3, n_pairs=2)
+    inp = inputs(sh, seed=12)
+    pt = sh.replace(angle_mode=1)
+    ip = dict(inp)
+    ip["theta"] = inp["dt"][..., None] * inp["theta"][None, None]
+    ys, yp = oracle.scan_fwd(sh, inp), oracle.scan_fwd(pt, ip)
+    np.testing.assert_allclose(yp["y"], ys["y"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(yp["hT"], ys["hT"], rtol=1e-12, atol=1e-12)
+    gs, gp = oracle.scan_bwd(sh, inp, inp["dy"]), oracle.scan_bwd(pt, ip, ip["dy"])
+    assert gp["dtheta"].shape == (sh.batch, sh.seqlen, sh.nheads, sh.n_pairs)
+    np.testing.assert_allclose(gp["ddt"] + (gp["dtheta"] * inp["theta"][None, None]).sum(-1),
+                               gs["ddt"], rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose((gp["dtheta"] * inp["dt"][..., None]).sum((0, 1)), gs["dtheta"],
+                               rtol=1e-10, atol=1e-10)
+    for k in ("dx", "dBm", "dCm", "dA_log", "dD", "dlam", "dh0", "dw0"):
+        np.testing.assert_allclose(gp[k], gs[k], rtol=1e-10, atol=1e-10, err_msg=k)
+
+
+def test_per_token_angles_equal_complex_modes():
+    """The 2x2 blocks with per-token angles against a complex-mode recurrence
+    whose eigenvalue of step t is exp(dt_t a + i theta_t)."""
+    sh = tiny(n_real=2, n_pairs=3, angle_mode=1)
+    inp = inputs(sh, seed=13)
+    out = oracle.scan_fwd(sh, inp)
+    Bt, L, H, P = sh.batch, sh.seqlen, sh.nheads, sh.headdim
+    nr, npr = sh.n_real, sh.n_pairs
+    y = np.zeros_like(out["y"])
+    for b in range(Bt):
+        for h in range(H):
+            g = group_of(sh, h)
+            a = np.array([decay_rate(sh, inp["A_log"], h, m) for m in range(nr + npr)])
+
+            def to_c(v):
+                return np.concatenate([v[:nr] + 0j, v[nr::2][:npr] + 1j * v[nr + 1::2][:npr]])
+
+            z = np.stack([to_c(inp["h0"][b, h][:, p]) for p in range(P)], axis=1)
+            wp = np.stack([to_c(inp["w0"][b, h][:, p]) for p in range(P)], axis=1)
+            for t in range(L):
+                dt = inp["dt"][b, t, h]
+                gam, bet = weights(sh, inp, b, t, h)
+                ph = np.concatenate([np.zeros(nr), inp["theta"][b, t, h]])
+                eig = np.exp(dt * a + 1j * ph)[:, None]
+                w = to_c(inp["Bm"][b, t, g, 0])[:, None] * inp["x"][b, t, h, 0][None, :]
+                z = eig * (z + bet * wp) + gam * w
+                c = to_c(inp["Cm"][b, t, g, 0])
+                y[b, t, h, 0] = np.real(np.conj(c)[:, None] * z).sum(0) + inp["D"][h] * inp["x"][b, t, h, 0]
+                wp = w
+    np.testing.assert_allclose(out["y"], y, rtol=1e-11, atol=1e-11)
+
+
+def test_per_token_angle_gradients_match_central_differences():
+    sh = tiny(batch=1, seqlen=12, nheads=2, headdim=2, n_real=2, n_pairs=2, angle_mode=1)
+    inp = inputs(sh, seed=14)
+    g = oracle.scan_bwd(sh, inp, inp["dy"])
+    eps = 1e-6
+    rng = np.random.default_rng(1)
+    for key, gkey in (("theta", "dtheta"), ("dt", "ddt"), ("A_log", "dA_log"), ("lam", "dlam")):
+        flat = inp[key].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 24), replace=False):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = _loss(sh, inp)
+            flat[i] = old - eps
+            lm = _loss(sh, inp)
+            flat[i] = old
+            fd = (lp - lm) / (2 * eps)
+            an = g[gkey].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (key, i, fd, an)
+
+
+# ---------------------------------------------------------------------------
+# real static rows (HybridMamba's row types: real static, real dynamic and
+# complex dynamic, sungsoo.github.io Part 08 item 3)
+# ---------------------------------------------------------------------------
+def test_static_rows_lti_vandermonde():
+    """dt, lam, B, C fixed in time: a convolution whose Vandermonde eigenvalues
+    are e^{a_n} on static rows (whatever dt) and e^{dt lam_n} on the others."""
+    sh = tiny(batch=1, seqlen=40, nheads=2, headdim=2, n_real=5, n_pairs=2, n_static=3)
+    inp = inputs(sh, seed=21, state=False)
+    L = sh.seqlen
+    for key in ("dt", "lam", "Bm", "Cm"):
+        inp[key] = np.broadcast_to(inp[key][:, :1], inp[key].shape).copy()
+    inp["dt"][:] = 0.3       # a step away from 1: static and dynamic rows differ
+    y = oracle.scan_fwd(sh, inp)["y"]
+    nr, npr = sh.n_real, sh.n_pairs
+    for h in range(sh.nheads):
+        g = group_of(sh, h)
+        dt = inp["dt"][0, 0, h]
+        gam, bet = weights(sh, inp, 0, 0, h)
+        lam = np.array([decay_rate(sh, inp["A_log"], h, n) + 0j for n in range(nr)] +
+                       [complex(decay_rate(sh, inp["A_log"], h, nr + j), inp["theta"][h, j])
+                        for j in range(npr)])
+        scale = np.array([1.0 if n < sh.n_static else dt for n in range(nr + npr)])
+        a = np.exp(scale * lam)
+        bv, cv = inp["Bm"][0, 0, g, 0], inp["Cm"][0, 0, g, 0]
+        bc = np.concatenate([bv[:nr] + 0j, bv[nr::2] + 1j * bv[nr + 1::2]])
+        cc = np.concatenate([cv[:nr] + 0j, cv[nr::2] + 1j * cv[nr + 1::2]])
+        V = a[:, None] ** np.arange(L)[None, :]
+        K = np.real((np.conj(cc) * bc) @ V) * (gam + bet)
+        K[0] = gam * np.real(np.conj(cc) @ bc)
+        for p in range(sh.headdim):
+            u = inp["x"][0, :, h, 0, p]
+            n = 2 * L
+            conv = np.fft.irfft(np.fft.rfft(K, n) * np.fft.rfft(u, n), n)[:L]
+            np.testing.assert_allclose(y[0, :, h, 0, p], conv + inp["D"][h] * u,
+                                       rtol=1e-9, atol=1e-10)
+
+
+def test_static_rows_equal_dynamic_rows_at_unit_step():
+    """With dt_t = 1 everywhere a static row and a dynamic row are the same row:
+    equal outputs and decay gradients; ddt loses exactly the static rows' a g_rho."""
+    sh = tiny(n_real=6, n_pairs=2, two_endpoint=1)
+    inp = inputs(sh, seed=22)
+    inp["dt"][:] = 1.0
+    st = sh.replace(n_static=4)
+    y0, y1 = oracle.scan_fwd(sh, inp), oracle.scan_fwd(st, inp)
+    np.testing.assert_allclose(y1["y"], y0["y"], rtol=1e-12, atol=1e-12)
+    g0, g1 = oracle.scan_bwd(sh, inp, inp["dy"]), oracle.scan_bwd(st, inp, inp["dy"])
+    for k in ("dx", "dBm", "dCm", "dA_log", "dtheta", "dD", "dlam", "dh0", "dw0"):
+        np.testing.assert_allclose(g1[k], g0[k], rtol=1e-10, atol=1e-10, err_msg=k)
+    assert np.abs(g1["ddt"] - g0["ddt"]).max() > 1e-3
+
+
+@pytest.mark.parametrize("decay_mode", [S.DECAY_PER_COORD, S.DECAY_PER_HEAD])
+def test_static_row_gradients_match_central_differences(decay_mode):
+    sh = tiny(batch=1, seqlen=12, nheads=2, headdim=2, n_real=4, n_pairs=2, n_static=2,
+              decay_mode=decay_mode)
+    inp = inputs(sh, seed=23)
+    g = oracle.scan_bwd(sh, inp, inp["dy"])
+    eps = 1e-6
+    rng = np.random.default_rng(2)
+    for key, gkey in (("A_log", "dA_log"), ("dt", "ddt"), ("Bm", "dBm"), ("x", "dx")):
+        flat = inp[key].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 16), replace=False):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = _loss(sh, inp)
+            flat[i] = old - eps
+            lm = _loss(sh, inp)
+            flat[i] = old
+            fd = (lp - lm) / (2 * eps)
+            an = g[gkey].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (key, i, fd, an)

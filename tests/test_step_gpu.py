@@ -31,9 +31,11 @@ def step_through(shape, inp, with_w=True):
     w = dev.w0.clone() if with_w else None
     y = torch.zeros((shape.batch, shape.seqlen, shape.nheads, shape.rank_out, shape.headdim),
                     dtype=scan.io_dtype(shape), device="cuda")
+    per_token = shape.angle_mode == S.ANGLE_PER_TOKEN and shape.n_pairs
     for t in range(shape.seqlen):
         lam_t = dev.lam[:, t] if shape.two_endpoint else None
-        abi.ssm_scan_step(desc, dev.x[:, t], dev.dt[:, t], dev.A_log, dev.theta, dev.Bm[:, t],
+        th = dev.theta[:, t].contiguous() if per_token else dev.theta   # dense [B][H][np]
+        abi.ssm_scan_step(desc, dev.x[:, t], dev.dt[:, t], dev.A_log, th, dev.Bm[:, t],
                           dev.Cm[:, t], dev.D, lam_t, h, w, y[:, t])
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
@@ -53,6 +55,28 @@ CASES = {
 def test_steps_match_sequence(name):
     shape = S.WORKLOADS[name].replace(**CASES[name])
     inp = S.make_inputs(shape, seed=11, with_dy=False, with_state=True)
+    y, h, w = step_through(shape, inp)
+    ref = oracle.scan_fwd(shape, inp)
+    compare("y", to_np(y), ref["y"], shape.dtype_io)
+    compare("hT", to_np(h), ref["hT"], shape.dtype_io)
+    compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
+
+
+def test_steps_with_per_token_angles():
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=7,
+                                               angle_mode=S.ANGLE_PER_TOKEN)
+    inp = S.make_inputs(shape, seed=14, with_dy=False, with_state=True)
+    y, h, w = step_through(shape, inp)
+    ref = oracle.scan_fwd(shape, inp)
+    compare("y", to_np(y), ref["y"], shape.dtype_io)
+    compare("hT", to_np(h), ref["hT"], shape.dtype_io)
+    compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
+
+
+def test_steps_with_static_rows():
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=7,
+                                               n_static=24)
+    inp = S.make_inputs(shape, seed=15, with_dy=False, with_state=True)
     y, h, w = step_through(shape, inp)
     ref = oracle.scan_fwd(shape, inp)
     compare("y", to_np(y), ref["y"], shape.dtype_io)

@@ -16,14 +16,24 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 
-@pytest.fixture(scope="module")
-def case():
+# one shape per chained tensor-core chain: per-coordinate (HybridMamba) and
+# scalar-decay (SSD-MIMO), each several chunks long
+CASES = {
+    "per_coordinate": (S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=320, nheads=4,
+                                                          ngroups=4), abi.ROUTE_CHUNKED),
+    "scalar_decay": (S.WORKLOADS["ssd_mimo_r4"].replace(batch=2, seqlen=150, nheads=4,
+                                                         ngroups=4), abi.ROUTE_SSD),
+}
+
+
+@pytest.fixture(scope="module", params=sorted(CASES))
+def case(request):
     from selective_diagonal_state_b200 import build
     build.build()
     abi.load_library()
-    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=320, nheads=4, ngroups=4)
+    shape, route = CASES[request.param]
     inp = S.make_inputs(shape, seed=61, with_state=True)
-    return shape, inp
+    return shape, inp, route
 
 
 def _timed_out(fn):
@@ -39,11 +49,11 @@ def _timed_out(fn):
 
 
 def test_forward_wait_gives_up_then_recovers(case):
-    shape, inp = case
+    shape, inp, route = case
     dev = scan.to_device(shape, inp)
     _timed_out(lambda: scan.scan_forward(shape, dev))
     y, hT, wT = scan.scan_forward(shape, dev)
-    assert abi.ssm_scan_last_route() == abi.ROUTE_CHUNKED
+    assert abi.ssm_scan_last_route() == route
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
     ref = oracle.scan_fwd(shape, inp)
@@ -52,7 +62,7 @@ def test_forward_wait_gives_up_then_recovers(case):
 
 
 def test_backward_wait_gives_up_then_recovers(case):
-    shape, inp = case
+    shape, inp, route = case
     dev = scan.to_device(shape, inp)
     wsf = scan.alloc_workspace(shape, abi.PASS_FWD)
     scan.scan_forward(shape, dev, workspace=wsf)
@@ -60,7 +70,7 @@ def test_backward_wait_gives_up_then_recovers(case):
     abi.ssm_scan_poll_device_error()
     _timed_out(lambda: scan.scan_backward(shape, dev, saved=wsf))
     g = scan.scan_backward(shape, dev, saved=wsf)
-    assert abi.ssm_scan_last_route() == abi.ROUTE_CHUNKED
+    assert abi.ssm_scan_last_route() == route
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
     gr = oracle.scan_bwd(shape, inp, inp["dy"])
