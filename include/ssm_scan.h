@@ -139,6 +139,10 @@ SSM_API void ssm_desc_set_contiguous(ssm_desc_t *d);
  * SSM_PASS_FWD size also writes the per-chunk products the backward reuses.  Returns 0 for an invalid descriptor (the
  * compute call then reports the error).  The workspace must be 256-byte
  * aligned; its contents need not be initialised and are clobbered.
+ * The SSM_PASS_BWD size is that of the kernels the call takes when every
+ * tensor base is 16-byte aligned (as allocators return them).  A backward
+ * whose tensors are not falls back to the recurrent kernels, which can need
+ * more: it then fails with SSM_ERR_WORKSPACE, and the message gives the size.
  */
 SSM_API size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass);
 

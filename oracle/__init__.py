@@ -31,6 +31,7 @@ class _Desc(ctypes.Structure):
         ("per_coord_decay", ctypes.c_int), ("two_endpoint", ctypes.c_int),
         ("angle_per_token", ctypes.c_int),
         ("n_static", ctypes.c_int),
+        ("zoh", ctypes.c_int),
     ]
 
 
@@ -60,7 +61,8 @@ def _desc(shape) -> _Desc:
     return _Desc(shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups,
                  shape.n_real, shape.n_pairs, shape.rank_in, shape.rank_out,
                  1 if shape.decay_mode == 1 else 0, shape.two_endpoint,
-                 1 if getattr(shape, "angle_mode", 0) == 1 else 0, getattr(shape, "n_static", 0))
+                 1 if getattr(shape, "angle_mode", 0) == 1 else 0, getattr(shape, "n_static", 0),
+                 1 if getattr(shape, "discretization", 0) == 1 else 0)
 
 
 def _p(a):

@@ -45,6 +45,14 @@
  *  Part 08 item 3): the transition of such a row is exp(a_n) at every step,
  *  independent of dt_t (read: "static" = not selective); its write is that of
  *  every other row.
+ *  Exact zero-order hold (zoh = 1; robocikowo.com glossary item 2 names ZOH as
+ *  a discretisation of the continuous system): with the input held constant
+ *  over the step, the continuous state x' = lam x + b u (lam = a on a real
+ *  row, a + i omega on a pair) moves by exactly
+ *      x_t = e^{dt lam} x_{t-1} + ((e^{dt lam} - 1) / lam) b u_t,
+ *  so the write W_t of mode m is scaled by Z = dt phi1(mu), mu = dt a + i phi
+ *  (phi the step's rotation angle), phi1(mu) = (e^mu - 1) / mu, instead of by
+ *  dt.  Only with the Euler form (two_endpoint = 0).
  *  Per-token rotation angles (angle_per_token = 1, the data-dependent angles of
  *  Mamba-3's complex state, sungsoo.github.io Part 05): phi = theta_t[j] is an
  *  input per (batch, token, head, pair) instead of dt_t theta_j, and its
@@ -63,6 +71,7 @@
  *   y, dy [B][L][H][O][P]  h0, w0, hT, wT [B][H][N][P]
  * Head h reads group g = h / (H / G).
  */
+#include <complex.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -81,6 +90,7 @@ typedef struct {
     int two_endpoint;    /* 0: lam == 1 (Euler write) */
     int angle_per_token; /* 0: phi = dt_t theta[h][j]; 1: phi = theta[b][t][h][j] */
     int n_static;        /* the first n_static real rows decay by exp(a_n) per step */
+    int zoh;             /* 1: exact zero-order-hold write (needs two_endpoint = 0, n_static = 0) */
 } oracle_desc;
 
 /* ---- index helpers ---------------------------------------------------- */
@@ -132,6 +142,86 @@ static void make_step(const oracle_desc *d, const double *A_log, const double *t
         sc->ep[j] = exp(dtv * a);
         sc->cp[j] = cos(phi);
         sc->sp[j] = sin(phi);
+    }
+}
+
+/* phi1(mu) = (e^mu - 1) / mu and its derivative, by their Taylor series near 0 */
+static double complex zoh_phi1(double complex mu) {
+    if (cabs(mu) < 0.05) {
+        double complex s = 0.0, term = 1.0;
+        for (int k = 0; k < 14; ++k) {   /* mu^k / (k + 1)! */
+            s += term;
+            term *= mu / (double)(k + 2);
+        }
+        return s;
+    }
+    return (cexp(mu) - 1.0) / mu;
+}
+static double complex zoh_phi1_d(double complex mu) {
+    if (cabs(mu) < 0.05) {
+        double complex s = 0.0, term = 0.5;   /* (k + 1) mu^k / (k + 2)! */
+        for (int k = 0; k < 14; ++k) {
+            s += (double)(k + 1) * term;
+            term *= mu / (double)(k + 3);
+        }
+        return s;
+    }
+    return (cexp(mu) * (mu - 1.0) + 1.0) / (mu * mu);
+}
+
+/* ZOH write coefficient Z_m of every mode m (real rows, then pairs) for one step,
+ * and the derivatives of Z_m with respect to dt, a_m and the angle (theta_j for
+ * static angles, phi_t for per-token ones). */
+typedef struct { double complex *z, *z_dt, *z_a, *z_w; } zoh_coef;
+
+static void make_zoh(const oracle_desc *d, const double *A_log, const double *theta, long b,
+                     long t, long h, double dtv, zoh_coef *zc) {
+    long nd = NDEC(d);
+    for (long m = 0; m < d->n_real + d->n_pairs; ++m) {
+        long n0 = m < d->n_real ? m : d->n_real + 2 * (m - d->n_real);
+        double a = -exp(A_log[h * nd + dec_of_row(d, n0)]);
+        double phi = 0.0, w = 0.0;
+        if (m >= d->n_real) {
+            long j = m - d->n_real;
+            if (d->angle_per_token) {
+                phi = theta[((b * d->seqlen + t) * d->nheads + h) * d->n_pairs + j];
+            } else {
+                w = theta[h * d->n_pairs + j];
+                phi = dtv * w;
+            }
+        }
+        double complex mu = dtv * a + I * phi;
+        double complex f1 = zoh_phi1(mu), f1d = zoh_phi1_d(mu);
+        zc->z[m] = dtv * f1;
+        zc->z_a[m] = dtv * dtv * f1d;
+        if (m >= d->n_real && d->angle_per_token) {
+            zc->z_dt[m] = f1 + dtv * a * f1d;   /* phi does not move with dt */
+            zc->z_w[m] = I * dtv * f1d;          /* d/dphi_t */
+        } else {
+            zc->z_dt[m] = MUT(13) ? f1 : cexp(mu);   /* d/ddt of (e^{dt lam} - 1) / lam */
+            zc->z_w[m] = I * dtv * dtv * f1d;    /* d/dtheta_j */
+        }
+    }
+}
+
+/* H += gamma W (Euler / two-endpoint) or H += Z (.) W per mode (ZOH) */
+static void add_write(const oracle_desc *d, const zoh_coef *zc, double gamma, const double *W,
+                      double *H) {
+    long P = d->headdim, NP = NST(d) * P;
+    if (!d->zoh) {
+        for (long i = 0; i < NP; ++i) H[i] += gamma * W[i];
+        return;
+    }
+    for (long n = 0; n < d->n_real; ++n)
+        for (long p = 0; p < P; ++p) H[n * P + p] += creal(zc->z[n]) * W[n * P + p];
+    for (long j = 0; j < d->n_pairs; ++j) {
+        long re = d->n_real + 2 * j, im = re + 1;
+        double zr = creal(zc->z[d->n_real + j]), zi = cimag(zc->z[d->n_real + j]);
+        for (long p = 0; p < P; ++p) {
+            double wr = W[re * P + p], wi = W[im * P + p];
+            H[re * P + p] += zr * wr - zi * wi;
+            H[im * P + p] += zi * wr + zr * wi;
+        }
     }
 }
 
@@ -205,6 +295,9 @@ static void fwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
     double *coef = tmp + NP;
     step_coef sc = {coef, coef + d->n_real, coef + d->n_real + d->n_pairs,
                     coef + d->n_real + 2 * d->n_pairs};
+    long nm = d->n_real + d->n_pairs;
+    double complex *zbuf = (double complex *)malloc(sizeof(double complex) * (4 * nm + 1));
+    zoh_coef zc = {zbuf, zbuf + nm, zbuf + 2 * nm, zbuf + 3 * nm};
     for (long i = 0; i < NP; ++i) {
         H[i] = h0 ? h0[ix_st(d, b, h, 0, 0) + i] : 0.0;
         Wp[i] = w0 ? w0[ix_st(d, b, h, 0, 0) + i] : 0.0;
@@ -213,10 +306,12 @@ static void fwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
         double gamma, beta, lv;
         step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
         make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
+        if (d->zoh) make_zoh(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &zc);
         make_write(d, x, Bm, b, t, h, g, W);
         for (long i = 0; i < NP; ++i) Z[i] = H[i] + (MUT(1) ? 0.0 : beta) * Wp[i];
         apply_transition(d, &sc, Z, tmp);
-        for (long i = 0; i < NP; ++i) H[i] = tmp[i] + gamma * W[i];
+        memcpy(H, tmp, sizeof(double) * NP);
+        add_write(d, &zc, gamma, W, H);
         for (long o = 0; o < d->rank_out; ++o)
             for (long p = 0; p < P; ++p) {
                 double acc = 0.0;
@@ -229,6 +324,7 @@ static void fwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
     }
     if (hT) memcpy(hT + ix_st(d, b, h, 0, 0), H, sizeof(double) * NP);
     if (wT) memcpy(wT + ix_st(d, b, h, 0, 0), Wp, sizeof(double) * NP);
+    free(zbuf);
 }
 
 static long unit_work_doubles(const oracle_desc *d) {
@@ -297,6 +393,10 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
     double *coef = (double *)calloc(d->n_real + 3 * d->n_pairs + 4, sizeof(double));
     step_coef sc = {coef, coef + d->n_real, coef + d->n_real + d->n_pairs,
                     coef + d->n_real + 2 * d->n_pairs};
+    long nm = d->n_real + d->n_pairs;
+    double complex *zbuf = (double complex *)calloc(4 * nm + 1, sizeof(double complex));
+    zoh_coef zc = {zbuf, zbuf + nm, zbuf + 2 * nm, zbuf + 3 * nm};
+    double *zoh_dphi = (double *)calloc(d->n_pairs + 1, sizeof(double));
     double *H = segH, *W = segW;
 
     /* pass 1: checkpoints */
@@ -312,10 +412,12 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
         double gamma, beta, lv;
         step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
         make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
+        if (d->zoh) make_zoh(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &zc);
         for (long i = 0; i < NP; ++i) Z[i] = H[i] + beta * W[i];
         apply_transition(d, &sc, Z, AZ);
         make_write(d, x, Bm, b, t, h, g, W);
-        for (long i = 0; i < NP; ++i) H[i] = AZ[i] + gamma * W[i];
+        memcpy(H, AZ, sizeof(double) * NP);
+        add_write(d, &zc, gamma, W, H);
     }
 
     /* pass 2: reverse, one segment at a time */
@@ -329,10 +431,12 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
             double gamma, beta, lv;
             step_weights(d, dt, lam, b, t, h, &gamma, &beta, &lv);
             make_step(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &sc);
+            if (d->zoh) make_zoh(d, A_log, theta, b, t, h, dt[ix_bl(d, b, t, h)], &zc);
             for (long i = 0; i < NP; ++i) Z[i] = segH[(k - 1) * NP + i] + beta * segW[(k - 1) * NP + i];
             apply_transition(d, &sc, Z, AZ);
             make_write(d, x, Bm, b, t, h, g, segW + k * NP);
-            for (long i = 0; i < NP; ++i) segH[k * NP + i] = AZ[i] + gamma * segW[k * NP + i];
+            memcpy(segH + k * NP, AZ, sizeof(double) * NP);
+            add_write(d, &zc, gamma, segW + k * NP, segH + k * NP);
         }
         for (long t = t1 - 1; t >= t0; --t) {
             long k = t - t0 + 1;
@@ -365,10 +469,45 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
                     dx[ix_x(d, b, t, h, r, p)] = v;
                 }
             /* H_t = A_t Z_t + gamma W_t */
-            double dgamma = 0.0;
-            for (long i = 0; i < NP; ++i) {
-                dW[i] = gamma * G[i] + Wbar[i];
-                dgamma += G[i] * Wt[i];
+            double dgamma = 0.0, ddt_zoh = 0.0;
+            if (!d->zoh) {
+                for (long i = 0; i < NP; ++i) {
+                    dW[i] = gamma * G[i] + Wbar[i];
+                    dgamma += G[i] * Wt[i];
+                }
+            } else {
+                /* H_t = A_t H_{t-1} + Z (.) W_t: dW = Z^T G, and the gradient of each
+                   mode's Z, g = dL/dRe Z + i dL/dIm Z, reaches dt, a and the angle */
+                make_zoh(d, A_log, theta, b, t, h, dtv, &zc);
+                for (long n = 0; n < d->n_real; ++n) {
+                    double z = creal(zc.z[n]), gz = 0.0;
+                    for (long p = 0; p < P; ++p) {
+                        dW[n * P + p] = z * G[n * P + p] + Wbar[n * P + p];
+                        gz += G[n * P + p] * Wt[n * P + p];
+                    }
+                    ddt_zoh += gz * creal(zc.z_dt[n]);
+                    dA_unit[dec_of_row(d, n)] += gz * creal(zc.z_a[n]);
+                }
+                for (long j = 0; j < d->n_pairs; ++j) {
+                    long m = d->n_real + j, re = d->n_real + 2 * j, im = re + 1;
+                    double zr = creal(zc.z[m]), zi = cimag(zc.z[m]), gr = 0.0, gi = 0.0;
+                    for (long p = 0; p < P; ++p) {
+                        double Gr = G[re * P + p], Gi = G[im * P + p];
+                        double wr = Wt[re * P + p], wi = Wt[im * P + p];
+                        double zt = MUT(14) ? -zi : zi;   /* the mutant applies Z, not Z^T */
+                        dW[re * P + p] = zr * Gr + zt * Gi + Wbar[re * P + p];
+                        dW[im * P + p] = -zt * Gr + zr * Gi + Wbar[im * P + p];
+                        gr += Gr * wr + Gi * wi;
+                        gi += -Gr * wi + Gi * wr;
+                    }
+                    ddt_zoh += gr * creal(zc.z_dt[m]) + gi * cimag(zc.z_dt[m]);
+                    dA_unit[dec_of_row(d, re)] += gr * creal(zc.z_a[m]) + gi * cimag(zc.z_a[m]);
+                    double gw = gr * creal(zc.z_w[m]) + gi * cimag(zc.z_w[m]);
+                    if (d->angle_per_token)
+                        zoh_dphi[j] = gw;
+                    else
+                        dth_unit[j] += gw;
+                }
             }
             for (long i = 0; i < NP; ++i) Z[i] = Hm[i] + beta * Wm[i];
             apply_transition(d, &sc, Z, AZ);
@@ -403,7 +542,8 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
                 dA_unit[di] += dtv * grho;
                 if (d->angle_per_token) {
                     /* phi is an input of its own: its gradient, per token */
-                    dtheta[((b * L + t) * d->nheads + h) * d->n_pairs + j] = MUT(12) ? -gphi : gphi;
+                    dtheta[((b * L + t) * d->nheads + h) * d->n_pairs + j] =
+                        (MUT(12) ? -gphi : gphi) + (d->zoh ? zoh_dphi[j] : 0.0);
                 } else {
                     double w = theta[h * d->n_pairs + j];
                     ddt_acc += w * gphi;
@@ -412,7 +552,7 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
             }
             double dbeta = 0.0;
             for (long i = 0; i < NP; ++i) dbeta += Gz[i] * (MUT(6) ? Wt[i] : Wm[i]);
-            ddt_acc += (MUT(7) ? 0.0 : lv * dgamma) + (1.0 - lv) * dbeta;
+            ddt_acc += (MUT(7) ? 0.0 : lv * dgamma) + (1.0 - lv) * dbeta + ddt_zoh;
             ddt[ix_bl(d, b, t, h)] = ddt_acc;
             if (dlam) dlam[ix_bl(d, b, t, h)] = d->two_endpoint ? dtv * (dgamma - dbeta) : 0.0;
             /* W_t = B_t u_t */
@@ -437,7 +577,7 @@ static void bwd_unit(const oracle_desc *d, long b, long h, const double *x, cons
     if (dh0) memcpy(dh0 + ix_st(d, b, h, 0, 0), G, sizeof(double) * NP);
     if (dw0) memcpy(dw0 + ix_st(d, b, h, 0, 0), Wbar, sizeof(double) * NP);
     free(ckH); free(ckW); free(segH); free(segW); free(G); free(Gz); free(Wbar);
-    free(dW); free(Z); free(AZ); free(coef);
+    free(dW); free(Z); free(AZ); free(coef); free(zbuf); free(zoh_dphi);
 }
 
 int oracle_scan_bwd(const oracle_desc *d, const double *x, const double *dt, const double *A_log,

@@ -339,6 +339,32 @@ SsdBwdWs ssd_bwd_layout(const ssm_desc_t *d) {
     return w;
 }
 
+// Stride conditions of the channel scan and of the scalar-decay chain, which the
+// descriptor alone decides (the kernels also need 16-byte aligned tensor bases,
+// known only at call time).
+bool m1_strides(const ssm_desc_t *d) {
+    auto m8 = [](int64_t v) { return v % 8 == 0; };
+    bool ok = d->stride_x[2] == 1 && d->stride_y[2] == 1 && d->stride_dt[2] == 1;
+    for (int k = 0; k < 2; ++k)
+        ok = ok && m8(d->stride_x[k]) && m8(d->stride_y[k]) && m8(d->stride_dt[k]);
+    if (d->two_endpoint)
+        ok = ok && d->stride_lambda[2] == 1 && m8(d->stride_lambda[0]) && m8(d->stride_lambda[1]);
+    for (int k = 0; k < 3; ++k) ok = ok && m8(d->stride_B[k]) && m8(d->stride_C[k]);
+    return ok;
+}
+bool ssd_strides(const ssm_desc_t *d) {
+    auto st16 = [](int64_t v) { return (v * 2) % 16 == 0; };
+    bool ok = true;
+    for (int k = 0; k < 3; ++k)
+        ok = ok && st16(d->stride_x[k]) && st16(d->stride_y[k]) && st16(d->stride_B[k]) &&
+             st16(d->stride_C[k]);
+    return ok;
+}
+size_t m1_bwd_bytes(const ssm_desc_t *d) {
+    return align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4) +
+           align256(ssm::m1_part_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
+}
+
 BwdWs bwd_layout(const ssm_desc_t *d) {
     BwdWs w;
     const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
@@ -441,19 +467,10 @@ size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass) {
         return (d->batch == 0 || d->seqlen == 0) ? 0 : fwd_layout(d).total_infer;
     if (pass != SSM_PASS_BWD) return 0;
     if (d->batch == 0 || d->seqlen == 0) return 0;
-    const size_t t = bwd_layout(d).total;
-    if (m1_shape(d)) {
-        const size_t t2 = align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4) +
-                          align256(ssm::m1_part_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
-        return t2 > t ? t2 : t;
-    }
-    if (ssd_shape(d)) {
-        // either chain may take the call (the scalar-decay one unless pointer
-        // alignment rules it out): room for both
-        const size_t t2 = ssd_bwd_layout(d).total;
-        return t2 > t ? t2 : t;
-    }
-    return t;
+    // the chain the call takes with 16-byte aligned tensors
+    if (m1_shape(d) && m1_strides(d)) return m1_bwd_bytes(d);
+    if (ssd_shape(d) && ssd_strides(d)) return ssd_bwd_layout(d).total;
+    return bwd_layout(d).total;
 }
 
 int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
@@ -699,11 +716,6 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     if (d->n_pairs > 0 && (rc = check_ptr(dtheta, "dtheta", 4))) return rc;
     if (dlambda && ((uintptr_t)dlambda % es)) return fail(SSM_ERR_ALIGN, "dlambda misaligned");
     const BwdWs lay = bwd_layout(d);
-    const size_t need_ws = ssm_scan_workspace_size(d, SSM_PASS_BWD);
-    if (!workspace || workspace_bytes < need_ws)
-        return fail(SSM_ERR_WORKSPACE, "backward needs %zu bytes of workspace, got %zu",
-                    need_ws, workspace ? workspace_bytes : (size_t)0);
-    if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
     if (saved) {
         const size_t need = fwd_layout(d).total;
         if (need == 0) {
@@ -731,7 +743,22 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     p.ws_blk = (float *)(ws + lay.off_blk);
     p.ws_blkc = (float *)(ws + lay.off_blkc);
     p.nc = (int)((d->seqlen + 63) / 64);
-    if (m1_shape(d) && ssm::m1_supported(p)) {
+    // the chain this call takes, and the workspace it needs
+    const bool use_m1 = m1_shape(d) && ssm::m1_supported(p);
+    const bool use_ssd = !use_m1 && ssd_shape(d) && ssm::ssd_supported(p) &&
+                         ((uintptr_t)dy & 15) == 0 && ((uintptr_t)dx & 15) == 0 &&
+                         (d->nheads != d->ngroups || ((((uintptr_t)dB | (uintptr_t)dC) & 15) == 0));
+    const size_t need_ws = use_m1 ? m1_bwd_bytes(d) : use_ssd ? ssd_bwd_layout(d).total : lay.total;
+    if (!workspace || workspace_bytes < need_ws)
+        return fail(SSM_ERR_WORKSPACE,
+                    "backward needs %zu bytes of workspace, got %zu%s", need_ws,
+                    workspace ? workspace_bytes : (size_t)0,
+                    need_ws > ssm_scan_workspace_size(d, SSM_PASS_BWD)
+                        ? " (tensors that are not 16-byte aligned take the recurrent kernels, "
+                          "which need more than ssm_scan_workspace_size reports)"
+                        : "");
+    if ((uintptr_t)workspace % 256) return fail(SSM_ERR_ALIGN, "workspace is not 256-byte aligned");
+    if (use_m1) {
         const size_t kb = align256(ssm::m1_kept_floats(d->batch, d->seqlen, d->nheads, nstate(d)) * 4);
         float *kept = (float *)ws;
         bool ready = false;
@@ -749,9 +776,7 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
         return SSM_OK;
     }
     if (saved && m1_shape(d)) saved = nullptr;   // states kept by the channel scan: not read here
-    if (ssd_shape(d) && ssm::ssd_supported(p) && ((uintptr_t)dy & 15) == 0 &&
-        ((uintptr_t)dx & 15) == 0 &&
-        (d->nheads != d->ngroups || ((((uintptr_t)dB | (uintptr_t)dC) & 15) == 0))) {
+    if (use_ssd) {
         // scalar-decay chain
         const SsdBwdWs sl = ssd_bwd_layout(d);
         ssm::Params pc = p;

@@ -142,81 +142,26 @@ __device__ __forceinline__ void chunk_scalars(const Params &p, float *f32, int t
     __syncthreads();
 }
 
-// ---- the carry between the chunks of a (b, h), tagged ------------------------------
-// Each fp32 value of the carried state (forward) or adjoint (backward) travels
-// with a 32-bit tag in one 8-byte word: the item of chunk step r (in walking
-// order) writes tag r + 1 into slot (r + 1) & 1 and the next item polls its own
-// words of that slot until every tag reads r + 1.  A word is written and read
-// with single 8-byte accesses, so a matching tag guarantees the value beside
-// it: no fence, no separate counter, one L2 round trip per step.  The slots
-// are zeroed on every call (tag 0 is never waited for).
-// Layout: [slot][b * H + h][column block cq (4)][column j (16)][state row n (128)],
-// so that a warp (32 consecutive rows) touches 256 contiguous bytes.
-__device__ __forceinline__ unsigned long long *ll_ptr(const Params &p, int slot, int bh, int cq,
-                                                      int j, int n) {
-    return reinterpret_cast<unsigned long long *>(p.ws_ring) +
-           ((((long long)slot * p.Bsz * p.H + bh) * 4 + cq) * 16 + j) * NP + n;
-}
-__device__ __forceinline__ void ll_store16(const Params &p, int slot, int bh, int cq, int n,
-                                           uint32_t tag, const float (&v)[16]) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const unsigned long long w =
-            ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v[j]);
-        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(ll_ptr(p, slot, bh, cq, j, n)),
-                     "l"(w)
-                     : "memory");
-    }
-}
-// Wait (at most p.wait_limit polls, none once the call's abort word is set) for
-// the 16 values of tag `tag`; false if they did not all arrive.
-__device__ __forceinline__ bool ll_load16(const Params &p, int slot, int bh, int cq, int n,
-                                          uint32_t tag, float (&v)[16]) {
-    uint32_t got = 0;
-    for (long long it = 0; it < p.wait_limit; ++it) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            if (!((got >> j) & 1u)) {
-                unsigned long long w;
-                asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];"
-                             : "=l"(w)
-                             : "l"(ll_ptr(p, slot, bh, cq, j, n))
-                             : "memory");
-                if ((uint32_t)(w >> 32) == tag) {
-                    v[j] = __uint_as_float((uint32_t)w);
-                    got |= 1u << j;
-                }
-            }
-        }
-        if (got == 0xffffu) return true;
-        if ((it & 15) == 15) {
-            int a;
-            asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];"
-                         : "=r"(a)
-                         : "l"(chain_abort_word(p))
-                         : "memory");
-            if (a) return false;
-        }
-        __nanosleep(32);
-    }
-    return false;
-}
-
-// K_in of thread (state row n, 16 columns from 16 cq): the tagged carry slot,
-// or h0 + beta_0 w0 for the first chunk; false if the carry did not arrive.
-__device__ __forceinline__ bool load_kin(const Params &p, int c, int b, int h, int n, int cq,
+// K_in of thread (state row n, 16 columns from 16 cq): the carry slot, or
+// h0 + beta_0 w0 for the first chunk.
+__device__ __forceinline__ void load_kin(const Params &p, int c, int b, int h, int n, int cq,
                                          float (&kc)[16]) {
-    if (c > 0) {
-        if (!ll_load16(p, c & 1, b * p.H + h, cq, n, (uint32_t)c, kc)) return false;
-        if (n >= p.N)
-#pragma unroll
-            for (int j = 0; j < 16; ++j) kc[j] = 0.f;
-        return true;
-    }
     if (n >= p.N) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) kc[j] = 0.f;
-        return true;
+        return;
+    }
+    if (c > 0) {
+        const float4 *src = carry_ptr(p, c & 1, b * p.H + h, cq, n);
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 v = __ldcg(src + j4 * NP);
+            kc[4 * j4] = v.x;
+            kc[4 * j4 + 1] = v.y;
+            kc[4 * j4 + 2] = v.z;
+            kc[4 * j4 + 3] = v.w;
+        }
+        return;
     }
     float beta0 = 0.f;
     if (p.two_ep)
@@ -228,7 +173,6 @@ __device__ __forceinline__ bool load_kin(const Params &p, int c, int b, int h, i
         if (p.w0) a = fmaf(beta0, p.w0[i0], a);
         kc[j] = a;
     }
-    return true;
 }
 
 // 8 bf16 of row `row`, logical 16-byte chunk `lc` of a 128-byte-swizzled tile
@@ -348,14 +292,6 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
             alog = __ldg(p.A_log + nx.h * p.ndec);
-            if (tid == 0) {   // the next item's tiles stream into L2 while this one runs
-                const int g2 = nx.h / p.hpg;
-                tma_prefetch_5d(&tmX, 0, 0, nx.h, nx.c * Qt, nx.b);
-                for (int kb = 0; kb < nbox; ++kb) {
-                    tma_prefetch_5d(&tmB, 64 * kb, 0, g2, nx.c * Qt, nx.b);
-                    if (want_y) tma_prefetch_5d(&tmC, 64 * kb, 0, g2, nx.c * Qt, nx.b);
-                }
-            }
         }
         {
             const bool okx = mbar_wait(bar_x, par, WAIT_LIMIT);
@@ -422,8 +358,14 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 ssd_raise_error(1);
                 chain_abort(p);
             }
+            if (tid == 0 && ok && c > 0 &&
+                !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
+                ssd_raise_error(2);
+                chain_abort(p);
+                ok = 0;
+            }
             fence_after_sync();
-            if (!__syncthreads_and(ok)) {
+            if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of K_in
                 aborted = true;
                 break;
             }
@@ -433,80 +375,66 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             issue_b(next);
             ++pc_b.issued;
         }
-        // The carry step is the only part of an item on the chain of its (b, h): S_c is
-        // read from TMEM before the wait, K_out leaves right after K_in arrives, and the
-        // K_in tiles (readout operand, saved copy) are written afterwards.
-        int kin_ok = 1;
-        {
+#pragma unroll 1
+        for (int cq = 2 * cb2; cq < 2 * cb2 + 2; ++cq) {
+            // K_in as the bf16 tile of the readout, in X''s place (S_c has read X')
             const int n = row;
+            float kc[16], sc[16];
+            load_kin(p, c, b, h, n, cq, kc);
+            tmem_ld16(t_sc + lane_q + 16u * cq, sc);
             const float E = f32[F_SC + 2];
             unsigned char *sv = p.ws_kp
                 ? reinterpret_cast<unsigned char *>(p.ws_kp + bhc(p, b, h, c) * SLOT_FLOATS)
                 : nullptr;
-            float sc2[2][16];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) tmem_ld16(t_sc + lane_q + 16u * (2 * cb2 + q), sc2[q]);
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float hi[8], lo[8];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int cq = 2 * cb2 + q;
-                float kc[16];
-                if (!load_kin(p, c, b, h, n, cq, kc)) {
-                    kin_ok = 0;
-                    break;
+                for (int j = 0; j < 8; ++j) {
+                    const float v = kc[8 * g8 + j];
+                    hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+                    lo[j] = v - hi[j];
                 }
-                float kn[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) kn[j] = n < N ? fmaf(E, kc[j], sc2[q][j]) : 0.f;
-                if (c + 1 < p.nc) {
-                    ll_store16(p, (c + 1) & 1, bh, cq, n, (uint32_t)(c + 1), kn);
-                } else if (n < N) {
-                    // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write
-                    // W_{L-1} = B_{L-1} u_{L-1} (summed over the R value rows)
-                    const int g = h / p.hpg, tl = L - 1;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
-                        if (p.hT) p.hT[i0] = kn[j];
-                        if (p.wT) {
-                            float w = 0.f;
-                            for (int r = 0; r < p.R; ++r)
-                                w = fmaf(ld_io(p.Bm, ix_B(p, b, tl, g, r, n), 1),
-                                         ld_io(p.x, ix_x(p, b, tl, h, r, 16 * cq + j), 1), w);
-                            p.wT[i0] = w;
-                        }
-                    }
+                const uint32_t off = sw_off(n, 2 * cq + g8);
+                const uint4 wh = pack8(hi);
+                *reinterpret_cast<uint4 *>(sm + SM_XS + off) = wh;
+                if (sv) {
+                    *reinterpret_cast<uint4 *>(sv + off) = wh;
+                    *reinterpret_cast<uint4 *>(sv + TILE + off) = pack8(lo);
                 }
-                // K_in as the bf16 tile of the readout, in X''s place (S_c has read X'),
-                // and its hi / lo tiles for the backward
+            }
+            float kn[16];
 #pragma unroll
-                for (int g8 = 0; g8 < 2; ++g8) {
-                    float hi[8], lo[8];
+            for (int j = 0; j < 16; ++j) kn[j] = n < N ? fmaf(E, kc[j], sc[j]) : 0.f;
+            if (c + 1 < p.nc) {
+                float4 *dst = carry_ptr(p, (c + 1) & 1, bh, cq, n);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float v = kc[8 * g8 + j];
-                        hi[j] = __bfloat162float(__float2bfloat16_rn(v));
-                        lo[j] = v - hi[j];
-                    }
-                    const uint32_t off = sw_off(n, 2 * cq + g8);
-                    const uint4 wh = pack8(hi);
-                    *reinterpret_cast<uint4 *>(sm + SM_XS + off) = wh;
-                    if (sv) {
-                        *reinterpret_cast<uint4 *>(sv + off) = wh;
-                        *reinterpret_cast<uint4 *>(sv + TILE + off) = pack8(lo);
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(kn[4 * j4], kn[4 * j4 + 1], kn[4 * j4 + 2],
+                                                      kn[4 * j4 + 3]));
+            } else if (n < N) {
+                // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write
+                // W_{L-1} = B_{L-1} u_{L-1} (summed over the R value rows)
+                const int g = h / p.hpg, tl = L - 1;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
+                    if (p.hT) p.hT[i0] = kn[j];
+                    if (p.wT) {
+                        float w = 0.f;
+                        for (int r = 0; r < p.R; ++r)
+                            w = fmaf(ld_io(p.Bm, ix_B(p, b, tl, g, r, n), 1),
+                                     ld_io(p.x, ix_x(p, b, tl, h, r, 16 * cq + j), 1), w);
+                        p.wT[i0] = w;
                     }
                 }
             }
         }
-        if (!kin_ok) {
-            ssd_raise_error(2);
-            chain_abort(p);
-        }
         fence_proxy_async();
         fence_before_sync();
-        if (!__syncthreads_and(kin_ok)) {
-            aborted = true;
-            break;
-        }
+        __syncthreads();
+        // the carry of (b, h) is in place: let the next chunk's item go (off the issue path)
+        if (tid == THREADS - 32 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
         if (want_y) {
             // ---- masked scores P = CB (.) W -> bf16 tile in B's place (CB and S_c have
             // read B; CB completed with S_c) -------------------------------------------------
@@ -698,6 +626,7 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     using namespace ssdb;
     using namespace umma;
     using chunkc::bhc;
+    using chunkc::carry_ptr;
     using chunkc::chain_abort;
     using chunkc::chain_abort_word;
     using chunkc::chain_ticket;
@@ -707,10 +636,10 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     using chunkc::ex2_fast;
     using chunkc::NP;
     using chunkc::PhaseCount;
+    using chunkc::publish_count;
     using chunkc::SLOT_FLOATS;
+    using chunkc::wait_count;
     using chunkc::WAIT_LIMIT;
-    using ssdk::ll_load16;
-    using ssdk::ll_store16;
     using ssdk::pack8;
     using ssdk::sw_off;
     using ssdk::unpack8;
@@ -816,16 +745,6 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = ssdk::tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
             alog = __ldg(p.A_log + nx.h * p.ndec);
-            if (tid == 0) {   // the next item's tiles stream into L2 while this one runs
-                const int g2 = nx.h / p.hpg;
-                tma_prefetch_5d(&tmX, 0, 0, nx.h, nx.c * Qt, nx.b);
-                tma_prefetch_5d(&tmDY, 0, 0, nx.h, nx.c * Qt, nx.b);
-                for (int kb = 0; kb < nbox; ++kb) {
-                    tma_prefetch_5d(&tmB, 64 * kb, 0, g2, nx.c * Qt, nx.b);
-                    tma_prefetch_5d(&tmC, 64 * kb, 0, g2, nx.c * Qt, nx.b);
-                }
-                bulk_prefetch_l2(p.ws_kp + bhc(p, nx.b, nx.h, nx.c) * SLOT_FLOATS, 2 * TILE);
-            }
         }
         const float a2 = f32[F_SC], E = f32[F_SC + 2];
         {
@@ -997,28 +916,34 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             }
         }
         // ---- chain step (needs only G_loc): G_in = E G_out + G_loc; Q = <G_out, E K_in> ----
-        // the adjoint leaving this chunk comes, tagged, from the item of chunk c + 1
+        {
+            int ok = 1;
+            // the adjoint leaving this chunk is published by the item of chunk c + 1
+            if (tid == 0 && rr > 0 &&
+                !wait_count(p.ws_flag + bh, rr, chain_abort_word(p), p.wait_limit)) {
+                ssd_raise_error(2);
+                chain_abort(p);
+                ok = 0;
+            }
+            if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of G_out
+                aborted = true;
+                break;
+            }
+        }
         float go[16];   // G_out of (state row `row`, 16 columns from 16 cb4), kept for phase 3
-        int gout_ok = 1;
         {
             const int n = row, cq = cb4;
-            // everything that does not need G_out first: the wait is the chain's only link
             float gl[16];
-            tmem_ld16(tb + T_GL + lane_q + 16u * cq, gl);
-            if (rr > 0) {
-                gout_ok = ll_load16(p, rr & 1, bh, cq, n, (uint32_t)rr, go) ? 1 : 0;
-                if (n >= N)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) go[j] = 0.f;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) go[j] = 0.f;
+            for (int j4 = 0; j4 < 4; ++j4) {
+                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rr > 0 && n < N) a4 = __ldcg(carry_ptr(p, rr & 1, bh, cq, n) + j4 * NP);
+                go[4 * j4] = a4.x;
+                go[4 * j4 + 1] = a4.y;
+                go[4 * j4 + 2] = a4.z;
+                go[4 * j4 + 3] = a4.w;
             }
-            float gi[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) gi[j] = n < N ? fmaf(E, go[j], gl[j]) : 0.f;
-            if (gout_ok && c > 0) ll_store16(p, (rr + 1) & 1, bh, cq, n, (uint32_t)(rr + 1), gi);
-            // Q = <G_out, E K_in> from the entering state's hi / lo tiles (off the chain)
+            tmem_ld16(tb + T_GL + lane_q + 16u * cq, gl);
             const unsigned char *kslot =
                 reinterpret_cast<const unsigned char *>(p.ws_kp + u * SLOT_FLOATS);
             float qb = 0.f;
@@ -1031,9 +956,16 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
 #pragma unroll
                 for (int j = 0; j < 8; ++j) qb = fmaf(go[8 * g8 + j], kh[j] + kl[j], qb);
             }
+            float gi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) gi[j] = n < N ? fmaf(E, go[j], gl[j]) : 0.f;
             float db0 = 0.f;
-            if (!gout_ok || c > 0) {
-                // the carry did not arrive (stop; nothing below is stored), or G_in has left
+            if (c > 0) {
+                float4 *dst = carry_ptr(p, (rr + 1) & 1, bh, cq, n);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4)
+                    __stcg(dst + j4 * NP, make_float4(gi[4 * j4], gi[4 * j4 + 1], gi[4 * j4 + 2],
+                                                      gi[4 * j4 + 3]));
             } else if (n < N) {
                 // the adjoint of K_{-1} = h0 + beta_0 w0: dh0, dw0 = beta_0 dh0, dbeta_0
                 float beta0 = 0.f;
@@ -1057,15 +989,10 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 f32[F_QB + 16 + warp] = db0;
             }
         }
-        if (!gout_ok) {
-            ssd_raise_error(2);
-            chain_abort(p);
-        }
         fence_before_sync();
-        if (!__syncthreads_and(gout_ok)) {
-            aborted = true;
-            break;
-        }
+        __syncthreads();
+        // the carry of chunk c - 1 is in place: let its item go (off the issue path)
+        if (tid == THREADS - 32 && c > 0) publish_count(p.ws_flag + bh, rr + 1);
         // ---- phase 2: dX_d = P^T dY, dC += dCB B, dB = dCB^T C ------------------------
         if (tid == 0) {
             fence_after_sync();
@@ -1438,10 +1365,10 @@ int sm_count();
 
 static int ssd_lg_rank(int R) { return R == 1 ? 0 : (R == 2 ? 1 : (R == 4 ? 2 : -1)); }
 
-// Bytes of the two tagged carry slots of every (b, h): 128 rows x 64 columns x 8 bytes each.
-size_t ssd_ring_bytes(long long B, long long H) { return (size_t)2 * B * H * 128 * 64 * 8; }
-
 // Tokens per chunk of the scalar-decay kernels (128 (token, rank) rows).
+// Bytes of the carry slots: two fp32 32 KB slots per (b, h).
+size_t ssd_ring_bytes(long long B, long long H) { return (size_t)2 * B * H * 128 * 64 * 4; }
+
 int ssd_chunk_tokens(int R) {
     const int lg = ssd_lg_rank(R);
     return lg < 0 ? 0 : (ssdk::ROWS >> lg);
@@ -1494,11 +1421,8 @@ cudaError_t ssd_forward(const Params &p, cudaStream_t st) {
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
         return e;
-    // tagged carry slots start at tag 0, which no item waits for
-    if ((e = cudaMemsetAsync(p.ws_ring, 0, ssd_ring_bytes(p.Bsz, p.H), st)) != cudaSuccess) return e;
-    // two CTAs per SM (shared memory, registers and TMEM columns allow it)
     const long long nitems = (long long)p.nc * p.H * p.Bsz;
-    const int grid = (int)(nitems < 2 * sm_count() ? nitems : 2 * sm_count());
+    const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
     k_ssd_fwd<<<grid, THREADS, SMEM_BYTES, st>>>(mx, mb, mc, my, p, lgR);
     profile_mark(st, "k_ssd_fwd");
     return cudaGetLastError();
@@ -1542,7 +1466,6 @@ cudaError_t ssd_backward(const Params &p, cudaStream_t st) {
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
         return e;
-    if ((e = cudaMemsetAsync(p.ws_ring, 0, ssd_ring_bytes(p.Bsz, p.H), st)) != cudaSuccess) return e;
     // dbeta_0 stays zero without a left endpoint
     if ((e = cudaMemsetAsync(p.sd_db0, 0, sizeof(float) * (size_t)p.Bsz * p.H, st)) != cudaSuccess)
         return e;

@@ -39,6 +39,8 @@ DECAY_PER_HEAD = 0
 DECAY_PER_COORD = 1
 ANGLE_STATIC = 0
 ANGLE_PER_TOKEN = 1
+DISC_EULER = 0
+DISC_ZOH = 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -67,6 +69,9 @@ class ScanShape:
     # the first n_static real rows are static: transition exp(a_n) per step,
     # independent of dt_t (HybridMamba's real static rows)
     n_static: int = 0
+    # 0: Euler / two-endpoint write (dt-scaled); 1: exact zero-order hold
+    # (write scaled by (e^{dt lam} - 1) / lam per mode; needs two_endpoint = 0)
+    discretization: int = 0
 
     @property
     def nstate(self) -> int:

@@ -20,6 +20,8 @@ MUTANTS = {
     10: "static rows decay by e^{dt a} instead of e^{a}",
     11: "static rows' decay gradient weighted by dt",
     12: "sign of the per-token angle gradient flipped",
+    13: "ZOH write's dt-derivative taken as phi1 instead of e^mu",
+    14: "ZOH backward applies Z instead of Z^T to a pair's adjoint",
 }
 
 PIN_CALLS = [
@@ -38,6 +40,8 @@ PIN_CALLS = [
     lambda: pins.test_static_row_gradients_match_central_differences(S.DECAY_PER_COORD),
     lambda: pins.test_per_token_angles_equal_complex_modes(),
     lambda: pins.test_per_token_angle_gradients_match_central_differences(),
+    lambda: pins.test_zoh_equals_matrix_exponential(dict()),
+    lambda: pins.test_zoh_gradients_match_central_differences(dict()),
 ]
 
 

@@ -533,3 +533,86 @@ def test_static_row_gradients_match_central_differences(decay_mode):
             fd = (lp - lm) / (2 * eps)
             an = g[gkey].reshape(-1)[i]
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (key, i, fd, an)
+
+
+# ---------------------------------------------------------------------------
+# exact zero-order-hold discretisation (robocikowo.com glossary item 2)
+# ---------------------------------------------------------------------------
+def _continuous_A(shape, inp, b, t, h):
+    """Real N x N generator of the continuous system of head h at step t:
+    a_n on real rows, [[a, -w], [w, a]] on pair j (w = theta_j, or the
+    per-token angle divided by the step)."""
+    nr, npr, N = shape.n_real, shape.n_pairs, shape.nstate
+    A = np.zeros((N, N))
+    dt = inp["dt"][b, t, h]
+    for n in range(nr):
+        A[n, n] = decay_rate(shape, inp["A_log"], h, n)
+    for j in range(npr):
+        a = decay_rate(shape, inp["A_log"], h, nr + j)
+        w = (inp["theta"][b, t, h, j] / dt if shape.angle_mode == S.ANGLE_PER_TOKEN
+             else inp["theta"][h, j])
+        r = nr + 2 * j
+        A[r:r + 2, r:r + 2] = [[a, -w], [w, a]]
+    return A
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(angle_mode=S.ANGLE_PER_TOKEN),
+                                dict(decay_mode=S.DECAY_PER_HEAD, n_pairs=0)])
+def test_zoh_equals_matrix_exponential(kw):
+    """Zero-order hold is exact for an input held over the step: the step's
+    transition and write are the blocks of expm([[A, I], [0, 0]] dt) (Van
+    Loan), computed here by scipy's matrix exponential on the real 2x2 form."""
+    from scipy.linalg import expm
+    sh = tiny(two_endpoint=0, discretization=S.DISC_ZOH, **kw)
+    inp = inputs(sh, seed=31)
+    out = oracle.scan_fwd(sh, inp)
+    N, P = sh.nstate, sh.headdim
+    y = np.zeros_like(out["y"])
+    for b in range(sh.batch):
+        for h in range(sh.nheads):
+            g = group_of(sh, h)
+            H = inp["h0"][b, h].copy()
+            for t in range(sh.seqlen):
+                M = np.zeros((2 * N, 2 * N))
+                M[:N, :N] = _continuous_A(sh, inp, b, t, h)
+                M[:N, N:] = np.eye(N)
+                E = expm(M * inp["dt"][b, t, h])
+                W = inp["Bm"][b, t, g, 0][:, None] * inp["x"][b, t, h, 0][None, :]
+                H = E[:N, :N] @ H + E[:N, N:] @ W
+                y[b, t, h, 0] = inp["Cm"][b, t, g, 0] @ H + inp["D"][h] * inp["x"][b, t, h, 0]
+    np.testing.assert_allclose(out["y"], y, rtol=1e-10, atol=1e-10)
+
+
+def test_zoh_tends_to_euler_for_slow_modes():
+    """|dt lam| -> 0: (e^{dt lam} - 1) / lam -> dt, the Euler write."""
+    sh = tiny(two_endpoint=0)
+    inp = inputs(sh, seed=32)
+    inp["A_log"][:] = -30.0
+    inp["theta"][:] = 1e-12
+    a = oracle.scan_fwd(sh, inp)["y"]
+    b = oracle.scan_fwd(sh.replace(discretization=S.DISC_ZOH), inp)["y"]
+    np.testing.assert_allclose(b, a, rtol=1e-9, atol=1e-9)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(angle_mode=S.ANGLE_PER_TOKEN),
+                                dict(decay_mode=S.DECAY_PER_HEAD)])
+def test_zoh_gradients_match_central_differences(kw):
+    sh = tiny(batch=1, seqlen=10, nheads=2, headdim=2, n_real=3, n_pairs=2, two_endpoint=0,
+              discretization=S.DISC_ZOH, **kw)
+    inp = inputs(sh, seed=33)
+    g = oracle.scan_bwd(sh, inp, inp["dy"])
+    eps = 1e-6
+    rng = np.random.default_rng(3)
+    for key, gkey in (("dt", "ddt"), ("A_log", "dA_log"), ("theta", "dtheta"), ("Bm", "dBm"),
+                      ("x", "dx"), ("Cm", "dCm"), ("h0", "dh0")):
+        flat = inp[key].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 12), replace=False):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = _loss(sh, inp)
+            flat[i] = old - eps
+            lm = _loss(sh, inp)
+            flat[i] = old
+            fd = (lp - lm) / (2 * eps)
+            an = g[gkey].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (key, i, fd, an)

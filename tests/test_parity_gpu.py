@@ -1,5 +1,7 @@
 """GPU parity: the CUDA scan (through the C ABI) against the fp64 oracle, element
 by element, on the same seeded inputs."""
+import re
+
 import numpy as np
 import pytest
 
@@ -187,7 +189,7 @@ def test_per_token_angles(kw):
 
 @pytest.mark.parametrize("kw", [
     dict(n_static=16),                        # HybridMamba heads: 16 static of 64 real rows
-    dict(n_real=96, n_pairs=16, n_static=48),  # another mixture of the three row types
+    dict(n_real=32, n_pairs=16, n_static=24),  # another mixture (N = 64)
     dict(n_static=64, dtype_io=S.DTYPE_F32),  # every real row static
     dict(n_static=8, decay_mode=S.DECAY_PER_HEAD, two_endpoint=0),
     dict(n_static=16, angle_mode=S.ANGLE_PER_TOKEN, seqlen=70),
@@ -291,6 +293,32 @@ def test_strided_views():
     torch.cuda.synchronize()
     got = yb[..., : y_ref.shape[3] * y_ref.shape[4]].reshape(y_ref.shape)
     assert float((got - y_ref).abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("name", ["mamba2_siso", "mamba1_siso"])
+def test_unaligned_tensors_take_recurrent_route(name):
+    """dy 2 bytes past a 16-byte boundary: the backward cannot take the chain
+    whose workspace ssm_scan_workspace_size reports, says so, and with the
+    recurrent kernels' workspace gives the oracle's gradients."""
+    shape = S.WORKLOADS[name].replace(**REDUCED[name])
+    inp = S.make_inputs(shape, seed=17)
+    dev = scan.to_device(shape, inp)
+    buf = torch.empty(dev.dy.numel() + 1, dtype=dev.dy.dtype, device="cuda")
+    dy_off = buf[1:].view(dev.dy.shape)
+    dy_off.copy_(dev.dy)
+    dev.dy = dy_off
+    with pytest.raises(abi.SsmError) as ei:
+        scan.scan_backward(shape, dev, workspace=scan.alloc_workspace(shape, abi.PASS_BWD))
+    assert ei.value.code == -6
+    need = int(re.search(r"needs (\d+) bytes", str(ei.value)).group(1))
+    ws = (torch.empty(need, dtype=torch.uint8, device="cuda"), need)
+    g = scan.scan_backward(shape, dev, workspace=ws)
+    assert abi.ssm_scan_last_route() == abi.ROUTE_RECURRENT
+    torch.cuda.synchronize()
+    gr = oracle.scan_bwd(shape, inp, inp["dy"])
+    for k, a, b in (("dx", g.dx, gr["dx"]), ("ddt", g.ddt, gr["ddt"]), ("dB", g.dBm, gr["dBm"]),
+                    ("dC", g.dCm, gr["dCm"]), ("dA_log", g.dA_log, gr["dA_log"])):
+        compare(k, to_np(a), b, shape.dtype_io)
 
 
 def test_backward_deterministic():
