@@ -68,6 +68,13 @@ enum ssm_decay_mode { SSM_DECAY_PER_HEAD = 0, SSM_DECAY_PER_COORD = 1 };
  * theta[b][t][h][j] (a data-dependent angle per token, the complex state of
  * Mamba-3 written as 2x2 rotations, sungsoo.github.io Part 05). */
 enum ssm_angle_mode { SSM_ANGLE_STATIC = 0, SSM_ANGLE_PER_TOKEN = 1 };
+/* Write of step t: SSM_DISC_EULER scales W_t = B_t u_t by dt_t (the two-endpoint
+ * form when two_endpoint == 1); SSM_DISC_ZOH is the exact zero-order hold
+ * ("State Space Models", robocikowo.com, glossary item 2): with the input held
+ * over the step, mode m (rate lam = a, or a + i omega on a pair) receives
+ * ((e^{dt lam} - 1) / lam) W_t, complex on a pair (= dt phi1(dt a + i phi),
+ * phi1(z) = (e^z - 1) / z, phi the step's rotation angle). */
+enum ssm_discretization { SSM_DISC_EULER = 0, SSM_DISC_ZOH = 1 };
 /* SSM_PASS_FWD: a forward that keeps what ssm_scan_bwd_saved reads;
  * SSM_PASS_FWD_INFER: a forward only (smaller workspace). */
 enum ssm_pass { SSM_PASS_FWD = 0, SSM_PASS_BWD = 1, SSM_PASS_FWD_INFER = 2 };
@@ -125,6 +132,9 @@ typedef struct ssm_desc {
                                    complex dynamic ones, sungsoo.github.io Part 08 item 3);
                                    their write is that of every row.  n_static > 0 is taken
                                    by the token-by-token recurrent kernels */
+    int32_t discretization;     /* enum ssm_discretization.  SSM_DISC_ZOH needs two_endpoint == 0
+                                   and n_static == 0, and is taken by the recurrent kernels */
+    int32_t reserved_;          /* must be 0 */
 } ssm_desc_t;
 
 /* Fill every stride of *d for dense tensors of the sizes already set. */

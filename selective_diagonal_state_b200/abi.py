@@ -50,6 +50,7 @@ class Desc(ctypes.Structure):
         ("stride_B", ctypes.c_int64 * 3), ("stride_C", ctypes.c_int64 * 3),
         ("stride_dt", ctypes.c_int64 * 3), ("stride_lambda", ctypes.c_int64 * 3),
         ("angle_mode", ctypes.c_int32), ("n_static", ctypes.c_int32),
+        ("discretization", ctypes.c_int32), ("reserved_", ctypes.c_int32),
     ]
 
 
@@ -115,6 +116,7 @@ def make_desc(shape: ScanShape) -> Desc:
     d.chunk, d.decay_mode = shape.chunk, shape.decay_mode
     d.two_endpoint, d.dtype_io = shape.two_endpoint, shape.dtype_io
     d.angle_mode, d.n_static = shape.angle_mode, shape.n_static
+    d.discretization = shape.discretization
     load_library().ssm_desc_set_contiguous(ctypes.byref(d))
     return d
 

@@ -155,6 +155,11 @@ int validate_desc(const ssm_desc_t *d) {
         return fail(SSM_ERR_ARG, "unknown angle_mode %d", d->angle_mode);
     if (d->n_static < 0 || d->n_static > d->n_real)
         return fail(SSM_ERR_ARG, "n_static (%d) must lie in [0, n_real = %d]", d->n_static, d->n_real);
+    if (d->discretization != SSM_DISC_EULER && d->discretization != SSM_DISC_ZOH)
+        return fail(SSM_ERR_ARG, "unknown discretization %d", d->discretization);
+    if (d->discretization == SSM_DISC_ZOH && (d->two_endpoint || d->n_static))
+        return fail(SSM_ERR_ARG, "the ZOH write needs two_endpoint == 0 and n_static == 0");
+    if (d->reserved_ != 0) return fail(SSM_ERR_ARG, "reserved descriptor field must be 0");
     if (d->batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch > 65535");
     if (d->seqlen > (1LL << 31) - 1 || d->nheads > (1 << 24) || d->headdim > (1 << 16))
         return fail(SSM_ERR_UNSUPPORTED, "sizes exceed the 32-bit index ranges of the kernels");
@@ -191,6 +196,7 @@ void fill_params(const ssm_desc_t *d, ssm::Params &p) {
     p.bf16 = d->dtype_io == SSM_BF16;
     p.angle_tok = d->angle_mode == SSM_ANGLE_PER_TOKEN && d->n_pairs > 0;
     p.nst = d->n_static;
+    p.zoh = d->discretization == SSM_DISC_ZOH;
     p.wait_limit = g_wait_limit.load();
     for (int k = 0; k < 3; ++k) {
         p.sx[k] = d->stride_x[k];
@@ -214,7 +220,7 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
     const bool static_angles = d->angle_mode == SSM_ANGLE_STATIC || d->n_pairs == 0;
     return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0 &&
-           static_angles && d->n_static == 0;
+           static_angles && d->n_static == 0 && d->discretization == SSM_DISC_EULER;
 }
 
 // Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and
@@ -224,7 +230,7 @@ bool ssd_shape(const ssm_desc_t *d) {
     return d->dtype_io == SSM_BF16 && d->decay_mode == SSM_DECAY_PER_HEAD && d->n_pairs == 0 &&
            d->headdim == 64 && (N == 64 || N == 128) && d->rank_in == d->rank_out &&
            (d->rank_in == 1 || d->rank_in == 2 || d->rank_in == 4) && d->chunk != 1 &&
-           d->seqlen > 0 && d->n_static == 0;
+           d->seqlen > 0 && d->n_static == 0 && d->discretization == SSM_DISC_EULER;
 }
 
 // Shapes of the channel scan (Mamba-1: head dim 1, 8 or 16 real state rows,
@@ -233,7 +239,8 @@ bool m1_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
     return d->dtype_io == SSM_BF16 && d->headdim == 1 && d->rank_in == 1 && d->rank_out == 1 &&
            d->n_pairs == 0 && (N == 8 || N == 16) && (d->nheads / d->ngroups) % 64 == 0 &&
-           d->chunk != 1 && d->seqlen > 0 && d->n_static == 0;
+           d->chunk != 1 && d->seqlen > 0 && d->n_static == 0 &&
+           d->discretization == SSM_DISC_EULER;
 }
 
 // Forward workspace of the tensor-core chain.  Every forward carries the fp32

@@ -19,6 +19,7 @@ struct Params {
     int two_ep, per_coord, bf16;
     int angle_tok;  // rotation angles given per token: theta / dtheta are [B][L][H][np]
     int nst;        // the first nst real rows are static (transition e^{a} whatever dt)
+    int zoh;        // exact zero-order-hold write (two_endpoint == 0, nst == 0)
     // element strides (batch, time, head-or-group)
     long long sx[3], sy[3], sB[3], sC[3], sdt[3], slam[3];
     // inputs
@@ -178,6 +179,52 @@ __device__ __forceinline__ void xreduce(float (&v)[K], int lane) {
             }
         }
     }
+}
+
+// ---- exact zero-order hold --------------------------------------------------
+// phi1(mu) = (e^mu - 1) / mu and phi1'(mu) = (e^mu (mu - 1) + 1) / mu^2 of a
+// complex mu = (mr, mi), by their Taylor series for |mu| < 1/2 (where the
+// closed forms cancel) and the closed forms above it.
+__device__ __forceinline__ void cmulf(float ar, float ai, float br, float bi, float &cr, float &ci) {
+    cr = ar * br - ai * bi;
+    ci = ar * bi + ai * br;
+}
+__device__ __forceinline__ void zoh_phi(float mr, float mi, float &f1r, float &f1i, float &fdr,
+                                        float &fdi) {
+    if (mr * mr + mi * mi < 0.25f) {
+        // sum_k mu^k / (k + 1)!  and  sum_k (k + 1) mu^k / (k + 2)!, 12 terms
+        float pr = 1.f, pi = 0.f;   // mu^k
+        f1r = f1i = fdr = fdi = 0.f;
+        float inv1 = 1.f, inv2 = 0.5f;   // 1 / (k + 1)!, 1 / (k + 2)!
+#pragma unroll
+        for (int k = 0; k < 12; ++k) {
+            f1r = fmaf(inv1, pr, f1r);
+            f1i = fmaf(inv1, pi, f1i);
+            fdr = fmaf((k + 1) * inv2, pr, fdr);
+            fdi = fmaf((k + 1) * inv2, pi, fdi);
+            float nr, ni;
+            cmulf(pr, pi, mr, mi, nr, ni);
+            pr = nr;
+            pi = ni;
+            inv1 *= 1.f / (float)(k + 2);
+            inv2 *= 1.f / (float)(k + 3);
+        }
+        return;
+    }
+    float sn, cs;
+    sincosf(mi, &sn, &cs);
+    const float ex = expf(mr);
+    const float s2 = sinf(0.5f * mi);
+    // e^mu - 1 without cancellation in its real part
+    const float er = fmaf(expm1f(mr), cs, -2.f * s2 * s2), ei = ex * sn;
+    const float d = 1.f / (mr * mr + mi * mi);   // 1 / |mu|^2
+    // (e^mu - 1) conj(mu) / |mu|^2
+    f1r = (er * mr + ei * mi) * d;
+    f1i = (ei * mr - er * mi) * d;
+    // phi1'(mu) = (e^mu - phi1(mu)) / mu
+    const float nr = ex * cs - f1r, ni = ex * sn - f1i;
+    fdr = (nr * mr + ni * mi) * d;
+    fdi = (ni * mr - nr * mi) * d;
 }
 
 // Timing hook (defined in abi.cu): call right after every kernel launch with

@@ -935,7 +935,7 @@ bool chunk_fwd_supported(const Params &p) {
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
     // y (forward) leaves by TMA stores
     const bool yok = !p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]));
-    return yok && !p.angle_tok && !p.nst && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
+    return yok && !p.angle_tok && !p.nst && !p.zoh && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
            (p.N == 64 || p.N == 128) &&
            p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
            st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) && st16(p.sB[2]) &&

@@ -42,6 +42,7 @@ struct Smem {
     float *corr;              // [HC][T][O][R]   -beta_{t+1} (C_t B_t)[o][r]   (or M for bwd)
     float *red;               // reduction buffer (kernel specific)
     float *misc;              // [HC][T][4]
+    float *zc;                // [HC][T][NSL]  ZOH write coefficient per slot (re, im per pair)
     int *slot;                // [N] slot of each state row
 };
 
@@ -93,6 +94,7 @@ __host__ __device__ inline size_t carve(Smem &s, float *base, const Params &p, i
     s.dy = with_dy ? take((size_t)g.HC * g.T * p.O * g.PP) : nullptr;
     s.corr = take((size_t)g.HC * g.T * p.O * p.R);
     s.misc = take((size_t)g.HC * g.T * 4);
+    s.zc = take(p.zoh ? (size_t)g.HC * g.T * NSL : 0);
     s.slot = reinterpret_cast<int *>(take((size_t)p.N));
     s.red = base ? base + off : nullptr;
     return off;
@@ -175,7 +177,7 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
         float dv = s.dt[hc * (T + 1) + tt], lv = s.lam[hc * (T + 1) + tt];
         float bnext = 0.f;
         if (t + 1 < p.L) bnext = (1.f - s.lam[hc * (T + 1) + tt + 1]) * s.dt[hc * (T + 1) + tt + 1];
-        s.sig[i] = lv * dv + bnext;
+        s.sig[i] = p.zoh ? 1.f : lv * dv + bnext;   // the ZOH write is scaled per mode
         s.bn[i] = bnext;
     }
     const int nmode = p.nr + p.np;
@@ -189,6 +191,25 @@ __device__ void stage_block(const Params &p, Smem &s, int b, int hbase, int gbas
                 float *cf = s.coef + (hc * T + tt) * NSL;
                 for (int m = l.tx; m < nmode; m += l.W) {
                     const float a = s.a[hc * p.ndec + (p.per_coord ? m : 0)];
+                    if (p.zoh) {
+                        // Z = dt phi1(dt a + i phi): the exact write of a held input
+                        float phi = 0.f;
+                        if (m >= p.nr) {
+                            const int j = m - p.nr;
+                            phi = p.angle_tok ? (tok_ok ? p.theta[ix_th(p, b, t0 + tt, h, j)] : 0.f)
+                                              : dv * s.w[hc * (p.np > 0 ? p.np : 1) + j];
+                        }
+                        float f1r, f1i, fdr, fdi;
+                        zoh_phi(dv * a, phi, f1r, f1i, fdr, fdi);
+                        float *zz = s.zc + (hc * T + tt) * NSL;
+                        if (m < p.nr) {
+                            zz[s.slot[m]] = dv * f1r;
+                        } else {
+                            const int sl = s.slot[p.nr + 2 * (m - p.nr)];
+                            zz[sl] = dv * f1r;
+                            zz[sl + 1] = dv * f1i;
+                        }
+                    }
                     if (m < p.nr) {
                         cf[s.slot[m]] = expf(m < p.nst ? a : dv * a);   // static rows: e^{a}
                     } else {
@@ -234,6 +255,8 @@ __device__ void init_rates(const Params &p, Smem &s, int hbase, int NSL, int NGL
     for (int n = threadIdx.x; n < p.N; n += blockDim.x) s.slot[n] = slot_of<NR, NPR>(n, p.nr, g.NQ);
     // padding slots must read as zero for the whole kernel
     for (int i = threadIdx.x; i < g.HC * g.T * NSL; i += blockDim.x) s.coef[i] = 0.f;
+    if (p.zoh)
+        for (int i = threadIdx.x; i < g.HC * g.T * NSL; i += blockDim.x) s.zc[i] = 0.f;
     for (int i = threadIdx.x; i < NGL * g.T * p.R * NSL; i += blockDim.x) s.Bp[i] = 0.f;
     for (int i = threadIdx.x; i < NGL * g.T * p.O * NSL; i += blockDim.x) s.Cp[i] = 0.f;
     __syncthreads();
@@ -251,6 +274,31 @@ __device__ __forceinline__ void step_fwd(float (&K)[NR + 2 * NPR], const float *
         const float kr = K[NR + 2 * j], ki = K[NR + 2 * j + 1];
         K[NR + 2 * j] = fmaf(ec, kr, fmaf(-es, ki, w[NR + 2 * j]));
         K[NR + 2 * j + 1] = fmaf(es, kr, fmaf(ec, ki, w[NR + 2 * j + 1]));
+    }
+}
+// w <- Z (.) w (ZOH write; complex product on a pair) and its transpose
+template <int NR, int NPR>
+__device__ __forceinline__ void zoh_apply(float (&w)[NR + 2 * NPR], const float *zz) {
+#pragma unroll
+    for (int i = 0; i < NR; ++i) w[i] *= zz[i];
+#pragma unroll
+    for (int j = 0; j < NPR; ++j) {
+        const float zr = zz[NR + 2 * j], zi = zz[NR + 2 * j + 1];
+        const float wr = w[NR + 2 * j], wi = w[NR + 2 * j + 1];
+        w[NR + 2 * j] = fmaf(zr, wr, -zi * wi);
+        w[NR + 2 * j + 1] = fmaf(zi, wr, zr * wi);
+    }
+}
+template <int NR, int NPR>
+__device__ __forceinline__ void zoh_apply_T(float (&g)[NR + 2 * NPR], const float *zz) {
+#pragma unroll
+    for (int i = 0; i < NR; ++i) g[i] *= zz[i];
+#pragma unroll
+    for (int j = 0; j < NPR; ++j) {
+        const float zr = zz[NR + 2 * j], zi = zz[NR + 2 * j + 1];
+        const float gr = g[NR + 2 * j], gi = g[NR + 2 * j + 1];
+        g[NR + 2 * j] = fmaf(zr, gr, zi * gi);
+        g[NR + 2 * j + 1] = fmaf(-zi, gr, zr * gi);
     }
 }
 // G <- A_t^T G
@@ -365,8 +413,14 @@ __global__ void __launch_bounds__(MAXT) k_fwd(Params p) {
 #pragma unroll
                 for (int sl = 0; sl < NS; ++sl) Wlast[sl] = w[sl];
             }
+            if (p.zoh) {
+                float zz[NS];
+                ld_slots<NS>(zz, s.zc + (ln.hc * T + tt) * NSL + ln.q * NS);
+                zoh_apply<NR, NPR>(w, zz);
+            } else {
 #pragma unroll
-            for (int sl = 0; sl < NS; ++sl) w[sl] *= sig;
+                for (int sl = 0; sl < NS; ++sl) w[sl] *= sig;
+            }
             float cf[NS];
             ld_slots<NS>(cf, s.coef + (ln.hc * T + tt) * NSL + ln.q * NS);
             step_fwd<NR, NPR>(K, cf, w);
@@ -489,6 +543,11 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep1(Params p) {
             float ws[NS];
 #pragma unroll
             for (int sl = 0; sl < NS; ++sl) ws[sl] = w[sl] * sig;
+            if (p.zoh) {
+                float zz[NS];
+                ld_slots<NS>(zz, s.zc + (ln.hc * T + tt) * NSL + ln.q * NS);
+                zoh_apply<NR, NPR>(ws, zz);
+            }
             step_fwd<NR, NPR>(K, cf, ws);
             // H_t = K_t - beta_{t+1} W_t ; values dy[o,p] * H[n,p]
             float v[KV];
@@ -567,7 +626,15 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
                     for (int sl = 0; sl < NS; ++sl) Gv[sl] = fmaf(cc[sl], dyo, Gv[sl]);
                 }
             }
-            // sum_p G[n,p] u[r,p]  and  sum_n B[n,r] G[n,p]
+            // sum_p G[n,p] u[r,p]  and  sum_n B[n,r] G[n,p] (ZOH: B^T Z^T G)
+            float gw[NS];
+#pragma unroll
+            for (int sl = 0; sl < NS; ++sl) gw[sl] = Gv[sl];
+            if (p.zoh) {
+                float zz[NS];
+                ld_slots<NS>(zz, s.zc + (ln.hc * T + tt) * NSL + ln.q * NS);
+                zoh_apply_T<NR, NPR>(gw, zz);
+            }
             float v[KV];
 #pragma unroll
             for (int r = 0; r < RM; ++r) {
@@ -578,7 +645,7 @@ __global__ void __launch_bounds__(MAXT) k_bwd_sweep2(Params p) {
 #pragma unroll
                 for (int sl = 0; sl < NS; ++sl) {
                     v[r * NS + sl] = Gv[sl] * ur;
-                    du = fmaf(bb[sl], Gv[sl], du);
+                    du = fmaf(bb[sl], gw[sl], du);
                 }
                 if (r < p.R) redB[(((ln.hc * T + tt) * RM + r) * NQ + ln.q) * PP + ln.pl] = du;
             }
@@ -774,21 +841,56 @@ __device__ __forceinline__ void units_local_item(const Params &p, float *smem, i
                 for (int r = 0; r < p.R; ++r) {
                     const float b0 = ld_io(p.Bm, ix_B(p, b, t, g, r, n0), p.bf16);
                     const float b1 = pair ? ld_io(p.Bm, ix_B(p, b, t, g, r, n0 + 1), p.bf16) : 0.f;
-                    const float g0 = sig * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0)];
-                    const float g1 = pair ? sig * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0 + 1)] : 0.f;
+                    const float g0 = p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0)];
+                    const float g1 = pair ? p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0 + 1)] : 0.f;
                     yr += b0 * g0 + b1 * g1;   // b * conj(g)
                     yi += b1 * g0 - b0 * g1;
+                }
+                float zoh_dt = 0.f, zoh_dw = 0.f;
+                if (p.zoh) {
+                    // the write of step t is Z b u: Y = Z b conj(g); the gradient of Z,
+                    // (yr, -yi), reaches dt, a and the angle through dZ/d.
+                    float phi = 0.f;
+                    if (pair)
+                        phi = p.angle_tok ? p.theta[ix_th(p, b, t, h, m - p.nr)]
+                                          : dv * p.theta[h * p.np + (m - p.nr)];
+                    float f1r, f1i, fdr, fdi;
+                    zoh_phi(dv * mi.a, phi, f1r, f1i, fdr, fdi);
+                    const float gzr = yr, gzi = -yi;
+                    float zdr, zdi;   // dZ / d dt
+                    if (pair && p.angle_tok) {
+                        zdr = fmaf(dv * mi.a, fdr, f1r);
+                        zdi = fmaf(dv * mi.a, fdi, f1i);
+                    } else {
+                        float sn, cs;
+                        sincosf(phi, &sn, &cs);
+                        const float ex = expf(dv * mi.a);
+                        zdr = ex * cs;
+                        zdi = ex * sn;
+                    }
+                    zoh_dt = fmaf(gzr, zdr, gzi * zdi);
+                    // dZ / da = dt^2 phi1'; dZ / dangle = i dt phi1' (per token) or i dt^2 phi1'
+                    dA = fmaf(dv * dv, fmaf(gzr, fdr, gzi * fdi), dA);
+                    const float wsc = (pair && p.angle_tok) ? dv : dv * dv;
+                    zoh_dw = wsc * fmaf(-gzr, fdi, gzi * fdr);
+                    float nr_, ni_;
+                    cmulf(dv * f1r, dv * f1i, yr, yi, nr_, ni_);
+                    yr = nr_;
+                    yi = ni_;
+                } else {
+                    yr *= sig;
+                    yi *= sig;
                 }
                 cr += xr - yr;
                 ci += xi - yi;
                 // a static row's log-transition is a itself: weight 1, nothing to ddt
                 const bool stat = m < p.nst;
                 dA = fmaf(stat ? 1.f : dv, cr, dA);
-                if (pair) dth = fmaf(dv, -ci, dth);
+                if (pair) dth = fmaf(dv, -ci, dth) + zoh_dw;
                 // per-token angle: the local part of dL/dphi_t (the carry from
                 // later time blocks is added by k_bwd_units_carry)
-                if (pair && p.angle_tok) p.dtheta[ix_th(p, b, t, h, m - p.nr)] = -ci;
-                contrib = stat ? 0.f : mi.a * cr + (pair ? -mi.w * ci : 0.f);
+                if (pair && p.angle_tok) p.dtheta[ix_th(p, b, t, h, m - p.nr)] = zoh_dw - ci;
+                contrib = stat ? 0.f : mi.a * cr + (pair ? -mi.w * ci : 0.f) + zoh_dt;
             }
             if (m == 0) {
                 sdt += dv;
@@ -924,11 +1026,31 @@ __global__ void k_bwd_units_final(Params p) {
                 dbeta = p.ws_par[((long long)b * p.H + h) * npar_of(p) + p.ndec + p.np + 1];
             dd += lv * ds + (1.f - lv) * dbeta;
             if (p.dlam) st_io(p.dlam, ix_lam(p, b, t, h), dv * (ds - dbeta), p.bf16);
-        } else {
+        } else if (!p.zoh) {   // the ZOH write's dt-dependence is in ws_ddt already
             dd += ds;
         }
         st_io(p.ddt, ix_dt(p, b, t, h), dd, p.bf16);
     }
+}
+
+// (Z^T gbu)[n] of head h at step t under the ZOH write: gbu scaled by the
+// mode's Z (transposed complex product on a pair)
+__device__ __forceinline__ float zoh_gbu(const Params &p, int b, int t, int h, int r, int n) {
+    const float dv = ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+    const bool pair = n >= p.nr;
+    const int m = pair ? p.nr + (n - p.nr) / 2 : n;
+    const float a = neg_exp(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
+    float phi = 0.f;
+    if (pair)
+        phi = p.angle_tok ? p.theta[ix_th(p, b, t, h, m - p.nr)] : dv * p.theta[h * p.np + (m - p.nr)];
+    float f1r, f1i, fdr, fdi;
+    zoh_phi(dv * a, phi, f1r, f1i, fdr, fdi);
+    const float zr = dv * f1r, zi = dv * f1i;
+    if (!pair) return zr * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n)];
+    const int n0 = p.nr + 2 * (m - p.nr);
+    const float gr = p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0)];
+    const float gi = p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n0 + 1)];
+    return n == n0 ? fmaf(zr, gr, zi * gi) : fmaf(-zi, gr, zr * gi);
 }
 
 // dB, dC per (b, t): sum over the heads of each group; per-head scalars first
@@ -953,7 +1075,12 @@ __device__ __forceinline__ void groups_item(const Params &p, float *smem, int t,
             if (k < p.R) {
                 const int r = k;
                 for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h) {
-                    float v = s_sig[h] * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n)];
+                    float v;
+                    if (p.zoh) {
+                        v = zoh_gbu(p, b, t, h, r, n);
+                    } else {
+                        v = s_sig[h] * p.ws_gbu[ix_wsk(p, b, t, h, r, p.R, n)];
+                    }
                     const float bnx = s_bn[h];
                     if (bnx != 0.f) {
                         const float *M2 = p.ws_M2 + ix_bth(p, b, t, h) * p.O * p.R;

@@ -292,6 +292,14 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
             alog = __ldg(p.A_log + nx.h * p.ndec);
+            if (tid == 0) {   // the next item's tiles stream into L2 while this one runs
+                const int g2 = nx.h / p.hpg;
+                tma_prefetch_5d(&tmX, 0, 0, nx.h, nx.c * Qt, nx.b);
+                for (int kb = 0; kb < nbox; ++kb) {
+                    tma_prefetch_5d(&tmB, 64 * kb, 0, g2, nx.c * Qt, nx.b);
+                    if (want_y) tma_prefetch_5d(&tmC, 64 * kb, 0, g2, nx.c * Qt, nx.b);
+                }
+            }
         }
         {
             const bool okx = mbar_wait(bar_x, par, WAIT_LIMIT);
@@ -745,6 +753,16 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = ssdk::tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
             alog = __ldg(p.A_log + nx.h * p.ndec);
+            if (tid == 0) {   // the next item's tiles stream into L2 while this one runs
+                const int g2 = nx.h / p.hpg;
+                tma_prefetch_5d(&tmX, 0, 0, nx.h, nx.c * Qt, nx.b);
+                tma_prefetch_5d(&tmDY, 0, 0, nx.h, nx.c * Qt, nx.b);
+                for (int kb = 0; kb < nbox; ++kb) {
+                    tma_prefetch_5d(&tmB, 64 * kb, 0, g2, nx.c * Qt, nx.b);
+                    tma_prefetch_5d(&tmC, 64 * kb, 0, g2, nx.c * Qt, nx.b);
+                }
+                bulk_prefetch_l2(p.ws_kp + bhc(p, nx.b, nx.h, nx.c) * SLOT_FLOATS, 2 * TILE);
+            }
         }
         const float a2 = f32[F_SC], E = f32[F_SC + 2];
         {

@@ -55,7 +55,13 @@ __global__ void __launch_bounds__(stepk::THREADS) k_scan_step(Params p, float *h
             const long long i0 = ix_st(p, b, h, n, q);
             const float wn = write_of(n);
             const float wp = (p.two_ep && ws) ? ws[i0] : 0.f;
-            const float hn = fmaf(e, fmaf(beta, wp, hs[i0]), gam * wn);
+            float wsc = gam;   // the write's scale: dt (Euler) or (e^{dt a} - 1) / a (ZOH)
+            if (p.zoh) {
+                float f1r, f1i, fdr, fdi;
+                zoh_phi(dt * a, 0.f, f1r, f1i, fdr, fdi);
+                wsc = dt * f1r;
+            }
+            const float hn = fmaf(e, fmaf(beta, wp, hs[i0]), wsc * wn);
             hs[i0] = hn;
             if (ws) ws[i0] = wn;
             readout(n, hn);
@@ -77,9 +83,18 @@ __global__ void __launch_bounds__(stepk::THREADS) k_scan_step(Params p, float *h
                 zr = fmaf(beta, ws[i0], zr);
                 zi = fmaf(beta, ws[i1], zi);
             }
-            // (er + i ei)(zr + i zi) + gamma W
-            const float hr = fmaf(er, zr, fmaf(-ei, zi, gam * wr));
-            const float hi = fmaf(er, zi, fmaf(ei, zr, gam * wi));
+            // (er + i ei)(zr + i zi) + gamma W  (ZOH: + Z W, complex)
+            float ur = gam * wr, ui = gam * wi;
+            if (p.zoh) {
+                float f1r, f1i, fdr, fdi;
+                const float phi = p.angle_tok ? p.theta[((long long)b * p.H + h) * p.np + j]
+                                              : dt * p.theta[h * p.np + j];
+                zoh_phi(dt * a, phi, f1r, f1i, fdr, fdi);
+                ur = dt * (f1r * wr - f1i * wi);
+                ui = dt * (f1i * wr + f1r * wi);
+            }
+            const float hr = fmaf(er, zr, fmaf(-ei, zi, ur));
+            const float hi = fmaf(er, zi, fmaf(ei, zr, ui));
             hs[i0] = hr;
             hs[i1] = hi;
             if (ws) {

@@ -43,8 +43,9 @@ def test_abi_version(lib):
 
 def test_desc_layout_matches_header(lib):
     """ssm_desc_t: five int64 sizes, eight int32 fields, six int64[3] stride
-    arrays, angle_mode and n_static: 200 bytes, no padding."""
-    assert ctypes.sizeof(abi.Desc) == 5 * 8 + 8 * 4 + 6 * 3 * 8 + 2 * 4
+    arrays, angle_mode, n_static, discretization and a reserved word: 208
+    bytes, no padding."""
+    assert ctypes.sizeof(abi.Desc) == 5 * 8 + 8 * 4 + 6 * 3 * 8 + 4 * 4
     assert abi.Desc.angle_mode.offset == 5 * 8 + 8 * 4 + 6 * 3 * 8
 
 
@@ -59,6 +60,18 @@ def test_angle_mode_validation(lib):
         d.n_static = bad
         assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
         assert b"n_static" in lib.ssm_scan_last_error()
+    d.n_static = 0
+    d.discretization = 2
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+    assert b"discretization" in lib.ssm_scan_last_error()
+    d.discretization = S.DISC_ZOH          # ZOH needs the Euler form (two_endpoint == 0)
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
+    assert b"ZOH" in lib.ssm_scan_last_error()
+    d.two_endpoint = 0
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0   # recurrent kernels: no workspace
+    d.discretization = 0
+    d.reserved_ = 1
+    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
     # static rows run on the recurrent kernels too
     st = abi.make_desc(sh.replace(n_static=16))
     assert st.n_static == 16

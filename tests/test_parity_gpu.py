@@ -29,7 +29,7 @@ def chunk_eligible(shape):
             and shape.rank_out == 1 and shape.nstate in (64, 128) and shape.n_real % 8 == 0
             and shape.seqlen > 0 and shape.chunk != 1
             and not (shape.angle_mode == S.ANGLE_PER_TOKEN and shape.n_pairs)
-            and shape.n_static == 0)
+            and shape.n_static == 0 and shape.discretization == S.DISC_EULER)
 
 
 def ssd_eligible(shape):
@@ -200,6 +200,23 @@ def test_static_rows(kw):
     base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=150)
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=93, with_state=True)
+    check_all(shape, inp, route=abi.ROUTE_RECURRENT)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),                                   # HybridMamba heads, Euler form, bf16
+    dict(dtype_io=S.DTYPE_F32),
+    dict(angle_mode=S.ANGLE_PER_TOKEN),
+    dict(decay_mode=S.DECAY_PER_HEAD, n_real=128, n_pairs=0, ngroups=2),
+    dict(rank_in=2, rank_out=2, n_real=16, n_pairs=8, seqlen=70),
+])
+def test_zoh_write(kw):
+    """Exact zero-order-hold write ((e^{dt lam} - 1) / lam per mode, complex on a
+    rotation pair) against the oracle, forward and backward."""
+    base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=150,
+                                              two_endpoint=0, discretization=S.DISC_ZOH)
+    shape = base.replace(**kw)
+    inp = S.make_inputs(shape, seed=95, with_state=True)
     check_all(shape, inp, route=abi.ROUTE_RECURRENT)
 
 

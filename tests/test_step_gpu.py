@@ -84,6 +84,18 @@ def test_steps_with_static_rows():
     compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(angle_mode=S.ANGLE_PER_TOKEN)])
+def test_steps_with_zoh_write(kw):
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=7,
+                                               two_endpoint=0, discretization=S.DISC_ZOH, **kw)
+    inp = S.make_inputs(shape, seed=16, with_dy=False, with_state=True)
+    y, h, w = step_through(shape, inp)
+    ref = oracle.scan_fwd(shape, inp)
+    compare("y", to_np(y), ref["y"], shape.dtype_io)
+    compare("hT", to_np(h), ref["hT"], shape.dtype_io)
+    compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
+
+
 def test_euler_write_needs_no_w():
     shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=6, two_endpoint=0)
     inp = S.make_inputs(shape, seed=12, with_dy=False, with_state=True)
