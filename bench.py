@@ -143,26 +143,51 @@ def kernel_bytes(shape, name: str) -> int:
 # keyed by the kernel's source file and the first 16 hex digits of its SHA-256
 # at capture time: an entry whose source has changed since is not reported
 # (traffic null) instead of going stale.
-NCU_TRAFFIC_PER_ROW = {}
+NCU_TRAFFIC_PER_ROW = {
+    # (workload, kernel): (dram read + write bytes per batch row of one launch, source hash)
+    # ncu --set full captures at batch 2 (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the
+    # full Mamba-2 size; the traffic of these kernels grows with the batch rows
+    ("hybridmamba", "k_chunk_fwd"): (421.24e6, "bc477f309b223f3c"),
+    ("hybridmamba", "k_chunk_bwd_fused"): (605.52e6, "6b57e6460b9284ec"),
+    ("ssd_mimo_r4", "k_ssd_fwd"): (1039.22e6, "3823fac94aef91bf"),
+    ("ssd_mimo_r4", "k_ssd_bwd"): (1740.24e6, "3823fac94aef91bf"),
+    ("mamba2_siso", "k_ssd_fwd"): (18.34e6, "3823fac94aef91bf"),
+    ("mamba2_siso", "k_ssd_bwd"): (76.70e6, "3823fac94aef91bf"),
+    ("mamba1_siso", "k_m1_fwd"): (60.60e6, "f3b528160f538458"),
+    ("mamba1_siso", "k_m1_bwd"): (119.65e6, "f3b528160f538458"),
+}
+
+# sources each kernel is compiled from: a traffic entry holds only while they
+# are byte-identical to the build the counters were taken on
+KERNEL_SOURCES = {
+    "k_chunk_fwd": ("scan_chunk.cu", "chunk_common.cuh", "umma.cuh", "common.cuh"),
+    "k_chunk_bwd_fused": ("scan_chunk_rev.cu", "chunk_common.cuh", "umma.cuh", "common.cuh"),
+    "k_ssd_fwd": ("scan_ssd.cu", "chunk_common.cuh", "umma.cuh", "common.cuh"),
+    "k_ssd_bwd": ("scan_ssd.cu", "chunk_common.cuh", "umma.cuh", "common.cuh"),
+    "k_m1_fwd": ("scan_m1.cu", "common.cuh"),
+    "k_m1_bwd": ("scan_m1.cu", "common.cuh"),
+}
 
 
-def _source_sha16(rel):
+def source_sha16(kernel):
     import hashlib
-    path = os.path.join(ROOT, "selective_diagonal_state_b200", "csrc", rel)
-    try:
-        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
-    except OSError:
-        return None
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES.get(kernel, ()):
+        try:
+            h.update(open(os.path.join(ROOT, "selective_diagonal_state_b200", "csrc", rel), "rb").read())
+        except OSError:
+            return None
+    return h.hexdigest()[:16] if kernel in KERNEL_SOURCES else None
 
 
 def ncu_traffic(shape, kernel):
     """Measured DRAM bytes of one launch of `kernel`, or None when there is no
-    capture of the kernel's current source."""
+    capture of the kernel's current sources."""
     ent = NCU_TRAFFIC_PER_ROW.get((shape.name, kernel))
     if ent is None:
         return None
-    per_row, src, sha = ent
-    if _source_sha16(src) != sha:
+    per_row, sha = ent
+    if source_sha16(kernel) != sha:
         return None
     return per_row * shape.batch
 

@@ -35,7 +35,7 @@ cudaError_t preact_backward(const Params &p, const PreactArgs &a, cudaStream_t s
 cudaError_t scan_step(const Params &p, float *h, float *w, cudaStream_t st);
 bool ssd_supported(const Params &p);
 int ssd_chunk_tokens(int R);
-size_t ssd_ring_bytes(long long B, long long H);
+size_t ssd_ring_bytes(long long B, long long H, long long L, int R);
 cudaError_t ssd_forward(const Params &p, cudaStream_t st);
 cudaError_t ssd_backward(const Params &p, cudaStream_t st);
 int ssd_error_take();
@@ -265,14 +265,15 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
         return w;
     }
     if (ssd_shape(d)) {
-        // scalar-decay chain: the two tagged carry slots and the counter of every (b, h),
-        // the ticket and abort words; a training forward also keeps the state entering
-        // every chunk of ssm::ssd_chunk_tokens tokens (bf16 hi + lo tiles, 32 KB)
+        // scalar-decay chain: the chain buffers (segment states and decays, a carry
+        // slot per CTA, the backward's adjoint slots), the counters of every (b, h), the
+        // ticket and abort words; a training forward also keeps the state entering every
+        // chunk of ssm::ssd_chunk_tokens tokens (bf16 hi + lo tiles, 32 KB)
         const size_t bh = (size_t)d->batch * d->nheads;
         const int qt = ssm::ssd_chunk_tokens(d->rank_in);
         const size_t units = bh * (size_t)((d->seqlen + qt - 1) / qt);
         const size_t slot = 128 * (size_t)d->headdim * 4;
-        size_t off = align256(ssm::ssd_ring_bytes(d->batch, d->nheads));   // tagged carry slots
+        size_t off = align256(ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, d->rank_in));
         w.off_flag = off;
         off = align256(off + (bh + 2) * 4);
         w.total_infer = off;
@@ -323,8 +324,8 @@ SsdBwdWs ssd_bwd_layout(const ssm_desc_t *d) {
     const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
     const size_t N = nstate(d);
     size_t off = 0;
-    w.off_ring = off;   // tagged carry slots
-    off = align256(off + ssm::ssd_ring_bytes(d->batch, d->nheads));
+    w.off_ring = off;   // carry slots and the forward's segment buffers
+    off = align256(off + ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, d->rank_in));
     w.off_flag = off;
     off = align256(off + (bh + 2) * 4);
     w.off_kp = off;

@@ -68,6 +68,11 @@ struct Params {
     float *sd_par;          // [B][H][NC][2] per chunk: sum_t dt_t drho_t, sum <dy, x>
     float *sd_db0;          // [B][H] dbeta_0 = <dL/dK_{-1}, w0>
     float *sd_dBh, *sd_dCh; // [B][L][H][R or O][N] fp32 per-head dB / dC (several heads per group)
+    // scalar-decay forward, segments of sd_G chunks: per (segment, b, h) the state the
+    // segment adds, then the state entering it ([nseg][B][H] 32 KB, in place), the
+    // segment's decay [nseg][B][H], and one 32 KB carry slot per CTA
+    float *sd_seg, *sd_sege, *sd_priv;
+    int sd_G, sd_nseg;
     Geometry geo;
 };
 

@@ -142,39 +142,6 @@ __device__ __forceinline__ void chunk_scalars(const Params &p, float *f32, int t
     __syncthreads();
 }
 
-// K_in of thread (state row n, 16 columns from 16 cq): the carry slot, or
-// h0 + beta_0 w0 for the first chunk.
-__device__ __forceinline__ void load_kin(const Params &p, int c, int b, int h, int n, int cq,
-                                         float (&kc)[16]) {
-    if (n >= p.N) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) kc[j] = 0.f;
-        return;
-    }
-    if (c > 0) {
-        const float4 *src = carry_ptr(p, c & 1, b * p.H + h, cq, n);
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-            const float4 v = __ldcg(src + j4 * NP);
-            kc[4 * j4] = v.x;
-            kc[4 * j4 + 1] = v.y;
-            kc[4 * j4 + 2] = v.z;
-            kc[4 * j4 + 3] = v.w;
-        }
-        return;
-    }
-    float beta0 = 0.f;
-    if (p.two_ep)
-        beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const long long i0 = ix_st(p, b, h, n, 16 * cq + j);
-        float a = p.h0 ? p.h0[i0] : 0.f;
-        if (p.w0) a = fmaf(beta0, p.w0[i0], a);
-        kc[j] = a;
-    }
-}
-
 // 8 bf16 of row `row`, logical 16-byte chunk `lc` of a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t sw_off(int row, int lc) {
     return (uint32_t)row * 128u + ((uint32_t)(lc ^ (row & 7)) << 4);
@@ -196,13 +163,218 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
     return w;
 }
 
+// ---- segments -----------------------------------------------------------------
+// The forward advances the state of a (b, h) a segment of G chunks at a time.  With
+// one decay per head the state a segment adds is one contraction over all its rows,
+//     S_seg = B_seg^T diag(e^{a (S_end - S_t)} sigma_t) X_seg,   E_seg = e^{a S_end}
+// (S the sum of dt inside the segment), the chunk state over a longer span: the
+// states entering the segments then come from a short elementwise pass over the
+// segments, and the forward's work items - whole segments, walked chunk by chunk
+// with the carry kept by the CTA - wait on no other item.
+// Slots as the carry: [segment][b * H + h][cq][j4][n][4] fp32.
+__device__ __forceinline__ float4 *seg_ptr(const Params &p, int s, int bh, int cq, int n) {
+    return reinterpret_cast<float4 *>(p.sd_seg) +
+           (((long long)(s * p.Bsz * p.H + bh) * 4 + cq) * 4) * NP + n;
+}
+__device__ __forceinline__ float4 *priv_ptr(const Params &p, int cta, int cq, int n) {
+    return reinterpret_cast<float4 *>(p.sd_priv) + (((long long)cta * 4 + cq) * 4) * NP + n;
+}
+__device__ __forceinline__ void ld_slot16(const float4 *src, float (&v)[16]) {
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+        const float4 w = __ldcg(src + j4 * NP);
+        v[4 * j4] = w.x;
+        v[4 * j4 + 1] = w.y;
+        v[4 * j4 + 2] = w.z;
+        v[4 * j4 + 3] = w.w;
+    }
+}
+__device__ __forceinline__ void st_slot16(float4 *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4)
+        __stcg(dst + j4 * NP, make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]));
+}
+
+// S_seg and E_seg of every (segment, b, h): the segment's chunks last to first, the
+// contraction accumulated in TMEM, each chunk's f_t scaled by the decay of the chunks
+// after it.  Work items are independent (no chain).
+__global__ void __launch_bounds__(THREADS, 2)
+k_ssd_seg_state(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                Params p, int lgR) {
+    const int BH = p.Bsz * p.H, G = p.sd_G;
+    const int nitems = p.sd_nseg * BH;
+    if ((int)blockIdx.x >= nitems) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *f32 = reinterpret_cast<float *>(sm + SM_F32);
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + SM_BAR);   // x and B of a chunk
+    uint64_t *bar_mma = bar_in + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int N = p.N, nbox = N / 64, Qt = ROWS >> lgR;
+    const int qd = warp & 3, cb2 = warp >> 2, row = 32 * qd + lane;
+    PhaseCount pc_in = {0u, 0u}, pc_m = {0u, 0u};   // issued: thread 0; done: every thread
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 0) tmem_alloc(tslot, 64);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t t_s = *tslot, lane_q = (32u * qd) << 16;
+    bool aborted = false;
+    for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
+        const int sg = item / BH, bh = item - sg * BH, b = bh / p.H, h = bh - b * p.H;
+        const int c0 = sg * G, glen = min(G, p.nc - c0);
+        const float alog = __ldg(p.A_log + h * p.ndec);
+        float P = 1.f;   // decay of the segment's chunks after the current one
+        for (int jj = glen - 1; jj >= 0; --jj) {
+            const int c = c0 + jj, t0 = c * Qt;
+            if (tid == 0) {
+                mbar_expect_tx(bar_in, TILE * (1 + nbox));
+                tma_load_5d(sm + SM_X, &tmX, bar_in, 0, 0, h, t0, b);
+                for (int k = 0; k < nbox; ++k)
+                    tma_load_5d(sm + SM_B + k * TILE, &tmB, bar_in, 64 * k, 0, h / p.hpg, t0, b);
+                ++pc_in.issued;
+            }
+            const Tok tok = tok_load_q(p, b, h, t0, Qt);
+            chunk_scalars(p, f32, t0, Qt, tok, alog);
+            int ok = mbar_wait(bar_in, pc_in.done & 1u, WAIT_LIMIT) ? 1 : 0;
+            pc_in.done += (uint32_t)ok;
+            if (!ok) ssd_raise_error(1);
+            if (!__syncthreads_and(ok)) {
+                aborted = true;
+                break;
+            }
+            // X' = diag(f P) X
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int ch = tid + THREADS * q;
+                const int r = ch >> 3;
+                const uint32_t off = (uint32_t)r * 128u + (uint32_t)(ch & 7) * 16u;
+                const float f = f32[F_FW + (r >> lgR)] * P;
+                float v[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + SM_X + off), v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] *= f;
+                *reinterpret_cast<uint4 *>(sm + SM_XS + off) = pack8(v);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t b_base = smem_u32(sm + SM_B), xs_base = smem_u32(sm + SM_XS);
+                const uint32_t id = idesc_bf16(128, 64, true, true);
+                for (int s2 = 0; s2 < ROWS / 16; ++s2)
+                    mma_bf16(t_s, sdesc(b_base + s2 * 2048u, TILE, 1024u, LAYOUT_SW128),
+                             sdesc(xs_base + s2 * 2048u, TILE, 1024u, LAYOUT_SW128), id,
+                             s2 > 0 || jj < glen - 1);
+                mma_commit(bar_mma);
+                ++pc_m.issued;
+            }
+            ok = mbar_wait(bar_mma, pc_m.done & 1u, WAIT_LIMIT) ? 1 : 0;
+            pc_m.done += (uint32_t)ok;
+            if (!ok) ssd_raise_error(1);
+            fence_after_sync();
+            P *= f32[F_SC + 2];
+            if (!__syncthreads_and(ok)) {   // also: every thread has read this chunk's scalars
+                aborted = true;
+                break;
+            }
+        }
+        if (aborted) break;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int cq = 2 * cb2 + q;
+            float v[16];
+            tmem_ld16(t_s + lane_q + 16u * cq, v);
+            if (row >= N)
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            st_slot16(seg_ptr(p, sg, bh, cq, row), v);
+        }
+        if (tid == 0) p.sd_sege[(long long)sg * BH + bh] = P;
+        fence_before_sync();
+        __syncthreads();   // TMEM is read before the next item's first MMA overwrites it
+        fence_after_sync();
+    }
+    if (aborted && tid == 0) {
+        drain_phases(bar_in, pc_in);
+        drain_phases(bar_mma, pc_m);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(t_s, 64);
+    }
+}
+
+// The state entering every segment of a (b, h), in place of S_seg: thread (row n,
+// column block cq, 4 columns j4) of (b, h) = blockIdx.y, segments in order, the
+// loads of the next PF segments in flight while the current one is carried.
+constexpr int SEG_PF = 4;
+__global__ void __launch_bounds__(256) k_ssd_seg_pass(Params p) {
+    const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H, BH = p.Bsz * p.H;
+    const int e = blockIdx.x * 256 + threadIdx.x;   // 0 .. 2047: (cq, j4, n)
+    const int n = e & 127, j4 = (e >> 7) & 3, cq = e >> 9;
+    float4 K = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n < p.N) {
+        float beta0 = 0.f;
+        if (p.two_ep)
+            beta0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), 1)) * ld_io(p.dt, ix_dt(p, b, 0, h), 1);
+        float v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const long long i0 = ix_st(p, b, h, n, 16 * cq + 4 * j4 + k);
+            v[k] = p.h0 ? p.h0[i0] : 0.f;
+            if (p.w0) v[k] = fmaf(beta0, p.w0[i0], v[k]);
+        }
+        K = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    const int ns = p.sd_nseg;
+    float4 buf[SEG_PF];
+    float eb[SEG_PF];
+#pragma unroll
+    for (int k = 0; k < SEG_PF; ++k) {
+        if (k < ns) {
+            buf[k] = __ldcg(seg_ptr(p, k, bh, cq, n) + j4 * NP);
+            eb[k] = p.sd_sege[(long long)k * BH + bh];
+        }
+    }
+    for (int s0 = 0; s0 < ns; s0 += SEG_PF) {
+#pragma unroll
+        for (int k = 0; k < SEG_PF; ++k) {
+            const int sg = s0 + k;
+            if (sg < ns) {
+                const float4 sv = buf[k];
+                const float E = eb[k];
+                if (sg + SEG_PF < ns) {   // refill this stage with a later segment
+                    buf[k] = __ldcg(seg_ptr(p, sg + SEG_PF, bh, cq, n) + j4 * NP);
+                    eb[k] = p.sd_sege[(long long)(sg + SEG_PF) * BH + bh];
+                }
+                __stcg(seg_ptr(p, sg, bh, cq, n) + j4 * NP, K);
+                K = make_float4(fmaf(E, K.x, sv.x), fmaf(E, K.y, sv.y), fmaf(E, K.z, sv.z),
+                                fmaf(E, K.w, sv.w));
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 2)
 k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
           Params p, int lgR) {
-    const int BH = p.Bsz * p.H;
-    const int nitems = p.nc * BH;
-    if ((int)blockIdx.x >= nitems) return;
+    const int BH = p.Bsz * p.H, G = p.sd_G;
+    const int nitems = p.nc * BH;            // chunk items (c * BH + bh); nitems = none
+    const int nseg_items = p.sd_nseg * BH;   // tickets: (segment, b, h), segment slowest
+    if ((int)blockIdx.x >= nseg_items) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,14 +421,16 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         if (want_y) tma_prefetch_desc(&tmY);
-        const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
+        // < nseg_items: the grid is <= nseg_items
+        const int first = atomicAdd(chain_ticket(p), 1);
         s_item[0] = first;
-        issue_x(first);
+        const int fitem = (first / BH) * G * BH + first % BH;   // its first chunk
+        issue_x(fitem);
         ++pc_x.issued;
-        issue_b(first);
+        issue_b(fitem);
         ++pc_b.issued;
         if (want_y) {   // C is read by the outputs only
-            issue_c(first);
+            issue_c(fitem);
             ++pc_c.issued;
         }
     }
@@ -267,7 +441,8 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     const uint32_t tbase = *tslot;
     const uint32_t t_cb = tbase, t_yo = tbase, t_sc = tbase + 128u, t_yd = tbase + 192u;
     const uint32_t lane_q = (32u * qd) << 16;
-    int item = s_item[0];
+    int tk = s_item[0], jj = 0;   // segment ticket, chunk inside the segment
+    int item = (tk / BH) * G * BH + tk % BH;
     Tok tok;
     float alog;
     {
@@ -278,16 +453,21 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     bool aborted = false;
 
     for (int k = 0; item < nitems; ++k) {
-        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
+        // the segment after this one, claimed at its first chunk
+        if (tid == 0 && jj == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const uint32_t par = (uint32_t)(k & 1);
         const ChunkItem it = chunk_item_cs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int bh = b * p.H + h;
         const int t0 = c * Qt;
+        const int sg = tk / BH, glen = min(G, p.nc - sg * G);
         // the previous item's y store has read the staging tile
         if (tid == 0) bulk_wait_read_all();
         chunk_scalars(p, f32, t0, Qt, tok, alog);
-        const int next = s_item[1];
+        // the next chunk: the segment's next, or the first of the next claimed segment
+        const int ntk = jj + 1 < glen ? tk : s_item[1];
+        const int njj = jj + 1 < glen ? jj + 1 : 0;
+        const int next = ntk < nseg_items ? ((ntk / BH) * G + njj) * BH + ntk % BH : nitems;
         if (next < nitems) {
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
@@ -366,14 +546,8 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                 ssd_raise_error(1);
                 chain_abort(p);
             }
-            if (tid == 0 && ok && c > 0 &&
-                !wait_count(p.ws_flag + bh, c, chain_abort_word(p), p.wait_limit)) {
-                ssd_raise_error(2);
-                chain_abort(p);
-                ok = 0;
-            }
             fence_after_sync();
-            if (!__syncthreads_and(ok)) {   // also orders the wait before the loads of K_in
+            if (!__syncthreads_and(ok)) {
                 aborted = true;
                 break;
             }
@@ -387,8 +561,9 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         for (int cq = 2 * cb2; cq < 2 * cb2 + 2; ++cq) {
             // K_in as the bf16 tile of the readout, in X''s place (S_c has read X')
             const int n = row;
+            // K_in: the state entering the segment (segment pass), then the CTA's own carry
             float kc[16], sc[16];
-            load_kin(p, c, b, h, n, cq, kc);
+            ld_slot16(jj == 0 ? seg_ptr(p, sg, bh, cq, n) : priv_ptr(p, blockIdx.x, cq, n), kc);
             tmem_ld16(t_sc + lane_q + 16u * cq, sc);
             const float E = f32[F_SC + 2];
             unsigned char *sv = p.ws_kp
@@ -415,11 +590,7 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
 #pragma unroll
             for (int j = 0; j < 16; ++j) kn[j] = n < N ? fmaf(E, kc[j], sc[j]) : 0.f;
             if (c + 1 < p.nc) {
-                float4 *dst = carry_ptr(p, (c + 1) & 1, bh, cq, n);
-#pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4)
-                    __stcg(dst + j4 * NP, make_float4(kn[4 * j4], kn[4 * j4 + 1], kn[4 * j4 + 2],
-                                                      kn[4 * j4 + 3]));
+                if (jj + 1 < glen) st_slot16(priv_ptr(p, blockIdx.x, cq, n), kn);
             } else if (n < N) {
                 // final state (beta_L = 0, so K_{L-1} = H_{L-1}) and the last write
                 // W_{L-1} = B_{L-1} u_{L-1} (summed over the R value rows)
@@ -441,8 +612,6 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        // the carry of (b, h) is in place: let the next chunk's item go (off the issue path)
-        if (tid == THREADS - 32 && c + 1 < p.nc) publish_count(p.ws_flag + bh, c + 1);
         if (want_y) {
             // ---- masked scores P = CB (.) W -> bf16 tile in B's place (CB and S_c have
             // read B; CB completed with S_c) -------------------------------------------------
@@ -546,6 +715,8 @@ k_ssd_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
             ++pc_x.issued;
         }
         item = next;
+        tk = ntk;
+        jj = njj;
     }
     if (tid == 0) bulk_wait_read_all();
     if (aborted && tid == 0) {
@@ -1384,8 +1555,32 @@ int sm_count();
 static int ssd_lg_rank(int R) { return R == 1 ? 0 : (R == 2 ? 1 : (R == 4 ? 2 : -1)); }
 
 // Tokens per chunk of the scalar-decay kernels (128 (token, rank) rows).
-// Bytes of the carry slots: two fp32 32 KB slots per (b, h).
-size_t ssd_ring_bytes(long long B, long long H) { return (size_t)2 * B * H * 128 * 64 * 4; }
+// Segments of the forward: about eight work items per resident CTA, at most one
+// 32 KB carry slot per CTA.
+constexpr int SSD_GRID_MAX = 296;
+constexpr long long SSD_ITEMS_TARGET = 8LL * SSD_GRID_MAX;
+static int ssd_nchunks(long long L, int R) {
+    const int qt = 128 >> (R == 4 ? 2 : R == 2 ? 1 : 0);
+    return (int)((L + qt - 1) / qt);
+}
+static int ssd_seg_chunks(long long B, long long H, long long L, int R) {
+    const long long nc = ssd_nchunks(L, R);
+    long long g = (nc * B * H + SSD_ITEMS_TARGET - 1) / SSD_ITEMS_TARGET;
+    if (g < 1) g = 1;
+    if (g > nc) g = nc;
+    return (int)g;
+}
+static size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
+// Bytes of the chain buffers: the backward's two 32 KB adjoint slots per (b, h),
+// then the forward's segment states (32 KB per (segment, b, h)), segment decays and
+// the per-CTA carry slots.
+size_t ssd_ring_bytes(long long B, long long H, long long L, int R) {
+    const size_t bh = (size_t)B * H, slot = 128 * 64 * 4;
+    const int nc = ssd_nchunks(L, R), G = ssd_seg_chunks(B, H, L, R);
+    const size_t nseg = (size_t)((nc + G - 1) / G);
+    return al256(2 * bh * slot) + al256(nseg * bh * slot) + al256(nseg * bh * 4) +
+           (size_t)SSD_GRID_MAX * slot;
+}
 
 int ssd_chunk_tokens(int R) {
     const int lg = ssd_lg_rank(R);
@@ -1433,15 +1628,35 @@ cudaError_t ssd_forward(const Params &p, cudaStream_t st) {
         !make_map5(&my, p.y, 64, p.O, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
-    static bool done[64] = {};
+    static bool done[64] = {}, done_s[64] = {};
     cudaError_t e;
     if ((e = ssd_set_smem(k_ssd_fwd, SMEM_BYTES, done)) != cudaSuccess) return e;
+    if ((e = ssd_set_smem(k_ssd_seg_state, SMEM_BYTES, done_s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
         return e;
-    const long long nitems = (long long)p.nc * p.H * p.Bsz;
-    const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
-    k_ssd_fwd<<<grid, THREADS, SMEM_BYTES, st>>>(mx, mb, mc, my, p, lgR);
+    // segment buffers after the adjoint slots (see ssd_ring_bytes)
+    Params q = p;
+    const size_t bh = (size_t)p.Bsz * p.H, slot = 128 * 64 * 4;
+    q.sd_G = ssd_seg_chunks(p.Bsz, p.H, p.L, p.R);
+    q.sd_nseg = (p.nc + q.sd_G - 1) / q.sd_G;
+    char *base = reinterpret_cast<char *>(p.ws_ring) + al256(2 * bh * slot);
+    q.sd_seg = reinterpret_cast<float *>(base);
+    base += al256((size_t)q.sd_nseg * bh * slot);
+    q.sd_sege = reinterpret_cast<float *>(base);
+    base += al256((size_t)q.sd_nseg * bh * 4);
+    q.sd_priv = reinterpret_cast<float *>(base);
+    const long long nitems = (long long)q.sd_nseg * bh;
+    int cap = 2 * sm_count();
+    if (cap > SSD_GRID_MAX) cap = SSD_GRID_MAX;
+    const int grid = (int)(nitems < cap ? nitems : cap);
+    k_ssd_seg_state<<<grid, THREADS, SMEM_BYTES, st>>>(mx, mb, q, lgR);
+    profile_mark(st, "k_ssd_seg_state");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_ssd_seg_pass<<<dim3(8, (unsigned)bh), 256, 0, st>>>(q);
+    profile_mark(st, "k_ssd_seg_pass");
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_ssd_fwd<<<grid, THREADS, SMEM_BYTES, st>>>(mx, mb, mc, my, q, lgR);
     profile_mark(st, "k_ssd_fwd");
     return cudaGetLastError();
 }

@@ -1,5 +1,5 @@
 """The timeout path of the chained tensor-core kernels, exercised without a
-fault: with a carry-wait limit of zero polls every wait of a call gives up,
+fault: with a carry-wait limit of zero polls every carry wait of a call gives up,
 the call stops early and reports SSM_ERR_TIMEOUT from the next device-error
 poll, and the next call with the normal limit is parity-green again.  Nothing
 here faults, traps or hangs the GPU: each wait returns after at most its
@@ -51,8 +51,19 @@ def _timed_out(fn):
 def test_forward_wait_gives_up_then_recovers(case):
     shape, inp, route = case
     dev = scan.to_device(shape, inp)
-    _timed_out(lambda: scan.scan_forward(shape, dev))
-    y, hT, wT = scan.scan_forward(shape, dev)
+    if route == abi.ROUTE_SSD:
+        # the scalar-decay forward walks whole segments and waits on no other work
+        # item: with no polls allowed it still completes, with no error
+        old = abi.ssm_scan_set_wait_limit(0)
+        try:
+            y, hT, wT = scan.scan_forward(shape, dev)
+            torch.cuda.synchronize()
+            abi.ssm_scan_poll_device_error()
+        finally:
+            abi.ssm_scan_set_wait_limit(old)
+    else:
+        _timed_out(lambda: scan.scan_forward(shape, dev))
+        y, hT, wT = scan.scan_forward(shape, dev)
     assert abi.ssm_scan_last_route() == route
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
