@@ -424,7 +424,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     uint64_t *bar_bc = bar_x + 2;                                       // raw B, C
     uint64_t *bar_mma = bar_x + 3;                                      // [2] phase A, B
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 5);
-    int *s_item = reinterpret_cast<int *>(bar_x + 6);                  // [3] claimed tickets
+    int *s_item = reinterpret_cast<int *>(bar_x + 6);                  // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
@@ -458,10 +458,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         tma_prefetch_desc(&tmX);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-        // tickets are claimed two items ahead, so the atomic's latency is hidden
         const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
         s_item[0] = first;
-        s_item[1] = atomicAdd(chain_ticket(p), 1);
         issue_x(first, 0);
         ++pc_x[0].issued;
         issue_bc(first);
@@ -491,9 +489,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 
     for (int k = 0; item < nitems; ++k) {
         // the item after this one (read by every thread after the next barrier)
-        // the ticket of the item after the next one (stored at the end of this item)
-        int pending = 0;
-        if (tid == 0) pending = atomicAdd(chain_ticket(p), 1);
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const int st = k & 1;
         const ChunkItem it = chunk_item_cs(p, item);
         const int c = it.c, h = it.h, b = it.b;
@@ -505,7 +501,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         // ---- this chunk's small inputs; K_c once the previous chunk has published it
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
-        const int next = s_item[(k + 1) % 3];
+        const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_cs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
@@ -660,6 +656,12 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             aborted = true;
             break;
         }
+        // raw B and C are consumed: fetch the next chunk's
+        if (tid == 0 && next < nitems) {
+            issue_bc(next);
+            ++pc_bc.issued;
+        }
+
         // ---- phase A: scores, chunk-local state --------------------------------
         if (tid == 0) {
             fence_after_sync();
@@ -673,11 +675,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                              id_sc, s > 0);
             mma_commit(&bar_mma[0]);
             ++pc_a.issued;
-            // raw B and C are consumed: fetch the next chunk's (after the MMAs are issued)
-            if (next < nitems) {
-                issue_bc(next);
-                ++pc_bc.issued;
-            }
         } else if (tid == 32) {
             fence_after_sync();
             const uint32_t x_base = smem_u32(sX);
@@ -874,7 +871,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             tma_store_4d(&tmY, sm + fwk::SM_P, 0, h, t0, b);
             bulk_commit();
         }
-        if (tid == 0) s_item[(k + 2) % 3] = pending;
         item = next;
     }
     if (tid == 0) bulk_wait_read_all();

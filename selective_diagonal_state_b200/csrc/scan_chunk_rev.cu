@@ -501,7 +501,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);   // [2]: x/dy/states, B/C
     uint64_t *bar_mma = bar_in + 2;                                      // [3] phases A, B, C
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 5);
-    int *s_item = reinterpret_cast<int *>(bar_in + 6);                  // [3] claimed tickets
+    int *s_item = reinterpret_cast<int *>(bar_in + 6);                  // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, nr = p.nr, L = p.L;
@@ -541,10 +541,8 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmDY);
-        // tickets are claimed two items ahead, so the atomic's latency is hidden
         const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
         s_item[0] = first;
-        s_item[1] = atomicAdd(chain_ticket(p), 1);
         issue_xs(first);
         ++pc_in[0].issued;
         issue_bc(first);
@@ -569,9 +567,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     for (int kit = 0; item < nitems; ++kit) {
         // the item after this one (read by every thread after the next barrier)
-        // the ticket of the item after the next one (stored at the end of this item)
-        int pending = 0;
-        if (tid == 0) pending = atomicAdd(chain_ticket(p), 1);
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const ChunkItem it = chunk_item_rcs(p, item);
         const int c = it.c, h = it.h, b = it.b;
         const int g = h / p.hpg;
@@ -581,7 +577,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t par = (uint32_t)(kit & 1);
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
-        const int next = s_item[(kit + 1) % 3];
+        const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
@@ -1226,7 +1222,6 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         fence_before_sync();
         __syncthreads();
-        if (tid == 0) s_item[(kit + 2) % 3] = pending;
         item = next;
     }
     if (aborted && tid == 0) {

@@ -834,7 +834,7 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     uint64_t *bar_k = bar_x + 1, *bar_bc = bar_x + 2;                 // K_in; B + C
     uint64_t *bar_p1 = bar_x + 3, *bar_p2 = bar_x + 4, *bar_p3 = bar_x + 5;   // MMA phases
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 6);
-    int *s_item = reinterpret_cast<int *>(bar_x + 7);                // [3] claimed tickets
+    int *s_item = reinterpret_cast<int *>(bar_x + 7);                // [2] claimed tickets
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, L = p.L;
@@ -876,10 +876,8 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         tma_prefetch_desc(&tmDY);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmC);
-        // tickets are claimed two items ahead, so the atomic's latency is hidden
         const int first = atomicAdd(chain_ticket(p), 1);   // < nitems: the grid is <= nitems
         s_item[0] = first;
-        s_item[1] = atomicAdd(chain_ticket(p), 1);
         issue_x(first);
         ++pc_x.issued;
         issue_k(first);
@@ -910,9 +908,7 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
     bool aborted = false;
 
     for (int k = 0; item < nitems; ++k) {
-        // the ticket of the item after the next one (stored at the end of this item)
-        int pending = 0;
-        if (tid == 0) pending = atomicAdd(chain_ticket(p), 1);
+        if (tid == 0) s_item[1] = atomicAdd(chain_ticket(p), 1);
         const uint32_t par = (uint32_t)(k & 1);
         const ChunkItem it = chunk_item_rcs(p, item);
         const int c = it.c, h = it.h, b = it.b;
@@ -923,7 +919,7 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         // the previous item's stores have read their staging tiles
         if (tid == 0) bulk_wait_read_all();
         ssdk::chunk_scalars(p, f32, t0, Qt, tok, alog, f32 + F_FE);
-        const int next = s_item[(k + 1) % 3];
+        const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = ssdk::tok_load_q(p, nx.b, nx.h, nx.c * Qt, Qt);
@@ -1444,7 +1440,6 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
         }
         fence_before_sync();
         __syncthreads();
-        if (tid == 0) s_item[(k + 2) % 3] = pending;
         item = next;
     }
     if (tid == 0) bulk_wait_read_all();
