@@ -145,16 +145,17 @@ def kernel_bytes(shape, name: str) -> int:
 # (traffic null) instead of going stale.
 NCU_TRAFFIC_PER_ROW = {
     # (workload, kernel): (dram read + write bytes per batch row of one launch, source hash)
-    # ncu --set full captures at batch 2 (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the
-    # full Mamba-2 size; the traffic of these kernels grows with the batch rows
-    ("hybridmamba", "k_chunk_fwd"): (421.24e6, "bc477f309b223f3c"),
-    ("hybridmamba", "k_chunk_bwd_fused"): (605.52e6, "6b57e6460b9284ec"),
-    ("ssd_mimo_r4", "k_ssd_fwd"): (1039.22e6, "3823fac94aef91bf"),
-    ("ssd_mimo_r4", "k_ssd_bwd"): (1740.24e6, "3823fac94aef91bf"),
-    ("mamba2_siso", "k_ssd_fwd"): (18.34e6, "3823fac94aef91bf"),
-    ("mamba2_siso", "k_ssd_bwd"): (76.70e6, "3823fac94aef91bf"),
-    ("mamba1_siso", "k_m1_fwd"): (60.60e6, "f3b528160f538458"),
-    ("mamba1_siso", "k_m1_bwd"): (119.65e6, "f3b528160f538458"),
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum captures at batch 2
+    # (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the full Mamba-2 size; the traffic of
+    # these kernels grows with the batch rows
+    ("hybridmamba", "k_chunk_fwd"): (420.8e6, "44f974fe96fa6c31"),
+    ("hybridmamba", "k_chunk_bwd_fused"): (603.45e6, "bf4b7047cc7bed68"),
+    ("ssd_mimo_r4", "k_ssd_fwd"): (1197.8e6, "968f48c9ed818efd"),
+    ("ssd_mimo_r4", "k_ssd_bwd"): (1736.5e6, "968f48c9ed818efd"),
+    ("mamba2_siso", "k_ssd_fwd"): (31.0e6, "968f48c9ed818efd"),
+    ("mamba2_siso", "k_ssd_bwd"): (75.25e6, "968f48c9ed818efd"),
+    ("mamba1_siso", "k_m1_fwd"): (60.55e6, "cab423aa329e9480"),
+    ("mamba1_siso", "k_m1_bwd"): (118.05e6, "cab423aa329e9480"),
 }
 
 # sources each kernel is compiled from: a traffic entry holds only while they
