@@ -124,8 +124,7 @@ typedef struct ssm_desc {
     int32_t two_endpoint;       /* 0: lambda not read (lam = 1); 1: lambda used */
     int32_t dtype_io;           /* enum ssm_dtype of x, dt, B, C, lambda, y and of their gradients */
     int64_t stride_x[3], stride_y[3], stride_B[3], stride_C[3], stride_dt[3], stride_lambda[3];
-    int32_t angle_mode;         /* enum ssm_angle_mode (ignored when n_pairs == 0).  Per-token
-                                   angles are taken by the token-by-token recurrent kernels */
+    int32_t angle_mode;         /* enum ssm_angle_mode (ignored when n_pairs == 0) */
     int32_t n_static;           /* 0 <= n_static <= n_real: the first n_static real rows are
                                    static, with the transition exp(a_n) at every step whatever
                                    dt_t (HybridMamba's real static rows next to its real and

@@ -217,10 +217,9 @@ struct BwdWs {
 // Shapes the tensor-core chain may take (pointer alignment is checked at call time).
 bool tensor_chain_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
-    const bool static_angles = d->angle_mode == SSM_ANGLE_STATIC || d->n_pairs == 0;
     return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0 &&
-           static_angles && d->n_static == 0 && d->discretization == SSM_DISC_EULER;
+           d->n_static == 0 && d->discretization == SSM_DISC_EULER;
 }
 
 // Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and

@@ -27,6 +27,11 @@ constexpr int F_W = 784;                  // [128] rotation frequency per mode
 constexpr int F_KRE = 912;                // [13][128] mode constants, real part
 constexpr int F_KIM = F_KRE + 13 * 128;   // [13][128] imaginary part
 constexpr int F_END = F_KIM + 13 * 128;
+// per-token rotation angles (p.angle_tok): inclusive prefix over the chunk's tokens,
+// pair-major with a padded row, Theta[j][t] at F_TH + j * TH_LD + t
+constexpr int TH_LD = 65;
+constexpr int F_TH = F_END;
+constexpr int F_END_TH = F_TH + 64 * TH_LD;
 
 constexpr uint32_t KM_LBO = 128, KM_SBO = 2048;  // K-major tiles with K = 128
 
@@ -164,11 +169,62 @@ __device__ __forceinline__ void sincos_red(float x, float *sn, float *cs) {
     __sincosf(r, sn, cs);
 }
 
+// Per-token angles of the chunk starting at token t0 into F_TH: Theta[j][t] = sum of
+// theta over tokens t0 .. t0 + t (tokens past L add nothing).  All threads; ends with
+// a barrier.
+__device__ __forceinline__ void chunk_angles(const Params &p, float *f32, int b, int h, int t0) {
+    const int np = p.np;
+    float *th = f32 + F_TH;
+    for (int i = threadIdx.x; i < 64 * np; i += blockDim.x) {   // coalesced over the pairs
+        const int t = i / np, j = i - t * np;
+        th[j * TH_LD + t] = (t0 + t < p.L) ? __ldg(p.theta + ix_th(p, b, t0 + t, h, j)) : 0.f;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int j = warp; j < np; j += nw) {   // a warp per pair: lane l takes tokens 2l, 2l + 1
+        float *row = th + j * TH_LD;
+        const float a0 = row[2 * lane], a1 = row[2 * lane + 1];
+        float v = a0 + a1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        const float base = v - (a0 + a1);
+        row[2 * lane] = base + a0;
+        row[2 * lane + 1] = base + a0 + a1;
+    }
+    __syncthreads();
+}
+// Theta of pair j at chunk token t (t = -1: the chunk start)
+__device__ __forceinline__ float th_at(const float *f32, int j, int t) {
+    return t < 0 ? 0.f : f32[F_TH + j * TH_LD + t];
+}
+// Rotation angle of pair j from chunk token tr to token t (tr = -1: the chunk start):
+// the pair's frequency times the step sum ds between them, or (TOK, per-token angles)
+// the angles summed over (tr, t].  The kernels are instantiated once per angle mode.
+template <bool TOK>
+__device__ __forceinline__ float pair_angle(const float *f32, int j, float w, float ds, int t,
+                                           int tr) {
+    if constexpr (TOK)
+        return th_at(f32, j, t) - th_at(f32, j, tr);
+    else
+        return w * ds;
+}
+template <bool TOK>
+__device__ __forceinline__ void pair_sincos(float ang, float *sn, float *cs) {
+    if constexpr (TOK)
+        sincos_red(ang, sn, cs);   // per-token angles can be any size
+    else
+        __sincosf(ang, sn, cs);
+}
+
 // Per-mode decay over each sub-block, E_k = e^{lam dS_k}, the products
 // F[i][j] = prod_{k=i}^{j-1} E_k (E_k itself is F[k][k+1]) and
 // G_i = conj(F[0][i]) into the F_KRE / F_KIM slots.  Four consecutive lanes
 // take one mode, lane k its sub-block k; the four factors are exchanged by
 // shuffles inside the group.  Needs F_S, F_A2, F_W; ends with a barrier.
+template <bool TOK>
 __device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32) {
     const int nmode = p.nr + p.np;
     for (int it = threadIdx.x; it < 4 * nmode; it += blockDim.x) {
@@ -181,7 +237,7 @@ __device__ __forceinline__ void chunk_mode_constants(const Params &p, float *f32
         float er = mag, ei = 0.f;
         if (m >= p.nr) {
             float sn, cs;
-            sincos_red(w * ds, &sn, &cs);
+            sincos_red(pair_angle<TOK>(f32, m - p.nr, w, ds, 16 * k + 15, 16 * k - 1), &sn, &cs);
             er = mag * cs;
             ei = mag * sn;
         }
@@ -229,7 +285,8 @@ __device__ __forceinline__ ModePrefetch mode_load(const Params &p, int h) {
     const int m = threadIdx.x;
     if (m < p.nr + p.np) {
         r.alog = __ldg(p.A_log + h * p.ndec + (p.per_coord ? m : 0));
-        if (m >= p.nr) r.w = __ldg(p.theta + h * p.np + (m - p.nr));
+        // per-token angles come from F_TH (chunk_angles), not from a frequency
+        if (m >= p.nr && !p.angle_tok) r.w = __ldg(p.theta + h * p.np + (m - p.nr));
     }
     return r;
 }

@@ -64,10 +64,12 @@ constexpr uint32_t SM_X = 16384;    // 8 KB  x (128B swizzle)
 constexpr uint32_t SM_BH = 24576;   // 16 KB Bh hi, MN-major (M = state rows, K = s)
 constexpr uint32_t SM_BHL = 40960;  // 16 KB Bh lo
 constexpr uint32_t SM_F32 = 57344;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+// the barriers follow the fp32 area, longer by the angle prefixes with per-token angles
+template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_TH : F_END) * 4; }
+template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
 }  // namespace stl
 
+template <bool TOK>
 __global__ void __launch_bounds__(stl::THREADS)
 k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                     Params p) {
@@ -76,7 +78,7 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + stl::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + stl::SM_BAR);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + stl::sm_bar<TOK>());
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 2);
 
@@ -101,7 +103,8 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     if (warp == 0) tmem_alloc(tslot, stl::TMEM_COLS);
     mode_rates(p, f32, h);
     chunk_tokens(p, f32, b, h, t0, true);
-    chunk_mode_constants(p, f32);
+    if constexpr (TOK) chunk_angles(p, f32, b, h, t0);
+    chunk_mode_constants<TOK>(p, f32);
     for (int m = tid; m < nmode; m += stl::THREADS) {
         float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
         ce[2 * m] = f32[F_KRE + fslot(0, 4) * NP + m];
@@ -144,7 +147,7 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 } else {
                     const int m = nr + ((r - nr) >> 1);
                     float sn, cs;
-                    __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                    pair_sincos<TOK>(pair_angle<TOK>(f32, m - nr, f32[F_W + m], ds, t, 16 * ib - 1), &sn, &cs);
                     const float eb = sig * ex2_fast(fminf(-f32[F_A2 + m] * ds, 120.f));
                     const float bi0 = eb * fmaf(rb[j], cs, rb[j + 1] * sn);
                     const float bi1 = eb * fmaf(rb[j + 1], cs, -rb[j] * sn);
@@ -370,10 +373,11 @@ constexpr uint32_t SM_BHL = 139264;   // 16 KB Bh lo
 constexpr uint32_t SM_KT = 155648;    // 16 KB K_c hi tile (MN-major: M = 64 p, K = 128 rows)
 constexpr uint32_t SM_P = 172032;     // 8 KB  P^T tiles, MN-major (N = 16 t, K = 64 s)
 constexpr uint32_t SM_F32 = 180224;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+// the barriers follow the fp32 area, longer by the angle prefixes with per-token angles
+template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_TH : F_END) * 4; }
+template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
 static_assert(THREADS * 16 == 8192, "one 16-byte piece of the saved P tiles per thread");
-static_assert(SM_BAR % 8 == 0 && SMEM_BYTES <= 232448, "shared memory map");
+static_assert(sm_bar<true>() % 8 == 0 && smem_bytes<true>() <= 232448, "shared memory map");
 }  // namespace fwk
 
 // K_c of thread (n, cq): the carry slot, or K_0 = h0 + beta_0 w0 for the first chunk
@@ -408,6 +412,7 @@ __device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int
     }
 }
 
+template <bool TOK>
 __global__ void __launch_bounds__(fwk::THREADS, 1)
 k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -420,7 +425,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + fwk::SM_F32);
-    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + fwk::SM_BAR);   // [2] x stages
+    uint64_t *bar_x = reinterpret_cast<uint64_t *>(sm + fwk::sm_bar<TOK>());   // [2] x stages
     uint64_t *bar_bc = bar_x + 2;                                       // raw B, C
     uint64_t *bar_mma = bar_x + 3;                                      // [2] phase A, B
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_x + 5);
@@ -501,6 +506,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         // ---- this chunk's small inputs; K_c once the previous chunk has published it
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
+        if constexpr (TOK) chunk_angles(p, f32, b, h, t0);
         const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_cs(p, next);
@@ -512,7 +518,7 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                 ++pc_x[st ^ 1].issued;
             }
         }
-        chunk_mode_constants(p, f32);
+        chunk_mode_constants<TOK>(p, f32);
         if (p.ws_ce && tid < p.nr + p.np) {
             float *ce = p.ws_ce + bhc(p, b, h, c) * (2 * NP);
             ce[2 * tid] = f32[F_KRE + fslot(0, 4) * NP + tid];
@@ -591,7 +597,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                         const int m = nr + ((r - nr) >> 1);
                         const float x = f32[F_A2 + m] * ds;
                         float sn, cs;
-                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        pair_sincos<TOK>(pair_angle<TOK>(f32, m - nr, f32[F_W + m], ds, t, 16 * ib - 1), &sn,
+                                         &cs);
                         // rotate by cis(-phi): (u + iv)(cs - i sn)
                         const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
                         const float ci0 = ec * fmaf(c0, cs, c1 * sn);
@@ -935,7 +942,7 @@ bool chunk_fwd_supported(const Params &p) {
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
     // y (forward) leaves by TMA stores
     const bool yok = !p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]));
-    return yok && !p.angle_tok && !p.nst && !p.zoh && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
+    return yok && !p.nst && !p.zoh && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
            (p.N == 64 || p.N == 128) &&
            p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
            st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) && st16(p.sB[2]) &&
@@ -980,6 +987,34 @@ static cudaError_t set_smem_once(K kern, uint32_t bytes, bool (&done)[64]) {
     return e;
 }
 
+template <bool TOK>
+static cudaError_t launch_state_local(const CUtensorMap &mx, const CUtensorMap &mb, const Params &p,
+                                      cudaStream_t st) {
+    using namespace chunkfwd;
+    static bool done[64] = {};
+    cudaError_t e;
+    if ((e = set_smem_once(k_chunk_state_local<TOK>, stl::smem_bytes<TOK>(), done)) != cudaSuccess)
+        return e;
+    k_chunk_state_local<TOK>
+        <<<dim3(p.nc, p.H, p.Bsz), stl::THREADS, stl::smem_bytes<TOK>(), st>>>(mx, mb, p);
+    return cudaSuccess;
+}
+
+template <bool TOK>
+static cudaError_t launch_fwd(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc,
+                              const CUtensorMap &my, const Params &p, int grid, cudaStream_t st) {
+    using namespace chunkfwd;
+    k_chunk_fwd<TOK><<<grid, fwk::THREADS, fwk::smem_bytes<TOK>(), st>>>(mx, mb, mc, my, p);
+    return cudaSuccess;
+}
+
+template <bool TOK>
+static cudaError_t fwd_smem(const Params &p) {
+    using namespace chunkfwd;
+    static bool done[64] = {};
+    return set_smem_once(k_chunk_fwd<TOK>, fwk::smem_bytes<TOK>(), done);
+}
+
 // The state entering every chunk (p.ws_kp) and the chunk decays (p.ws_ce);
 // also hT and the last write when p.hT / p.wT are set.
 cudaError_t chunk_states(const Params &p, cudaStream_t st) {
@@ -988,10 +1023,9 @@ cudaError_t chunk_states(const Params &p, cudaStream_t st) {
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
         !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true))
         return cudaErrorInvalidValue;
-    static bool a1[64] = {};
-    cudaError_t e;
-    if ((e = set_smem_once(k_chunk_state_local, stl::SMEM_BYTES, a1)) != cudaSuccess) return e;
-    k_chunk_state_local<<<dim3(p.nc, p.H, p.Bsz), stl::THREADS, stl::SMEM_BYTES, st>>>(mx, mb, p);
+    cudaError_t e = p.angle_tok ? launch_state_local<true>(mx, mb, p, st)
+                                : launch_state_local<false>(mx, mb, p, st);
+    if (e != cudaSuccess) return e;
     profile_mark(st, "k_chunk_state_local");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_chunk_state_pass<<<dim3(p.H, p.Bsz), pas::THREADS, 0, st>>>(p);
@@ -1007,9 +1041,8 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         !make_map(&mc, p.Cm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
-    static bool a3[64] = {};
     cudaError_t e;
-    if ((e = set_smem_once(k_chunk_fwd, fwk::SMEM_BYTES, a3)) != cudaSuccess) return e;
+    if ((e = p.angle_tok ? fwd_smem<true>(p) : fwd_smem<false>(p)) != cudaSuccess) return e;
     // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
@@ -1019,7 +1052,10 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     CUtensorMap my;
     if (!make_map(&my, p.y, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
-    k_chunk_fwd<<<grid, fwk::THREADS, fwk::SMEM_BYTES, st>>>(mx, mb, mc, my, p);
+    if (p.angle_tok)
+        launch_fwd<true>(mx, mb, mc, my, p, grid, st);
+    else
+        launch_fwd<false>(mx, mb, mc, my, p, grid, st);
     profile_mark(st, "k_chunk_fwd");
     return cudaGetLastError();
 }

@@ -59,10 +59,12 @@ constexpr uint32_t SM_BH = 98304;     // 16 KB Bh (stored MN-major with M = rows
 constexpr uint32_t SM_P = 114688;     // 8 KB  P^T, K-major (rows s, K = t)
 constexpr uint32_t SM_GC = 122880;    // 16 KB Gc bf16, MN-major B operand (N = p, K = state rows)
 constexpr uint32_t SM_F32 = 139264;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+// the barriers follow the fp32 area, longer by the angle prefixes with per-token angles
+template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_TH : F_END) * 4; }
+template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
 }  // namespace dxk
 
+template <bool TOK>
 __global__ void __launch_bounds__(dxk::THREADS, 1)
 k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                const __grid_constant__ CUtensorMap tmDY, Params p) {
@@ -71,7 +73,7 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + dxk::SM_F32);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dxk::SM_BAR);
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + dxk::sm_bar<TOK>());
     uint64_t *bar_mma = bar_tma + 1;   // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_tma + 3);
 
@@ -105,7 +107,8 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
         for (int i = tid; i < (int)((dxk::SM_P - dxk::SM_CI) / 16); i += dxk::THREADS)
             reinterpret_cast<uint4 *>(sm + dxk::SM_CI)[i] = make_uint4(0, 0, 0, 0);
     chunk_tokens(p, f32, b, h, t0, true);
-    chunk_mode_constants(p, f32);
+    if constexpr (TOK) chunk_angles(p, f32, b, h, t0);
+    chunk_mode_constants<TOK>(p, f32);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -160,7 +163,8 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
                         const int m = nr + ((r - nr) >> 1);
                         const float x = f32[F_A2 + m] * ds;
                         float sn, cs;
-                        __sincosf(f32[F_W + m] * ds, &sn, &cs);
+                        pair_sincos<TOK>(pair_angle<TOK>(f32, m - nr, f32[F_W + m], ds, t, 16 * ib - 1),
+                                         &sn, &cs);
                         const float ec = ex2_fast(x), eb = sig * ex2_fast(fminf(-x, 120.f));
                         vCI[j] = ec * fmaf(c0, cs, c1 * sn);
                         vCI[j + 1] = ec * fmaf(c1, cs, -c0 * sn);
@@ -469,8 +473,10 @@ constexpr uint32_t SM_KTL = 147456;   // 16 KB K_prev lo
 constexpr uint32_t SM_GC = 163840;    // 16 KB Gc hi (rows n, K = p)
 constexpr uint32_t SM_GCL = 180224;   // 16 KB Gc lo
 constexpr uint32_t SM_F32 = 196608;
-constexpr uint32_t SM_BAR = SM_F32 + F_END * 4;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 64 + 1024;
+// the barriers follow the fp32 area, longer by the angle prefixes with per-token angles
+template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_TH : F_END) * 4; }
+template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
+static_assert(smem_bytes<true>() <= 232448, "shared memory map");
 constexpr int RED_LD = 65;            // row stride of the column reductions (floats)
 // after phase B the Bo .. G regions are free: two [128][RED_LD] reductions and exchange space
 constexpr uint32_t SM_RED = SM_BO;
@@ -486,6 +492,7 @@ __device__ __forceinline__ uint32_t e_col(int j, int k) {   // k >= j
     return 352u + 16u * (uint32_t)((j == 0 ? 0 : (j == 1 ? 4 : (j == 2 ? 7 : 9))) + (k - j));
 }
 
+template <bool TOK>
 __global__ void __launch_bounds__(fuk::THREADS, 1)
 k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
@@ -498,7 +505,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *f32 = reinterpret_cast<float *>(sm + fuk::SM_F32);
-    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::SM_BAR);   // [2]: x/dy/states, B/C
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + fuk::sm_bar<TOK>());   // [2]: x/dy/states, B/C
     uint64_t *bar_mma = bar_in + 2;                                      // [3] phases A, B, C
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_in + 5);
     int *s_item = reinterpret_cast<int *>(bar_in + 6);                  // [2] claimed tickets
@@ -577,13 +584,14 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t par = (uint32_t)(kit & 1);
         mode_rates_from(p, f32, mp);
         chunk_tokens_from(p, f32, t0, tok, true);
+        if constexpr (TOK) chunk_angles(p, f32, b, h, t0);
         const int next = s_item[1];
         if (next < nitems) {
             const ChunkItem nx = chunk_item_rcs(p, next);
             tok = tok_load(p, nx.b, nx.h, nx.c * Q);
             mp = mode_load(p, nx.h);
         }
-        chunk_mode_constants(p, f32);
+        chunk_mode_constants<TOK>(p, f32);
         const bool ok0 = mbar_wait(&bar_in[0], par, WAIT_LIMIT);
         const bool ok1 = ok0 && mbar_wait(&bar_in[1], par, WAIT_LIMIT);
         if (tid == 0) {
@@ -630,11 +638,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                         const int m = nr + ((r - nr) >> 1);
                         const float a = f32[F_A2 + m], w = f32[F_W + m];
                         float sn, cs;
-                        __sincosf(w * dsb, &sn, &cs);
+                        pair_sincos<TOK>(pair_angle<TOK>(f32, m - nr, w, dsb, t, 16 * kb - 1), &sn, &cs);
                         const float eb = sig * ex2_fast(fminf(-a * dsb, 120.f));
                         vb[j] = eb * fmaf(rb[j], cs, rb[j + 1] * sn);
                         vb[j + 1] = eb * fmaf(rb[j + 1], cs, -rb[j] * sn);
-                        __sincosf(w * dse, &sn, &cs);
+                        pair_sincos<TOK>(pair_angle<TOK>(f32, m - nr, w, dse, t, 16 * kb + 15), &sn, &cs);
                         const float ec = ex2_fast(fminf(a * dse, 120.f));
                         vc[j] = ec * fmaf(rc[j], cs, rc[j + 1] * sn);
                         vc[j + 1] = ec * fmaf(rc[j + 1], cs, -rc[j] * sn);
@@ -975,6 +983,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const bool pr_row = valid && n >= nr;
         const bool im_row = pr_row && ((n - nr) & 1);
         const float a2 = valid ? f32[F_A2 + m] : 0.f, w = valid ? f32[F_W + m] : 0.f;
+        const int jp = pr_row ? (n - nr) >> 1 : 0;   // rotation pair of the row
         const int tc = 16 * i;
 
         // part 1: dCK_t = e^{lam S_t} V + e^{lam (S_t - Sb_i)} sum_k F[k][i] D_{i,k}
@@ -1009,7 +1018,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 float er = mag, ei = 0.f;
                 if (pr_row) {
                     float sn, cs;
-                    __sincosf(w * ds, &sn, &cs);
+                    pair_sincos<TOK>(pair_angle<TOK>(f32, jp, w, ds, tc + j, 16 * i - 1), &sn, &cs);
                     er = mag * cs;
                     ei = mag * sn;
                 }
@@ -1027,7 +1036,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
 
         // part 2: gbu, the decay-gradient suffix sums, dB / dC, walking backwards
-        const float coef = !valid ? 0.f : (im_row ? -w : a2 * 0.6931471805599453f);
+        // per token and row: the ddt term of the suffix sum (a for the decay, -w for the
+        // angle); with per-token angles the imaginary rows keep -(suffix sum), the angle's
+        // own gradient, which leaves through dtheta instead
+        const float coef = !valid ? 0.f
+                                  : (im_row ? (TOK ? -1.f : -w) : a2 * 0.6931471805599453f);
         const bool one_head = p.hpg == 1;
         const long long tstride = (long long)p.H * p.N;
         float *gdst = p.ws_gbu + ix_wsk(p, b, t0, h, 0, 1, valid ? n : 0);
@@ -1066,7 +1079,7 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 float er = mag, ei = 0.f;
                 if (pr_row) {
                     float sn, cs;
-                    __sincosf(w * ds, &sn, &cs);
+                    pair_sincos<TOK>(pair_angle<TOK>(f32, jp, w, ds, tc + 15, t), &sn, &cs);
                     er = mag * cs;
                     ei = mag * sn;
                 }
@@ -1143,6 +1156,14 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (later != 0.f) {
             const float add = coef * later;
             for (int t = tc; t < tc + 16; ++t) red2[n * fuk::RED_LD + t] += add;
+        }
+        if (TOK && im_row) {
+            // dL/dtheta_t of this pair, the part from inside the chunk (the carry from
+            // later chunks is added by the block-carry pass); kept out of ddt
+            for (int t = tc; t < tc + 16; ++t) {
+                if (t0 + t < L) p.dtheta[ix_th(p, b, t0 + t, h, jp)] = red2[n * fuk::RED_LD + t];
+                red2[n * fuk::RED_LD + t] = 0.f;
+            }
         }
         dacc += (im_row ? -later : later) * sdt;
         xch[(fuk::TQ + i) * 128 + n] = dacc;
@@ -1261,6 +1282,16 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool (&done)[64]) {
 cudaError_t chunk_states(const Params &p, cudaStream_t st);
 int sm_count();
 
+// Shared memory opt-in of the dx and fused kernels of one angle mode.
+template <bool TOK>
+static cudaError_t rev_smem() {
+    using namespace chunkrev;
+    static bool a3[64] = {}, a4[64] = {};
+    cudaError_t e;
+    if ((e = set_smem(k_chunk_bwd_dx<TOK>, dxk::smem_bytes<TOK>(), a3)) != cudaSuccess) return e;
+    return set_smem(k_chunk_bwd_fused<TOK>, fuk::smem_bytes<TOK>(), a4);
+}
+
 // The state entering every chunk for the tensor-core backward (p.ws_kp,
 // p.ws_ce), unless the forward's are given (p.states_ready).
 cudaError_t chunk_bwd_states(const Params &p, cudaStream_t st) {
@@ -1280,10 +1311,8 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         !make_map(&mdy, p.dy, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
-    static bool a3[64] = {}, a4[64] = {};
     cudaError_t e;
-    if ((e = set_smem(k_chunk_bwd_dx, dxk::SMEM_BYTES, a3)) != cudaSuccess) return e;
-    if ((e = set_smem(k_chunk_bwd_fused, fuk::SMEM_BYTES, a4)) != cudaSuccess) return e;
+    if ((e = p.angle_tok ? rev_smem<true>() : rev_smem<false>()) != cudaSuccess) return e;
     // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
@@ -1297,7 +1326,12 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
             (!make_map(&mdb, p.dBm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
              !make_map(&mdc, p.dCm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true)))
             return cudaErrorInvalidValue;
-        k_chunk_bwd_fused<<<pgrid, fuk::THREADS, fuk::SMEM_BYTES, st>>>(mx, mb, mc, mdy, mdb, mdc, p);
+        if (p.angle_tok)
+            k_chunk_bwd_fused<true>
+                <<<pgrid, fuk::THREADS, fuk::smem_bytes<true>(), st>>>(mx, mb, mc, mdy, mdb, mdc, p);
+        else
+            k_chunk_bwd_fused<false>
+                <<<pgrid, fuk::THREADS, fuk::smem_bytes<false>(), st>>>(mx, mb, mc, mdy, mdb, mdc, p);
     }
     profile_mark(st, "k_chunk_bwd_fused");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1309,7 +1343,10 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
         profile_mark(st, "k_chunk_bwd_dx_saved");
     } else {
-        k_chunk_bwd_dx<<<grid, dxk::THREADS, dxk::SMEM_BYTES, st>>>(mb, mc, mdy, p);
+        if (p.angle_tok)
+            k_chunk_bwd_dx<true><<<grid, dxk::THREADS, dxk::smem_bytes<true>(), st>>>(mb, mc, mdy, p);
+        else
+            k_chunk_bwd_dx<false><<<grid, dxk::THREADS, dxk::smem_bytes<false>(), st>>>(mb, mc, mdy, p);
         profile_mark(st, "k_chunk_bwd_dx");
     }
     return cudaGetLastError();

@@ -76,10 +76,11 @@ def test_angle_mode_validation(lib):
     st = abi.make_desc(sh.replace(n_static=16))
     assert st.n_static == 16
     assert abi.ssm_scan_workspace_size(st, abi.PASS_FWD) == 0
-    # per-token angles run on the recurrent kernels: no chunk workspace
+    # per-token angles take the tensor-core chain as static ones do: the same
+    # chunk workspace
     pt = abi.make_desc(sh.replace(angle_mode=S.ANGLE_PER_TOKEN))
-    assert abi.ssm_scan_workspace_size(pt, abi.PASS_FWD) == 0
-    assert abi.ssm_scan_workspace_size(abi.make_desc(sh), abi.PASS_FWD) > 0
+    assert abi.ssm_scan_workspace_size(pt, abi.PASS_FWD) == \
+        abi.ssm_scan_workspace_size(abi.make_desc(sh), abi.PASS_FWD) > 0
 
 
 def test_wait_limit_setter(lib):

@@ -28,7 +28,6 @@ def chunk_eligible(shape):
     return (shape.dtype_io == S.DTYPE_BF16 and shape.headdim == 64 and shape.rank_in == 1
             and shape.rank_out == 1 and shape.nstate in (64, 128) and shape.n_real % 8 == 0
             and shape.seqlen > 0 and shape.chunk != 1
-            and not (shape.angle_mode == S.ANGLE_PER_TOKEN and shape.n_pairs)
             and shape.n_static == 0 and shape.discretization == S.DISC_EULER)
 
 
@@ -178,13 +177,14 @@ def test_channel_scan_shapes(kw):
 def test_per_token_angles(kw):
     """Per-token rotation angles theta[b][t][h][j] (the complex state of
     Mamba-3): forward, and the per-token angle gradient across several 64-token
-    blocks of the finalize scan."""
+    chunks -- on the tensor-core chain for the bf16 HybridMamba heads, on the
+    recurrent kernels for the others."""
     base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=150,
                                               angle_mode=S.ANGLE_PER_TOKEN)
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=91, with_state=True)
     assert inp["theta"].shape == (shape.batch, shape.seqlen, shape.nheads, shape.n_pairs)
-    check_all(shape, inp, route=abi.ROUTE_RECURRENT)
+    check_all(shape, inp)   # the tensor-core chain for bf16 HybridMamba heads
 
 
 @pytest.mark.parametrize("kw", [
@@ -418,7 +418,8 @@ def test_moderate_decay_stays_chunked():
 
 @pytest.mark.parametrize("kw", [dict(), dict(seqlen=64), dict(seqlen=1),
                                 dict(decay_mode=S.DECAY_PER_HEAD, two_endpoint=0, n_real=128,
-                                     n_pairs=0, ngroups=2)])
+                                     n_pairs=0, ngroups=2),
+                                dict(angle_mode=S.ANGLE_PER_TOKEN)])
 def test_backward_from_saved_states(kw):
     """The backward that reads the forward's chunk states gives the same
     gradients as the one that recomputes them, and the oracle's.  Everything but
