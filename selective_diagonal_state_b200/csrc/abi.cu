@@ -223,14 +223,18 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
 }
 
 // Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and
-// SSD-MIMO with R = O in {1, 2, 4} (pointer alignment is checked at call time).
+// SSD-MIMO with R, O in {1, 2, 4} (pointer alignment is checked at call time).
 bool ssd_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
+    auto rank_ok = [](int r) { return r == 1 || r == 2 || r == 4; };
     return d->dtype_io == SSM_BF16 && d->decay_mode == SSM_DECAY_PER_HEAD && d->n_pairs == 0 &&
-           d->headdim == 64 && (N == 64 || N == 128) && d->rank_in == d->rank_out &&
-           (d->rank_in == 1 || d->rank_in == 2 || d->rank_in == 4) && d->chunk != 1 &&
-           d->seqlen > 0 && d->n_static == 0 && d->discretization == SSM_DISC_EULER;
+           d->headdim == 64 && (N == 64 || N == 128) && rank_ok(d->rank_in) &&
+           rank_ok(d->rank_out) && d->chunk != 1 && d->seqlen > 0 && d->n_static == 0 &&
+           d->discretization == SSM_DISC_EULER;
 }
+// (token, rank) rows per token of the scalar-decay chain: the wider of the two ranks
+// (the narrower side's extra rows are zero)
+static int ssd_rank(const ssm_desc_t *d) { return d->rank_in > d->rank_out ? d->rank_in : d->rank_out; }
 
 // Shapes of the channel scan (Mamba-1: head dim 1, 8 or 16 real state rows,
 // groups of a multiple of 64 channels).
@@ -269,10 +273,10 @@ FwdWs fwd_layout(const ssm_desc_t *d) {
         // ticket and abort words; a training forward also keeps the state entering every
         // chunk of ssm::ssd_chunk_tokens tokens (bf16 hi + lo tiles, 32 KB)
         const size_t bh = (size_t)d->batch * d->nheads;
-        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        const int qt = ssm::ssd_chunk_tokens(ssd_rank(d));
         const size_t units = bh * (size_t)((d->seqlen + qt - 1) / qt);
         const size_t slot = 128 * (size_t)d->headdim * 4;
-        size_t off = align256(ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, d->rank_in));
+        size_t off = align256(ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, ssd_rank(d)));
         w.off_flag = off;
         off = align256(off + (bh + 2) * 4);
         w.total_infer = off;
@@ -317,14 +321,14 @@ struct SsdBwdWs {
 SsdBwdWs ssd_bwd_layout(const ssm_desc_t *d) {
     SsdBwdWs w;
     const size_t bh = (size_t)d->batch * d->nheads;
-    const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+    const int qt = ssm::ssd_chunk_tokens(ssd_rank(d));
     const size_t nc = (size_t)((d->seqlen + qt - 1) / qt);
     const size_t slot = 128 * (size_t)d->headdim * 4;
     const size_t BLH = (size_t)d->batch * d->seqlen * d->nheads;
     const size_t N = nstate(d);
     size_t off = 0;
     w.off_ring = off;   // carry slots and the forward's segment buffers
-    off = align256(off + ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, d->rank_in));
+    off = align256(off + ssm::ssd_ring_bytes(d->batch, d->nheads, d->seqlen, ssd_rank(d)));
     w.off_flag = off;
     off = align256(off + (bh + 2) * 4);
     w.off_kp = off;
@@ -622,7 +626,7 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         p.ws_ring = (float *)(ws + lay.off_ring);
         p.ws_flag = (int *)(ws + lay.off_flag);
         if (workspace_bytes >= lay.total) p.ws_kp = (float *)(ws + lay.off_kp);
-        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        const int qt = ssm::ssd_chunk_tokens(ssd_rank(d));
         p.nc = (int)((d->seqlen + qt - 1) / qt);
         profile_begin(st);
         const cudaError_t e = ssm::ssd_forward(p, st);
@@ -797,7 +801,7 @@ int bwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
             pc.sd_dBh = (float *)(ws + sl.off_dBh);
             pc.sd_dCh = (float *)(ws + sl.off_dCh);
         }
-        const int qt = ssm::ssd_chunk_tokens(d->rank_in);
+        const int qt = ssm::ssd_chunk_tokens(ssd_rank(d));
         pc.nc = (int)((d->seqlen + qt - 1) / qt);
         if (saved) {
             pc.ws_kp = (float *)((const char *)saved + fwd_layout(d).off_kp);

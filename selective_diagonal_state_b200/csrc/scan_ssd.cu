@@ -2,7 +2,7 @@
 // SSD-MIMO configurations ("When a Diagonal State Is Not Enough",
 // sungsoo.github.io, Part 03 "Selective SSM and masked linear attention" and
 // "SISO and MIMO"; Part 08 item 3), bf16 I/O, fp32 state, head dim 64, 64 or
-// 128 state rows, rank R = O in {1, 2, 4}, optional two-endpoint writes.
+// 128 state rows, ranks R, O in {1, 2, 4}, optional two-endpoint writes.
 //
 // With one decay a per head the transition between tokens s < t is the scalar
 // exp(a (S_t - S_s)), S the cumulative sum of dt, so the state-mediated part
@@ -22,7 +22,12 @@
 //     E = exp(a S_end).
 // Every exponent is <= 0, so no range condition applies.
 //
-// A chunk has 128 (token, rank) rows: 128 / R tokens.  Per chunk, on the
+// A chunk has 128 (token, rank) rows: 128 / max(R, O) tokens.  When R != O the
+// narrower side's extra rank rows are zero: the tensor maps of x, B (R ranks) and
+// of y, C, dy (O ranks) all use a box of max(R, O) ranks, TMA fills the rows past
+// a tensor's own rank count with zeros on a load and drops them on a store, so a
+// zero source row adds nothing and a zero target row is never written.  Per chunk,
+// on the
 // tensor cores (M = 128 everywhere, fp32 accumulators in TMEM):
 //     CB   = C (128 j x N) . B^T (N x 128 i)
 //     S_c  = B^T (N x 128 i) . X' (128 i x 64 p),   X' = diag(f) X
@@ -1331,9 +1336,11 @@ k_ssd_bwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUten
                         for (int j = 0; j < 8; ++j) o8[j] = v[8 * q + j];
                         *reinterpret_cast<uint4 *>(stg + sw_off(row, 4 * (cb4 & 1) + q)) = pack8(o8);
                     }
-                } else if (tvalid && n0 < N) {
+                } else if (tvalid && n0 < N && (row & Rm) < (half ? p.O : p.R)) {
+                    // the (token, rank) row's own rank: a source rank of dB (< R) or a
+                    // target rank of dC (< O)
                     float *dst = (half ? p.sd_dCh : p.sd_dBh) +
-                                 ix_wsk(p, b, t0 + ti, h, row & Rm, p.R, n0);
+                                 ix_wsk(p, b, t0 + ti, h, row & Rm, half ? p.O : p.R, n0);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         reinterpret_cast<float4 *>(dst)[q] =
@@ -1498,13 +1505,16 @@ __global__ void k_ssd_params(Params p) {
             }
         const float a = -expf(__ldg(p.A_log + h * p.ndec));
         p.dA_log[h * p.ndec] = a * sa;
-        if (p.dD) p.dD[h] = sd;
+        if (p.dD) p.dD[h] = p.R == p.O ? sd : 0.f;   // D is used only when O == R
     }
 }
 
 // dB / dC of groups with several heads: the fixed-order sum of the per-head parts.
+// Rank rr of a token is a source rank of dB when rr < R and a target rank of dC
+// when rr < O.
 __global__ void k_ssd_group_sum(Params p) {
-    const int RN = p.R * p.N;
+    const int Rp = p.R > p.O ? p.R : p.O;
+    const int RN = Rp * p.N;
     const long long total = (long long)p.Bsz * p.L * p.G * RN;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
          i += (long long)gridDim.x * blockDim.x) {
@@ -1514,30 +1524,33 @@ __global__ void k_ssd_group_sum(Params p) {
         const long long r2 = r / p.G;
         const int t = (int)(r2 % p.L), b = (int)(r2 / p.L);
         const int rr = e / p.N, n = e % p.N;
+        // a rank past one side's count reads that side's last rank and stores nothing
+        const int rb = min(rr, p.R - 1), rc = min(rr, p.O - 1);
         float sb = 0.f, sc = 0.f;
         for (int k = 0; k < p.hpg; ++k) {
             const int h = g * p.hpg + k;
-            sb += p.sd_dBh[ix_wsk(p, b, t, h, rr, p.R, n)];
-            sc += p.sd_dCh[ix_wsk(p, b, t, h, rr, p.O, n)];
+            sb += p.sd_dBh[ix_wsk(p, b, t, h, rb, p.R, n)];
+            sc += p.sd_dCh[ix_wsk(p, b, t, h, rc, p.O, n)];
         }
-        st_io(p.dBm, ix_B(p, b, t, g, rr, n), sb, 1);
-        st_io(p.dCm, ix_C(p, b, t, g, rr, n), sc, 1);
+        if (rr < p.R) st_io(p.dBm, ix_B(p, b, t, g, rr, n), sb, 1);
+        if (rr < p.O) st_io(p.dCm, ix_C(p, b, t, g, rr, n), sc, 1);
     }
 }
 
 namespace ssdk {
 
-// 5-D bf16 map over (inner, rank, head-or-group, time, batch), box
-// (64, rank, 1, tokens, 1), 128-byte swizzle: one box is the chunk's 128
-// (token, rank) rows of 64 elements.
-static bool make_map5(CUtensorMap *m, const void *base, uint64_t inner, uint64_t R, uint64_t d2,
-                      uint64_t L, uint64_t B, uint64_t sR, uint64_t s2, uint64_t sL, uint64_t sB,
-                      uint32_t Qt) {
+// 5-D bf16 map over (inner, rank, head-or-group, time, batch) of a tensor with R
+// ranks, box (64, Rb, 1, tokens, 1) with Rb = max(R, O) >= R, 128-byte swizzle: one
+// box is the chunk's 128 (token, rank) rows of 64 elements, rank rows R .. Rb - 1
+// out of bounds (zero-filled by a load, dropped by a store).
+static bool make_map5(CUtensorMap *m, const void *base, uint64_t inner, uint64_t R, uint32_t Rb,
+                      uint64_t d2, uint64_t L, uint64_t B, uint64_t sR, uint64_t s2, uint64_t sL,
+                      uint64_t sB, uint32_t Qt) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
+    if (!fn || Rb < R) return false;
     cuuint64_t dims[5] = {inner, R, d2, L, B};
     cuuint64_t strides[4] = {sR * 2, s2 * 2, sL * 2, sB * 2};
-    cuuint32_t box[5] = {64, (cuuint32_t)R, 1, Qt, 1};
+    cuuint32_t box[5] = {64, Rb, 1, Qt, 1};
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1553,8 +1566,11 @@ static bool make_map5(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 int sm_count();
 
 static int ssd_lg_rank(int R) { return R == 1 ? 0 : (R == 2 ? 1 : (R == 4 ? 2 : -1)); }
+// (token, rank) rows per token: the wider of the two ranks
+static int ssd_rows_per_token(const Params &p) { return p.R > p.O ? p.R : p.O; }
 
-// Tokens per chunk of the scalar-decay kernels (128 (token, rank) rows).
+// Tokens per chunk of the scalar-decay kernels (128 (token, rank) rows); R here and
+// below is the rows per token, max(R, O).
 // Segments of the forward: about eight work items per resident CTA, at most one
 // 32 KB carry slot per CTA.
 constexpr int SSD_GRID_MAX = 296;
@@ -1593,7 +1609,7 @@ bool ssd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ptr == nullptr || ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
     return p.bf16 && !p.per_coord && p.np == 0 && p.P == 64 && (p.N == 64 || p.N == 128) &&
-           p.R == p.O && ssd_lg_rank(p.R) >= 0 && p.L > 0 && al16(p.x) && al16(p.Bm) &&
+           ssd_lg_rank(p.R) >= 0 && ssd_lg_rank(p.O) >= 0 && p.L > 0 && al16(p.x) && al16(p.Bm) &&
            al16(p.Cm) && al16(p.y) && st16(p.sx[0]) && st16(p.sx[1]) && st16(p.sx[2]) &&
            st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]) && st16(p.sB[0]) && st16(p.sB[1]) &&
            st16(p.sB[2]) && st16(p.sC[0]) && st16(p.sC[1]) && st16(p.sC[2]) &&
@@ -1616,16 +1632,16 @@ static cudaError_t ssd_set_smem(K kern, uint32_t bytes, bool (&done)[64]) {
 // backward.  Needs p.ws_ring, p.ws_flag and p.nc = chunks of ssd_chunk_tokens.
 cudaError_t ssd_forward(const Params &p, cudaStream_t st) {
     using namespace ssdk;
-    const int lgR = ssd_lg_rank(p.R);
+    const int Rp = ssd_rows_per_token(p), lgR = ssd_lg_rank(Rp);
     const uint32_t Qt = (uint32_t)(ROWS >> lgR);
     CUtensorMap mx, mb, mc, my;
-    if (!make_map5(&mx, p.x, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
-        !make_map5(&mb, p.Bm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
-        !make_map5(&mc, p.Cm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt))
+    if (!make_map5(&mx, p.x, 64, p.R, Rp, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
+        !make_map5(&mb, p.Bm, p.N, p.R, Rp, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+        !make_map5(&mc, p.Cm, p.N, p.O, Rp, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt))
         return cudaErrorInvalidValue;
     my = mx;
     if (p.y &&
-        !make_map5(&my, p.y, 64, p.O, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt))
+        !make_map5(&my, p.y, 64, p.O, Rp, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
     static bool done[64] = {}, done_s[64] = {};
@@ -1638,7 +1654,7 @@ cudaError_t ssd_forward(const Params &p, cudaStream_t st) {
     // segment buffers after the adjoint slots (see ssd_ring_bytes)
     Params q = p;
     const size_t bh = (size_t)p.Bsz * p.H, slot = 128 * 64 * 4;
-    q.sd_G = ssd_seg_chunks(p.Bsz, p.H, p.L, p.R);
+    q.sd_G = ssd_seg_chunks(p.Bsz, p.H, p.L, Rp);
     q.sd_nseg = (p.nc + q.sd_G - 1) / q.sd_G;
     char *base = reinterpret_cast<char *>(p.ws_ring) + al256(2 * bh * slot);
     q.sd_seg = reinterpret_cast<float *>(base);
@@ -1676,20 +1692,20 @@ cudaError_t ssd_backward(const Params &p, cudaStream_t st) {
         pf.wT = nullptr;
         if ((e = ssd_forward(pf, st)) != cudaSuccess) return e;
     }
-    const int lgR = ssd_lg_rank(p.R);
+    const int Rp = ssd_rows_per_token(p), lgR = ssd_lg_rank(Rp);
     const uint32_t Qt = (uint32_t)(ROWS >> lgR);
     CUtensorMap mx, mdy, mb, mc, mdx, mdb, mdc;
-    if (!make_map5(&mx, p.x, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
-        !make_map5(&mdy, p.dy, 64, p.O, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt) ||
-        !make_map5(&mb, p.Bm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
-        !make_map5(&mc, p.Cm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt) ||
-        !make_map5(&mdx, p.dx, 64, p.R, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt))
+    if (!make_map5(&mx, p.x, 64, p.R, Rp, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt) ||
+        !make_map5(&mdy, p.dy, 64, p.O, Rp, p.H, p.L, p.Bsz, p.P, p.sy[2], p.sy[1], p.sy[0], Qt) ||
+        !make_map5(&mb, p.Bm, p.N, p.R, Rp, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+        !make_map5(&mc, p.Cm, p.N, p.O, Rp, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt) ||
+        !make_map5(&mdx, p.dx, 64, p.R, Rp, p.H, p.L, p.Bsz, p.P, p.sx[2], p.sx[1], p.sx[0], Qt))
         return cudaErrorInvalidValue;
     mdb = mb;
     mdc = mc;
     if (p.hpg == 1 &&
-        (!make_map5(&mdb, p.dBm, p.N, p.R, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
-         !make_map5(&mdc, p.dCm, p.N, p.O, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt)))
+        (!make_map5(&mdb, p.dBm, p.N, p.R, Rp, p.G, p.L, p.Bsz, p.N, p.sB[2], p.sB[1], p.sB[0], Qt) ||
+         !make_map5(&mdc, p.dCm, p.N, p.O, Rp, p.G, p.L, p.Bsz, p.N, p.sC[2], p.sC[1], p.sC[0], Qt)))
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag || !p.ws_kp || !p.sd_tok || !p.sd_par || !p.sd_db0 ||
         (p.hpg != 1 && (!p.sd_dBh || !p.sd_dCh)))
@@ -1715,7 +1731,7 @@ cudaError_t ssd_backward(const Params &p, cudaStream_t st) {
     profile_mark(st, "k_ssd_tokens");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.hpg != 1) {
-        const long long tg = (long long)p.Bsz * p.L * p.G * p.R * p.N;
+        const long long tg = (long long)p.Bsz * p.L * p.G * Rp * p.N;
         int gb = (int)((tg + 255) / 256);
         if (gb > 148 * 16) gb = 148 * 16;
         k_ssd_group_sum<<<gb, 256, 0, st>>>(p);

@@ -35,7 +35,7 @@ def ssd_eligible(shape):
     """Shapes the scalar-decay (per-head) tensor-core kernels take."""
     return (shape.dtype_io == S.DTYPE_BF16 and shape.decay_mode == S.DECAY_PER_HEAD
             and shape.n_pairs == 0 and shape.headdim == 64 and shape.nstate in (64, 128)
-            and shape.rank_in == shape.rank_out and shape.rank_in in (1, 2, 4)
+            and shape.rank_in in (1, 2, 4) and shape.rank_out in (1, 2, 4)
             and shape.seqlen > 0 and shape.chunk != 1)
 
 
@@ -218,6 +218,25 @@ def test_zoh_write(kw):
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=95, with_state=True)
     check_all(shape, inp, route=abi.ROUTE_RECURRENT)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(rank_in=1, rank_out=2),
+    dict(rank_in=2, rank_out=1, ngroups=2),                   # two heads per group
+    dict(rank_in=1, rank_out=4),
+    dict(rank_in=4, rank_out=1, ngroups=2),
+    dict(rank_in=2, rank_out=4, two_endpoint=1, ngroups=2),
+    dict(rank_in=4, rank_out=2, n_real=64, seqlen=97),         # 64 state rows
+])
+def test_scalar_decay_unequal_ranks(kw):
+    """SSD-MIMO with R source and O != R target rows per token on the scalar-decay
+    tensor-core chain (chunks of 128 / max(R, O) tokens; the narrower side's rank
+    rows are zero-filled on load and dropped on store): every output against the
+    oracle, with groups of one head and of two."""
+    base = S.WORKLOADS["ssd_mimo_r4"].replace(batch=2, seqlen=150, nheads=4, ngroups=4)
+    shape = base.replace(**kw)
+    inp = S.make_inputs(shape, seed=97, with_state=True)
+    check_all(shape, inp, route=abi.ROUTE_SSD)
 
 
 @pytest.mark.parametrize("name", S.WORKLOAD_ORDER)
