@@ -219,7 +219,7 @@ bool tensor_chain_shape(const ssm_desc_t *d) {
     const int N = d->n_real + 2 * d->n_pairs;
     return d->dtype_io == SSM_BF16 && d->headdim == 64 && d->rank_in == 1 && d->rank_out == 1 &&
            (N == 64 || N == 128) && d->n_real % 8 == 0 && d->chunk != 1 && d->seqlen > 0 &&
-           d->n_static == 0 && d->discretization == SSM_DISC_EULER;
+           d->n_static == 0;
 }
 
 // Shapes of the scalar-decay (per-head) tensor-core chain: Mamba-2 SISO and

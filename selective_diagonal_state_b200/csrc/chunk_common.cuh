@@ -5,6 +5,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "umma.cuh"
 
@@ -217,6 +219,39 @@ __device__ __forceinline__ void pair_sincos(float ang, float *sn, float *cs) {
         sincos_red(ang, sn, cs);   // per-token angles can be any size
     else
         __sincosf(ang, sn, cs);
+}
+
+// Exact zero-order-hold write (ZOH): the write of chunk token t on mode m is
+// scaled by Z = dt phi1(dt a + i phi), phi1(z) = (e^z - 1) / z, in place of sigma_t
+// (the Euler form's dt), phi the token's rotation angle on a pair (dt theta_j, or
+// the token's own angle with per-token angles) and 0 on a real row.  Tokens past
+// the sequence end have dt = 0 and so Z = 0.
+__device__ __forceinline__ float zoh_real(const float *f32, int m, int t) {
+    const float dv = f32[F_DT + t];
+    float f1r, f1i, fdr, fdi;
+    zoh_phi(dv * f32[F_A2 + m] * 0.6931471805599453f, 0.f, f1r, f1i, fdr, fdi);
+    return dv * f1r;
+}
+// the token's own rotation angle on pair j (m its mode, w its frequency)
+template <bool TOK>
+__device__ __forceinline__ float tok_angle(const float *f32, int j, float w, int t) {
+    if constexpr (TOK)
+        return th_at(f32, j, t) - th_at(f32, j, t - 1);
+    else
+        return f32[F_DT + t] * w;
+}
+// (b0 + i b1) <- Z (b0 + i b1) on pair j of mode m
+template <bool TOK>
+__device__ __forceinline__ void zoh_pair(const float *f32, int m, int j, int t, float &b0,
+                                         float &b1) {
+    const float dv = f32[F_DT + t];
+    float f1r, f1i, fdr, fdi;
+    zoh_phi(dv * f32[F_A2 + m] * 0.6931471805599453f, tok_angle<TOK>(f32, j, f32[F_W + m], t), f1r,
+            f1i, fdr, fdi);
+    const float zr = dv * f1r, zi = dv * f1i;
+    const float r = fmaf(zr, b0, -zi * b1);
+    b1 = fmaf(zi, b0, zr * b1);
+    b0 = r;
 }
 
 // Per-mode decay over each sub-block, E_k = e^{lam dS_k}, the products
@@ -505,6 +540,17 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t 
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Host: calls fn(tok, zoh) with std::integral_constant<bool, ...> arguments for the
+// call's angle mode (per-token angles) and write form (ZOH), so that each kernel
+// runs the instantiation compiled for them.
+template <typename Fn>
+static cudaError_t by_variant(const Params &p, Fn &&fn) {
+    using T = std::true_type;
+    using F = std::false_type;
+    if (p.angle_tok) return p.zoh ? fn(T{}, T{}) : fn(T{}, F{});
+    return p.zoh ? fn(F{}, T{}) : fn(F{}, F{});
 }
 
 }  // namespace chunkc

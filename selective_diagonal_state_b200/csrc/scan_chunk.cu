@@ -69,7 +69,7 @@ template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_T
 template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
 }  // namespace stl
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 __global__ void __launch_bounds__(stl::THREADS)
 k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                     Params p) {
@@ -122,7 +122,8 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const int ib = t >> 4;
         const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
         const float ds = f32[F_S + t] - Sb;
-        const float sig = f32[F_SIG + t];
+        // the write's scale: sigma_t, or per mode Z (ZOH, applied to b below)
+        const float sig = ZOH ? 1.f : f32[F_SIG + t];
         const unsigned char *sB = sm + stl::SM_B;
         unsigned char *sv = p.sv_Bh ? p.sv_Bh + bhc(p, b, h, c) * 16384 : nullptr;
 #pragma unroll 1
@@ -139,6 +140,15 @@ k_chunk_state_local(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
                 const int r = r0 + j;
+                if constexpr (ZOH) {
+                    if (r < nr) {
+                        rb[j] *= zoh_real(f32, r, t);
+                        rb[j + 1] *= zoh_real(f32, r + 1, t);
+                    } else {
+                        const int m = nr + ((r - nr) >> 1);
+                        zoh_pair<TOK>(f32, m, m - nr, t, rb[j], rb[j + 1]);
+                    }
+                }
                 if (r < nr) {
                     v[j] = sig * rb[j] * ex2_fast(fminf(-f32[F_A2 + r] * ds, 120.f)) *
                            f32[F_KRE + fslot(ib, 4) * NP + r];
@@ -412,7 +422,7 @@ __device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int
     }
 }
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 __global__ void __launch_bounds__(fwk::THREADS, 1)
 k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -547,7 +557,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             const int ib = t >> 4;
             const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
             const float ds = f32[F_S + t] - Sb;
-            const float sig = f32[F_SIG + t];
+            // the write's scale: sigma_t, or per mode Z (ZOH, applied to b below)
+            const float sig = ZOH ? 1.f : f32[F_SIG + t];
             unsigned char *sv = p.sv_Bh ? p.sv_Bh + bhc(p, b, h, c) * 16384 : nullptr;
             float corr = 0.f;
 #pragma unroll 1
@@ -567,8 +578,17 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                     const int r = r0 + j;
                     // two rows at a time: real rows r, r+1 or one pair (re, im)
                     const float c0 = rc[j], c1 = rc[j + 1];
-                    const float b0 = rb[j], b1 = rb[j + 1];
+                    float b0 = rb[j], b1 = rb[j + 1];
                     corr = fmaf(c0, b0, fmaf(c1, b1, corr));
+                    if constexpr (ZOH) {
+                        if (r < nr) {
+                            b0 *= zoh_real(f32, r, t);
+                            b1 *= zoh_real(f32, r + 1, t);
+                        } else {
+                            const int m = nr + ((r - nr) >> 1);
+                            zoh_pair<TOK>(f32, m, m - nr, t, b0, b1);
+                        }
+                    }
                     if (r < nr) {
                         const int m0 = r, m1 = r + 1;
                         const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
@@ -942,7 +962,7 @@ bool chunk_fwd_supported(const Params &p) {
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
     // y (forward) leaves by TMA stores
     const bool yok = !p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]));
-    return yok && !p.nst && !p.zoh && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
+    return yok && !p.nst && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
            (p.N == 64 || p.N == 128) &&
            p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
            st16(p.sx[1]) && st16(p.sx[2]) && st16(p.sB[0]) && st16(p.sB[1]) && st16(p.sB[2]) &&
@@ -987,32 +1007,30 @@ static cudaError_t set_smem_once(K kern, uint32_t bytes, bool (&done)[64]) {
     return e;
 }
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 static cudaError_t launch_state_local(const CUtensorMap &mx, const CUtensorMap &mb, const Params &p,
                                       cudaStream_t st) {
     using namespace chunkfwd;
     static bool done[64] = {};
     cudaError_t e;
-    if ((e = set_smem_once(k_chunk_state_local<TOK>, stl::smem_bytes<TOK>(), done)) != cudaSuccess)
+    if ((e = set_smem_once(k_chunk_state_local<TOK, ZOH>, stl::smem_bytes<TOK>(), done)) !=
+        cudaSuccess)
         return e;
-    k_chunk_state_local<TOK>
+    k_chunk_state_local<TOK, ZOH>
         <<<dim3(p.nc, p.H, p.Bsz), stl::THREADS, stl::smem_bytes<TOK>(), st>>>(mx, mb, p);
     return cudaSuccess;
 }
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 static cudaError_t launch_fwd(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc,
                               const CUtensorMap &my, const Params &p, int grid, cudaStream_t st) {
     using namespace chunkfwd;
-    k_chunk_fwd<TOK><<<grid, fwk::THREADS, fwk::smem_bytes<TOK>(), st>>>(mx, mb, mc, my, p);
-    return cudaSuccess;
-}
-
-template <bool TOK>
-static cudaError_t fwd_smem(const Params &p) {
-    using namespace chunkfwd;
     static bool done[64] = {};
-    return set_smem_once(k_chunk_fwd<TOK>, fwk::smem_bytes<TOK>(), done);
+    cudaError_t e;
+    if ((e = set_smem_once(k_chunk_fwd<TOK, ZOH>, fwk::smem_bytes<TOK>(), done)) != cudaSuccess)
+        return e;
+    k_chunk_fwd<TOK, ZOH><<<grid, fwk::THREADS, fwk::smem_bytes<TOK>(), st>>>(mx, mb, mc, my, p);
+    return cudaSuccess;
 }
 
 // The state entering every chunk (p.ws_kp) and the chunk decays (p.ws_ce);
@@ -1023,8 +1041,10 @@ cudaError_t chunk_states(const Params &p, cudaStream_t st) {
     if (!make_map(&mx, p.x, PD, p.H, p.L, p.Bsz, p.sx[2], p.sx[1], p.sx[0], PD, true) ||
         !make_map(&mb, p.Bm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true))
         return cudaErrorInvalidValue;
-    cudaError_t e = p.angle_tok ? launch_state_local<true>(mx, mb, p, st)
-                                : launch_state_local<false>(mx, mb, p, st);
+    // one instantiation per angle mode and write form
+    cudaError_t e = by_variant(p, [&](auto tok, auto zoh) {
+        return launch_state_local<decltype(tok)::value, decltype(zoh)::value>(mx, mb, p, st);
+    });
     if (e != cudaSuccess) return e;
     profile_mark(st, "k_chunk_state_local");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1042,7 +1062,6 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
     cudaError_t e;
-    if ((e = p.angle_tok ? fwd_smem<true>(p) : fwd_smem<false>(p)) != cudaSuccess) return e;
     // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
@@ -1052,10 +1071,11 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
     CUtensorMap my;
     if (!make_map(&my, p.y, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
-    if (p.angle_tok)
-        launch_fwd<true>(mx, mb, mc, my, p, grid, st);
-    else
-        launch_fwd<false>(mx, mb, mc, my, p, grid, st);
+    if ((e = by_variant(p, [&](auto tok, auto zoh) {
+             return launch_fwd<decltype(tok)::value, decltype(zoh)::value>(mx, mb, mc, my, p, grid,
+                                                                            st);
+         })) != cudaSuccess)
+        return e;
     profile_mark(st, "k_chunk_fwd");
     return cudaGetLastError();
 }

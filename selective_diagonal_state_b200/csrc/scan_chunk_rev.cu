@@ -64,7 +64,7 @@ template <bool TOK> constexpr uint32_t sm_bar() { return SM_F32 + (TOK ? F_END_T
 template <bool TOK> constexpr uint32_t smem_bytes() { return sm_bar<TOK>() + 64 + 1024; }
 }  // namespace dxk
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 __global__ void __launch_bounds__(dxk::THREADS, 1)
 k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                const __grid_constant__ CUtensorMap tmDY, Params p) {
@@ -124,7 +124,8 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
             const int ib = t >> 4;
             const float Sb = ib == 0 ? 0.f : f32[F_S + 16 * ib - 1];
             const float ds = f32[F_S + t] - Sb;
-            const float sig = f32[F_SIG + t];
+            // the write's scale: sigma_t, or per mode Z (ZOH, applied to b below)
+            const float sig = ZOH ? 1.f : f32[F_SIG + t];
             const unsigned char *sB = sm + dxk::SM_B, *sC = sm + dxk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
@@ -138,8 +139,17 @@ k_chunk_bwd_dx(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ 
                 for (int j = 0; j < 8; j += 2) {
                     const int r = r0 + j;
                     const float c0 = rc[j], c1 = rc[j + 1];
-                    const float b0 = rb[j], b1 = rb[j + 1];
+                    float b0 = rb[j], b1 = rb[j + 1];
                     corr = fmaf(c0, b0, fmaf(c1, b1, corr));
+                    if constexpr (ZOH) {
+                        if (r < nr) {
+                            b0 *= zoh_real(f32, r, t);
+                            b1 *= zoh_real(f32, r + 1, t);
+                        } else {
+                            const int m = nr + ((r - nr) >> 1);
+                            zoh_pair<TOK>(f32, m, m - nr, t, b0, b1);
+                        }
+                    }
                     if (r < nr) {
                         const int m0 = r, m1 = r + 1;
                         const float x0 = f32[F_A2 + m0] * ds, x1 = f32[F_A2 + m1] * ds;
@@ -492,7 +502,7 @@ __device__ __forceinline__ uint32_t e_col(int j, int k) {   // k >= j
     return 352u + 16u * (uint32_t)((j == 0 ? 0 : (j == 1 ? 4 : (j == 2 ? 7 : 9))) + (k - j));
 }
 
-template <bool TOK>
+template <bool TOK, bool ZOH>
 __global__ void __launch_bounds__(fuk::THREADS, 1)
 k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmDY,
@@ -614,7 +624,8 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const float St = f32[F_S + t];
             const float dsb = St - (kb == 0 ? 0.f : f32[F_S + 16 * kb - 1]);   // >= 0
             const float dse = St - f32[F_S + 16 * kb + 15];                     // <= 0
-            const float sig = f32[F_SIG + t];
+            // the write's scale: sigma_t, or per mode Z (ZOH, applied to b below)
+            const float sig = ZOH ? 1.f : f32[F_SIG + t];
             const unsigned char *sB = sm + fuk::SM_B, *sC = sm + fuk::SM_C;
             float corr = 0.f;
 #pragma unroll 1
@@ -628,6 +639,15 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 for (int j = 0; j < 8; j += 2) {
                     const int r = r0 + j;
                     corr = fmaf(rc[j], rb[j], fmaf(rc[j + 1], rb[j + 1], corr));
+                    if constexpr (ZOH) {
+                        if (r < nr) {
+                            rb[j] *= zoh_real(f32, r, t);
+                            rb[j + 1] *= zoh_real(f32, r + 1, t);
+                        } else {
+                            const int m = nr + ((r - nr) >> 1);
+                            zoh_pair<TOK>(f32, m, m - nr, t, rb[j], rb[j + 1]);
+                        }
+                    }
                     if (r < nr) {
                         const float a0 = f32[F_A2 + r], a1 = f32[F_A2 + r + 1];
                         vb[j] = sig * rb[j] * ex2_fast(fminf(-a0 * dsb, 120.f));
@@ -1103,10 +1123,48 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 const float bt = ld_row1(sB, t, n), ct = ld_row1(sC, t, n);
                 const float k_ = kk[j];                          // dCK_t
                 const float dCt = fmaf(-bn * m2, bt, k_);        // dC_t
-                const float gg = sig * res;
                 const float co = __shfl_xor_sync(0xffffffffu, ct, 1);
                 const float ko = __shfl_xor_sync(0xffffffffu, k_, 1);
                 const float bo = __shfl_xor_sync(0xffffffffu, bt, 1);
+                // gg: the write's adjoint scale applied to gbu (sigma_t, or conj(Z) per mode)
+                float gg, zd = 0.f, zw = 0.f;
+                if constexpr (ZOH) {
+                    // Z = dt phi1(mu), mu = dt a + i phi; the pair's (re, im) of gbu and b
+                    const float ro = __shfl_xor_sync(0xffffffffu, res, 1);
+                    const float g_r = im_row ? ro : res, g_i = im_row ? res : ro;
+                    const float b_r = im_row ? bo : bt, b_i = im_row ? bt : bo;
+                    const float an = a2 * 0.6931471805599453f;
+                    const float ph = pr_row ? tok_angle<TOK>(f32, jp, w, t) : 0.f;
+                    float f1r, f1i, fdr, fdi;
+                    zoh_phi(dtv * an, ph, f1r, f1i, fdr, fdi);
+                    const float zr = dtv * f1r, zi = dtv * f1i;
+                    gg = !pr_row ? zr * res : (im_row ? fmaf(-zi, g_r, zr * g_i) : fmaf(zr, g_r, zi * g_i));
+                    // dL/dZ = (Re s, -Im s), s = b conj(gbu); it reaches dt through
+                    // dZ/d dt, a through dt^2 phi1' and the angle through i dt^2 phi1'
+                    // (i dt phi1' for a per-token angle)
+                    const float gzr = pr_row ? fmaf(b_r, g_r, b_i * g_i) : bt * res;
+                    const float gzi = pr_row ? fmaf(b_r, g_i, -b_i * g_r) : 0.f;
+                    float zdr, zdi;
+                    if (TOK && pr_row) {
+                        zdr = fmaf(dtv * an, fdr, f1r);
+                        zdi = fmaf(dtv * an, fdi, f1i);
+                    } else {
+                        float sn, cs;
+                        sincosf(ph, &sn, &cs);
+                        const float ex = expf(dtv * an);
+                        zdr = ex * cs;
+                        zdi = ex * sn;
+                    }
+                    if (tv && !im_row) {   // once per mode: a real row or a pair's re row
+                        zd = fmaf(gzr, zdr, gzi * zdi);
+                        dacc = fmaf(dtv * dtv, fmaf(gzr, fdr, gzi * fdi), dacc);
+                    } else if (tv) {
+                        zw = (TOK ? dtv : dtv * dtv) * fmaf(-gzr, fdi, gzi * fdr);
+                        if (!TOK) dacc += zw;   // the pair's angle-gradient partial
+                    }
+                } else {
+                    gg = sig * res;
+                }
                 const float go = __shfl_xor_sync(0xffffffffu, gg, 1);
                 float v;
                 if (!pr_row)
@@ -1119,7 +1177,8 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 cum += v;
                 dacc = fmaf(dtv, im_row ? -cum : cum, dacc);
                 sdt += dtv;
-                red2[n * fuk::RED_LD + t] = coef * cum;
+                // ddt terms; with a per-token angle the im row's entry is the angle's gradient
+                red2[n * fuk::RED_LD + t] = coef * cum + (ZOH ? (im_row ? (TOK ? zw : 0.f) : zd) : 0.f);
                 red[n * fuk::RED_LD + t] = tv ? res * bt : 0.f;
                 if (one_head) {
                     // dB / dC replace the (t, n) element of the raw B / C tiles that only this
@@ -1282,14 +1341,14 @@ static cudaError_t set_smem(K kern, uint32_t bytes, bool (&done)[64]) {
 cudaError_t chunk_states(const Params &p, cudaStream_t st);
 int sm_count();
 
-// Shared memory opt-in of the dx and fused kernels of one angle mode.
-template <bool TOK>
+// Shared memory opt-in of the dx and fused kernels of one angle mode and write form.
+template <bool TOK, bool ZOH>
 static cudaError_t rev_smem() {
     using namespace chunkrev;
     static bool a3[64] = {}, a4[64] = {};
     cudaError_t e;
-    if ((e = set_smem(k_chunk_bwd_dx<TOK>, dxk::smem_bytes<TOK>(), a3)) != cudaSuccess) return e;
-    return set_smem(k_chunk_bwd_fused<TOK>, fuk::smem_bytes<TOK>(), a4);
+    if ((e = set_smem(k_chunk_bwd_dx<TOK, ZOH>, dxk::smem_bytes<TOK>(), a3)) != cudaSuccess) return e;
+    return set_smem(k_chunk_bwd_fused<TOK, ZOH>, fuk::smem_bytes<TOK>(), a4);
 }
 
 // The state entering every chunk for the tensor-core backward (p.ws_kp,
@@ -1312,7 +1371,10 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     if (!p.ws_ring || !p.ws_flag) return cudaErrorInvalidValue;
     cudaError_t e;
-    if ((e = p.angle_tok ? rev_smem<true>() : rev_smem<false>()) != cudaSuccess) return e;
+    if ((e = by_variant(p, [&](auto tok, auto zoh) {
+             return rev_smem<decltype(tok)::value, decltype(zoh)::value>();
+         })) != cudaSuccess)
+        return e;
     // the per-(b, h) carry counters, the ticket and the abort word start at zero on every call
     if ((e = cudaMemsetAsync(p.ws_flag, 0, sizeof(int) * ((size_t)p.Bsz * p.H + 2), st)) !=
         cudaSuccess)
@@ -1326,12 +1388,12 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
             (!make_map(&mdb, p.dBm, p.N, p.G, p.L, p.Bsz, p.sB[2], p.sB[1], p.sB[0], 64, true) ||
              !make_map(&mdc, p.dCm, p.N, p.G, p.L, p.Bsz, p.sC[2], p.sC[1], p.sC[0], 64, true)))
             return cudaErrorInvalidValue;
-        if (p.angle_tok)
-            k_chunk_bwd_fused<true>
-                <<<pgrid, fuk::THREADS, fuk::smem_bytes<true>(), st>>>(mx, mb, mc, mdy, mdb, mdc, p);
-        else
-            k_chunk_bwd_fused<false>
-                <<<pgrid, fuk::THREADS, fuk::smem_bytes<false>(), st>>>(mx, mb, mc, mdy, mdb, mdc, p);
+        by_variant(p, [&](auto tok, auto zoh) {
+            constexpr bool T = decltype(tok)::value, Z = decltype(zoh)::value;
+            k_chunk_bwd_fused<T, Z>
+                <<<pgrid, fuk::THREADS, fuk::smem_bytes<T>(), st>>>(mx, mb, mc, mdy, mdb, mdc, p);
+            return cudaSuccess;
+        });
     }
     profile_mark(st, "k_chunk_bwd_fused");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1343,10 +1405,11 @@ cudaError_t chunk_bwd_reverse(const Params &p, cudaStream_t st) {
         k_chunk_bwd_dx_saved<<<grid, dxs::THREADS, dxs::SMEM_BYTES, st>>>(mdy, p);
         profile_mark(st, "k_chunk_bwd_dx_saved");
     } else {
-        if (p.angle_tok)
-            k_chunk_bwd_dx<true><<<grid, dxk::THREADS, dxk::smem_bytes<true>(), st>>>(mb, mc, mdy, p);
-        else
-            k_chunk_bwd_dx<false><<<grid, dxk::THREADS, dxk::smem_bytes<false>(), st>>>(mb, mc, mdy, p);
+        by_variant(p, [&](auto tok, auto zoh) {
+            constexpr bool T = decltype(tok)::value, Z = decltype(zoh)::value;
+            k_chunk_bwd_dx<T, Z><<<grid, dxk::THREADS, dxk::smem_bytes<T>(), st>>>(mb, mc, mdy, p);
+            return cudaSuccess;
+        });
         profile_mark(st, "k_chunk_bwd_dx");
     }
     return cudaGetLastError();

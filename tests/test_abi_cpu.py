@@ -68,7 +68,10 @@ def test_angle_mode_validation(lib):
     assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0
     assert b"ZOH" in lib.ssm_scan_last_error()
     d.two_endpoint = 0
-    assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0   # recurrent kernels: no workspace
+    # the ZOH write takes the tensor-core chain: the same workspace as the Euler form
+    zoh_ws = abi.ssm_scan_workspace_size(d, abi.PASS_FWD)
+    d.discretization = 0
+    assert zoh_ws == abi.ssm_scan_workspace_size(d, abi.PASS_FWD) > 0
     d.discretization = 0
     d.reserved_ = 1
     assert abi.ssm_scan_workspace_size(d, abi.PASS_FWD) == 0

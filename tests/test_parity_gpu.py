@@ -27,8 +27,7 @@ def chunk_eligible(shape):
     """Shapes the per-coordinate tensor-core kernels take."""
     return (shape.dtype_io == S.DTYPE_BF16 and shape.headdim == 64 and shape.rank_in == 1
             and shape.rank_out == 1 and shape.nstate in (64, 128) and shape.n_real % 8 == 0
-            and shape.seqlen > 0 and shape.chunk != 1
-            and shape.n_static == 0 and shape.discretization == S.DISC_EULER)
+            and shape.seqlen > 0 and shape.chunk != 1 and shape.n_static == 0)
 
 
 def ssd_eligible(shape):
@@ -36,7 +35,8 @@ def ssd_eligible(shape):
     return (shape.dtype_io == S.DTYPE_BF16 and shape.decay_mode == S.DECAY_PER_HEAD
             and shape.n_pairs == 0 and shape.headdim == 64 and shape.nstate in (64, 128)
             and shape.rank_in in (1, 2, 4) and shape.rank_out in (1, 2, 4)
-            and shape.seqlen > 0 and shape.chunk != 1)
+            and shape.seqlen > 0 and shape.chunk != 1
+            and shape.n_static == 0 and shape.discretization == S.DISC_EULER)
 
 
 def channel_eligible(shape):
@@ -204,7 +204,7 @@ def test_static_rows(kw):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(),                                   # HybridMamba heads, Euler form, bf16
+    dict(),                                   # HybridMamba heads (Euler write off), bf16
     dict(dtype_io=S.DTYPE_F32),
     dict(angle_mode=S.ANGLE_PER_TOKEN),
     dict(decay_mode=S.DECAY_PER_HEAD, n_real=128, n_pairs=0, ngroups=2),
@@ -212,12 +212,14 @@ def test_static_rows(kw):
 ])
 def test_zoh_write(kw):
     """Exact zero-order-hold write ((e^{dt lam} - 1) / lam per mode, complex on a
-    rotation pair) against the oracle, forward and backward."""
+    rotation pair) against the oracle, forward and backward: on the per-coordinate
+    tensor-core chain for bf16 heads of 64 channels, on the recurrent kernels
+    otherwise."""
     base = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=4, ngroups=4, seqlen=150,
                                               two_endpoint=0, discretization=S.DISC_ZOH)
     shape = base.replace(**kw)
     inp = S.make_inputs(shape, seed=95, with_state=True)
-    check_all(shape, inp, route=abi.ROUTE_RECURRENT)
+    check_all(shape, inp)
 
 
 @pytest.mark.parametrize("kw", [
@@ -438,7 +440,10 @@ def test_moderate_decay_stays_chunked():
 @pytest.mark.parametrize("kw", [dict(), dict(seqlen=64), dict(seqlen=1),
                                 dict(decay_mode=S.DECAY_PER_HEAD, two_endpoint=0, n_real=128,
                                      n_pairs=0, ngroups=2),
-                                dict(angle_mode=S.ANGLE_PER_TOKEN)])
+                                dict(angle_mode=S.ANGLE_PER_TOKEN),
+                                dict(two_endpoint=0, discretization=S.DISC_ZOH),
+                                dict(two_endpoint=0, discretization=S.DISC_ZOH,
+                                     angle_mode=S.ANGLE_PER_TOKEN, ngroups=2)])
 def test_backward_from_saved_states(kw):
     """The backward that reads the forward's chunk states gives the same
     gradients as the one that recomputes them, and the oracle's.  Everything but
