@@ -50,7 +50,24 @@ def parse():
                     help="target wall time of the bounded oracle sample")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the batch size (small cases for profiling only)")
+    ap.add_argument("--variant", default="none", choices=sorted(VARIANTS),
+                    help="a variant of the workload's scan (per-token angles, ZOH write, ...)")
+    ap.add_argument("--op", default="scan", choices=["scan", "preact", "step"],
+                    help="scan: forward + backward (the headline); preact: the dt / lambda "
+                         "pre-activations, forward + backward; step: one decoding step")
     return ap.parse_args()
+
+
+# Variants of a workload's scan (rows beyond the hot path): the descriptor fields
+# they change.
+VARIANTS = {
+    "none": {},
+    "per_token_angles": dict(angle_mode=S.ANGLE_PER_TOKEN),
+    "zoh": dict(two_endpoint=0, discretization=S.DISC_ZOH),
+    "static_rows": dict(n_static=16),
+    "rank_out_1": dict(rank_out=1),
+    "rank_out_2": dict(rank_out=2),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -60,6 +77,7 @@ def tensor_bytes(shape: S.ScanShape) -> dict:
     s = shape
     e = 2 if s.dtype_io == S.DTYPE_BF16 else 4
     BL = s.batch * s.seqlen
+    per_token = s.angle_mode == S.ANGLE_PER_TOKEN and s.n_pairs
     return {
         "x": BL * s.nheads * s.rank_in * s.headdim * e,
         "y": BL * s.nheads * s.rank_out * s.headdim * e,
@@ -67,18 +85,20 @@ def tensor_bytes(shape: S.ScanShape) -> dict:
         "C": BL * s.ngroups * s.rank_out * s.nstate * e,
         "dt": BL * s.nheads * e,
         "lam": BL * s.nheads * e if s.two_endpoint else 0,
+        # per-token rotation angles (fp32), read by both directions, their gradient written
+        "theta": BL * s.nheads * s.n_pairs * 4 if per_token else 0,
     }
 
 
 def fwd_bytes(shape):
     t = tensor_bytes(shape)
-    return t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["y"]
+    return t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["theta"] + t["y"]
 
 
 def bwd_bytes(shape):
     t = tensor_bytes(shape)
-    reads = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["y"]  # y-sized dy
-    writes = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
+    reads = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["theta"] + t["y"]  # y-sized dy
+    writes = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["theta"]
     return reads + writes
 
 
@@ -90,7 +110,7 @@ def kernel_bytes(shape, name: str) -> int:
     s = shape
     t = tensor_bytes(shape)
     BLH = s.batch * s.seqlen * s.nheads
-    ins = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"]
+    ins = t["x"] + t["B"] + t["C"] + t["dt"] + t["lam"] + t["theta"]
     dy = t["y"]
     if name in ("k_fwd", "k_chunk_fwd"):
         return ins + t["y"]
@@ -114,7 +134,7 @@ def kernel_bytes(shape, name: str) -> int:
         return dy + t["x"]
     if name == "k_chunk_bwd_fused":   # x, B, C, dt, lambda, dy -> dB, dC (one head per group)
         out = t["B"] + t["C"] if s.nheads == s.ngroups else 0
-        return ins + dy + out
+        return ins + dy + out + t["theta"]   # and the per-token angle gradient
     if name == "k_bwd_units_final":   # dt, lambda -> ddt, dlambda
         return 2 * (t["dt"] + t["lam"])
     # scalar-decay chain
@@ -307,7 +327,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    shape = S.WORKLOADS[args.workload]
+    shape = S.WORKLOADS[args.workload].replace(**VARIANTS[args.variant])
     per_step_target = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     units, L, cores = oracle_sample_plan(shape, per_step_target)
     for _ in range(args.warmup):
@@ -371,10 +391,164 @@ def roofline_of(shape, dom, ms_launch, peaks):
             "ms_per_launch": ms_launch, "peak_source": src}
 
 
+def _clock_index(local):
+    if "CUDA_VISIBLE_DEVICES" not in os.environ:
+        return local
+    return int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+
+
+def _peaks():
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    return json.load(open(pk)) if os.path.exists(pk) else {}
+
+
+def run_op(args, shape):
+    """--op preact | step: a row beyond the hot path on one GPU, timed like the
+    scan (CUDA events on the launching stream around K calls after W warm-up
+    calls, clocks sampled meanwhile, L2 flushed between calls when the data fit
+    in it) against the HBM roofline of its algorithmic bytes.
+
+    preact: ssm_preact_fwd + ssm_preact_bwd over the workload's (batch, L, heads):
+      reads z (and the lambda logits), writes dt (and lambda); then reads z,
+      ddt (and the logits, dlambda), writes dz (and dlambda_logit).
+    step:   one ssm_scan_step for a decoding batch (--batch, default 128 rows) of
+      the workload's heads: the fp32 state (and the previous write) read and
+      written once, one token's x, dt, lambda, B, C read and y written."""
+    import torch
+
+    from selective_diagonal_state_b200 import abi, scan
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--op preact / step run on one GPU")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    abi.load_library()
+    e = 2 if shape.dtype_io == S.DTYPE_BF16 else 4
+    two = bool(shape.two_endpoint)
+    dtype = scan.io_dtype(shape)
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    stream = torch.cuda.current_stream()
+    if args.op == "preact":
+        inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1, with_dy=False,
+                            with_raw=True)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dtype).cuda()  # noqa: E731
+        z, lg = dev(inp["z"]), dev(inp["lam_logit"])
+        bias = torch.from_numpy(inp["dt_bias"]).cuda()
+        dt, lam = torch.empty_like(z), torch.empty_like(lg)
+        ddt = torch.randn(z.shape, generator=gen, device="cuda").to(dtype)
+        dlam = torch.randn(z.shape, generator=gen, device="cuda").to(dtype)
+        dz, dlg = torch.empty_like(z), torch.empty_like(lg)
+        dbias = torch.empty(shape.nheads, dtype=torch.float32, device="cuda")
+        desc = abi.make_desc(shape)
+
+        def call():
+            abi.ssm_preact_fwd(desc, z, bias, lg if two else None, dt, lam if two else None)
+            abi.ssm_preact_bwd(desc, z, bias, lg if two else None, ddt, dlam if two else None,
+                               dz, dbias, dlg if two else None)
+
+        BLH = shape.batch * shape.seqlen * shape.nheads
+        nbytes = BLH * e * (5 + 5 * two)
+        tokens = shape.batch * shape.seqlen
+        launches = 2
+        cfg = {"batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads}
+        metric = "pre-activation (softplus dt, sigmoid lambda) fwd+bwd tokens/s"
+    else:
+        B = args.batch or 128
+        sh = shape.replace(batch=B, seqlen=1)
+        inp = S.make_inputs(sh, seed=S.WORKLOAD_ORDER.index(shape.name) + 1, with_dy=False,
+                            with_state=True)
+        d = scan.to_device(sh, inp)
+        desc = abi.make_desc(sh)
+        h = d.h0.clone()
+        w = d.w0.clone() if two else None
+        y = torch.empty((B, 1, sh.nheads, sh.rank_out, sh.headdim), dtype=dtype, device="cuda")
+        per_token = sh.angle_mode == S.ANGLE_PER_TOKEN and sh.n_pairs
+        th = d.theta[:, 0].contiguous() if per_token else d.theta
+
+        def call():
+            abi.ssm_scan_step(desc, d.x, d.dt, d.A_log, th, d.Bm, d.Cm, d.D,
+                              d.lam if two else None, h, w, y)
+
+        st = B * sh.nheads * sh.nstate * sh.headdim * 4
+        tb = tensor_bytes(sh)
+        nbytes = 2 * st * (2 if two else 1) + sum(tb.values())
+        tokens = B
+        launches = 1
+        cfg = {"batch": B, "nheads": sh.nheads, "state_bytes": st * (2 if two else 1)}
+        metric = "decode step tokens/s (one token per batch row and call)"
+    flush = nbytes < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    abi.ssm_scan_poll_device_error()
+    # per-kernel device times (events around each launch, in a separate pass)
+    abi.ssm_scan_profile_start(launches * args.steps)
+    for _ in range(args.steps):
+        call()
+    prof = abi.ssm_scan_profile_stop()
+    kernel_ms = {n: tot / max(1, c) for n, (c, tot) in prof.items()}
+    # the timed calls replay a CUDA graph of one call: these ops take microseconds,
+    # so launching them from Python would time the host instead of the device
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    torch.cuda.synchronize()
+    call = graph.replay
+    clocks = ClockSampler(_clock_index(int(os.environ.get("LOCAL_RANK", "0"))))
+    clocks.start()
+    time.sleep(0.3)
+    clocks.mark(True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps if flush else 1)]
+    if flush:
+        for a, b in evs:
+            scratch.fill_(1.0)
+            a.record(stream)
+            call()
+            b.record(stream)
+    else:
+        evs[0][0].record(stream)
+        for _ in range(args.steps):
+            call()
+        evs[0][1].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    abi.ssm_scan_poll_device_error()
+    peaks = _peaks()
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    ach = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": metric, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype_io == S.DTYPE_BF16 else "f32", "data": "synthetic",
+        "op": args.op,
+        "config": dict(cfg, workload=shape.name, variant=args.variant,
+                       l2=("data below twice L2: each call timed alone, L2 flushed between "
+                           "calls" if flush else "data larger than twice L2; no flush")),
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                     "frac": ach / hbm, "traffic": None, "algorithmic_bytes": nbytes,
+                     "peak_source": "measured" if peaks.get("hbm_gbs") else "fallback"},
+        "kernel_ms": kernel_ms,
+        "timing": "CUDA graph replays of one call, CUDA events on the stream",
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.op != "scan":
+        shape = S.WORKLOADS[args.workload].replace(**VARIANTS[args.variant])
+        if args.batch and args.op != "step":
+            shape = shape.replace(batch=args.batch)
+        run_op(args, shape)
         return
     import torch
     import torch.distributed as dist
@@ -393,7 +567,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     abi.load_library()
-    shape = S.WORKLOADS[args.workload]
+    shape = S.WORKLOADS[args.workload].replace(**VARIANTS[args.variant])
     if args.batch:
         shape = shape.replace(batch=args.batch)
     inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1000 * rank)
@@ -620,7 +794,8 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if shape.dtype_io == S.DTYPE_BF16 else "f32",
         "data": "synthetic",
-        "config": {"workload": shape.name, "batch_per_gpu": shape.batch, "seqlen": shape.seqlen,
+        "config": {"workload": shape.name, "variant": args.variant,
+                   "batch_per_gpu": shape.batch, "seqlen": shape.seqlen,
                    "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
                    "state": f"{shape.n_real} real + {shape.n_pairs} rotation pairs",
                    "rank_in": shape.rank_in, "rank_out": shape.rank_out,

@@ -283,7 +283,8 @@ SSM_API int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_b
 /*
  * Gradients through the pre-activations, from ddt and dlambda (as written by
  * ssm_scan_bwd):  dz = ddt * sigmoid(z + dt_bias),
- * ddt_bias[h] = sum over (b, t) of dz (fp32, written, fixed summation order),
+ * ddt_bias[h] = sum over (b, t) of the dz returned (in dtype_io; fp32 sum, written, fixed
+ * summation order),
  * dlambda_logit = dlambda * lambda (1 - lambda).  dz may alias ddt and
  * dlambda_logit may alias dlambda; ddt_bias may be NULL; the lambda pointers
  * may be NULL when two_endpoint == 0.

@@ -228,9 +228,9 @@ __device__ __forceinline__ void pair_sincos(float ang, float *sn, float *cs) {
 // the sequence end have dt = 0 and so Z = 0.
 __device__ __forceinline__ float zoh_real(const float *f32, int m, int t) {
     const float dv = f32[F_DT + t];
-    float f1r, f1i, fdr, fdi;
-    zoh_phi(dv * f32[F_A2 + m] * 0.6931471805599453f, 0.f, f1r, f1i, fdr, fdi);
-    return dv * f1r;
+    float f1, fd;
+    zoh_phi_real(dv * f32[F_A2 + m] * 0.6931471805599453f, f1, fd);
+    return dv * f1;
 }
 // the token's own rotation angle on pair j (m its mode, w its frequency)
 template <bool TOK>

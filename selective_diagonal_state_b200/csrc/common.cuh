@@ -232,6 +232,26 @@ __device__ __forceinline__ void zoh_phi(float mr, float mi, float &f1r, float &f
     fdi = (ni * mr - nr * mi) * d;
 }
 
+// The same for a real argument: phi1(m) and phi1'(m).
+__device__ __forceinline__ void zoh_phi_real(float m, float &f1, float &fd) {
+    if (m * m < 0.25f) {
+        float pw = 1.f, inv1 = 1.f, inv2 = 0.5f;
+        f1 = fd = 0.f;
+#pragma unroll
+        for (int k = 0; k < 12; ++k) {
+            f1 = fmaf(inv1, pw, f1);
+            fd = fmaf((k + 1) * inv2, pw, fd);
+            pw *= m;
+            inv1 *= 1.f / (float)(k + 2);
+            inv2 *= 1.f / (float)(k + 3);
+        }
+        return;
+    }
+    const float d = 1.f / m;
+    f1 = expm1f(m) * d;
+    fd = (expf(m) - f1) * d;
+}
+
 // Timing hook (defined in abi.cu): call right after every kernel launch with
 // the kernel's name.
 void profile_mark(cudaStream_t st, const char *name);

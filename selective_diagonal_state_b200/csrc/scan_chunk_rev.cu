@@ -1135,8 +1135,11 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const float b_r = im_row ? bo : bt, b_i = im_row ? bt : bo;
                     const float an = a2 * 0.6931471805599453f;
                     const float ph = pr_row ? tok_angle<TOK>(f32, jp, w, t) : 0.f;
-                    float f1r, f1i, fdr, fdi;
-                    zoh_phi(dtv * an, ph, f1r, f1i, fdr, fdi);
+                    float f1r, f1i = 0.f, fdr, fdi = 0.f;
+                    if (pr_row)   // (a warp holds rows of one kind: no divergence)
+                        zoh_phi(dtv * an, ph, f1r, f1i, fdr, fdi);
+                    else
+                        zoh_phi_real(dtv * an, f1r, fdr);
                     const float zr = dtv * f1r, zi = dtv * f1i;
                     gg = !pr_row ? zr * res : (im_row ? fmaf(-zi, g_r, zr * g_i) : fmaf(zr, g_r, zi * g_i));
                     // dL/dZ = (Re s, -Im s), s = b conj(gbu); it reaches dt through
@@ -1145,15 +1148,13 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const float gzr = pr_row ? fmaf(b_r, g_r, b_i * g_i) : bt * res;
                     const float gzi = pr_row ? fmaf(b_r, g_i, -b_i * g_r) : 0.f;
                     float zdr, zdi;
-                    if (TOK && pr_row) {
+                    if (TOK && pr_row) {   // phi1 + dt a phi1'
                         zdr = fmaf(dtv * an, fdr, f1r);
                         zdi = fmaf(dtv * an, fdi, f1i);
-                    } else {
-                        float sn, cs;
-                        sincosf(ph, &sn, &cs);
-                        const float ex = expf(dtv * an);
-                        zdr = ex * cs;
-                        zdi = ex * sn;
+                    } else {               // e^mu = 1 + mu phi1, mu = dt a + i phi
+                        const float mr = dtv * an;
+                        zdr = 1.f + fmaf(mr, f1r, -ph * f1i);
+                        zdi = fmaf(mr, f1i, ph * f1r);
                     }
                     if (tv && !im_row) {   // once per mode: a real row or a pair's re row
                         zd = fmaf(gzr, zdr, gzi * zdi);
@@ -1217,10 +1218,17 @@ k_chunk_bwd_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             for (int t = tc; t < tc + 16; ++t) red2[n * fuk::RED_LD + t] += add;
         }
         if (TOK && im_row) {
-            // dL/dtheta_t of this pair, the part from inside the chunk (the carry from
-            // later chunks is added by the block-carry pass); kept out of ddt
+            // dL/dtheta_t of this pair, kept out of ddt: the part from inside the chunk and
+            // the carry from later chunks, minus the imaginary part of the exact value at
+            // the chunk's end boundary (published with the adjoint this item waited for)
+            float cai = 0.f;
+            if (p.ws_qb && c + 1 < p.nc) {
+                const float *q = p.ws_qb + ((long long)bh * p.nc + c + 1) * 4 * (long long)N;
+#pragma unroll
+                for (int w2 = 0; w2 < 4; ++w2) cai += __ldcg(q + w2 * N + n);
+            }
             for (int t = tc; t < tc + 16; ++t) {
-                if (t0 + t < L) p.dtheta[ix_th(p, b, t0 + t, h, jp)] = red2[n * fuk::RED_LD + t];
+                if (t0 + t < L) p.dtheta[ix_th(p, b, t0 + t, h, jp)] = red2[n * fuk::RED_LD + t] - cai;
                 red2[n * fuk::RED_LD + t] = 0.f;
             }
         }

@@ -968,7 +968,8 @@ __global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
             dA += blk[4 * m + 2] + car * (stat ? ntok : sdt);
             if (mi.pair) dth += blk[4 * m + 3] - cai * sdt;
             contrib = stat ? 0.f : mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
-            if (mi.pair && p.angle_tok && cai != 0.f) {
+            // per-token angles: the chunked backward subtracts the exact carry itself
+            if (mi.pair && p.angle_tok && cai != 0.f && !p.ws_qb) {
                 const int tend = min(p.L, (tb + 1) * TBL);
                 for (int t = tb * TBL; t < tend; ++t)
                     p.dtheta[ix_th(p, b, t, h, m - p.nr)] -= cai;

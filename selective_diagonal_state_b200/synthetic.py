@@ -141,14 +141,17 @@ def _sigmoid(v):
 
 
 def make_inputs(shape: ScanShape, seed: int, with_dy: bool = True,
-                with_state: bool = False) -> dict:
+                with_state: bool = False, with_raw: bool = False) -> dict:
     """Draw every input of one scan (and the upstream gradient ``dy``).
 
     Returns float32 numpy arrays holding values exactly representable in the
     storage dtype (bf16-rounded where ``dtype_io`` is bf16).  Layouts:
     ``x [B,L,H,R,P]``, ``dt/lam [B,L,H]``, ``A_log [H,n_decay]``,
     ``theta [H,n_pairs]``, ``D [H]``, ``Bm [B,L,G,R,N]``, ``Cm [B,L,G,O,N]``,
-    ``dy [B,L,H,O,P]``; optional ``h0``/``w0`` ``[B,H,N,P]``.
+    ``dy [B,L,H,O,P]``; optional ``h0``/``w0`` ``[B,H,N,P]``; with ``with_raw``
+    also the pre-activation inputs ``z``, ``lam_logit`` ``[B,L,H]`` and
+    ``dt_bias [H]`` that ``dt`` and ``lam`` were made from (the draws are the
+    same either way).
     """
     s = shape
     g = np.random.Generator(np.random.PCG64(seed))
@@ -178,8 +181,11 @@ def make_inputs(shape: ScanShape, seed: int, with_dy: bool = True,
     if with_state:
         out["h0"] = g.standard_normal((Bt, H, N, P), dtype=f32) * f32(0.5)
         out["w0"] = g.standard_normal((Bt, H, N, P), dtype=f32) * f32(0.5)
+    if with_raw:
+        out["z"], out["lam_logit"] = z, lam_logit
+        out["dt_bias"] = dt_bias.astype(f32)
     if s.dtype_io == DTYPE_BF16:
-        for k in ("dt", "lam", "Bm", "Cm", "x", "dy"):
+        for k in ("dt", "lam", "Bm", "Cm", "x", "dy", "z", "lam_logit"):
             if k in out:
                 out[k] = round_bf16(out[k])
     if s.angle_mode == ANGLE_PER_TOKEN:

@@ -38,13 +38,15 @@ def _dev(a, shape):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(scan.io_dtype(shape)).cuda()
 
 
-@pytest.mark.parametrize("name", ["tiny_hybrid_fp32", "hybridmamba", "mamba1_siso"])
-def test_preact_forward_and_backward(name):
+@pytest.mark.parametrize("name,heads", [("tiny_hybrid_fp32", 0), ("hybridmamba", 4),
+                                        ("mamba1_siso", 96), ("hybridmamba", 3),
+                                        ("tiny_hybrid_fp32", 5)])
+def test_preact_forward_and_backward(name, heads):
+    """Both pre-activation passes against the oracle: dense layouts with an even
+    head count take two heads per thread, odd head counts one element per thread."""
     shape = S.WORKLOADS[name].replace(batch=2, seqlen=37)
-    if name == "mamba1_siso":
-        shape = shape.replace(nheads=96)
-    if name == "hybridmamba":
-        shape = shape.replace(nheads=4, ngroups=4)
+    if heads:
+        shape = shape.replace(nheads=heads, ngroups=heads if name != "mamba1_siso" else 1)
     z, bias, logit = _raw(shape, 5)
     desc = abi.make_desc(shape)
     zd, ld = _dev(z, shape), _dev(logit, shape)

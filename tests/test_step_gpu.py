@@ -96,6 +96,31 @@ def test_steps_with_zoh_write(kw):
     compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
 
 
+@pytest.mark.parametrize("kw", [
+    # sixteen channels per head, up to nine heads per CTA, ranks 8: the staged kernel
+    # with 83 KB of coefficients (above the default shared-memory limit)
+    dict(headdim=16, nheads=18, ngroups=9, n_real=96, n_pairs=16, rank_in=8, rank_out=8),
+    # 256 state rows at ranks 8: 166 KB of coefficients, too large for shared memory,
+    # the per-channel kernel
+    dict(headdim=16, nheads=9, ngroups=9, n_real=128, n_pairs=64, rank_in=8, rank_out=8),
+    # one channel per head: the per-channel kernel
+    dict(headdim=1, nheads=256, ngroups=2, n_real=12, n_pairs=2, rank_in=2, rank_out=3),
+    # a head width that does not divide the CTA (its heads straddle CTAs)
+    dict(headdim=48, nheads=5, ngroups=5, n_real=9, n_pairs=3),
+])
+def test_steps_kernel_layouts(kw):
+    """The step's CTA layouts: several heads per CTA, heads straddling CTAs, and the
+    per-channel kernel taken for one-channel heads or coefficients too large for
+    shared memory."""
+    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(batch=2, seqlen=5, **kw)
+    inp = S.make_inputs(shape, seed=17, with_dy=False, with_state=True)
+    y, h, w = step_through(shape, inp)
+    ref = oracle.scan_fwd(shape, inp)
+    compare("y", to_np(y), ref["y"], shape.dtype_io)
+    compare("hT", to_np(h), ref["hT"], shape.dtype_io)
+    compare("last_write", to_np(w), ref["wT"], shape.dtype_io)
+
+
 def test_euler_write_needs_no_w():
     shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=6, two_endpoint=0)
     inp = S.make_inputs(shape, seed=12, with_dy=False, with_state=True)
