@@ -15,6 +15,9 @@ the per-head parameter gradients.
   the per-channel parameter gradients (sums over the batch) come from every
   batch row of sampled channels.
 * SSD-MIMO rank 4 (4 x 16384, 16 heads, B and C per head): sampled heads.
+* Variants at the HybridMamba / SSD-MIMO sizes: per-token rotation angles and
+  the ZOH write on the per-coordinate tensor-core chain, one target row per
+  token (O = 1, R = 4) on the scalar-decay chain; sampled heads.
 """
 import numpy as np
 import pytest
@@ -31,13 +34,14 @@ torch = pytest.importorskip("torch")
 PER_TOKEN = ("x", "dt", "lam", "Bm", "Cm", "dy")
 
 
-def _train_step(name, seed):
-    """Training forward (saving workspace) + backward on the full workload;
-    outputs as float64 numpy arrays and the route both calls took."""
+def _train_step(name, seed, **variant):
+    """Training forward (saving workspace) + backward on the full workload (with
+    the descriptor changes `variant`); outputs as float64 numpy arrays and the
+    route both calls took."""
     from selective_diagonal_state_b200 import build
     build.build()
     abi.load_library()
-    shape = S.WORKLOADS[name]
+    shape = S.WORKLOADS[name].replace(**variant)
     inp = S.make_inputs(shape, seed=seed)
     dev = scan.to_device(shape, inp)
     wsf = scan.alloc_workspace(shape, abi.PASS_FWD)
@@ -67,7 +71,9 @@ def _sub_inputs(inp, heads, groups=None, batch=None):
             si[k] = a if groups is None else a[:, :, groups]
         else:
             si[k] = a[:, :, heads]
-    si.update(A_log=inp["A_log"][heads], theta=inp["theta"][heads], D=inp["D"][heads])
+    th = inp["theta"]
+    th = th[bsl][:, :, heads] if th.ndim == 4 else th[heads]   # per-token angles [B,L,H,np]
+    si.update(A_log=inp["A_log"][heads], theta=th, D=inp["D"][heads])
     return si
 
 
@@ -90,7 +96,8 @@ def _check(prefix, shape, out, ref, grad, heads, groups=None, batch=None, fields
     if shape.two_endpoint:
         pairs["dlambda"] = (out["dlam"][bsl][:, :, heads], grad["dlam"])
     if shape.n_pairs:
-        pairs["dtheta"] = (out["dtheta"][heads], grad["dtheta"])
+        dth = out["dtheta"]
+        pairs["dtheta"] = (dth[bsl][:, :, heads] if dth.ndim == 4 else dth[heads], grad["dtheta"])
     for k, (a, b) in pairs.items():
         if fields is None or k in fields:
             compare(k, a, b, dt)
@@ -176,4 +183,52 @@ def test_mimo_sampled_head(mimo_run, h):
     sub = shape.replace(nheads=1, ngroups=1)
     si = _sub_inputs(inp, hs, groups=hs)
     _check("mimo", shape, out, oracle.scan_fwd(sub, si), oracle.scan_bwd(sub, si, si["dy"]),
+           hs, groups=hs)
+
+
+# ---- variants at full size ----------------------------------------------------------
+@pytest.fixture(scope="module")
+def per_token_run():
+    return _train_step("hybridmamba", seed=8, angle_mode=S.ANGLE_PER_TOKEN)
+
+
+@pytest.mark.parametrize("h", (5, 30))
+def test_per_token_angles_sampled_head(per_token_run, h):
+    shape, inp, out, routes = per_token_run
+    assert routes == (abi.ROUTE_CHUNKED, abi.ROUTE_CHUNKED)
+    hs = slice(h, h + 1)
+    sub = shape.replace(nheads=1, ngroups=1)
+    si = _sub_inputs(inp, hs, groups=hs)
+    _check("per-token", shape, out, oracle.scan_fwd(sub, si), oracle.scan_bwd(sub, si, si["dy"]),
+           hs, groups=hs)
+
+
+@pytest.fixture(scope="module")
+def zoh_run():
+    return _train_step("hybridmamba", seed=9, two_endpoint=0, discretization=S.DISC_ZOH)
+
+
+@pytest.mark.parametrize("h", (2, 27))
+def test_zoh_write_sampled_head(zoh_run, h):
+    shape, inp, out, routes = zoh_run
+    assert routes == (abi.ROUTE_CHUNKED, abi.ROUTE_CHUNKED)
+    hs = slice(h, h + 1)
+    sub = shape.replace(nheads=1, ngroups=1)
+    si = _sub_inputs(inp, hs, groups=hs)
+    _check("zoh", shape, out, oracle.scan_fwd(sub, si), oracle.scan_bwd(sub, si, si["dy"]),
+           hs, groups=hs)
+
+
+@pytest.fixture(scope="module")
+def mimo_o1_run():
+    return _train_step("ssd_mimo_r4", seed=10, rank_out=1)
+
+
+def test_mimo_one_target_row_sampled_head(mimo_o1_run):
+    shape, inp, out, routes = mimo_o1_run
+    assert routes == (abi.ROUTE_SSD, abi.ROUTE_SSD)
+    hs = slice(9, 10)
+    sub = shape.replace(nheads=1, ngroups=1)
+    si = _sub_inputs(inp, hs, groups=hs)
+    _check("mimo-o1", shape, out, oracle.scan_fwd(sub, si), oracle.scan_bwd(sub, si, si["dy"]),
            hs, groups=hs)
