@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define SSM_SCAN_ABI_VERSION 2
+#define SSM_SCAN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define SSM_API __attribute__((visibility("default")))
@@ -292,6 +292,81 @@ SSM_API int ssm_preact_fwd(const ssm_desc_t *d, const void *z, const float *dt_b
 SSM_API int ssm_preact_bwd(const ssm_desc_t *d, const void *z, const float *dt_bias,
                            const void *lambda_logit, const void *ddt, const void *dlambda,
                            void *dz, float *ddt_bias, void *dlambda_logit, void *stream);
+
+/*
+ * Sequence sharding (context parallelism).  A sequence split into nseg
+ * consecutive segments (one per rank, or processed one after another) is
+ * scanned exactly by scanning every segment and exchanging per-segment
+ * boundary values.  The recurrence is linear in its state (sungsoo.github.io,
+ * Part 03: the chunked form composes the state carried between chunks the same
+ * way), so with Phi_k the product of segment k's transitions and beta_0(k) the
+ * left-endpoint weight of its first token:
+ *     forward:  K_in(0) = h0, W_in(0) = prev_write,
+ *               K_in(k+1) = Phi_k (K_in(k) + beta_0(k) W_in(k)) + hT_loc(k),
+ *               W_in(k+1) = last write of segment k,
+ *     where hT_loc(k) is segment k's end state scanned from zero (h0 = 0,
+ *     prev_write = 0); scanning segment k again from (K_in(k), W_in(k)) gives
+ *     its exact y and hT.
+ *     backward: dK_end(nseg-1) = dhT (NULL = 0),
+ *               dK_end(k) = dh0_loc(k+1) + Phi_{k+1}^T dK_end(k+1),
+ *               dW_end(k) = beta_0(k+1) dK_end(k)   (0 for the last segment),
+ *     where dh0_loc(k+1) is the dh0 of segment k+1's backward with no end
+ *     adjoint; segment k's backward with end adjoint dK_end(k) gives its exact
+ *     gradients once dW_end(k) is added to its last token's write
+ *     (ssm_cp_write_adjoint), and the per-head parameter gradients are the sums
+ *     over segments.
+ * The end adjoint enters a segment's backward through ssm_cp_tail_rows(d)
+ * trailing rows of its buffers (ssm_cp_fill_tail): the backward runs over
+ * seqlen + tail rows with the same strides.  Every call below takes the
+ * segment's own descriptor (seqlen = the segment's length, strides of its
+ * buffers).  Layouts: states [B][H][N][P] fp32; phi [B][H][n_real + n_pairs][2]
+ * fp32 (re, im; im = 0 on a real row); beta0 [B][H] fp32; a gathered array
+ * ("_all") stacks nseg of them, segment k at index k.
+ */
+
+/* Trailing rows ssm_cp_fill_tail writes: N (fp32 I/O) or 2 N (bf16: the end
+ * adjoint as bf16 value + remainder).  -1 for a bad descriptor. */
+SSM_API int ssm_cp_tail_rows(const ssm_desc_t *d);
+
+/* phi and beta0 of the segment described by d (its dt, lambda, theta: the
+ * same inputs as ssm_scan_fwd).  n_pairs up to 64. */
+SSM_API int ssm_cp_segment_transition(const ssm_desc_t *d, const void *dt, const float *A_log,
+                                      const float *theta, const void *lambda, float *phi,
+                                      float *beta0, void *stream);
+
+/* K_in(seg) -> h_in and W_in(seg) -> w_in from the gathered hT_loc / last
+ * writes / phi / beta0 of the segments before seg, starting from h0 /
+ * prev_write (NULL = zero).  The gathered arrays are not read when seg == 0. */
+SSM_API int ssm_cp_state_combine(const ssm_desc_t *d, int nseg, int seg, const float *hT_all,
+                                 const float *wT_all, const float *phi_all,
+                                 const float *beta0_all, const float *h0, const float *w0,
+                                 float *h_in, float *w_in, void *stream);
+
+/* dK_end(seg) -> dh_end and dW_end(seg) -> dw_end from the gathered dh0_loc /
+ * phi / beta0 of the segments after seg and the adjoint dhT of the whole
+ * sequence's final state (NULL = zero).  The gathered arrays are not read when
+ * seg == nseg - 1. */
+SSM_API int ssm_cp_adjoint_combine(const ssm_desc_t *d, int nseg, int seg, const float *dh0_all,
+                                   const float *phi_all, const float *beta0_all,
+                                   const float *dhT, float *dh_end, float *dw_end, void *stream);
+
+/* Writes the trailing rows t = seqlen .. seqlen + tail - 1 of the segment's
+ * x, dt, B, C, lambda (two_endpoint) and dy buffers (which must hold them at
+ * the descriptor's strides): dt, x and B zero, lambda 1, so the state passes
+ * through unchanged; C row 0 of trailing token s N + k is the unit vector e_k
+ * and its dy row 0 carries part s of dh_end[:, k, :] (NULL = zero).  A
+ * backward over seqlen + tail tokens then has dh_end as the adjoint of the
+ * segment's end state, and the trailing rows add nothing to the parameter
+ * gradients (they are weighted by dt or x).  Not for per-token angles or
+ * static rows (SSM_ERR_UNSUPPORTED). */
+SSM_API int ssm_cp_fill_tail(const ssm_desc_t *d, void *x, void *dt, void *B, void *C,
+                             void *lambda, void *dy, const float *dh_end, void *stream);
+
+/* Adds dw_end, the adjoint of the segment's last write W_{L-1} = B_{L-1} u_{L-1},
+ * to dx and dB of its last token (dx += B^T dw_end per head, dB += the group's
+ * sum of dw_end u^T); dx / dB as written by ssm_scan_bwd. */
+SSM_API int ssm_cp_write_adjoint(const ssm_desc_t *d, const void *x, const void *B,
+                                 const float *dw_end, void *dx, void *dB, void *stream);
 
 /* Message describing the last failing call on this host thread ("" if none). */
 SSM_API const char *ssm_scan_last_error(void);

@@ -25,7 +25,9 @@ EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd"
             "ssm_scan_bwd", "ssm_scan_last_error", "ssm_scan_poll_device_error",
             "ssm_scan_abi_version", "ssm_scan_profile_start", "ssm_scan_profile_stop",
             "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
-            "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd", "ssm_scan_set_wait_limit"]
+            "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd", "ssm_scan_set_wait_limit",
+            "ssm_cp_tail_rows", "ssm_cp_segment_transition", "ssm_cp_state_combine",
+            "ssm_cp_adjoint_combine", "ssm_cp_fill_tail", "ssm_cp_write_adjoint"]
 ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT, ROUTE_SSD, ROUTE_CHANNEL = 0, 1, 2, 3, 4
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -86,6 +88,20 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_preact_fwd.restype = ctypes.c_int
     lib.ssm_preact_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 9
     lib.ssm_preact_bwd.restype = ctypes.c_int
+    lib.ssm_cp_tail_rows.argtypes = [ctypes.POINTER(Desc)]
+    lib.ssm_cp_tail_rows.restype = ctypes.c_int
+    lib.ssm_cp_segment_transition.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 7
+    lib.ssm_cp_segment_transition.restype = ctypes.c_int
+    lib.ssm_cp_state_combine.argtypes = ([ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_int] +
+                                         [_vp] * 9)
+    lib.ssm_cp_state_combine.restype = ctypes.c_int
+    lib.ssm_cp_adjoint_combine.argtypes = ([ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_int] +
+                                           [_vp] * 7)
+    lib.ssm_cp_adjoint_combine.restype = ctypes.c_int
+    lib.ssm_cp_fill_tail.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 8
+    lib.ssm_cp_fill_tail.restype = ctypes.c_int
+    lib.ssm_cp_write_adjoint.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 6
+    lib.ssm_cp_write_adjoint.restype = ctypes.c_int
     lib.ssm_scan_last_error.argtypes = []
     lib.ssm_scan_last_error.restype = ctypes.c_char_p
     lib.ssm_scan_poll_device_error.argtypes = [_vp]
@@ -166,6 +182,49 @@ def ssm_scan_step(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h, w, y, stream
     rc = lib.ssm_scan_step(ctypes.byref(desc), *[_ptr(t) for t in (
         x, dt, A_log, theta, B, C, D, lam, h, w, y)], _stream(stream))
     _check(rc, "ssm_scan_step")
+
+
+def ssm_cp_tail_rows(desc: Desc) -> int:
+    n = int(load_library().ssm_cp_tail_rows(ctypes.byref(desc)))
+    _check(SSM_OK if n >= 0 else -1, "ssm_cp_tail_rows")
+    return n
+
+
+def ssm_cp_segment_transition(desc: Desc, dt, A_log, theta, lam, phi, beta0, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_cp_segment_transition(ctypes.byref(desc), *[_ptr(t) for t in (
+        dt, A_log, theta, lam, phi, beta0)], _stream(stream))
+    _check(rc, "ssm_cp_segment_transition")
+
+
+def ssm_cp_state_combine(desc: Desc, nseg: int, seg: int, hT_all, wT_all, phi_all, beta0_all,
+                         h0, w0, h_in, w_in, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_cp_state_combine(ctypes.byref(desc), nseg, seg, *[_ptr(t) for t in (
+        hT_all, wT_all, phi_all, beta0_all, h0, w0, h_in, w_in)], _stream(stream))
+    _check(rc, "ssm_cp_state_combine")
+
+
+def ssm_cp_adjoint_combine(desc: Desc, nseg: int, seg: int, dh0_all, phi_all, beta0_all, dhT,
+                           dh_end, dw_end, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_cp_adjoint_combine(ctypes.byref(desc), nseg, seg, *[_ptr(t) for t in (
+        dh0_all, phi_all, beta0_all, dhT, dh_end, dw_end)], _stream(stream))
+    _check(rc, "ssm_cp_adjoint_combine")
+
+
+def ssm_cp_fill_tail(desc: Desc, x, dt, B, C, lam, dy, dh_end, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_cp_fill_tail(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, B, C, lam, dy, dh_end)], _stream(stream))
+    _check(rc, "ssm_cp_fill_tail")
+
+
+def ssm_cp_write_adjoint(desc: Desc, x, B, dw_end, dx, dB, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_cp_write_adjoint(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, B, dw_end, dx, dB)], _stream(stream))
+    _check(rc, "ssm_cp_write_adjoint")
 
 
 def ssm_preact_fwd(desc: Desc, z, dt_bias, lam_logit, dt, lam, stream=None) -> None:

@@ -45,6 +45,15 @@ size_t m1_part_floats(long long B, long long L, long long H, int N);
 cudaError_t m1_forward(const Params &p, float *kept, cudaStream_t st);
 cudaError_t m1_backward(const Params &p, float *kept, bool kept_ready, float *part,
                         cudaStream_t st);
+cudaError_t cp_transition(const Params &p, float *phi, float *beta0, cudaStream_t st);
+cudaError_t cp_state_combine(const Params &p, int seg, const float *hT_all, const float *wT_all,
+                             const float *phi_all, const float *beta0_all, const float *h0,
+                             const float *w0, float *h_in, float *w_in, cudaStream_t st);
+cudaError_t cp_adjoint_combine(const Params &p, int nseg, int seg, const float *dh0_all,
+                               const float *phi_all, const float *beta0_all, const float *dhT,
+                               float *dh_end, float *dw_end, cudaStream_t st);
+cudaError_t cp_write_adjoint(const Params &p, const float *dw_end, cudaStream_t st);
+cudaError_t cp_fill_tail(const Params &p, int nv, const float *dh_end, cudaStream_t st);
 }  // namespace ssm
 
 namespace {
@@ -991,6 +1000,134 @@ int ssm_scan_profile_stop(char *names, int name_len, int *counts, double *total_
     return n;
 }
 
+
+// ---- sequence sharding ---------------------------------------------------------------
+int ssm_cp_tail_rows(const ssm_desc_t *d) {
+    if (validate_desc(d)) return -1;
+    return (d->dtype_io == SSM_BF16 ? 2 : 1) * nstate(d);
+}
+
+int ssm_cp_segment_transition(const ssm_desc_t *d, const void *dt, const float *A_log,
+                              const float *theta, const void *lambda, float *phi, float *beta0,
+                              void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(dt, "dt", es)) || (rc = check_ptr(A_log, "A_log", 4)) ||
+        (rc = check_ptr(phi, "phi", 4)) || (rc = check_ptr(beta0, "beta0", 4)))
+        return rc;
+    if (d->n_pairs && (rc = check_ptr(theta, "theta", 4))) return rc;
+    if (d->two_endpoint && (rc = check_ptr(lambda, "lambda", es))) return rc;
+    if (d->n_pairs > 64)
+        return fail(SSM_ERR_UNSUPPORTED, "ssm_cp_segment_transition: n_pairs %d above 64", d->n_pairs);
+    ssm::Params p;
+    fill_params(d, p);
+    p.dt = dt; p.A_log = A_log; p.theta = theta; p.lam = lambda;
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::cp_transition(p, phi, beta0, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_cp_segment_transition launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_cp_state_combine(const ssm_desc_t *d, int nseg, int seg, const float *hT_all,
+                         const float *wT_all, const float *phi_all, const float *beta0_all,
+                         const float *h0, const float *w0, float *h_in, float *w_in,
+                         void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (nseg < 1 || seg < 0 || seg >= nseg)
+        return fail(SSM_ERR_ARG, "ssm_cp_state_combine: segment %d of %d", seg, nseg);
+    if ((rc = check_ptr(h_in, "h_in", 4)) || (rc = check_ptr(w_in, "w_in", 4))) return rc;
+    if (seg > 0 && ((rc = check_ptr(hT_all, "hT_all", 4)) || (rc = check_ptr(wT_all, "wT_all", 4)) ||
+                    (rc = check_ptr(phi_all, "phi_all", 4)) ||
+                    (rc = check_ptr(beta0_all, "beta0_all", 4))))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e =
+        ssm::cp_state_combine(p, seg, hT_all, wT_all, phi_all, beta0_all, h0, w0, h_in, w_in, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_cp_state_combine launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_cp_adjoint_combine(const ssm_desc_t *d, int nseg, int seg, const float *dh0_all,
+                           const float *phi_all, const float *beta0_all, const float *dhT,
+                           float *dh_end, float *dw_end, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (nseg < 1 || seg < 0 || seg >= nseg)
+        return fail(SSM_ERR_ARG, "ssm_cp_adjoint_combine: segment %d of %d", seg, nseg);
+    if ((rc = check_ptr(dh_end, "dh_end", 4)) || (rc = check_ptr(dw_end, "dw_end", 4))) return rc;
+    if (seg + 1 < nseg &&
+        ((rc = check_ptr(dh0_all, "dh0_all", 4)) || (rc = check_ptr(phi_all, "phi_all", 4)) ||
+         (rc = check_ptr(beta0_all, "beta0_all", 4))))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::cp_adjoint_combine(p, nseg, seg, dh0_all, phi_all, beta0_all, dhT,
+                                                  dh_end, dw_end, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_cp_adjoint_combine launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_cp_fill_tail(const ssm_desc_t *d, void *x, void *dt, void *B, void *C, void *lambda,
+                     void *dy, const float *dh_end, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (d->angle_mode == SSM_ANGLE_PER_TOKEN && d->n_pairs)
+        return fail(SSM_ERR_UNSUPPORTED, "ssm_cp_fill_tail: per-token angles");
+    if (d->n_static)
+        return fail(SSM_ERR_UNSUPPORTED,
+                    "ssm_cp_fill_tail: static rows (their transition does not vanish with dt)");
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(x, "x", es)) || (rc = check_ptr(dt, "dt", es)) ||
+        (rc = check_ptr(B, "B", es)) || (rc = check_ptr(C, "C", es)) || (rc = check_ptr(dy, "dy", es)))
+        return rc;
+    if (d->two_endpoint && (rc = check_ptr(lambda, "lambda", es))) return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    p.x = x; p.dt = dt; p.Bm = B; p.Cm = C; p.lam = lambda; p.dy = dy;
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::cp_fill_tail(p, ssm_cp_tail_rows(d), dh_end, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_cp_fill_tail launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+int ssm_cp_write_adjoint(const ssm_desc_t *d, const void *x, const void *B, const float *dw_end,
+                         void *dx, void *dB, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (d->batch == 0 || d->seqlen == 0) return SSM_OK;
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(x, "x", es)) || (rc = check_ptr(B, "B", es)) ||
+        (rc = check_ptr(dw_end, "dw_end", 4)) || (rc = check_ptr(dx, "dx", es)) ||
+        (rc = check_ptr(dB, "dB", es)))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    p.x = x; p.Bm = B; p.dx = dx; p.dBm = dB;
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::cp_write_adjoint(p, dw_end, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_cp_write_adjoint launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
 
 }  // extern "C"
 

@@ -1,0 +1,313 @@
+// Sequence sharding (context parallelism): the pieces that join scans of
+// consecutive segments of one sequence into the scan of the whole sequence.
+//
+// The recurrence is linear in its state, so a segment run from a zero state
+// and a zero left endpoint gives its local end state, and the true end state is
+// that plus the segment's whole transition applied to what enters it
+// ("When a Diagonal State Is Not Enough", sungsoo.github.io, Part 03: the state
+// carried between chunks of the chunked form is the same composition):
+//     K_in(k + 1) = Phi_k (K_in(k) + beta_0(k) W_in(k)) + hT_loc(k),
+//     W_in(k + 1) = last write of segment k,
+// Phi_k = prod over the segment of A_t (per mode: e^{a sum dt} and a rotation
+// by the summed angle), beta_0(k) the left-endpoint weight of its first token.
+// The backward is the mirror image: the adjoint entering the end of segment k
+// is the full adjoint of the next segment's initial state,
+//     dK_end(k) = dh0_loc(k + 1) + Phi_{k+1}^T dK_end(k + 1),
+// and the last write of segment k receives beta_0(k + 1) times it.
+//
+// Kernels: the segment transition, the two combines (an ordered scan over the
+// gathered per-segment values, elementwise over (b, h, mode, channel)), the
+// adjoint of the boundary write (added to dx / dB of the segment's last token),
+// and the fill of the trailing rows through which a segment's backward receives
+// its end adjoint (one-hot C rows read the state out; their dy carries it).
+#include "common.cuh"
+
+namespace ssm {
+
+namespace cpk {
+constexpr int THREADS = 256;
+}
+
+// Phi of every (b, h, mode) of the segment ([B][H][nmode][2], (re, im)) and
+// beta_0 ([B][H]).  One CTA per (b, h): the sums of dt (and of the per-token
+// angles) over the segment in a fixed order, then one thread per mode.
+__global__ void __launch_bounds__(cpk::THREADS) k_cp_transition(Params p, float *phi, float *beta0) {
+    __shared__ float red[cpk::THREADS];
+    __shared__ float th[64 * 8];   // per-token angle partial sums [pair][warp]
+    const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float s = 0.f;
+    for (int t = tid; t < p.L; t += cpk::THREADS) s += ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+    red[tid] = s;
+    // per-token angles: warp w sums tokens w, w + 8, ...; lane j (and j + 32) one pair
+    if (p.angle_tok && p.np) {
+        for (int j = lane; j < p.np; j += 32) {
+            float a = 0.f;
+            for (int t = warp; t < p.L; t += cpk::THREADS / 32) a += p.theta[ix_th(p, b, t, h, j)];
+            th[j * 8 + warp] = a;
+        }
+    }
+    __syncthreads();
+    for (int w = cpk::THREADS / 2; w >= 1; w >>= 1) {
+        if (tid < w) red[tid] += red[tid + w];
+        __syncthreads();
+    }
+    const float S = red[0];
+    const int nmode = p.nr + p.np;
+    for (int m = tid; m < nmode; m += cpk::THREADS) {
+        const float a = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
+        float re, im = 0.f;
+        if (m < p.nr) {
+            re = expf(a * (m < p.nst ? (float)p.L : S));   // static rows: e^{a} per token
+        } else {
+            const int j = m - p.nr;
+            float ang;
+            if (p.angle_tok) {
+                ang = 0.f;
+                for (int w = 0; w < cpk::THREADS / 32; ++w) ang += th[j * 8 + w];
+            } else {
+                ang = p.theta[h * p.np + j] * S;
+            }
+            float sn, cs;
+            sincosf(ang, &sn, &cs);
+            const float mag = expf(a * S);
+            re = mag * cs;
+            im = mag * sn;
+        }
+        float *o = phi + ((long long)bh * nmode + m) * 2;
+        o[0] = re;
+        o[1] = im;
+    }
+    if (tid == 0) {
+        float b0 = 0.f;
+        if (p.two_ep && p.L > 0)
+            b0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), p.bf16)) * ld_io(p.dt, ix_dt(p, b, 0, h), p.bf16);
+        beta0[bh] = b0;
+    }
+}
+
+// Unit (b, h, mode m, channel q): a real mode is one state row, a pair mode its
+// (re, im) rows.
+struct CpUnit {
+    int b, h, m, q, n0;
+    bool pair;
+};
+__device__ __forceinline__ CpUnit cp_unit(const Params &p, long long u) {
+    const int nmode = p.nr + p.np;
+    CpUnit c;
+    c.q = (int)(u % p.P);
+    long long r = u / p.P;
+    c.m = (int)(r % nmode);
+    r /= nmode;
+    c.h = (int)(r % p.H);
+    c.b = (int)(r / p.H);
+    c.pair = c.m >= p.nr;
+    c.n0 = c.pair ? p.nr + 2 * (c.m - p.nr) : c.m;
+    return c;
+}
+
+// State and left endpoint entering segment `seg` from the gathered local end
+// states hT_all / last writes wT_all ([nseg][B][H][N][P]), transitions phi_all
+// ([nseg][B][H][nmode][2]) and beta0_all ([nseg][B][H]) of the segments before
+// it, starting from h0 / w0 (NULL = zero).
+__global__ void __launch_bounds__(cpk::THREADS)
+    k_cp_state_combine(Params p, int seg, const float *hT_all, const float *wT_all,
+                       const float *phi_all, const float *beta0_all, const float *h0,
+                       const float *w0, float *h_in, float *w_in) {
+    const int nmode = p.nr + p.np;
+    const long long units = (long long)p.Bsz * p.H * nmode * p.P;
+    const long long st = (long long)p.Bsz * p.H * p.N * p.P;   // one segment's state
+    const long long bhs = (long long)p.Bsz * p.H;
+    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+         u += (long long)gridDim.x * blockDim.x) {
+        const CpUnit c = cp_unit(p, u);
+        const long long i0 = ix_st(p, c.b, c.h, c.n0, c.q);
+        const long long i1 = c.pair ? ix_st(p, c.b, c.h, c.n0 + 1, c.q) : i0;
+        float hr = h0 ? h0[i0] : 0.f, hi = (c.pair && h0) ? h0[i1] : 0.f;
+        float wr = w0 ? w0[i0] : 0.f, wi = (c.pair && w0) ? w0[i1] : 0.f;
+        const long long bh = (long long)c.b * p.H + c.h;
+        for (int k = 0; k < seg; ++k) {
+            const float be = beta0_all[k * bhs + bh];
+            const float *ph = phi_all + ((k * bhs + bh) * nmode + c.m) * 2;
+            const float zr = fmaf(be, wr, hr), zi = fmaf(be, wi, hi);
+            hr = fmaf(ph[0], zr, -ph[1] * zi) + hT_all[k * st + i0];
+            hi = c.pair ? fmaf(ph[1], zr, ph[0] * zi) + hT_all[k * st + i1] : 0.f;
+            wr = wT_all[k * st + i0];
+            wi = c.pair ? wT_all[k * st + i1] : 0.f;
+        }
+        h_in[i0] = hr;
+        w_in[i0] = wr;
+        if (c.pair) {
+            h_in[i1] = hi;
+            w_in[i1] = wi;
+        }
+    }
+}
+
+// Adjoint entering the end of segment `seg` (and the adjoint of its last write)
+// from the gathered local initial-state adjoints dh0_all ([nseg][B][H][N][P]) and
+// transitions of the segments after it, starting from dhT (NULL = zero) at the
+// end of the last segment.
+__global__ void __launch_bounds__(cpk::THREADS)
+    k_cp_adjoint_combine(Params p, int nseg, int seg, const float *dh0_all,
+                         const float *phi_all, const float *beta0_all, const float *dhT,
+                         float *dh_end, float *dw_end) {
+    const int nmode = p.nr + p.np;
+    const long long units = (long long)p.Bsz * p.H * nmode * p.P;
+    const long long st = (long long)p.Bsz * p.H * p.N * p.P;
+    const long long bhs = (long long)p.Bsz * p.H;
+    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+         u += (long long)gridDim.x * blockDim.x) {
+        const CpUnit c = cp_unit(p, u);
+        const long long i0 = ix_st(p, c.b, c.h, c.n0, c.q);
+        const long long i1 = c.pair ? ix_st(p, c.b, c.h, c.n0 + 1, c.q) : i0;
+        float gr = dhT ? dhT[i0] : 0.f, gi = (c.pair && dhT) ? dhT[i1] : 0.f;
+        const long long bh = (long long)c.b * p.H + c.h;
+        for (int k = nseg - 1; k > seg; --k) {
+            // full adjoint of segment k's initial state: its own part + Phi_k^T g
+            const float *ph = phi_all + ((k * bhs + bh) * nmode + c.m) * 2;
+            const float nr_ = fmaf(ph[0], gr, ph[1] * gi) + dh0_all[k * st + i0];
+            const float ni_ = c.pair ? fmaf(-ph[1], gr, ph[0] * gi) + dh0_all[k * st + i1] : 0.f;
+            gr = nr_;
+            gi = ni_;
+        }
+        const float be = seg + 1 < nseg ? beta0_all[(seg + 1) * bhs + bh] : 0.f;
+        dh_end[i0] = gr;
+        dw_end[i0] = be * gr;
+        if (c.pair) {
+            dh_end[i1] = gi;
+            dw_end[i1] = be * gi;
+        }
+    }
+}
+
+// dW of the segment's last token (t = L - 1) receives dw_end: dx += B^T dw_end per
+// head, dB += sum over the group's heads of dw_end u^T.  Thread (b, h, r, q) for dx,
+// then (b, g, r, n) for dB.
+__global__ void __launch_bounds__(cpk::THREADS) k_cp_write_adjoint(Params p, const float *dw_end) {
+    const int t = p.L - 1;
+    const long long nx = (long long)p.Bsz * p.H * p.R * p.P;
+    const long long nb = (long long)p.Bsz * p.G * p.R * p.N;
+    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < nx + nb;
+         u += (long long)gridDim.x * blockDim.x) {
+        if (u < nx) {
+            const int q = (int)(u % p.P);
+            long long r_ = u / p.P;
+            const int r = (int)(r_ % p.R);
+            r_ /= p.R;
+            const int h = (int)(r_ % p.H), b = (int)(r_ / p.H), g = h / p.hpg;
+            float acc = 0.f;
+            for (int n = 0; n < p.N; ++n)
+                acc = fmaf(ld_io(p.Bm, ix_B(p, b, t, g, r, n), p.bf16), dw_end[ix_st(p, b, h, n, q)], acc);
+            const long long ix = ix_x(p, b, t, h, r, q);
+            st_io(p.dx, ix, ld_io(p.dx, ix, p.bf16) + acc, p.bf16);
+        } else {
+            const long long v = u - nx;
+            const int n = (int)(v % p.N);
+            long long r_ = v / p.N;
+            const int r = (int)(r_ % p.R);
+            r_ /= p.R;
+            const int g = (int)(r_ % p.G), b = (int)(r_ / p.G);
+            float acc = 0.f;
+            for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h)
+                for (int q = 0; q < p.P; ++q)
+                    acc = fmaf(dw_end[ix_st(p, b, h, n, q)], ld_io(p.x, ix_x(p, b, t, h, r, q), p.bf16), acc);
+            const long long ib = ix_B(p, b, t, g, r, n);
+            st_io(p.dBm, ib, ld_io(p.dBm, ib, p.bf16) + acc, p.bf16);
+        }
+    }
+}
+
+// Trailing rows t = L .. L + nv - 1 of a segment's buffers (p.L = the segment's
+// own length, the buffers hold L + nv tokens): zero dt, x, B, lambda 1 (static
+// angles, no static rows), so the state passes through unchanged and nothing is
+// written; C row o = 0 of trailing token L + s N + k is e_k (the others zero),
+// and its dy carries part s of dh_end[:, k, :] (bf16: s = 0 the bf16 value,
+// s = 1 the remainder; fp32: one part).  The backward over L + nv tokens then
+// receives dh_end as the adjoint of the segment's end state; every gradient a
+// trailing row adds to the parameters is weighted by its dt (zero) or its input
+// (zero).
+__global__ void __launch_bounds__(cpk::THREADS) k_cp_fill_tail(Params p, int nv, const float *dh_end) {
+    const int nsets = nv / p.N;
+    const long long per_tok = (long long)p.Bsz * p.H;   // (b, h) pairs per trailing token
+    const long long units = (long long)nv * per_tok;
+    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+         u += (long long)gridDim.x * blockDim.x) {
+        const int v = (int)(u / per_tok);
+        const long long bh = u - (long long)v * per_tok;
+        const int b = (int)(bh / p.H), h = (int)(bh - (long long)b * p.H);
+        const int g = h / p.hpg, t = p.L + v, s = v / p.N, k = v - s * p.N;
+        st_io((void *)p.dt, ix_dt(p, b, t, h), 0.f, p.bf16);
+        if (p.two_ep) st_io((void *)p.lam, ix_lam(p, b, t, h), 1.f, p.bf16);
+        for (int r = 0; r < p.R; ++r)
+            for (int q = 0; q < p.P; ++q) st_io((void *)p.x, ix_x(p, b, t, h, r, q), 0.f, p.bf16);
+        for (int o = 0; o < p.O; ++o)
+            for (int q = 0; q < p.P; ++q) {
+                float val = 0.f;
+                if (o == 0) {
+                    const float d = dh_end ? dh_end[ix_st(p, b, h, k, q)] : 0.f;
+                    const float hi = p.bf16 ? __bfloat162float(__float2bfloat16_rn(d)) : d;
+                    val = (nsets == 1 || s == 0) ? hi : d - hi;
+                }
+                st_io((void *)p.dy, ix_y(p, b, t, h, o, q), val, p.bf16);
+            }
+        if (h == g * p.hpg) {   // B and C rows once per group
+            for (int r = 0; r < p.R; ++r)
+                for (int n = 0; n < p.N; ++n) st_io((void *)p.Bm, ix_B(p, b, t, g, r, n), 0.f, p.bf16);
+            for (int o = 0; o < p.O; ++o)
+                for (int n = 0; n < p.N; ++n)
+                    st_io((void *)p.Cm, ix_C(p, b, t, g, o, n), (o == 0 && n == k) ? 1.f : 0.f, p.bf16);
+        }
+    }
+}
+
+static int cp_blocks(long long units) {
+    long long b = (units + cpk::THREADS - 1) / cpk::THREADS;
+    if (b > 148 * 16) b = 148 * 16;
+    return b < 1 ? 1 : (int)b;
+}
+
+cudaError_t cp_transition(const Params &p, float *phi, float *beta0, cudaStream_t st) {
+    if (p.Bsz * p.H == 0) return cudaSuccess;
+    k_cp_transition<<<p.Bsz * p.H, cpk::THREADS, 0, st>>>(p, phi, beta0);
+    profile_mark(st, "k_cp_transition");
+    return cudaGetLastError();
+}
+
+cudaError_t cp_state_combine(const Params &p, int seg, const float *hT_all, const float *wT_all,
+                             const float *phi_all, const float *beta0_all, const float *h0,
+                             const float *w0, float *h_in, float *w_in, cudaStream_t st) {
+    const long long units = (long long)p.Bsz * p.H * (p.nr + p.np) * p.P;
+    k_cp_state_combine<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, seg, hT_all, wT_all, phi_all,
+                                                                  beta0_all, h0, w0, h_in, w_in);
+    profile_mark(st, "k_cp_state_combine");
+    return cudaGetLastError();
+}
+
+cudaError_t cp_adjoint_combine(const Params &p, int nseg, int seg, const float *dh0_all,
+                               const float *phi_all, const float *beta0_all, const float *dhT,
+                               float *dh_end, float *dw_end, cudaStream_t st) {
+    const long long units = (long long)p.Bsz * p.H * (p.nr + p.np) * p.P;
+    k_cp_adjoint_combine<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, nseg, seg, dh0_all, phi_all,
+                                                                    beta0_all, dhT, dh_end, dw_end);
+    profile_mark(st, "k_cp_adjoint_combine");
+    return cudaGetLastError();
+}
+
+cudaError_t cp_write_adjoint(const Params &p, const float *dw_end, cudaStream_t st) {
+    if (p.L < 1) return cudaSuccess;
+    const long long units = (long long)p.Bsz * p.H * p.R * p.P + (long long)p.Bsz * p.G * p.R * p.N;
+    k_cp_write_adjoint<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, dw_end);
+    profile_mark(st, "k_cp_write_adjoint");
+    return cudaGetLastError();
+}
+
+cudaError_t cp_fill_tail(const Params &p, int nv, const float *dh_end, cudaStream_t st) {
+    const long long units = (long long)nv * p.Bsz * p.H;
+    if (units == 0) return cudaSuccess;
+    k_cp_fill_tail<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, nv, dh_end);
+    profile_mark(st, "k_cp_fill_tail");
+    return cudaGetLastError();
+}
+
+}  // namespace ssm

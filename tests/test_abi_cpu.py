@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert abi.ssm_scan_abi_version() == 2
+    assert abi.ssm_scan_abi_version() == 3
 
 
 def test_desc_layout_matches_header(lib):
