@@ -168,14 +168,14 @@ NCU_TRAFFIC_PER_ROW = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum captures at batch 2
     # (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the full Mamba-2 size; the traffic of
     # these kernels grows with the batch rows
-    ("hybridmamba", "k_chunk_fwd"): (420.8e6, "44f974fe96fa6c31"),
-    ("hybridmamba", "k_chunk_bwd_fused"): (603.45e6, "bf4b7047cc7bed68"),
-    ("ssd_mimo_r4", "k_ssd_fwd"): (1197.8e6, "968f48c9ed818efd"),
-    ("ssd_mimo_r4", "k_ssd_bwd"): (1736.5e6, "968f48c9ed818efd"),
-    ("mamba2_siso", "k_ssd_fwd"): (31.0e6, "968f48c9ed818efd"),
-    ("mamba2_siso", "k_ssd_bwd"): (75.25e6, "968f48c9ed818efd"),
-    ("mamba1_siso", "k_m1_fwd"): (60.55e6, "cab423aa329e9480"),
-    ("mamba1_siso", "k_m1_bwd"): (118.05e6, "cab423aa329e9480"),
+    ("hybridmamba", "k_chunk_fwd"): (420.69e6, "98ef2b7812470817"),
+    ("hybridmamba", "k_chunk_bwd_fused"): (603.48e6, "ea6b3d47ea94be38"),
+    ("ssd_mimo_r4", "k_ssd_fwd"): (1181.88e6, "92ad5153603b560e"),
+    ("ssd_mimo_r4", "k_ssd_bwd"): (1734.67e6, "92ad5153603b560e"),
+    ("mamba2_siso", "k_ssd_fwd"): (31.14e6, "92ad5153603b560e"),
+    ("mamba2_siso", "k_ssd_bwd"): (75.71e6, "92ad5153603b560e"),
+    ("mamba1_siso", "k_m1_fwd"): (60.46e6, "c4d8b182de0d5666"),
+    ("mamba1_siso", "k_m1_bwd"): (118.59e6, "c4d8b182de0d5666"),
 }
 
 # sources each kernel is compiled from: a traffic entry holds only while they
