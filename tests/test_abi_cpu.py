@@ -229,3 +229,31 @@ def test_preact_argument_checks(lib):
     assert fwd(z=FAKE + 1) == -3        # bf16 tensors need 2-byte alignment
     assert lib.ssm_preact_bwd(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
                               None) == -1
+
+
+def test_sequence_sharding_calls_validate_before_launch(lib):
+    """The ssm_cp_* calls check their arguments on the host (nothing is launched)."""
+    sh = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=100)
+    d = abi.make_desc(sh)
+    assert lib.ssm_cp_tail_rows(ctypes.byref(d)) == 2 * sh.nstate        # bf16: value + remainder
+    d32 = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"])
+    assert lib.ssm_cp_tail_rows(ctypes.byref(d32)) == S.WORKLOADS["tiny_hybrid_fp32"].nstate
+    bad = abi.make_desc(sh)
+    bad.ngroups = 5
+    assert lib.ssm_cp_tail_rows(ctypes.byref(bad)) == -1
+    p = [FAKE] * 8
+    # segment index out of range
+    assert lib.ssm_cp_state_combine(ctypes.byref(d), 2, 2, *p, None) == -1
+    assert "segment" in lib.ssm_scan_last_error().decode()
+    assert lib.ssm_cp_adjoint_combine(ctypes.byref(d), 0, 0, *p[:6], None) == -1
+    # missing outputs
+    assert lib.ssm_cp_state_combine(ctypes.byref(d), 2, 1, FAKE, FAKE, FAKE, FAKE, None, None,
+                                    None, FAKE, None) == -1
+    assert "h_in" in lib.ssm_scan_last_error().decode()
+    # the end-adjoint rows cannot carry per-token angles or static rows through
+    for kw in (dict(angle_mode=S.ANGLE_PER_TOKEN), dict(n_static=8)):
+        dd = abi.make_desc(sh.replace(**kw))
+        assert lib.ssm_cp_fill_tail(ctypes.byref(dd), *([FAKE] * 7), None) == -2
+    # transition: n_pairs above 64
+    wide = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(n_real=0, n_pairs=65))
+    assert lib.ssm_cp_segment_transition(ctypes.byref(wide), *([FAKE] * 6), None) == -2
