@@ -171,3 +171,27 @@ def preact_bwd(z, dt_bias, lam_logit, ddt, dlam=None):
         lam = _sigmoid(np.asarray(lam_logit, dtype=np.float64))
         dlogit = np.asarray(dlam, dtype=np.float64) * lam * (1.0 - lam)
     return dz, dbias, dlogit
+
+
+# ---- output gate of the mixer ------------------------------------------------------
+# The pages' fused kernel merges the state update with the gating and the output
+# projection of the mixer ("Diagonal Equivalence in State Space Models", kongchang.com:
+# the kernel-performance paragraph).  Reading (the gate's form is not given there): the
+# Mamba-style output gate y_g = y * silu(z), z of y's shape, silu(z) = z sigmoid(z).
+def gate_fwd(y, z):
+    """y_g = y * silu(z), elementwise."""
+    y = np.asarray(y, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    return y * z * _sigmoid(z)
+
+
+def gate_bwd(y, z, dyg):
+    """Chain rule through gate_fwd: (dy, dz) for the upstream gradient dyg."""
+    y = np.asarray(y, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    g = np.asarray(dyg, dtype=np.float64)
+    s = _sigmoid(z)
+    dy = g * z * s
+    dz = g * y * s * (1.0 + z * (1.0 - s))
+    return dy, dz
+
