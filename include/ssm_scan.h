@@ -171,6 +171,35 @@ SSM_API int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, con
                  void *stream);
 
 /*
+ * Forward scan followed by the mixer's output gate (the pages' fused kernel
+ * merges the state update with the gating and output projection of the mixer:
+ * "Diagonal Equivalence in State Space Models", kongchang.com, the
+ * kernel-performance paragraph; the gate's form is read as Mamba's):
+ *     y_gated = y * silu(z),   silu(z) = z / (1 + e^{-z}),
+ * with z in y's layout and strides (dtype_io).  Inputs and hT / last_write as
+ * ssm_scan_fwd; y_pre (may be NULL) receives the pre-gate y, which
+ * ssm_gate_bwd needs.  The per-coordinate tensor-core chain applies the gate in
+ * its output epilogue (z read there, y_gated and y_pre leaving by TMA stores);
+ * the other chains write y to y_gated and gate it in place with one
+ * elementwise pass.  Same workspace as ssm_scan_fwd.
+ */
+SSM_API int ssm_scan_fwd_gated(const ssm_desc_t *d, const void *x, const void *dt,
+                               const float *A_log, const float *theta, const void *B,
+                               const void *C, const float *D, const void *lambda,
+                               const float *h0, const float *prev_write, const void *z,
+                               void *y_gated, void *y_pre, float *hT, float *last_write,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Gradient through the output gate, for the upstream gradient dy_gated of
+ * y_gated: dy = dy_gated * silu(z) (the dy of ssm_scan_bwd) and
+ * dz = dy_gated * y_pre * sigmoid(z) (1 + z (1 - sigmoid(z))); all in y's
+ * layout and dtype_io.  dy may alias dy_gated.
+ */
+SSM_API int ssm_gate_bwd(const ssm_desc_t *d, const void *z, const void *y_pre,
+                         const void *dy_gated, void *dy, void *dz, void *stream);
+
+/*
  * Backward scan: gradients of sum(dy * y) with respect to every input of
  * ssm_scan_fwd, recomputing the forward states (nothing is saved between the
  * calls).  Inputs as for ssm_scan_fwd plus dy.  Outputs dx, ddt, dB, dC (in

@@ -27,7 +27,8 @@ EXPORTED = ["ssm_desc_set_contiguous", "ssm_scan_workspace_size", "ssm_scan_fwd"
             "ssm_scan_bwd_noalloc", "ssm_scan_last_route", "ssm_scan_bwd_saved",
             "ssm_scan_step", "ssm_preact_fwd", "ssm_preact_bwd", "ssm_scan_set_wait_limit",
             "ssm_cp_tail_rows", "ssm_cp_segment_transition", "ssm_cp_state_combine",
-            "ssm_cp_adjoint_combine", "ssm_cp_fill_tail", "ssm_cp_write_adjoint"]
+            "ssm_cp_adjoint_combine", "ssm_cp_fill_tail", "ssm_cp_write_adjoint",
+            "ssm_scan_fwd_gated", "ssm_gate_bwd"]
 ROUTE_CHUNKED, ROUTE_RANGE_FALLBACK, ROUTE_RECURRENT, ROUTE_SSD, ROUTE_CHANNEL = 0, 1, 2, 3, 4
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -88,6 +89,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_preact_fwd.restype = ctypes.c_int
     lib.ssm_preact_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 9
     lib.ssm_preact_bwd.restype = ctypes.c_int
+    lib.ssm_scan_fwd_gated.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 16 + [ctypes.c_size_t, _vp]
+    lib.ssm_scan_fwd_gated.restype = ctypes.c_int
+    lib.ssm_gate_bwd.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 6
+    lib.ssm_gate_bwd.restype = ctypes.c_int
     lib.ssm_cp_tail_rows.argtypes = [ctypes.POINTER(Desc)]
     lib.ssm_cp_tail_rows.restype = ctypes.c_int
     lib.ssm_cp_segment_transition.argtypes = [ctypes.POINTER(Desc)] + [_vp] * 7
@@ -182,6 +187,23 @@ def ssm_scan_step(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h, w, y, stream
     rc = lib.ssm_scan_step(ctypes.byref(desc), *[_ptr(t) for t in (
         x, dt, A_log, theta, B, C, D, lam, h, w, y)], _stream(stream))
     _check(rc, "ssm_scan_step")
+
+
+def ssm_scan_fwd_gated(desc: Desc, x, dt, A_log, theta, B, C, D, lam, h0, prev_write, z,
+                       y_gated, y_pre=None, hT=None, last_write=None, workspace=None,
+                       workspace_bytes: int = 0, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_scan_fwd_gated(ctypes.byref(desc), *[_ptr(t) for t in (
+        x, dt, A_log, theta, B, C, D, lam, h0, prev_write, z, y_gated, y_pre, hT, last_write,
+        workspace)], workspace_bytes, _stream(stream))
+    _check(rc, "ssm_scan_fwd_gated")
+
+
+def ssm_gate_bwd(desc: Desc, z, y_pre, dy_gated, dy, dz, stream=None) -> None:
+    lib = load_library()
+    rc = lib.ssm_gate_bwd(ctypes.byref(desc), *[_ptr(t) for t in (z, y_pre, dy_gated, dy, dz)],
+                          _stream(stream))
+    _check(rc, "ssm_gate_bwd")
 
 
 def ssm_cp_tail_rows(desc: Desc) -> int:

@@ -54,6 +54,8 @@ cudaError_t cp_adjoint_combine(const Params &p, int nseg, int seg, const float *
                                float *dh_end, float *dw_end, cudaStream_t st);
 cudaError_t cp_write_adjoint(const Params &p, const float *dw_end, cudaStream_t st);
 cudaError_t cp_fill_tail(const Params &p, int nv, const float *dh_end, cudaStream_t st);
+cudaError_t gate_forward(const Params &p, cudaStream_t st);
+cudaError_t gate_backward(const Params &p, const void *dyg, void *dy, void *dz, cudaStream_t st);
 }  // namespace ssm
 
 namespace {
@@ -582,22 +584,34 @@ int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, const floa
     return SSM_OK;
 }
 
-int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
-                 const float *theta, const void *B, const void *C, const float *D,
-                 const void *lambda, const float *h0, const float *prev_write, void *y,
-                 float *hT, float *last_write, void *workspace, size_t workspace_bytes,
-                 void *stream) {
+}  // extern "C"
+
+namespace {
+// Forward of both entry points; z (may be NULL: no gate) is the mixer's output gate,
+// applied in the per-coordinate tensor-core epilogue or by an elementwise pass after
+// the other chains, y_pre (may be NULL) keeps the pre-gate y.
+int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+             const float *theta, const void *B, const void *C, const float *D,
+             const void *lambda, const float *h0, const float *prev_write, const void *z,
+             void *y, void *y_pre, float *hT, float *last_write, void *workspace,
+             size_t workspace_bytes, void *stream) {
     int rc = validate_desc(d);
     if (rc) return rc;
     if (d->batch == 0) return SSM_OK;
     if (d->seqlen > 0) {
         if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
-        if ((rc = check_ptr(y, "y", d->dtype_io == SSM_BF16 ? 2 : 4))) return rc;
+        const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+        if ((rc = check_ptr(y, "y", es))) return rc;
+        if (z && (uintptr_t)z % es) return fail(SSM_ERR_ALIGN, "z is not %zu-byte aligned", es);
+        if (y_pre && (uintptr_t)y_pre % es)
+            return fail(SSM_ERR_ALIGN, "y_pre is not %zu-byte aligned", es);
     }
     ssm::Params p;
     fill_params(d, p);
     p.x = x; p.dt = dt; p.A_log = A_log; p.theta = theta; p.Bm = B; p.Cm = C; p.D = D;
     p.lam = lambda; p.h0 = h0; p.w0 = prev_write; p.y = y; p.hT = hT; p.wT = last_write;
+    p.gz = d->seqlen > 0 ? z : nullptr;
+    p.ypre = p.gz ? y_pre : nullptr;
     // chunk == 1 asks for the token-by-token recurrent kernels
     if (m1_shape(d) && ssm::m1_supported(p)) {
         const FwdWs lay = fwd_layout(d);
@@ -608,7 +622,8 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         }
         cudaStream_t st = (cudaStream_t)stream;
         profile_begin(st);
-        const cudaError_t e = ssm::m1_forward(p, kept, st);
+        cudaError_t e = ssm::m1_forward(p, kept, st);
+        if (e == cudaSuccess && p.gz) e = ssm::gate_forward(p, st);
         profile_end();
         g_last_gate = nullptr;
         g_last_route = SSM_ROUTE_CHANNEL;
@@ -638,7 +653,8 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
         const int qt = ssm::ssd_chunk_tokens(ssd_rank(d));
         p.nc = (int)((d->seqlen + qt - 1) / qt);
         profile_begin(st);
-        const cudaError_t e = ssm::ssd_forward(p, st);
+        cudaError_t e = ssm::ssd_forward(p, st);
+        if (e == cudaSuccess && p.gz) e = ssm::gate_forward(p, st);
         profile_end();
         g_last_gate = nullptr;
         g_last_route = SSM_ROUTE_SSD;
@@ -685,16 +701,67 @@ int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float
             ps.gate = gate;
             ps.gate_on = 1;
             e = ssm::simt_forward(ps, st);
+            // the tensor-core epilogue gates its own y; the recurrent chain's is gated here
+            if (e == cudaSuccess && p.gz) e = ssm::gate_forward(ps, st);
         }
         g_last_gate = gate;
         g_last_route = SSM_ROUTE_CHUNKED;
     } else {
         e = ssm::simt_forward(p, st);
+        if (e == cudaSuccess && p.gz) e = ssm::gate_forward(p, st);
         g_last_gate = nullptr;
         g_last_route = SSM_ROUTE_RECURRENT;
     }
     profile_end();
     if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_fwd launch");
+    g_last_error.clear();
+    return SSM_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                 const float *theta, const void *B, const void *C, const float *D,
+                 const void *lambda, const float *h0, const float *prev_write, void *y,
+                 float *hT, float *last_write, void *workspace, size_t workspace_bytes,
+                 void *stream) {
+    return fwd_impl(d, x, dt, A_log, theta, B, C, D, lambda, h0, prev_write, nullptr, y, nullptr,
+                    hT, last_write, workspace, workspace_bytes, stream);
+}
+
+int ssm_scan_fwd_gated(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
+                       const float *theta, const void *B, const void *C, const float *D,
+                       const void *lambda, const float *h0, const float *prev_write,
+                       const void *z, void *y_gated, void *y_pre, float *hT, float *last_write,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (d && d->batch > 0 && d->seqlen > 0) {
+        const int rc = check_ptr(z, "z", d->dtype_io == SSM_BF16 ? 2 : 4);
+        if (rc) return rc;
+    }
+    return fwd_impl(d, x, dt, A_log, theta, B, C, D, lambda, h0, prev_write, z, y_gated, y_pre,
+                    hT, last_write, workspace, workspace_bytes, stream);
+}
+
+int ssm_gate_bwd(const ssm_desc_t *d, const void *z, const void *y_pre, const void *dy_gated,
+                 void *dy, void *dz, void *stream) {
+    int rc = validate_desc(d);
+    if (rc) return rc;
+    if (d->batch == 0 || d->seqlen == 0) return SSM_OK;
+    const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
+    if ((rc = check_ptr(z, "z", es)) || (rc = check_ptr(y_pre, "y_pre", es)) ||
+        (rc = check_ptr(dy_gated, "dy_gated", es)) || (rc = check_ptr(dy, "dy", es)) ||
+        (rc = check_ptr(dz, "dz", es)))
+        return rc;
+    ssm::Params p;
+    fill_params(d, p);
+    p.gz = z;
+    p.ypre = const_cast<void *>(y_pre);
+    cudaStream_t st = (cudaStream_t)stream;
+    profile_begin(st);
+    const cudaError_t e = ssm::gate_backward(p, dy_gated, dy, dz, st);
+    profile_end();
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_gate_bwd launch");
     g_last_error.clear();
     return SSM_OK;
 }

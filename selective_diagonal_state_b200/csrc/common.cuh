@@ -28,6 +28,10 @@ struct Params {
     // forward outputs
     void *y;
     float *hT, *wT;
+    // output gate of the mixer (null: none): y_g = y * silu(z), z in y's layout; the
+    // pre-gate y is kept in ypre when set
+    const void *gz;
+    void *ypre;
     // backward outputs
     void *dx, *ddt, *dBm, *dCm, *dlam;
     float *dA_log, *dtheta, *dD, *dh0, *dw0;
