@@ -52,9 +52,11 @@ def parse():
                     help="override the batch size (small cases for profiling only)")
     ap.add_argument("--variant", default="none", choices=sorted(VARIANTS),
                     help="a variant of the workload's scan (per-token angles, ZOH write, ...)")
-    ap.add_argument("--op", default="scan", choices=["scan", "preact", "step"],
+    ap.add_argument("--op", default="scan", choices=["scan", "preact", "step", "gate"],
                     help="scan: forward + backward (the headline); preact: the dt / lambda "
-                         "pre-activations, forward + backward; step: one decoding step")
+                         "pre-activations, forward + backward; step: one decoding step; "
+                         "gate: the forward with the mixer's output gate against the plain "
+                         "forward")
     return ap.parse_args()
 
 
@@ -451,6 +453,39 @@ def run_op(args, shape):
         launches = 2
         cfg = {"batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads}
         metric = "pre-activation (softplus dt, sigmoid lambda) fwd+bwd tokens/s"
+    elif args.op == "gate":
+        inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1,
+                            with_dy=False)
+        d = scan.to_device(shape, inp)
+        desc = abi.make_desc(shape)
+        y, hT, wT = scan.alloc_fwd(shape)
+        z = torch.randn(y.shape, generator=gen, device="cuda").to(dtype)
+        ws, nb = scan.alloc_workspace(shape, abi.PASS_FWD_INFER, desc=desc)
+
+        def plain():
+            abi.ssm_scan_fwd(desc, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam, None, None,
+                             y, hT, wT, ws, nb)
+
+        def call():
+            abi.ssm_scan_fwd_gated(desc, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam,
+                                   None, None, z, y, None, hT, wT, ws, nb)
+
+        tb = tensor_bytes(shape)
+        nbytes = fwd_bytes(shape) + tb["y"]   # the scan's bytes and z
+        tokens = shape.batch * shape.seqlen
+        launches = 0   # counted by the profile session below
+        cfg = {"batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads}
+        metric = "forward with the mixer's output gate, tokens/s"
+        for _ in range(3):
+            plain()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            plain()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        plain_ms = e0.elapsed_time(e1) / args.steps
     else:
         B = args.batch or 128
         sh = shape.replace(batch=B, seqlen=1)
@@ -482,11 +517,13 @@ def run_op(args, shape):
     torch.cuda.synchronize()
     abi.ssm_scan_poll_device_error()
     # per-kernel device times (events around each launch, in a separate pass)
-    abi.ssm_scan_profile_start(launches * args.steps)
+    abi.ssm_scan_profile_start(max(launches, 16) * args.steps)
     for _ in range(args.steps):
         call()
     prof = abi.ssm_scan_profile_stop()
     kernel_ms = {n: tot / max(1, c) for n, (c, tot) in prof.items()}
+    if not launches:
+        launches = int(round(sum(c for c, _ in prof.values()) / args.steps))
     # the timed calls replay a CUDA graph of one call: these ops take microseconds,
     # so launching them from Python would time the host instead of the device
     graph = torch.cuda.CUDAGraph()
@@ -533,6 +570,7 @@ def run_op(args, shape):
                      "peak_source": "measured" if peaks.get("hbm_gbs") else "fallback"},
         "kernel_ms": kernel_ms,
         "timing": "CUDA graph replays of one call, CUDA events on the stream",
+        "plain_forward_ms": plain_ms if args.op == "gate" else None,
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }

@@ -178,10 +178,10 @@ SSM_API int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, con
  *     y_gated = y * silu(z),   silu(z) = z / (1 + e^{-z}),
  * with z in y's layout and strides (dtype_io).  Inputs and hT / last_write as
  * ssm_scan_fwd; y_pre (may be NULL) receives the pre-gate y, which
- * ssm_gate_bwd needs.  The per-coordinate tensor-core chain applies the gate in
- * its output epilogue (z read there, y_gated and y_pre leaving by TMA stores);
- * the other chains write y to y_gated and gate it in place with one
- * elementwise pass.  Same workspace as ssm_scan_fwd.
+ * ssm_gate_bwd needs.  The scan writes y to y_gated and one elementwise pass
+ * gates it in place right after, while y is still in L2 (inside the
+ * instruction-bound tensor-core epilogue the gate was measured slower).  Same
+ * workspace as ssm_scan_fwd.
  */
 SSM_API int ssm_scan_fwd_gated(const ssm_desc_t *d, const void *x, const void *dt,
                                const float *A_log, const float *theta, const void *B,

@@ -588,8 +588,8 @@ int ssm_scan_step(const ssm_desc_t *d, const void *x, const void *dt, const floa
 
 namespace {
 // Forward of both entry points; z (may be NULL: no gate) is the mixer's output gate,
-// applied in the per-coordinate tensor-core epilogue or by an elementwise pass after
-// the other chains, y_pre (may be NULL) keeps the pre-gate y.
+// applied by one elementwise pass after the chain that ran; y_pre (may be NULL)
+// keeps the pre-gate y.
 int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,
              const float *theta, const void *B, const void *C, const float *D,
              const void *lambda, const float *h0, const float *prev_write, const void *z,
@@ -701,9 +701,9 @@ int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
             ps.gate = gate;
             ps.gate_on = 1;
             e = ssm::simt_forward(ps, st);
-            // the tensor-core epilogue gates its own y; the recurrent chain's is gated here
-            if (e == cudaSuccess && p.gz) e = ssm::gate_forward(ps, st);
         }
+        // whichever chain ran wrote y: one gate pass (it reads y while it is in L2)
+        if (e == cudaSuccess && p.gz) e = ssm::gate_forward(p, st);
         g_last_gate = gate;
         g_last_route = SSM_ROUTE_CHUNKED;
     } else {

@@ -1,9 +1,10 @@
 // The mixer's output gate around the scan: y_g = y * silu(z), silu(z) = z sigmoid(z),
 // z in y's layout.  The pages' fused kernel merges the state update with the gating
 // and the output projection of the mixer ("Diagonal Equivalence in State Space
-// Models", kongchang.com: the kernel-performance paragraph); the per-coordinate
-// tensor-core forward applies the gate in its epilogue, and these elementwise passes
-// apply it after the other kernels (forward) and take its gradient (backward):
+// Models", kongchang.com: the kernel-performance paragraph).  These elementwise passes
+// apply it right after the scan's forward, while y is still in L2 (inside the
+// instruction-bound tensor-core epilogue it was measured slower), and take its
+// gradient (backward):
 //     dy = dy_g silu(z),   dz = dy_g y sigmoid(z) (1 + z (1 - sigmoid(z))).
 #include "common.cuh"
 
@@ -39,13 +40,38 @@ __device__ __forceinline__ long long gate_index(const Params &p, long long i, lo
 }
 
 // y (the scan's output, in p.y) -> y * silu(z) in place, the pre-gate y copied to
-// p.ypre when set.  Runs only on the chain the device-side range check selected
-// (p.gate), like the recurrent kernels behind the tensor-core forward.
-__global__ void __launch_bounds__(256) k_gate_fwd(Params p) {
+// p.ypre when set.  `vec`: dense layouts and 16-byte aligned tensors, 16 bytes per
+// access.
+__global__ void __launch_bounds__(256) k_gate_fwd(Params p, int vec) {
     if (gated_off(p)) return;
     const long long total = (long long)p.Bsz * p.L * p.H * p.O * p.P;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    if (vec) {
+        const int per = p.bf16 ? 8 : 4;   // elements per 16 bytes
+        const long long nv = total / per;
+        for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < nv; v += stride) {
+            const uint4 yw = reinterpret_cast<const uint4 *>(p.y)[v];
+            const uint4 zw = reinterpret_cast<const uint4 *>(p.gz)[v];
+            if (p.ypre) reinterpret_cast<uint4 *>(p.ypre)[v] = yw;
+            uint32_t yu[4] = {yw.x, yw.y, yw.z, yw.w}, zu[4] = {zw.x, zw.y, zw.z, zw.w}, o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (p.bf16) {
+                    const float y0 = __uint_as_float(yu[k] << 16), y1 = __uint_as_float(yu[k] & 0xffff0000u);
+                    const float z0 = __uint_as_float(zu[k] << 16), z1 = __uint_as_float(zu[k] & 0xffff0000u);
+                    const __nv_bfloat162 r = __floats2bfloat162_rn(y0 * z0 * gate_sigmoid(z0),
+                                                                   y1 * z1 * gate_sigmoid(z1));
+                    o[k] = *reinterpret_cast<const uint32_t *>(&r);
+                } else {
+                    const float y = __uint_as_float(yu[k]), z = __uint_as_float(zu[k]);
+                    o[k] = __float_as_uint(y * z * gate_sigmoid(z));
+                }
+            }
+            reinterpret_cast<uint4 *>(p.y)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        return;
+    }
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += stride) {
         const long long ix = gate_index(p, i, total);
         const float y = ld_io(p.y, ix, p.bf16), z = ld_io(p.gz, ix, p.bf16);
         if (p.ypre) st_io(p.ypre, ix, y, p.bf16);
@@ -72,8 +98,18 @@ static int gate_blocks(const Params &p) {
     return b < 1 ? 1 : (int)b;
 }
 
+// dense [B][L][H][O][P] with 16-byte aligned tensors and a whole number of 16-byte pieces
+static int gate_vec(const Params &p) {
+    const long long P = p.P, OP = (long long)p.O * P, HOP = p.H * OP, LHOP = p.L * HOP;
+    const long long total = p.Bsz * LHOP;
+    const int per = p.bf16 ? 8 : 4;
+    auto a16 = [](const void *q) { return q == nullptr || ((uintptr_t)q & 15) == 0; };
+    return p.sy[2] == OP && p.sy[1] == HOP && p.sy[0] == LHOP && total % per == 0 && a16(p.y) &&
+           a16(p.gz) && a16(p.ypre);
+}
+
 cudaError_t gate_forward(const Params &p, cudaStream_t st) {
-    k_gate_fwd<<<gate_blocks(p), 256, 0, st>>>(p);
+    k_gate_fwd<<<gate_blocks(p), 256, 0, st>>>(p, gate_vec(p));
     profile_mark(st, "k_gate_fwd");
     return cudaGetLastError();
 }

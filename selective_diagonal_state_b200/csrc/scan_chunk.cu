@@ -422,11 +422,11 @@ __device__ __forceinline__ void load_k(const Params &p, int c, int b, int h, int
     }
 }
 
-template <bool TOK, bool ZOH, bool GATE>
+template <bool TOK, bool ZOH>
 __global__ void __launch_bounds__(fwk::THREADS, 1)
 k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
-            const __grid_constant__ CUtensorMap tmYP, Params p) {
+            Params p) {
     if (gated_off(p)) return;
     const int BH = p.Bsz * p.H;
     const int nitems = p.nc * BH;
@@ -870,14 +870,11 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             break;
         }
         // ---- epilogue: y_t[p] = Y^T[p][t] + corr_t u_t[p], staged in the P tiles'
-        // place (phase B is done with them) and written by one TMA store; with the
-        // mixer's output gate, y_t[p] silu(z_t[p]) instead, and the pre-gate y (when
-        // kept) staged in the consumed K_c tile's place for a second store --------
-        constexpr bool gate = GATE;   // instantiated with and without the gate
+        // place (phase B is done with them) and written by one TMA store --------
         {
             const int qd = warp & 3, part = warp >> 2;   // TMEM quarter, column block
             const int pp = 16 * qd + (lane & 15);
-            unsigned char *ys = sm + fwk::SM_P, *yp = sm + fwk::SM_KT;
+            unsigned char *ys = sm + fwk::SM_P;
             constexpr int CPW = 64 / (fwk::THREADS / 128);
             for (int c16 = 0; c16 < CPW / 16; ++c16) {
                 float v[16];
@@ -888,16 +885,8 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                     for (int j = 0; j < 16; ++j) {
                         const int t = tc + j;
                         const float u = bf(sX + off_sw128(t, pp));
-                        float yv = fmaf(f32[F_CORR + t], u, v[j]);
-                        if constexpr (gate) {
-                            const float z = t0 + t < L ? ld_io(p.gz, ix_y(p, b, t0 + t, h, 0, pp), 1) : 0.f;
-                            if (p.ypre)
-                                *reinterpret_cast<__nv_bfloat16 *>(yp + off_sw128(t, pp)) =
-                                    __float2bfloat16_rn(yv);
-                            yv *= z * __frcp_rn(1.f + __expf(-z));
-                        }
                         *reinterpret_cast<__nv_bfloat16 *>(ys + off_sw128(t, pp)) =
-                            __float2bfloat16_rn(yv);
+                            __float2bfloat16_rn(fmaf(f32[F_CORR + t], u, v[j]));
                     }
                 }
             }
@@ -907,7 +896,6 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         __syncthreads();
         if (tid == 0) {   // tokens past the sequence end are clipped by the store
             tma_store_4d(&tmY, sm + fwk::SM_P, 0, h, t0, b);
-            if (GATE && p.ypre) tma_store_4d(&tmYP, sm + fwk::SM_KT, 0, h, t0, b);
             bulk_commit();
         }
         item = next;
@@ -973,8 +961,7 @@ bool chunk_fwd_supported(const Params &p) {
     auto al16 = [](const void *ptr) { return ((uintptr_t)ptr & 15) == 0; };
     auto st16 = [](long long s) { return (s * 2) % 16 == 0; };
     // y (forward) leaves by TMA stores
-    const bool yok = (!p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]))) &&
-                     al16(p.ypre);   // the kept pre-gate y leaves by a TMA store too
+    const bool yok = !p.y || (al16(p.y) && st16(p.sy[0]) && st16(p.sy[1]) && st16(p.sy[2]));
     return yok && !p.nst && p.bf16 && p.P == chunkc::PD && p.R == 1 && p.O == 1 &&
            (p.N == 64 || p.N == 128) &&
            p.nr % 8 == 0 && p.L > 0 && al16(p.x) && al16(p.Bm) && al16(p.Cm) && st16(p.sx[0]) &&
@@ -1034,18 +1021,15 @@ static cudaError_t launch_state_local(const CUtensorMap &mx, const CUtensorMap &
     return cudaSuccess;
 }
 
-template <bool TOK, bool ZOH, bool GATE>
+template <bool TOK, bool ZOH>
 static cudaError_t launch_fwd(const CUtensorMap &mx, const CUtensorMap &mb, const CUtensorMap &mc,
-                              const CUtensorMap &my, const CUtensorMap &myp, const Params &p,
-                              int grid, cudaStream_t st) {
+                              const CUtensorMap &my, const Params &p, int grid, cudaStream_t st) {
     using namespace chunkfwd;
     static bool done[64] = {};
     cudaError_t e;
-    if ((e = set_smem_once(k_chunk_fwd<TOK, ZOH, GATE>, fwk::smem_bytes<TOK>(), done)) !=
-        cudaSuccess)
+    if ((e = set_smem_once(k_chunk_fwd<TOK, ZOH>, fwk::smem_bytes<TOK>(), done)) != cudaSuccess)
         return e;
-    k_chunk_fwd<TOK, ZOH, GATE>
-        <<<grid, fwk::THREADS, fwk::smem_bytes<TOK>(), st>>>(mx, mb, mc, my, myp, p);
+    k_chunk_fwd<TOK, ZOH><<<grid, fwk::THREADS, fwk::smem_bytes<TOK>(), st>>>(mx, mb, mc, my, p);
     return cudaSuccess;
 }
 
@@ -1084,18 +1068,12 @@ cudaError_t chunk_forward(const Params &p, cudaStream_t st) {
         return e;
     const long long nitems = (long long)p.nc * p.H * p.Bsz;
     const int grid = (int)(nitems < sm_count() ? nitems : sm_count());
-    CUtensorMap my, myp;
+    CUtensorMap my;
     if (!make_map(&my, p.y, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
         return cudaErrorInvalidValue;
-    myp = my;   // the pre-gate y (same layout as y) when the gate keeps it
-    if (p.gz && p.ypre &&
-        !make_map(&myp, p.ypre, PD, p.H, p.L, p.Bsz, p.sy[2], p.sy[1], p.sy[0], PD, true))
-        return cudaErrorInvalidValue;
-    // one instantiation per angle mode, write form and output gate
     if ((e = by_variant(p, [&](auto tok, auto zoh) {
-             constexpr bool T = decltype(tok)::value, Z = decltype(zoh)::value;
-             return p.gz ? launch_fwd<T, Z, true>(mx, mb, mc, my, myp, p, grid, st)
-                         : launch_fwd<T, Z, false>(mx, mb, mc, my, myp, p, grid, st);
+             return launch_fwd<decltype(tok)::value, decltype(zoh)::value>(mx, mb, mc, my, p, grid,
+                                                                            st);
          })) != cudaSuccess)
         return e;
     profile_mark(st, "k_chunk_fwd");
