@@ -170,14 +170,14 @@ NCU_TRAFFIC_PER_ROW = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum captures at batch 2
     # (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the full Mamba-2 size; the traffic of
     # these kernels grows with the batch rows
-    ("hybridmamba", "k_chunk_fwd"): (420.69e6, "98ef2b7812470817"),
-    ("hybridmamba", "k_chunk_bwd_fused"): (603.48e6, "ea6b3d47ea94be38"),
-    ("ssd_mimo_r4", "k_ssd_fwd"): (1181.88e6, "92ad5153603b560e"),
-    ("ssd_mimo_r4", "k_ssd_bwd"): (1734.67e6, "92ad5153603b560e"),
-    ("mamba2_siso", "k_ssd_fwd"): (31.14e6, "92ad5153603b560e"),
-    ("mamba2_siso", "k_ssd_bwd"): (75.71e6, "92ad5153603b560e"),
-    ("mamba1_siso", "k_m1_fwd"): (60.46e6, "c4d8b182de0d5666"),
-    ("mamba1_siso", "k_m1_bwd"): (118.59e6, "c4d8b182de0d5666"),
+    ("hybridmamba", "k_chunk_fwd"): (420.81e6, "add66e7439dff3bc"),
+    ("hybridmamba", "k_chunk_bwd_fused"): (603.87e6, "7a7cb7c7d5e041ac"),
+    ("ssd_mimo_r4", "k_ssd_fwd"): (1198.19e6, "18e295a1b6f32936"),
+    ("ssd_mimo_r4", "k_ssd_bwd"): (1739.86e6, "18e295a1b6f32936"),
+    ("mamba2_siso", "k_ssd_fwd"): (31.04e6, "18e295a1b6f32936"),
+    ("mamba2_siso", "k_ssd_bwd"): (75.87e6, "18e295a1b6f32936"),
+    ("mamba1_siso", "k_m1_fwd"): (60.85e6, "21950b673a9f6706"),
+    ("mamba1_siso", "k_m1_bwd"): (118.78e6, "21950b673a9f6706"),
 }
 
 # sources each kernel is compiled from: a traffic entry holds only while they
