@@ -19,7 +19,6 @@ the per-head parameter gradients.
   the ZOH write on the per-coordinate tensor-core chain, one target row per
   token (O = 1, R = 4) on the scalar-decay chain; sampled heads.
 """
-import numpy as np
 import pytest
 
 import oracle

@@ -1,6 +1,5 @@
 """The pins must catch plausible mistakes: each mutant oracle (one planted error,
 compiled with -DORACLE_MUTANT=k) has to fail at least one pin."""
-import numpy as np
 import pytest
 
 import oracle
