@@ -161,7 +161,10 @@ SSM_API size_t ssm_scan_workspace_size(const ssm_desc_t *d, int pass);
  * two_endpoint == 0), h0 and prev_write (NULL = zero initial state and zero
  * left endpoint).  Writes y and, when non-NULL, hT = H_{L-1} and
  * last_write = W_{L-1} = B_{L-1} u_{L-1}; passing (hT, last_write) as
- * (h0, prev_write) of the next call continues the sequence exactly.
+ * (h0, prev_write) of the next call continues the sequence exactly.  y may be
+ * NULL (a state-only forward: hT / last_write only; the per-coordinate
+ * tensor-core chain then builds every chunk's state at once and needs the
+ * SSM_PASS_FWD workspace size).
  * stream is a cudaStream_t (NULL = legacy default stream).
  */
 SSM_API int ssm_scan_fwd(const ssm_desc_t *d, const void *x, const void *dt, const float *A_log,

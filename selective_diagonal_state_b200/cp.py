@@ -20,10 +20,10 @@ backward  1. the segment's backward with no end adjoint -> its local dh0;
              tokens; the per-head parameter gradients are summed over ranks.
 
 Every step runs in the CUDA library; this module holds the buffers, the
-order of the calls and the collectives.  Each scan runs twice (step 1 and
-step 3 of each direction); a correction pass that only reads the entering
-state out through C (instead of a second scan) is the cheaper form this
-leaves for later.  Per-token rotation angles and static rows are not sharded
+order of the calls and the collectives.  The forward's step 1 writes no y
+(a state-only forward); the backward runs twice (its step 1 for the local
+dh0).  A readout-only correction (instead of the second forward scan) and an
+adjoint-only first backward are the cheaper forms left for later.  Per-token rotation angles and static rows are not sharded
 (the trailing rows cannot pass them through unchanged).
 """
 from __future__ import annotations
@@ -103,6 +103,8 @@ class SegmentScan:
         self.desc = abi.Desc.from_buffer_copy(self.desc_ext)
         self.desc.seqlen = shape.seqlen
         self.ws_f = scan.alloc_workspace(shape, abi.PASS_FWD_INFER, device, self.desc)
+        # the state-only forward of step 1 (y not written) takes the training size
+        self.ws_s = scan.alloc_workspace(shape, abi.PASS_FWD, device, self.desc)
         self.ws_b = scan.alloc_workspace(self.ext, abi.PASS_BWD, device, self.desc_ext)
 
     # ---- inputs ---------------------------------------------------------------------
@@ -132,10 +134,11 @@ class SegmentScan:
 
     # ---- forward ----------------------------------------------------------------------
     def forward_local(self) -> Boundary:
-        """Step 1: the segment from a zero state, and its transition."""
+        """Step 1: the segment's end state from a zero state (a state-only forward:
+        no y), and its transition."""
         d, b = self.dev, self.bnd
         abi.ssm_scan_fwd(self.desc, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam, None,
-                         None, self.out[0], b.hT, b.wT, self.ws_f[0], self.ws_f[1])
+                         None, None, b.hT, b.wT, self.ws_s[0], self.ws_s[1])
         abi.ssm_cp_segment_transition(self.desc, d.dt, d.A_log, d.theta, d.lam, b.phi, b.beta0)
         return b
 

@@ -21,6 +21,7 @@ cudaError_t chunk_range_check(const Params &p, int *gate, cudaStream_t st);
 bool chunk_bwd_supported(const Params &p);
 bool chunk_fwd_supported(const Params &p);
 cudaError_t chunk_forward(const Params &p, cudaStream_t st);
+cudaError_t chunk_states(const Params &p, cudaStream_t st);
 int chunk_error_take();
 int chunk_rev_error_take();
 bool step_supported(const Params &p);
@@ -601,7 +602,12 @@ int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
     if (d->seqlen > 0) {
         if ((rc = common_inputs(d, x, dt, A_log, theta, B, C, D, lambda))) return rc;
         const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
-        if ((rc = check_ptr(y, "y", es))) return rc;
+        // y may be NULL for a state-only forward (hT / last_write), not with a gate
+        if (y || z) {
+            if ((rc = check_ptr(y, "y", es))) return rc;
+        } else if (!hT && !last_write) {
+            return fail(SSM_ERR_ARG, "y, hT and last_write are all NULL");
+        }
         if (z && (uintptr_t)z % es) return fail(SSM_ERR_ALIGN, "z is not %zu-byte aligned", es);
         if (y_pre && (uintptr_t)y_pre % es)
             return fail(SSM_ERR_ALIGN, "y_pre is not %zu-byte aligned", es);
@@ -662,8 +668,15 @@ int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
         g_last_error.clear();
         return SSM_OK;
     }
+    // state-only forward on the per-coordinate chain: every chunk's state at once and
+    // the carry pass (the backward's state rebuild), into the training workspace
+    const bool states_only = chunked && !y && d->seqlen > 0;
     if (chunked) {
         const FwdWs lay = fwd_layout(d);
+        if (states_only && (!workspace || workspace_bytes < lay.total))
+            return fail(SSM_ERR_WORKSPACE,
+                        "a state-only forward needs %zu bytes of workspace, got %zu", lay.total,
+                        workspace ? workspace_bytes : (size_t)0);
         if (!workspace || workspace_bytes < lay.total_infer)
             return fail(SSM_ERR_WORKSPACE,
                         "forward needs %zu bytes of workspace (%zu to save for the backward), got %zu",
@@ -695,7 +708,16 @@ int fwd_impl(const ssm_desc_t *d, const void *x, const void *dt, const float *A_
         ssm::Params pc = p;
         pc.gate = gate;
         pc.gate_on = 0;
-        if (e == cudaSuccess) e = ssm::chunk_forward(pc, st);
+        if (e == cudaSuccess) {
+            if (states_only) {
+                pc.sv_P = nullptr;   // nothing else of the training forward is kept
+                pc.sv_Bh = nullptr;
+                pc.sv_corr = nullptr;
+                e = ssm::chunk_states(pc, st);
+            } else {
+                e = ssm::chunk_forward(pc, st);
+            }
+        }
         if (e == cudaSuccess && fallback) {
             ssm::Params ps = p;
             ps.gate = gate;

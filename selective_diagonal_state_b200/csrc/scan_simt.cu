@@ -437,9 +437,10 @@ __global__ void __launch_bounds__(MAXT) k_fwd(Params p) {
             }
         }
         __syncthreads();
-        // y = C K - beta_{t+1} M u + D u, summed over the row groups
+        // y = C K - beta_{t+1} M u + D u, summed over the row groups (not written by a
+        // state-only forward)
         const Lanes2D l2 = lanes2d(p.P);
-        for (int row = l2.ty; row < HC * T * p.O; row += l2.ny)
+        for (int row = l2.ty; p.y && row < HC * T * p.O; row += l2.ny)
         for (int q = l2.tx; q < p.P; q += l2.W) {
             const int o = row % p.O, tt = (row / p.O) % T, hc = row / (p.O * T);
             int h = ln.hbase + hc, t = t0 + tt;

@@ -473,3 +473,25 @@ def test_backward_from_saved_states(kw):
     compare("dx", to_np(g_saved.dx), gr["dx"], dt)
     compare("dA_log", to_np(g_saved.dA_log), gr["dA_log"], dt)
     compare("ddt", to_np(g_saved.ddt), gr["ddt"], dt)
+
+
+@pytest.mark.parametrize("name", S.WORKLOAD_ORDER)
+def test_state_only_forward(name):
+    """y = NULL: only the final state and last write, equal to the full forward's."""
+    shape = S.WORKLOADS[name].replace(**REDUCED[name])
+    inp = S.make_inputs(shape, seed=120, with_state=True)
+    dev = scan.to_device(shape, inp)
+    desc = abi.make_desc(shape)
+    y_ref, hT_ref, wT_ref = scan.scan_forward(shape, dev)
+    route = abi.ssm_scan_last_route()
+    hT, wT = torch.empty_like(hT_ref), torch.empty_like(wT_ref)
+    ws, nb = scan.alloc_workspace(shape, abi.PASS_FWD, desc=desc)
+    abi.ssm_scan_fwd(desc, dev.x, dev.dt, dev.A_log, dev.theta, dev.Bm, dev.Cm, dev.D, dev.lam,
+                     dev.h0, dev.w0, None, hT, wT, ws, nb)
+    assert abi.ssm_scan_last_route() == route
+    torch.cuda.synchronize()
+    abi.ssm_scan_poll_device_error()
+    ref = oracle.scan_fwd(shape, inp)
+    compare("hT", to_np(hT), ref["hT"], shape.dtype_io)
+    compare("last_write", to_np(wT), ref["wT"], shape.dtype_io)
+    assert float((hT - hT_ref).abs().max()) <= 1e-3 * max(1.0, float(hT_ref.abs().max()))
