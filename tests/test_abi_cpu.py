@@ -257,3 +257,22 @@ def test_sequence_sharding_calls_validate_before_launch(lib):
     # transition: n_pairs above 64
     wide = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(n_real=0, n_pairs=65))
     assert lib.ssm_cp_segment_transition(ctypes.byref(wide), *([FAKE] * 6), None) == -2
+
+
+def test_gated_forward_and_state_only_forward_validate(lib):
+    """The gated forward needs z and y; a plain forward may drop y (state only)
+    but not every output."""
+    d = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"])
+    ins = [FAKE] * 10   # x, dt, A_log, theta, B, C, D, lambda, h0, prev_write
+    # z missing
+    rc = lib.ssm_scan_fwd_gated(ctypes.byref(d), *ins, None, FAKE, None, FAKE, None, None, 0, None)
+    assert rc == -1 and "z" in lib.ssm_scan_last_error().decode()
+    # y_gated missing
+    rc = lib.ssm_scan_fwd_gated(ctypes.byref(d), *ins, FAKE, None, None, FAKE, None, None, 0, None)
+    assert rc == -1 and "y" in lib.ssm_scan_last_error().decode()
+    # state-only forward with nothing to write
+    rc = lib.ssm_scan_fwd(ctypes.byref(d), *ins, None, None, None, None, 0, None)
+    assert rc == -1 and "NULL" in lib.ssm_scan_last_error().decode()
+    # the gate's backward checks every pointer
+    rc = lib.ssm_gate_bwd(ctypes.byref(d), FAKE, None, FAKE, FAKE, FAKE, None)
+    assert rc == -1 and "y_pre" in lib.ssm_scan_last_error().decode()
