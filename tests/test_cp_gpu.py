@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import oracle
-from selective_diagonal_state_b200 import abi, cp
+from selective_diagonal_state_b200 import abi, cp, scan
 from selective_diagonal_state_b200 import synthetic as S
 from tests.parity_util import compare, to_np
 
@@ -92,3 +92,35 @@ def test_one_segment_is_the_plain_scan():
     compare("y", to_np(fwd[0][0]), ref["y"], shape.dtype_io)
     gr = oracle.scan_bwd(shape, inp, inp["dy"])
     compare("dx", to_np(grads[0].dx[:, :shape.seqlen]), gr["dx"], shape.dtype_io)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(angle_mode=S.ANGLE_PER_TOKEN), dict(n_static=16),
+                                dict(two_endpoint=0)])
+def test_segment_transition(kw):
+    """phi of a segment is the product of its tokens' transitions: e^{a sum dt} on a
+    real row (e^{a L} on a static one), times a rotation by theta sum dt (or by the
+    sum of the per-token angles) on a pair; beta_0 the first token's (1 - lam) dt."""
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=3, ngroups=3, seqlen=77, **kw)
+    inp = S.make_inputs(shape, seed=51)
+    dev = scan.to_device(shape, inp)
+    nmode = shape.n_real + shape.n_pairs
+    phi = torch.empty((2, 3, nmode, 2), dtype=torch.float32, device="cuda")
+    beta0 = torch.empty((2, 3), dtype=torch.float32, device="cuda")
+    abi.ssm_cp_segment_transition(abi.make_desc(shape), dev.dt, dev.A_log, dev.theta, dev.lam,
+                                  phi, beta0)
+    torch.cuda.synchronize()
+    a = -np.exp(inp["A_log"].astype(np.float64))                     # [H, nmode]
+    sdt = inp["dt"].astype(np.float64).sum(axis=1)                    # [B, H]
+    mag = np.exp(a[None] * sdt[:, :, None])
+    mag[:, :, :shape.n_static] = np.exp(a[None, :, :shape.n_static] * shape.seqlen)
+    if shape.angle_mode == S.ANGLE_PER_TOKEN:
+        ang = inp["theta"].astype(np.float64).sum(axis=1)             # [B, H, np]
+    else:
+        ang = inp["theta"].astype(np.float64)[None] * sdt[:, :, None]
+    ref = np.zeros((2, 3, nmode, 2))
+    ref[:, :, :shape.n_real, 0] = mag[:, :, :shape.n_real]
+    ref[:, :, shape.n_real:, 0] = mag[:, :, shape.n_real:] * np.cos(ang)
+    ref[:, :, shape.n_real:, 1] = mag[:, :, shape.n_real:] * np.sin(ang)
+    np.testing.assert_allclose(to_np(phi), ref, rtol=2e-4, atol=1e-6)
+    b0 = ((1.0 - inp["lam"][:, 0]) * inp["dt"][:, 0]) if shape.two_endpoint else np.zeros((2, 3))
+    np.testing.assert_allclose(to_np(beta0), b0, rtol=1e-5, atol=1e-7)
