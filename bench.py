@@ -170,12 +170,12 @@ NCU_TRAFFIC_PER_ROW = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum captures at batch 2
     # (HybridMamba, Mamba-1), 1 (SSD-MIMO) and the full Mamba-2 size; the traffic of
     # these kernels grows with the batch rows
-    ("hybridmamba", "k_chunk_fwd"): (420.81e6, "add66e7439dff3bc"),
+    ("hybridmamba", "k_chunk_fwd"): (421.30e6, "45bd0acc068dc92e"),
     ("hybridmamba", "k_chunk_bwd_fused"): (603.87e6, "7a7cb7c7d5e041ac"),
-    ("ssd_mimo_r4", "k_ssd_fwd"): (1198.19e6, "18e295a1b6f32936"),
-    ("ssd_mimo_r4", "k_ssd_bwd"): (1739.86e6, "18e295a1b6f32936"),
-    ("mamba2_siso", "k_ssd_fwd"): (31.04e6, "18e295a1b6f32936"),
-    ("mamba2_siso", "k_ssd_bwd"): (75.87e6, "18e295a1b6f32936"),
+    ("ssd_mimo_r4", "k_ssd_fwd"): (1182.60e6, "b0388a47d161e1c7"),
+    ("ssd_mimo_r4", "k_ssd_bwd"): (1739.96e6, "b0388a47d161e1c7"),
+    ("mamba2_siso", "k_ssd_fwd"): (31.07e6, "b0388a47d161e1c7"),
+    ("mamba2_siso", "k_ssd_bwd"): (75.35e6, "b0388a47d161e1c7"),
     ("mamba1_siso", "k_m1_fwd"): (60.85e6, "21950b673a9f6706"),
     ("mamba1_siso", "k_m1_bwd"): (118.78e6, "21950b673a9f6706"),
 }

@@ -927,7 +927,31 @@ k_chunk_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 // kernels take the call instead (their chain is launched behind the same gate).
 constexpr float RANGE_LOG2 = 100.f;
 
-__global__ void k_range_check(Params p, int *gate) {
+constexpr int RANGE_HMAX = 256;   // heads whose largest rate a block tabulates once
+
+__device__ __forceinline__ float largest_log_rate(const Params &p, int h) {
+    float amax = p.A_log[h * p.ndec];
+    for (int m = 1; m < p.ndec; ++m) amax = fmaxf(amax, p.A_log[h * p.ndec + m]);
+    return amax;
+}
+
+__global__ void __launch_bounds__(256) k_range_check(Params p, int *gate) {
+    // the largest log-rate of every head, once per block: one warp per head, its lanes
+    // reading consecutive modes (fmaxf drops NaN unless every rate of the head is NaN,
+    // as the sequential maximum does)
+    __shared__ float s_amax[RANGE_HMAX];
+    const bool tab = p.H <= RANGE_HMAX;
+    if (tab) {
+        const int lane = threadIdx.x & 31;
+        for (int h = threadIdx.x >> 5; h < p.H; h += blockDim.x >> 5) {
+            float v = __int_as_float(0x7fffffff);
+            for (int m = lane; m < p.ndec; m += 32) v = fmaxf(v, p.A_log[h * p.ndec + m]);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) s_amax[h] = v;
+        }
+        __syncthreads();
+    }
     const int nsb = (p.L + 15) / 16;
     const long long items = (long long)p.Bsz * nsb * p.H;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < items;
@@ -935,8 +959,7 @@ __global__ void k_range_check(Params p, int *gate) {
         const int h = (int)(i % p.H);
         const long long r = i / p.H;
         const int sb = (int)(r % nsb), b = (int)(r / nsb);
-        float amax = p.A_log[h * p.ndec];
-        for (int m = 1; m < p.ndec; ++m) amax = fmaxf(amax, p.A_log[h * p.ndec + m]);
+        const float amax = tab ? s_amax[h] : largest_log_rate(p, h);
         float span = 0.f;
         for (int k = 0; k < 16; ++k) {
             const int t = 16 * sb + k;

@@ -937,62 +937,131 @@ __global__ void __launch_bounds__(256) k_bwd_units_local(Params p) {
 }
 
 // carry the block totals across time blocks: per (b, h), one thread per mode
-__global__ void __launch_bounds__(256) k_bwd_units_carry(Params p) {
+constexpr int CARRY_GROUP = 32;   // time blocks per group when the carries are exact
+
+// sum over the block's threads of v[0 .. nthr) by warp 0 (lane-strided partials, then a
+// shuffle tree: a fixed order); the total is valid in lane 0
+__device__ __forceinline__ float sum_modes(const float *v, int nthr, int lane) {
+    float acc = 0.f;
+    for (int k = lane; k < nthr; k += 32) acc += v[k];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+}
+
+__host__ __device__ inline int carry_threads(const Params &p) {   // one per mode
+    const int n = ((p.nr + p.np + 31) / 32) * 32;
+    return n < 32 ? 32 : n;
+}
+
+__global__ void __launch_bounds__(1024) k_bwd_units_carry(Params p) {
     if (gated_off(p)) return;
     extern __shared__ __align__(16) float smem[];
     const int h = blockIdx.x, b = blockIdx.y;
-    const int m = threadIdx.x, nthr = blockDim.x;
+    // thread (mode m, slice s): with exact carries the slices take interleaved time blocks
+    const int nthr = carry_threads(p), nsub = blockDim.x / nthr;
+    const int m = threadIdx.x % nthr, sl = threadIdx.x / nthr;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NTB = ntb_of(p), nmode = p.nr + p.np;
+    const long long bstride = 4 * (long long)nmode + 2;
+    const float *blk0 = p.ws_blk + ((long long)b * p.H + h) * NTB * bstride;
+    float *blkc = p.ws_blkc + ((long long)b * p.H + h) * NTB;
     const ModeInfo mi = mode_info(p, h, m);
-    float *s_c = smem;  // [nthr]
+    float *s_c = smem;  // [nthr], or [CARRY_GROUP][nthr] when the carries are exact
     float car = 0.f, cai = 0.f, dA = 0.f, dth = 0.f, dD = 0.f;
-    for (int tb = NTB - 1; tb >= 0; --tb) {
-        const float *blk = p.ws_blk + (((long long)b * p.H + h) * NTB + tb) * (4 * (long long)nmode + 2);
-        const float sdt = blk[4 * nmode + 0];
-        if (p.ws_qb && mi.valid) {
-            // exact carry from the chunk boundary: sum_p conj(Gbar) A K_prev at the next block start
-            car = 0.f;
-            cai = 0.f;
-            if (tb + 1 < NTB) {
-                const float *q = p.ws_qb + (((long long)b * p.H + h) * p.nc + (tb + 1)) * 4 * (long long)p.N;
-                for (int w2 = 0; w2 < 4; ++w2) {   // four partial sums over column blocks of p
-                    car += q[w2 * p.N + mi.n0];
-                    if (mi.pair) cai += q[w2 * p.N + mi.n0 + 1];
+    if (p.ws_qb) {
+        // The chunked chain left the exact carry at every block start (sum_p conj(Gbar) A
+        // K_prev at the next block's start, four partial sums over column blocks of p), so
+        // the blocks are independent: groups of CARRY_GROUP blocks, the slices forming
+        // their modes' terms of interleaved blocks, then one warp per block summing the
+        // modes.
+        const float *q0 = p.ws_qb + ((long long)b * p.H + h) * p.nc * 4 * (long long)p.N;
+        for (int g0 = NTB - 1; g0 >= 0; g0 -= CARRY_GROUP) {
+            const int ng = min(CARRY_GROUP, g0 + 1);
+#pragma unroll 4
+            for (int j = sl; j < ng; j += nsub) {
+                const int tb = g0 - j;
+                const float *blk = blk0 + tb * bstride;
+                float contrib = 0.f;
+                if (mi.valid) {
+                    float cr = 0.f, ci = 0.f;
+                    if (tb + 1 < NTB) {
+                        const float *q = q0 + (long long)(tb + 1) * 4 * p.N;
+                        for (int w2 = 0; w2 < 4; ++w2) {
+                            cr += q[w2 * p.N + mi.n0];
+                            if (mi.pair) ci += q[w2 * p.N + mi.n0 + 1];
+                        }
+                    }
+                    const bool stat = m < p.nst;
+                    const float sdt = blk[4 * nmode + 0];
+                    const float ntok = (float)(min(p.L, (tb + 1) * TBL) - tb * TBL);
+                    dA += blk[4 * m + 2] + cr * (stat ? ntok : sdt);
+                    if (mi.pair) dth += blk[4 * m + 3] - ci * sdt;
+                    contrib = stat ? 0.f : mi.a * cr + (mi.pair ? -mi.w * ci : 0.f);
+                }
+                s_c[j * nthr + m] = contrib;
+                if (m == 0) dD += blk[4 * nmode + 1];
+            }
+            __syncthreads();
+            for (int j = warp; j < ng; j += blockDim.x >> 5) {
+                const float acc = sum_modes(s_c + j * nthr, nthr, lane);
+                if (lane == 0) blkc[g0 - j] = acc;
+            }
+            __syncthreads();
+        }
+        // the slices' partial sums, added in slice order
+        s_c[sl * nthr + m] = dA;
+        s_c[(nsub + sl) * nthr + m] = dth;
+        s_c[(2 * nsub + sl) * nthr + m] = dD;
+        __syncthreads();
+        if (sl == 0) {
+            dA = dth = dD = 0.f;
+            for (int k = 0; k < nsub; ++k) {
+                dA += s_c[k * nthr + m];
+                dth += s_c[(nsub + k) * nthr + m];
+                dD += s_c[(2 * nsub + k) * nthr + m];
+            }
+        }
+        __syncthreads();
+    } else {
+        for (int tb = NTB - 1; tb >= 0; --tb) {
+            const float *blk = blk0 + tb * bstride;
+            const float sdt = blk[4 * nmode + 0];
+            float contrib = 0.f;
+            if (mi.valid) {
+                const bool stat = m < p.nst;
+                // static rows: the carried sum counts once per token of the block
+                const float ntok = (float)(min(p.L, (tb + 1) * TBL) - tb * TBL);
+                dA += blk[4 * m + 2] + car * (stat ? ntok : sdt);
+                if (mi.pair) dth += blk[4 * m + 3] - cai * sdt;
+                contrib = stat ? 0.f : mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
+                // per-token angles: the angle's gradient takes the carry at every token
+                if (mi.pair && p.angle_tok && cai != 0.f) {
+                    const int tend = min(p.L, (tb + 1) * TBL);
+                    for (int t = tb * TBL; t < tend; ++t)
+                        p.dtheta[ix_th(p, b, t, h, m - p.nr)] -= cai;
                 }
             }
-        }
-        float contrib = 0.f;
-        if (mi.valid) {
-            const bool stat = m < p.nst;
-            // static rows: the carried sum counts once per token of the block
-            const float ntok = (float)(min(p.L, (tb + 1) * TBL) - tb * TBL);
-            dA += blk[4 * m + 2] + car * (stat ? ntok : sdt);
-            if (mi.pair) dth += blk[4 * m + 3] - cai * sdt;
-            contrib = stat ? 0.f : mi.a * car + (mi.pair ? -mi.w * cai : 0.f);
-            // per-token angles: the chunked backward subtracts the exact carry itself
-            if (mi.pair && p.angle_tok && cai != 0.f && !p.ws_qb) {
-                const int tend = min(p.L, (tb + 1) * TBL);
-                for (int t = tb * TBL; t < tend; ++t)
-                    p.dtheta[ix_th(p, b, t, h, m - p.nr)] -= cai;
+            s_c[m] = contrib;
+            __syncthreads();
+            if (warp == 0) {
+                const float acc = sum_modes(s_c, nthr, lane);
+                if (lane == 0) {
+                    blkc[tb] = acc;
+                    dD += blk[4 * nmode + 1];
+                }
             }
+            if (mi.valid) {
+                car += blk[4 * m + 0];
+                cai += blk[4 * m + 1];
+            }
+            __syncthreads();
         }
-        s_c[m] = contrib;
-        __syncthreads();
-        if (m == 0) {
-            float acc = 0.f;
-            for (int j = 0; j < nthr; ++j) acc += s_c[j];
-            p.ws_blkc[((long long)b * p.H + h) * NTB + tb] = acc;
-            dD += blk[4 * nmode + 1];
-        }
-        if (mi.valid && !p.ws_qb) {
-            car += blk[4 * m + 0];
-            cai += blk[4 * m + 1];
-        }
-        __syncthreads();
     }
     float *part = p.ws_par + ((long long)b * p.H + h) * npar_of(p);
-    s_c[m] = dA;
+    if (sl == 0) s_c[m] = dA;
     __syncthreads();
+    if (sl != 0) return;
     if (p.per_coord) {
         if (mi.valid) part[m] = dA;
     } else if (m == 0) {
@@ -1313,7 +1382,13 @@ static cudaError_t bwd_finalize(const Params &p, cudaStream_t st, bool local, bo
         profile_mark(st, "k_bwd_units_local");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    k_bwd_units_carry<<<dim3(p.H, p.Bsz), nthr, (size_t)nthr * 4, st>>>(p);
+    {
+        // with exact carries, up to four slices of the modes' threads take interleaved blocks
+        const int cthr = carry_threads(p);
+        const int nsub = p.ws_qb ? (1024 / cthr < 4 ? 1024 / cthr : 4) : 1;
+        k_bwd_units_carry<<<dim3(p.H, p.Bsz), cthr * nsub,
+                            (size_t)(p.ws_qb ? CARRY_GROUP : 1) * cthr * 4, st>>>(p);
+    }
     profile_mark(st, "k_bwd_units_carry");
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long total = (long long)p.Bsz * p.L * p.H;

@@ -1492,17 +1492,38 @@ __global__ void k_ssd_tokens(Params p) {
     }
 }
 
-// Per-head parameter gradients (fixed summation order over batch rows and
-// chunks): dA_log = a sum dt drho, dD = sum <dy, x>.
-__global__ void k_ssd_params(Params p) {
-    for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < p.H; h += gridDim.x * blockDim.x) {
-        float sa = 0.f, sd = 0.f;
-        for (int b = 0; b < p.Bsz; ++b)
-            for (int c = 0; c < p.nc; ++c) {
-                const long long u = chunkc::bhc(p, b, h, c);
-                sa += p.sd_par[2 * u];
-                sd += p.sd_par[2 * u + 1];
-            }
+// Per-head parameter gradients: dA_log = a sum dt drho, dD = sum <dy, x>, summed over
+// batch rows and chunks by one block per head in a fixed order (thread-strided
+// partials, a shuffle tree per warp, then the warps in order).
+constexpr int SSD_PARAM_THREADS = 256;
+
+__global__ void __launch_bounds__(SSD_PARAM_THREADS) k_ssd_params(Params p) {
+    __shared__ float s_part[2][SSD_PARAM_THREADS / 32];
+    const int h = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = p.Bsz * p.nc;
+    float sa = 0.f, sd = 0.f;
+    for (int k = threadIdx.x; k < n; k += SSD_PARAM_THREADS) {
+        const int b = k / p.nc, c = k - b * p.nc;
+        const long long u = chunkc::bhc(p, b, h, c);
+        sa += p.sd_par[2 * u];
+        sd += p.sd_par[2 * u + 1];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, o);
+        sd += __shfl_xor_sync(0xffffffffu, sd, o);
+    }
+    if (lane == 0) {
+        s_part[0][warp] = sa;
+        s_part[1][warp] = sd;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        sa = sd = 0.f;
+        for (int w = 0; w < SSD_PARAM_THREADS / 32; ++w) {
+            sa += s_part[0][w];
+            sd += s_part[1][w];
+        }
         const float a = -expf(__ldg(p.A_log + h * p.ndec));
         p.dA_log[h * p.ndec] = a * sa;
         if (p.dD) p.dD[h] = p.R == p.O ? sd : 0.f;   // D is used only when O == R
@@ -1738,7 +1759,7 @@ cudaError_t ssd_backward(const Params &p, cudaStream_t st) {
         profile_mark(st, "k_ssd_group_sum");
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    k_ssd_params<<<(p.H + 127) / 128, 128, 0, st>>>(p);
+    k_ssd_params<<<p.H, SSD_PARAM_THREADS, 0, st>>>(p);
     profile_mark(st, "k_ssd_params");
     return cudaGetLastError();
 }
