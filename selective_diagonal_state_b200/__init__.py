@@ -8,6 +8,8 @@ and SSD-MIMO rank-R routing, as a C-ABI CUDA library (``include/ssm_scan.h``).
 Modules:
   ``abi``        ctypes binding with the C entry-point names
   ``scan``       torch device-buffer helpers around the binding
+  ``cp``         sequence sharding: segment scans joined through boundary values
+  ``dist``       data-parallel plumbing (parameter-gradient all-reduce)
   ``synthetic``  seeded input generators (no scan arithmetic)
   ``build``      nvcc build of ``libssm_scan.so`` for sm_100a
 """
