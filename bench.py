@@ -52,11 +52,14 @@ def parse():
                     help="override the batch size (small cases for profiling only)")
     ap.add_argument("--variant", default="none", choices=sorted(VARIANTS),
                     help="a variant of the workload's scan (per-token angles, ZOH write, ...)")
-    ap.add_argument("--op", default="scan", choices=["scan", "preact", "step", "gate"],
+    ap.add_argument("--op", default="scan", choices=["scan", "preact", "step", "gate", "cp"],
                     help="scan: forward + backward (the headline); preact: the dt / lambda "
                          "pre-activations, forward + backward; step: one decoding step; "
                          "gate: the forward with the mixer's output gate against the plain "
-                         "forward")
+                         "forward; cp: the sequence-sharded training step with every "
+                         "segment on this GPU, against the whole-sequence step")
+    ap.add_argument("--segments", type=int, default=4,
+                    help="--op cp: segments the sequence is cut into")
     return ap.parse_args()
 
 
@@ -405,7 +408,7 @@ def _peaks():
 
 
 def run_op(args, shape):
-    """--op preact | step: a row beyond the hot path on one GPU, timed like the
+    """--op preact | step | gate | cp: a row beyond the hot path on one GPU, timed like the
     scan (CUDA events on the launching stream around K calls after W warm-up
     calls, clocks sampled meanwhile, L2 flushed between calls when the data fit
     in it) against the HBM roofline of its algorithmic bytes.
@@ -415,12 +418,17 @@ def run_op(args, shape):
       ddt (and the logits, dlambda), writes dz (and dlambda_logit).
     step:   one ssm_scan_step for a decoding batch (--batch, default 128 rows) of
       the workload's heads: the fp32 state (and the previous write) read and
-      written once, one token's x, dt, lambda, B, C read and y written."""
+      written once, one token's x, dt, lambda, B, C read and y written.
+    gate:   the forward with the output gate, beside the plain forward.
+    cp:     the sequence cut into --segments segments, each scanned by its own
+      buffers (state-only forward, exact forward, two backwards and the boundary
+      combines) one after another on this GPU, beside the whole-sequence step;
+      the roofline counts the whole sequence's scan bytes once."""
     import torch
 
     from selective_diagonal_state_b200 import abi, scan
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:
-        raise SystemExit("--op preact / step run on one GPU")
+        raise SystemExit("--op preact / step / gate / cp run on one GPU")
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
     abi.load_library()
@@ -476,6 +484,51 @@ def run_op(args, shape):
         launches = 0   # counted by the profile session below
         cfg = {"batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads}
         metric = "forward with the mixer's output gate, tokens/s"
+        for _ in range(3):
+            plain()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            plain()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        plain_ms = e0.elapsed_time(e1) / args.steps
+    elif args.op == "cp":
+        from selective_diagonal_state_b200 import cp
+        nseg = args.segments
+        if nseg < 1 or nseg > shape.seqlen:
+            raise SystemExit("--segments must be in [1, seqlen]")
+        inp = S.make_inputs(shape, seed=S.WORKLOAD_ORDER.index(shape.name) + 1)
+        segs = []
+        for k in range(nseg):
+            a, b_ = cp.segment_bounds(shape.seqlen, nseg, k)
+            sg = cp.SegmentScan(shape.replace(seqlen=b_ - a))
+            sg.load(inp, a, b_)
+            segs.append(sg)
+
+        def call():
+            cp.run_sharded(segs)
+
+        # the whole-sequence training step on the same inputs, for the overhead
+        d = scan.to_device(shape, inp)
+        desc = abi.make_desc(shape)
+        out, grads = scan.alloc_fwd(shape), scan.alloc_bwd(shape)
+        wsf = scan.alloc_workspace(shape, abi.PASS_FWD, desc=desc)
+        wsb = scan.alloc_workspace(shape, abi.PASS_BWD, desc=desc)
+
+        def plain():
+            scan.scan_forward(shape, d, out=out, desc=desc, workspace=wsf)
+            scan.scan_backward(shape, d, grads=grads, workspace=wsb, desc=desc, saved=wsf)
+
+        nbytes = fwd_bytes(shape) + bwd_bytes(shape)   # the whole sequence's scan bytes
+        tokens = shape.batch * shape.seqlen
+        launches = 0   # counted by the profile session below
+        cfg = {"batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads,
+               "segments": nseg,
+               "emulation": "every segment's kernels on this GPU one after another; the "
+                            "all-gathers are stacks of the segments' boundary values"}
+        metric = "sequence-sharded training step (all segments on one GPU) tokens/s"
         for _ in range(3):
             plain()
         torch.cuda.synchronize()
@@ -571,6 +624,7 @@ def run_op(args, shape):
         "kernel_ms": kernel_ms,
         "timing": "CUDA graph replays of one call, CUDA events on the stream",
         "plain_forward_ms": plain_ms if args.op == "gate" else None,
+        "plain_step_ms": plain_ms if args.op == "cp" else None,
         "gpu_launches": launches * args.steps,
         "clocks": clk,
     }

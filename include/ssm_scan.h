@@ -222,8 +222,8 @@ SSM_API int ssm_scan_bwd(const ssm_desc_t *d, const void *x, const void *dt, con
 /*
  * Backward that reuses the forward's chunk states: identical to ssm_scan_bwd,
  * except that fwd_workspace is the workspace of a preceding ssm_scan_fwd call
- * with the same descriptor and the same inputs (x, dt, A_log, theta, B, lambda,
- * h0, prev_write), left unchanged since.  The tensor-core backward then reads
+ * with the same descriptor and the same inputs (x, dt, A_log, theta, B, C, D,
+ * lambda, h0, prev_write; dy may differ), left unchanged since.  The tensor-core backward then reads
  * the states entering every 64-token chunk from it instead of recomputing them
  * (the training step "forward saving chunk states, then backward").  For
  * descriptors whose forward needs no workspace it behaves as ssm_scan_bwd.

@@ -21,8 +21,8 @@ backward  1. the segment's backward with no end adjoint -> its local dh0;
 
 Every step runs in the CUDA library; this module holds the buffers, the
 order of the calls and the collectives.  The forward's step 1 writes no y
-(a state-only forward); the backward runs twice (its step 1 for the local
-dh0).  A readout-only correction (instead of the second forward scan) and an
+(a state-only forward); the exact forward keeps its chunk states, and both
+backwards (step 1 for the local dh0, step 3 the exact one) read them.  A readout-only correction (instead of the second forward scan) and an
 adjoint-only first backward are the cheaper forms left for later.  Per-token rotation angles and static rows are not sharded
 (the trailing rows cannot pass them through unchanged).
 """
@@ -102,9 +102,11 @@ class SegmentScan:
         self.desc_ext = abi.make_desc(self.ext)
         self.desc = abi.Desc.from_buffer_copy(self.desc_ext)
         self.desc.seqlen = shape.seqlen
-        self.ws_f = scan.alloc_workspace(shape, abi.PASS_FWD_INFER, device, self.desc)
         # the state-only forward of step 1 (y not written) takes the training size
         self.ws_s = scan.alloc_workspace(shape, abi.PASS_FWD, device, self.desc)
+        # the exact forward runs over the extended rows and keeps its chunk states,
+        # which both backwards read
+        self.ws_f = scan.alloc_workspace(self.ext, abi.PASS_FWD, device, self.desc_ext)
         self.ws_b = scan.alloc_workspace(self.ext, abi.PASS_BWD, device, self.desc_ext)
 
     # ---- inputs ---------------------------------------------------------------------
@@ -144,25 +146,38 @@ class SegmentScan:
 
     def forward_exact(self, nseg, seg, gathered: Boundary, h0=None, w0=None):
         """Step 3: the entering state from the gathered boundaries, then the
-        segment from it.  Returns (y of the segment's tokens, hT, last write)."""
+        segment from it, over the extended rows (the trailing rows pass the state
+        through unchanged and change no y of the segment's tokens), keeping the
+        chunk states for the backward.  Returns (y of the segment's tokens, hT,
+        last write); the last write is the segment's own, from step 1."""
         d = self.dev
         abi.ssm_cp_state_combine(self.desc, nseg, seg, gathered.hT, gathered.wT, gathered.phi,
                                  gathered.beta0, h0, w0, self.h_in, self.w_in)
+        # the trailing rows' inputs as the backward reads them (its end adjoint only
+        # changes their dy, which the forward does not read)
+        abi.ssm_cp_fill_tail(self.desc, d.x, d.dt, d.Bm, d.Cm, d.lam, d.dy, None)
         y, hT, wT = self.out
-        abi.ssm_scan_fwd(self.desc, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam,
+        abi.ssm_scan_fwd(self.desc_ext, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam,
                          self.h_in, self.w_in, y, hT, wT, self.ws_f[0], self.ws_f[1])
-        return y[:, :self.shape.seqlen], hT, wT
+        return y[:, :self.shape.seqlen], hT, self.bnd.wT
 
     # ---- backward ---------------------------------------------------------------------
     def _backward(self, dh_end):
+        # reads the chunk states the exact forward kept (same inputs, entering
+        # state and trailing rows; only the trailing rows' dy differ)
         d, g = self.dev, self.grads
         abi.ssm_cp_fill_tail(self.desc, d.x, d.dt, d.Bm, d.Cm, d.lam, d.dy, dh_end)
-        abi.ssm_scan_bwd(self.desc_ext, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam,
-                         self.h_in, self.w_in, d.dy, g.dx, g.ddt, g.dA_log, g.dtheta, g.dBm,
-                         g.dCm, g.dD, g.dlam, g.dh0, g.dw0, self.ws_b[0], self.ws_b[1])
+        args = (self.desc_ext, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam, self.h_in,
+                self.w_in, d.dy, g.dx, g.ddt, g.dA_log, g.dtheta, g.dBm, g.dCm, g.dD, g.dlam,
+                g.dh0, g.dw0)
+        if self.ws_f[1]:
+            abi.ssm_scan_bwd_saved(*args, self.ws_f[0], self.ws_f[1], self.ws_b[0], self.ws_b[1])
+        else:   # a forward that keeps nothing (the recurrent kernels)
+            abi.ssm_scan_bwd(*args, self.ws_b[0], self.ws_b[1])
 
     def backward_local(self):
-        """Step 1: the backward with no end adjoint -> the local dh0."""
+        """Step 1: the backward with no end adjoint -> the local dh0 (after
+        ``forward_exact``, whose kept chunk states it reads)."""
         self._backward(None)
         self.dh0_loc.copy_(self.grads.dh0)
         return self.dh0_loc

@@ -185,36 +185,51 @@ __global__ void __launch_bounds__(cpk::THREADS)
 // head, dB += sum over the group's heads of dw_end u^T.  Thread (b, h, r, q) for dx,
 // then (b, g, r, n) for dB.
 __global__ void __launch_bounds__(cpk::THREADS) k_cp_write_adjoint(Params p, const float *dw_end) {
+    // dx of the last token: one thread per (b, h, r, q), the sum over the state rows
     const int t = p.L - 1;
     const long long nx = (long long)p.Bsz * p.H * p.R * p.P;
-    const long long nb = (long long)p.Bsz * p.G * p.R * p.N;
-    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < nx + nb;
+    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < nx;
          u += (long long)gridDim.x * blockDim.x) {
-        if (u < nx) {
-            const int q = (int)(u % p.P);
-            long long r_ = u / p.P;
-            const int r = (int)(r_ % p.R);
-            r_ /= p.R;
-            const int h = (int)(r_ % p.H), b = (int)(r_ / p.H), g = h / p.hpg;
-            float acc = 0.f;
-            for (int n = 0; n < p.N; ++n)
-                acc = fmaf(ld_io(p.Bm, ix_B(p, b, t, g, r, n), p.bf16), dw_end[ix_st(p, b, h, n, q)], acc);
-            const long long ix = ix_x(p, b, t, h, r, q);
-            st_io(p.dx, ix, ld_io(p.dx, ix, p.bf16) + acc, p.bf16);
-        } else {
-            const long long v = u - nx;
-            const int n = (int)(v % p.N);
-            long long r_ = v / p.N;
-            const int r = (int)(r_ % p.R);
-            r_ /= p.R;
-            const int g = (int)(r_ % p.G), b = (int)(r_ / p.G);
-            float acc = 0.f;
-            for (int h = g * p.hpg; h < (g + 1) * p.hpg; ++h)
-                for (int q = 0; q < p.P; ++q)
-                    acc = fmaf(dw_end[ix_st(p, b, h, n, q)], ld_io(p.x, ix_x(p, b, t, h, r, q), p.bf16), acc);
-            const long long ib = ix_B(p, b, t, g, r, n);
-            st_io(p.dBm, ib, ld_io(p.dBm, ib, p.bf16) + acc, p.bf16);
-        }
+        const int q = (int)(u % p.P);
+        long long r_ = u / p.P;
+        const int r = (int)(r_ % p.R);
+        r_ /= p.R;
+        const int h = (int)(r_ % p.H), b = (int)(r_ / p.H), g = h / p.hpg;
+        float acc = 0.f;
+        for (int n = 0; n < p.N; ++n)
+            acc = fmaf(ld_io(p.Bm, ix_B(p, b, t, g, r, n), p.bf16), dw_end[ix_st(p, b, h, n, q)], acc);
+        const long long ix = ix_x(p, b, t, h, r, q);
+        st_io(p.dx, ix, ld_io(p.dx, ix, p.bf16) + acc, p.bf16);
+    }
+}
+
+// dB of the last token: one block per (b, g, r, n), the sum over the group's
+// (head, channel) pairs in a fixed order (thread-strided partials, a shuffle
+// tree per warp, then the warps in order)
+__global__ void __launch_bounds__(cpk::THREADS) k_cp_write_adjoint_b(Params p, const float *dw_end) {
+    __shared__ float part[cpk::THREADS / 32];
+    const int t = p.L - 1;
+    int u = blockIdx.x;
+    const int n = u % p.N;
+    u /= p.N;
+    const int r = u % p.R;
+    u /= p.R;
+    const int g = u % p.G, b = u / p.G;
+    const int cnt = p.hpg * p.P;
+    float acc = 0.f;
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const int h = g * p.hpg + i / p.P, q = i % p.P;
+        acc = fmaf(dw_end[ix_st(p, b, h, n, q)], ld_io(p.x, ix_x(p, b, t, h, r, q), p.bf16), acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float sum = 0.f;
+        for (int w = 0; w < cpk::THREADS / 32; ++w) sum += part[w];
+        const long long ib = ix_B(p, b, t, g, r, n);
+        st_io(p.dBm, ib, ld_io(p.dBm, ib, p.bf16) + sum, p.bf16);
     }
 }
 
@@ -228,35 +243,45 @@ __global__ void __launch_bounds__(cpk::THREADS) k_cp_write_adjoint(Params p, con
 // trailing row adds to the parameters is weighted by its dt (zero) or its input
 // (zero).
 __global__ void __launch_bounds__(cpk::THREADS) k_cp_fill_tail(Params p, int nv, const float *dh_end) {
+    // one block per trailing row (b, v); its threads take each field's elements with
+    // the innermost index fastest, so the stores of a warp are contiguous
     const int nsets = nv / p.N;
-    const long long per_tok = (long long)p.Bsz * p.H;   // (b, h) pairs per trailing token
-    const long long units = (long long)nv * per_tok;
-    for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
-         u += (long long)gridDim.x * blockDim.x) {
-        const int v = (int)(u / per_tok);
-        const long long bh = u - (long long)v * per_tok;
-        const int b = (int)(bh / p.H), h = (int)(bh - (long long)b * p.H);
-        const int g = h / p.hpg, t = p.L + v, s = v / p.N, k = v - s * p.N;
-        st_io((void *)p.dt, ix_dt(p, b, t, h), 0.f, p.bf16);
-        if (p.two_ep) st_io((void *)p.lam, ix_lam(p, b, t, h), 1.f, p.bf16);
-        for (int r = 0; r < p.R; ++r)
-            for (int q = 0; q < p.P; ++q) st_io((void *)p.x, ix_x(p, b, t, h, r, q), 0.f, p.bf16);
-        for (int o = 0; o < p.O; ++o)
-            for (int q = 0; q < p.P; ++q) {
-                float val = 0.f;
-                if (o == 0) {
-                    const float d = dh_end ? dh_end[ix_st(p, b, h, k, q)] : 0.f;
-                    const float hi = p.bf16 ? __bfloat162float(__float2bfloat16_rn(d)) : d;
-                    val = (nsets == 1 || s == 0) ? hi : d - hi;
-                }
-                st_io((void *)p.dy, ix_y(p, b, t, h, o, q), val, p.bf16);
+    const int rows = p.Bsz * nv;
+    const int nx = p.H * p.R * p.P, ny = p.H * p.O * p.P;
+    const int nb = p.G * p.R * p.N, nc = p.G * p.O * p.N;
+    for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+        const int b = row / nv, v = row - b * nv, t = p.L + v;
+        const int s = v / p.N, k = v - s * p.N;
+        // dt = 0 and lambda = 1
+        for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
+            st_io((void *)p.dt, ix_dt(p, b, t, h), 0.f, p.bf16);
+            if (p.two_ep) st_io((void *)p.lam, ix_lam(p, b, t, h), 1.f, p.bf16);
+        }
+        // x = 0
+        for (int i = threadIdx.x; i < nx; i += blockDim.x) {
+            const int q = i % p.P, r1 = i / p.P, rr = r1 % p.R, h = r1 / p.R;
+            st_io((void *)p.x, ix_x(p, b, t, h, rr, q), 0.f, p.bf16);
+        }
+        // dy: in target rank 0 of trailing row v = s N + k, row k of the end adjoint
+        // (s = 0: its io-precision value; s = 1: the remainder), zero elsewhere
+        for (int i = threadIdx.x; i < ny; i += blockDim.x) {
+            const int q = i % p.P, r1 = i / p.P, o = r1 % p.O, h = r1 / p.O;
+            float val = 0.f;
+            if (o == 0) {
+                const float d = dh_end ? dh_end[ix_st(p, b, h, k, q)] : 0.f;
+                const float hi = p.bf16 ? __bfloat162float(__float2bfloat16_rn(d)) : d;
+                val = (nsets == 1 || s == 0) ? hi : d - hi;
             }
-        if (h == g * p.hpg) {   // B and C rows once per group
-            for (int r = 0; r < p.R; ++r)
-                for (int n = 0; n < p.N; ++n) st_io((void *)p.Bm, ix_B(p, b, t, g, r, n), 0.f, p.bf16);
-            for (int o = 0; o < p.O; ++o)
-                for (int n = 0; n < p.N; ++n)
-                    st_io((void *)p.Cm, ix_C(p, b, t, g, o, n), (o == 0 && n == k) ? 1.f : 0.f, p.bf16);
+            st_io((void *)p.dy, ix_y(p, b, t, h, o, q), val, p.bf16);
+        }
+        // B = 0; C = e_k in target rank 0
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+            const int n = i % p.N, r1 = i / p.N, rr = r1 % p.R, g = r1 / p.R;
+            st_io((void *)p.Bm, ix_B(p, b, t, g, rr, n), 0.f, p.bf16);
+        }
+        for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+            const int n = i % p.N, r1 = i / p.N, o = r1 % p.O, g = r1 / p.O;
+            st_io((void *)p.Cm, ix_C(p, b, t, g, o, n), (o == 0 && n == k) ? 1.f : 0.f, p.bf16);
         }
     }
 }
@@ -296,16 +321,22 @@ cudaError_t cp_adjoint_combine(const Params &p, int nseg, int seg, const float *
 
 cudaError_t cp_write_adjoint(const Params &p, const float *dw_end, cudaStream_t st) {
     if (p.L < 1) return cudaSuccess;
-    const long long units = (long long)p.Bsz * p.H * p.R * p.P + (long long)p.Bsz * p.G * p.R * p.N;
+    const long long units = (long long)p.Bsz * p.H * p.R * p.P;
     k_cp_write_adjoint<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, dw_end);
     profile_mark(st, "k_cp_write_adjoint");
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long nbo = (long long)p.Bsz * p.G * p.R * p.N;
+    if (nbo == 0) return cudaSuccess;
+    k_cp_write_adjoint_b<<<(unsigned)nbo, cpk::THREADS, 0, st>>>(p, dw_end);
+    profile_mark(st, "k_cp_write_adjoint_b");
     return cudaGetLastError();
 }
 
 cudaError_t cp_fill_tail(const Params &p, int nv, const float *dh_end, cudaStream_t st) {
-    const long long units = (long long)nv * p.Bsz * p.H;
-    if (units == 0) return cudaSuccess;
-    k_cp_fill_tail<<<cp_blocks(units), cpk::THREADS, 0, st>>>(p, nv, dh_end);
+    const long long rows = (long long)nv * p.Bsz;
+    if (rows == 0) return cudaSuccess;
+    k_cp_fill_tail<<<(int)(rows < 148 * 16 ? rows : 148 * 16), cpk::THREADS, 0, st>>>(p, nv, dh_end);
     profile_mark(st, "k_cp_fill_tail");
     return cudaGetLastError();
 }
