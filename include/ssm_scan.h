@@ -389,8 +389,12 @@ SSM_API int ssm_cp_adjoint_combine(const ssm_desc_t *d, int nseg, int seg, const
  * and its dy row 0 carries part s of dh_end[:, k, :] (NULL = zero).  A
  * backward over seqlen + tail tokens then has dh_end as the adjoint of the
  * segment's end state, and the trailing rows add nothing to the parameter
- * gradients (they are weighted by dt or x).  Not for per-token angles or
- * static rows (SSM_ERR_UNSUPPORTED). */
+ * gradients (they are weighted by dt or x).  A forward over the seqlen + tail
+ * rows after this call gives the segment's own y and hT unchanged (its last
+ * write is the trailing rows' zero write; the segment's own is that of its
+ * local forward), and since calls with another dh_end change only dy, the
+ * backwards may read that forward's workspace (ssm_scan_bwd_saved).  Not for
+ * per-token angles or static rows (SSM_ERR_UNSUPPORTED). */
 SSM_API int ssm_cp_fill_tail(const ssm_desc_t *d, void *x, void *dt, void *B, void *C,
                              void *lambda, void *dy, const float *dh_end, void *stream);
 
