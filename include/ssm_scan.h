@@ -393,8 +393,10 @@ SSM_API int ssm_cp_adjoint_combine(const ssm_desc_t *d, int nseg, int seg, const
  * rows after this call gives the segment's own y and hT unchanged (its last
  * write is the trailing rows' zero write; the segment's own is that of its
  * local forward), and since calls with another dh_end change only dy, the
- * backwards may read that forward's workspace (ssm_scan_bwd_saved).  Not for
- * per-token angles or static rows (SSM_ERR_UNSUPPORTED). */
+ * backwards may read that forward's workspace (ssm_scan_bwd_saved).  With x,
+ * dt, B, C and lambda all NULL only the dy rows are written (the other rows as
+ * an earlier call left them).  Not for per-token angles or static rows
+ * (SSM_ERR_UNSUPPORTED). */
 SSM_API int ssm_cp_fill_tail(const ssm_desc_t *d, void *x, void *dt, void *B, void *C,
                              void *lambda, void *dy, const float *dh_end, void *stream);
 

@@ -166,7 +166,8 @@ class SegmentScan:
         # reads the chunk states the exact forward kept (same inputs, entering
         # state and trailing rows; only the trailing rows' dy differ)
         d, g = self.dev, self.grads
-        abi.ssm_cp_fill_tail(self.desc, d.x, d.dt, d.Bm, d.Cm, d.lam, d.dy, dh_end)
+        # the trailing rows' other inputs were written before the exact forward
+        abi.ssm_cp_fill_tail(self.desc, None, None, None, None, None, d.dy, dh_end)
         args = (self.desc_ext, d.x, d.dt, d.A_log, d.theta, d.Bm, d.Cm, d.D, d.lam, self.h_in,
                 self.w_in, d.dy, g.dx, g.ddt, g.dA_log, g.dtheta, g.dBm, g.dCm, g.dD, g.dlam,
                 g.dh0, g.dw0)

@@ -1180,10 +1180,15 @@ int ssm_cp_fill_tail(const ssm_desc_t *d, void *x, void *dt, void *B, void *C, v
         return fail(SSM_ERR_UNSUPPORTED,
                     "ssm_cp_fill_tail: static rows (their transition does not vanish with dt)");
     const size_t es = d->dtype_io == SSM_BF16 ? 2 : 4;
-    if ((rc = check_ptr(x, "x", es)) || (rc = check_ptr(dt, "dt", es)) ||
-        (rc = check_ptr(B, "B", es)) || (rc = check_ptr(C, "C", es)) || (rc = check_ptr(dy, "dy", es)))
-        return rc;
-    if (d->two_endpoint && (rc = check_ptr(lambda, "lambda", es))) return rc;
+    // x, dt, B, C and lambda all NULL: only the dy rows (the rest as an earlier call left them)
+    const bool dy_only = !x && !dt && !B && !C && !lambda;
+    if ((rc = check_ptr(dy, "dy", es))) return rc;
+    if (!dy_only) {
+        if ((rc = check_ptr(x, "x", es)) || (rc = check_ptr(dt, "dt", es)) ||
+            (rc = check_ptr(B, "B", es)) || (rc = check_ptr(C, "C", es)))
+            return rc;
+        if (d->two_endpoint && (rc = check_ptr(lambda, "lambda", es))) return rc;
+    }
     ssm::Params p;
     fill_params(d, p);
     p.x = x; p.dt = dt; p.Bm = B; p.Cm = C; p.lam = lambda; p.dy = dy;

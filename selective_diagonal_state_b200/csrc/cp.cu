@@ -249,16 +249,17 @@ __global__ void __launch_bounds__(cpk::THREADS) k_cp_fill_tail(Params p, int nv,
     const int rows = p.Bsz * nv;
     const int nx = p.H * p.R * p.P, ny = p.H * p.O * p.P;
     const int nb = p.G * p.R * p.N, nc = p.G * p.O * p.N;
+    const bool all = p.x != nullptr;   // else only the dy rows
     for (int row = blockIdx.x; row < rows; row += gridDim.x) {
         const int b = row / nv, v = row - b * nv, t = p.L + v;
         const int s = v / p.N, k = v - s * p.N;
         // dt = 0 and lambda = 1
-        for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
+        for (int h = threadIdx.x; all && h < p.H; h += blockDim.x) {
             st_io((void *)p.dt, ix_dt(p, b, t, h), 0.f, p.bf16);
             if (p.two_ep) st_io((void *)p.lam, ix_lam(p, b, t, h), 1.f, p.bf16);
         }
         // x = 0
-        for (int i = threadIdx.x; i < nx; i += blockDim.x) {
+        for (int i = threadIdx.x; all && i < nx; i += blockDim.x) {
             const int q = i % p.P, r1 = i / p.P, rr = r1 % p.R, h = r1 / p.R;
             st_io((void *)p.x, ix_x(p, b, t, h, rr, q), 0.f, p.bf16);
         }
@@ -275,11 +276,11 @@ __global__ void __launch_bounds__(cpk::THREADS) k_cp_fill_tail(Params p, int nv,
             st_io((void *)p.dy, ix_y(p, b, t, h, o, q), val, p.bf16);
         }
         // B = 0; C = e_k in target rank 0
-        for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        for (int i = threadIdx.x; all && i < nb; i += blockDim.x) {
             const int n = i % p.N, r1 = i / p.N, rr = r1 % p.R, g = r1 / p.R;
             st_io((void *)p.Bm, ix_B(p, b, t, g, rr, n), 0.f, p.bf16);
         }
-        for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+        for (int i = threadIdx.x; all && i < nc; i += blockDim.x) {
             const int n = i % p.N, r1 = i / p.N, o = r1 % p.O, g = r1 / p.O;
             st_io((void *)p.Cm, ix_C(p, b, t, g, o, n), (o == 0 && n == k) ? 1.f : 0.f, p.bf16);
         }

@@ -254,6 +254,12 @@ def test_sequence_sharding_calls_validate_before_launch(lib):
     for kw in (dict(angle_mode=S.ANGLE_PER_TOKEN), dict(n_static=8)):
         dd = abi.make_desc(sh.replace(**kw))
         assert lib.ssm_cp_fill_tail(ctypes.byref(dd), *([FAKE] * 7), None) == -2
+    # the fill takes every input row buffer or none of them (dy only), and always dy
+    assert lib.ssm_cp_fill_tail(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                None) == -1
+    assert "x" in lib.ssm_scan_last_error().decode()
+    assert lib.ssm_cp_fill_tail(ctypes.byref(d), *([None] * 5), None, None, None) == -1
+    assert "dy" in lib.ssm_scan_last_error().decode()
     # transition: n_pairs above 64
     wide = abi.make_desc(S.WORKLOADS["tiny_hybrid_fp32"].replace(n_real=0, n_pairs=65))
     assert lib.ssm_cp_segment_transition(ctypes.byref(wide), *([FAKE] * 6), None) == -2
