@@ -37,6 +37,11 @@ CASES = [
     ("ssd_mimo_r4", dict(batch=1, nheads=2, ngroups=2, seqlen=200), 2),
     # channel scan
     ("mamba1_siso", dict(batch=2, nheads=64, seqlen=150), 3),
+    # eight segments of 65 tokens (a full chunk and a one-token chunk each)
+    ("hybridmamba", dict(batch=1, nheads=2, ngroups=2, seqlen=520), 8),
+    # segments of one and two tokens, on the tensor-core chain and the recurrent kernels
+    ("hybridmamba", dict(batch=1, nheads=2, ngroups=2, seqlen=10), 8),
+    ("tiny_hybrid_fp32", dict(seqlen=9), 8),
 ]
 
 
