@@ -28,6 +28,30 @@ namespace cpk {
 constexpr int THREADS = 256;
 }
 
+// phi of mode m of head h from the segment's dt sum S (with per-token angles, ang_tok
+// is the pair's summed angle): e^{a S} on a dynamic real row, e^{a L} on a static one,
+// and e^{a S} times the rotation by the summed angle on a pair
+__device__ __forceinline__ void cp_mode_phi(const Params &p, int h, int m, float S, float ang_tok,
+                                            float &re, float &im) {
+    const float a = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
+    im = 0.f;
+    if (m < p.nr) {
+        re = expf(a * (m < p.nst ? (float)p.L : S));   // static rows: e^{a} per token
+    } else {
+        const float ang = p.angle_tok ? ang_tok : p.theta[h * p.np + (m - p.nr)] * S;
+        float sn, cs;
+        sincosf(ang, &sn, &cs);
+        const float mag = expf(a * S);
+        re = mag * cs;
+        im = mag * sn;
+    }
+}
+
+__device__ __forceinline__ float cp_beta0(const Params &p, int b, int h) {
+    if (!p.two_ep || p.L < 1) return 0.f;
+    return (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), p.bf16)) * ld_io(p.dt, ix_dt(p, b, 0, h), p.bf16);
+}
+
 // Phi of every (b, h, mode) of the segment ([B][H][nmode][2], (re, im)) and
 // beta_0 ([B][H]).  One CTA per (b, h): the sums of dt (and of the per-token
 // angles) over the segment in a fixed order, then one thread per mode.
@@ -55,34 +79,51 @@ __global__ void __launch_bounds__(cpk::THREADS) k_cp_transition(Params p, float 
     const float S = red[0];
     const int nmode = p.nr + p.np;
     for (int m = tid; m < nmode; m += cpk::THREADS) {
-        const float a = -expf(p.A_log[h * p.ndec + (p.per_coord ? m : 0)]);
-        float re, im = 0.f;
-        if (m < p.nr) {
-            re = expf(a * (m < p.nst ? (float)p.L : S));   // static rows: e^{a} per token
-        } else {
-            const int j = m - p.nr;
-            float ang;
-            if (p.angle_tok) {
-                ang = 0.f;
-                for (int w = 0; w < cpk::THREADS / 32; ++w) ang += th[j * 8 + w];
-            } else {
-                ang = p.theta[h * p.np + j] * S;
-            }
-            float sn, cs;
-            sincosf(ang, &sn, &cs);
-            const float mag = expf(a * S);
-            re = mag * cs;
-            im = mag * sn;
-        }
+        float ang = 0.f;
+        if (p.angle_tok && m >= p.nr)
+            for (int w = 0; w < cpk::THREADS / 32; ++w) ang += th[(m - p.nr) * 8 + w];
+        float re, im;
+        cp_mode_phi(p, h, m, S, ang, re, im);
         float *o = phi + ((long long)bh * nmode + m) * 2;
         o[0] = re;
         o[1] = im;
     }
-    if (tid == 0) {
-        float b0 = 0.f;
-        if (p.two_ep && p.L > 0)
-            b0 = (1.f - ld_io(p.lam, ix_lam(p, b, 0, h), p.bf16)) * ld_io(p.dt, ix_dt(p, b, 0, h), p.bf16);
-        beta0[bh] = b0;
+    if (tid == 0) beta0[bh] = cp_beta0(p, b, h);
+}
+
+// The same for many heads (no per-token angles): one CTA per (32-head tile, b),
+// the lane a head (so a warp's dt loads are contiguous), the warps interleaved
+// tokens, their partial sums added in warp order.
+__global__ void __launch_bounds__(cpk::THREADS) k_cp_transition_cols(Params p, float *phi,
+                                                                     float *beta0) {
+    constexpr int NW = cpk::THREADS / 32;
+    __shared__ float part[NW][32];
+    __shared__ float s_sum[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h0 = blockIdx.x * 32, b = blockIdx.y, h = h0 + lane;
+    float s = 0.f;
+    if (h < p.H) {
+#pragma unroll 4
+        for (int t = warp; t < p.L; t += NW) s += ld_io(p.dt, ix_dt(p, b, t, h), p.bf16);
+    }
+    part[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0) {
+        float S = 0.f;
+        for (int w = 0; w < NW; ++w) S += part[w][lane];
+        s_sum[lane] = S;
+        if (h < p.H) beta0[(long long)b * p.H + h] = cp_beta0(p, b, h);
+    }
+    __syncthreads();
+    const int nmode = p.nr + p.np;
+    const int nh = min(32, p.H - h0);
+    for (int i = threadIdx.x; i < nh * nmode; i += blockDim.x) {
+        const int hl = i / nmode, m = i - hl * nmode;
+        float re, im;
+        cp_mode_phi(p, h0 + hl, m, s_sum[hl], 0.f, re, im);
+        float *o = phi + (((long long)b * p.H + h0 + hl) * nmode + m) * 2;
+        o[0] = re;
+        o[1] = im;
     }
 }
 
@@ -295,8 +336,13 @@ static int cp_blocks(long long units) {
 
 cudaError_t cp_transition(const Params &p, float *phi, float *beta0, cudaStream_t st) {
     if (p.Bsz * p.H == 0) return cudaSuccess;
-    k_cp_transition<<<p.Bsz * p.H, cpk::THREADS, 0, st>>>(p, phi, beta0);
-    profile_mark(st, "k_cp_transition");
+    if (p.H >= 256 && !(p.angle_tok && p.np)) {   // many heads: a CTA per 32-head tile
+        k_cp_transition_cols<<<dim3((p.H + 31) / 32, p.Bsz), cpk::THREADS, 0, st>>>(p, phi, beta0);
+        profile_mark(st, "k_cp_transition_cols");
+    } else {
+        k_cp_transition<<<p.Bsz * p.H, cpk::THREADS, 0, st>>>(p, phi, beta0);
+        profile_mark(st, "k_cp_transition");
+    }
     return cudaGetLastError();
 }
 

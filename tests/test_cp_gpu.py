@@ -42,6 +42,8 @@ CASES = [
     # segments of one and two tokens, on the tensor-core chain and the recurrent kernels
     ("hybridmamba", dict(batch=1, nheads=2, ngroups=2, seqlen=10), 8),
     ("tiny_hybrid_fp32", dict(seqlen=9), 8),
+    # many channels: the head-tiled segment transition
+    ("mamba1_siso", dict(batch=1, nheads=320, seqlen=64), 2),
 ]
 
 
@@ -100,17 +102,21 @@ def test_one_segment_is_the_plain_scan():
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(angle_mode=S.ANGLE_PER_TOKEN), dict(n_static=16),
-                                dict(two_endpoint=0)])
+                                dict(two_endpoint=0),
+                                # many heads: the head-tiled kernel, a partial last tile
+                                dict(nheads=300, ngroups=300)])
 def test_segment_transition(kw):
     """phi of a segment is the product of its tokens' transitions: e^{a sum dt} on a
     real row (e^{a L} on a static one), times a rotation by theta sum dt (or by the
     sum of the per-token angles) on a pair; beta_0 the first token's (1 - lam) dt."""
-    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, nheads=3, ngroups=3, seqlen=77, **kw)
+    kw = dict(dict(nheads=3, ngroups=3), **kw)
+    shape = S.WORKLOADS["hybridmamba"].replace(batch=2, seqlen=77, **kw)
+    H = shape.nheads
     inp = S.make_inputs(shape, seed=51)
     dev = scan.to_device(shape, inp)
     nmode = shape.n_real + shape.n_pairs
-    phi = torch.empty((2, 3, nmode, 2), dtype=torch.float32, device="cuda")
-    beta0 = torch.empty((2, 3), dtype=torch.float32, device="cuda")
+    phi = torch.empty((2, H, nmode, 2), dtype=torch.float32, device="cuda")
+    beta0 = torch.empty((2, H), dtype=torch.float32, device="cuda")
     abi.ssm_cp_segment_transition(abi.make_desc(shape), dev.dt, dev.A_log, dev.theta, dev.lam,
                                   phi, beta0)
     torch.cuda.synchronize()
@@ -122,10 +128,10 @@ def test_segment_transition(kw):
         ang = inp["theta"].astype(np.float64).sum(axis=1)             # [B, H, np]
     else:
         ang = inp["theta"].astype(np.float64)[None] * sdt[:, :, None]
-    ref = np.zeros((2, 3, nmode, 2))
+    ref = np.zeros((2, H, nmode, 2))
     ref[:, :, :shape.n_real, 0] = mag[:, :, :shape.n_real]
     ref[:, :, shape.n_real:, 0] = mag[:, :, shape.n_real:] * np.cos(ang)
     ref[:, :, shape.n_real:, 1] = mag[:, :, shape.n_real:] * np.sin(ang)
     np.testing.assert_allclose(to_np(phi), ref, rtol=2e-4, atol=1e-6)
-    b0 = ((1.0 - inp["lam"][:, 0]) * inp["dt"][:, 0]) if shape.two_endpoint else np.zeros((2, 3))
+    b0 = ((1.0 - inp["lam"][:, 0]) * inp["dt"][:, 0]) if shape.two_endpoint else np.zeros((2, H))
     np.testing.assert_allclose(to_np(beta0), b0, rtol=1e-5, atol=1e-7)
