@@ -1,5 +1,6 @@
 """Host side of sequence sharding (no GPU): segment bounds, the shapes that are
-refused, and the all-gather of boundary values over world-size-2 gloo ranks."""
+refused, the all-gather of boundary values over world-size-2 gloo ranks, and
+the segment composition itself on the fp64 oracle."""
 import os
 
 import pytest
@@ -63,3 +64,59 @@ def test_all_gather_stacks_in_rank_order():
     for r in range(2):
         g = res[r]
         assert [row[0][0] for row in g] == [1.0, 2.0]   # segment k at index k
+
+
+def _segment_inputs(inp, a, b, h0=None, w0=None):
+    tok = ("x", "dt", "Bm", "Cm", "lam", "dy")
+    sub = {k: (v[:, a:b] if k in tok and v is not None else v) for k, v in inp.items()}
+    sub["h0"], sub["w0"] = h0, w0
+    return sub
+
+
+def _apply_phi(X, mag, ang, nr):
+    """Phi applied to states [B][H][N][P]: real rows scaled by e^{a S}; a pair's
+    (re, im) rows multiplied by e^{a S} e^{i angle}."""
+    import numpy as np
+    Y = X.copy()
+    Y[:, :, :nr] *= mag[:, :, :nr, None]
+    re, im = X[:, :, nr::2], X[:, :, nr + 1::2]
+    m, c, s = mag[:, :, nr:, None], np.cos(ang)[..., None], np.sin(ang)[..., None]
+    Y[:, :, nr::2] = m * (c * re - s * im)
+    Y[:, :, nr + 1::2] = m * (s * re + c * im)
+    return Y
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 5])
+def test_segment_composition_on_the_oracle(nseg):
+    """The composition the sharded scan rests on, on the fp64 oracle alone:
+    segments scanned from a zero state and joined by
+    K_in(k+1) = Phi_k (K_in(k) + beta_0(k) W_in(k)) + hT_loc(k), W_in(k+1) = last
+    write of segment k (Phi_k: e^{a sum dt} and the rotation by theta sum dt;
+    beta_0(k) = (1 - lambda) dt of the segment's first token) give the whole
+    sequence's final state and last write, and each segment scanned again from
+    (K_in(k), W_in(k)) gives the whole sequence's y on its tokens."""
+    import numpy as np
+
+    import oracle
+    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=41)
+    inp = S.make_inputs(shape, seed=61, with_state=True)
+    whole = oracle.scan_fwd(shape, inp)
+    a_rate = -np.exp(inp["A_log"].astype(np.float64))                 # [H, nmode]
+    theta = inp["theta"].astype(np.float64)                            # [H, n_pairs]
+    K, W = inp["h0"].astype(np.float64), inp["w0"].astype(np.float64)
+    for k in range(nseg):
+        a, b = cp.segment_bounds(shape.seqlen, nseg, k)
+        seg = shape.replace(seqlen=b - a)
+        # the exact forward of the segment from what enters it
+        y = oracle.scan_fwd(seg, _segment_inputs(inp, a, b, K, W))["y"]
+        np.testing.assert_allclose(y, whole["y"][:, a:b], rtol=1e-10, atol=1e-12)
+        loc = oracle.scan_fwd(seg, _segment_inputs(inp, a, b))
+        S_dt = inp["dt"][:, a:b].astype(np.float64).sum(axis=1)        # [B, H]
+        mag = np.exp(a_rate[None] * S_dt[:, :, None])                  # [B, H, nmode]
+        ang = theta[None] * S_dt[:, :, None]                           # [B, H, n_pairs]
+        lam0, dt0 = (inp[k][:, a].astype(np.float64) for k in ("lam", "dt"))
+        beta0 = (1.0 - lam0) * dt0                                     # [B, H]
+        K = _apply_phi(K + beta0[:, :, None, None] * W, mag, ang, shape.n_real) + loc["hT"]
+        W = loc["wT"]
+    np.testing.assert_allclose(K, whole["hT"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(W, whole["wT"], rtol=1e-10, atol=1e-12)
