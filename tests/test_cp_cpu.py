@@ -120,3 +120,88 @@ def test_segment_composition_on_the_oracle(nseg):
         W = loc["wT"]
     np.testing.assert_allclose(K, whole["hT"], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(W, whole["wT"], rtol=1e-10, atol=1e-12)
+
+
+def test_backward_composition_on_the_oracle():
+    """The backward half on the fp64 oracle alone.  The adjoint entering the end of
+    segment k is dK_end(k) = dh0_loc(k+1) + Phi_{k+1}^T dK_end(k+1), where
+    dh0_loc(k+1) is that segment's dh0 with no end adjoint.  Fed through trailing
+    rows (dt = x = B = 0, lambda = 1, C rows e_n, dy rows the end adjoint), with
+    beta_0(k+1) dK_end(k) added as the adjoint of the segment's last write, each
+    segment's backward gives the whole sequence's gradients on its tokens.  The
+    parameter gradients are the segments' sums, and dh0 / dprev_write are those
+    of the first segment."""
+    import numpy as np
+
+    import oracle
+    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=37)
+    nseg, N, nr = 3, shape.nstate, shape.n_real
+    inp = S.make_inputs(shape, seed=62, with_state=True)
+    whole = oracle.scan_bwd(shape, inp, inp["dy"])
+    a_rate = -np.exp(inp["A_log"].astype(np.float64))
+    theta = inp["theta"].astype(np.float64)
+    bounds = [cp.segment_bounds(shape.seqlen, nseg, k) for k in range(nseg)]
+    f64 = lambda v: v.astype(np.float64)  # noqa: E731
+
+    def phi_of(a, b):
+        S_dt = f64(inp["dt"][:, a:b]).sum(axis=1)
+        return np.exp(a_rate[None] * S_dt[:, :, None]), theta[None] * S_dt[:, :, None]
+
+    def beta0_of(a):
+        return (1.0 - f64(inp["lam"][:, a])) * f64(inp["dt"][:, a])
+
+    # forward: the states entering every segment (the forward composition)
+    K, W = f64(inp["h0"]), f64(inp["w0"])
+    enter = []
+    for k, (a, b) in enumerate(bounds):
+        enter.append((K, W))
+        loc = oracle.scan_fwd(shape.replace(seqlen=b - a), _segment_inputs(inp, a, b))
+        mag, ang = phi_of(a, b)
+        K = _apply_phi(K + beta0_of(a)[:, :, None, None] * W, mag, ang, nr) + loc["hT"]
+        W = loc["wT"]
+    # backward: local dh0, then the end adjoints from the last segment back
+    dh0_loc = [oracle.scan_bwd(shape.replace(seqlen=b - a), _segment_inputs(inp, a, b, *enter[k]),
+                               inp["dy"][:, a:b])["dh0"] for k, (a, b) in enumerate(bounds)]
+    dK_end = [None] * nseg
+    dK_end[-1] = np.zeros_like(dh0_loc[0])
+    for k in range(nseg - 2, -1, -1):
+        a1, b1 = bounds[k + 1]
+        mag, ang = phi_of(a1, b1)
+        dK_end[k] = dh0_loc[k + 1] + _apply_phi(dK_end[k + 1], mag, -ang, nr)   # Phi^T
+    sums = {n: 0.0 for n in ("dA_log", "dtheta", "dD")}
+    for k, (a, b) in enumerate(bounds):
+        L = b - a
+        ext = shape.replace(seqlen=L + N)
+        sub = _segment_inputs(inp, a, b, *enter[k])
+        pad = lambda v: np.concatenate([v, np.zeros((v.shape[0], N) + v.shape[2:], v.dtype)],  # noqa: E731
+                                       axis=1)
+        for name in ("x", "dt", "Bm", "Cm"):
+            sub[name] = pad(sub[name])
+        sub["lam"] = np.concatenate([sub["lam"], np.ones((shape.batch, N, shape.nheads),
+                                                         sub["lam"].dtype)], axis=1)
+        for n in range(N):
+            sub["Cm"][:, L + n, :, 0, n] = 1.0
+        dy = pad(f64(inp["dy"][:, a:b]))                                # fp64: the end adjoint rows
+        dy[:, L:, :, 0, :] = np.transpose(dK_end[k], (0, 2, 1, 3))     # row n <- dK_end[:, :, n]
+        g = oracle.scan_bwd(ext, sub, dy)
+        # the last write's adjoint: dx += B^T dW, dB += sum over the group's heads of dW x^T
+        dW = (beta0_of(bounds[k + 1][0])[:, :, None, None] * dK_end[k]) if k + 1 < nseg \
+            else np.zeros_like(dK_end[k])
+        hpg = shape.nheads // shape.ngroups
+        for h in range(shape.nheads):
+            gi = h // hpg
+            for r in range(shape.rank_in):
+                Bl = f64(inp["Bm"][:, b - 1, gi, r])                    # [B, N]
+                xl = f64(inp["x"][:, b - 1, h, r])                      # [B, P]
+                g["dx"][:, L - 1, h, r] += np.einsum("bn,bnp->bp", Bl, dW[:, h])
+                g["dBm"][:, L - 1, gi, r] += np.einsum("bnp,bp->bn", dW[:, h], xl)
+        for name in ("dx", "ddt", "dBm", "dCm", "dlam"):
+            np.testing.assert_allclose(g[name][:, :L], whole[name][:, a:b], rtol=1e-9, atol=1e-11,
+                                       err_msg=f"segment {k} {name}")
+        for name in sums:
+            sums[name] = sums[name] + g[name]
+        if k == 0:
+            np.testing.assert_allclose(g["dh0"], whole["dh0"], rtol=1e-9, atol=1e-11)
+            np.testing.assert_allclose(g["dw0"], whole["dw0"], rtol=1e-9, atol=1e-11)
+    for name, v in sums.items():
+        np.testing.assert_allclose(v, whole[name], rtol=1e-9, atol=1e-11, err_msg=name)
