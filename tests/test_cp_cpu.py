@@ -86,8 +86,10 @@ def _apply_phi(X, mag, ang, nr):
     return Y
 
 
-@pytest.mark.parametrize("nseg", [2, 3, 5])
-def test_segment_composition_on_the_oracle(nseg):
+@pytest.mark.parametrize("nseg,kw", [(2, {}), (3, {}), (5, {}),
+                                     # exact zero-order hold (single endpoint: beta_0 = 0)
+                                     (3, dict(two_endpoint=0, discretization=S.DISC_ZOH))])
+def test_segment_composition_on_the_oracle(nseg, kw):
     """The composition the sharded scan rests on, on the fp64 oracle alone:
     segments scanned from a zero state and joined by
     K_in(k+1) = Phi_k (K_in(k) + beta_0(k) W_in(k)) + hT_loc(k), W_in(k+1) = last
@@ -98,7 +100,7 @@ def test_segment_composition_on_the_oracle(nseg):
     import numpy as np
 
     import oracle
-    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=41)
+    shape = S.WORKLOADS["tiny_hybrid_fp32"].replace(seqlen=41, **kw)
     inp = S.make_inputs(shape, seed=61, with_state=True)
     whole = oracle.scan_fwd(shape, inp)
     a_rate = -np.exp(inp["A_log"].astype(np.float64))                 # [H, nmode]
@@ -114,8 +116,10 @@ def test_segment_composition_on_the_oracle(nseg):
         S_dt = inp["dt"][:, a:b].astype(np.float64).sum(axis=1)        # [B, H]
         mag = np.exp(a_rate[None] * S_dt[:, :, None])                  # [B, H, nmode]
         ang = theta[None] * S_dt[:, :, None]                           # [B, H, n_pairs]
-        lam0, dt0 = (inp[k][:, a].astype(np.float64) for k in ("lam", "dt"))
-        beta0 = (1.0 - lam0) * dt0                                     # [B, H]
+        beta0 = np.zeros(inp["dt"][:, a].shape)                        # [B, H]
+        if shape.two_endpoint:
+            lam0, dt0 = (inp[k][:, a].astype(np.float64) for k in ("lam", "dt"))
+            beta0 = (1.0 - lam0) * dt0
         K = _apply_phi(K + beta0[:, :, None, None] * W, mag, ang, shape.n_real) + loc["hT"]
         W = loc["wT"]
     np.testing.assert_allclose(K, whole["hT"], rtol=1e-10, atol=1e-12)
